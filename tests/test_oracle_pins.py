@@ -1,0 +1,557 @@
+"""Pins of the CPU oracle against things other than itself: hand-derived
+cases, brute force, closed forms, invariants and an exact-arithmetic softmax.
+CPU only."""
+import decimal
+import itertools
+import os
+
+import numpy as np
+import pytest
+
+from oracle import (FLAG_CAPACITY, FLAG_RANGE, CapacityError, OracleCache, bf16_to_f64,
+                    dense_attention_f64, mask_words_to_bool, pack_codes, quantize_groups,
+                    quantize_stream_oneshot, to_fp16, unpack_codes)
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ----------------------------------------------------------------- fp16 rounding
+
+def _all_finite_fp16():
+    pats = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    vals = pats.view(np.float16).astype(np.float64)
+    ok = np.isfinite(vals)
+    return vals[ok], pats[ok]
+
+
+def test_fp16_rounding_is_nearest_ties_even_bruteforce():
+    vals, pats = _all_finite_fp16()
+    order = np.argsort(vals, kind="stable")
+    vals, pats = vals[order], pats[order]
+    # drop -0 duplicate so neighbours are distinct
+    keep = np.ones(len(vals), bool)
+    keep[1:] = vals[1:] != vals[:-1]
+    vals, pats = vals[keep], pats[keep]
+    rng = np.random.default_rng(7)
+    mags = np.exp(rng.uniform(np.log(2.0 ** -26), np.log(65000.0), 4000))
+    x = (mags * rng.choice([-1, 1], 4000)).astype(np.float32)
+    # exact midpoints between neighbours (ties) inside the normal range
+    mid = ((vals[1000:1100] + vals[1001:1101]) / 2).astype(np.float32)
+    x = np.concatenate([x, mid[mid.astype(np.float64) == (vals[1000:1100] + vals[1001:1101]) / 2]])
+    got = to_fp16(x).astype(np.float64)
+    for xi, gi in zip(x.astype(np.float64), got):
+        dist = np.abs(vals - xi)
+        best = np.nonzero(dist == dist.min())[0]
+        if len(best) == 1:
+            want = vals[best[0]]
+        else:  # tie: the neighbour with an even last significand bit
+            evens = [i for i in best if (int(pats[i]) & 1) == 0]
+            assert len(evens) == 1
+            want = vals[evens[0]]
+        assert gi == want, (xi, gi, want)
+    # overflow: at and beyond max + half an ulp (65520) rounds to infinity
+    assert np.isinf(to_fp16(np.float32(65520.0)))
+    assert to_fp16(np.float32(65519.0)) == np.float16(65504.0)
+
+
+# ----------------------------------------------------------------- quantizer
+
+def _golden_quantizer_cases():
+    cases = []
+    with open(os.path.join(GOLDEN, "quantizer_cases.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            b, xs, ks, s, z, qs = [p.strip() for p in line.split("|")]
+            cases.append((int(b), [float(v) for v in xs.split()],
+                          [bool(int(v)) for v in ks.split()], float(s), float(z),
+                          [int(v) for v in qs.split()]))
+    return cases
+
+
+@pytest.mark.parametrize("case", _golden_quantizer_cases())
+def test_quantizer_hand_derived_cases(case):
+    bits, xs, keep, s, z, codes = case
+    q, sh, zh = quantize_groups(np.array([xs], np.float32), np.array([keep]), bits)
+    assert float(sh[0]) == s
+    assert float(zh[0]) == z
+    assert q[0].tolist() == codes
+
+
+def _random_groups(rng, G, n, outliers=True):
+    x = rng.standard_normal((G, n)).astype(np.float32)
+    if outliers:
+        x[: G // 4] *= 10
+    return synth.bf16_bits_to_f32(synth.f32_to_bf16_bits(x))
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_quantizer_extremes_and_error_bound(bits):
+    rng = np.random.default_rng(bits)
+    x = _random_groups(rng, 512, 32)
+    q, s, z = quantize_groups(x, np.ones_like(x, bool), bits)
+    levels = 2 ** bits - 1
+    rows = np.arange(x.shape[0])
+    # z is the group minimum (bf16 values in fp16's normal range convert exactly)
+    assert np.all(z.astype(np.float32) == x.min(1))
+    assert np.all(q[rows, x.argmin(1)] == 0)
+    assert np.all(q[rows, x.argmax(1)] == levels)
+    s64 = s.astype(np.float64)
+    xhat = q * s64[:, None] + z.astype(np.float64)[:, None]
+    s_f = (x.max(1).astype(np.float64) - x.min(1)) / levels
+    ulp16 = 2.0 ** (np.floor(np.log2(s_f)) - 10)
+    bound = s64 / 2 + levels * ulp16 / 2 + s64 * 2.0 ** -19
+    assert np.all(np.abs(x - xhat) <= bound[:, None])
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_quantizer_picks_nearest_code_bruteforce(bits):
+    rng = np.random.default_rng(100 + bits)
+    x = _random_groups(rng, 64, 32)
+    keep = rng.random(x.shape) > 0.1
+    keep[:, 0] = True
+    q, s, z = quantize_groups(x, keep, bits)
+    codes = np.arange(2 ** bits, dtype=np.float64)
+    for gi in range(x.shape[0]):
+        cand = codes * float(s[gi]) + float(z[gi])
+        for j in range(x.shape[1]):
+            if not keep[gi, j]:
+                assert q[gi, j] == 0
+                continue
+            err = np.abs(cand - float(x[gi, j]))
+            assert err[q[gi, j]] <= err.min() + float(s[gi]) * 2.0 ** -19
+
+
+def test_quantizer_constant_group_is_exact():
+    x = np.full((3, 32), 1.75, np.float32)
+    x[1] = -0.125
+    x[2] = 0.0
+    q, s, z = quantize_groups(x, np.ones_like(x, bool), 4)
+    assert np.all(q == 0) and np.all(s == 0)
+    assert np.all(z.astype(np.float32)[:, None] == x)
+
+
+def test_quantizer_exact_grid_recovered():
+    """Values on a grid z0 + q*s0 (s0 a power of two) with codes 0 and
+    2^b - 1 present are quantized without error."""
+    rng = np.random.default_rng(3)
+    for bits in (2, 4):
+        lv = 2 ** bits - 1
+        q0 = rng.integers(0, lv + 1, (100, 32))
+        q0[:, 0], q0[:, 1] = 0, lv
+        e = rng.integers(-6, 2, 100).astype(np.float64)
+        z0 = rng.integers(-40, 40, 100) * 2.0 ** e
+        x = (z0[:, None] + q0 * (2.0 ** e)[:, None]).astype(np.float32)
+        q, s, z = quantize_groups(x, np.ones_like(x, bool), bits)
+        assert np.all(q == q0)
+        assert np.all(s.astype(np.float64) == 2.0 ** e)
+        assert np.all(z.astype(np.float64) == z0)
+
+
+# ----------------------------------------------------------------- packing
+
+def _golden_packing():
+    out = []
+    with open(os.path.join(GOLDEN, "packing_words.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            b, cs, ws = [p.strip() for p in line.split("|")]
+            out.append((int(b), [int(v) for v in cs.split()], [int(v, 16) for v in ws.split()]))
+    return out
+
+
+@pytest.mark.parametrize("case", _golden_packing())
+def test_packing_hand_derived_words(case):
+    bits, codes, words = case
+    got = pack_codes(np.array(codes, np.uint8), bits)
+    assert got.tolist() == words
+    assert unpack_codes(got, bits, len(codes)).tolist() == codes
+
+
+@pytest.mark.parametrize("bits,n", [(2, 32), (2, 64), (4, 32), (4, 64), (4, 128)])
+def test_pack_unpack_roundtrip(bits, n):
+    rng = np.random.default_rng(bits * n)
+    c = rng.integers(0, 2 ** bits, (7, 5, n)).astype(np.uint8)
+    assert np.array_equal(unpack_codes(pack_codes(c, bits), bits, n), c)
+
+
+def test_mask_words():
+    w = np.array([0x80000001, 0x2], np.uint32)
+    m = mask_words_to_bool(w, 64)
+    assert np.nonzero(m)[0].tolist() == [0, 31, 33]
+
+
+# ----------------------------------------------------------------- commit
+
+def _cache(w, cap=None, P=None, **over):
+    w = w.with_(**over) if over else w
+    cap = cap if cap is not None else w.L + 4 * max(w.k_group, w.blk)
+    P = P if P is not None else max(8, 2 * int(round(w.prot_frac * cap)) + 8)
+    return w, OracleCache(w.B, w.Hq, w.Hkv, w.d, w.blk, w.k_bits, w.v_bits,
+                          w.k_group, w.v_group, P, cap)
+
+
+SMALL = synth.WORKLOADS["batch32"].with_(B=2, Hq=4, Hkv=2, L=256, prot_frac=0.05)
+
+
+@pytest.mark.parametrize("kb,vb,gk,gv", [(4, 4, 32, 32), (2, 2, 64, 64), (2, 4, 128, 32),
+                                         (4, 2, 64, 128)])
+def test_incremental_commits_equal_one_shot(kb, vb, gk, gv):
+    w, c = _cache(SMALL, k_bits=kb, v_bits=vb, k_group=gk, v_group=gv)
+    n_blocks = w.L // w.blk + 1          # ends with an incomplete K group when gk > blk
+    per_unit = {}
+    for i in range(n_blocks):
+        K, V, M = synth.block_inputs(w, i)
+        c.commit(K, V, M)
+        for b in range(w.B):
+            for h in range(w.Hkv):
+                per_unit.setdefault((b, h), []).append((K[b, h], V[b, h], M[b, h]))
+    snap = c.snapshot()
+    for (b, h), blocks in per_unit.items():
+        u = b * w.Hkv + h
+        Ks = np.concatenate([x[0] for x in blocks])
+        Vs = np.concatenate([x[1] for x in blocks])
+        prot = np.concatenate([mask_words_to_bool(x[2], w.blk) for x in blocks])
+        ref = quantize_stream_oneshot(Ks, Vs, prot, kb, vb, gk, gv, c.P)
+        nG = ref["k_codes"].shape[0]
+        assert np.array_equal(snap["k_codes"][u], ref["k_codes"])
+        assert np.array_equal(snap["k_sz"][u].view(np.uint16), ref["k_sz"].view(np.uint16))
+        assert np.array_equal(snap["v_codes"][u], ref["v_codes"])
+        assert np.array_equal(snap["v_sz"][u].view(np.uint16), ref["v_sz"].view(np.uint16))
+        n = int(snap["prot_count"][u])
+        assert np.array_equal(snap["prot_pos"][u, :n], ref["prot_pos"])
+        assert np.array_equal(snap["prot_k"][u, :n], ref["prot_k"])
+        # the tail holds the incomplete group's bf16 K verbatim
+        assert np.array_equal(snap["k_tail"][u], Ks[nG * gk:])
+
+
+def test_protected_entries_exact_and_excluded():
+    w, c = _cache(SMALL, k_bits=4, v_bits=4, k_group=32, v_group=32)
+    K, V, M = synth.block_inputs(w, 0)
+    c.commit(K, V, M)
+    prot = mask_words_to_bool(M.reshape(w.B * w.Hkv, -1), w.blk)
+    snap = c.snapshot()
+    for u in range(w.B * w.Hkv):
+        want = np.nonzero(prot[u])[0]
+        assert snap["prot_count"][u] == len(want)
+        assert snap["prot_pos"][u, :len(want)].tolist() == want.tolist()
+        Ku = K.reshape(w.B * w.Hkv, w.blk, w.d)[u]
+        assert np.array_equal(snap["prot_k"][u, :len(want)], Ku[want])
+        # protected slot codes are 0 in every channel
+        codes = unpack_codes(snap["k_codes"][u, 0], 4, 32)     # [d, 32]
+        assert np.all(codes[:, want] == 0)
+        # dequantized K reproduces protected rows exactly
+        kh = c.dequant_k(u)
+        assert np.array_equal(kh[want], bf16_to_f64(Ku[want]))
+    # changing the protected tokens' K values changes nothing else
+    K2 = K.copy().reshape(w.B * w.Hkv, w.blk, w.d)
+    for u in range(w.B * w.Hkv):
+        K2[u, prot[u]] = synth.f32_to_bf16_bits(np.full((prot[u].sum(), w.d), 1000.0, np.float32))
+    _, c2 = _cache(SMALL, k_bits=4, v_bits=4, k_group=32, v_group=32)
+    c2.commit(K2.reshape(K.shape), V, M)
+    s2 = c2.snapshot()
+    assert np.array_equal(snap["k_codes"], s2["k_codes"])
+    assert np.array_equal(snap["k_sz"].view(np.uint16), s2["k_sz"].view(np.uint16))
+
+
+def test_all_protected_group_has_zero_scale_and_zero():
+    w, c = _cache(SMALL.with_(B=1, Hkv=1, Hq=1), k_bits=2, v_bits=2, k_group=32, v_group=32, P=64)
+    K, V, _ = synth.block_inputs(w, 0)
+    M = np.full((1, 1, 1), 0xFFFFFFFF, np.uint32)
+    c.commit(K, V, M)
+    assert np.all(c.k_sz[0, 0] == 0) and np.all(c.k_codes[0, 0] == 0)
+    assert np.array_equal(c.dequant_k(0), bf16_to_f64(K[0, 0]))
+
+
+def test_side_table_overflow_keeps_first_and_flags():
+    w = SMALL.with_(B=1, Hkv=1, Hq=1)
+    K, V, _ = synth.block_inputs(w, 0)
+    want = [1, 5, 9, 20, 30]
+    M = synth.positions_to_mask(want, 32).reshape(1, 1, 1)
+    _, c = _cache(w, k_bits=4, v_bits=4, k_group=32, v_group=32, P=3)
+    f = c.commit(K, V, M)
+    assert f & FLAG_CAPACITY
+    assert c.prot_pos[0, :3].tolist() == [1, 5, 9]
+    # the excess tokens are quantized as if never protected
+    _, c_ref = _cache(w, k_bits=4, v_bits=4, k_group=32, v_group=32, P=3)
+    c_ref.commit(K, V, synth.positions_to_mask([1, 5, 9], 32).reshape(1, 1, 1))
+    assert np.array_equal(c.k_codes, c_ref.k_codes)
+    assert np.array_equal(c.k_sz.view(np.uint16), c_ref.k_sz.view(np.uint16))
+    assert c_ref.flags == 0
+
+
+def test_capacity_error_leaves_state():
+    w, c = _cache(SMALL, cap=64)
+    for i in range(2):
+        c.commit(*synth.block_inputs(w, i))
+    before = c.snapshot()
+    with pytest.raises(CapacityError):
+        c.commit(*synth.block_inputs(w, 2))
+    after = c.snapshot()
+    assert before["len"] == after["len"] == 64
+    assert np.array_equal(before["v_codes"], after["v_codes"])
+
+
+def test_range_flag_and_clamp():
+    w, c = _cache(SMALL.with_(B=1, Hkv=1, Hq=1), k_bits=4, v_bits=4, k_group=32, v_group=32)
+    K, V, _ = synth.block_inputs(w, 0)
+    V = V.copy()
+    V[0, 0, 3, 7] = synth.f32_to_bf16_bits(np.array([1e6], np.float32))[0]
+    f = c.commit(K, V, None)
+    assert f & FLAG_RANGE
+    vh = c.dequant_v(0)
+    # the value was clamped to the fp16 maximum before quantization
+    assert np.all(np.isfinite(vh))
+    assert abs(vh[3, 7] - 65504.0) <= float(c.v_sz[0, 3, 0, 0]) / 2 + 16
+
+
+# ----------------------------------------------------------------- attention
+
+def _decimal_attention(q, K, V, scale):
+    """Softmax attention in 40-digit decimal arithmetic, loops only."""
+    ctx = decimal.Context(prec=40)
+    D = lambda v: decimal.Decimal(float(v))  # noqa: E731
+    out = []
+    for qi in q:
+        logits = [ctx.multiply(D(scale), sum((ctx.multiply(D(a), D(b)) for a, b in zip(qi, kj)),
+                                             decimal.Decimal(0))) for kj in K]
+        m = max(logits)
+        e = [ctx.exp(ctx.subtract(x, m)) for x in logits]
+        tot = sum(e, decimal.Decimal(0))
+        row = []
+        for c in range(len(V[0])):
+            num = sum((ctx.multiply(ei, D(V[j][c])) for j, ei in enumerate(e)), decimal.Decimal(0))
+            row.append(float(ctx.divide(num, tot)))
+        out.append(row)
+    return np.array(out)
+
+
+def test_dense_attention_matches_exact_arithmetic():
+    rng = np.random.default_rng(11)
+    for (n, m, d) in [(1, 1, 1), (2, 5, 3), (3, 7, 4)]:
+        q = rng.standard_normal((n, d)) * 3
+        K = rng.standard_normal((m, d))
+        V = rng.standard_normal((m, d))
+        got = dense_attention_f64(q, K, V, 0.7)
+        want = _decimal_attention(q, K, V, 0.7)
+        assert np.allclose(got, want, rtol=0, atol=1e-13)
+
+
+def _filled(w, n_blocks, **over):
+    w, c = _cache(w, **over)
+    for i in range(n_blocks):
+        c.commit(*synth.block_inputs(w, i))
+    return w, c
+
+
+def test_passthrough_equals_dense_attention():
+    w, c = _filled(SMALL, 5, k_bits=16, v_bits=16)
+    Q = synth.queries_bits(w, 0)
+    Ka, Va = synth.active_block_bits(w, 0)
+    O = c.block_attention(Q, Ka, Va, w.softmax_scale)
+    g = w.Hq // w.Hkv
+    for b in range(w.B):
+        for hq in range(w.Hq):
+            h = hq // g
+            Ks = np.concatenate([synth.unit_kv_bits(w, b, h, 5 * w.blk)[0], Ka[b, h]])
+            Vs = np.concatenate([synth.unit_kv_bits(w, b, h, 5 * w.blk)[1], Va[b, h]])
+            ref = _decimal_attention(bf16_to_f64(Q[b, hq, :2]), bf16_to_f64(Ks), bf16_to_f64(Vs),
+                                     w.softmax_scale) if (b, hq) == (0, 0) else \
+                dense_attention_f64(bf16_to_f64(Q[b, hq]), bf16_to_f64(Ks), bf16_to_f64(Vs),
+                                    w.softmax_scale)
+            rows = ref.shape[0]
+            assert np.allclose(O[b, hq, :rows], ref, rtol=0, atol=1e-12)
+
+
+def _grid_block(rng, blk, d, bits, GK, GV, prot_rows):
+    """K with every (group, channel) on a grid z0 + q*2^e (codes 0 and 2^b-1
+    present among non-protected tokens) and V with every (token, channel
+    group) on such a grid: quantization is then lossless."""
+    lv = 2 ** bits - 1
+    K = np.zeros((blk, d))
+    keep = np.ones(blk, bool)
+    keep[prot_rows] = False
+    kidx = np.nonzero(keep)[0]
+    for g0 in range(0, blk, GK):
+        for ch in range(d):
+            e = rng.integers(-4, 1)
+            q = rng.integers(0, lv + 1, GK)
+            ks = [i - g0 for i in kidx if g0 <= i < g0 + GK]
+            q[ks[0]], q[ks[1]] = 0, lv
+            z0 = rng.integers(-30, 30)
+            K[g0:g0 + GK, ch] = (z0 + q) * 2.0 ** e
+    for r in prot_rows:
+        K[r] = rng.standard_normal(d) * 5
+    V = np.zeros((blk, d))
+    for t in range(blk):
+        for c0 in range(0, d, GV):
+            e = rng.integers(-4, 1)
+            q = rng.integers(0, lv + 1, GV)
+            q[0], q[-1] = 0, lv
+            V[t, c0:c0 + GV] = (rng.integers(-30, 30) + q) * 2.0 ** e
+    return synth.f32_to_bf16_bits(K.astype(np.float32)), synth.f32_to_bf16_bits(V.astype(np.float32))
+
+
+@pytest.mark.parametrize("bits,GK,GV", [(4, 32, 32), (2, 32, 64), (2, 32, 32), (4, 32, 128)])
+def test_grid_exact_cache_attention_equals_dense(bits, GK, GV):
+    """Commit + dequant + attention in quantized mode equal dense attention
+    over the original K/V when the inputs sit on each group's grid."""
+    rng = np.random.default_rng(bits * GK + GV)
+    B, Hq, Hkv, d, blk = 1, 4, 2, 128, 32
+    nb = 4
+    c = OracleCache(B, Hq, Hkv, d, blk, bits, bits, GK, GV, 16, 256)
+    allK = [[[] for _ in range(Hkv)] for _ in range(B)]
+    allV = [[[] for _ in range(Hkv)] for _ in range(B)]
+    for i in range(nb):
+        K = np.zeros((B, Hkv, blk, d), np.uint16)
+        V = np.zeros_like(K)
+        M = np.zeros((B, Hkv, 1), np.uint32)
+        for h in range(Hkv):
+            prot = [3 + h, 17] if i % 2 == 0 else []
+            K[0, h], V[0, h] = _grid_block(rng, blk, d, bits, GK, GV, prot)
+            M[0, h] = synth.positions_to_mask(prot, blk)
+            allK[0][h].append(K[0, h])
+            allV[0][h].append(V[0, h])
+        c.commit(K, V, M)
+    Q = synth.f32_to_bf16_bits(rng.standard_normal((B, Hq, blk, d)).astype(np.float32))
+    Ka = synth.f32_to_bf16_bits(rng.standard_normal((B, Hkv, blk, d)).astype(np.float32))
+    Va = synth.f32_to_bf16_bits(rng.standard_normal((B, Hkv, blk, d)).astype(np.float32))
+    O = c.block_attention(Q, Ka, Va, 0.09)
+    for hq in range(Hq):
+        h = hq // 2
+        Ks = np.concatenate(allK[0][h] + [Ka[0, h]])
+        Vs = np.concatenate(allV[0][h] + [Va[0, h]])
+        ref = dense_attention_f64(bf16_to_f64(Q[0, hq]), bf16_to_f64(Ks), bf16_to_f64(Vs), 0.09)
+        assert np.allclose(O[0, hq], ref, rtol=0, atol=1e-12)
+
+
+def test_grid_exact_with_64_token_groups_and_tail():
+    """Same as above with K groups of 64 spanning two commits, ending with
+    a 32-token bf16 tail."""
+    rng = np.random.default_rng(64)
+    B, Hq, Hkv, d, blk, GK, GV, bits = 1, 2, 1, 128, 32, 64, 32, 2
+    c = OracleCache(B, Hq, Hkv, d, blk, bits, bits, GK, GV, 16, 256)
+    Kg, Vg = _grid_block(rng, 192, d, bits, GK, GV, [5, 70, 130])
+    prot = np.zeros(192, bool)
+    prot[[5, 70, 130]] = True
+    for i in range(6):
+        sl = slice(32 * i, 32 * (i + 1))
+        M = synth.positions_to_mask(np.nonzero(prot[sl])[0], 32).reshape(1, 1, 1)
+        c.commit(Kg[sl].reshape(1, 1, 32, d), Vg[sl].reshape(1, 1, 32, d), M)
+    Kt, Vt = _grid_block(rng, 32, d, bits, 32, GV, [])
+    c.commit(Kt.reshape(1, 1, 32, d), Vt.reshape(1, 1, 32, d), None)   # stays in the tail
+    assert c.n_quantized == 192 and c.len == 224
+    Q = synth.f32_to_bf16_bits(rng.standard_normal((B, Hq, blk, d)).astype(np.float32))
+    Ka = synth.f32_to_bf16_bits(rng.standard_normal((B, Hkv, blk, d)).astype(np.float32))
+    Va = synth.f32_to_bf16_bits(rng.standard_normal((B, Hkv, blk, d)).astype(np.float32))
+    O = c.block_attention(Q, Ka, Va, 0.09)
+    Ks = np.concatenate([Kg, Kt, Ka[0, 0]])
+    Vs = np.concatenate([Vg, Vt, Va[0, 0]])
+    for hq in range(Hq):
+        ref = dense_attention_f64(bf16_to_f64(Q[0, hq]), bf16_to_f64(Ks), bf16_to_f64(Vs), 0.09)
+        assert np.allclose(O[0, hq], ref, rtol=0, atol=1e-12)
+
+
+def test_empty_cache_attends_active_block_only():
+    w, c = _filled(SMALL, 0)
+    Q = synth.queries_bits(w, 1)
+    Ka, Va = synth.active_block_bits(w, 1)
+    O = c.block_attention(Q, Ka, Va, w.softmax_scale)
+    g = w.Hq // w.Hkv
+    for b, hq in itertools.product(range(w.B), range(w.Hq)):
+        ref = dense_attention_f64(bf16_to_f64(Q[b, hq]), bf16_to_f64(Ka[b, hq // g]),
+                                  bf16_to_f64(Va[b, hq // g]), w.softmax_scale)
+        assert np.allclose(O[b, hq], ref, rtol=0, atol=1e-13)
+
+
+def test_zero_queries_give_mean_of_values():
+    w, c = _filled(SMALL, 6)
+    Q = np.zeros((w.B, w.Hq, w.blk, w.d), np.uint16)
+    Ka, Va = synth.active_block_bits(w, 2)
+    O = c.block_attention(Q, Ka, Va, w.softmax_scale)
+    g = w.Hq // w.Hkv
+    for b, hq in itertools.product(range(w.B), range(w.Hq)):
+        u = b * w.Hkv + hq // g
+        allv = np.concatenate([c.dequant_v(u), bf16_to_f64(Va[b, hq // g])])
+        assert np.allclose(O[b, hq], allv.mean(0)[None, :], rtol=0, atol=1e-12)
+
+
+def test_constant_values_give_constant_output():
+    w, c = _cache(SMALL)
+    cval = synth.f32_to_bf16_bits(np.float32(-0.6875))
+    for i in range(5):
+        K, V, M = synth.block_inputs(w, i)
+        c.commit(K, np.full_like(V, cval), M)
+    Q = synth.queries_bits(w, 3)
+    Ka, _ = synth.active_block_bits(w, 3)
+    O = c.block_attention(Q, Ka, np.full_like(Ka, cval), w.softmax_scale)
+    assert np.allclose(O, -0.6875, rtol=0, atol=1e-13)
+
+
+def test_permuting_whole_groups_leaves_output():
+    w, c = _filled(SMALL.with_(k_group=32), 6)
+    Q = synth.queries_bits(w, 4)
+    Ka, Va = synth.active_block_bits(w, 4)
+    O = c.block_attention(Q, Ka, Va, w.softmax_scale)
+    # rebuild the committed stream with K-groups (and their V rows) permuted
+    perm = [3, 0, 5, 1, 4, 2]
+    _, c2 = _cache(SMALL.with_(k_group=32))
+    for i in perm:
+        c2.commit(*synth.block_inputs(w, i))
+    O2 = c2.block_attention(Q, Ka, Va, w.softmax_scale)
+    assert np.allclose(O, O2, rtol=0, atol=1e-12)
+
+
+def test_gqa_equals_mha_with_replicated_kv():
+    w = SMALL.with_(B=1, Hq=4, Hkv=2)
+    _, c = _cache(w)
+    w4 = w.with_(Hkv=4)
+    _, c4 = _cache(w4)
+    for i in range(5):
+        K, V, M = synth.block_inputs(w, i)
+        c.commit(K, V, M)
+        rep = [0, 0, 1, 1]
+        c4.commit(K[:, rep], V[:, rep], M[:, rep])
+    Q = synth.queries_bits(w, 5)
+    Ka, Va = synth.active_block_bits(w, 5)
+    O = c.block_attention(Q, Ka, Va, 0.1)
+    O4 = c4.block_attention(Q, Ka[:, [0, 0, 1, 1]], Va[:, [0, 0, 1, 1]], 0.1)
+    assert np.array_equal(O, O4)
+
+
+def test_quantized_attention_uses_dequantized_cache():
+    """Quantized attention equals dense attention over K_hat, V_hat built
+    here from the stored codes with x_hat = q*s + z (per-channel K groups,
+    per-token V groups) and the side table's rows."""
+    w, c = _filled(SMALL.with_(k_group=64, v_group=32, k_bits=2, v_bits=4), 5)
+    Q = synth.queries_bits(w, 6)
+    Ka, Va = synth.active_block_bits(w, 6)
+    O = c.block_attention(Q, Ka, Va, w.softmax_scale)
+    u, b, h = 1, 0, 1
+    n_q = c.n_quantized
+    khat = np.zeros((c.len, w.d))
+    for j in range(n_q // 64):
+        for ch in range(w.d):
+            codes = unpack_codes(c.k_codes[u, j, ch], 2, 64)
+            s, z = c.k_sz[u, j, ch]
+            khat[64 * j:64 * j + 64, ch] = codes * float(s) + float(z)
+    for i in range(c.prot_count[u]):
+        khat[c.prot_pos[u, i]] = bf16_to_f64(c.prot_k[u, i])
+    khat[n_q:] = bf16_to_f64(c.k_tail[u, :c.len - n_q])
+    vhat = np.zeros((c.len, w.d))
+    for t in range(c.len):
+        codes = unpack_codes(c.v_codes[u, t], 4, w.d)
+        for g0 in range(w.d // 32):
+            s, z = c.v_sz[u, t, g0]
+            vhat[t, 32 * g0:32 * g0 + 32] = codes[32 * g0:32 * g0 + 32] * float(s) + float(z)
+    g = w.Hq // w.Hkv
+    for hq in range(h * g, h * g + g):
+        ref = dense_attention_f64(bf16_to_f64(Q[b, hq]),
+                                  np.concatenate([khat, bf16_to_f64(Ka[b, h])]),
+                                  np.concatenate([vhat, bf16_to_f64(Va[b, h])]),
+                                  w.softmax_scale)
+        assert np.allclose(O[b, hq], ref, rtol=0, atol=1e-12)
