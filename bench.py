@@ -1,0 +1,619 @@
+#!/usr/bin/env python
+"""Benchmark of the low-bit block-diffusion KV-cache hot path on B200.
+
+One step = dkv_commit_block of one 32-token block (quantize-on-commit) +
+dkv_block_attention of the next active block's queries over the committed
+cache (one denoising step).  Every max(1, k_group/block) steps a cache is
+rolled back with dkv_cache_truncate to its starting length, so the committed
+length stays at the workload's L (+ at most k_group tokens) however many
+steps run.  Inputs are seeded synthetic data from `synth`, resident in HBM
+before the timed region; caches are replicated R times and used round-robin
+so that the bytes touched between two uses of one cache exceed the L2.
+
+Output: one JSON line (rank 0).  `value` = algorithmic HBM bytes of all steps
+(packed cache + scales + side table + tail read by attention, Q / active
+block / output, commit reads and writes) / device time of the timed region,
+summed over ranks (weak scaling: each rank runs its own copy of the
+workload).  `--impl reference` times the CPU oracle instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = ("block-attention HBM GB/s & % of 8 TB/s roofline; commit tokens/s (1×B200)")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------ accounting
+
+def _n_prot(w: synth.Workload, L: int) -> float:
+    """Expected protected positions per unit among the first L tokens."""
+    return w.prot_frac * L
+
+
+def attn_bytes(w: synth.Workload, L: int) -> float:
+    """Algorithmic HBM bytes of one dkv_block_attention at committed length L."""
+    U, d = w.B * w.Hkv, w.d
+    if w.k_bits < 16:
+        Lq = (L // w.k_group) * w.k_group
+        nG = Lq // w.k_group
+        kb = Lq * d * w.k_bits / 8 + nG * d * 4 + (nG + 1) * 4 + (L - Lq) * d * 2
+        kb += _n_prot(w, Lq) * (d * 2 + 4)
+    else:
+        kb = L * d * 2
+    vb = L * (d * w.v_bits / 8 + (d // w.v_group) * 4) if w.v_bits < 16 else L * d * 2
+    io = w.B * w.Hq * w.blk * d * 2 * 2 + 2 * U * w.blk * d * 2
+    return U * (kb + vb) + io
+
+
+def attn_flops(w: synth.Workload, L: int) -> float:
+    """QK^T and PV multiply-adds x 2 over committed + active tokens."""
+    return 4.0 * w.rows * w.d * (L + w.blk) * w.B * w.Hkv
+
+
+def commit_bytes(w: synth.Workload, L_before: int) -> float:
+    U, d, blk = w.B * w.Hkv, w.d, w.blk
+    b = 2 * blk * d * 2 + 4                                   # K, V block + mask
+    b += blk * (d * w.v_bits / 8 + (d // w.v_group) * 4) if w.v_bits < 16 else blk * d * 2
+    if w.k_bits < 16:
+        n_tail = L_before % w.k_group
+        if n_tail + blk >= w.k_group:                        # completes a group
+            b += n_tail * d * 2 + w.k_group * d * w.k_bits / 8 + d * 4 + 8
+            b += _n_prot(w, w.k_group) * (d * 2 + 4)
+        else:
+            b += blk * d * 2
+    else:
+        b += blk * d * 2
+    return U * b
+
+
+def cycle_len(w: synth.Workload) -> int:
+    return max(1, w.k_group // w.blk) if w.k_bits < 16 else 1
+
+
+def step_lengths(w: synth.Workload, K: int, R: int):
+    """Committed length before the commit of each step k (cache k % R)."""
+    C = cycle_len(w)
+    pos = [0] * R
+    out = []
+    for k in range(K):
+        r = k % R
+        out.append(w.L + pos[r] * w.blk)
+        pos[r] = (pos[r] + 1) % C
+    return out
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def traffic_record():
+    """ncu DRAM traffic per launch of the dominant kernel, if the committed
+    record matches the kernel source as it is now (else None)."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return {}
+    with open(p) as f:
+        rec = json.load(f)
+    out = {}
+    for wl, r in rec.items():
+        src = os.path.join(ROOT, r.get("source", ""))
+        if not os.path.exists(src):
+            continue
+        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        if h == r.get("source_sha256_16"):
+            out[wl] = r
+    return out
+
+
+# ------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-i", gpu_id, "-lms", "100"], stdout=subprocess.PIPE,
+                stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, pw, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in out.splitlines():
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+                pw.append(float(f[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        busy = [s for s, p in zip(sm, pw) if p > 200.0] or sm
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm), "samples_under_load": len(busy),
+                "power_w_max": max(pw)}
+
+
+# ------------------------------------------------------------ GPU arm
+
+def _dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def run_gpu(w: synth.Workload, K: int, W: int, want_e2e=True, log=print, kernel=0):
+    import torch
+    import quantized_kv_cache_dkv_b200 as dkv
+
+    world, rank, local = _dist()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    props = torch.cuda.get_device_properties(dev)
+    l2 = getattr(props, "L2_cache_size", 126 * 2 ** 20)
+    C = cycle_len(w)
+    cache_bytes = attn_bytes(w, w.L)
+    R = 1 if cache_bytes >= 2 * l2 else min(8, math.ceil(3 * l2 / cache_bytes))
+    unit = max(w.k_group, w.blk)
+    cap = ((w.L + C * w.blk + unit - 1) // unit) * unit
+    P = int(round(w.prot_frac * cap)) * 2 + 64
+    cfg = dkv.make_config(w.B, w.Hq, w.Hkv, w.d, w.blk, w.k_bits, w.v_bits, w.k_group,
+                          w.v_group, P, cap)
+    caches = [dkv.dkv_cache_alloc(cfg) for _ in range(R)]
+    if kernel:
+        for c in caches:
+            dkv.dkv_cache_set_option(c, dkv.DKV_OPT_ATTN_KERNEL, kernel)
+
+    def up(bits):
+        import numpy as np
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(
+            torch.bfloat16)
+
+    def upw(words):
+        import numpy as np
+        return torch.from_numpy(np.ascontiguousarray(words).view(np.int32)).to(dev)
+
+    t0 = time.time()
+    nb = w.L // w.blk
+    for i in range(nb):
+        K_, V_, M_ = synth.block_inputs(w, i)
+        Kd, Vd, Md = up(K_), up(V_), upw(M_)
+        for c in caches:
+            dkv.dkv_commit_block(c, Kd, Vd, Md)
+    torch.cuda.synchronize()
+    t_prefill = time.time() - t0
+
+    # per-step inputs: C blocks to commit, S distinct query / active blocks
+    blocks = [synth.block_inputs(w, nb + c) for c in range(C)]
+    host_blocks = blocks
+    dblocks = [(up(a), up(b), upw(m)) for a, b, m in blocks]
+    S = min(K, R * C) if K > 0 else 1
+    S = max(S, 1)
+    host_steps = [(synth.queries_bits(w, s),) + tuple(synth.active_block_bits(w, s))
+                  for s in range(S)]
+    dsteps = [(up(q), up(ka), up(va)) for q, ka, va in host_steps]
+    outs = [torch.empty((w.B, w.Hq, w.blk, w.d), dtype=torch.bfloat16, device=dev)
+            for _ in range(S)]
+
+    pos = [0] * R
+    launches = [0]
+
+    def step(k):
+        r = k % R
+        c = pos[r]
+        Kd, Vd, Md = dblocks[c]
+        dkv.dkv_commit_block(caches[r], Kd, Vd, Md)
+        q, ka, va = dsteps[k % S]
+        dkv.dkv_block_attention(caches[r], q, ka, va, w.softmax_scale, outs[k % S])
+        launches[0] += 1 + dkv.dkv_last_attention_plan(caches[r])[2]
+        pos[r] += 1
+        if pos[r] == C:  # back to the starting length
+            dkv.dkv_cache_truncate(caches[r], w.L)
+            launches[0] += 1 if w.k_bits < 16 else 0
+            pos[r] = 0
+
+    def finish():
+        for r in range(R):
+            if pos[r]:
+                dkv.dkv_cache_truncate(caches[r], w.L)
+                launches[0] += 1 if w.k_bits < 16 else 0
+                pos[r] = 0
+
+    # warm-up (eager), then capture exactly K steps in one CUDA graph
+    for k in range(W):
+        step(k)
+    finish()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    launches[0] = 0
+    with torch.cuda.graph(g):
+        for k in range(K):
+            step(k)
+        finish()
+    graph_launches = launches[0]
+    plan = dkv.dkv_last_attention_plan(caches[0])
+    g.replay()
+    torch.cuda.synchronize()
+
+    # clocks sampled over a window of back-to-back replays around the timed one
+    gpu_id = str(getattr(props, "uuid", local))
+    gpu_id = gpu_id if gpu_id.startswith("GPU-") or not hasattr(props, "uuid") else "GPU-" + gpu_id
+    sampler = ClockSampler(gpu_id)
+    t_end = time.time() + 0.6
+    while time.time() < t_end:
+        g.replay()
+        torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    stream = torch.cuda.current_stream()
+    e0.record(stream)
+    g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = e0.elapsed_time(e1)
+    t_end = time.time() + 0.4
+    while time.time() < t_end:
+        g.replay()
+        torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    Ls = step_lengths(w, K, R)
+    step_bytes = sum(attn_bytes(w, L + w.blk) + commit_bytes(w, L) for L in Ls)
+    value = world * step_bytes / (ms / 1e3) / 1e9
+
+    # profiling pass: device time of each kernel kind (eager launches)
+    for c in caches:
+        dkv.dkv_cache_set_option(c, dkv.DKV_OPT_PROFILE, 1)
+    Kp = max(K, 2 * R * C)
+    for k in range(Kp):
+        step(k)
+    finish()
+    torch.cuda.synchronize()
+    prof = {}
+    for kind, name in ((dkv.DKV_KERNEL_ATTENTION, "attention"), (dkv.DKV_KERNEL_COMBINE, "combine"),
+                       (dkv.DKV_KERNEL_COMMIT, "commit"), (dkv.DKV_KERNEL_TRUNCATE, "truncate")):
+        tot, n = 0.0, 0
+        for c in caches:
+            a, b = dkv.dkv_profile_read(c, kind)
+            tot += a
+            n += b
+        prof[name] = (tot, n)
+    for c in caches:
+        dkv.dkv_cache_set_option(c, dkv.DKV_OPT_PROFILE, 0)
+    Lp = step_lengths(w, Kp, R)
+    att_ms, att_n = prof["attention"]
+    att_bytes = sum(attn_bytes(w, L + w.blk) for L in Lp)
+    att_flops = sum(attn_flops(w, L + w.blk) for L in Lp)
+    com_ms, com_n = prof["commit"]
+
+    # end to end through the public API from pinned host memory
+    e2e = None
+    if want_e2e:
+        pin = lambda a: torch.from_numpy(a).pin_memory()  # noqa: E731
+        import numpy as np
+        hb = [(pin(a.view(np.int16)), pin(b.view(np.int16)), pin(m.view(np.int32)))
+              for a, b, m in host_blocks]
+        hs = [(pin(q.view(np.int16)), pin(ka.view(np.int16)), pin(va.view(np.int16)))
+              for q, ka, va in host_steps]
+        hout = torch.empty((w.B, w.Hq, w.blk, w.d), dtype=torch.int16).pin_memory()
+        dK = torch.empty((w.B, w.Hkv, w.blk, w.d), dtype=torch.int16, device=dev)
+        dV, dKa, dVa = torch.empty_like(dK), torch.empty_like(dK), torch.empty_like(dK)
+        dM = torch.empty((w.B, w.Hkv, w.blk // 32), dtype=torch.int32, device=dev)
+        dQ = torch.empty((w.B, w.Hq, w.blk, w.d), dtype=torch.int16, device=dev)
+        dO = torch.empty_like(dQ)
+        h2d = (dK.numel() * 2 * 2 + dM.numel() * 4 + dQ.numel() * 2 + dKa.numel() * 2 * 2)
+        d2h = dO.numel() * 2
+
+        def e2e_step(k):
+            r = k % R
+            c = pos[r]
+            dK.copy_(hb[c][0], non_blocking=True)
+            dV.copy_(hb[c][1], non_blocking=True)
+            dM.copy_(hb[c][2], non_blocking=True)
+            dkv.dkv_commit_block(caches[r], dK, dV, dM)
+            q, ka, va = hs[k % S]
+            dQ.copy_(q, non_blocking=True)
+            dKa.copy_(ka, non_blocking=True)
+            dVa.copy_(va, non_blocking=True)
+            dkv.dkv_block_attention(caches[r], dQ, dKa, dVa, w.softmax_scale, dO)
+            hout.copy_(dO, non_blocking=True)
+            pos[r] += 1
+            if pos[r] == C:
+                dkv.dkv_cache_truncate(caches[r], w.L)
+                pos[r] = 0
+
+        for k in range(W):
+            e2e_step(k)
+        finish()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for k in range(K):
+            e2e_step(k)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        ems = e0.elapsed_time(e1)
+        finish()
+        if world > 1:
+            t = torch.tensor([ems], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        e2e = {"value": world * step_bytes / (ems / 1e3) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": ems / K}
+
+    for c in caches:
+        dkv.dkv_cache_free(c)
+    return {
+        "ms": ms, "value": value, "R": R, "C": C, "cap": cap, "P": P, "plan": plan,
+        "graph_launches": graph_launches, "clocks": clocks, "t_prefill_s": t_prefill,
+        "att_ms": att_ms, "att_n": att_n, "att_bytes": att_bytes, "att_flops": att_flops,
+        "combine_ms": prof["combine"][0], "combine_n": prof["combine"][1],
+        "commit_ms": com_ms, "commit_n": com_n, "e2e": e2e, "L_mean": sum(Ls) / len(Ls) + w.blk,
+        "step_bytes": step_bytes / K,
+    }
+
+
+def roofline(w: synth.Workload, r: dict, peaks: dict, peak_kind: str, traffic):
+    """Roofline of the dominant kernel (the split attention kernel)."""
+    avg_s = r["att_ms"] / max(r["att_n"], 1) / 1e3
+    bytes_launch = r["att_bytes"] / max(r["att_n"], 1)
+    flops_launch = r["att_flops"] / max(r["att_n"], 1)
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    bound = "tensor" if flops_launch / bytes_launch > ridge else "hbm"
+    if bound == "hbm":
+        ach, peak, unit = bytes_launch / avg_s / 1e9, peaks["hbm_gbs"], "GB/s"
+    else:
+        ach, peak, unit = flops_launch / avg_s / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+    tr = None
+    if traffic and w.name in traffic:
+        t = traffic[w.name]
+        tr = t["traffic_bytes_per_launch"] * (bytes_launch / t["algorithmic_bytes_per_launch"]) \
+            if t.get("scale_by_bytes") else t["traffic_bytes_per_launch"]
+    return {"bound": bound, "achieved": round(ach, 2), "peak": peak, "unit": unit,
+            "frac": round(ach / peak, 4), "traffic": tr,
+            "peak_source": f"{peak_kind} ({'hbm_gbs' if bound == 'hbm' else 'bf16_tflops burst'})",
+            "kernel": "attention split kernel", "avg_launch_us": round(avg_s * 1e6, 3),
+            "algorithmic_bytes_per_launch": int(bytes_launch),
+            "algorithmic_flops_per_launch": int(flops_launch),
+            "hbm_gbs_at_kernel": round(bytes_launch / avg_s / 1e9, 1),
+            "pct_of_8tbs_at_kernel": round(100 * bytes_launch / avg_s / 8e12, 2)}
+
+
+# ------------------------------------------------------------ CPU oracle arm
+
+def _blas_threads() -> int:
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        n = [i.get("num_threads", 1) for i in info if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample(w: synth.Workload, seconds: float, max_steps=None, warmup=0):
+    """Time the oracle (as it stands) on sampled units of the workload: each
+    step = commit of one block + one block attention, per sampled unit.
+    Returns (GB/s, steps, elapsed, description)."""
+    from oracle import OracleCache
+    nb = w.L // w.blk
+    C = cycle_len(w)
+    units = [(0, 0)] if w.L >= 16384 else [(0, 0), (w.B - 1, w.Hkv - 1)]
+    cap = w.L + C * w.blk + max(w.k_group, w.blk)
+    P = int(round(w.prot_frac * cap)) * 2 + 64
+    ocs = []
+    for (b, h) in units:
+        oc = OracleCache(1, w.g, 1, w.d, w.blk, w.k_bits, w.v_bits, w.k_group, w.v_group, P, cap)
+        for i in range(nb):
+            Kb, Vb = synth.kv_block_bits(w, b, h, i)
+            oc.commit(Kb[None, None], Vb[None, None],
+                      synth.block_protect_words(w, b, h, i)[None, None])
+        ocs.append(oc)
+    blocks = {}
+    for (b, h) in units:
+        for c in range(C):
+            Kb, Vb = synth.kv_block_bits(w, b, h, nb + c)
+            blocks[(b, h, c)] = (Kb[None, None], Vb[None, None],
+                                 synth.block_protect_words(w, b, h, nb + c)[None, None])
+    q = synth.queries_bits(w, 0)
+    ka, va = synth.active_block_bits(w.with_(B=1, Hkv=1, Hq=w.g), 0)
+    U = w.B * w.Hkv
+    pos = 0
+    per_unit_bytes = 0.0
+    steps = 0
+    elapsed = 0.0
+    k = 0
+    while True:
+        if max_steps is not None and steps >= max_steps:
+            break
+        if max_steps is None and elapsed >= seconds and steps > 0:
+            break
+        L_before = w.L + pos * w.blk
+        t0 = time.perf_counter()
+        for (b, h), oc in zip(units, ocs):
+            oc.commit(*blocks[(b, h, pos)])
+            oc.block_attention(q[b:b + 1, h * w.g:(h + 1) * w.g], ka, va, w.softmax_scale)
+        dt = time.perf_counter() - t0
+        pos += 1
+        if pos == C:
+            for oc in ocs:
+                oc.truncate(w.L)
+            pos = 0
+        k += 1
+        if k <= warmup:
+            continue
+        elapsed += dt
+        steps += 1
+        per_unit_bytes += (attn_bytes(w, L_before + w.blk) + commit_bytes(w, L_before)) / U
+    gbs = per_unit_bytes * len(units) / elapsed / 1e9
+    desc = (f"{len(units)} of {U} (batch, kv-head) units x {steps} steps (commit + attention), "
+            f"L={w.L}; numpy/BLAS fp64")
+    return gbs, steps, elapsed, desc
+
+
+# ------------------------------------------------------------ main
+
+def base_line(w, args, value, ms_per_step, world):
+    return {
+        "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 6),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp16", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
+                   "L": w.L, "block": w.blk, "k_bits": w.k_bits, "v_bits": w.v_bits,
+                   "k_group": w.k_group, "v_group": w.v_group, "prot_frac": w.prot_frac,
+                   "parallelism": f"replicas{world}" if world > 1 else "single"},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=64)
+    ap.add_argument("--warmup", type=int, default=4)
+    ap.add_argument("--impl", choices=["dkv", "reference"], default="dkv")
+    ap.add_argument("--workload", default="mha8b", choices=list(synth.WORKLOADS))
+    ap.add_argument("--all-workloads", action="store_true",
+                    help="also run the other workloads and add a summary per workload")
+    ap.add_argument("--kernel", type=int, default=0, choices=[0, 1, 2],
+                    help="attention kernel: 0 = library's choice, 1 = mma.sync, 2 = tcgen05")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = _dist()
+    w = synth.WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        gbs, steps, el, desc = oracle_sample(w, 0, max_steps=args.steps, warmup=args.warmup)
+        line = base_line(w, args, gbs, el / max(steps, 1) * 1e3, world)
+        line["dtype"] = "f64"
+        line["impl"] = "reference"
+        cores = _blas_threads()
+        line["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": cores,
+                                "kind": "oracle", "sample": desc}
+        line["e2e"] = {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                       "d2h_bytes_per_step": 0}
+        print(json.dumps(line), flush=True)
+        return
+
+    import torch
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    peaks, peak_kind = load_peaks()
+    traffic = traffic_record()
+    r = run_gpu(w, args.steps, args.warmup, log=lambda *a: None, kernel=args.kernel)
+    line = base_line(w, args, r["value"], r["ms"] / args.steps, world)
+    line["config"]["L2_policy"] = (f"{r['R']} cache replicas used round-robin"
+                                   if r["R"] > 1 else "cache larger than L2")
+    line["config"]["L_mean"] = r["L_mean"]
+    line["config"]["step"] = (f"1 commit + 1 attention; truncate to L every {r['C']} steps; "
+                              "timed region = one CUDA graph replay of the steps")
+    line["roofline"] = roofline(w, r, peaks, peak_kind, traffic)
+    line["clocks"] = r["clocks"]
+    line["e2e"] = r["e2e"]
+    line["gpu_launches"] = r["graph_launches"]
+    line["attention_gbs"] = round(r["att_bytes"] / (r["att_ms"] / 1e3) / 1e9, 1)
+    line["pct_of_8tbs"] = round(100 * line["attention_gbs"] / 8000.0, 2)
+    line["commit_tokens_per_s"] = round(w.B * w.blk * r["commit_n"] / (r["commit_ms"] / 1e3), 1) \
+        if r["commit_ms"] > 0 else None
+    line["kernel_ms"] = {"attention": round(r["att_ms"] / max(r["att_n"], 1), 5),
+                         "combine": round(r["combine_ms"] / max(r["combine_n"], 1), 5),
+                         "commit": round(r["commit_ms"] / max(r["commit_n"], 1), 5)}
+    line["attention_plan"] = {"kernel": ["", "mma.sync", "tcgen05"][r["plan"][0]],
+                              "splits": r["plan"][1], "launches": r["plan"][2]}
+    if args.all_workloads:
+        line["workloads"] = {}
+        for name in synth.WORKLOAD_ORDER:
+            if name == w.name:
+                continue
+            ww = synth.WORKLOADS[name]
+            kern = args.kernel if (args.kernel != 2 or ww.rows == 128) else 0
+            rr = run_gpu(ww, min(args.steps, 16), args.warmup, want_e2e=False, kernel=kern)
+            rf = roofline(ww, rr, peaks, peak_kind, traffic)
+            line["workloads"][name] = {
+                "value_gbs": round(rr["value"], 1),
+                "attention_gbs": round(rr["att_bytes"] / (rr["att_ms"] / 1e3) / 1e9, 1),
+                "attention_us": round(rr["att_ms"] / max(rr["att_n"], 1) * 1e3, 2),
+                "roofline": {k: rf[k] for k in ("bound", "achieved", "peak", "unit", "frac")},
+                "commit_tokens_per_s": round(ww.B * ww.blk * rr["commit_n"] /
+                                             (rr["commit_ms"] / 1e3), 1),
+                "plan": rr["plan"], "clocks_sm_mhz": (rr["clocks"] or {}).get("sm_mhz")}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        gbs, steps, el, desc = oracle_sample(w, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": _blas_threads(),
+                                "kind": "oracle", "sample": desc}
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

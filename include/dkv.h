@@ -1,0 +1,198 @@
+/*
+ * libdkv -- quantize-on-commit and bidirectional block attention over a
+ * low-bit block-diffusion KV cache, for NVIDIA B200 (sm_100a).
+ *
+ * The operations follow three passages of the source pages:
+ *   - "SoloQ: Calibration-Free Quantization for Diffusion Language Models",
+ *     block-diffusion paragraph: KV entries are quantized only when a block
+ *     is committed, the block being denoised stays in full precision, and
+ *     keys use KIVI-style per-channel asymmetric quantization.
+ *   - "KV Cache Quantization for Diffusion Language Models" (Tai et al.,
+ *     Findings of EMNLP 2026), abstract: KIVI adapted to prefix-cache reuse;
+ *     KProtect keeps chosen K entries in high precision while V gets
+ *     standard low-bit quantization.
+ *   - MaskAhead / Q-MaskAhead abstract: block-diffusion models attend to the
+ *     cache at every denoising step, computing attention directly from the
+ *     low-bit KV.
+ *
+ * Quantizer of one group (b bits): s = fp16((max - min) / (2^b - 1)),
+ * z = fp16(min), q = clamp(rint((x - z) / s), 0, 2^b - 1), all fp32 with
+ * round-to-nearest-even; dequantized value q * s + z.  K groups are
+ * k_group consecutive tokens of one channel (positions aligned to 0); V
+ * groups are v_group consecutive channels of one token.  Protected K
+ * positions are left out of their group's min/max, get code 0, and keep
+ * their bf16 vector in a side table.
+ *
+ * Conventions for every call:
+ *   - Return value: DKV_OK (0) or a DKV_ERR_* code.  On an error detected on
+ *     the host no state changes and nothing is launched; dkv_last_error()
+ *     gives a message (thread-local, valid until the next call).
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Commit and
+ *     attention are asynchronous and stream-ordered; alloc, free, status and
+ *     export synchronize `stream`.
+ *   - Caller buffers are device memory (cudaMalloc or torch), contiguous,
+ *     16-byte aligned, bf16 = IEEE bfloat16 bit patterns.  The library keeps
+ *     no caller pointer past the call.  Calls on the current CUDA device,
+ *     which must be the one the cache was allocated on.
+ *   - Errors found while kernels run (protected side table full, committed
+ *     value out of fp16 range) are sticky flags read by dkv_cache_status.
+ */
+#ifndef DKV_H
+#define DKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  DKV_OK = 0,
+  DKV_ERR_INVALID_ARG = 1, /* NULL/misaligned pointer, bad size */
+  DKV_ERR_UNSUPPORTED = 2, /* shape or bit width outside the built set */
+  DKV_ERR_CAPACITY = 3,    /* len + block would exceed max_tokens */
+  DKV_ERR_CUDA = 4         /* a CUDA runtime call failed */
+};
+
+/* sticky device-side flags (dkv_cache_status) */
+enum {
+  DKV_FLAG_CAPACITY = 0x1, /* side table full: later protected tokens were quantized normally */
+  DKV_FLAG_RANGE = 0x2,    /* a committed K/V value was NaN/Inf or |x| > 65504; the
+                              quantizer used NaN -> 0 and clamped to +-65504 */
+  DKV_FLAG_TIMEOUT = 0x4   /* an attention CTA gave up waiting on one of its own
+                              pipeline stages (bounded wait, about 1 s); that call's
+                              output is undefined */
+};
+
+/* Cache shape.  Supported: head_dim == 128; block a multiple of 32, <= 128;
+ * q_heads a multiple of kv_heads with (q_heads/kv_heads)*block <= 256;
+ * k_bits, v_bits in {2, 4, 16} (16 = store bf16, quantization off);
+ * k_group in {32, 64, 128} with k_group % block == 0 or block % k_group == 0;
+ * v_group in {32, 64, 128}; max_tokens a multiple of max(k_group, block). */
+typedef struct dkv_config {
+  int32_t batch;         /* B: sequences (all share one committed length) */
+  int32_t q_heads;       /* Hq */
+  int32_t kv_heads;      /* Hkv; query head h reads kv-head h / (Hq/Hkv) */
+  int32_t head_dim;      /* d */
+  int32_t block;         /* blk: tokens per committed / active block */
+  int32_t k_bits;        /* bK */
+  int32_t v_bits;        /* bV */
+  int32_t k_group;       /* GK: tokens per K group (per channel) */
+  int32_t v_group;       /* GV: channels per V group (per token) */
+  int32_t max_protected; /* side-table capacity per (sequence, kv-head) */
+  int64_t max_tokens;    /* capacity per sequence */
+} dkv_config;
+
+typedef struct dkv_cache dkv_cache; /* opaque; owns its device memory */
+
+/* Allocate an empty cache (len = 0) on the current device.  Device memory is
+ * owned by the handle until dkv_cache_free.  Synchronizes `stream`. */
+int dkv_cache_alloc(const dkv_config* cfg, void* stream, dkv_cache** out);
+
+/* Release the handle and its device memory (synchronizes the device). */
+int dkv_cache_free(dkv_cache* cache);
+
+/* Commit one block: k, v are bf16 [B, Hkv, block, d]; protect_words is a
+ * device array uint32 [B, Hkv, block/32] whose bit t marks token t of the
+ * block as a protected K position, or NULL for none.  V is quantized per
+ * token at once; K tokens wait in a bf16 tail until their K group is
+ * complete, then the group is quantized.  len grows by `block` (host side,
+ * at once).  Returns DKV_ERR_CAPACITY if len + block > max_tokens. */
+int dkv_commit_block(dkv_cache* cache, const void* k, const void* v,
+                     const uint32_t* protect_words, void* stream);
+
+/* One denoising-step attention: q bf16 [B, Hq, block, d], the active block
+ * k_act, v_act bf16 [B, Hkv, block, d] (kept in full precision), out bf16
+ * [B, Hq, block, d].  Every query attends to every committed token and every
+ * active-block token (bidirectional, no mask): out = softmax(softmax_scale *
+ * q K^T) V with K, V the dequantized cache, the bf16 K tail and the active
+ * block; fp32 softmax, bf16 (round-to-nearest-even) output.  q, k_act,
+ * v_act must hold values within the fp16 range. */
+int dkv_block_attention(dkv_cache* cache, const void* q, const void* k_act,
+                        const void* v_act, float softmax_scale, void* out,
+                        void* stream);
+
+/* Roll the cache back to its first new_len committed tokens (for instance to
+ * reuse a shared prefix, the prefix-cache reuse of the Tai et al. abstract).
+ * new_len must be a multiple of `block` and, when k_bits < 16, of k_group, so
+ * that no incomplete K group remains; 0 <= new_len <= len.  The side table
+ * keeps the entries of the surviving groups.  Stream-ordered; len changes
+ * at once on the host. */
+int dkv_cache_truncate(dkv_cache* cache, int64_t new_len, void* stream);
+
+/* Committed tokens per sequence (host mirror, no synchronization). */
+int dkv_cache_len(const dkv_cache* cache, int64_t* len);
+
+/* Synchronize `stream`, return the sticky DKV_FLAG_* bits and clear them. */
+int dkv_cache_status(dkv_cache* cache, void* stream, uint32_t* flags);
+
+/* Host copies of the committed state in the canonical layout (U = B*Hkv
+ * units, u = b*Hkv + h; L = len; Lq = tokens whose K group is complete,
+ * = L when k_bits == 16; nG = Lq / k_group).  Every pointer is a host buffer
+ * owned by the caller, or NULL to skip that array.  Synchronizes `stream`.
+ *   k_codes   uint32 [U, nG, d, k_group*k_bits/32]  codes of one (group,
+ *             channel) packed along its tokens: token t at bits
+ *             [k_bits*t mod 32, +k_bits) of word k_bits*t/32
+ *   k_sz      uint16 [U, nG, d, 2]    fp16 (scale, zero) per (group, channel)
+ *   k_raw     uint16 [U, L, d]        bf16 K when k_bits == 16
+ *   k_tail    uint16 [U, L - Lq, d]   bf16 K of the incomplete group
+ *   tail_mask uint32 [U, ceil(k_group/32)]  protect bits of the tail slots
+ *   v_codes   uint32 [U, L, d*v_bits/32]    per token, packed along channels
+ *   v_sz      uint16 [U, L, d/v_group, 2]   fp16 (scale, zero)
+ *   v_raw     uint16 [U, L, d]        bf16 V when v_bits == 16
+ *   prot_count  int32 [U]             side-table entries in use
+ *   prot_pos    int32 [U, max_protected]    their positions, ascending
+ *               (unused slots: -1)
+ *   prot_k      uint16 [U, max_protected, d] their bf16 K vectors
+ *   prot_gstart int32 [U, nG + 1]     entries stored before group j */
+typedef struct dkv_export {
+  uint32_t* k_codes;
+  uint16_t* k_sz;
+  uint16_t* k_raw;
+  uint16_t* k_tail;
+  uint32_t* tail_mask;
+  uint32_t* v_codes;
+  uint16_t* v_sz;
+  uint16_t* v_raw;
+  int32_t* prot_count;
+  int32_t* prot_pos;
+  uint16_t* prot_k;
+  int32_t* prot_gstart;
+} dkv_export;
+
+int dkv_cache_export(dkv_cache* cache, void* stream, dkv_export* out);
+
+/* Tuning knobs (testing and benchmarking).  Values persist on the handle.
+ *   DKV_OPT_SPLITS: token splits per (sequence, kv-head) in attention;
+ *     0 = chosen from the SM count (default).  Results agree within fp32
+ *     rounding for any split count.
+ *   DKV_OPT_ATTN_KERNEL: 0 = best available (default), 1 = warp-level
+ *     mma.sync kernel, 2 = tcgen05 tensor-memory kernel (DKV_ERR_UNSUPPORTED
+ *     if the shape has no tcgen05 variant). */
+enum { DKV_OPT_SPLITS = 1, DKV_OPT_ATTN_KERNEL = 2, DKV_OPT_PROFILE = 3 };
+int dkv_cache_set_option(dkv_cache* cache, int32_t key, int64_t value);
+
+/* With DKV_OPT_PROFILE = 1, every kernel launch on this handle (outside CUDA
+ * graph capture) is bracketed by CUDA events recorded on its stream.  This
+ * call waits for them and returns, per kernel kind, the summed device time in
+ * milliseconds and the launch count since the last read, then resets them.
+ * kind: DKV_KERNEL_ATTENTION (the split attention kernel), DKV_KERNEL_COMBINE,
+ * DKV_KERNEL_COMMIT, DKV_KERNEL_TRUNCATE. */
+enum { DKV_KERNEL_ATTENTION = 0, DKV_KERNEL_COMBINE = 1, DKV_KERNEL_COMMIT = 2,
+       DKV_KERNEL_TRUNCATE = 3 };
+int dkv_profile_read(dkv_cache* cache, int32_t kind, double* total_ms, int64_t* launches);
+
+/* Launch description of the last dkv_block_attention on this handle: the
+ * kernel used (1 = mma.sync, 2 = tcgen05), its split count, and how many
+ * kernels it launched. */
+int dkv_last_attention_plan(const dkv_cache* cache, int32_t* kernel,
+                            int32_t* splits, int32_t* launches);
+
+/* Message of the last error on this thread ("" if none). */
+const char* dkv_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DKV_H */

@@ -306,6 +306,20 @@ class OracleCache:
         self.prot_gstart[u, j + 1] = count
         return flag
 
+    # -- roll back to an earlier prefix
+    def truncate(self, new_len: int) -> None:
+        """Drop the committed tokens [new_len, len): new_len must be a
+        multiple of the block and of the K group (so no incomplete group
+        remains).  The side table keeps the entries of the surviving groups."""
+        if new_len < 0 or new_len > self.len or new_len % self.blk:
+            raise ValueError("new_len must be a multiple of the block within [0, len]")
+        if self.kb < 16:
+            if new_len % self.GK:
+                raise ValueError("new_len must be a multiple of k_group")
+            self.prot_count[:] = self.prot_gstart[:, new_len // self.GK]
+            self.tail_prot[:] = False
+        self.len = new_len
+
     # -- dequantization (fp64)
     def dequant_k(self, u) -> np.ndarray:
         """K_hat [len, d] fp64 of unit u: quantized groups (protected rows

@@ -1,0 +1,280 @@
+// Quantize-on-commit ("KV entries are quantized only when a block is
+// committed; the block still being denoised stays in full precision; keys use
+// KIVI-style per-channel asymmetric quantization" -- SoloQ, block-diffusion
+// paragraph; protected K entries kept in high precision with standard low-bit
+// V -- "KV Cache Quantization for Diffusion Language Models", abstract).
+//
+// One CTA of 128 threads per (sequence, kv-head) unit.  V: one item per
+// (token, channel group).  K: thread c owns channel c of every K group that
+// this commit completes; tokens of an incomplete group wait in the bf16 tail.
+//
+// This file is compiled with -fmad=false and uses only correctly rounded fp32
+// operations (__fsub_rn, __fdiv_rn, __float2half_rn, __float2int_rn), so the
+// codes, scales and zero-points are bit-identical to any other IEEE fp32
+// evaluation of the same formulas.
+#include "dkv_internal.cuh"
+
+namespace dkv {
+namespace {
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) {
+  return __uint_as_float(uint32_t(b) << 16);
+}
+
+// NaN, +-Inf or beyond the fp16 range
+__device__ __forceinline__ bool out_of_range(float x) { return !(fabsf(x) <= 65504.f); }
+
+__device__ __forceinline__ float sanitize(float x) {
+  if (x != x) return 0.f;
+  return fminf(fmaxf(x, -65504.f), 65504.f);
+}
+
+struct GroupQuant {
+  float s32, z32;  // stored fp16 scale / zero, widened
+  __half2 sz;      // (scale, zero)
+};
+
+// s = fp16((mx - mn) / levels), z = fp16(mn)
+__device__ __forceinline__ GroupQuant make_quant(float mn, float mx, int levels) {
+  const float s_f = __fdiv_rn(__fsub_rn(mx, mn), float(levels));
+  const __half s = __float2half_rn(s_f);
+  const __half z = __float2half_rn(mn);
+  GroupQuant q;
+  q.s32 = __half2float(s);
+  q.z32 = __half2float(z);
+  q.sz = __halves2half2(s, z);
+  return q;
+}
+
+// q = clamp(rint((x - z) / s), 0, levels); 0 when s == 0
+__device__ __forceinline__ uint32_t code_of(float x, const GroupQuant& q, int levels) {
+  if (!(q.s32 > 0.f)) return 0u;
+  const float t = __fdiv_rn(__fsub_rn(x, q.z32), q.s32);
+  int c = __float2int_rn(t);
+  c = c < 0 ? 0 : (c > levels ? levels : c);
+  return uint32_t(c);
+}
+
+constexpr int kThreads = 128;
+
+template <int KB, int VB>
+__global__ void __launch_bounds__(kThreads)
+commit_kernel(CacheView c, const uint16_t* __restrict__ k, const uint16_t* __restrict__ v,
+              const uint32_t* __restrict__ pw, int64_t p0) {
+  const int u = blockIdx.x;
+  const int tid = threadIdx.x;
+  const int d = kHeadDim;
+  const int blk = c.blk;
+  const uint16_t* ku = k + size_t(u) * blk * d;
+  const uint16_t* vu = v + size_t(u) * blk * d;
+  const int nbw = blk / 32;
+  bool range = false;
+
+  // ------------------------------------------------------------------ V
+  if constexpr (VB == 16) {
+    const uint4* src = reinterpret_cast<const uint4*>(vu);
+    uint4* dst = reinterpret_cast<uint4*>(c.v_raw + (size_t(u) * c.cap + p0) * d);
+    for (int i = tid; i < blk * d / 8; i += kThreads) {
+      const uint4 x = src[i];
+      const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        range |= out_of_range(bf16_bits_to_f32(uint16_t(w[j] & 0xFFFF)));
+        range |= out_of_range(bf16_bits_to_f32(uint16_t(w[j] >> 16)));
+      }
+      dst[i] = x;
+    }
+  } else {
+    constexpr int levels = (1 << VB) - 1;
+    constexpr int per = 32 / VB;
+    const int GV = c.GV;
+    const int ngr = d / GV;
+    for (int it = tid; it < blk * ngr; it += kThreads) {
+      const int t = it / ngr, gi = it % ngr;
+      const uint16_t* x = vu + t * d + gi * GV;
+      float mn = __int_as_float(0x7f800000), mx = -__int_as_float(0x7f800000);
+      for (int i = 0; i < GV; ++i) {
+        float f = bf16_bits_to_f32(x[i]);
+        range |= out_of_range(f);
+        f = sanitize(f);
+        mn = fminf(mn, f);
+        mx = fmaxf(mx, f);
+      }
+      const GroupQuant q = make_quant(mn, mx, levels);
+      uint32_t* dst = c.v_codes + (size_t(u) * c.cap + p0 + t) * c.vw + gi * GV / per;
+      for (int w = 0; w < GV / per; ++w) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int e = 0; e < per; ++e)
+          word |= code_of(sanitize(bf16_bits_to_f32(x[w * per + e])), q, levels) << (e * VB);
+        dst[w] = word;
+      }
+      c.v_sz[(size_t(u) * c.cap + p0 + t) * ngr + gi] = q.sz;
+    }
+  }
+
+  // ------------------------------------------------------------------ K
+  if constexpr (KB == 16) {
+    const uint4* src = reinterpret_cast<const uint4*>(ku);
+    uint4* dst = reinterpret_cast<uint4*>(c.k_raw + (size_t(u) * c.cap + p0) * d);
+    for (int i = tid; i < blk * d / 8; i += kThreads) {
+      const uint4 x = src[i];
+      const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        range |= out_of_range(bf16_bits_to_f32(uint16_t(w[j] & 0xFFFF)));
+        range |= out_of_range(bf16_bits_to_f32(uint16_t(w[j] >> 16)));
+      }
+      dst[i] = x;
+    }
+  } else {
+    constexpr int levels = (1 << KB) - 1;
+    constexpr int per = 32 / KB;
+    const int GK = c.GK;
+    const int n_tail = int(p0 % GK);
+    uint16_t* tail = c.k_tail + size_t(u) * GK * d;
+    uint32_t* tmask = c.tail_mask + size_t(u) * c.twords;
+    if (n_tail + blk < GK) {
+      // the group stays incomplete: append the block to the bf16 tail
+      const uint4* src = reinterpret_cast<const uint4*>(ku);
+      uint4* dst = reinterpret_cast<uint4*>(tail + size_t(n_tail) * d);
+      for (int i = tid; i < blk * d / 8; i += kThreads) {
+        const uint4 x = src[i];
+        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          range |= out_of_range(bf16_bits_to_f32(uint16_t(w[j] & 0xFFFF)));
+          range |= out_of_range(bf16_bits_to_f32(uint16_t(w[j] >> 16)));
+        }
+        dst[i] = x;
+      }
+      if (tid < nbw) tmask[n_tail / 32 + tid] = pw ? pw[size_t(u) * nbw + tid] : 0u;
+    } else {
+      // pending stream = tail[0, n_tail) ++ block[0, blk); quantize every
+      // complete group (k_group and block divide one another, so nothing is
+      // left over)
+      const int npend = n_tail + blk;
+      const int nfull = npend / GK;
+      const int ch = tid;  // channel
+      auto pend_raw = [&](int pt) -> uint16_t {
+        return pt < n_tail ? tail[size_t(pt) * d + ch] : ku[size_t(pt - n_tail) * d + ch];
+      };
+      int count = c.prot_count[u];
+      const int64_t j0 = (p0 - n_tail) / GK;
+      for (int gi = 0; gi < nfull; ++gi) {
+        const int64_t j = j0 + gi;
+        uint32_t gm[4] = {0u, 0u, 0u, 0u};
+        for (int w = 0; w < GK / 32; ++w) {
+          const int pwi = gi * GK / 32 + w;  // word of the pending stream
+          if (pwi < n_tail / 32)
+            gm[w] = tmask[pwi];
+          else
+            gm[w] = pw ? pw[size_t(u) * nbw + (pwi - n_tail / 32)] : 0u;
+        }
+        // side table full: keep the first `room` protected tokens by position
+        int want = 0;
+        for (int w = 0; w < GK / 32; ++w) want += __popc(gm[w]);
+        const int room = c.P - count;
+        if (want > room) {
+          int kept = 0;
+          for (int w = 0; w < GK / 32; ++w) {
+            uint32_t m = gm[w], nm = 0u;
+            while (m && kept < room) {
+              const uint32_t low = m & (0u - m);
+              nm |= low;
+              m ^= low;
+              ++kept;
+            }
+            gm[w] = nm;
+          }
+          if (tid == 0) atomicOr(c.status, uint32_t(DKV_FLAG_CAPACITY));
+        }
+        // min / max over the group's non-protected tokens of channel ch
+        float mn = __int_as_float(0x7f800000), mx = -__int_as_float(0x7f800000);
+        for (int t = 0; t < GK; ++t) {
+          const int pt = gi * GK + t;
+          float f = bf16_bits_to_f32(pend_raw(pt));
+          if (pt >= n_tail) range |= out_of_range(f);
+          f = sanitize(f);
+          if (!((gm[t >> 5] >> (t & 31)) & 1u)) {
+            mn = fminf(mn, f);
+            mx = fmaxf(mx, f);
+          }
+        }
+        if (mn > mx) mn = mx = 0.f;  // every token protected
+        const GroupQuant q = make_quant(mn, mx, levels);
+        uint32_t* dst = c.k_codes + ((size_t(u) * c.nG + j) * d + ch) * c.kw;
+        for (int w = 0; w < GK / per; ++w) {
+          uint32_t word = 0;
+          for (int e = 0; e < per; ++e) {
+            const int t = w * per + e;
+            if ((gm[t >> 5] >> (t & 31)) & 1u) continue;  // protected slot: code 0
+            word |= code_of(sanitize(bf16_bits_to_f32(pend_raw(gi * GK + t))), q, levels) << (e * KB);
+          }
+          dst[w] = word;
+        }
+        c.k_sz[(size_t(u) * c.nG + j) * d + ch] = q.sz;
+        // side-table entries, ascending positions
+        for (int w = 0; w < GK / 32; ++w) {
+          uint32_t m = gm[w];
+          while (m) {
+            const int b = __ffs(m) - 1;
+            m &= m - 1u;
+            const int t = w * 32 + b;
+            if (tid == 0) c.prot_pos[size_t(u) * c.P + count] = int32_t(j * GK + t);
+            c.prot_k[(size_t(u) * c.P + count) * d + ch] = pend_raw(gi * GK + t);
+            ++count;
+          }
+        }
+        if (tid == 0) c.prot_gstart[size_t(u) * (c.nG + 1) + j + 1] = count;
+      }
+      if (tid == 0) c.prot_count[u] = count;
+      if (tid < c.twords) tmask[tid] = 0u;
+    }
+  }
+  if (range) atomicOr(c.status, uint32_t(DKV_FLAG_RANGE));
+}
+
+// Roll back to new_len (a multiple of the K group): the side table keeps the
+// entries stored before group new_len / GK; the tail is empty.
+__global__ void truncate_kernel(CacheView c, int64_t new_len) {
+  const int u = blockIdx.x * blockDim.x + threadIdx.x;
+  if (u >= c.U) return;
+  c.prot_count[u] = c.prot_gstart[size_t(u) * (c.nG + 1) + new_len / c.GK];
+  for (int w = 0; w < c.twords; ++w) c.tail_mask[size_t(u) * c.twords + w] = 0u;
+}
+
+template <int KB, int VB>
+cudaError_t launch_kv(const CacheView& c, const uint16_t* k, const uint16_t* v,
+                      const uint32_t* pw, int64_t p0, cudaStream_t s) {
+  commit_kernel<KB, VB><<<c.U, kThreads, 0, s>>>(c, k, v, pw, p0);
+  return cudaGetLastError();
+}
+
+template <int KB>
+cudaError_t launch_k(const CacheView& c, const uint16_t* k, const uint16_t* v,
+                     const uint32_t* pw, int64_t p0, cudaStream_t s) {
+  switch (c.vb) {
+    case 2: return launch_kv<KB, 2>(c, k, v, pw, p0, s);
+    case 4: return launch_kv<KB, 4>(c, k, v, pw, p0, s);
+    default: return launch_kv<KB, 16>(c, k, v, pw, p0, s);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_truncate(const CacheView& c, int64_t new_len, cudaStream_t s) {
+  truncate_kernel<<<(c.U + 127) / 128, 128, 0, s>>>(c, new_len);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_commit(const CacheView& c, const uint16_t* k, const uint16_t* v,
+                          const uint32_t* pw, int64_t p0, cudaStream_t s) {
+  switch (c.kb) {
+    case 2: return launch_k<2>(c, k, v, pw, p0, s);
+    case 4: return launch_k<4>(c, k, v, pw, p0, s);
+    default: return launch_k<16>(c, k, v, pw, p0, s);
+  }
+}
+
+}  // namespace dkv

@@ -1,0 +1,107 @@
+// Packed-code -> fp16 conversion used by the attention kernels.
+//
+// A 4-bit word holds 8 codes (element e at bits 4e), a 2-bit word 16 codes
+// (element e at bits 2e).  Codes are moved into the low mantissa bits of the
+// fp16 constant 1024 (bit pattern 0x6400, whose ulp is 1), giving 1024 + c or
+// 1024 + 2^k c exactly; one fp16 fma removes the offset and the 2^k factor
+// exactly, and a second fp16 fma gives q * s + z with a single rounding.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+namespace dkv {
+
+__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t mask, uint32_t bits) {
+  uint32_t r;  // (a & mask) | bits
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(a), "r"(mask), "r"(bits));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
+}
+
+__device__ __forceinline__ __half2 u2h(uint32_t x) { return *reinterpret_cast<__half2*>(&x); }
+__device__ __forceinline__ uint32_t h2u(__half2 x) { return *reinterpret_cast<uint32_t*>(&x); }
+
+__device__ __forceinline__ __half2 h2c(float a) { return __float2half2_rn(a); }
+
+constexpr uint32_t kMagic1024 = 0x64006400u;
+
+// (1024 + 2^k c) -> c, exactly
+__device__ __forceinline__ __half2 unbias(uint32_t x, float inv, float off) {
+  return __hfma2(u2h(x), h2c(inv), h2c(off));
+}
+
+// 8 four-bit codes -> 8 halves q*s+z, element order
+__device__ __forceinline__ uint4 dequant4x8(uint32_t w, __half2 s2, __half2 z2) {
+  const uint32_t w8 = w >> 8;
+  const __half2 n04 = unbias(and_or(w, 0x000F000Fu, kMagic1024), 1.f, -1024.f);
+  const __half2 n15 = unbias(and_or(w, 0x00F000F0u, kMagic1024), 0.0625f, -64.f);
+  const __half2 n26 = unbias(and_or(w8, 0x000F000Fu, kMagic1024), 1.f, -1024.f);
+  const __half2 n37 = unbias(and_or(w8, 0x00F000F0u, kMagic1024), 0.0625f, -64.f);
+  const uint32_t v04 = h2u(__hfma2(n04, s2, z2));
+  const uint32_t v15 = h2u(__hfma2(n15, s2, z2));
+  const uint32_t v26 = h2u(__hfma2(n26, s2, z2));
+  const uint32_t v37 = h2u(__hfma2(n37, s2, z2));
+  uint4 r;
+  r.x = prmt(v04, v15, 0x5410);  // e0 e1
+  r.y = prmt(v26, v37, 0x5410);  // e2 e3
+  r.z = prmt(v04, v15, 0x7632);  // e4 e5
+  r.w = prmt(v26, v37, 0x7632);  // e6 e7
+  return r;
+}
+
+// 16 two-bit codes -> 16 halves q*s+z, element order (lo = e0..e7, hi = e8..e15)
+__device__ __forceinline__ void dequant2x16(uint32_t w, __half2 s2, __half2 z2, uint4& lo,
+                                            uint4& hi) {
+  const uint32_t w8 = w >> 8;
+  uint32_t v[8];
+  v[0] = h2u(__hfma2(unbias(and_or(w, 0x00030003u, kMagic1024), 1.f, -1024.f), s2, z2));
+  v[1] = h2u(__hfma2(unbias(and_or(w, 0x000C000Cu, kMagic1024), 0.25f, -256.f), s2, z2));
+  v[2] = h2u(__hfma2(unbias(and_or(w, 0x00300030u, kMagic1024), 0.0625f, -64.f), s2, z2));
+  v[3] = h2u(__hfma2(unbias(and_or(w, 0x00C000C0u, kMagic1024), 0.015625f, -16.f), s2, z2));
+  v[4] = h2u(__hfma2(unbias(and_or(w8, 0x00030003u, kMagic1024), 1.f, -1024.f), s2, z2));
+  v[5] = h2u(__hfma2(unbias(and_or(w8, 0x000C000Cu, kMagic1024), 0.25f, -256.f), s2, z2));
+  v[6] = h2u(__hfma2(unbias(and_or(w8, 0x00300030u, kMagic1024), 0.0625f, -64.f), s2, z2));
+  v[7] = h2u(__hfma2(unbias(and_or(w8, 0x00C000C0u, kMagic1024), 0.015625f, -16.f), s2, z2));
+  // v[i] = (e_i, e_{i+8})
+  lo.x = prmt(v[0], v[1], 0x5410);
+  lo.y = prmt(v[2], v[3], 0x5410);
+  lo.z = prmt(v[4], v[5], 0x5410);
+  lo.w = prmt(v[6], v[7], 0x5410);
+  hi.x = prmt(v[0], v[1], 0x7632);
+  hi.y = prmt(v[2], v[3], 0x7632);
+  hi.z = prmt(v[4], v[5], 0x7632);
+  hi.w = prmt(v[6], v[7], 0x7632);
+}
+
+// 8 bf16 -> 8 fp16 (exact inside fp16's normal range)
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 x) {
+  auto cvt = [](uint32_t w) -> uint32_t {
+    const float a = __uint_as_float(w << 16);
+    const float b = __uint_as_float(w & 0xFFFF0000u);
+    return h2u(__floats2half2_rn(a, b));
+  };
+  uint4 r;
+  r.x = cvt(x.x);
+  r.y = cvt(x.y);
+  r.z = cvt(x.z);
+  r.w = cvt(x.w);
+  return r;
+}
+
+__device__ __forceinline__ __half bf16_to_half(uint16_t b) {
+  return __float2half_rn(__uint_as_float(uint32_t(b) << 16));
+}
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+}  // namespace dkv

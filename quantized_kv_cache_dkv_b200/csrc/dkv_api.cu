@@ -1,0 +1,455 @@
+// C-ABI entry points of libdkv: argument checks, device memory, split
+// planning and kernel launches.  Every step of the path runs in the kernels
+// of commit.cu, attn_mma.cu and attn_tc.cu; this file only plans and launches.
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "dkv_internal.cuh"
+
+namespace {
+// CUDA events bracketing kernel launches (DKV_OPT_PROFILE)
+struct ProfRecord {
+  cudaEvent_t start, stop;
+  int kind;
+};
+}  // namespace
+
+struct dkv_cache {
+  dkv_config cfg;
+  dkv::CacheView v;
+  int device = 0;
+  int num_sms = 148;
+  int64_t len = 0;
+  void* arena = nullptr;
+  size_t arena_bytes = 0;
+  float* part_o = nullptr;
+  float2* part_ml = nullptr;
+  int32_t max_splits = 1;
+  int32_t opt_splits = 0;
+  int32_t opt_kernel = 0;
+  int32_t last_kernel = 0, last_splits = 0, last_launches = 0;
+  bool profile = false;
+  std::vector<ProfRecord> prof;  // event pool; the first prof_used are pending
+  size_t prof_used = 0;
+};
+
+namespace {
+
+thread_local std::string g_err;
+
+int fail(int code, const std::string& msg) {
+  g_err = msg;
+  return code;
+}
+
+#define DKV_CUDA(expr)                                                              \
+  do {                                                                              \
+    cudaError_t e_ = (expr);                                                        \
+    if (e_ != cudaSuccess)                                                          \
+      return fail(DKV_ERR_CUDA, std::string(#expr) + ": " + cudaGetErrorString(e_)); \
+  } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+int check_config(const dkv_config* c) {
+  if (!c) return fail(DKV_ERR_INVALID_ARG, "config is NULL");
+  if (c->batch < 1 || c->q_heads < 1 || c->kv_heads < 1 || c->head_dim < 1 || c->block < 1 ||
+      c->max_tokens < 1 || c->max_protected < 0)
+    return fail(DKV_ERR_INVALID_ARG, "non-positive size in config");
+  if (c->q_heads % c->kv_heads)
+    return fail(DKV_ERR_INVALID_ARG, "q_heads must be a multiple of kv_heads");
+  if (c->head_dim != dkv::kHeadDim) return fail(DKV_ERR_UNSUPPORTED, "head_dim must be 128");
+  if (c->block % 32 || c->block > 128)
+    return fail(DKV_ERR_UNSUPPORTED, "block must be a multiple of 32 and <= 128");
+  if ((c->q_heads / c->kv_heads) * c->block > 256)
+    return fail(DKV_ERR_UNSUPPORTED, "(q_heads/kv_heads)*block must be <= 256");
+  auto okbits = [](int b) { return b == 2 || b == 4 || b == 16; };
+  if (!okbits(c->k_bits) || !okbits(c->v_bits))
+    return fail(DKV_ERR_UNSUPPORTED, "k_bits/v_bits must be 2, 4 or 16");
+  auto okgrp = [](int g) { return g == 32 || g == 64 || g == 128; };
+  if (c->k_bits < 16) {
+    if (!okgrp(c->k_group)) return fail(DKV_ERR_UNSUPPORTED, "k_group must be 32, 64 or 128");
+    if (c->k_group % c->block && c->block % c->k_group)
+      return fail(DKV_ERR_UNSUPPORTED, "k_group and block must divide one another");
+  }
+  if (c->v_bits < 16 && !okgrp(c->v_group))
+    return fail(DKV_ERR_UNSUPPORTED, "v_group must be 32, 64 or 128");
+  int64_t unit = c->block;
+  if (c->k_bits < 16) unit = std::max<int64_t>(unit, c->k_group);
+  if (c->max_tokens % unit)
+    return fail(DKV_ERR_INVALID_ARG, "max_tokens must be a multiple of max(k_group, block)");
+  if (c->max_tokens > (int64_t(1) << 30))
+    return fail(DKV_ERR_INVALID_ARG, "max_tokens too large (limit 2^30)");
+  return DKV_OK;
+}
+
+// Runs `launch` on stream s; when profiling (and s is not capturing a graph)
+// records a pair of events around it.
+template <class F>
+cudaError_t timed_launch(dkv_cache* c, int kind, cudaStream_t s, F&& launch) {
+  bool rec = c->profile;
+  if (rec) {
+    cudaStreamCaptureStatus st = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &st) != cudaSuccess || st != cudaStreamCaptureStatusNone) rec = false;
+  }
+  if (!rec) return launch();
+  if (c->prof_used == c->prof.size()) {
+    ProfRecord r{};
+    cudaError_t e = cudaEventCreate(&r.start);
+    if (e == cudaSuccess) e = cudaEventCreate(&r.stop);
+    if (e != cudaSuccess) return e;
+    c->prof.push_back(r);
+  }
+  ProfRecord& r = c->prof[c->prof_used++];
+  r.kind = kind;
+  cudaError_t e = cudaEventRecord(r.start, s);
+  if (e == cudaSuccess) e = launch();
+  if (e == cudaSuccess) e = cudaEventRecord(r.stop, s);
+  return e;
+}
+
+int split_cap(int U, int sms) {
+  int64_t s = ceil_div(int64_t(8) * sms, U);
+  return int(std::min<int64_t>(64, std::max<int64_t>(4, s)));
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* dkv_last_error(void) { return g_err.c_str(); }
+
+int dkv_cache_alloc(const dkv_config* cfg, void* stream, dkv_cache** out) {
+  g_err.clear();
+  if (!out) return fail(DKV_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  int rc = check_config(cfg);
+  if (rc) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  dkv_cache* c = new (std::nothrow) dkv_cache();
+  if (!c) return fail(DKV_ERR_INVALID_ARG, "host allocation failed");
+  c->cfg = *cfg;
+  dkv::CacheView& v = c->v;
+  v.B = cfg->batch;
+  v.Hq = cfg->q_heads;
+  v.Hkv = cfg->kv_heads;
+  v.d = cfg->head_dim;
+  v.blk = cfg->block;
+  v.g = v.Hq / v.Hkv;
+  v.rows = v.g * v.blk;
+  v.kb = cfg->k_bits;
+  v.vb = cfg->v_bits;
+  v.GK = cfg->k_bits < 16 ? cfg->k_group : cfg->block;
+  v.GV = cfg->v_bits < 16 ? cfg->v_group : 32;
+  v.P = cfg->k_bits < 16 ? cfg->max_protected : 0;
+  v.cap = cfg->max_tokens;
+  v.nG = v.cap / v.GK;
+  v.kw = v.kb < 16 ? v.GK * v.kb / 32 : 0;
+  v.vw = v.vb < 16 ? v.d * v.vb / 32 : 0;
+  v.vgroups = v.d / v.GV;
+  v.twords = (v.GK + 31) / 32;
+  v.U = v.B * v.Hkv;
+  const size_t U = size_t(v.U);
+
+  cudaError_t e = cudaGetDevice(&c->device);
+  if (e == cudaSuccess)
+    e = cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, c->device);
+  if (e != cudaSuccess) {
+    delete c;
+    return fail(DKV_ERR_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(e));
+  }
+  c->max_splits = split_cap(v.U, c->num_sms);
+
+  // one arena; 256-byte aligned regions
+  struct Region { size_t off, bytes; };
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    Region r{off, bytes};
+    off = align256(off + bytes);
+    return r;
+  };
+  const bool kq = v.kb < 16, vq = v.vb < 16;
+  Region r_kc = take(kq ? U * v.nG * v.d * v.kw * 4 : 0);
+  Region r_ksz = take(kq ? U * v.nG * v.d * 4 : 0);
+  Region r_kraw = take(kq ? 0 : U * v.cap * v.d * 2);
+  Region r_tail = take(kq ? U * v.GK * v.d * 2 : 0);
+  Region r_tm = take(U * v.twords * 4);
+  Region r_vc = take(vq ? U * v.cap * v.vw * 4 : 0);
+  Region r_vsz = take(vq ? U * v.cap * v.vgroups * 4 : 0);
+  Region r_vraw = take(vq ? 0 : U * v.cap * v.d * 2);
+  Region r_pc = take(U * 4);
+  Region r_pp = take(U * size_t(v.P) * 4);
+  Region r_pk = take(U * size_t(v.P) * v.d * 2);
+  Region r_pg = take(U * (v.nG + 1) * 4);
+  Region r_st = take(4);
+  Region r_po = take(U * size_t(c->max_splits) * v.rows * v.d * 4);
+  Region r_pml = take(U * size_t(c->max_splits) * v.rows * 8);
+  c->arena_bytes = off;
+
+  e = cudaMalloc(&c->arena, c->arena_bytes);
+  if (e != cudaSuccess) {
+    delete c;
+    return fail(DKV_ERR_CUDA, std::string("cudaMalloc: ") + cudaGetErrorString(e));
+  }
+  char* base = static_cast<char*>(c->arena);
+  auto at = [&](const Region& r) -> void* { return r.bytes ? base + r.off : nullptr; };
+  v.k_codes = static_cast<uint32_t*>(at(r_kc));
+  v.k_sz = static_cast<__half2*>(at(r_ksz));
+  v.k_raw = static_cast<uint16_t*>(at(r_kraw));
+  v.k_tail = static_cast<uint16_t*>(at(r_tail));
+  v.tail_mask = static_cast<uint32_t*>(at(r_tm));
+  v.v_codes = static_cast<uint32_t*>(at(r_vc));
+  v.v_sz = static_cast<__half2*>(at(r_vsz));
+  v.v_raw = static_cast<uint16_t*>(at(r_vraw));
+  v.prot_count = static_cast<int32_t*>(at(r_pc));
+  v.prot_pos = static_cast<int32_t*>(at(r_pp));
+  v.prot_k = static_cast<uint16_t*>(at(r_pk));
+  v.prot_gstart = static_cast<int32_t*>(at(r_pg));
+  v.status = static_cast<uint32_t*>(at(r_st));
+  c->part_o = static_cast<float*>(at(r_po));
+  c->part_ml = static_cast<float2*>(at(r_pml));
+
+  // zero everything that carries state (counters, masks, status) -- and the
+  // rest, so exports of unused slots are deterministic; prot_pos unused = -1
+  e = cudaMemsetAsync(c->arena, 0, r_po.off, s);
+  if (e == cudaSuccess && r_pp.bytes) e = cudaMemsetAsync(base + r_pp.off, 0xFF, r_pp.bytes, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) {
+    cudaFree(c->arena);
+    delete c;
+    return fail(DKV_ERR_CUDA, std::string("cache init: ") + cudaGetErrorString(e));
+  }
+  *out = c;
+  return DKV_OK;
+}
+
+int dkv_cache_free(dkv_cache* c) {
+  g_err.clear();
+  if (!c) return fail(DKV_ERR_INVALID_ARG, "cache is NULL");
+  cudaError_t e = cudaDeviceSynchronize();
+  cudaError_t e2 = cudaFree(c->arena);
+  for (auto& r : c->prof) {
+    cudaEventDestroy(r.start);
+    cudaEventDestroy(r.stop);
+  }
+  delete c;
+  if (e != cudaSuccess) return fail(DKV_ERR_CUDA, std::string("sync: ") + cudaGetErrorString(e));
+  if (e2 != cudaSuccess) return fail(DKV_ERR_CUDA, std::string("cudaFree: ") + cudaGetErrorString(e2));
+  return DKV_OK;
+}
+
+int dkv_cache_len(const dkv_cache* c, int64_t* len) {
+  g_err.clear();
+  if (!c || !len) return fail(DKV_ERR_INVALID_ARG, "NULL argument");
+  *len = c->len;
+  return DKV_OK;
+}
+
+int dkv_cache_truncate(dkv_cache* c, int64_t new_len, void* stream) {
+  g_err.clear();
+  if (!c) return fail(DKV_ERR_INVALID_ARG, "cache is NULL");
+  if (new_len < 0 || new_len > c->len || new_len % c->v.blk)
+    return fail(DKV_ERR_INVALID_ARG, "new_len must be a multiple of block within [0, len]");
+  if (c->v.kb < 16) {
+    if (new_len % c->v.GK) return fail(DKV_ERR_INVALID_ARG, "new_len must be a multiple of k_group");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = timed_launch(c, DKV_KERNEL_TRUNCATE, s,
+                                 [&] { return dkv::launch_truncate(c->v, new_len, s); });
+    if (e != cudaSuccess)
+      return fail(DKV_ERR_CUDA, std::string("truncate launch: ") + cudaGetErrorString(e));
+  }
+  c->len = new_len;
+  return DKV_OK;
+}
+
+int dkv_commit_block(dkv_cache* c, const void* k, const void* v, const uint32_t* protect_words,
+                     void* stream) {
+  g_err.clear();
+  if (!c || !k || !v) return fail(DKV_ERR_INVALID_ARG, "NULL cache, k or v");
+  if (!aligned16(k) || !aligned16(v) ||
+      (reinterpret_cast<uintptr_t>(protect_words) & 3u))
+    return fail(DKV_ERR_INVALID_ARG, "k and v must be 16-byte aligned, protect_words 4-byte");
+  if (c->len + c->v.blk > c->v.cap)
+    return fail(DKV_ERR_CAPACITY, "len + block exceeds max_tokens");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = timed_launch(c, DKV_KERNEL_COMMIT, s, [&] {
+    return dkv::launch_commit(c->v, static_cast<const uint16_t*>(k),
+                              static_cast<const uint16_t*>(v), protect_words, c->len, s);
+  });
+  if (e != cudaSuccess) return fail(DKV_ERR_CUDA, std::string("commit launch: ") + cudaGetErrorString(e));
+  c->len += c->v.blk;
+  return DKV_OK;
+}
+
+int dkv_block_attention(dkv_cache* c, const void* q, const void* k_act, const void* v_act,
+                        float softmax_scale, void* out, void* stream) {
+  g_err.clear();
+  if (!c || !q || !k_act || !v_act || !out) return fail(DKV_ERR_INVALID_ARG, "NULL argument");
+  if (!aligned16(q) || !aligned16(k_act) || !aligned16(v_act) || !aligned16(out))
+    return fail(DKV_ERR_INVALID_ARG, "q, k_act, v_act and out must be 16-byte aligned");
+  if (!(softmax_scale == softmax_scale) || softmax_scale > 3.0e38f || softmax_scale < -3.0e38f)
+    return fail(DKV_ERR_INVALID_ARG, "softmax_scale must be finite");
+  const dkv::CacheView& v = c->v;
+  dkv::AttnArgs a{};
+  a.c = v;
+  a.q = static_cast<const uint16_t*>(q);
+  a.k_act = static_cast<const uint16_t*>(k_act);
+  a.v_act = static_cast<const uint16_t*>(v_act);
+  a.out = static_cast<uint16_t*>(out);
+  a.part_o = c->part_o;
+  a.part_ml = c->part_ml;
+  a.scale_log2 = softmax_scale * 1.4426950408889634f;
+  a.L = c->len;
+  a.Lq = v.kb < 16 ? (c->len / v.GK) * v.GK : c->len;
+  a.n_tok = c->len + v.blk;
+
+  int kernel = c->opt_kernel;
+  if (kernel == 0) kernel = dkv::tc_supported(v) ? 2 : 1;
+  if (kernel == 2 && !dkv::tc_supported(v))
+    return fail(DKV_ERR_UNSUPPORTED, "no tcgen05 attention variant for this shape");
+  const int tile = kernel == 2 ? dkv::kTcTile : dkv::kMmaTile;
+  const int64_t n_tiles = ceil_div(a.n_tok, tile);
+  int64_t ns;
+  if (c->opt_splits > 0) {
+    ns = c->opt_splits;
+  } else {
+    // enough CTAs for two waves over the SMs, each split at least 2 tiles
+    ns = ceil_div(int64_t(2) * c->num_sms, v.U);
+    ns = std::min<int64_t>(ns, std::max<int64_t>(1, n_tiles / 2));
+  }
+  ns = std::max<int64_t>(1, std::min<int64_t>({ns, n_tiles, c->max_splits}));
+  const int64_t tps = ceil_div(n_tiles, ns);
+  ns = ceil_div(n_tiles, tps);  // no empty split
+  a.nsplit = int(ns);
+  a.tiles_per_split = int(tps);
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = timed_launch(c, DKV_KERNEL_ATTENTION, s, [&] {
+    return kernel == 2 ? dkv::launch_attention_tc(a, s) : dkv::launch_attention_mma(a, s);
+  });
+  if (e != cudaSuccess) return fail(DKV_ERR_CUDA, std::string("attention launch: ") + cudaGetErrorString(e));
+  int launches = 1;
+  if (a.nsplit > 1) {
+    e = timed_launch(c, DKV_KERNEL_COMBINE, s, [&] { return dkv::launch_combine(a, s); });
+    if (e != cudaSuccess) return fail(DKV_ERR_CUDA, std::string("combine launch: ") + cudaGetErrorString(e));
+    launches = 2;
+  }
+  c->last_kernel = kernel;
+  c->last_splits = a.nsplit;
+  c->last_launches = launches;
+  return DKV_OK;
+}
+
+int dkv_cache_status(dkv_cache* c, void* stream, uint32_t* flags) {
+  g_err.clear();
+  if (!c || !flags) return fail(DKV_ERR_INVALID_ARG, "NULL argument");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  DKV_CUDA(cudaStreamSynchronize(s));
+  DKV_CUDA(cudaMemcpy(flags, c->v.status, 4, cudaMemcpyDeviceToHost));
+  DKV_CUDA(cudaMemset(c->v.status, 0, 4));
+  return DKV_OK;
+}
+
+int dkv_cache_export(dkv_cache* c, void* stream, dkv_export* o) {
+  g_err.clear();
+  if (!c || !o) return fail(DKV_ERR_INVALID_ARG, "NULL argument");
+  const dkv::CacheView& v = c->v;
+  DKV_CUDA(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+  const int64_t L = c->len;
+  const int64_t Lq = v.kb < 16 ? (L / v.GK) * v.GK : L;
+  const int64_t nGq = v.kb < 16 ? Lq / v.GK : 0;
+  const size_t U = size_t(v.U);
+  auto copy2d = [&](void* dst, const void* src, size_t width, size_t pitch) -> cudaError_t {
+    if (!dst || !src || width == 0) return cudaSuccess;
+    return cudaMemcpy2D(dst, width, src, pitch, width, U, cudaMemcpyDeviceToHost);
+  };
+  if (v.kb < 16) {
+    DKV_CUDA(copy2d(o->k_codes, v.k_codes, nGq * v.d * v.kw * 4, v.nG * v.d * v.kw * 4));
+    DKV_CUDA(copy2d(o->k_sz, v.k_sz, nGq * v.d * 4, v.nG * v.d * 4));
+    DKV_CUDA(copy2d(o->k_tail, v.k_tail, (L - Lq) * v.d * 2, size_t(v.GK) * v.d * 2));
+    DKV_CUDA(copy2d(o->tail_mask, v.tail_mask, v.twords * 4, v.twords * 4));
+    DKV_CUDA(copy2d(o->prot_count, v.prot_count, 4, 4));
+    DKV_CUDA(copy2d(o->prot_pos, v.prot_pos, size_t(v.P) * 4, size_t(v.P) * 4));
+    DKV_CUDA(copy2d(o->prot_k, v.prot_k, size_t(v.P) * v.d * 2, size_t(v.P) * v.d * 2));
+    DKV_CUDA(copy2d(o->prot_gstart, v.prot_gstart, (nGq + 1) * 4, (v.nG + 1) * 4));
+  } else {
+    DKV_CUDA(copy2d(o->k_raw, v.k_raw, L * v.d * 2, v.cap * v.d * 2));
+    if (o->prot_count) std::memset(o->prot_count, 0, U * 4);
+  }
+  if (v.vb < 16) {
+    DKV_CUDA(copy2d(o->v_codes, v.v_codes, L * v.vw * 4, v.cap * v.vw * 4));
+    DKV_CUDA(copy2d(o->v_sz, v.v_sz, L * v.vgroups * 4, v.cap * v.vgroups * 4));
+  } else {
+    DKV_CUDA(copy2d(o->v_raw, v.v_raw, L * v.d * 2, v.cap * v.d * 2));
+  }
+  return DKV_OK;
+}
+
+int dkv_cache_set_option(dkv_cache* c, int32_t key, int64_t value) {
+  g_err.clear();
+  if (!c) return fail(DKV_ERR_INVALID_ARG, "cache is NULL");
+  switch (key) {
+    case DKV_OPT_SPLITS:
+      if (value < 0 || value > c->max_splits)
+        return fail(DKV_ERR_INVALID_ARG, "splits must be in [0, " + std::to_string(c->max_splits) + "]");
+      c->opt_splits = int32_t(value);
+      return DKV_OK;
+    case DKV_OPT_ATTN_KERNEL:
+      if (value < 0 || value > 2) return fail(DKV_ERR_INVALID_ARG, "kernel must be 0, 1 or 2");
+      if (value == 2 && !dkv::tc_supported(c->v))
+        return fail(DKV_ERR_UNSUPPORTED, "no tcgen05 attention variant for this shape");
+      c->opt_kernel = int32_t(value);
+      return DKV_OK;
+    case DKV_OPT_PROFILE:
+      if (value != 0 && value != 1) return fail(DKV_ERR_INVALID_ARG, "profile must be 0 or 1");
+      c->profile = value == 1;
+      return DKV_OK;
+    default:
+      return fail(DKV_ERR_INVALID_ARG, "unknown option key");
+  }
+}
+
+int dkv_profile_read(dkv_cache* c, int32_t kind, double* total_ms, int64_t* launches) {
+  g_err.clear();
+  if (!c || !total_ms || !launches) return fail(DKV_ERR_INVALID_ARG, "NULL argument");
+  double ms = 0.0;
+  int64_t n = 0;
+  for (size_t i = 0; i < c->prof_used; ++i) {
+    ProfRecord& r = c->prof[i];
+    DKV_CUDA(cudaEventSynchronize(r.stop));
+    if (r.kind != kind) continue;
+    float t = 0.f;
+    DKV_CUDA(cudaEventElapsedTime(&t, r.start, r.stop));
+    ms += t;
+    ++n;
+  }
+  // records of other kinds stay readable: compact them to the front
+  size_t keep = 0;
+  for (size_t i = 0; i < c->prof_used; ++i)
+    if (c->prof[i].kind != kind) std::swap(c->prof[keep++], c->prof[i]);
+  c->prof_used = keep;
+  *total_ms = ms;
+  *launches = n;
+  return DKV_OK;
+}
+
+int dkv_last_attention_plan(const dkv_cache* c, int32_t* kernel, int32_t* splits,
+                            int32_t* launches) {
+  g_err.clear();
+  if (!c) return fail(DKV_ERR_INVALID_ARG, "cache is NULL");
+  if (kernel) *kernel = c->last_kernel;
+  if (splits) *splits = c->last_splits;
+  if (launches) *launches = c->last_launches;
+  return DKV_OK;
+}
+
+}  // extern "C"

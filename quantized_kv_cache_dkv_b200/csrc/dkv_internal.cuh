@@ -1,0 +1,75 @@
+// Internal declarations shared by the host API and the kernels of libdkv.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "dkv.h"
+
+namespace dkv {
+
+constexpr int kHeadDim = 128;
+constexpr int kChunk = 32;  // token granularity of every segment boundary
+
+// Device-side view of one cache.  Array layouts are the canonical ones of
+// dkv.h with the capacity (not the length) as the token extent.
+struct CacheView {
+  int32_t B, Hq, Hkv, d, blk, g, rows;
+  int32_t kb, vb, GK, GV, P;
+  int64_t cap;     // tokens per unit
+  int64_t nG;      // cap / GK (K groups per unit)
+  int32_t kw;      // uint32 words per (K group, channel) = GK*kb/32
+  int32_t vw;      // uint32 words per V token = d*vb/32
+  int32_t vgroups; // d / GV
+  int32_t twords;  // ceil(GK/32)
+  int32_t U;
+
+  uint32_t* k_codes;    // [U][nG][d][kw]
+  __half2* k_sz;        // [U][nG][d]
+  uint16_t* k_raw;      // [U][cap][d]          (kb == 16)
+  uint16_t* k_tail;     // [U][GK][d]
+  uint32_t* tail_mask;  // [U][twords]
+  uint32_t* v_codes;    // [U][cap][vw]
+  __half2* v_sz;        // [U][cap][vgroups]
+  uint16_t* v_raw;      // [U][cap][d]          (vb == 16)
+  int32_t* prot_count;  // [U]
+  int32_t* prot_pos;    // [U][P]
+  uint16_t* prot_k;     // [U][P][d]
+  int32_t* prot_gstart; // [U][nG + 1]
+  uint32_t* status;     // sticky DKV_FLAG_* bits
+};
+
+// Arguments of one attention call.
+struct AttnArgs {
+  CacheView c;
+  const uint16_t* q;      // [B][Hq][blk][d] bf16
+  const uint16_t* k_act;  // [B][Hkv][blk][d] bf16
+  const uint16_t* v_act;  // [B][Hkv][blk][d] bf16
+  uint16_t* out;          // [B][Hq][blk][d] bf16
+  float* part_o;          // [U][nsplit][rows][d] fp32 (unnormalised)
+  float2* part_ml;        // [U][nsplit][rows] (running max in log2 units, sum)
+  float scale_log2;       // softmax_scale * log2(e)
+  int64_t L;              // committed tokens
+  int64_t Lq;             // tokens whose K is in complete groups (or raw)
+  int64_t n_tok;          // L + blk
+  int32_t nsplit;
+  int32_t tiles_per_split;  // in units of the kernel's token tile
+};
+
+cudaError_t launch_commit(const CacheView& c, const uint16_t* k, const uint16_t* v,
+                          const uint32_t* protect_words, int64_t p0, cudaStream_t s);
+cudaError_t launch_truncate(const CacheView& c, int64_t new_len, cudaStream_t s);
+
+// mma.sync kernel: token tile of 64.
+constexpr int kMmaTile = 64;
+cudaError_t launch_attention_mma(const AttnArgs& a, cudaStream_t s);
+cudaError_t launch_combine(const AttnArgs& a, cudaStream_t s);
+
+// tcgen05 kernel: token tile of 128, rows == 128.
+constexpr int kTcTile = 128;
+bool tc_supported(const CacheView& c);
+cudaError_t launch_attention_tc(const AttnArgs& a, cudaStream_t s);
+
+}  // namespace dkv

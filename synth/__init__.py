@@ -19,7 +19,8 @@ one (batch, kv-head) unit comes from its own PCG64 stream keyed by
 from __future__ import annotations
 
 import math
-from dataclasses import dataclass, field, replace
+import functools
+from dataclasses import dataclass, replace
 
 import numpy as np
 
@@ -53,7 +54,6 @@ class Workload:
     softmax_scale: float
     seed: int = 0
     attn_steps: int = 1  # denoising-step attentions the workload runs per block
-    extra: dict = field(default_factory=dict)
 
     @property
     def g(self) -> int:
@@ -142,6 +142,7 @@ def _rng(*key: int) -> np.random.Generator:
     return np.random.Generator(np.random.PCG64(np.random.SeedSequence(list(key))))
 
 
+@functools.lru_cache(maxsize=4096)
 def outlier_channels(w: Workload, h: int) -> np.ndarray:
     """K channels of kv-head h scaled by the outlier factor (same for every b)."""
     if w.n_outlier == 0:
@@ -185,6 +186,7 @@ def unit_kv_bits(w: Workload, b: int, h: int, n_tokens: int):
     return np.concatenate(ks), np.concatenate(vs)
 
 
+@functools.lru_cache(maxsize=4096)
 def prefill_protected_positions(w: Workload, b: int, h: int) -> np.ndarray:
     """round(prot_frac * L) distinct positions of [0, L), uniform, sorted."""
     n = w.n_prot_prefill

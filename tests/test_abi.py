@@ -1,0 +1,75 @@
+"""The C-ABI library loads, exports every function include/dkv.h declares, and
+rejects bad configurations on the host before touching the GPU.  CPU only:
+no call here launches a kernel."""
+import ctypes
+import subprocess
+
+import pytest
+
+import quantized_kv_cache_dkv_b200 as dkv
+
+
+def test_library_exports_every_header_symbol():
+    names = dkv.header_symbols()
+    assert "dkv_commit_block" in names and "dkv_block_attention" in names
+    out = subprocess.run(["nm", "-D", "--defined-only", dkv.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {ln.split()[-1] for ln in out.splitlines() if ln.strip()}
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    lib = ctypes.CDLL(dkv.LIB_PATH)
+    for n in names:
+        assert getattr(lib, n) is not None
+
+
+def _alloc_rc(**over):
+    cfg = dict(B=1, Hq=4, Hkv=1, d=128, blk=32, k_bits=4, v_bits=4, k_group=32, v_group=32,
+               max_protected=0, max_tokens=256)
+    cfg.update(over)
+    c = dkv.make_config(**cfg)
+    h = ctypes.c_void_p()
+    return dkv._alloc(ctypes.byref(c), None, ctypes.byref(h)), dkv._lib.dkv_last_error().decode()
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(d=64), dkv.DKV_ERR_UNSUPPORTED),
+    (dict(k_bits=3), dkv.DKV_ERR_UNSUPPORTED),
+    (dict(v_bits=8), dkv.DKV_ERR_UNSUPPORTED),
+    (dict(k_group=48), dkv.DKV_ERR_UNSUPPORTED),
+    (dict(v_group=16), dkv.DKV_ERR_UNSUPPORTED),
+    (dict(blk=48), dkv.DKV_ERR_UNSUPPORTED),
+    (dict(Hq=6, Hkv=4), dkv.DKV_ERR_INVALID_ARG),
+    (dict(Hq=16, Hkv=1, blk=32), dkv.DKV_ERR_UNSUPPORTED),     # 512 query rows per kv-head
+    (dict(max_tokens=100), dkv.DKV_ERR_INVALID_ARG),
+    (dict(k_group=64, max_tokens=96), dkv.DKV_ERR_INVALID_ARG),
+    (dict(B=0), dkv.DKV_ERR_INVALID_ARG),
+    (dict(max_protected=-1), dkv.DKV_ERR_INVALID_ARG),
+])
+def test_bad_config_rejected_on_host(over, code):
+    rc, msg = _alloc_rc(**over)
+    assert rc == code
+    assert msg
+
+
+def test_null_arguments_rejected():
+    P = ctypes.c_void_p
+    assert dkv._commit(None, P(16), P(16), None, None) == dkv.DKV_ERR_INVALID_ARG
+    assert dkv._attn(None, P(16), P(16), P(16), ctypes.c_float(1.0), P(16), None) == \
+        dkv.DKV_ERR_INVALID_ARG
+    n = ctypes.c_int64()
+    assert dkv._len(None, ctypes.byref(n)) == dkv.DKV_ERR_INVALID_ARG
+    assert dkv._free(None) == dkv.DKV_ERR_INVALID_ARG
+    assert dkv._setopt(None, 1, 0) == dkv.DKV_ERR_INVALID_ARG
+    assert "NULL" in dkv._lib.dkv_last_error().decode()
+
+
+def test_package_refuses_to_load_without_library(tmp_path):
+    """The binding has no fallback: a copy of the package without the .so
+    fails at import."""
+    import shutil
+    import sys
+    pkg = tmp_path / "quantized_kv_cache_dkv_b200"
+    shutil.copytree(dkv.__path__[0], pkg, ignore=shutil.ignore_patterns("*.so", "_build"))
+    r = subprocess.run([sys.executable, "-c", "import quantized_kv_cache_dkv_b200"],
+                       cwd=tmp_path, capture_output=True, text=True)
+    assert r.returncode != 0 and "libdkv.so is missing" in r.stderr

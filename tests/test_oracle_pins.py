@@ -555,3 +555,28 @@ def test_quantized_attention_uses_dequantized_cache():
                                   np.concatenate([vhat, bf16_to_f64(Va[b, h])]),
                                   w.softmax_scale)
         assert np.allclose(O[b, hq], ref, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("gk", [32, 64])
+def test_truncate_then_recommit_equals_fresh_cache(gk):
+    """Rolling back to a prefix and committing new blocks gives the same
+    state as committing prefix + new blocks into an empty cache."""
+    w = SMALL.with_(k_group=gk, prot_frac=0.1)
+    _, c = _cache(w)
+    for i in range(7):
+        c.commit(*synth.block_inputs(w, i))
+    c.truncate(128)
+    for i in (9, 10, 11):
+        c.commit(*synth.block_inputs(w, i))
+    _, f = _cache(w)
+    for i in (0, 1, 2, 3, 9, 10, 11):
+        f.commit(*synth.block_inputs(w, i))
+    a, b = c.snapshot(), f.snapshot()
+    for key in ("k_codes", "v_codes", "k_tail", "tail_mask", "prot_count", "prot_gstart"):
+        assert np.array_equal(a[key], b[key]), key
+    for u in range(c.U):
+        n = int(b["prot_count"][u])
+        assert np.array_equal(a["prot_pos"][u, :n], b["prot_pos"][u, :n])
+        assert np.array_equal(a["prot_k"][u, :n], b["prot_k"][u, :n])
+    with pytest.raises(ValueError):
+        c.truncate(32 if gk == 64 else 33)
