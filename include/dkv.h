@@ -121,6 +121,34 @@ int dkv_block_attention(dkv_cache* cache, const void* q, const void* k_act,
  * at once on the host. */
 int dkv_cache_truncate(dkv_cache* cache, int64_t new_len, void* stream);
 
+/* dkv_block_attention for callers that cannot call cudaMalloc -- code that
+ * runs while a CUDA stream capture is active (cudaMalloc is a prohibited call
+ * there and would invalidate the capture), or a plugin inside a host
+ * application that owns and budgets all device memory.  The pages have no
+ * counterpart to this call; it computes exactly what dkv_block_attention
+ * computes, with the same arguments, launch plan and error codes, but takes
+ * its split scratch (the per-split partial outputs merged by the combine
+ * kernel) from a fixed buffer compiled into the library instead of the
+ * handle's workspace, and allocates nothing: no cudaMalloc, cudaFree or
+ * allocating library routine.  The cache handle is an input created
+ * beforehand (dkv_cache_alloc).
+ *   - The buffer is a static __device__ array of DKV_NOALLOC_SCRATCH_BYTES
+ *     (16 MiB); every GPU that loads libdkv holds it until the process exits.
+ *   - A plan needing more scratch than that (B*Hkv * splits *
+ *     (q_heads/kv_heads)*block * (4*head_dim + 8) bytes, when splits > 1)
+ *     returns DKV_ERR_UNSUPPORTED with a message; lower DKV_OPT_SPLITS.
+ *   - The first call on each device looks up the buffer's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - Every call on a device shares the one buffer, which keeps the last
+ *     call's contents (each call overwrites what it reads).  Calls that
+ *     overlap on the GPU -- on different streams without ordering between
+ *     them -- race on it; serialize them. */
+#define DKV_NOALLOC_SCRATCH_BYTES (16u << 20)
+int dkv_block_attention_noalloc(dkv_cache* cache, const void* q, const void* k_act,
+                                const void* v_act, float softmax_scale, void* out,
+                                void* stream);
+
 /* Committed tokens per sequence (host mirror, no synchronization). */
 int dkv_cache_len(const dkv_cache* cache, int64_t* len);
 

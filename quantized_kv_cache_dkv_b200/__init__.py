@@ -66,6 +66,8 @@ _alloc = _sig("dkv_cache_alloc", [ctypes.POINTER(dkv_config), _P, ctypes.POINTER
 _free = _sig("dkv_cache_free", [_P])
 _commit = _sig("dkv_commit_block", [_P, _P, _P, _P, _P])
 _attn = _sig("dkv_block_attention", [_P, _P, _P, _P, ctypes.c_float, _P, _P])
+_attn_noalloc = _sig("dkv_block_attention_noalloc", [_P, _P, _P, _P, ctypes.c_float, _P, _P])
+DKV_NOALLOC_SCRATCH_BYTES = 16 << 20
 _len = _sig("dkv_cache_len", [_P, ctypes.POINTER(ctypes.c_int64)])
 _truncate = _sig("dkv_cache_truncate", [_P, ctypes.c_int64, _P])
 _status = _sig("dkv_cache_status", [_P, _P, ctypes.POINTER(ctypes.c_uint32)])
@@ -172,6 +174,25 @@ def dkv_block_attention(cache: Cache, q, k_act, v_act, softmax_scale: float, out
                   (torch.bfloat16, torch.int16))
     _check(_attn(cache.h, _ptr(q), _ptr(k_act), _ptr(v_act), ctypes.c_float(softmax_scale),
                  _ptr(out), _stream(stream)))
+
+
+def dkv_block_attention_noalloc(cache: Cache, q, k_act, v_act, softmax_scale: float, out,
+                                stream=None) -> None:
+    """dkv_block_attention for callers that cannot call cudaMalloc (under CUDA
+    stream capture, or inside a host application that owns all device
+    memory): split scratch comes from a fixed 16 MiB buffer inside libdkv and
+    nothing is allocated.  Calls overlapping on the GPU share that buffer and
+    race; the first call on a device should come before any stream capture."""
+    import torch
+    c = cache.cfg
+    _tensor_check(q, (c.batch, c.q_heads, c.block, c.head_dim), "q", (torch.bfloat16, torch.int16))
+    shp = (c.batch, c.kv_heads, c.block, c.head_dim)
+    _tensor_check(k_act, shp, "k_act", (torch.bfloat16, torch.int16))
+    _tensor_check(v_act, shp, "v_act", (torch.bfloat16, torch.int16))
+    _tensor_check(out, (c.batch, c.q_heads, c.block, c.head_dim), "out",
+                  (torch.bfloat16, torch.int16))
+    _check(_attn_noalloc(cache.h, _ptr(q), _ptr(k_act), _ptr(v_act),
+                         ctypes.c_float(softmax_scale), _ptr(out), _stream(stream)))
 
 
 def dkv_cache_truncate(cache: Cache, new_len: int, stream=None) -> None:

@@ -123,6 +123,23 @@ int split_cap(int U, int sms) {
 
 }  // namespace
 
+namespace dkv {
+
+bool cache_info(const dkv_cache* c, CacheInfo* out) {
+  if (!c || !out) return false;
+  out->v = c->v;
+  out->len = c->len;
+  out->num_sms = c->num_sms;
+  out->opt_splits = c->opt_splits;
+  out->opt_kernel = c->opt_kernel;
+  out->max_splits = c->max_splits;
+  return true;
+}
+
+int report_error(int code, const char* msg) { return fail(code, msg); }
+
+}  // namespace dkv
+
 extern "C" {
 
 const char* dkv_last_error(void) { return g_err.c_str(); }

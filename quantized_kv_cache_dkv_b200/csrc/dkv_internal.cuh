@@ -72,4 +72,15 @@ constexpr int kTcTile = 128;
 bool tc_supported(const CacheView& c);
 cudaError_t launch_attention_tc(const AttnArgs& a, cudaStream_t s);
 
+// Read-only view of a cache handle, and the thread-local error message, for
+// entry points defined outside dkv_api.cu.
+struct CacheInfo {
+  CacheView v;
+  int64_t len;
+  int num_sms;
+  int32_t opt_splits, opt_kernel, max_splits;
+};
+bool cache_info(const dkv_cache* c, CacheInfo* out);
+int report_error(int code, const char* msg);
+
 }  // namespace dkv
