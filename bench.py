@@ -184,6 +184,32 @@ def _dist():
     return world, rank, local
 
 
+def max_over_ranks(x: float) -> float:
+    """Max of a per-rank scalar over all ranks (identity without a process
+    group); NCCL reduces a device tensor, other backends a host tensor."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    dev = torch.device("cuda", torch.cuda.current_device()) if dist.get_backend() == "nccl" \
+        else torch.device("cpu")
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.barrier()
+
+
+def whole_job_gbs(bytes_per_rank: float, max_ms: float, world: int) -> float:
+    """Weak scaling: every rank moves bytes_per_rank; the job's time is the
+    slowest rank's."""
+    return world * bytes_per_rank / (max_ms / 1e3) / 1e9
+
+
 def run_gpu(w: synth.Workload, K: int, W: int, want_e2e=True, log=print, kernel=0):
     import torch
     import quantized_kv_cache_dkv_b200 as dkv
@@ -285,9 +311,7 @@ def run_gpu(w: synth.Workload, K: int, W: int, want_e2e=True, log=print, kernel=
     while time.time() < t_end:
         g.replay()
         torch.cuda.synchronize()
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
+    barrier()
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
@@ -296,22 +320,18 @@ def run_gpu(w: synth.Workload, K: int, W: int, want_e2e=True, log=print, kernel=
     g.replay()
     e1.record(stream)
     torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
+    barrier()
     ms = e0.elapsed_time(e1)
     t_end = time.time() + 0.4
     while time.time() < t_end:
         g.replay()
         torch.cuda.synchronize()
     clocks = sampler.stop()
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms)
 
     Ls = step_lengths(w, K, R)
     step_bytes = sum(attn_bytes(w, L + w.blk) + commit_bytes(w, L) for L in Ls)
-    value = world * step_bytes / (ms / 1e3) / 1e9
+    value = whole_job_gbs(step_bytes, ms, world)
 
     # profiling pass: device time of each kernel kind (eager launches)
     for c in caches:
@@ -378,23 +398,18 @@ def run_gpu(w: synth.Workload, K: int, W: int, want_e2e=True, log=print, kernel=
             e2e_step(k)
         finish()
         torch.cuda.synchronize()
-        if world > 1:
-            dist.barrier()
+        barrier()
         torch.cuda.synchronize()
         e0.record(stream)
         for k in range(K):
             e2e_step(k)
         e1.record(stream)
         torch.cuda.synchronize()
-        if world > 1:
-            dist.barrier()
+        barrier()
         ems = e0.elapsed_time(e1)
         finish()
-        if world > 1:
-            t = torch.tensor([ems], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
-        e2e = {"value": world * step_bytes / (ems / 1e3) / 1e9, "unit": "GB/s",
+        ems = max_over_ranks(ems)
+        e2e = {"value": whole_job_gbs(step_bytes, ems, world), "unit": "GB/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": ems / K}
 
@@ -534,6 +549,8 @@ def main():
                     help="also run the other workloads and add a summary per workload")
     ap.add_argument("--kernel", type=int, default=0, choices=[0, 1, 2],
                     help="attention kernel: 0 = library's choice, 1 = mma.sync, 2 = tcgen05")
+    ap.add_argument("--B", type=int, default=0, help="override the workload's batch (profiling)")
+    ap.add_argument("--L", type=int, default=0, help="override the committed length (profiling)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -541,6 +558,10 @@ def main():
         args.warmup = 3
     world, rank, local = _dist()
     w = synth.WORKLOADS[args.workload]
+    if args.B:
+        w = w.with_(B=args.B)
+    if args.L:
+        w = w.with_(L=args.L)
 
     if args.impl == "reference":
         if rank != 0:

@@ -22,7 +22,6 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 std::mutex g_mu;
 void* g_scratch_addr[kMaxDevices] = {};  // device address per device ordinal
 
-int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -67,29 +66,12 @@ extern "C" int dkv_block_attention_noalloc(dkv_cache* cache, const void* q, cons
   a.v_act = static_cast<const uint16_t*>(v_act);
   a.out = static_cast<uint16_t*>(out);
   a.scale_log2 = softmax_scale * 1.4426950408889634f;
-  a.L = ci.len;
-  a.Lq = v.kb < 16 ? (ci.len / v.GK) * v.GK : ci.len;
-  a.n_tok = ci.len + v.blk;
 
   // the launch plan of dkv_block_attention
-  int kernel = ci.opt_kernel;
-  if (kernel == 0) kernel = dkv::tc_supported(v) ? 2 : 1;
-  if (kernel == 2 && !dkv::tc_supported(v))
-    return report_error(DKV_ERR_UNSUPPORTED, "no tcgen05 attention variant for this shape");
-  const int tile = kernel == 2 ? dkv::kTcTile : dkv::kMmaTile;
-  const int64_t n_tiles = ceil_div(a.n_tok, tile);
-  int64_t ns;
-  if (ci.opt_splits > 0) {
-    ns = ci.opt_splits;
-  } else {
-    ns = ceil_div(int64_t(2) * ci.num_sms, v.U);
-    ns = std::min<int64_t>(ns, std::max<int64_t>(1, n_tiles / 2));
-  }
-  ns = std::max<int64_t>(1, std::min<int64_t>({ns, n_tiles, int64_t(ci.max_splits)}));
-  const int64_t tps = ceil_div(n_tiles, ns);
-  ns = ceil_div(n_tiles, tps);
-  a.nsplit = int(ns);
-  a.tiles_per_split = int(tps);
+  int kernel = 0;
+  const char* perr = nullptr;
+  const int prc = dkv::plan_attention(ci, &a, &kernel, &perr);
+  if (prc != DKV_OK) return report_error(prc, perr);
 
   if (a.nsplit > 1) {
     const size_t rows_total = size_t(v.U) * size_t(a.nsplit) * size_t(v.rows);

@@ -1,9 +1,10 @@
 // Bidirectional block attention over the low-bit cache on the 5th-generation
-// tensor cores (tcgen05 + tensor memory), for query groups of 128 rows
-// (query heads per kv-head x block = 128).  Attention is computed "directly
+// tensor cores (tcgen05 + tensor memory).  A query group (query heads per
+// kv-head x block tokens, 32..256 rows) is processed in row blocks of at most
+// 128 rows, each padded with zero queries to the M = 128 MMA shape.  Attention is computed "directly
 // from low-bit KV" (MaskAhead / Q-MaskAhead abstract) at every denoising step.
 //
-// CTA = (unit, token split), one CTA per SM, 13 warps:
+// CTA = (unit, token split), one CTA per SM, 14 warps:
 //   warps 0-3   softmax: thread r owns query row r (= TMEM lane r); loads Q
 //               into TMEM, runs the online softmax on S, writes P (fp16) back
 //               into TMEM, rescales O when the running max grows by > 2^8,
@@ -14,6 +15,11 @@
 //               contiguous: MN-major, 128-byte swizzle)
 //   warp 12     allocates TMEM; one lane issues the MMAs:
 //               S_j = Q K_j^T (A = Q from TMEM), O += P_j V_j (A = P from TMEM)
+//   warp 13     one lane streams each tile's packed K/V codes and fp16
+//               (scale, zero) pairs -- four contiguous ranges of the cache --
+//               into a 3-stage shared-memory ring with 1-D bulk copies
+//               (cp.async.bulk, completion counted on an mbarrier), so HBM
+//               latency overlaps the dequantization and the MMAs
 // Tensor memory (512 columns x 128 lanes x 32 bit): O [0,128), S0 [128,256),
 // S1 [256,384), Q [384,448); P_j (fp16 pairs) overwrites the first 64
 // columns of S_(j mod 2) once the softmax has read them.
@@ -28,9 +34,12 @@ namespace dkv {
 namespace {
 
 constexpr int TT = kTcTile;              // tokens per tile
-constexpr int kWarps = 13;
+constexpr int kWarps = 14;
 constexpr int kThreads = kWarps * 32;
 constexpr int kMmaWarp = 12;
+constexpr int kLoadWarp = 13;
+constexpr int kStages = 3;  // ring of packed tiles
+constexpr int kStagedProt = 24;  // protected K rows staged per tile (more: read from global)
 constexpr uint32_t kTileBytes = 128 * 128 * 2;
 constexpr uint32_t kColO = 0, kColS0 = 128, kColS1 = 256, kColQ = 384, kTmemCols = 512;
 constexpr uint64_t kTimeoutNs = 1000000000ull;
@@ -42,11 +51,23 @@ constexpr uint32_t kIdesc = (1u << 4) | (0u << 7) | (0u << 10) | (0u << 15) | (1
 struct Smem {
   // offsets into the 1024-byte aligned dynamic shared memory
   static constexpr uint32_t kK0 = 0, kK1 = kTileBytes, kV0 = 2 * kTileBytes, kV1 = 3 * kTileBytes;
-  static constexpr uint32_t kBar = 4 * kTileBytes;  // 16 mbarriers
-  static constexpr uint32_t kMisc = kBar + 16 * 8;  // tmem base, abort flag
+  // one ring stage: packed K codes (<= 8 KB: 128 tokens x 128 channels x 4 bit),
+  // K (scale, zero) (<= 2 KB), packed V codes (<= 8 KB), V (scale, zero) (<= 2 KB)
+  static constexpr uint32_t kRKc = 0, kRKsz = 8192, kRVc = 10240, kRVsz = 18432;
+  // side-table slice of the tile's K groups: header {entries n, first entry
+  // g0, index base of the staged positions}, positions (aligned superset),
+  // and the bf16 K rows of the first kStagedProt entries
+  static constexpr uint32_t kRHdr = 20480, kRPos = 20496, kRPk = 20624;
+  static constexpr uint32_t kStageBytes = 27648;
+  static constexpr uint32_t kRing = 4 * kTileBytes;
+  static constexpr uint32_t kBar = kRing + kStages * kStageBytes;  // 24 mbarriers
+  static constexpr uint32_t kMisc = kBar + 24 * 8;  // tmem base, abort flag
   static constexpr uint32_t kBytes = kMisc + 16;
 };
-enum Bar { KFULL = 0, KEMPTY = 2, VFULL = 4, VEMPTY = 6, SFULL = 8, PFULL = 10, QREADY = 12, DONE = 13 };
+enum Bar {
+  KFULL = 0, KEMPTY = 2, VFULL = 4, VEMPTY = 6, SFULL = 8, PFULL = 10, QREADY = 12, DONE = 13,
+  RFULL = 14, REMPTY = 14 + kStages
+};
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -78,15 +99,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Waits for the phase of `parity`; false on abort or after ~1 s (then the
-// CTA-wide abort flag and the sticky timeout flag are set).
+// Waits for the phase of `parity`; false on abort (unless drain) or after
+// ~1 s (then the CTA-wide abort flag and the sticky timeout flag are set).
+// `drain` waits that ignore the abort flag are used only for the CTA's own
+// copies and MMAs in flight before it releases shared and tensor memory.
 __device__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                          uint32_t* status) {
+                          uint32_t* status, bool drain = false) {
   uint64_t t0 = 0;
   for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 63u) {
-      if (*abort_flag) return false;
+      if (!drain && *abort_flag) return false;
       const uint64_t now = globaltimer();
       if (t0 == 0) {
         t0 = now;
@@ -97,6 +120,21 @@ __device__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_fla
       }
     }
   }
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+// 1-D bulk copy global -> shared (no multicast); completion counted on `bar`
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes,
+                                         uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
 }
 
 __device__ __forceinline__ void tc_fence_before() {
@@ -198,9 +236,13 @@ __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
 
 // ------------------------------------------------------------------ producers
 
-// K tile: thread `c` (channel) fills tokens [32q, 32q+32) of the tile for q = 0..3
+// K tile: thread `c` (channel) fills tokens [32q, 32q+32) of the tile for
+// q = 0..3.  Codes and (scale, zero) of the quantized part come from the ring
+// stage `rs` (groups of the tile in order, [group][channel][kw words]); the
+// bf16 tail, the active block and bits = 16 come straight from global memory.
 template <int KB>
-__device__ void fill_k_tile(const AttnArgs& a, int u, int64_t tile_start, uint8_t* kt, int c) {
+__device__ void fill_k_tile(const AttnArgs& a, int u, int64_t tile_start, uint8_t* kt,
+                            const uint8_t* rs, int c) {
   const CacheView& cv = a.c;
   const int d = kHeadDim;
 #pragma unroll 1
@@ -217,23 +259,23 @@ __device__ void fill_k_tile(const AttnArgs& a, int u, int64_t tile_start, uint8_
     } else if (pos0 < a.n_tok) {
       raw = a.k_act + (size_t(u) * cv.blk + (pos0 - a.L)) * d;
     }
-    int64_t j = 0;
     if (codes) {
       if constexpr (KB < 16) {
-        j = pos0 / cv.GK;
-        const int o = int(pos0 % cv.GK);
-        const size_t base = ((size_t(u) * cv.nG + j) * d + c) * cv.kw + size_t(o) * KB / 32;
-        const __half2 sz = cv.k_sz[(size_t(u) * cv.nG + j) * d + c];
+        const int gi = (32 * q) / cv.GK;  // group within the tile
+        const int o = (32 * q) % cv.GK;
+        const uint32_t* kc = reinterpret_cast<const uint32_t*>(rs + Smem::kRKc) +
+                             (gi * d + c) * cv.kw + o * KB / 32;
+        const __half2 sz = reinterpret_cast<const __half2*>(rs + Smem::kRKsz)[gi * d + c];
         const __half2 s2 = __half2half2(__low2half(sz));
         const __half2 z2 = __half2half2(__high2half(sz));
         if constexpr (KB == 4) {
-          const uint4 w = __ldg(reinterpret_cast<const uint4*>(cv.k_codes + base));
+          const uint4 w = *reinterpret_cast<const uint4*>(kc);
           out[0] = dequant4x8(w.x, s2, z2);
           out[1] = dequant4x8(w.y, s2, z2);
           out[2] = dequant4x8(w.z, s2, z2);
           out[3] = dequant4x8(w.w, s2, z2);
         } else {
-          const uint2 w = __ldg(reinterpret_cast<const uint2*>(cv.k_codes + base));
+          const uint2 w = *reinterpret_cast<const uint2*>(kc);
           dequant2x16(w.x, s2, z2, out[0], out[1]);
           dequant2x16(w.y, s2, z2, out[2], out[3]);
         }
@@ -257,15 +299,22 @@ __device__ void fill_k_tile(const AttnArgs& a, int u, int64_t tile_start, uint8_
       *reinterpret_cast<uint4*>(kt + kt_off(c, 32 * q + 8 * i)) = out[i];
     if constexpr (KB < 16) {
       if (codes) {
-        // protected rows of this chunk: their bf16 K from the side table
-        const int g0 = cv.prot_gstart[size_t(u) * (cv.nG + 1) + j];
-        const int g1 = cv.prot_gstart[size_t(u) * (cv.nG + 1) + j + 1];
-        for (int e = g0; e < g1; ++e) {
-          const int pos = cv.prot_pos[size_t(u) * cv.P + e];
+        // protected rows of this chunk: their bf16 K from the staged side-table
+        // slice (entries past kStagedProt from global memory)
+        const int* hdr = reinterpret_cast<const int*>(rs + Smem::kRHdr);
+        const int n = hdr[0], g0 = hdr[1], pbase = hdr[2];
+        const int* rpos = reinterpret_cast<const int*>(rs + Smem::kRPos);
+        const uint16_t* rpk = reinterpret_cast<const uint16_t*>(rs + Smem::kRPk);
+        for (int i = 0; i < n; ++i) {
+          const int pos = i < kStagedProt ? rpos[g0 + i - pbase]
+                                          : __ldg(cv.prot_pos + size_t(u) * cv.P + g0 + i);
           if (pos >= pos0 && pos < pos0 + 32) {
             const int t = 32 * q + int(pos - pos0);
+            const uint16_t kv = i < kStagedProt
+                                    ? rpk[i * d + c]
+                                    : __ldg(cv.prot_k + (size_t(u) * cv.P + g0 + i) * d + c);
             __half* dst = reinterpret_cast<__half*>(kt + kt_off(c, t & ~7)) + (t & 7);
-            *dst = bf16_to_half(cv.prot_k[(size_t(u) * cv.P + e) * d + c]);
+            *dst = bf16_to_half(kv);
           }
         }
       }
@@ -273,37 +322,48 @@ __device__ void fill_k_tile(const AttnArgs& a, int u, int64_t tile_start, uint8_
   }
 }
 
-// V tile: thread `t` (token of the tile) fills its 128 channels
+// V tile: thread `tid` fills items (token t, channel quarter qq) with
+// qq = item % 4, t = item / 4, item = tid + 128 r (r = 0..3), so a warp reads
+// 512 contiguous bytes of the ring stage ([token][vw words]).
 template <int VB>
-__device__ void fill_v_tile(const AttnArgs& a, int u, int64_t tile_start, uint8_t* vt, int t) {
+__device__ void fill_v_tile(const AttnArgs& a, int u, int64_t tile_start, uint8_t* vt,
+                            const uint8_t* rs, int tid) {
   const CacheView& cv = a.c;
   const int d = kHeadDim;
-  const int64_t pos = tile_start + t;
-  const uint16_t* raw = nullptr;
-  bool codes = false;
-  if (pos < a.L) {
-    if constexpr (VB < 16) codes = true;
-    else raw = cv.v_raw + (size_t(u) * cv.cap + pos) * d;
-  } else if (pos < a.n_tok) {
-    raw = a.v_act + (size_t(u) * cv.blk + (pos - a.L)) * d;
-  }
 #pragma unroll 1
-  for (int qq = 0; qq < 4; ++qq) {
+  for (int r = 0; r < 4; ++r) {
+    const int item = tid + 128 * r;
+    const int t = item >> 2, qq = item & 3;
+    const int64_t pos = tile_start + t;
     uint4 out[4];
+    const uint16_t* raw = nullptr;
+    bool codes = false;
+    if (pos < a.L) {
+      if constexpr (VB < 16) codes = true;
+      else raw = cv.v_raw + (size_t(u) * cv.cap + pos) * d;
+    } else if (pos < a.n_tok) {
+      raw = a.v_act + (size_t(u) * cv.blk + (pos - a.L)) * d;
+    }
+    // out[i] holds channels 32qq + 8((i + rot) & 3): lanes of a quarter warp
+    // (tokens t, t+1 x quarters 0..3) then store to 8 distinct bank groups
+    const int rot = qq & 2;
     if (codes) {
       if constexpr (VB < 16) {
-        const size_t tok = size_t(u) * cv.cap + pos;
-        const __half2 sz = cv.v_sz[tok * cv.vgroups + (qq * 32) / cv.GV];
+        const __half2 sz =
+            reinterpret_cast<const __half2*>(rs + Smem::kRVsz)[t * cv.vgroups + (qq * 32) / cv.GV];
         const __half2 s2 = __half2half2(__low2half(sz));
         const __half2 z2 = __half2half2(__high2half(sz));
+        const uint32_t* vc = reinterpret_cast<const uint32_t*>(rs + Smem::kRVc) + t * cv.vw;
         if constexpr (VB == 4) {
-          const uint4 w = __ldg(reinterpret_cast<const uint4*>(cv.v_codes + tok * cv.vw + qq * 4));
+          uint4 w = *reinterpret_cast<const uint4*>(vc + qq * 4);
+          if (rot) w = make_uint4(w.z, w.w, w.x, w.y);
           out[0] = dequant4x8(w.x, s2, z2);
           out[1] = dequant4x8(w.y, s2, z2);
           out[2] = dequant4x8(w.z, s2, z2);
           out[3] = dequant4x8(w.w, s2, z2);
         } else {
-          const uint2 w = __ldg(reinterpret_cast<const uint2*>(cv.v_codes + tok * cv.vw + qq * 2));
+          uint2 w = *reinterpret_cast<const uint2*>(vc + qq * 2);
+          if (rot) w = make_uint2(w.y, w.x);
           dequant2x16(w.x, s2, z2, out[0], out[1]);
           dequant2x16(w.y, s2, z2, out[2], out[3]);
         }
@@ -311,14 +371,15 @@ __device__ void fill_v_tile(const AttnArgs& a, int u, int64_t tile_start, uint8_
     } else if (raw) {
 #pragma unroll
       for (int i = 0; i < 4; ++i)
-        out[i] = bf16x8_to_f16x8(__ldg(reinterpret_cast<const uint4*>(raw + qq * 32 + 8 * i)));
+        out[i] = bf16x8_to_f16x8(
+            __ldg(reinterpret_cast<const uint4*>(raw + qq * 32 + 8 * ((i + rot) & 3))));
     } else {
 #pragma unroll
       for (int i = 0; i < 4; ++i) out[i] = make_uint4(0u, 0u, 0u, 0u);
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-      *reinterpret_cast<uint4*>(vt + vt_off(t, 32 * qq + 8 * i)) = out[i];
+      *reinterpret_cast<uint4*>(vt + vt_off(t, 32 * qq + 8 * ((i + rot) & 3))) = out[i];
   }
 }
 
@@ -336,8 +397,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + Smem::kMisc + 4);
 
   const CacheView& cv = a.c;
-  const int u = blockIdx.x / a.nsplit;
-  const int sp = blockIdx.x % a.nsplit;
+  // CTA = (unit, split, row block): a query group of more than 128 rows is
+  // cut into row blocks of rows/nrb; smaller blocks are zero-padded to M = 128
+  const int nrb = (cv.rows + 127) / 128;
+  const int rpb = cv.rows / nrb;
+  const int rb = blockIdx.x % nrb;
+  const int u = (blockIdx.x / nrb) / a.nsplit;
+  const int sp = (blockIdx.x / nrb) % a.nsplit;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t n_tiles = (a.n_tok + TT - 1) / TT;
   const int64_t t_begin = int64_t(sp) * a.tiles_per_split;
@@ -355,6 +421,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
     }
     mbar_init(bar(QREADY), 128);
     mbar_init(bar(DONE), 1);
+    for (int st = 0; st < kStages; ++st) {
+      mbar_init(bar(RFULL + st), 1);
+      mbar_init(bar(REMPTY + st), 256);
+    }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -371,16 +441,21 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
 
   if (warp < 4) {
     // ------------------------------------------------------------ softmax
-    const int r = threadIdx.x;  // query row = TMEM lane
+    const int lr = threadIdx.x;         // TMEM lane = row of this block
+    const bool row_ok = lr < rpb;       // padding rows carry Q = 0 and write nothing
+    // a warp holding only padding rows skips the softmax arithmetic (its P
+    // rows feed only padding rows of O, which are never read)
+    const bool warp_rows = warp * 32 < rpb;
+    const int r = rb * rpb + lr;        // query row of the unit
     const uint32_t lane_base = tmem + (uint32_t(warp * 32) << 16);
     {
-      const uint4* qrow = reinterpret_cast<const uint4*>(a.q + (size_t(u) * cv.rows + r) * kHeadDim);
+      const uint4* qrow = reinterpret_cast<const uint4*>(a.q + (size_t(u) * cv.rows + (row_ok ? r : 0)) * kHeadDim);
       uint32_t qv[32];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const uint4 y = bf16x8_to_f16x8(__ldg(qrow + h * 8 + i));
+          const uint4 y = row_ok ? bf16x8_to_f16x8(__ldg(qrow + h * 8 + i)) : make_uint4(0u, 0u, 0u, 0u);
           qv[4 * i + 0] = y.x;
           qv[4 * i + 1] = y.y;
           qv[4 * i + 2] = y.z;
@@ -404,22 +479,38 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
         break;
       }
       tc_fence_after();
+      if (!warp_rows) {
+        mbar_arrive(bar(PFULL + b));
+        continue;
+      }
       const int64_t tile_start = (t_begin + j) * TT;
       const int valid = a.n_tok - tile_start < TT ? int(a.n_tok - tile_start) : TT;
-      // pass 1: row max of this tile
+      // pass 1: row max of this tile (full tiles with scale >= 0: max of the
+      // raw scores times the scale; otherwise per element with masking)
+      const bool fast = valid >= TT && a.scale_log2 >= 0.f;
       float mx = -__int_as_float(0x7f800000);
 #pragma unroll 1
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t s[32];
-        tmem_ld32(lane_base + s_col + 32 * ch, s);
+      for (int ch = 0; ch < 4; ch += 2) {
+        uint32_t s0[32], s1[32];
+        tmem_ld32(lane_base + s_col + 32 * ch, s0);
+        tmem_ld32(lane_base + s_col + 32 * ch + 32, s1);
         tmem_ld_wait();
+        if (fast) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float x = 32 * ch + i < valid ? __uint_as_float(s[i]) * a.scale_log2
-                                              : -__int_as_float(0x7f800000);
-          mx = fmaxf(mx, x);
+          for (int i = 0; i < 32; ++i)
+            mx = fmaxf(mx, fmaxf(__uint_as_float(s0[i]), __uint_as_float(s1[i])));
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float x0 = 32 * ch + i < valid ? __uint_as_float(s0[i]) * a.scale_log2
+                                                 : -__int_as_float(0x7f800000);
+            const float x1 = 32 * ch + 32 + i < valid ? __uint_as_float(s1[i]) * a.scale_log2
+                                                      : -__int_as_float(0x7f800000);
+            mx = fmaxf(mx, fmaxf(x0, x1));
+          }
         }
       }
+      if (fast) mx *= a.scale_log2;
       // lazy rescale: keep the reference max unless the new one exceeds it by
       // 8 (P <= 2^8); decided per warp, rows whose max did not grow get alpha 1
       if (__any_sync(0xffffffffu, mx > m_used + 8.f)) {
@@ -447,25 +538,41 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
         l *= alpha;
         m_used = m_new;
       }
-      // pass 2: P = 2^(x - m_used) as fp16 into the first 64 columns of S_b
+      // pass 2: P = 2^(s*scale - m_used) as fp16 into the first 64 columns of S_b
+      const float nm = -m_used;
 #pragma unroll 1
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t s[32];
-        tmem_ld32(lane_base + s_col + 32 * ch, s);
+      for (int ch = 0; ch < 4; ch += 2) {
+        uint32_t s0[32], s1[32];
+        tmem_ld32(lane_base + s_col + 32 * ch, s0);
+        tmem_ld32(lane_base + s_col + 32 * ch + 32, s1);
         tmem_ld_wait();
-        uint32_t p[16];
+        uint32_t p0[16], p1[16];
+        if (valid >= TT) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int c0 = 32 * ch + 2 * i;
-          const float x0 = c0 < valid ? __uint_as_float(s[2 * i]) * a.scale_log2 - m_used
-                                      : -__int_as_float(0x7f800000);
-          const float x1 = c0 + 1 < valid ? __uint_as_float(s[2 * i + 1]) * a.scale_log2 - m_used
-                                          : -__int_as_float(0x7f800000);
-          const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
-          l += p0 + p1;
-          p[i] = pack_h2(p0, p1);
+          for (int i = 0; i < 16; ++i) {
+            const float a0 = fast_exp2(fmaf(__uint_as_float(s0[2 * i]), a.scale_log2, nm));
+            const float a1 = fast_exp2(fmaf(__uint_as_float(s0[2 * i + 1]), a.scale_log2, nm));
+            const float b0 = fast_exp2(fmaf(__uint_as_float(s1[2 * i]), a.scale_log2, nm));
+            const float b1 = fast_exp2(fmaf(__uint_as_float(s1[2 * i + 1]), a.scale_log2, nm));
+            l += (a0 + a1) + (b0 + b1);
+            p0[i] = pack_h2(a0, a1);
+            p1[i] = pack_h2(b0, b1);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int c0 = 32 * ch + 2 * i, c1 = c0 + 32;
+            const float a0 = c0 < valid ? fast_exp2(fmaf(__uint_as_float(s0[2 * i]), a.scale_log2, nm)) : 0.f;
+            const float a1 = c0 + 1 < valid ? fast_exp2(fmaf(__uint_as_float(s0[2 * i + 1]), a.scale_log2, nm)) : 0.f;
+            const float b0 = c1 < valid ? fast_exp2(fmaf(__uint_as_float(s1[2 * i]), a.scale_log2, nm)) : 0.f;
+            const float b1 = c1 + 1 < valid ? fast_exp2(fmaf(__uint_as_float(s1[2 * i + 1]), a.scale_log2, nm)) : 0.f;
+            l += (a0 + a1) + (b0 + b1);
+            p0[i] = pack_h2(a0, a1);
+            p1[i] = pack_h2(b0, b1);
+          }
         }
-        tmem_st16(lane_base + s_col + 16 * ch, p);
+        tmem_st16(lane_base + s_col + 16 * ch, p0);
+        tmem_st16(lane_base + s_col + 16 * ch + 16, p1);
       }
       tmem_st_wait();
       tc_fence_before();
@@ -477,7 +584,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
       ok = __all_sync(0xffffffffu,
                       mbar_wait(bar(VEMPTY + (jl & 1)), (jl >> 1) & 1, abort_flag, cv.status));
     }
-    if (ok) {
+    if (ok && warp_rows) {
       tc_fence_after();
       const float inv = 1.f / l;
 #pragma unroll 1
@@ -485,7 +592,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
         uint32_t o[32];
         tmem_ld32(lane_base + kColO + 32 * ch, o);
         tmem_ld_wait();
-        if (a.nsplit == 1) {
+        if (!row_ok) {
+          // padding row: nothing to write
+        } else if (a.nsplit == 1) {
           uint4* dst = reinterpret_cast<uint4*>(a.out + (size_t(u) * cv.rows + r) * kHeadDim + 32 * ch);
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
@@ -507,28 +616,117 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
                                  __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
         }
       }
-      if (a.nsplit > 1) a.part_ml[(size_t(u) * a.nsplit + sp) * cv.rows + r] = make_float2(m_used, l);
+      if (a.nsplit > 1 && row_ok)
+        a.part_ml[(size_t(u) * a.nsplit + sp) * cv.rows + r] = make_float2(m_used, l);
     }
   } else if (warp < 8) {
     // ------------------------------------------------------------ K producer
     const int c = threadIdx.x - 128;
     for (int j = 0; j < nt; ++j) {
-      const int b = j & 1;
+      const int b = j & 1, st = j % kStages;
       if (!mbar_wait(bar(KEMPTY + b), ((j >> 1) & 1) ^ 1, abort_flag, cv.status)) break;
-      fill_k_tile<KB>(a, u, (t_begin + j) * TT, sm + (b ? Smem::kK1 : Smem::kK0), c);
+      if (!mbar_wait(bar(RFULL + st), (j / kStages) & 1, abort_flag, cv.status)) break;
+      fill_k_tile<KB>(a, u, (t_begin + j) * TT, sm + (b ? Smem::kK1 : Smem::kK0),
+                      sm + Smem::kRing + st * Smem::kStageBytes, c);
       fence_async_smem();
       mbar_arrive(bar(KFULL + b));
+      mbar_arrive(bar(REMPTY + st));
     }
   } else if (warp < 12) {
     // ------------------------------------------------------------ V producer
     const int t = threadIdx.x - 256;
     for (int j = 0; j < nt; ++j) {
-      const int b = j & 1;
+      const int b = j & 1, st = j % kStages;
       if (!mbar_wait(bar(VEMPTY + b), ((j >> 1) & 1) ^ 1, abort_flag, cv.status)) break;
-      fill_v_tile<VB>(a, u, (t_begin + j) * TT, sm + (b ? Smem::kV1 : Smem::kV0), t);
+      if (!mbar_wait(bar(RFULL + st), (j / kStages) & 1, abort_flag, cv.status)) break;
+      fill_v_tile<VB>(a, u, (t_begin + j) * TT, sm + (b ? Smem::kV1 : Smem::kV0),
+                      sm + Smem::kRing + st * Smem::kStageBytes, t);
       fence_async_smem();
       mbar_arrive(bar(VFULL + b));
+      mbar_arrive(bar(REMPTY + st));
     }
+  } else if (warp == kLoadWarp) {
+    // ------------------------------------------------------------ loader
+    // lanes prefetch the side-table group index of 32 tiles at a time; lane 0
+    // issues the bulk copies of each tile
+    int issued = 0;
+    int pf0 = 0, pf1 = 0;  // this lane's prefetched gstart values (tile j0 + lane)
+    for (int j = 0; j < nt; ++j) {
+      if constexpr (KB < 16) {
+        if ((j & 31) == 0) {
+          pf0 = pf1 = 0;
+          const int jj = j + lane;
+          const int64_t ts = (t_begin + jj) * TT;
+          if (jj < nt && ts < a.Lq && cv.P > 0) {
+            const int64_t q_end = ts + TT < a.Lq ? ts + TT : a.Lq;
+            const int32_t* gs = cv.prot_gstart + size_t(u) * (cv.nG + 1);
+            pf0 = __ldg(gs + ts / cv.GK);
+            pf1 = __ldg(gs + q_end / cv.GK);
+          }
+        }
+      }
+      const int g0 = __shfl_sync(0xffffffffu, pf0, j & 31);
+      const int g1 = __shfl_sync(0xffffffffu, pf1, j & 31);
+      const int st = j % kStages;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(REMPTY + st), ((j / kStages) & 1) ^ 1,
+                                             abort_flag, cv.status)))
+        break;
+      ++issued;
+      if (lane == 0) {
+        const int64_t ts = (t_begin + j) * TT;
+        const uint32_t dst = sm_base + Smem::kRing + st * Smem::kStageBytes;
+        uint32_t kc_b = 0, ksz_b = 0, vc_b = 0, vsz_b = 0, pos_b = 0, pk_b = 0;
+        int64_t g_lo = 0, pidx0 = 0;
+        const int n = g1 - g0;
+        if (KB < 16 && ts < a.Lq) {
+          g_lo = ts / cv.GK;
+          const int64_t q_end = ts + TT < a.Lq ? ts + TT : a.Lq;  // multiple of GK
+          const uint32_t ng = uint32_t(q_end / cv.GK - g_lo);
+          kc_b = ng * kHeadDim * uint32_t(cv.kw) * 4u;
+          ksz_b = ng * kHeadDim * 4u;
+          if (n > 0) {
+            const int nst = n < kStagedProt ? n : kStagedProt;
+            const int64_t e0 = int64_t(u) * cv.P + g0;       // first entry, global index
+            pidx0 = e0 & ~int64_t(3);                        // 16-byte aligned superset
+            pos_b = uint32_t(((e0 + nst + 3) & ~int64_t(3)) - pidx0) * 4u;
+            pk_b = uint32_t(nst) * kHeadDim * 2u;
+          }
+        }
+        if (VB < 16 && ts < a.L) {
+          const int64_t v_end = ts + TT < a.L ? ts + TT : a.L;
+          const uint32_t nv = uint32_t(v_end - ts);
+          vc_b = nv * uint32_t(cv.vw) * 4u;
+          vsz_b = nv * uint32_t(cv.vgroups) * 4u;
+        }
+        int* hdr = reinterpret_cast<int*>(sm + Smem::kRing + st * Smem::kStageBytes + Smem::kRHdr);
+        hdr[0] = kc_b ? n : 0;
+        hdr[1] = g0;
+        hdr[2] = int(pidx0 - int64_t(u) * cv.P);
+        mbar_arrive_expect_tx(bar(RFULL + st), kc_b + ksz_b + vc_b + vsz_b + pos_b + pk_b);
+        if (kc_b) {
+          bulk_g2s(dst + Smem::kRKc, cv.k_codes + (size_t(u) * cv.nG + g_lo) * kHeadDim * cv.kw,
+                   kc_b, bar(RFULL + st));
+          bulk_g2s(dst + Smem::kRKsz, cv.k_sz + (size_t(u) * cv.nG + g_lo) * kHeadDim, ksz_b,
+                   bar(RFULL + st));
+        }
+        if (pos_b) {
+          bulk_g2s(dst + Smem::kRPos, cv.prot_pos + pidx0, pos_b, bar(RFULL + st));
+          bulk_g2s(dst + Smem::kRPk, cv.prot_k + (size_t(u) * cv.P + g0) * kHeadDim, pk_b,
+                   bar(RFULL + st));
+        }
+        if (vc_b) {
+          bulk_g2s(dst + Smem::kRVc, cv.v_codes + (size_t(u) * cv.cap + ts) * cv.vw, vc_b,
+                   bar(RFULL + st));
+          bulk_g2s(dst + Smem::kRVsz, cv.v_sz + (size_t(u) * cv.cap + ts) * cv.vgroups, vsz_b,
+                   bar(RFULL + st));
+        }
+      }
+      __syncwarp();
+    }
+    // drain: the last copies issued have landed before shared memory is released
+    if (lane == 0)
+      for (int j = issued > kStages ? issued - kStages : 0; j < issued; ++j)
+        mbar_wait(bar(RFULL + j % kStages), (j / kStages) & 1, abort_flag, cv.status, true);
   } else if (lane == 0) {
     // ------------------------------------------------------------ MMA issuer
     bool ok = mbar_wait(bar(QREADY), 0, abort_flag, cv.status);
@@ -564,7 +762,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
     if (ok && nt > 0) ok = issue_pv(nt - 1);
     // drain: every MMA issued above completes before TMEM is released
     mma_commit(bar(DONE));
-    mbar_wait(bar(DONE), 0, abort_flag, cv.status);
+    mbar_wait(bar(DONE), 0, abort_flag, cv.status, /*drain=*/true);
   }
 
   tc_fence_before();
@@ -581,7 +779,8 @@ cudaError_t launch_kv(const AttnArgs& a, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<KB, VB>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
-  attn_tc_kernel<KB, VB><<<unsigned(a.c.U) * unsigned(a.nsplit), kThreads, smem, s>>>(a);
+  const unsigned nrb = unsigned((a.c.rows + 127) / 128);
+  attn_tc_kernel<KB, VB><<<unsigned(a.c.U) * unsigned(a.nsplit) * nrb, kThreads, smem, s>>>(a);
   return cudaGetLastError();
 }
 
@@ -596,7 +795,10 @@ cudaError_t launch_k(const AttnArgs& a, cudaStream_t s) {
 
 }  // namespace
 
-bool tc_supported(const CacheView& c) { return c.rows == 128 && c.d == kHeadDim; }
+// any query group of 32..256 rows (a multiple of 32): M = 128 per row block
+bool tc_supported(const CacheView& c) {
+  return c.d == kHeadDim && c.rows >= 32 && c.rows <= 256 && c.rows % 32 == 0;
+}
 
 cudaError_t launch_attention_tc(const AttnArgs& a, cudaStream_t s) {
   if (!tc_supported(a.c)) return cudaErrorNotSupported;

@@ -4,7 +4,9 @@
 // paragraph; protected K entries kept in high precision with standard low-bit
 // V -- "KV Cache Quantization for Diffusion Language Models", abstract).
 //
-// One CTA of 128 threads per (sequence, kv-head) unit.  V: one item per
+// One CTA of 128 threads per (sequence, kv-head) unit.  The block's V and,
+// when a K group completes, the pending K stream (bf16 tail + block) are first
+// staged in shared memory with coalesced 16-byte loads.  V: one item per
 // (token, channel group).  K: thread c owns channel c of every K group that
 // this commit completes; tokens of an incomplete group wait in the bf16 tail.
 //
@@ -56,11 +58,33 @@ __device__ __forceinline__ uint32_t code_of(float x, const GroupQuant& q, int le
 }
 
 constexpr int kThreads = 128;
+constexpr int kRowPad = kHeadDim + 8;  // shared-memory row stride in halves (272 B)
 
+__device__ __forceinline__ void range_check8(uint4 x, bool& range) {
+  const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    range |= out_of_range(bf16_bits_to_f32(uint16_t(w[j] & 0xFFFF)));
+    range |= out_of_range(bf16_bits_to_f32(uint16_t(w[j] >> 16)));
+  }
+}
+
+// rows [0, n) of a [n][d] bf16 block -> shared rows of kRowPad halves
+__device__ __forceinline__ void stage_rows(uint16_t* dst, const uint16_t* src, int n, int tid) {
+  for (int i = tid; i < n * (kHeadDim / 8); i += kThreads) {
+    const int t = i / (kHeadDim / 8), o = i % (kHeadDim / 8);
+    *reinterpret_cast<uint4*>(dst + t * kRowPad + o * 8) =
+        __ldg(reinterpret_cast<const uint4*>(src + size_t(t) * kHeadDim + o * 8));
+  }
+}
+
+// Shared memory: the V block [blk][kRowPad] (quantized V), then the pending
+// K stream [max(k_group, blk)][kRowPad] (quantized K, when a group completes).
 template <int KB, int VB>
 __global__ void __launch_bounds__(kThreads)
 commit_kernel(CacheView c, const uint16_t* __restrict__ k, const uint16_t* __restrict__ v,
               const uint32_t* __restrict__ pw, int64_t p0) {
+  extern __shared__ __align__(16) uint16_t sbuf[];
   const int u = blockIdx.x;
   const int tid = threadIdx.x;
   const int d = kHeadDim;
@@ -69,6 +93,19 @@ commit_kernel(CacheView c, const uint16_t* __restrict__ k, const uint16_t* __res
   const uint16_t* vu = v + size_t(u) * blk * d;
   const int nbw = blk / 32;
   bool range = false;
+  uint16_t* sv = sbuf;
+  uint16_t* sk = sbuf + (VB < 16 ? blk * kRowPad : 0);
+  const int GK = c.GK;
+  const int n_tail = KB < 16 ? int(p0 % GK) : 0;
+  const bool completes = KB < 16 && n_tail + blk >= GK;
+
+  // ------------------------------------------------------------------ stage
+  if constexpr (VB < 16) stage_rows(sv, vu, blk, tid);
+  if (completes) {
+    stage_rows(sk, c.k_tail + size_t(u) * GK * d, n_tail, tid);
+    stage_rows(sk + n_tail * kRowPad, ku, blk, tid);
+  }
+  __syncthreads();
 
   // ------------------------------------------------------------------ V
   if constexpr (VB == 16) {
@@ -76,12 +113,7 @@ commit_kernel(CacheView c, const uint16_t* __restrict__ k, const uint16_t* __res
     uint4* dst = reinterpret_cast<uint4*>(c.v_raw + (size_t(u) * c.cap + p0) * d);
     for (int i = tid; i < blk * d / 8; i += kThreads) {
       const uint4 x = src[i];
-      const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        range |= out_of_range(bf16_bits_to_f32(uint16_t(w[j] & 0xFFFF)));
-        range |= out_of_range(bf16_bits_to_f32(uint16_t(w[j] >> 16)));
-      }
+      range_check8(x, range);
       dst[i] = x;
     }
   } else {
@@ -91,14 +123,19 @@ commit_kernel(CacheView c, const uint16_t* __restrict__ k, const uint16_t* __res
     const int ngr = d / GV;
     for (int it = tid; it < blk * ngr; it += kThreads) {
       const int t = it / ngr, gi = it % ngr;
-      const uint16_t* x = vu + t * d + gi * GV;
+      const uint16_t* x = sv + t * kRowPad + gi * GV;
       float mn = __int_as_float(0x7f800000), mx = -__int_as_float(0x7f800000);
-      for (int i = 0; i < GV; ++i) {
-        float f = bf16_bits_to_f32(x[i]);
-        range |= out_of_range(f);
-        f = sanitize(f);
-        mn = fminf(mn, f);
-        mx = fmaxf(mx, f);
+      for (int i8 = 0; i8 < GV; i8 += 8) {
+        const uint4 q8 = *reinterpret_cast<const uint4*>(x + i8);
+        const uint32_t w[4] = {q8.x, q8.y, q8.z, q8.w};
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          float f = bf16_bits_to_f32(uint16_t(w[j >> 1] >> (16 * (j & 1))));
+          range |= out_of_range(f);
+          f = sanitize(f);
+          mn = fminf(mn, f);
+          mx = fmaxf(mx, f);
+        }
       }
       const GroupQuant q = make_quant(mn, mx, levels);
       uint32_t* dst = c.v_codes + (size_t(u) * c.cap + p0 + t) * c.vw + gi * GV / per;
@@ -119,46 +156,32 @@ commit_kernel(CacheView c, const uint16_t* __restrict__ k, const uint16_t* __res
     uint4* dst = reinterpret_cast<uint4*>(c.k_raw + (size_t(u) * c.cap + p0) * d);
     for (int i = tid; i < blk * d / 8; i += kThreads) {
       const uint4 x = src[i];
-      const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        range |= out_of_range(bf16_bits_to_f32(uint16_t(w[j] & 0xFFFF)));
-        range |= out_of_range(bf16_bits_to_f32(uint16_t(w[j] >> 16)));
-      }
+      range_check8(x, range);
       dst[i] = x;
     }
   } else {
     constexpr int levels = (1 << KB) - 1;
     constexpr int per = 32 / KB;
-    const int GK = c.GK;
-    const int n_tail = int(p0 % GK);
     uint16_t* tail = c.k_tail + size_t(u) * GK * d;
     uint32_t* tmask = c.tail_mask + size_t(u) * c.twords;
-    if (n_tail + blk < GK) {
+    if (!completes) {
       // the group stays incomplete: append the block to the bf16 tail
       const uint4* src = reinterpret_cast<const uint4*>(ku);
       uint4* dst = reinterpret_cast<uint4*>(tail + size_t(n_tail) * d);
       for (int i = tid; i < blk * d / 8; i += kThreads) {
         const uint4 x = src[i];
-        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          range |= out_of_range(bf16_bits_to_f32(uint16_t(w[j] & 0xFFFF)));
-          range |= out_of_range(bf16_bits_to_f32(uint16_t(w[j] >> 16)));
-        }
+        range_check8(x, range);
         dst[i] = x;
       }
       if (tid < nbw) tmask[n_tail / 32 + tid] = pw ? pw[size_t(u) * nbw + tid] : 0u;
     } else {
-      // pending stream = tail[0, n_tail) ++ block[0, blk); quantize every
-      // complete group (k_group and block divide one another, so nothing is
-      // left over)
+      // pending stream = tail[0, n_tail) ++ block[0, blk) (staged in sk);
+      // quantize every complete group (k_group and block divide one another,
+      // so nothing is left over)
       const int npend = n_tail + blk;
       const int nfull = npend / GK;
       const int ch = tid;  // channel
-      auto pend_raw = [&](int pt) -> uint16_t {
-        return pt < n_tail ? tail[size_t(pt) * d + ch] : ku[size_t(pt - n_tail) * d + ch];
-      };
+      auto pend_raw = [&](int pt) -> uint16_t { return sk[pt * kRowPad + ch]; };
       int count = c.prot_count[u];
       const int64_t j0 = (p0 - n_tail) / GK;
       for (int gi = 0; gi < nfull; ++gi) {
@@ -247,7 +270,15 @@ __global__ void truncate_kernel(CacheView c, int64_t new_len) {
 template <int KB, int VB>
 cudaError_t launch_kv(const CacheView& c, const uint16_t* k, const uint16_t* v,
                       const uint32_t* pw, int64_t p0, cudaStream_t s) {
-  commit_kernel<KB, VB><<<c.U, kThreads, 0, s>>>(c, k, v, pw, p0);
+  const int krows = KB < 16 ? (c.GK > c.blk ? c.GK : c.blk) : 0;
+  const int vrows = VB < 16 ? c.blk : 0;
+  const size_t smem = size_t(krows + vrows) * kRowPad * 2;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(commit_kernel<KB, VB>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return e;
+  }
+  commit_kernel<KB, VB><<<c.U, kThreads, smem, s>>>(c, k, v, pw, p0);
   return cudaGetLastError();
 }
 

@@ -138,6 +138,50 @@ bool cache_info(const dkv_cache* c, CacheInfo* out) {
 
 int report_error(int code, const char* msg) { return fail(code, msg); }
 
+int plan_attention(const CacheInfo& ci, AttnArgs* a, int* kernel_out, const char** err) {
+  const CacheView& v = ci.v;
+  a->L = ci.len;
+  a->Lq = v.kb < 16 ? (ci.len / v.GK) * v.GK : ci.len;
+  a->n_tok = ci.len + v.blk;
+  int kernel = ci.opt_kernel;
+  if (kernel == 0) kernel = tc_supported(v) ? 2 : 1;
+  if (kernel == 2 && !tc_supported(v)) {
+    *err = "no tcgen05 attention variant for this shape";
+    return DKV_ERR_UNSUPPORTED;
+  }
+  const int tile = kernel == 2 ? kTcTile : kMmaTile;
+  const int64_t n_tiles = ceil_div(a->n_tok, tile);
+  const int64_t nrb = kernel == 2 ? (v.rows + 127) / 128 : 1;
+  const int64_t cap = std::max<int64_t>(1, std::min<int64_t>(n_tiles, ci.max_splits));
+  int64_t ns;
+  if (ci.opt_splits > 0) {
+    ns = std::min<int64_t>(ci.opt_splits, cap);
+  } else {
+    // minimise waves x (tiles per split + 2 tiles of per-CTA overhead) plus
+    // the combine's traffic (U*rows*(4d+8) bytes per split, ~5.2 MB per tile
+    // time), one CTA per SM
+    const double comb = double(v.U) * v.rows * (4.0 * v.d + 8.0) / 5.2e6;
+    double best = 1e300;
+    ns = 1;
+    for (int64_t s = 1; s <= cap; ++s) {
+      const int64_t tps = ceil_div(n_tiles, s);
+      const int64_t se = ceil_div(n_tiles, tps);
+      if (se != s) continue;
+      const int64_t waves = ceil_div(v.U * nrb * se, ci.num_sms);
+      const double cost = double(waves) * double(tps + 2) + (se > 1 ? comb * se : 0.0);
+      if (cost < best - 1e-9) {
+        best = cost;
+        ns = se;
+      }
+    }
+  }
+  const int64_t tps = ceil_div(n_tiles, ns);
+  a->nsplit = int(ceil_div(n_tiles, tps));  // no empty split
+  a->tiles_per_split = int(tps);
+  *kernel_out = kernel;
+  return DKV_OK;
+}
+
 }  // namespace dkv
 
 extern "C" {
@@ -325,29 +369,12 @@ int dkv_block_attention(dkv_cache* c, const void* q, const void* k_act, const vo
   a.part_o = c->part_o;
   a.part_ml = c->part_ml;
   a.scale_log2 = softmax_scale * 1.4426950408889634f;
-  a.L = c->len;
-  a.Lq = v.kb < 16 ? (c->len / v.GK) * v.GK : c->len;
-  a.n_tok = c->len + v.blk;
-
-  int kernel = c->opt_kernel;
-  if (kernel == 0) kernel = dkv::tc_supported(v) ? 2 : 1;
-  if (kernel == 2 && !dkv::tc_supported(v))
-    return fail(DKV_ERR_UNSUPPORTED, "no tcgen05 attention variant for this shape");
-  const int tile = kernel == 2 ? dkv::kTcTile : dkv::kMmaTile;
-  const int64_t n_tiles = ceil_div(a.n_tok, tile);
-  int64_t ns;
-  if (c->opt_splits > 0) {
-    ns = c->opt_splits;
-  } else {
-    // enough CTAs for two waves over the SMs, each split at least 2 tiles
-    ns = ceil_div(int64_t(2) * c->num_sms, v.U);
-    ns = std::min<int64_t>(ns, std::max<int64_t>(1, n_tiles / 2));
-  }
-  ns = std::max<int64_t>(1, std::min<int64_t>({ns, n_tiles, c->max_splits}));
-  const int64_t tps = ceil_div(n_tiles, ns);
-  ns = ceil_div(n_tiles, tps);  // no empty split
-  a.nsplit = int(ns);
-  a.tiles_per_split = int(tps);
+  dkv::CacheInfo ci;
+  dkv::cache_info(c, &ci);
+  int kernel = 0;
+  const char* perr = nullptr;
+  const int prc = dkv::plan_attention(ci, &a, &kernel, &perr);
+  if (prc != DKV_OK) return fail(prc, perr);
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = timed_launch(c, DKV_KERNEL_ATTENTION, s, [&] {

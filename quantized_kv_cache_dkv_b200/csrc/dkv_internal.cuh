@@ -81,6 +81,11 @@ struct CacheInfo {
   int32_t opt_splits, opt_kernel, max_splits;
 };
 bool cache_info(const dkv_cache* c, CacheInfo* out);
+
+// Launch plan of one attention call (kernel, split count, tiles per split);
+// fills a->L, Lq, n_tok, nsplit, tiles_per_split.  Returns DKV_OK or an error
+// code with *err set.
+int plan_attention(const CacheInfo& ci, AttnArgs* a, int* kernel, const char** err);
 int report_error(int code, const char* msg);
 
 }  // namespace dkv

@@ -92,14 +92,22 @@ def output_bound(ref64: np.ndarray) -> np.ndarray:
     return ATOL_MAX + half_ulp
 
 
+def bf16_round(ref64: np.ndarray) -> np.ndarray:
+    """fp64 -> bf16 (nearest even, through fp32) -> fp64."""
+    return bf16_to_f64(synth.f32_to_bf16_bits(np.asarray(ref64, np.float64).astype(np.float32)))
+
+
 def assert_close(got_bits: np.ndarray, ref64: np.ndarray, what=""):
-    """GPU bf16 output vs the fp64 oracle: every element within
-    output_bound, mean absolute error <= 1e-3."""
+    """GPU bf16 output vs the fp64 oracle: every element within output_bound
+    of the exact value; mean absolute difference to the oracle rounded to
+    bf16 <= 1e-3 (the mean of bf16's own rounding alone is ulp/4, about 1e-3
+    at |o| ~ 0.5-1, so the mean is taken between two bf16 results)."""
     got = bf16_to_f64(got_bits)
     ref = np.asarray(ref64, np.float64)
     assert np.all(np.isfinite(got)), what
     err = np.abs(got - ref)
     ratio = err / output_bound(ref)
     assert ratio.max() <= 1.0, (what, float(err.max()), float(ratio.max()))
-    assert err.mean() <= ATOL_MEAN, (what, float(err.mean()))
-    return float(err.max()), float(err.mean())
+    mean = float(np.abs(got - bf16_round(ref)).mean())
+    assert mean <= ATOL_MEAN, (what, mean)
+    return float(err.max()), mean

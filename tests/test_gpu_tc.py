@@ -1,5 +1,6 @@
-"""The tcgen05 (tensor-memory) attention kernel against the CPU oracle, for
-query groups of 128 rows, on the same cases as the warp-level kernel."""
+"""The tcgen05 (tensor-memory) attention kernel against the CPU oracle:
+query groups of 32 rows (zero-padded to M = 128), 128 rows, and 224 rows (two
+row blocks of 112)."""
 import pytest
 
 import synth
@@ -11,6 +12,10 @@ TC_CASES = {
     "tiny": SHRUNK["tiny"],
     "batch32": SHRUNK["batch32"],
     "longprompt": SHRUNK["longprompt"],
+    "mha8b": SHRUNK["mha8b"],
+    "gqa7b": SHRUNK["gqa7b"],
+    "rows64": SHRUNK["batch32"].with_(Hq=4, Hkv=2),
+    "rows256": SHRUNK["gqa7b"].with_(Hq=32, Hkv=4, B=1),
 }
 
 
