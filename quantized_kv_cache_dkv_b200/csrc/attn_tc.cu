@@ -4,18 +4,19 @@
 // 128 rows, each padded with zero queries to the M = 128 MMA shape.  Attention is computed "directly
 // from low-bit KV" (MaskAhead / Q-MaskAhead abstract) at every denoising step.
 //
-// CTA = (unit, token split), one CTA per SM, 14 warps:
+// CTA = (unit, token split, row block), one CTA per SM, 22 warps:
 //   warps 0-3   softmax: thread r owns query row r (= TMEM lane r); loads Q
 //               into TMEM, runs the online softmax on S, writes P (fp16) back
 //               into TMEM, rescales O when the running max grows by > 2^8,
 //               and writes the output / split partial at the end
-//   warps 4-7   K producer: dequantizes 128-token K tiles into shared memory
-//               (channel rows, tokens contiguous: MN-major, 128-byte swizzle)
-//   warps 8-11  V producer: dequantizes V tiles (token rows, channels
-//               contiguous: MN-major, 128-byte swizzle)
-//   warp 12     allocates TMEM; one lane issues the MMAs:
+//   warps 4-11  K producers: dequantize 128-token K tiles into shared memory
+//               (channel rows, tokens contiguous: MN-major, 128-byte swizzle);
+//               two warps per SM sub-partition, half a tile each
+//   warps 12-19 V producers: dequantize V tiles (token rows, channels
+//               contiguous: MN-major, 128-byte swizzle), half a tile each
+//   warp 20     allocates TMEM; one lane issues the MMAs:
 //               S_j = Q K_j^T (A = Q from TMEM), O += P_j V_j (A = P from TMEM)
-//   warp 13     one lane streams each tile's packed K/V codes and fp16
+//   warp 21     one lane streams each tile's packed K/V codes and fp16
 //               (scale, zero) pairs -- four contiguous ranges of the cache --
 //               into a 3-stage shared-memory ring with 1-D bulk copies
 //               (cp.async.bulk, completion counted on an mbarrier), so HBM
@@ -27,6 +28,8 @@
 // Every wait is bounded (about one second of %globaltimer): on expiry the
 // CTA raises DKV_FLAG_TIMEOUT, all roles leave their loops, the MMA lane waits
 // (bounded) for its own MMAs, and TMEM is released before returning.
+#include <type_traits>
+
 #include "dequant.cuh"
 #include "dkv_internal.cuh"
 
@@ -34,10 +37,10 @@ namespace dkv {
 namespace {
 
 constexpr int TT = kTcTile;              // tokens per tile
-constexpr int kWarps = 14;
+constexpr int kWarps = 22;
 constexpr int kThreads = kWarps * 32;
-constexpr int kMmaWarp = 12;
-constexpr int kLoadWarp = 13;
+constexpr int kMmaWarp = 20;
+constexpr int kLoadWarp = 21;
 constexpr int kStages = 3;  // ring of packed tiles
 constexpr int kStagedProt = 24;  // protected K rows staged per tile (more: read from global)
 constexpr uint32_t kTileBytes = 128 * 128 * 2;
@@ -87,14 +90,16 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
+// try_wait suspends the thread until the phase completes or the hint (ns)
+// expires, so waiting warps do not take issue slots from working ones
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "r"(200000u)
       : "memory");
   return ok != 0;
 }
@@ -108,7 +113,7 @@ __device__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_fla
   uint64_t t0 = 0;
   for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 63u) {
+    if ((it & 7u) == 7u) {
       if (!drain && *abort_flag) return false;
       const uint64_t now = globaltimer();
       if (t0 == 0) {
@@ -236,17 +241,69 @@ __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
 
 // ------------------------------------------------------------------ producers
 
-// K tile: thread `c` (channel) fills tokens [32q, 32q+32) of the tile for
-// q = 0..3.  Codes and (scale, zero) of the quantized part come from the ring
+// K tile: thread (c, qh) fills tokens [32q, 32q+32) of channel c for
+// q = 2qh, 2qh+1.  Codes and (scale, zero) of the quantized part come from the ring
 // stage `rs` (groups of the tile in order, [group][channel][kw words]); the
 // bf16 tail, the active block and bits = 16 come straight from global memory.
 template <int KB>
 __device__ void fill_k_tile(const AttnArgs& a, int u, int64_t tile_start, uint8_t* kt,
-                            const uint8_t* rs, int c) {
+                            const uint8_t* rs, int c, int qh) {
   const CacheView& cv = a.c;
   const int d = kHeadDim;
+  if constexpr (KB < 16) {
+    if (tile_start + TT <= a.Lq) {
+      // whole tile quantized: issue every shared-memory load, then dequantize
+      using W = typename std::conditional<KB == 4, uint4, uint2>::type;
+      W w[2];
+      __half2 sz[2];
+#pragma unroll
+      for (int qi = 0; qi < 2; ++qi) {
+        const int q = 2 * qh + qi;
+        const int gi = (32 * q) / cv.GK, o = (32 * q) % cv.GK;
+        w[qi] = *reinterpret_cast<const W*>(reinterpret_cast<const uint32_t*>(rs + Smem::kRKc) +
+                                            (gi * d + c) * cv.kw + o * KB / 32);
+        sz[qi] = reinterpret_cast<const __half2*>(rs + Smem::kRKsz)[gi * d + c];
+      }
+#pragma unroll
+      for (int qi = 0; qi < 2; ++qi) {
+        const int q = 2 * qh + qi;
+        const __half2 s2 = __half2half2(__low2half(sz[qi]));
+        const __half2 z2 = __half2half2(__high2half(sz[qi]));
+        uint4 out[4];
+        if constexpr (KB == 4) {
+          out[0] = dequant4x8(w[qi].x, s2, z2);
+          out[1] = dequant4x8(w[qi].y, s2, z2);
+          out[2] = dequant4x8(w[qi].z, s2, z2);
+          out[3] = dequant4x8(w[qi].w, s2, z2);
+        } else {
+          dequant2x16(w[qi].x, s2, z2, out[0], out[1]);
+          dequant2x16(w[qi].y, s2, z2, out[2], out[3]);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          *reinterpret_cast<uint4*>(kt + kt_off(c, 32 * q + 8 * i)) = out[i];
+      }
+      // protected rows of this thread's two chunks
+      const int* hdr = reinterpret_cast<const int*>(rs + Smem::kRHdr);
+      const int n = hdr[0], g0 = hdr[1], pbase = hdr[2];
+      const int* rpos = reinterpret_cast<const int*>(rs + Smem::kRPos);
+      const uint16_t* rpk = reinterpret_cast<const uint16_t*>(rs + Smem::kRPk);
+      for (int i = 0; i < n; ++i) {
+        const int pos = i < kStagedProt ? rpos[g0 + i - pbase]
+                                        : __ldg(cv.prot_pos + size_t(u) * cv.P + g0 + i);
+        const int t = int(pos - tile_start);
+        if ((t >> 6) != qh) continue;
+        const uint16_t kv = i < kStagedProt
+                                ? rpk[i * d + c]
+                                : __ldg(cv.prot_k + (size_t(u) * cv.P + g0 + i) * d + c);
+        __half* dst = reinterpret_cast<__half*>(kt + kt_off(c, t & ~7)) + (t & 7);
+        *dst = bf16_to_half(kv);
+      }
+      return;
+    }
+  }
 #pragma unroll 1
-  for (int q = 0; q < 4; ++q) {
+  for (int q = 2 * qh; q < 2 * qh + 2; ++q) {
     const int64_t pos0 = tile_start + 32 * q;
     uint4 out[4];
     const uint16_t* raw = nullptr;
@@ -322,17 +379,57 @@ __device__ void fill_k_tile(const AttnArgs& a, int u, int64_t tile_start, uint8_
   }
 }
 
-// V tile: thread `tid` fills items (token t, channel quarter qq) with
-// qq = item % 4, t = item / 4, item = tid + 128 r (r = 0..3), so a warp reads
+// V tile: thread `tid` (0..255) fills items (token t, channel quarter qq) with
+// qq = item % 4, t = item / 4, item = tid + 256 r (r = 0, 1), so a warp reads
 // 512 contiguous bytes of the ring stage ([token][vw words]).
 template <int VB>
 __device__ void fill_v_tile(const AttnArgs& a, int u, int64_t tile_start, uint8_t* vt,
                             const uint8_t* rs, int tid) {
   const CacheView& cv = a.c;
   const int d = kHeadDim;
+  if constexpr (VB < 16) {
+    if (tile_start + TT <= a.L) {
+      // whole tile quantized: issue every shared-memory load, then dequantize
+      using W = typename std::conditional<VB == 4, uint4, uint2>::type;
+      W w[2];
+      __half2 sz[2];
+      const int qq = tid & 3, rot = qq & 2;
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int t = (tid + 256 * r) >> 2;
+        w[r] = *reinterpret_cast<const W*>(reinterpret_cast<const uint32_t*>(rs + Smem::kRVc) +
+                                           t * cv.vw + qq * (VB == 4 ? 4 : 2));
+        sz[r] = reinterpret_cast<const __half2*>(rs + Smem::kRVsz)[t * cv.vgroups + (qq * 32) / cv.GV];
+      }
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int t = (tid + 256 * r) >> 2;
+        const __half2 s2 = __half2half2(__low2half(sz[r]));
+        const __half2 z2 = __half2half2(__high2half(sz[r]));
+        uint4 out[4];
+        if constexpr (VB == 4) {
+          uint4 x = w[r];
+          if (rot) x = make_uint4(x.z, x.w, x.x, x.y);
+          out[0] = dequant4x8(x.x, s2, z2);
+          out[1] = dequant4x8(x.y, s2, z2);
+          out[2] = dequant4x8(x.z, s2, z2);
+          out[3] = dequant4x8(x.w, s2, z2);
+        } else {
+          uint2 x = w[r];
+          if (rot) x = make_uint2(x.y, x.x);
+          dequant2x16(x.x, s2, z2, out[0], out[1]);
+          dequant2x16(x.y, s2, z2, out[2], out[3]);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          *reinterpret_cast<uint4*>(vt + vt_off(t, 32 * qq + 8 * ((i + rot) & 3))) = out[i];
+      }
+      return;
+    }
+  }
 #pragma unroll 1
-  for (int r = 0; r < 4; ++r) {
-    const int item = tid + 128 * r;
+  for (int r = 0; r < 2; ++r) {
+    const int item = tid + 256 * r;
     const int t = item >> 2, qq = item & 3;
     const int64_t pos = tile_start + t;
     uint4 out[4];
@@ -412,9 +509,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
 
   if (threadIdx.x == 0) {
     for (int b = 0; b < 2; ++b) {
-      mbar_init(bar(KFULL + b), 128);
+      mbar_init(bar(KFULL + b), 256);
       mbar_init(bar(KEMPTY + b), 1);
-      mbar_init(bar(VFULL + b), 128);
+      mbar_init(bar(VFULL + b), 256);
       mbar_init(bar(VEMPTY + b), 1);
       mbar_init(bar(SFULL + b), 1);
       mbar_init(bar(PFULL + b), 128);
@@ -423,7 +520,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
     mbar_init(bar(DONE), 1);
     for (int st = 0; st < kStages; ++st) {
       mbar_init(bar(RFULL + st), 1);
-      mbar_init(bar(REMPTY + st), 256);
+      mbar_init(bar(REMPTY + st), 512);
     }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -490,25 +587,27 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
       const bool fast = valid >= TT && a.scale_log2 >= 0.f;
       float mx = -__int_as_float(0x7f800000);
 #pragma unroll 1
-      for (int ch = 0; ch < 4; ch += 2) {
-        uint32_t s0[32], s1[32];
-        tmem_ld32(lane_base + s_col + 32 * ch, s0);
-        tmem_ld32(lane_base + s_col + 32 * ch + 32, s1);
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t sv[32];
+        tmem_ld32(lane_base + s_col + 32 * ch, sv);
         tmem_ld_wait();
+        float m4[4];
         if (fast) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            mx = fmaxf(mx, fmaxf(__uint_as_float(s0[i]), __uint_as_float(s1[i])));
+          for (int i = 0; i < 4; ++i) m4[i] = __uint_as_float(sv[i]);
+#pragma unroll
+          for (int i = 4; i < 32; ++i) m4[i & 3] = fmaxf(m4[i & 3], __uint_as_float(sv[i]));
         } else {
 #pragma unroll
+          for (int i = 0; i < 4; ++i) m4[i] = -__int_as_float(0x7f800000);
+#pragma unroll
           for (int i = 0; i < 32; ++i) {
-            const float x0 = 32 * ch + i < valid ? __uint_as_float(s0[i]) * a.scale_log2
-                                                 : -__int_as_float(0x7f800000);
-            const float x1 = 32 * ch + 32 + i < valid ? __uint_as_float(s1[i]) * a.scale_log2
-                                                      : -__int_as_float(0x7f800000);
-            mx = fmaxf(mx, fmaxf(x0, x1));
+            const float x = 32 * ch + i < valid ? __uint_as_float(sv[i]) * a.scale_log2
+                                                : -__int_as_float(0x7f800000);
+            m4[i & 3] = fmaxf(m4[i & 3], x);
           }
         }
+        mx = fmaxf(mx, fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])));
       }
       if (fast) mx *= a.scale_log2;
       // lazy rescale: keep the reference max unless the new one exceeds it by
@@ -540,40 +639,37 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
       }
       // pass 2: P = 2^(s*scale - m_used) as fp16 into the first 64 columns of S_b
       const float nm = -m_used;
+      float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
-      for (int ch = 0; ch < 4; ch += 2) {
-        uint32_t s0[32], s1[32];
-        tmem_ld32(lane_base + s_col + 32 * ch, s0);
-        tmem_ld32(lane_base + s_col + 32 * ch + 32, s1);
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t sv[32];
+        tmem_ld32(lane_base + s_col + 32 * ch, sv);
         tmem_ld_wait();
-        uint32_t p0[16], p1[16];
+        uint32_t pv[16];
         if (valid >= TT) {
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float a0 = fast_exp2(fmaf(__uint_as_float(s0[2 * i]), a.scale_log2, nm));
-            const float a1 = fast_exp2(fmaf(__uint_as_float(s0[2 * i + 1]), a.scale_log2, nm));
-            const float b0 = fast_exp2(fmaf(__uint_as_float(s1[2 * i]), a.scale_log2, nm));
-            const float b1 = fast_exp2(fmaf(__uint_as_float(s1[2 * i + 1]), a.scale_log2, nm));
-            l += (a0 + a1) + (b0 + b1);
-            p0[i] = pack_h2(a0, a1);
-            p1[i] = pack_h2(b0, b1);
+            const float p0 = fast_exp2(fmaf(__uint_as_float(sv[2 * i]), a.scale_log2, nm));
+            const float p1 = fast_exp2(fmaf(__uint_as_float(sv[2 * i + 1]), a.scale_log2, nm));
+            l4[i & 3] += p0 + p1;
+            pv[i] = pack_h2(p0, p1);
           }
         } else {
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const int c0 = 32 * ch + 2 * i, c1 = c0 + 32;
-            const float a0 = c0 < valid ? fast_exp2(fmaf(__uint_as_float(s0[2 * i]), a.scale_log2, nm)) : 0.f;
-            const float a1 = c0 + 1 < valid ? fast_exp2(fmaf(__uint_as_float(s0[2 * i + 1]), a.scale_log2, nm)) : 0.f;
-            const float b0 = c1 < valid ? fast_exp2(fmaf(__uint_as_float(s1[2 * i]), a.scale_log2, nm)) : 0.f;
-            const float b1 = c1 + 1 < valid ? fast_exp2(fmaf(__uint_as_float(s1[2 * i + 1]), a.scale_log2, nm)) : 0.f;
-            l += (a0 + a1) + (b0 + b1);
-            p0[i] = pack_h2(a0, a1);
-            p1[i] = pack_h2(b0, b1);
+            const int c0 = 32 * ch + 2 * i;
+            const float p0 =
+                c0 < valid ? fast_exp2(fmaf(__uint_as_float(sv[2 * i]), a.scale_log2, nm)) : 0.f;
+            const float p1 =
+                c0 + 1 < valid ? fast_exp2(fmaf(__uint_as_float(sv[2 * i + 1]), a.scale_log2, nm))
+                               : 0.f;
+            l4[i & 3] += p0 + p1;
+            pv[i] = pack_h2(p0, p1);
           }
         }
-        tmem_st16(lane_base + s_col + 16 * ch, p0);
-        tmem_st16(lane_base + s_col + 16 * ch + 16, p1);
+        tmem_st16(lane_base + s_col + 16 * ch, pv);
       }
+      l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar(PFULL + b));
@@ -619,22 +715,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
       if (a.nsplit > 1 && row_ok)
         a.part_ml[(size_t(u) * a.nsplit + sp) * cv.rows + r] = make_float2(m_used, l);
     }
-  } else if (warp < 8) {
+  } else if (warp < 12) {
     // ------------------------------------------------------------ K producer
-    const int c = threadIdx.x - 128;
+    const int c = (threadIdx.x - 128) & 127;   // channel
+    const int qh = (threadIdx.x - 128) >> 7;    // chunks 2qh, 2qh+1 of each tile
     for (int j = 0; j < nt; ++j) {
       const int b = j & 1, st = j % kStages;
       if (!mbar_wait(bar(KEMPTY + b), ((j >> 1) & 1) ^ 1, abort_flag, cv.status)) break;
       if (!mbar_wait(bar(RFULL + st), (j / kStages) & 1, abort_flag, cv.status)) break;
       fill_k_tile<KB>(a, u, (t_begin + j) * TT, sm + (b ? Smem::kK1 : Smem::kK0),
-                      sm + Smem::kRing + st * Smem::kStageBytes, c);
+                      sm + Smem::kRing + st * Smem::kStageBytes, c, qh);
       fence_async_smem();
       mbar_arrive(bar(KFULL + b));
       mbar_arrive(bar(REMPTY + st));
     }
-  } else if (warp < 12) {
+  } else if (warp < 20) {
     // ------------------------------------------------------------ V producer
-    const int t = threadIdx.x - 256;
+    const int t = threadIdx.x - 384;
     for (int j = 0; j < nt; ++j) {
       const int b = j & 1, st = j % kStages;
       if (!mbar_wait(bar(VEMPTY + b), ((j >> 1) & 1) ^ 1, abort_flag, cv.status)) break;

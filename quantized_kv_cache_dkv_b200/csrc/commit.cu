@@ -4,11 +4,13 @@
 // paragraph; protected K entries kept in high precision with standard low-bit
 // V -- "KV Cache Quantization for Diffusion Language Models", abstract).
 //
-// One CTA of 128 threads per (sequence, kv-head) unit.  The block's V and,
+// One CTA of 256 threads per (sequence, kv-head) unit.  The block's V and,
 // when a K group completes, the pending K stream (bf16 tail + block) are first
 // staged in shared memory with coalesced 16-byte loads.  V: one item per
-// (token, channel group).  K: thread c owns channel c of every K group that
-// this commit completes; tokens of an incomplete group wait in the bf16 tail.
+// (token, channel group), threads 128..255.  K: thread c < 128 owns channel c
+// of every K group that this commit completes; tokens of an incomplete group
+// wait in the bf16 tail.  Group sizes are compile-time constants, so each
+// group's loads and divisions are unrolled and independent.
 //
 // This file is compiled with -fmad=false and uses only correctly rounded fp32
 // operations (__fsub_rn, __fdiv_rn, __float2half_rn, __float2int_rn), so the
@@ -57,7 +59,7 @@ __device__ __forceinline__ uint32_t code_of(float x, const GroupQuant& q, int le
   return uint32_t(c);
 }
 
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;         // 128 K channels and up to 128 V groups side by side
 constexpr int kRowPad = kHeadDim + 8;  // shared-memory row stride in halves (272 B)
 
 __device__ __forceinline__ void range_check8(uint4 x, bool& range) {
@@ -78,8 +80,93 @@ __device__ __forceinline__ void stage_rows(uint16_t* dst, const uint16_t* src, i
   }
 }
 
+__device__ __forceinline__ float bf16_at(const uint16_t* p) { return bf16_bits_to_f32(*p); }
+
+// One V group: G consecutive channels of one token (x: shared memory, 16-byte
+// aligned).  Fully unrolled so the loads and the divisions are independent.
+template <int VB, int G>
+__device__ __forceinline__ void quant_v_group(const uint16_t* x, uint32_t* codes, __half2* sz,
+                                              bool& range) {
+  constexpr int levels = (1 << VB) - 1;
+  constexpr int per = 32 / VB;
+  float mn4[4], mx4[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    mn4[i] = __int_as_float(0x7f800000);
+    mx4[i] = -__int_as_float(0x7f800000);
+  }
+#pragma unroll
+  for (int i8 = 0; i8 < G; i8 += 8) {
+    const uint4 q8 = *reinterpret_cast<const uint4*>(x + i8);
+    const uint32_t w[4] = {q8.x, q8.y, q8.z, q8.w};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      float f = bf16_bits_to_f32(uint16_t(w[j >> 1] >> (16 * (j & 1))));
+      range |= out_of_range(f);
+      f = sanitize(f);
+      mn4[j & 3] = fminf(mn4[j & 3], f);
+      mx4[j & 3] = fmaxf(mx4[j & 3], f);
+    }
+  }
+  const float mn = fminf(fminf(mn4[0], mn4[1]), fminf(mn4[2], mn4[3]));
+  const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+  const GroupQuant q = make_quant(mn, mx, levels);
+#pragma unroll
+  for (int w = 0; w < G / per; ++w) {
+    uint32_t word = 0;
+#pragma unroll
+    for (int e = 0; e < per; ++e)
+      word |= code_of(sanitize(bf16_at(x + w * per + e)), q, levels) << (e * VB);
+    codes[w] = word;
+  }
+  *sz = q.sz;
+}
+
+// One K group of channel ch: G tokens of the pending stream (rows of sk),
+// protected tokens (bits of gm) left out of min/max and given code 0.
+template <int KB, int G>
+__device__ __forceinline__ GroupQuant quant_k_group(const uint16_t* sk, int row0, int ch,
+                                                    const uint32_t (&gm)[4], bool check_from,
+                                                    int check_row, uint32_t* codes, bool& range) {
+  constexpr int levels = (1 << KB) - 1;
+  constexpr int per = 32 / KB;
+  float mn4[4], mx4[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    mn4[i] = __int_as_float(0x7f800000);
+    mx4[i] = -__int_as_float(0x7f800000);
+  }
+#pragma unroll
+  for (int t = 0; t < G; ++t) {
+    float f = bf16_at(sk + (row0 + t) * kRowPad + ch);
+    if (check_from && row0 + t >= check_row) range |= out_of_range(f);
+    f = sanitize(f);
+    if (!((gm[t >> 5] >> (t & 31)) & 1u)) {
+      mn4[t & 3] = fminf(mn4[t & 3], f);
+      mx4[t & 3] = fmaxf(mx4[t & 3], f);
+    }
+  }
+  float mn = fminf(fminf(mn4[0], mn4[1]), fminf(mn4[2], mn4[3]));
+  float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+  if (mn > mx) mn = mx = 0.f;  // every token protected
+  const GroupQuant q = make_quant(mn, mx, levels);
+#pragma unroll
+  for (int w = 0; w < G / per; ++w) {
+    uint32_t word = 0;
+#pragma unroll
+    for (int e = 0; e < per; ++e) {
+      const int t = w * per + e;
+      const uint32_t cq = code_of(sanitize(bf16_at(sk + (row0 + t) * kRowPad + ch)), q, levels);
+      if (!((gm[t >> 5] >> (t & 31)) & 1u)) word |= cq << (e * KB);  // protected slot: code 0
+    }
+    codes[w] = word;
+  }
+  return q;
+}
+
 // Shared memory: the V block [blk][kRowPad] (quantized V), then the pending
 // K stream [max(k_group, blk)][kRowPad] (quantized K, when a group completes).
+// Threads [0, 128): K (channel = thread); threads [128, 256): V groups.
 template <int KB, int VB>
 __global__ void __launch_bounds__(kThreads)
 commit_kernel(CacheView c, const uint16_t* __restrict__ k, const uint16_t* __restrict__ v,
@@ -116,37 +203,17 @@ commit_kernel(CacheView c, const uint16_t* __restrict__ k, const uint16_t* __res
       range_check8(x, range);
       dst[i] = x;
     }
-  } else {
-    constexpr int levels = (1 << VB) - 1;
-    constexpr int per = 32 / VB;
+  } else if (tid >= 128) {
     const int GV = c.GV;
     const int ngr = d / GV;
-    for (int it = tid; it < blk * ngr; it += kThreads) {
+    for (int it = tid - 128; it < blk * ngr; it += 128) {
       const int t = it / ngr, gi = it % ngr;
       const uint16_t* x = sv + t * kRowPad + gi * GV;
-      float mn = __int_as_float(0x7f800000), mx = -__int_as_float(0x7f800000);
-      for (int i8 = 0; i8 < GV; i8 += 8) {
-        const uint4 q8 = *reinterpret_cast<const uint4*>(x + i8);
-        const uint32_t w[4] = {q8.x, q8.y, q8.z, q8.w};
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          float f = bf16_bits_to_f32(uint16_t(w[j >> 1] >> (16 * (j & 1))));
-          range |= out_of_range(f);
-          f = sanitize(f);
-          mn = fminf(mn, f);
-          mx = fmaxf(mx, f);
-        }
-      }
-      const GroupQuant q = make_quant(mn, mx, levels);
-      uint32_t* dst = c.v_codes + (size_t(u) * c.cap + p0 + t) * c.vw + gi * GV / per;
-      for (int w = 0; w < GV / per; ++w) {
-        uint32_t word = 0;
-#pragma unroll
-        for (int e = 0; e < per; ++e)
-          word |= code_of(sanitize(bf16_bits_to_f32(x[w * per + e])), q, levels) << (e * VB);
-        dst[w] = word;
-      }
-      c.v_sz[(size_t(u) * c.cap + p0 + t) * ngr + gi] = q.sz;
+      uint32_t* codes = c.v_codes + (size_t(u) * c.cap + p0 + t) * c.vw + gi * GV * VB / 32;
+      __half2* sz = c.v_sz + (size_t(u) * c.cap + p0 + t) * ngr + gi;
+      if (GV == 32) quant_v_group<VB, 32>(x, codes, sz, range);
+      else if (GV == 64) quant_v_group<VB, 64>(x, codes, sz, range);
+      else quant_v_group<VB, 128>(x, codes, sz, range);
     }
   }
 
@@ -160,8 +227,6 @@ commit_kernel(CacheView c, const uint16_t* __restrict__ k, const uint16_t* __res
       dst[i] = x;
     }
   } else {
-    constexpr int levels = (1 << KB) - 1;
-    constexpr int per = 32 / KB;
     uint16_t* tail = c.k_tail + size_t(u) * GK * d;
     uint32_t* tmask = c.tail_mask + size_t(u) * c.twords;
     if (!completes) {
@@ -174,33 +239,37 @@ commit_kernel(CacheView c, const uint16_t* __restrict__ k, const uint16_t* __res
         dst[i] = x;
       }
       if (tid < nbw) tmask[n_tail / 32 + tid] = pw ? pw[size_t(u) * nbw + tid] : 0u;
-    } else {
+    } else if (tid < 128) {
       // pending stream = tail[0, n_tail) ++ block[0, blk) (staged in sk);
       // quantize every complete group (k_group and block divide one another,
       // so nothing is left over)
       const int npend = n_tail + blk;
       const int nfull = npend / GK;
       const int ch = tid;  // channel
-      auto pend_raw = [&](int pt) -> uint16_t { return sk[pt * kRowPad + ch]; };
       int count = c.prot_count[u];
       const int64_t j0 = (p0 - n_tail) / GK;
       for (int gi = 0; gi < nfull; ++gi) {
         const int64_t j = j0 + gi;
         uint32_t gm[4] = {0u, 0u, 0u, 0u};
-        for (int w = 0; w < GK / 32; ++w) {
-          const int pwi = gi * GK / 32 + w;  // word of the pending stream
-          if (pwi < n_tail / 32)
-            gm[w] = tmask[pwi];
-          else
-            gm[w] = pw ? pw[size_t(u) * nbw + (pwi - n_tail / 32)] : 0u;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          if (w < GK / 32) {
+            const int pwi = gi * GK / 32 + w;  // word of the pending stream
+            if (pwi < n_tail / 32)
+              gm[w] = tmask[pwi];
+            else
+              gm[w] = pw ? pw[size_t(u) * nbw + (pwi - n_tail / 32)] : 0u;
+          }
         }
         // side table full: keep the first `room` protected tokens by position
         int want = 0;
-        for (int w = 0; w < GK / 32; ++w) want += __popc(gm[w]);
+#pragma unroll
+        for (int w = 0; w < 4; ++w) want += __popc(gm[w]);
         const int room = c.P - count;
         if (want > room) {
           int kept = 0;
-          for (int w = 0; w < GK / 32; ++w) {
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
             uint32_t m = gm[w], nm = 0u;
             while (m && kept < room) {
               const uint32_t low = m & (0u - m);
@@ -212,40 +281,22 @@ commit_kernel(CacheView c, const uint16_t* __restrict__ k, const uint16_t* __res
           }
           if (tid == 0) atomicOr(c.status, uint32_t(DKV_FLAG_CAPACITY));
         }
-        // min / max over the group's non-protected tokens of channel ch
-        float mn = __int_as_float(0x7f800000), mx = -__int_as_float(0x7f800000);
-        for (int t = 0; t < GK; ++t) {
-          const int pt = gi * GK + t;
-          float f = bf16_bits_to_f32(pend_raw(pt));
-          if (pt >= n_tail) range |= out_of_range(f);
-          f = sanitize(f);
-          if (!((gm[t >> 5] >> (t & 31)) & 1u)) {
-            mn = fminf(mn, f);
-            mx = fmaxf(mx, f);
-          }
-        }
-        if (mn > mx) mn = mx = 0.f;  // every token protected
-        const GroupQuant q = make_quant(mn, mx, levels);
-        uint32_t* dst = c.k_codes + ((size_t(u) * c.nG + j) * d + ch) * c.kw;
-        for (int w = 0; w < GK / per; ++w) {
-          uint32_t word = 0;
-          for (int e = 0; e < per; ++e) {
-            const int t = w * per + e;
-            if ((gm[t >> 5] >> (t & 31)) & 1u) continue;  // protected slot: code 0
-            word |= code_of(sanitize(bf16_bits_to_f32(pend_raw(gi * GK + t))), q, levels) << (e * KB);
-          }
-          dst[w] = word;
-        }
+        uint32_t* codes = c.k_codes + ((size_t(u) * c.nG + j) * d + ch) * c.kw;
+        GroupQuant q;
+        if (GK == 32) q = quant_k_group<KB, 32>(sk, gi * GK, ch, gm, true, n_tail, codes, range);
+        else if (GK == 64) q = quant_k_group<KB, 64>(sk, gi * GK, ch, gm, true, n_tail, codes, range);
+        else q = quant_k_group<KB, 128>(sk, gi * GK, ch, gm, true, n_tail, codes, range);
         c.k_sz[(size_t(u) * c.nG + j) * d + ch] = q.sz;
         // side-table entries, ascending positions
-        for (int w = 0; w < GK / 32; ++w) {
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
           uint32_t m = gm[w];
           while (m) {
             const int b = __ffs(m) - 1;
             m &= m - 1u;
             const int t = w * 32 + b;
             if (tid == 0) c.prot_pos[size_t(u) * c.P + count] = int32_t(j * GK + t);
-            c.prot_k[(size_t(u) * c.P + count) * d + ch] = pend_raw(gi * GK + t);
+            c.prot_k[(size_t(u) * c.P + count) * d + ch] = sk[(gi * GK + t) * kRowPad + ch];
             ++count;
           }
         }
