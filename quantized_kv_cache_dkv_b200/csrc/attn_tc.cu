@@ -4,26 +4,32 @@
 // 128 rows, each padded with zero queries to the M = 128 MMA shape.  Attention is computed "directly
 // from low-bit KV" (MaskAhead / Q-MaskAhead abstract) at every denoising step.
 //
-// CTA = (unit, token split, row block), one CTA per SM, 22 warps:
-//   warps 0-3   softmax: thread r owns query row r (= TMEM lane r); loads Q
-//               into TMEM, runs the online softmax on S, writes P (fp16) back
-//               into TMEM, rescales O when the running max grows by > 2^8,
-//               and writes the output / split partial at the end
-//   warps 4-11  K producers: dequantize 128-token K tiles into shared memory
+// CTA = (unit, token split, row block), one CTA per SM, 24 warps (six
+// warpgroups; setmaxnreg moves registers from the producers and the control
+// warps to the softmax warpgroup):
+//   warps 0-7   softmax, two warpgroups: thread (r, h) owns query row r (=
+//               TMEM lane r) and columns [64h, 64h+64) of each S tile; loads
+//               its half of Q into TMEM, runs the online softmax (row maxima
+//               of the two halves exchanged through shared memory on an
+//               mbarrier), writes P (fp16) into its own half of S, rescales
+//               its half of O when the running max grows by > 2^8, and writes
+//               its half of the output / split partial at the end
+//   warps 8-15  K producers: dequantize 128-token K tiles into shared memory
 //               (channel rows, tokens contiguous: MN-major, 128-byte swizzle);
 //               two warps per SM sub-partition, half a tile each
-//   warps 12-19 V producers: dequantize V tiles (token rows, channels
+//   warps 16-23 V producers: dequantize V tiles (token rows, channels
 //               contiguous: MN-major, 128-byte swizzle), half a tile each
-//   warp 20     allocates TMEM; one lane issues the MMAs:
+//   warp 24     allocates TMEM; one lane issues the MMAs:
 //               S_j = Q K_j^T (A = Q from TMEM), O += P_j V_j (A = P from TMEM)
-//   warp 21     one lane streams each tile's packed K/V codes and fp16
+//   warp 25     one lane streams each tile's packed K/V codes and fp16
 //               (scale, zero) pairs -- four contiguous ranges of the cache --
 //               into a 3-stage shared-memory ring with 1-D bulk copies
 //               (cp.async.bulk, completion counted on an mbarrier), so HBM
 //               latency overlaps the dequantization and the MMAs
 // Tensor memory (512 columns x 128 lanes x 32 bit): O [0,128), S0 [128,256),
-// S1 [256,384), Q [384,448); P_j (fp16 pairs) overwrites the first 64
-// columns of S_(j mod 2) once the softmax has read them.
+// S1 [256,384), Q [384,448).  P_j (fp16 pairs) overwrites, per half h, the
+// columns [64h, 64h+32) of S_(j mod 2) once that half's scores are read; the
+// PV MMAs take their A operand from those two 32-column pieces.
 // Hand-offs are mbarriers; MMA completion arrives through tcgen05.commit.
 // Every wait is bounded (about one second of %globaltimer): on expiry the
 // CTA raises DKV_FLAG_TIMEOUT, all roles leave their loops, the MMA lane waits
@@ -37,10 +43,10 @@ namespace dkv {
 namespace {
 
 constexpr int TT = kTcTile;              // tokens per tile
-constexpr int kWarps = 22;
+constexpr int kWarps = 28;  // seven warpgroups; warps 26, 27 only complete the last one
 constexpr int kThreads = kWarps * 32;
-constexpr int kMmaWarp = 20;
-constexpr int kLoadWarp = 21;
+constexpr int kMmaWarp = 24;
+constexpr int kLoadWarp = 25;
 constexpr int kStages = 3;  // ring of packed tiles
 constexpr int kStagedProt = 24;  // protected K rows staged per tile (more: read from global)
 constexpr uint32_t kTileBytes = 128 * 128 * 2;
@@ -63,13 +69,15 @@ struct Smem {
   static constexpr uint32_t kRHdr = 20480, kRPos = 20496, kRPk = 20624;
   static constexpr uint32_t kStageBytes = 27648;
   static constexpr uint32_t kRing = 4 * kTileBytes;
-  static constexpr uint32_t kBar = kRing + kStages * kStageBytes;  // 24 mbarriers
-  static constexpr uint32_t kMisc = kBar + 24 * 8;  // tmem base, abort flag
+  static constexpr uint32_t kBar = kRing + kStages * kStageBytes;  // 32 mbarriers
+  static constexpr uint32_t kXch = kBar + 32 * 8;   // [2 parities][2 halves][128] row maxima
+  static constexpr uint32_t kLsum = kXch + 2048;    // [2 halves][128] row sums
+  static constexpr uint32_t kMisc = kLsum + 1024;   // tmem base, abort flag
   static constexpr uint32_t kBytes = kMisc + 16;
 };
 enum Bar {
   KFULL = 0, KEMPTY = 2, VFULL = 4, VEMPTY = 6, SFULL = 8, PFULL = 10, QREADY = 12, DONE = 13,
-  RFULL = 14, REMPTY = 14 + kStages
+  RFULL = 14, REMPTY = 14 + kStages, XCH = 14 + 2 * kStages, LSUM = XCH + 2
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -203,6 +211,26 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t addr, uint32_t lbo, uin
   return d;
 }
 
+// Register budgets per warpgroup after setmaxnreg (launch: 72 per thread x
+// 896 threads = 64512): softmax keeps 72 (2 x 128 threads), producers rise to
+// 80 (512 threads), control drops to 40 (128 threads): 18432 + 40960 + 5120.
+constexpr int kRegProducer = 80, kRegControl = 40;
+
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // D[tmem] (+)= A[tmem] * B[smem]^T
 __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
                                        uint32_t accumulate) {
@@ -245,9 +273,20 @@ __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
 // q = 2qh, 2qh+1.  Codes and (scale, zero) of the quantized part come from the ring
 // stage `rs` (groups of the tile in order, [group][channel][kw words]); the
 // bf16 tail, the active block and bits = 16 come straight from global memory.
+// Byte offsets of the 16-byte chunks a K producer thread (c, qh) stores:
+// chunk i (0..7) holds tokens 64 qh + 8 i .. +7 of channel c.
+struct KOffsets {
+  uint32_t o[8];
+  __device__ explicit KOffsets(int c, int qh) {
+    const uint32_t base = uint32_t(((c >> 3) * 2 + qh) * 1024 + (c & 7) * 128);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[i] = base + uint32_t(((i ^ (c & 7)) & 7) << 4);
+  }
+};
+
 template <int KB>
 __device__ void fill_k_tile(const AttnArgs& a, int u, int64_t tile_start, uint8_t* kt,
-                            const uint8_t* rs, int c, int qh) {
+                            const uint8_t* rs, int c, int qh, const KOffsets& ko) {
   const CacheView& cv = a.c;
   const int d = kHeadDim;
   if constexpr (KB < 16) {
@@ -266,7 +305,6 @@ __device__ void fill_k_tile(const AttnArgs& a, int u, int64_t tile_start, uint8_
       }
 #pragma unroll
       for (int qi = 0; qi < 2; ++qi) {
-        const int q = 2 * qh + qi;
         const __half2 s2 = __half2half2(__low2half(sz[qi]));
         const __half2 z2 = __half2half2(__high2half(sz[qi]));
         uint4 out[4];
@@ -280,8 +318,7 @@ __device__ void fill_k_tile(const AttnArgs& a, int u, int64_t tile_start, uint8_
           dequant2x16(w[qi].y, s2, z2, out[2], out[3]);
         }
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-          *reinterpret_cast<uint4*>(kt + kt_off(c, 32 * q + 8 * i)) = out[i];
+        for (int i = 0; i < 4; ++i) *reinterpret_cast<uint4*>(kt + ko.o[4 * qi + i]) = out[i];
       }
       // protected rows of this thread's two chunks
       const int* hdr = reinterpret_cast<const int*>(rs + Smem::kRHdr);
@@ -382,9 +419,21 @@ __device__ void fill_k_tile(const AttnArgs& a, int u, int64_t tile_start, uint8_
 // V tile: thread `tid` (0..255) fills items (token t, channel quarter qq) with
 // qq = item % 4, t = item / 4, item = tid + 256 r (r = 0, 1), so a warp reads
 // 512 contiguous bytes of the ring stage ([token][vw words]).
+// Byte offsets of the 16-byte chunks a V producer thread stores: item r
+// (token (tid >> 2) + 64 r, quarter tid & 3), store i = chunk (i + rot) & 3.
+struct VOffsets {
+  uint32_t base, x[4];
+  __device__ explicit VOffsets(int tid) {
+    const int qq = tid & 3, t7 = (tid >> 2) & 7, rot = qq & 2;
+    base = uint32_t(((tid >> 5) * 2 + (qq >> 1)) * 1024 + t7 * 128);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) x[i] = uint32_t(((4 * (qq & 1) + ((i + rot) & 3)) ^ t7) << 4);
+  }
+};
+
 template <int VB>
 __device__ void fill_v_tile(const AttnArgs& a, int u, int64_t tile_start, uint8_t* vt,
-                            const uint8_t* rs, int tid) {
+                            const uint8_t* rs, int tid, const VOffsets& vo) {
   const CacheView& cv = a.c;
   const int d = kHeadDim;
   if constexpr (VB < 16) {
@@ -403,7 +452,6 @@ __device__ void fill_v_tile(const AttnArgs& a, int u, int64_t tile_start, uint8_
       }
 #pragma unroll
       for (int r = 0; r < 2; ++r) {
-        const int t = (tid + 256 * r) >> 2;
         const __half2 s2 = __half2half2(__low2half(sz[r]));
         const __half2 z2 = __half2half2(__high2half(sz[r]));
         uint4 out[4];
@@ -422,7 +470,7 @@ __device__ void fill_v_tile(const AttnArgs& a, int u, int64_t tile_start, uint8_
         }
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-          *reinterpret_cast<uint4*>(vt + vt_off(t, 32 * qq + 8 * ((i + rot) & 3))) = out[i];
+          *reinterpret_cast<uint4*>(vt + vo.base + 16384u * r + vo.x[i]) = out[i];
       }
       return;
     }
@@ -514,9 +562,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
       mbar_init(bar(VFULL + b), 256);
       mbar_init(bar(VEMPTY + b), 1);
       mbar_init(bar(SFULL + b), 1);
-      mbar_init(bar(PFULL + b), 128);
+      mbar_init(bar(PFULL + b), 256);
+      mbar_init(bar(XCH + b), 256);
     }
-    mbar_init(bar(QREADY), 128);
+    mbar_init(bar(QREADY), 256);
+    mbar_init(bar(LSUM), 256);
     mbar_init(bar(DONE), 1);
     for (int st = 0; st < kStages; ++st) {
       mbar_init(bar(RFULL + st), 1);
@@ -536,162 +586,178 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp < 4) {
+  if (warp < 8) {
     // ------------------------------------------------------------ softmax
-    const int lr = threadIdx.x;         // TMEM lane = row of this block
+    const int lr = threadIdx.x & 127;   // TMEM lane = row of this block
+    const int h = threadIdx.x >> 7;     // column half of S, O and Q
     const bool row_ok = lr < rpb;       // padding rows carry Q = 0 and write nothing
     // a warp holding only padding rows skips the softmax arithmetic (its P
     // rows feed only padding rows of O, which are never read)
-    const bool warp_rows = warp * 32 < rpb;
+    const bool warp_rows = (warp & 3) * 32 < rpb;
     const int r = rb * rpb + lr;        // query row of the unit
-    const uint32_t lane_base = tmem + (uint32_t(warp * 32) << 16);
+    const uint32_t lane_base = tmem + (uint32_t((warp & 3) * 32) << 16);
+    float* xmax = reinterpret_cast<float*>(sm + Smem::kXch);   // [parity][half][row]
+    float* lsum = reinterpret_cast<float*>(sm + Smem::kLsum);  // [half][row]
+    // a negative scale is folded into Q (an exact fp16 sign flip), so scores
+    // are always multiplied by sc > 0; scale 0 (uniform weights) uses 1e-30
+    const bool qneg = a.scale_log2 < 0.f;
+    const float sc = fmaxf(fabsf(a.scale_log2), 1e-30f);
     {
-      const uint4* qrow = reinterpret_cast<const uint4*>(a.q + (size_t(u) * cv.rows + (row_ok ? r : 0)) * kHeadDim);
+      const uint4* qrow = reinterpret_cast<const uint4*>(
+          a.q + (size_t(u) * cv.rows + (row_ok ? r : 0)) * kHeadDim + 64 * h);
       uint32_t qv[32];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint4 y = row_ok ? bf16x8_to_f16x8(__ldg(qrow + h * 8 + i)) : make_uint4(0u, 0u, 0u, 0u);
-          qv[4 * i + 0] = y.x;
-          qv[4 * i + 1] = y.y;
-          qv[4 * i + 2] = y.z;
-          qv[4 * i + 3] = y.w;
-        }
-        tmem_st32(lane_base + kColQ + 32 * h, qv);
+      for (int i = 0; i < 8; ++i) {
+        uint4 y = row_ok ? bf16x8_to_f16x8(__ldg(qrow + i)) : make_uint4(0u, 0u, 0u, 0u);
+        if (qneg) y = make_uint4(y.x ^ 0x80008000u, y.y ^ 0x80008000u, y.z ^ 0x80008000u,
+                                 y.w ^ 0x80008000u);
+        qv[4 * i + 0] = y.x;
+        qv[4 * i + 1] = y.y;
+        qv[4 * i + 2] = y.z;
+        qv[4 * i + 3] = y.w;
       }
+      tmem_st32(lane_base + kColQ + 32 * h, qv);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar(QREADY));
     }
     float m_used = -__int_as_float(0x7f800000);  // reference max (log2 units)
-    float l = 0.f;
+    float l = 0.f;                                 // this half's row sum relative to m_used
     bool ok = true;
     for (int j = 0; j < nt && ok; ++j) {
       const int b = j & 1;
-      const uint32_t s_col = b ? kColS1 : kColS0;
+      const uint32_t s_col = (b ? kColS1 : kColS0) + 64 * h;
       // tcgen05.ld/st are warp-collective: every branch around them is warp-uniform
       if (!__all_sync(0xffffffffu, mbar_wait(bar(SFULL + b), (j >> 1) & 1, abort_flag, cv.status))) {
         ok = false;
         break;
       }
       tc_fence_after();
+      const int64_t tile_start = (t_begin + j) * TT;
+      const int valid = a.n_tok - tile_start < TT ? int(a.n_tok - tile_start) : TT;
+      // pass 1: max of this half's raw scores (masked tokens excluded)
+      float pm = -__int_as_float(0x7f800000);
+      if (warp_rows) {
+#pragma unroll 1
+        for (int ch = 0; ch < 2; ++ch) {
+          uint32_t sv[32];
+          tmem_ld32(lane_base + s_col + 32 * ch, sv);
+          tmem_ld_wait();
+          const int c0 = 64 * h + 32 * ch;  // first column of this chunk
+          float m4[4];
+          if (c0 + 32 <= valid) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) m4[i] = __uint_as_float(sv[i]);
+#pragma unroll
+            for (int i = 4; i < 32; i += 2)
+              m4[(i >> 1) & 3] =
+                  max3f(m4[(i >> 1) & 3], __uint_as_float(sv[i]), __uint_as_float(sv[i + 1]));
+          } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) m4[i] = -__int_as_float(0x7f800000);
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (c0 + i < valid) m4[i & 3] = fmaxf(m4[i & 3], __uint_as_float(sv[i]));
+          }
+          pm = fmaxf(pm, fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])));
+        }
+      }
+      // the row max over both halves (mbarrier exchange, bounded wait)
+      xmax[((b * 2) + h) * 128 + lr] = pm;
+      mbar_arrive(bar(XCH + b));
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(XCH + b), (j >> 1) & 1, abort_flag, cv.status))) {
+        ok = false;
+        break;
+      }
       if (!warp_rows) {
         mbar_arrive(bar(PFULL + b));
         continue;
       }
-      const int64_t tile_start = (t_begin + j) * TT;
-      const int valid = a.n_tok - tile_start < TT ? int(a.n_tok - tile_start) : TT;
-      // pass 1: row max of this tile (full tiles with scale >= 0: max of the
-      // raw scores times the scale; otherwise per element with masking)
-      const bool fast = valid >= TT && a.scale_log2 >= 0.f;
-      float mx = -__int_as_float(0x7f800000);
-#pragma unroll 1
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t sv[32];
-        tmem_ld32(lane_base + s_col + 32 * ch, sv);
-        tmem_ld_wait();
-        float m4[4];
-        if (fast) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) m4[i] = __uint_as_float(sv[i]);
-#pragma unroll
-          for (int i = 4; i < 32; ++i) m4[i & 3] = fmaxf(m4[i & 3], __uint_as_float(sv[i]));
-        } else {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) m4[i] = -__int_as_float(0x7f800000);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float x = 32 * ch + i < valid ? __uint_as_float(sv[i]) * a.scale_log2
-                                                : -__int_as_float(0x7f800000);
-            m4[i & 3] = fmaxf(m4[i & 3], x);
-          }
-        }
-        mx = fmaxf(mx, fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])));
-      }
-      if (fast) mx *= a.scale_log2;
+      const float mx = fmaxf(pm, xmax[((b * 2) + (h ^ 1)) * 128 + lr]) * sc;
       // lazy rescale: keep the reference max unless the new one exceeds it by
-      // 8 (P <= 2^8); decided per warp, rows whose max did not grow get alpha 1
-      if (__any_sync(0xffffffffu, mx > m_used + 8.f)) {
+      // 8 (P <= 2^8); both halves of a row decide alike, per warp; rows whose
+      // max did not grow get alpha 1
+      const bool rescale = __any_sync(0xffffffffu, mx > m_used + 8.f);
+      float alpha = 1.f;
+      if (rescale) {
         const float m_new = fmaxf(m_used, mx);
-        const float alpha = fast_exp2(m_used - m_new);  // 0 on the first tile
-        if (j > 0) {
-          // O must not be in use by PV(j-1)
-          const int pb = (j - 1) & 1;
-          if (!__all_sync(0xffffffffu, mbar_wait(bar(VEMPTY + pb), ((j - 1) >> 1) & 1,
-                                                 abort_flag, cv.status))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-#pragma unroll 1
-          for (int ch = 0; ch < 4; ++ch) {
-            uint32_t o[32];
-            tmem_ld32(lane_base + kColO + 32 * ch, o);
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st32(lane_base + kColO + 32 * ch, o);
-          }
-        }
+        alpha = fast_exp2(m_used - m_new);  // 0 on the first tile
         l *= alpha;
         m_used = m_new;
       }
-      // pass 2: P = 2^(s*scale - m_used) as fp16 into the first 64 columns of S_b
+      // pass 2: P = 2^(s*sc - m_used) as fp16 into columns [64h, 64h+32) of S_b
       const float nm = -m_used;
       float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
-      for (int ch = 0; ch < 4; ++ch) {
+      for (int ch = 0; ch < 2; ++ch) {
         uint32_t sv[32];
         tmem_ld32(lane_base + s_col + 32 * ch, sv);
         tmem_ld_wait();
+        const int c0 = 64 * h + 32 * ch;
+        if (c0 + 32 > valid) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (c0 + i >= valid) sv[i] = 0xff800000u;  // -inf: masked token, weight 0
+        }
         uint32_t pv[16];
-        if (valid >= TT) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float p0 = fast_exp2(fmaf(__uint_as_float(sv[2 * i]), a.scale_log2, nm));
-            const float p1 = fast_exp2(fmaf(__uint_as_float(sv[2 * i + 1]), a.scale_log2, nm));
-            l4[i & 3] += p0 + p1;
-            pv[i] = pack_h2(p0, p1);
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int c0 = 32 * ch + 2 * i;
-            const float p0 =
-                c0 < valid ? fast_exp2(fmaf(__uint_as_float(sv[2 * i]), a.scale_log2, nm)) : 0.f;
-            const float p1 =
-                c0 + 1 < valid ? fast_exp2(fmaf(__uint_as_float(sv[2 * i + 1]), a.scale_log2, nm))
-                               : 0.f;
-            l4[i & 3] += p0 + p1;
-            pv[i] = pack_h2(p0, p1);
-          }
+        for (int i = 0; i < 16; ++i) {
+          const float p0 = fast_exp2(fmaf(__uint_as_float(sv[2 * i]), sc, nm));
+          const float p1 = fast_exp2(fmaf(__uint_as_float(sv[2 * i + 1]), sc, nm));
+          l4[i & 3] += p0 + p1;
+          pv[i] = pack_h2(p0, p1);
         }
         tmem_st16(lane_base + s_col + 16 * ch, pv);
       }
       l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+      if (rescale && j > 0) {
+        // this half of O must not be in use by PV(j-1); PV(j) waits for the arrive
+        const int pb = (j - 1) & 1;
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(VEMPTY + pb), ((j - 1) >> 1) & 1,
+                                               abort_flag, cv.status))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll 1
+        for (int ch = 0; ch < 2; ++ch) {
+          uint32_t o[32];
+          tmem_ld32(lane_base + kColO + 64 * h + 32 * ch, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(lane_base + kColO + 64 * h + 32 * ch, o);
+        }
+      }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar(PFULL + b));
     }
-    // epilogue: wait for the last PV, then read O
+    // epilogue: wait for the last PV, combine the halves' row sums, write O
     if (ok && nt > 0) {
       const int jl = nt - 1;
       ok = __all_sync(0xffffffffu,
                       mbar_wait(bar(VEMPTY + (jl & 1)), (jl >> 1) & 1, abort_flag, cv.status));
     }
+    if (ok) {
+      lsum[h * 128 + lr] = l;
+      mbar_arrive(bar(LSUM));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(LSUM), 0, abort_flag, cv.status));
+    }
     if (ok && warp_rows) {
       tc_fence_after();
-      const float inv = 1.f / l;
+      const float lt = l + lsum[(h ^ 1) * 128 + lr];
+      const float inv = 1.f / lt;
 #pragma unroll 1
-      for (int ch = 0; ch < 4; ++ch) {
+      for (int ch = 0; ch < 2; ++ch) {
         uint32_t o[32];
-        tmem_ld32(lane_base + kColO + 32 * ch, o);
+        tmem_ld32(lane_base + kColO + 64 * h + 32 * ch, o);
         tmem_ld_wait();
+        const int col = 64 * h + 32 * ch;
         if (!row_ok) {
           // padding row: nothing to write
         } else if (a.nsplit == 1) {
-          uint4* dst = reinterpret_cast<uint4*>(a.out + (size_t(u) * cv.rows + r) * kHeadDim + 32 * ch);
+          uint4* dst = reinterpret_cast<uint4*>(a.out + (size_t(u) * cv.rows + r) * kHeadDim + col);
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             uint32_t w[4];
@@ -705,44 +771,51 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
           }
         } else {
           float4* dst = reinterpret_cast<float4*>(
-              a.part_o + ((size_t(u) * a.nsplit + sp) * cv.rows + r) * kHeadDim + 32 * ch);
+              a.part_o + ((size_t(u) * a.nsplit + sp) * cv.rows + r) * kHeadDim + col);
 #pragma unroll
           for (int i = 0; i < 8; ++i)
             dst[i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
                                  __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
         }
       }
-      if (a.nsplit > 1 && row_ok)
-        a.part_ml[(size_t(u) * a.nsplit + sp) * cv.rows + r] = make_float2(m_used, l);
+      if (a.nsplit > 1 && row_ok && h == 0)
+        a.part_ml[(size_t(u) * a.nsplit + sp) * cv.rows + r] = make_float2(m_used, lt);
     }
-  } else if (warp < 12) {
+  } else if (warp < 24) {
+    regs_inc<kRegProducer>();
+    if (warp < 16) {
     // ------------------------------------------------------------ K producer
-    const int c = (threadIdx.x - 128) & 127;   // channel
-    const int qh = (threadIdx.x - 128) >> 7;    // chunks 2qh, 2qh+1 of each tile
+    const int c = (threadIdx.x - 256) & 127;   // channel
+    const int qh = (threadIdx.x - 256) >> 7;    // chunks 2qh, 2qh+1 of each tile
+    const KOffsets ko(c, qh);
     for (int j = 0; j < nt; ++j) {
       const int b = j & 1, st = j % kStages;
       if (!mbar_wait(bar(KEMPTY + b), ((j >> 1) & 1) ^ 1, abort_flag, cv.status)) break;
       if (!mbar_wait(bar(RFULL + st), (j / kStages) & 1, abort_flag, cv.status)) break;
       fill_k_tile<KB>(a, u, (t_begin + j) * TT, sm + (b ? Smem::kK1 : Smem::kK0),
-                      sm + Smem::kRing + st * Smem::kStageBytes, c, qh);
+                      sm + Smem::kRing + st * Smem::kStageBytes, c, qh, ko);
       fence_async_smem();
       mbar_arrive(bar(KFULL + b));
       mbar_arrive(bar(REMPTY + st));
     }
-  } else if (warp < 20) {
+    } else {
     // ------------------------------------------------------------ V producer
-    const int t = threadIdx.x - 384;
+    const int t = threadIdx.x - 512;
+    const VOffsets vo(t);
     for (int j = 0; j < nt; ++j) {
       const int b = j & 1, st = j % kStages;
       if (!mbar_wait(bar(VEMPTY + b), ((j >> 1) & 1) ^ 1, abort_flag, cv.status)) break;
       if (!mbar_wait(bar(RFULL + st), (j / kStages) & 1, abort_flag, cv.status)) break;
       fill_v_tile<VB>(a, u, (t_begin + j) * TT, sm + (b ? Smem::kV1 : Smem::kV0),
-                      sm + Smem::kRing + st * Smem::kStageBytes, t);
+                      sm + Smem::kRing + st * Smem::kStageBytes, t, vo);
       fence_async_smem();
       mbar_arrive(bar(VFULL + b));
       mbar_arrive(bar(REMPTY + st));
     }
-  } else if (warp == kLoadWarp) {
+    }
+  } else {
+    regs_dec<kRegControl>();
+    if (warp == kLoadWarp) {
     // ------------------------------------------------------------ loader
     // lanes prefetch the side-table group index of 32 tiles at a time; lane 0
     // issues the bulk copies of each tile
@@ -824,7 +897,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
     if (lane == 0)
       for (int j = issued > kStages ? issued - kStages : 0; j < issued; ++j)
         mbar_wait(bar(RFULL + j % kStages), (j / kStages) & 1, abort_flag, cv.status, true);
-  } else if (lane == 0) {
+    } else if (warp == kMmaWarp && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
     bool ok = mbar_wait(bar(QREADY), 0, abort_flag, cv.status);
     tc_fence_after();
@@ -836,9 +909,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
       const uint32_t vbase = sm_base + (bb ? Smem::kV1 : Smem::kV0);
       const uint32_t p_col = bb ? kColS1 : kColS0;
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        mma_ts(tmem + kColO, tmem + p_col + 8 * kk, sdesc_sw128(vbase + 4096 * kk, 1024, 2048),
-               (i > 0 || kk > 0) ? 1u : 0u);
+      for (int kk = 0; kk < 8; ++kk)  // tokens 16kk..: P half kk/4, packed column 8(kk%4)
+        mma_ts(tmem + kColO, tmem + p_col + 64 * (kk >> 2) + 8 * (kk & 3),
+               sdesc_sw128(vbase + 4096 * kk, 1024, 2048), (i > 0 || kk > 0) ? 1u : 0u);
       mma_commit(bar(VEMPTY + bb));
       return true;
     };
@@ -860,6 +933,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
     // drain: every MMA issued above completes before TMEM is released
     mma_commit(bar(DONE));
     mbar_wait(bar(DONE), 0, abort_flag, cv.status, /*drain=*/true);
+    }
   }
 
   tc_fence_before();
