@@ -70,14 +70,14 @@ struct Smem {
   static constexpr uint32_t kStageBytes = 27648;
   static constexpr uint32_t kRing = 4 * kTileBytes;
   static constexpr uint32_t kBar = kRing + kStages * kStageBytes;  // 32 mbarriers
-  static constexpr uint32_t kXch = kBar + 32 * 8;   // [2 parities][2 halves][128] row maxima
-  static constexpr uint32_t kLsum = kXch + 2048;    // [2 halves][128] row sums
-  static constexpr uint32_t kMisc = kLsum + 1024;   // tmem base, abort flag
+  static constexpr uint32_t kRef = kBar + 32 * 8;   // [tile parity][128] reference max per row
+  static constexpr uint32_t kLsum = kRef + 1024;    // [warpgroup][128] row sum, then its reference
+  static constexpr uint32_t kMisc = kLsum + 2048;   // tmem base, abort flag
   static constexpr uint32_t kBytes = kMisc + 16;
 };
 enum Bar {
   KFULL = 0, KEMPTY = 2, VFULL = 4, VEMPTY = 6, SFULL = 8, PFULL = 10, QREADY = 12, DONE = 13,
-  RFULL = 14, REMPTY = 14 + kStages, XCH = 14 + 2 * kStages, LSUM = XCH + 2
+  RFULL = 14, REMPTY = 14 + kStages, RREADY = 14 + 2 * kStages, LSUM = RREADY + 2
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -108,6 +108,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(bar), "r"(parity), "r"(200000u)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
       : "memory");
   return ok != 0;
 }
@@ -184,6 +196,22 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       : "memory");
 }
 
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(
+                   taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+               "r"(r[7])
+               : "memory");
+}
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
@@ -212,9 +240,9 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t addr, uint32_t lbo, uin
 }
 
 // Register budgets per warpgroup after setmaxnreg (launch: 72 per thread x
-// 896 threads = 64512): softmax keeps 72 (2 x 128 threads), producers rise to
-// 80 (512 threads), control drops to 40 (128 threads): 18432 + 40960 + 5120.
-constexpr int kRegProducer = 80, kRegControl = 40;
+// 896 threads = 64512): softmax rises to 88 (2 x 128 threads), producers keep
+// 72 (512 threads), control drops to 40 (128 threads): 22528 + 36864 + 5120.
+constexpr int kRegSoftmax = 88, kRegControl = 40;
 
 template <int N>
 __device__ __forceinline__ void regs_inc() {
@@ -225,6 +253,31 @@ __device__ __forceinline__ void regs_dec() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
+// Packed fp32 pairs (sm_100 f32x2 arithmetic): one instruction for two lanes'
+// worth of fma / add / mul, operands as 64-bit register pairs {lo, hi}.
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t x, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(x));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
 __device__ __forceinline__ float max3f(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
@@ -285,8 +338,17 @@ struct KOffsets {
 };
 
 template <int KB>
-__device__ void fill_k_tile(const AttnArgs& a, int u, int64_t tile_start, uint8_t* kt,
-                            const uint8_t* rs, int c, int qh, const KOffsets& ko) {
+__device__ __noinline__ void fill_k_general(const AttnArgs& a, int u, int64_t tile_start,
+                                            uint8_t* kt, const uint8_t* rs, int c, int qh);
+
+// K tile, channel c, token chunks 2qh, 2qh+1.  The whole-quantized-tile case
+// is inline; tiles that reach the bf16 tail or the active block take the
+// out-of-line general path (at most two per call), which keeps the hot loop's
+// code small.
+template <int KB>
+__device__ __forceinline__ void fill_k_tile(const AttnArgs& a, int u, int64_t tile_start,
+                                            uint8_t* kt, const uint8_t* rs, int c, int qh,
+                                            const KOffsets& ko) {
   const CacheView& cv = a.c;
   const int d = kHeadDim;
   if constexpr (KB < 16) {
@@ -339,6 +401,14 @@ __device__ void fill_k_tile(const AttnArgs& a, int u, int64_t tile_start, uint8_
       return;
     }
   }
+  fill_k_general<KB>(a, u, tile_start, kt, rs, c, qh);
+}
+
+template <int KB>
+__device__ __noinline__ void fill_k_general(const AttnArgs& a, int u, int64_t tile_start,
+                                            uint8_t* kt, const uint8_t* rs, int c, int qh) {
+  const CacheView& cv = a.c;
+  const int d = kHeadDim;
 #pragma unroll 1
   for (int q = 2 * qh; q < 2 * qh + 2; ++q) {
     const int64_t pos0 = tile_start + 32 * q;
@@ -432,10 +502,15 @@ struct VOffsets {
 };
 
 template <int VB>
-__device__ void fill_v_tile(const AttnArgs& a, int u, int64_t tile_start, uint8_t* vt,
-                            const uint8_t* rs, int tid, const VOffsets& vo) {
+__device__ __noinline__ void fill_v_general(const AttnArgs& a, int u, int64_t tile_start,
+                                            uint8_t* vt, const uint8_t* rs, int tid);
+
+// V tile: the whole-quantized-tile case inline, the rest out of line
+template <int VB>
+__device__ __forceinline__ void fill_v_tile(const AttnArgs& a, int u, int64_t tile_start,
+                                            uint8_t* vt, const uint8_t* rs, int tid,
+                                            const VOffsets& vo) {
   const CacheView& cv = a.c;
-  const int d = kHeadDim;
   if constexpr (VB < 16) {
     if (tile_start + TT <= a.L) {
       // whole tile quantized: issue every shared-memory load, then dequantize
@@ -475,6 +550,14 @@ __device__ void fill_v_tile(const AttnArgs& a, int u, int64_t tile_start, uint8_
       return;
     }
   }
+  fill_v_general<VB>(a, u, tile_start, vt, rs, tid);
+}
+
+template <int VB>
+__device__ __noinline__ void fill_v_general(const AttnArgs& a, int u, int64_t tile_start,
+                                            uint8_t* vt, const uint8_t* rs, int tid) {
+  const CacheView& cv = a.c;
+  const int d = kHeadDim;
 #pragma unroll 1
   for (int r = 0; r < 2; ++r) {
     const int item = tid + 256 * r;
@@ -531,7 +614,7 @@ __device__ void fill_v_tile(const AttnArgs& a, int u, int64_t tile_start, uint8_
 // ------------------------------------------------------------------ kernel
 
 template <int KB, int VB>
-__global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
+__global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~uintptr_t(1023));
@@ -562,8 +645,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
       mbar_init(bar(VFULL + b), 256);
       mbar_init(bar(VEMPTY + b), 1);
       mbar_init(bar(SFULL + b), 1);
-      mbar_init(bar(PFULL + b), 256);
-      mbar_init(bar(XCH + b), 256);
+      mbar_init(bar(PFULL + b), 128);
+      mbar_init(bar(RREADY + b), 128);
     }
     mbar_init(bar(QREADY), 256);
     mbar_init(bar(LSUM), 256);
@@ -588,16 +671,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
 
   if (warp < 8) {
     // ------------------------------------------------------------ softmax
+    regs_inc<kRegSoftmax>();
     const int lr = threadIdx.x & 127;   // TMEM lane = row of this block
-    const int h = threadIdx.x >> 7;     // column half of S, O and Q
+    const int h = threadIdx.x >> 7;     // warpgroup: tiles j = h (mod 2); Q / output half h
     const bool row_ok = lr < rpb;       // padding rows carry Q = 0 and write nothing
     // a warp holding only padding rows skips the softmax arithmetic (its P
     // rows feed only padding rows of O, which are never read)
     const bool warp_rows = (warp & 3) * 32 < rpb;
     const int r = rb * rpb + lr;        // query row of the unit
     const uint32_t lane_base = tmem + (uint32_t((warp & 3) * 32) << 16);
-    float* xmax = reinterpret_cast<float*>(sm + Smem::kXch);   // [parity][half][row]
-    float* lsum = reinterpret_cast<float*>(sm + Smem::kLsum);  // [half][row]
+    float* ref = reinterpret_cast<float*>(sm + Smem::kRef);    // [tile parity][row]
+    float* lsum = reinterpret_cast<float*>(sm + Smem::kLsum);  // [warpgroup][row], then refs
     // a negative scale is folded into Q (an exact fp16 sign flip), so scores
     // are always multiplied by sc > 0; scale 0 (uniform weights) uses 1e-30
     const bool qneg = a.scale_log2 < 0.f;
@@ -621,119 +705,143 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
       tc_fence_before();
       mbar_arrive(bar(QREADY));
     }
-    float m_used = -__int_as_float(0x7f800000);  // reference max (log2 units)
-    float l = 0.f;                                 // this half's row sum relative to m_used
+    // Every tile j has one reference max per row, r_j (log2 units), non-
+    // decreasing in j: r_j = r_(j-1) unless the tile's max exceeds it by more
+    // than 8 (P <= 2^8), then r_j = max(r_(j-1), tile max).  O always holds
+    // its sum relative to the reference of the last PV; this warpgroup's row
+    // sum l is relative to r_w, the reference of its own last tile.
+    float r_w = -__int_as_float(0x7f800000);
+    float l = 0.f;
     bool ok = true;
-    for (int j = 0; j < nt && ok; ++j) {
-      const int b = j & 1;
-      const uint32_t s_col = (b ? kColS1 : kColS0) + 64 * h;
+    for (int j = h; j < nt && ok; j += 2) {
+      const int b = h;  // S buffer, reference slot and barriers of this warpgroup's tiles
+      const uint32_t s_col = b ? kColS1 : kColS0;
       // tcgen05.ld/st are warp-collective: every branch around them is warp-uniform
       if (!__all_sync(0xffffffffu, mbar_wait(bar(SFULL + b), (j >> 1) & 1, abort_flag, cv.status))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const int64_t tile_start = (t_begin + j) * TT;
-      const int valid = a.n_tok - tile_start < TT ? int(a.n_tok - tile_start) : TT;
-      // pass 1: max of this half's raw scores (masked tokens excluded)
-      float pm = -__int_as_float(0x7f800000);
-      if (warp_rows) {
-#pragma unroll 1
-        for (int ch = 0; ch < 2; ++ch) {
-          uint32_t sv[32];
-          tmem_ld32(lane_base + s_col + 32 * ch, sv);
-          tmem_ld_wait();
-          const int c0 = 64 * h + 32 * ch;  // first column of this chunk
-          float m4[4];
-          if (c0 + 32 <= valid) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) m4[i] = __uint_as_float(sv[i]);
-#pragma unroll
-            for (int i = 4; i < 32; i += 2)
-              m4[(i >> 1) & 3] =
-                  max3f(m4[(i >> 1) & 3], __uint_as_float(sv[i]), __uint_as_float(sv[i + 1]));
-          } else {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) m4[i] = -__int_as_float(0x7f800000);
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (c0 + i < valid) m4[i & 3] = fmaxf(m4[i & 3], __uint_as_float(sv[i]));
-          }
-          pm = fmaxf(pm, fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])));
-        }
-      }
-      // the row max over both halves (mbarrier exchange, bounded wait)
-      xmax[((b * 2) + h) * 128 + lr] = pm;
-      mbar_arrive(bar(XCH + b));
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(XCH + b), (j >> 1) & 1, abort_flag, cv.status))) {
-        ok = false;
-        break;
-      }
       if (!warp_rows) {
+        mbar_arrive(bar(RREADY + b));
         mbar_arrive(bar(PFULL + b));
         continue;
       }
-      const float mx = fmaxf(pm, xmax[((b * 2) + (h ^ 1)) * 128 + lr]) * sc;
-      // lazy rescale: keep the reference max unless the new one exceeds it by
-      // 8 (P <= 2^8); both halves of a row decide alike, per warp; rows whose
-      // max did not grow get alpha 1
-      const bool rescale = __any_sync(0xffffffffu, mx > m_used + 8.f);
-      float alpha = 1.f;
-      if (rescale) {
-        const float m_new = fmaxf(m_used, mx);
-        alpha = fast_exp2(m_used - m_new);  // 0 on the first tile
-        l *= alpha;
-        m_used = m_new;
-      }
-      // pass 2: P = 2^(s*sc - m_used) as fp16 into columns [64h, 64h+32) of S_b
-      const float nm = -m_used;
-      float l4[4] = {0.f, 0.f, 0.f, 0.f};
+      const int64_t tile_start = (t_begin + j) * TT;
+      const int valid = a.n_tok - tile_start < TT ? int(a.n_tok - tile_start) : TT;
+      // pass 1: max of the raw scores (masked tokens excluded), 64 columns per wait
+      float pm = -__int_as_float(0x7f800000);
 #pragma unroll 1
-      for (int ch = 0; ch < 2; ++ch) {
-        uint32_t sv[32];
-        tmem_ld32(lane_base + s_col + 32 * ch, sv);
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t sv[32], sw[32];
+        tmem_ld32(lane_base + s_col + 64 * hh, sv);
+        tmem_ld32(lane_base + s_col + 64 * hh + 32, sw);
         tmem_ld_wait();
-        const int c0 = 64 * h + 32 * ch;
-        if (c0 + 32 > valid) {
+        if (64 * hh + 64 > valid) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (c0 + i >= valid) sv[i] = 0xff800000u;  // -inf: masked token, weight 0
+          for (int i = 0; i < 32; ++i) {
+            if (64 * hh + i >= valid) sv[i] = 0xff800000u;
+            if (64 * hh + 32 + i >= valid) sw[i] = 0xff800000u;
+          }
         }
-        uint32_t pv[16];
+        float m4[4];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float p0 = fast_exp2(fmaf(__uint_as_float(sv[2 * i]), sc, nm));
-          const float p1 = fast_exp2(fmaf(__uint_as_float(sv[2 * i + 1]), sc, nm));
-          l4[i & 3] += p0 + p1;
+        for (int i = 0; i < 4; ++i) m4[i] = fmaxf(__uint_as_float(sv[i]), __uint_as_float(sw[i]));
+#pragma unroll
+        for (int i = 4; i < 32; ++i)
+          m4[i & 3] = max3f(m4[i & 3], __uint_as_float(sv[i]), __uint_as_float(sw[i]));
+        pm = max3f(pm, fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+      }
+      const float mx = pm * sc;
+      // the previous tile's reference (bounded wait on the other warpgroup)
+      float r_prev = -__int_as_float(0x7f800000);
+      if (j > 0) {
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(RREADY + (b ^ 1)), ((j - 1) >> 1) & 1,
+                                               abort_flag, cv.status))) {
+          ok = false;
+          break;
+        }
+        r_prev = ref[(b ^ 1) * 128 + lr];
+      }
+      // lazy rescale, decided per warp; rows whose max did not grow keep r_prev
+      const bool rescale = __any_sync(0xffffffffu, mx > r_prev + 8.f);
+      const float r_j = rescale ? fmaxf(r_prev, mx) : r_prev;
+      ref[b * 128 + lr] = r_j;
+      mbar_arrive(bar(RREADY + b));
+      l *= fast_exp2(r_w - r_j);  // 1 when unchanged, 0 on this warpgroup's first tile
+      r_w = r_j;
+      // pass 2: P = 2^(s*sc - r_j) as fp16 pairs into columns [0, 64) of S_b;
+      // 16-column chunks, the load of chunk c+1 in flight while chunk c is computed
+      const uint64_t sc2 = f2pack(sc, sc), nm2 = f2pack(-r_j, -r_j);
+      uint64_t l2[2] = {0ull, 0ull};  // two packed pairs of partial row sums
+      uint32_t va[16], vb[16];
+      auto chunk = [&](uint32_t (&v)[16], int c) {
+        if (16 * c + 16 > valid) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            if (16 * c + i >= valid) v[i] = 0xff800000u;  // -inf: masked token, weight 0
+        }
+        uint32_t pv[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          float x0, x1;
+          f2unpack(ffma2(f2pack(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])), sc2, nm2),
+                   x0, x1);
+          const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+          l2[i & 1] = fadd2(l2[i & 1], f2pack(p0, p1));
           pv[i] = pack_h2(p0, p1);
         }
-        tmem_st16(lane_base + s_col + 16 * ch, pv);
+        tmem_st8(lane_base + s_col + 8 * c, pv);
+      };
+      tmem_ld16(lane_base + s_col, va);
+      tmem_ld_wait();
+#pragma unroll 1
+      for (int c = 0; c < 8; c += 2) {
+        tmem_ld16(lane_base + s_col + 16 * (c + 1), vb);
+        chunk(va, c);
+        tmem_ld_wait();
+        if (c + 2 < 8) tmem_ld16(lane_base + s_col + 16 * (c + 2), va);
+        chunk(vb, c + 1);
+        if (c + 2 < 8) tmem_ld_wait();
       }
-      l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+      {
+        float a0, a1, b0, b1;
+        f2unpack(l2[0], a0, a1);
+        f2unpack(l2[1], b0, b1);
+        l += (a0 + b0) + (a1 + b1);
+      }
       if (rescale && j > 0) {
-        // this half of O must not be in use by PV(j-1); PV(j) waits for the arrive
-        const int pb = (j - 1) & 1;
-        if (!__all_sync(0xffffffffu, mbar_wait(bar(VEMPTY + pb), ((j - 1) >> 1) & 1,
+        // O holds PV(j-1) relative to r_prev: scale it to r_j once PV(j-1) is
+        // done; PV(j) waits for this warpgroup's arrive below
+        const float alpha = fast_exp2(r_prev - r_j);
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(VEMPTY + (b ^ 1)), ((j - 1) >> 1) & 1,
                                                abort_flag, cv.status))) {
           ok = false;
           break;
         }
         tc_fence_after();
 #pragma unroll 1
-        for (int ch = 0; ch < 2; ++ch) {
+        for (int ch = 0; ch < 4; ++ch) {
           uint32_t o[32];
-          tmem_ld32(lane_base + kColO + 64 * h + 32 * ch, o);
+          tmem_ld32(lane_base + kColO + 32 * ch, o);
           tmem_ld_wait();
+          const uint64_t al2 = f2pack(alpha, alpha);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(lane_base + kColO + 64 * h + 32 * ch, o);
+          for (int i = 0; i < 32; i += 2) {
+            float x0, x1;
+            f2unpack(fmul2(f2pack(__uint_as_float(o[i]), __uint_as_float(o[i + 1])), al2), x0, x1);
+            o[i] = __float_as_uint(x0);
+            o[i + 1] = __float_as_uint(x1);
+          }
+          tmem_st32(lane_base + kColO + 32 * ch, o);
         }
       }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar(PFULL + b));
     }
-    // epilogue: wait for the last PV, combine the halves' row sums, write O
+    // epilogue: wait for the last PV, combine the two warpgroups' row sums at
+    // the final reference (the largest, references never decrease), write O
     if (ok && nt > 0) {
       const int jl = nt - 1;
       ok = __all_sync(0xffffffffu,
@@ -741,12 +849,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
     }
     if (ok) {
       lsum[h * 128 + lr] = l;
+      lsum[256 + h * 128 + lr] = r_w;
       mbar_arrive(bar(LSUM));
       ok = __all_sync(0xffffffffu, mbar_wait(bar(LSUM), 0, abort_flag, cv.status));
     }
     if (ok && warp_rows) {
       tc_fence_after();
-      const float lt = l + lsum[(h ^ 1) * 128 + lr];
+      const float lo = lsum[(h ^ 1) * 128 + lr], ro = lsum[256 + (h ^ 1) * 128 + lr];
+      const float rf = fmaxf(r_w, ro);
+      // a warpgroup without tiles has l = 0 and reference -inf: weight 2^-inf = 0
+      const float lt = l * fast_exp2(r_w - rf) + lo * fast_exp2(ro - rf);
       const float inv = 1.f / lt;
 #pragma unroll 1
       for (int ch = 0; ch < 2; ++ch) {
@@ -779,10 +891,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
         }
       }
       if (a.nsplit > 1 && row_ok && h == 0)
-        a.part_ml[(size_t(u) * a.nsplit + sp) * cv.rows + r] = make_float2(m_used, lt);
+        a.part_ml[(size_t(u) * a.nsplit + sp) * cv.rows + r] = make_float2(rf, lt);
     }
   } else if (warp < 24) {
-    regs_inc<kRegProducer>();
     if (warp < 16) {
     // ------------------------------------------------------------ K producer
     const int c = (threadIdx.x - 256) & 127;   // channel
@@ -901,35 +1012,64 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
     // ------------------------------------------------------------ MMA issuer
     bool ok = mbar_wait(bar(QREADY), 0, abort_flag, cv.status);
     tc_fence_after();
-    auto issue_pv = [&](int i) -> bool {
-      const int bb = i & 1;
-      if (!mbar_wait(bar(PFULL + bb), (i >> 1) & 1, abort_flag, cv.status)) return false;
-      if (!mbar_wait(bar(VFULL + bb), (i >> 1) & 1, abort_flag, cv.status)) return false;
-      tc_fence_after();
-      const uint32_t vbase = sm_base + (bb ? Smem::kV1 : Smem::kV0);
-      const uint32_t p_col = bb ? kColS1 : kColS0;
+    // QK(j) needs K_j (KFULL) and S_(j mod 2) free, i.e. PV(j-2) issued; PV(i)
+    // needs P_i (PFULL) and V_i (VFULL).  Whichever is ready is issued, PV
+    // first, so a late K tile never holds back a ready PV.  Barrier phases
+    // cannot run ahead: each next phase needs an MMA issued here first.
+    int nq = 0, np = 0;
+    uint64_t t0 = 0;
+    uint32_t idle = 0;
+    while (ok && np < nt) {
+      bool progress = false;
+      if (np < nq && mbar_test(bar(PFULL + (np & 1)), (np >> 1) & 1) &&
+          mbar_test(bar(VFULL + (np & 1)), (np >> 1) & 1)) {
+        tc_fence_after();
+        const int bb = np & 1;
+        const uint32_t vbase = sm_base + (bb ? Smem::kV1 : Smem::kV0);
+        const uint32_t p_col = bb ? kColS1 : kColS0;
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk)  // tokens 16kk..: P half kk/4, packed column 8(kk%4)
-        mma_ts(tmem + kColO, tmem + p_col + 64 * (kk >> 2) + 8 * (kk & 3),
-               sdesc_sw128(vbase + 4096 * kk, 1024, 2048), (i > 0 || kk > 0) ? 1u : 0u);
-      mma_commit(bar(VEMPTY + bb));
-      return true;
-    };
-    for (int j = 0; j < nt && ok; ++j) {
-      const int b = j & 1;
-      if (!mbar_wait(bar(KFULL + b), (j >> 1) & 1, abort_flag, cv.status)) { ok = false; break; }
-      tc_fence_after();
-      const uint32_t kbase = sm_base + (b ? Smem::kK1 : Smem::kK0);
-      const uint32_t s_col = b ? kColS1 : kColS0;
+        for (int kk = 0; kk < 8; ++kk)  // tokens 16kk..16kk+15: packed P columns 8kk..8kk+7
+          mma_ts(tmem + kColO, tmem + p_col + 8 * kk, sdesc_sw128(vbase + 4096 * kk, 1024, 2048),
+                 (np > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(bar(VEMPTY + bb));
+        ++np;
+        progress = true;
+      }
+      if (nq < nt && nq <= np + 1 && mbar_test(bar(KFULL + (nq & 1)), (nq >> 1) & 1)) {
+        tc_fence_after();
+        const int b = nq & 1;
+        const uint32_t kbase = sm_base + (b ? Smem::kK1 : Smem::kK0);
+        const uint32_t s_col = b ? kColS1 : kColS0;
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        mma_ts(tmem + s_col, tmem + kColQ + 8 * kk, sdesc_sw128(kbase + 4096 * kk, 1024, 2048),
-               kk > 0 ? 1u : 0u);
-      mma_commit(bar(KEMPTY + b));
-      mma_commit(bar(SFULL + b));
-      if (j > 0 && !issue_pv(j - 1)) { ok = false; break; }
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tmem + s_col, tmem + kColQ + 8 * kk, sdesc_sw128(kbase + 4096 * kk, 1024, 2048),
+                 kk > 0 ? 1u : 0u);
+        mma_commit(bar(KEMPTY + b));
+        mma_commit(bar(SFULL + b));
+        ++nq;
+        progress = true;
+      }
+      if (progress) {
+        t0 = 0;
+        idle = 0;
+      } else if ((++idle & 15u) == 0) {
+        // bounded: give up on another thread's abort or after kTimeoutNs
+        if (*abort_flag) {
+          ok = false;
+        } else {
+          const uint64_t now = globaltimer();
+          if (t0 == 0) {
+            t0 = now;
+          } else if (now - t0 > kTimeoutNs) {
+            *abort_flag = 1;
+            atomicOr(cv.status, uint32_t(DKV_FLAG_TIMEOUT));
+            ok = false;
+          }
+        }
+      } else {
+        __nanosleep(32);
+      }
     }
-    if (ok && nt > 0) ok = issue_pv(nt - 1);
     // drain: every MMA issued above completes before TMEM is released
     mma_commit(bar(DONE));
     mbar_wait(bar(DONE), 0, abort_flag, cv.status, /*drain=*/true);
