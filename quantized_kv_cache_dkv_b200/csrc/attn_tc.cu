@@ -330,10 +330,18 @@ __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
 // chunk i (0..7) holds tokens 64 qh + 8 i .. +7 of channel c.
 struct KOffsets {
   uint32_t o[8];
-  __device__ explicit KOffsets(int c, int qh) {
+  uint32_t w[2], z[2];  // ring offsets of chunk 2qh+qi: code words (uint32), (scale, zero) pairs
+  __device__ KOffsets(int c, int qh, int GK, int kw, int kb) {
     const uint32_t base = uint32_t(((c >> 3) * 2 + qh) * 1024 + (c & 7) * 128);
 #pragma unroll
     for (int i = 0; i < 8; ++i) o[i] = base + uint32_t(((i ^ (c & 7)) & 7) << 4);
+#pragma unroll
+    for (int qi = 0; qi < 2; ++qi) {
+      const int q = 2 * qh + qi;
+      const int gi = (32 * q) / GK, off = (32 * q) % GK;
+      w[qi] = uint32_t((gi * kHeadDim + c) * kw + off * kb / 32);
+      z[qi] = uint32_t(gi * kHeadDim + c);
+    }
   }
 };
 
@@ -353,40 +361,37 @@ __device__ __forceinline__ void fill_k_tile(const AttnArgs& a, int u, int64_t ti
   const int d = kHeadDim;
   if constexpr (KB < 16) {
     if (tile_start + TT <= a.Lq) {
-      // whole tile quantized: issue every shared-memory load, then dequantize
+      // whole tile quantized: one 32-token chunk per iteration (a rolled
+      // loop keeps the hot code small)
       using W = typename std::conditional<KB == 4, uint4, uint2>::type;
-      W w[2];
-      __half2 sz[2];
-#pragma unroll
+#pragma unroll 1
       for (int qi = 0; qi < 2; ++qi) {
-        const int q = 2 * qh + qi;
-        const int gi = (32 * q) / cv.GK, o = (32 * q) % cv.GK;
-        w[qi] = *reinterpret_cast<const W*>(reinterpret_cast<const uint32_t*>(rs + Smem::kRKc) +
-                                            (gi * d + c) * cv.kw + o * KB / 32);
-        sz[qi] = reinterpret_cast<const __half2*>(rs + Smem::kRKsz)[gi * d + c];
-      }
-#pragma unroll
-      for (int qi = 0; qi < 2; ++qi) {
-        const __half2 s2 = __half2half2(__low2half(sz[qi]));
-        const __half2 z2 = __half2half2(__high2half(sz[qi]));
+        const W w = *reinterpret_cast<const W*>(reinterpret_cast<const uint32_t*>(rs + Smem::kRKc) +
+                                                (qi ? ko.w[1] : ko.w[0]));
+        const __half2 sz = reinterpret_cast<const __half2*>(rs + Smem::kRKsz)[qi ? ko.z[1] : ko.z[0]];
+        const __half2 s2 = __half2half2(__low2half(sz));
+        const __half2 z2 = __half2half2(__high2half(sz));
         uint4 out[4];
         if constexpr (KB == 4) {
-          out[0] = dequant4x8(w[qi].x, s2, z2);
-          out[1] = dequant4x8(w[qi].y, s2, z2);
-          out[2] = dequant4x8(w[qi].z, s2, z2);
-          out[3] = dequant4x8(w[qi].w, s2, z2);
+          out[0] = dequant4x8(w.x, s2, z2);
+          out[1] = dequant4x8(w.y, s2, z2);
+          out[2] = dequant4x8(w.z, s2, z2);
+          out[3] = dequant4x8(w.w, s2, z2);
         } else {
-          dequant2x16(w[qi].x, s2, z2, out[0], out[1]);
-          dequant2x16(w[qi].y, s2, z2, out[2], out[3]);
+          dequant2x16(w.x, s2, z2, out[0], out[1]);
+          dequant2x16(w.y, s2, z2, out[2], out[3]);
         }
+        // chunk 1's offsets are chunk 0's shifted by +-64 bytes (bit 2 of the swizzle)
+        uint8_t* dst = kt + (qi ? int(ko.o[4]) - int(ko.o[0]) : 0);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) *reinterpret_cast<uint4*>(kt + ko.o[4 * qi + i]) = out[i];
+        for (int i = 0; i < 4; ++i) *reinterpret_cast<uint4*>(dst + ko.o[i]) = out[i];
       }
       // protected rows of this thread's two chunks
       const int* hdr = reinterpret_cast<const int*>(rs + Smem::kRHdr);
       const int n = hdr[0], g0 = hdr[1], pbase = hdr[2];
       const int* rpos = reinterpret_cast<const int*>(rs + Smem::kRPos);
       const uint16_t* rpk = reinterpret_cast<const uint16_t*>(rs + Smem::kRPk);
+#pragma unroll 1
       for (int i = 0; i < n; ++i) {
         const int pos = i < kStagedProt ? rpos[g0 + i - pbase]
                                         : __ldg(cv.prot_pos + size_t(u) * cv.P + g0 + i);
@@ -493,11 +498,18 @@ __device__ __noinline__ void fill_k_general(const AttnArgs& a, int u, int64_t ti
 // (token (tid >> 2) + 64 r, quarter tid & 3), store i = chunk (i + rot) & 3.
 struct VOffsets {
   uint32_t base, x[4];
-  __device__ explicit VOffsets(int tid) {
+  uint32_t w[2], z[2];  // ring offsets of item r: code words (uint32), (scale, zero) pairs
+  __device__ VOffsets(int tid, int vw, int vgroups, int GV, int vb) {
     const int qq = tid & 3, t7 = (tid >> 2) & 7, rot = qq & 2;
     base = uint32_t(((tid >> 5) * 2 + (qq >> 1)) * 1024 + t7 * 128);
 #pragma unroll
     for (int i = 0; i < 4; ++i) x[i] = uint32_t(((4 * (qq & 1) + ((i + rot) & 3)) ^ t7) << 4);
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int t = (tid + 256 * r) >> 2;
+      w[r] = uint32_t(t * vw + qq * (vb == 4 ? 4 : 2));
+      z[r] = uint32_t(t * vgroups + (qq * 32) / GV);
+    }
   }
 };
 
@@ -513,39 +525,32 @@ __device__ __forceinline__ void fill_v_tile(const AttnArgs& a, int u, int64_t ti
   const CacheView& cv = a.c;
   if constexpr (VB < 16) {
     if (tile_start + TT <= a.L) {
-      // whole tile quantized: issue every shared-memory load, then dequantize
+      // whole tile quantized: one item per iteration (a rolled loop keeps
+      // the hot code small)
       using W = typename std::conditional<VB == 4, uint4, uint2>::type;
-      W w[2];
-      __half2 sz[2];
-      const int qq = tid & 3, rot = qq & 2;
-#pragma unroll
+      const bool rot = (tid & 2) != 0;
+#pragma unroll 1
       for (int r = 0; r < 2; ++r) {
-        const int t = (tid + 256 * r) >> 2;
-        w[r] = *reinterpret_cast<const W*>(reinterpret_cast<const uint32_t*>(rs + Smem::kRVc) +
-                                           t * cv.vw + qq * (VB == 4 ? 4 : 2));
-        sz[r] = reinterpret_cast<const __half2*>(rs + Smem::kRVsz)[t * cv.vgroups + (qq * 32) / cv.GV];
-      }
-#pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        const __half2 s2 = __half2half2(__low2half(sz[r]));
-        const __half2 z2 = __half2half2(__high2half(sz[r]));
+        W x = *reinterpret_cast<const W*>(reinterpret_cast<const uint32_t*>(rs + Smem::kRVc) +
+                                          (r ? vo.w[1] : vo.w[0]));
+        const __half2 sz = reinterpret_cast<const __half2*>(rs + Smem::kRVsz)[r ? vo.z[1] : vo.z[0]];
+        const __half2 s2 = __half2half2(__low2half(sz));
+        const __half2 z2 = __half2half2(__high2half(sz));
         uint4 out[4];
         if constexpr (VB == 4) {
-          uint4 x = w[r];
           if (rot) x = make_uint4(x.z, x.w, x.x, x.y);
           out[0] = dequant4x8(x.x, s2, z2);
           out[1] = dequant4x8(x.y, s2, z2);
           out[2] = dequant4x8(x.z, s2, z2);
           out[3] = dequant4x8(x.w, s2, z2);
         } else {
-          uint2 x = w[r];
           if (rot) x = make_uint2(x.y, x.x);
           dequant2x16(x.x, s2, z2, out[0], out[1]);
           dequant2x16(x.y, s2, z2, out[2], out[3]);
         }
+        uint8_t* dst = vt + vo.base + 16384u * uint32_t(r);
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-          *reinterpret_cast<uint4*>(vt + vo.base + 16384u * r + vo.x[i]) = out[i];
+        for (int i = 0; i < 4; ++i) *reinterpret_cast<uint4*>(dst + vo.x[i]) = out[i];
       }
       return;
     }
@@ -713,6 +718,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     float r_w = -__int_as_float(0x7f800000);
     float l = 0.f;
     bool ok = true;
+#pragma unroll 1
     for (int j = h; j < nt && ok; j += 2) {
       const int b = h;  // S buffer, reference slot and barriers of this warpgroup's tiles
       const uint32_t s_col = b ? kColS1 : kColS0;
@@ -729,21 +735,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       }
       const int64_t tile_start = (t_begin + j) * TT;
       const int valid = a.n_tok - tile_start < TT ? int(a.n_tok - tile_start) : TT;
-      // pass 1: max of the raw scores (masked tokens excluded), 64 columns per wait
+      // Token counts are multiples of 32, so a tile holds n32 = valid / 32
+      // whole 32-column chunks of scores; columns past them are never read
+      // (and the PV MMAs stop at the same token).
+      const int n32 = valid >> 5;
+      // pass 1: max of the raw scores, two chunks per wait (an odd last chunk
+      // is loaded twice, which leaves the max unchanged)
       float pm = -__int_as_float(0x7f800000);
 #pragma unroll 1
-      for (int hh = 0; hh < 2; ++hh) {
+      for (int cc = 0; cc < n32; cc += 2) {
         uint32_t sv[32], sw[32];
-        tmem_ld32(lane_base + s_col + 64 * hh, sv);
-        tmem_ld32(lane_base + s_col + 64 * hh + 32, sw);
+        tmem_ld32(lane_base + s_col + 32 * cc, sv);
+        tmem_ld32(lane_base + s_col + 32 * (cc + 1 < n32 ? cc + 1 : cc), sw);
         tmem_ld_wait();
-        if (64 * hh + 64 > valid) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            if (64 * hh + i >= valid) sv[i] = 0xff800000u;
-            if (64 * hh + 32 + i >= valid) sw[i] = 0xff800000u;
-          }
-        }
         float m4[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) m4[i] = fmaxf(__uint_as_float(sv[i]), __uint_as_float(sw[i]));
@@ -775,12 +779,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       const uint64_t sc2 = f2pack(sc, sc), nm2 = f2pack(-r_j, -r_j);
       uint64_t l2[2] = {0ull, 0ull};  // two packed pairs of partial row sums
       uint32_t va[16], vb[16];
-      auto chunk = [&](uint32_t (&v)[16], int c) {
-        if (16 * c + 16 > valid) {
-#pragma unroll
-          for (int i = 0; i < 16; ++i)
-            if (16 * c + i >= valid) v[i] = 0xff800000u;  // -inf: masked token, weight 0
-        }
+      auto chunk = [&](const uint32_t (&v)[16], int c) {
         uint32_t pv[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -793,16 +792,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         }
         tmem_st8(lane_base + s_col + 8 * c, pv);
       };
+      const int n16 = 2 * n32;
       tmem_ld16(lane_base + s_col, va);
       tmem_ld_wait();
 #pragma unroll 1
-      for (int c = 0; c < 8; c += 2) {
+      for (int c = 0; c < n16; c += 2) {
         tmem_ld16(lane_base + s_col + 16 * (c + 1), vb);
         chunk(va, c);
         tmem_ld_wait();
-        if (c + 2 < 8) tmem_ld16(lane_base + s_col + 16 * (c + 2), va);
+        if (c + 2 < n16) tmem_ld16(lane_base + s_col + 16 * (c + 2), va);
         chunk(vb, c + 1);
-        if (c + 2 < 8) tmem_ld_wait();
+        if (c + 2 < n16) tmem_ld_wait();
       }
       {
         float a0, a1, b0, b1;
@@ -898,7 +898,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     // ------------------------------------------------------------ K producer
     const int c = (threadIdx.x - 256) & 127;   // channel
     const int qh = (threadIdx.x - 256) >> 7;    // chunks 2qh, 2qh+1 of each tile
-    const KOffsets ko(c, qh);
+    const KOffsets ko(c, qh, cv.GK, cv.kw, KB < 16 ? KB : 16);
+#pragma unroll 1
     for (int j = 0; j < nt; ++j) {
       const int b = j & 1, st = j % kStages;
       if (!mbar_wait(bar(KEMPTY + b), ((j >> 1) & 1) ^ 1, abort_flag, cv.status)) break;
@@ -912,7 +913,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     } else {
     // ------------------------------------------------------------ V producer
     const int t = threadIdx.x - 512;
-    const VOffsets vo(t);
+    const VOffsets vo(t, cv.vw, cv.vgroups, cv.GV, VB < 16 ? VB : 16);
+#pragma unroll 1
     for (int j = 0; j < nt; ++j) {
       const int b = j & 1, st = j % kStages;
       if (!mbar_wait(bar(VEMPTY + b), ((j >> 1) & 1) ^ 1, abort_flag, cv.status)) break;
@@ -929,20 +931,25 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     if (warp == kLoadWarp) {
     // ------------------------------------------------------------ loader
     // lanes prefetch the side-table group index of 32 tiles at a time; lane 0
-    // issues the bulk copies of each tile
+    // issues the bulk copies of each tile.  Token positions fit in 32 bits
+    // (capacity <= 2^30) and K groups are 32, 64 or 128 tokens, so the group
+    // arithmetic is 32-bit shifts.
+    const int gks = KB < 16 ? __ffs(cv.GK) - 1 : 0;
+    const int Lq = int(a.Lq), Lc = int(a.L), t0 = int(t_begin) * TT;
+    const int32_t* gs = cv.prot_gstart + size_t(u) * size_t(cv.nG + 1);
     int issued = 0;
     int pf0 = 0, pf1 = 0;  // this lane's prefetched gstart values (tile j0 + lane)
+#pragma unroll 1
     for (int j = 0; j < nt; ++j) {
       if constexpr (KB < 16) {
         if ((j & 31) == 0) {
           pf0 = pf1 = 0;
           const int jj = j + lane;
-          const int64_t ts = (t_begin + jj) * TT;
-          if (jj < nt && ts < a.Lq && cv.P > 0) {
-            const int64_t q_end = ts + TT < a.Lq ? ts + TT : a.Lq;
-            const int32_t* gs = cv.prot_gstart + size_t(u) * (cv.nG + 1);
-            pf0 = __ldg(gs + ts / cv.GK);
-            pf1 = __ldg(gs + q_end / cv.GK);
+          const int ts = t0 + jj * TT;
+          if (jj < nt && ts < Lq && cv.P > 0) {
+            const int q_end = ts + TT < Lq ? ts + TT : Lq;
+            pf0 = __ldg(gs + (ts >> gks));
+            pf1 = __ldg(gs + (q_end >> gks));
           }
         }
       }
@@ -954,52 +961,53 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         break;
       ++issued;
       if (lane == 0) {
-        const int64_t ts = (t_begin + j) * TT;
+        const int ts = t0 + j * TT;
         const uint32_t dst = sm_base + Smem::kRing + st * Smem::kStageBytes;
         uint32_t kc_b = 0, ksz_b = 0, vc_b = 0, vsz_b = 0, pos_b = 0, pk_b = 0;
-        int64_t g_lo = 0, pidx0 = 0;
+        int g_lo = 0, pidx0 = 0;  // pidx0: first staged position, relative to the unit
         const int n = g1 - g0;
-        if (KB < 16 && ts < a.Lq) {
-          g_lo = ts / cv.GK;
-          const int64_t q_end = ts + TT < a.Lq ? ts + TT : a.Lq;  // multiple of GK
-          const uint32_t ng = uint32_t(q_end / cv.GK - g_lo);
+        if (KB < 16 && ts < Lq) {
+          g_lo = ts >> gks;
+          const int q_end = ts + TT < Lq ? ts + TT : Lq;  // multiple of GK
+          const uint32_t ng = uint32_t((q_end >> gks) - g_lo);
           kc_b = ng * kHeadDim * uint32_t(cv.kw) * 4u;
           ksz_b = ng * kHeadDim * 4u;
           if (n > 0) {
             const int nst = n < kStagedProt ? n : kStagedProt;
-            const int64_t e0 = int64_t(u) * cv.P + g0;       // first entry, global index
-            pidx0 = e0 & ~int64_t(3);                        // 16-byte aligned superset
-            pos_b = uint32_t(((e0 + nst + 3) & ~int64_t(3)) - pidx0) * 4u;
+            // 16-byte aligned superset of the staged positions (the unit's
+            // slice starts at u * P entries)
+            const int64_t e0 = int64_t(u) * cv.P + g0;
+            const int64_t ea = e0 & ~int64_t(3);
+            pidx0 = int(ea - int64_t(u) * cv.P);
+            pos_b = uint32_t(((e0 + nst + 3) & ~int64_t(3)) - ea) * 4u;
             pk_b = uint32_t(nst) * kHeadDim * 2u;
           }
         }
-        if (VB < 16 && ts < a.L) {
-          const int64_t v_end = ts + TT < a.L ? ts + TT : a.L;
-          const uint32_t nv = uint32_t(v_end - ts);
+        if (VB < 16 && ts < Lc) {
+          const uint32_t nv = uint32_t((ts + TT < Lc ? ts + TT : Lc) - ts);
           vc_b = nv * uint32_t(cv.vw) * 4u;
           vsz_b = nv * uint32_t(cv.vgroups) * 4u;
         }
         int* hdr = reinterpret_cast<int*>(sm + Smem::kRing + st * Smem::kStageBytes + Smem::kRHdr);
         hdr[0] = kc_b ? n : 0;
         hdr[1] = g0;
-        hdr[2] = int(pidx0 - int64_t(u) * cv.P);
+        hdr[2] = pidx0;
         mbar_arrive_expect_tx(bar(RFULL + st), kc_b + ksz_b + vc_b + vsz_b + pos_b + pk_b);
+        const size_t ug = size_t(u) * size_t(cv.nG) + size_t(g_lo);
         if (kc_b) {
-          bulk_g2s(dst + Smem::kRKc, cv.k_codes + (size_t(u) * cv.nG + g_lo) * kHeadDim * cv.kw,
-                   kc_b, bar(RFULL + st));
-          bulk_g2s(dst + Smem::kRKsz, cv.k_sz + (size_t(u) * cv.nG + g_lo) * kHeadDim, ksz_b,
-                   bar(RFULL + st));
+          bulk_g2s(dst + Smem::kRKc, cv.k_codes + ug * kHeadDim * cv.kw, kc_b, bar(RFULL + st));
+          bulk_g2s(dst + Smem::kRKsz, cv.k_sz + ug * kHeadDim, ksz_b, bar(RFULL + st));
         }
         if (pos_b) {
-          bulk_g2s(dst + Smem::kRPos, cv.prot_pos + pidx0, pos_b, bar(RFULL + st));
-          bulk_g2s(dst + Smem::kRPk, cv.prot_k + (size_t(u) * cv.P + g0) * kHeadDim, pk_b,
+          const size_t e = size_t(u) * size_t(cv.P);
+          bulk_g2s(dst + Smem::kRPos, cv.prot_pos + e + size_t(pidx0), pos_b, bar(RFULL + st));
+          bulk_g2s(dst + Smem::kRPk, cv.prot_k + (e + size_t(g0)) * kHeadDim, pk_b,
                    bar(RFULL + st));
         }
         if (vc_b) {
-          bulk_g2s(dst + Smem::kRVc, cv.v_codes + (size_t(u) * cv.cap + ts) * cv.vw, vc_b,
-                   bar(RFULL + st));
-          bulk_g2s(dst + Smem::kRVsz, cv.v_sz + (size_t(u) * cv.cap + ts) * cv.vgroups, vsz_b,
-                   bar(RFULL + st));
+          const size_t ut = size_t(u) * size_t(cv.cap) + size_t(ts);
+          bulk_g2s(dst + Smem::kRVc, cv.v_codes + ut * cv.vw, vc_b, bar(RFULL + st));
+          bulk_g2s(dst + Smem::kRVsz, cv.v_sz + ut * cv.vgroups, vsz_b, bar(RFULL + st));
         }
       }
       __syncwarp();
@@ -1013,62 +1021,51 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     bool ok = mbar_wait(bar(QREADY), 0, abort_flag, cv.status);
     tc_fence_after();
     // QK(j) needs K_j (KFULL) and S_(j mod 2) free, i.e. PV(j-2) issued; PV(i)
-    // needs P_i (PFULL) and V_i (VFULL).  Whichever is ready is issued, PV
-    // first, so a late K tile never holds back a ready PV.  Barrier phases
-    // cannot run ahead: each next phase needs an MMA issued here first.
+    // needs P_i (PFULL) and V_i (VFULL).  Every QK that is ready and allowed
+    // is issued at once; otherwise the lane sleeps (suspending mbarrier wait)
+    // on the barrier it needs next: P of the oldest un-issued PV, or K of the
+    // next QK when no PV is pending.  Barrier phases cannot run ahead: each
+    // next phase needs an MMA issued here first.
     int nq = 0, np = 0;
-    uint64_t t0 = 0;
-    uint32_t idle = 0;
+    auto issue_qk = [&]() {
+      tc_fence_after();
+      const int b = nq & 1;
+      const uint32_t kbase = sm_base + (b ? Smem::kK1 : Smem::kK0);
+      const uint32_t s_col = b ? kColS1 : kColS0;
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_ts(tmem + s_col, tmem + kColQ + 8 * kk, sdesc_sw128(kbase + 4096 * kk, 1024, 2048),
+               kk > 0 ? 1u : 0u);
+      mma_commit(bar(KEMPTY + b));
+      mma_commit(bar(SFULL + b));
+      ++nq;
+    };
+#pragma unroll 1
     while (ok && np < nt) {
-      bool progress = false;
-      if (np < nq && mbar_test(bar(PFULL + (np & 1)), (np >> 1) & 1) &&
-          mbar_test(bar(VFULL + (np & 1)), (np >> 1) & 1)) {
-        tc_fence_after();
-        const int bb = np & 1;
-        const uint32_t vbase = sm_base + (bb ? Smem::kV1 : Smem::kV0);
-        const uint32_t p_col = bb ? kColS1 : kColS0;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)  // tokens 16kk..16kk+15: packed P columns 8kk..8kk+7
-          mma_ts(tmem + kColO, tmem + p_col + 8 * kk, sdesc_sw128(vbase + 4096 * kk, 1024, 2048),
-                 (np > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(bar(VEMPTY + bb));
-        ++np;
-        progress = true;
+      while (nq < nt && nq <= np + 1 && mbar_test(bar(KFULL + (nq & 1)), (nq >> 1) & 1)) issue_qk();
+      if (np == nq) {
+        // nothing to multiply by P yet: wait for the next K tile
+        ok = mbar_wait(bar(KFULL + (nq & 1)), (nq >> 1) & 1, abort_flag, cv.status);
+        if (ok) issue_qk();
+        continue;
       }
-      if (nq < nt && nq <= np + 1 && mbar_test(bar(KFULL + (nq & 1)), (nq >> 1) & 1)) {
-        tc_fence_after();
-        const int b = nq & 1;
-        const uint32_t kbase = sm_base + (b ? Smem::kK1 : Smem::kK0);
-        const uint32_t s_col = b ? kColS1 : kColS0;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + s_col, tmem + kColQ + 8 * kk, sdesc_sw128(kbase + 4096 * kk, 1024, 2048),
-                 kk > 0 ? 1u : 0u);
-        mma_commit(bar(KEMPTY + b));
-        mma_commit(bar(SFULL + b));
-        ++nq;
-        progress = true;
+      const int bb = np & 1;
+      if (!mbar_wait(bar(PFULL + bb), (np >> 1) & 1, abort_flag, cv.status) ||
+          !mbar_wait(bar(VFULL + bb), (np >> 1) & 1, abort_flag, cv.status)) {
+        ok = false;
+        break;
       }
-      if (progress) {
-        t0 = 0;
-        idle = 0;
-      } else if ((++idle & 15u) == 0) {
-        // bounded: give up on another thread's abort or after kTimeoutNs
-        if (*abort_flag) {
-          ok = false;
-        } else {
-          const uint64_t now = globaltimer();
-          if (t0 == 0) {
-            t0 = now;
-          } else if (now - t0 > kTimeoutNs) {
-            *abort_flag = 1;
-            atomicOr(cv.status, uint32_t(DKV_FLAG_TIMEOUT));
-            ok = false;
-          }
-        }
-      } else {
-        __nanosleep(32);
-      }
+      tc_fence_after();
+      const uint32_t vbase = sm_base + (bb ? Smem::kV1 : Smem::kV0);
+      const uint32_t p_col = bb ? kColS1 : kColS0;
+      const int64_t pv_start = (t_begin + np) * TT;
+      const int nk = a.n_tok - pv_start < TT ? int(a.n_tok - pv_start) >> 4 : TT / 16;
+#pragma unroll 1
+      for (int kk = 0; kk < nk; ++kk)  // tokens 16kk..16kk+15: packed P columns 8kk..8kk+7
+        mma_ts(tmem + kColO, tmem + p_col + 8 * kk, sdesc_sw128(vbase + 4096 * kk, 1024, 2048),
+               (np > 0 || kk > 0) ? 1u : 0u);
+      mma_commit(bar(VEMPTY + bb));
+      ++np;
     }
     // drain: every MMA issued above completes before TMEM is released
     mma_commit(bar(DONE));
