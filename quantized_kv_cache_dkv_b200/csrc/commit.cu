@@ -35,6 +35,7 @@ __device__ __forceinline__ float sanitize(float x) {
 
 struct GroupQuant {
   float s32, z32;  // stored fp16 scale / zero, widened
+  float rs;        // correctly rounded 1 / s32 (0 when s32 == 0)
   __half2 sz;      // (scale, zero)
 };
 
@@ -46,14 +47,23 @@ __device__ __forceinline__ GroupQuant make_quant(float mn, float mx, int levels)
   GroupQuant q;
   q.s32 = __half2float(s);
   q.z32 = __half2float(z);
+  q.rs = q.s32 > 0.f ? __frcp_rn(q.s32) : 0.f;
   q.sz = __halves2half2(s, z);
   return q;
 }
 
-// q = clamp(rint((x - z) / s), 0, levels); 0 when s == 0
+// q = clamp(rint((x - z) / s), 0, levels) with (x - z) / s the correctly
+// rounded fp32 quotient; 0 when s == 0.  The quotient is estimated as
+// (x - z) * fl(1/s), within a few ulp of it.  Inside the clamp range
+// (|quotient| <= levels + 1 <= 16) those few ulp are below 2^-17, so the
+// estimate rounds to the same integer unless it lies within 2^-12 of a tie
+// (k + 1/2); only then is the exact division taken.  Outside the range both
+// clamp alike.  The code is therefore the division-based one, bit for bit.
 __device__ __forceinline__ uint32_t code_of(float x, const GroupQuant& q, int levels) {
   if (!(q.s32 > 0.f)) return 0u;
-  const float t = __fdiv_rn(__fsub_rn(x, q.z32), q.s32);
+  const float num = __fsub_rn(x, q.z32);
+  float t = __fmul_rn(num, q.rs);
+  if (fabsf(fabsf(__fsub_rn(t, rintf(t))) - 0.5f) < 2.44140625e-4f) t = __fdiv_rn(num, q.s32);
   int c = __float2int_rn(t);
   c = c < 0 ? 0 : (c > levels ? levels : c);
   return uint32_t(c);

@@ -31,6 +31,7 @@ _TAG_KV_BLOCK = 3
 _TAG_PROT_PREFILL = 4
 _TAG_PROT_LATE = 5
 _TAG_ACTIVE = 6
+_TAG_GRID = 7
 
 
 @dataclass(frozen=True)
@@ -224,6 +225,28 @@ def block_inputs(w: Workload, block: int, units=None):
         K[b, h], V[b, h] = kv_block_bits(w, b, h, block)
         M[b, h] = block_protect_words(w, b, h, block)
     return K, V, M
+
+
+def grid_block_bits(w: Workload, block: int, levels: int):
+    """K, V bf16 bits [B, Hkv, blk, d] on a grid of multiples of 1/64 in
+    [0, levels], each (token, 32-channel) row of V and each (channel, 32-token)
+    column of K holding both ends 0 and levels.  With group min 0 and max
+    `levels` the scale is 1 or close to it, so many (x - z) / s quotients land
+    exactly on or next to a rounding tie k + 1/2.  Seeded like the others."""
+    r = _rng(w.seed, _TAG_GRID, block, levels)
+    shape = (w.B, w.Hkv, w.blk, w.d)
+    x = r.integers(0, 64 * levels + 1, size=(2,) + shape).astype(np.float32) / np.float32(64)
+    K, V = x[0], x[1]
+    V[..., 0::32] = 0.0
+    V[..., 1::32] = float(levels)
+    K[..., 0, :] = 0.0
+    K[..., 1, :] = float(levels)
+    # every other token row of V and channel of K slightly stretched, so that
+    # its scale is not exactly 1 and quotients fall next to the ties
+    f = np.array([1.0, 1.0 - 1.0 / 256, 1.0 + 1.0 / 256, 1.0 - 3.0 / 512], np.float32)
+    V[:, :, 1::2, :] *= f[r.integers(0, 4, size=V[:, :, 1::2, :1].shape)]
+    K[..., 1::2] *= f[r.integers(0, 4, size=K[..., :1, 1::2].shape)]
+    return f32_to_bf16_bits(K), f32_to_bf16_bits(V)
 
 
 def queries_bits(w: Workload, step: int) -> np.ndarray:

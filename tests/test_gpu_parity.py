@@ -180,6 +180,24 @@ def test_all_protected_group_and_side_table_overflow(dkv):
     assert_close(host_bits(out), oc.block_attention(Q, Ka, Va, w.softmax_scale))
 
 
+@pytest.mark.parametrize("bits,group", [(2, 32), (4, 32), (2, 64), (4, 64)])
+def test_commit_codes_at_rounding_ties(dkv, bits, group):
+    """Grid inputs put many (x - z) / s quotients exactly on k + 1/2 or within
+    an ulp of it: the codes must still be those of the correctly rounded
+    division with round-half-even."""
+    w = SHRUNK["tiny"].with_(k_bits=bits, v_bits=bits, k_group=group, v_group=group,
+                             prot_frac=0.0)
+    levels = (1 << bits) - 1
+    cap = 256
+    cache = dkv.dkv_cache_alloc(gpu_config(dkv, w, cap, 8))
+    oc = oracle_cache(w, cap, 8)
+    for i in range(6):
+        K, V = synth.grid_block_bits(w, i, levels)
+        dkv.dkv_commit_block(cache, dev_bf16(K), dev_bf16(V), None)
+        oc.commit(K, V, None)
+    compare_exports(dkv.dkv_cache_export(cache), oc.snapshot())
+
+
 def test_range_flag_and_clamp(dkv):
     w = SHRUNK["tiny"]
     cache = dkv.dkv_cache_alloc(gpu_config(dkv, w, 128, 8))
