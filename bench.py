@@ -275,16 +275,14 @@ def run_gpu(w: synth.Workload, K: int, W: int, want_e2e=True, log=print, kernel=
         dkv.dkv_block_attention(caches[r], q, ka, va, w.softmax_scale, outs[k % S])
         launches[0] += 1 + dkv.dkv_last_attention_plan(caches[r])[2]
         pos[r] += 1
-        if pos[r] == C:  # back to the starting length
+        if pos[r] == C:  # back to the starting length (recorded; the next commit applies it)
             dkv.dkv_cache_truncate(caches[r], w.L)
-            launches[0] += 1 if w.k_bits < 16 else 0
             pos[r] = 0
 
     def finish():
         for r in range(R):
             if pos[r]:
                 dkv.dkv_cache_truncate(caches[r], w.L)
-                launches[0] += 1 if w.k_bits < 16 else 0
                 pos[r] = 0
 
     # warm-up (eager), then capture exactly K steps in one CUDA graph

@@ -117,8 +117,11 @@ int dkv_block_attention(dkv_cache* cache, const void* q, const void* k_act,
  * reuse a shared prefix, the prefix-cache reuse of the Tai et al. abstract).
  * new_len must be a multiple of `block` and, when k_bits < 16, of k_group, so
  * that no incomplete K group remains; 0 <= new_len <= len.  The side table
- * keeps the entries of the surviving groups.  Stream-ordered; len changes
- * at once on the host. */
+ * keeps the entries of the surviving groups.  len changes at once on the
+ * host.  No kernel runs here: the device-side count of side-table entries
+ * and the tail mask are reset by the next dkv_commit_block, or by
+ * dkv_cache_export if that comes first (on its stream), which is all that
+ * reads them; dkv_block_attention reads neither.  `stream` is unused. */
 int dkv_cache_truncate(dkv_cache* cache, int64_t new_len, void* stream);
 
 /* dkv_block_attention for callers that cannot call cudaMalloc -- code that

@@ -59,11 +59,13 @@ __device__ __forceinline__ GroupQuant make_quant(float mn, float mx, int levels)
 // estimate rounds to the same integer unless it lies within 2^-12 of a tie
 // (k + 1/2); only then is the exact division taken.  Outside the range both
 // clamp alike.  The code is therefore the division-based one, bit for bit.
+__device__ __noinline__ float exact_quotient(float num, float s) { return __fdiv_rn(num, s); }
+
 __device__ __forceinline__ uint32_t code_of(float x, const GroupQuant& q, int levels) {
   if (!(q.s32 > 0.f)) return 0u;
   const float num = __fsub_rn(x, q.z32);
   float t = __fmul_rn(num, q.rs);
-  if (fabsf(fabsf(__fsub_rn(t, rintf(t))) - 0.5f) < 2.44140625e-4f) t = __fdiv_rn(num, q.s32);
+  if (fabsf(fabsf(__fsub_rn(t, rintf(t))) - 0.5f) < 2.44140625e-4f) t = exact_quotient(num, q.s32);
   int c = __float2int_rn(t);
   c = c < 0 ? 0 : (c > levels ? levels : c);
   return uint32_t(c);
@@ -93,19 +95,16 @@ __device__ __forceinline__ void stage_rows(uint16_t* dst, const uint16_t* src, i
 __device__ __forceinline__ float bf16_at(const uint16_t* p) { return bf16_bits_to_f32(*p); }
 
 // One V group: G consecutive channels of one token (x: shared memory, 16-byte
-// aligned).  Fully unrolled so the loads and the divisions are independent.
-template <int VB, int G>
-__device__ __forceinline__ void quant_v_group(const uint16_t* x, uint32_t* codes, __half2* sz,
-                                              bool& range) {
+// aligned).  Rolled loops over 8-channel chunks and code words keep the code
+// small (each warp runs it once, so its instructions come from the cache).
+template <int VB>
+__device__ __forceinline__ void quant_v_group(const uint16_t* x, int G, uint32_t* codes,
+                                              __half2* sz, bool& range) {
   constexpr int levels = (1 << VB) - 1;
   constexpr int per = 32 / VB;
-  float mn4[4], mx4[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    mn4[i] = __int_as_float(0x7f800000);
-    mx4[i] = -__int_as_float(0x7f800000);
-  }
-#pragma unroll
+  float mn2[2] = {__int_as_float(0x7f800000), __int_as_float(0x7f800000)};
+  float mx2[2] = {-__int_as_float(0x7f800000), -__int_as_float(0x7f800000)};
+#pragma unroll 1
   for (int i8 = 0; i8 < G; i8 += 8) {
     const uint4 q8 = *reinterpret_cast<const uint4*>(x + i8);
     const uint32_t w[4] = {q8.x, q8.y, q8.z, q8.w};
@@ -114,14 +113,12 @@ __device__ __forceinline__ void quant_v_group(const uint16_t* x, uint32_t* codes
       float f = bf16_bits_to_f32(uint16_t(w[j >> 1] >> (16 * (j & 1))));
       range |= out_of_range(f);
       f = sanitize(f);
-      mn4[j & 3] = fminf(mn4[j & 3], f);
-      mx4[j & 3] = fmaxf(mx4[j & 3], f);
+      mn2[j & 1] = fminf(mn2[j & 1], f);
+      mx2[j & 1] = fmaxf(mx2[j & 1], f);
     }
   }
-  const float mn = fminf(fminf(mn4[0], mn4[1]), fminf(mn4[2], mn4[3]));
-  const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-  const GroupQuant q = make_quant(mn, mx, levels);
-#pragma unroll
+  const GroupQuant q = make_quant(fminf(mn2[0], mn2[1]), fmaxf(mx2[0], mx2[1]), levels);
+#pragma unroll 1
   for (int w = 0; w < G / per; ++w) {
     uint32_t word = 0;
 #pragma unroll
@@ -133,41 +130,44 @@ __device__ __forceinline__ void quant_v_group(const uint16_t* x, uint32_t* codes
 }
 
 // One K group of channel ch: G tokens of the pending stream (rows of sk),
-// protected tokens (bits of gm) left out of min/max and given code 0.
-template <int KB, int G>
-__device__ __forceinline__ GroupQuant quant_k_group(const uint16_t* sk, int row0, int ch,
-                                                    const uint32_t (&gm)[4], bool check_from,
-                                                    int check_row, uint32_t* codes, bool& range) {
+// protected tokens (bits of gm) left out of min/max and given code 0.  Rolled
+// loops as above.
+template <int KB>
+__device__ __forceinline__ GroupQuant quant_k_group(const uint16_t* sk, int G, int row0, int ch,
+                                                    const uint32_t (&gm)[4], int check_row,
+                                                    uint32_t* codes, bool& range) {
   constexpr int levels = (1 << KB) - 1;
   constexpr int per = 32 / KB;
-  float mn4[4], mx4[4];
+  float mn2[2] = {__int_as_float(0x7f800000), __int_as_float(0x7f800000)};
+  float mx2[2] = {-__int_as_float(0x7f800000), -__int_as_float(0x7f800000)};
+#pragma unroll 1
+  for (int t8 = 0; t8 < G; t8 += 8) {
+    const uint32_t m8 = (gm[t8 >> 5] >> (t8 & 31)) & 0xFFu;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    mn4[i] = __int_as_float(0x7f800000);
-    mx4[i] = -__int_as_float(0x7f800000);
-  }
-#pragma unroll
-  for (int t = 0; t < G; ++t) {
-    float f = bf16_at(sk + (row0 + t) * kRowPad + ch);
-    if (check_from && row0 + t >= check_row) range |= out_of_range(f);
-    f = sanitize(f);
-    if (!((gm[t >> 5] >> (t & 31)) & 1u)) {
-      mn4[t & 3] = fminf(mn4[t & 3], f);
-      mx4[t & 3] = fmaxf(mx4[t & 3], f);
+    for (int i = 0; i < 8; ++i) {
+      const int t = t8 + i;
+      float f = bf16_at(sk + (row0 + t) * kRowPad + ch);
+      if (row0 + t >= check_row) range |= out_of_range(f);
+      f = sanitize(f);
+      if (!((m8 >> i) & 1u)) {
+        mn2[i & 1] = fminf(mn2[i & 1], f);
+        mx2[i & 1] = fmaxf(mx2[i & 1], f);
+      }
     }
   }
-  float mn = fminf(fminf(mn4[0], mn4[1]), fminf(mn4[2], mn4[3]));
-  float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+  float mn = fminf(mn2[0], mn2[1]);
+  float mx = fmaxf(mx2[0], mx2[1]);
   if (mn > mx) mn = mx = 0.f;  // every token protected
   const GroupQuant q = make_quant(mn, mx, levels);
-#pragma unroll
+#pragma unroll 1
   for (int w = 0; w < G / per; ++w) {
+    const uint32_t mw = (gm[(w * per) >> 5] >> ((w * per) & 31));  // per <= 16 bits of mask
     uint32_t word = 0;
 #pragma unroll
     for (int e = 0; e < per; ++e) {
-      const int t = w * per + e;
-      const uint32_t cq = code_of(sanitize(bf16_at(sk + (row0 + t) * kRowPad + ch)), q, levels);
-      if (!((gm[t >> 5] >> (t & 31)) & 1u)) word |= cq << (e * KB);  // protected slot: code 0
+      const uint32_t cq =
+          code_of(sanitize(bf16_at(sk + (row0 + w * per + e) * kRowPad + ch)), q, levels);
+      if (!((mw >> e) & 1u)) word |= cq << (e * KB);  // protected slot: code 0
     }
     codes[w] = word;
   }
@@ -180,7 +180,7 @@ __device__ __forceinline__ GroupQuant quant_k_group(const uint16_t* sk, int row0
 template <int KB, int VB>
 __global__ void __launch_bounds__(kThreads)
 commit_kernel(CacheView c, const uint16_t* __restrict__ k, const uint16_t* __restrict__ v,
-              const uint32_t* __restrict__ pw, int64_t p0) {
+              const uint32_t* __restrict__ pw, int64_t p0, int truncated) {
   extern __shared__ __align__(16) uint16_t sbuf[];
   const int u = blockIdx.x;
   const int tid = threadIdx.x;
@@ -195,6 +195,14 @@ commit_kernel(CacheView c, const uint16_t* __restrict__ k, const uint16_t* __res
   const int GK = c.GK;
   const int n_tail = KB < 16 ? int(p0 % GK) : 0;
   const bool completes = KB < 16 && n_tail + blk >= GK;
+
+  // a roll-back to p0 (a multiple of the K group) recorded since the last
+  // commit: the side table keeps the entries of the groups before p0, the
+  // tail is empty; applied here, before any thread reads either
+  if (KB < 16 && truncated) {
+    if (tid == 0) c.prot_count[u] = c.prot_gstart[size_t(u) * size_t(c.nG + 1) + size_t(p0 / GK)];
+    if (tid < c.twords) c.tail_mask[size_t(u) * c.twords + tid] = 0u;
+  }
 
   // ------------------------------------------------------------------ stage
   if constexpr (VB < 16) stage_rows(sv, vu, blk, tid);
@@ -221,9 +229,7 @@ commit_kernel(CacheView c, const uint16_t* __restrict__ k, const uint16_t* __res
       const uint16_t* x = sv + t * kRowPad + gi * GV;
       uint32_t* codes = c.v_codes + (size_t(u) * c.cap + p0 + t) * c.vw + gi * GV * VB / 32;
       __half2* sz = c.v_sz + (size_t(u) * c.cap + p0 + t) * ngr + gi;
-      if (GV == 32) quant_v_group<VB, 32>(x, codes, sz, range);
-      else if (GV == 64) quant_v_group<VB, 64>(x, codes, sz, range);
-      else quant_v_group<VB, 128>(x, codes, sz, range);
+      quant_v_group<VB>(x, GV, codes, sz, range);
     }
   }
 
@@ -292,10 +298,7 @@ commit_kernel(CacheView c, const uint16_t* __restrict__ k, const uint16_t* __res
           if (tid == 0) atomicOr(c.status, uint32_t(DKV_FLAG_CAPACITY));
         }
         uint32_t* codes = c.k_codes + ((size_t(u) * c.nG + j) * d + ch) * c.kw;
-        GroupQuant q;
-        if (GK == 32) q = quant_k_group<KB, 32>(sk, gi * GK, ch, gm, true, n_tail, codes, range);
-        else if (GK == 64) q = quant_k_group<KB, 64>(sk, gi * GK, ch, gm, true, n_tail, codes, range);
-        else q = quant_k_group<KB, 128>(sk, gi * GK, ch, gm, true, n_tail, codes, range);
+        const GroupQuant q = quant_k_group<KB>(sk, GK, gi * GK, ch, gm, n_tail, codes, range);
         c.k_sz[(size_t(u) * c.nG + j) * d + ch] = q.sz;
         // side-table entries, ascending positions
 #pragma unroll
@@ -330,7 +333,7 @@ __global__ void truncate_kernel(CacheView c, int64_t new_len) {
 
 template <int KB, int VB>
 cudaError_t launch_kv(const CacheView& c, const uint16_t* k, const uint16_t* v,
-                      const uint32_t* pw, int64_t p0, cudaStream_t s) {
+                      const uint32_t* pw, int64_t p0, bool truncated, cudaStream_t s) {
   const int krows = KB < 16 ? (c.GK > c.blk ? c.GK : c.blk) : 0;
   const int vrows = VB < 16 ? c.blk : 0;
   const size_t smem = size_t(krows + vrows) * kRowPad * 2;
@@ -339,17 +342,17 @@ cudaError_t launch_kv(const CacheView& c, const uint16_t* k, const uint16_t* v,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     if (e != cudaSuccess) return e;
   }
-  commit_kernel<KB, VB><<<c.U, kThreads, smem, s>>>(c, k, v, pw, p0);
+  commit_kernel<KB, VB><<<c.U, kThreads, smem, s>>>(c, k, v, pw, p0, truncated ? 1 : 0);
   return cudaGetLastError();
 }
 
 template <int KB>
 cudaError_t launch_k(const CacheView& c, const uint16_t* k, const uint16_t* v,
-                     const uint32_t* pw, int64_t p0, cudaStream_t s) {
+                     const uint32_t* pw, int64_t p0, bool truncated, cudaStream_t s) {
   switch (c.vb) {
-    case 2: return launch_kv<KB, 2>(c, k, v, pw, p0, s);
-    case 4: return launch_kv<KB, 4>(c, k, v, pw, p0, s);
-    default: return launch_kv<KB, 16>(c, k, v, pw, p0, s);
+    case 2: return launch_kv<KB, 2>(c, k, v, pw, p0, truncated, s);
+    case 4: return launch_kv<KB, 4>(c, k, v, pw, p0, truncated, s);
+    default: return launch_kv<KB, 16>(c, k, v, pw, p0, truncated, s);
   }
 }
 
@@ -361,11 +364,11 @@ cudaError_t launch_truncate(const CacheView& c, int64_t new_len, cudaStream_t s)
 }
 
 cudaError_t launch_commit(const CacheView& c, const uint16_t* k, const uint16_t* v,
-                          const uint32_t* pw, int64_t p0, cudaStream_t s) {
+                          const uint32_t* pw, int64_t p0, bool truncated, cudaStream_t s) {
   switch (c.kb) {
-    case 2: return launch_k<2>(c, k, v, pw, p0, s);
-    case 4: return launch_k<4>(c, k, v, pw, p0, s);
-    default: return launch_k<16>(c, k, v, pw, p0, s);
+    case 2: return launch_k<2>(c, k, v, pw, p0, truncated, s);
+    case 4: return launch_k<4>(c, k, v, pw, p0, truncated, s);
+    default: return launch_k<16>(c, k, v, pw, p0, truncated, s);
   }
 }
 

@@ -28,6 +28,7 @@ struct dkv_cache {
   size_t arena_bytes = 0;
   float* part_o = nullptr;
   float2* part_ml = nullptr;
+  bool trunc_pending = false;  // a dkv_cache_truncate not yet applied on the device
   int32_t max_splits = 1;
   int32_t opt_splits = 0;
   int32_t opt_kernel = 0;
@@ -322,13 +323,25 @@ int dkv_cache_truncate(dkv_cache* c, int64_t new_len, void* stream) {
     return fail(DKV_ERR_INVALID_ARG, "new_len must be a multiple of block within [0, len]");
   if (c->v.kb < 16) {
     if (new_len % c->v.GK) return fail(DKV_ERR_INVALID_ARG, "new_len must be a multiple of k_group");
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = timed_launch(c, DKV_KERNEL_TRUNCATE, s,
-                                 [&] { return dkv::launch_truncate(c->v, new_len, s); });
-    if (e != cudaSuccess)
-      return fail(DKV_ERR_CUDA, std::string("truncate launch: ") + cudaGetErrorString(e));
+    // The device side (side-table count, tail mask) is read only by the next
+    // commit and by export, so the roll-back is recorded here and applied by
+    // whichever of them comes first: no launch of its own.
+    c->trunc_pending = true;
   }
+  (void)stream;
   c->len = new_len;
+  return DKV_OK;
+}
+
+// Applies a recorded roll-back to the device state (export without an
+// intervening commit).
+static int apply_pending_truncate(dkv_cache* c, cudaStream_t s) {
+  if (!c->trunc_pending) return DKV_OK;
+  cudaError_t e = timed_launch(c, DKV_KERNEL_TRUNCATE, s,
+                               [&] { return dkv::launch_truncate(c->v, c->len, s); });
+  if (e != cudaSuccess)
+    return fail(DKV_ERR_CUDA, std::string("truncate launch: ") + cudaGetErrorString(e));
+  c->trunc_pending = false;
   return DKV_OK;
 }
 
@@ -344,9 +357,11 @@ int dkv_commit_block(dkv_cache* c, const void* k, const void* v, const uint32_t*
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = timed_launch(c, DKV_KERNEL_COMMIT, s, [&] {
     return dkv::launch_commit(c->v, static_cast<const uint16_t*>(k),
-                              static_cast<const uint16_t*>(v), protect_words, c->len, s);
+                              static_cast<const uint16_t*>(v), protect_words, c->len,
+                              c->trunc_pending, s);
   });
   if (e != cudaSuccess) return fail(DKV_ERR_CUDA, std::string("commit launch: ") + cudaGetErrorString(e));
+  c->trunc_pending = false;
   c->len += c->v.blk;
   return DKV_OK;
 }
@@ -407,6 +422,8 @@ int dkv_cache_export(dkv_cache* c, void* stream, dkv_export* o) {
   g_err.clear();
   if (!c || !o) return fail(DKV_ERR_INVALID_ARG, "NULL argument");
   const dkv::CacheView& v = c->v;
+  const int trc = apply_pending_truncate(c, static_cast<cudaStream_t>(stream));
+  if (trc != DKV_OK) return trc;
   DKV_CUDA(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
   const int64_t L = c->len;
   const int64_t Lq = v.kb < 16 ? (L / v.GK) * v.GK : L;

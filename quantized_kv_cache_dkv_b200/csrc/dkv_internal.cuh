@@ -59,7 +59,7 @@ struct AttnArgs {
 };
 
 cudaError_t launch_commit(const CacheView& c, const uint16_t* k, const uint16_t* v,
-                          const uint32_t* protect_words, int64_t p0, cudaStream_t s);
+                          const uint32_t* pw, int64_t p0, bool truncated, cudaStream_t s);
 cudaError_t launch_truncate(const CacheView& c, int64_t new_len, cudaStream_t s);
 
 // mma.sync kernel: token tile of 64.

@@ -247,6 +247,31 @@ def test_truncate_then_recommit(dkv, gk):
         dkv.dkv_cache_truncate(cache, 32 if gk == 64 else 33)
 
 
+@pytest.mark.parametrize("gk", [32, 64])
+def test_truncate_recorded_then_attention_export_commit(dkv, gk):
+    """Truncation only records the new length: attention right after it, two
+    truncations in a row, export applying it, and a later commit must all
+    agree with the oracle."""
+    torch = _torch()
+    w = SHRUNK["batch32"].with_(k_group=gk, prot_frac=0.1)
+    cap = default_cap(w, 12)
+    P = 64
+    cache = dkv.dkv_cache_alloc(gpu_config(dkv, w, cap, P))
+    oc = oracle_cache(w, cap, P)
+    commit_both(dkv, cache, oc, w, range(7))
+    for n in (192, 128):
+        dkv.dkv_cache_truncate(cache, n)
+        oc.truncate(n)
+    Q = synth.queries_bits(w, 1)
+    Ka, Va = synth.active_block_bits(w, 1)
+    out = torch.empty((w.B, w.Hq, w.blk, w.d), dtype=torch.bfloat16, device="cuda")
+    dkv.dkv_block_attention(cache, dev_bf16(Q), dev_bf16(Ka), dev_bf16(Va), w.softmax_scale, out)
+    assert_close(host_bits(out), oc.block_attention(Q, Ka, Va, w.softmax_scale))
+    compare_exports(dkv.dkv_cache_export(cache), oc.snapshot())
+    commit_both(dkv, cache, oc, w, (8, 9, 10))
+    compare_exports(dkv.dkv_cache_export(cache), oc.snapshot())
+
+
 def test_null_protect_mask_means_none(dkv):
     w = SHRUNK["batch32"]
     cap = default_cap(w, 4)
