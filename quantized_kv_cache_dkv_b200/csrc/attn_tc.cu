@@ -240,9 +240,9 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t addr, uint32_t lbo, uin
 }
 
 // Register budgets per warpgroup after setmaxnreg (launch: 72 per thread x
-// 896 threads = 64512): softmax rises to 88 (2 x 128 threads), producers keep
-// 72 (512 threads), control drops to 40 (128 threads): 22528 + 36864 + 5120.
-constexpr int kRegSoftmax = 88, kRegControl = 40;
+// 896 threads = 64512): softmax rises to 96 (2 x 128 threads), producers drop
+// to 64 (512 threads), control to 56 (128 threads): 24576 + 32768 + 7168.
+constexpr int kRegSoftmax = 96, kRegProducer = 64, kRegControl = 56;
 
 template <int N>
 __device__ __forceinline__ void regs_inc() {
@@ -328,6 +328,19 @@ __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
 // bf16 tail, the active block and bits = 16 come straight from global memory.
 // Byte offsets of the 16-byte chunks a K producer thread (c, qh) stores:
 // chunk i (0..7) holds tokens 64 qh + 8 i .. +7 of channel c.
+// Tiles whose K is wholly quantized are stored in the order the prmt-free
+// dequantization produces: the token at tile position kpos(t) is t, permuted
+// within groups of 16 (2-bit codes) or 8 (4-bit codes).  The V tile of such a
+// tile puts token t's row at the same position, so P V pairs every score with
+// its own value row; the softmax does not depend on column order.  Other
+// tiles (K tail, active block, bf16 K) keep the natural order.
+template <int KB>
+__device__ __forceinline__ int kpos(int t) {
+  if constexpr (KB == 2) return (t & ~15) | (8 * ((t >> 2) & 1) + 2 * (t & 3) + ((t >> 3) & 1));
+  else if constexpr (KB == 4) return (t & ~7) | (2 * (t & 3) + ((t >> 2) & 1));
+  else return t;
+}
+
 struct KOffsets {
   uint32_t o[8];
   uint32_t w[2], z[2];  // ring offsets of chunk 2qh+qi: code words (uint32), (scale, zero) pairs
@@ -371,15 +384,15 @@ __device__ __forceinline__ void fill_k_tile(const AttnArgs& a, int u, int64_t ti
         const __half2 sz = reinterpret_cast<const __half2*>(rs + Smem::kRKsz)[qi ? ko.z[1] : ko.z[0]];
         const __half2 s2 = __half2half2(__low2half(sz));
         const __half2 z2 = __half2half2(__high2half(sz));
-        uint4 out[4];
+        uint4 out[4];  // tokens in kpos order
         if constexpr (KB == 4) {
-          out[0] = dequant4x8(w.x, s2, z2);
-          out[1] = dequant4x8(w.y, s2, z2);
-          out[2] = dequant4x8(w.z, s2, z2);
-          out[3] = dequant4x8(w.w, s2, z2);
+          out[0] = dequant4x8_raw(w.x, s2, z2);
+          out[1] = dequant4x8_raw(w.y, s2, z2);
+          out[2] = dequant4x8_raw(w.z, s2, z2);
+          out[3] = dequant4x8_raw(w.w, s2, z2);
         } else {
-          dequant2x16(w.x, s2, z2, out[0], out[1]);
-          dequant2x16(w.y, s2, z2, out[2], out[3]);
+          dequant2x16_raw(w.x, s2, z2, out[0], out[1]);
+          dequant2x16_raw(w.y, s2, z2, out[2], out[3]);
         }
         // chunk 1's offsets are chunk 0's shifted by +-64 bytes (bit 2 of the swizzle)
         uint8_t* dst = kt + (qi ? int(ko.o[4]) - int(ko.o[0]) : 0);
@@ -400,7 +413,8 @@ __device__ __forceinline__ void fill_k_tile(const AttnArgs& a, int u, int64_t ti
         const uint16_t kv = i < kStagedProt
                                 ? rpk[i * d + c]
                                 : __ldg(cv.prot_k + (size_t(u) * cv.P + g0 + i) * d + c);
-        __half* dst = reinterpret_cast<__half*>(kt + kt_off(c, t & ~7)) + (t & 7);
+        const int p = kpos<KB>(t);
+        __half* dst = reinterpret_cast<__half*>(kt + kt_off(c, p & ~7)) + (p & 7);
         *dst = bf16_to_half(kv);
       }
       return;
@@ -496,12 +510,15 @@ __device__ __noinline__ void fill_k_general(const AttnArgs& a, int u, int64_t ti
 // 512 contiguous bytes of the ring stage ([token][vw words]).
 // Byte offsets of the 16-byte chunks a V producer thread stores: item r
 // (token (tid >> 2) + 64 r, quarter tid & 3), store i = chunk (i + rot) & 3.
+template <int KB>
 struct VOffsets {
   uint32_t base, x[4];
   uint32_t w[2], z[2];  // ring offsets of item r: code words (uint32), (scale, zero) pairs
   __device__ VOffsets(int tid, int vw, int vgroups, int GV, int vb) {
-    const int qq = tid & 3, t7 = (tid >> 2) & 7, rot = qq & 2;
-    base = uint32_t(((tid >> 5) * 2 + (qq >> 1)) * 1024 + t7 * 128);
+    // row of token tid >> 2 (and + 64): its kpos position (identity for bf16 K)
+    const int p = kpos<KB>(tid >> 2);
+    const int qq = tid & 3, t7 = p & 7, rot = qq & 2;
+    base = uint32_t(((p >> 3) * 2 + (qq >> 1)) * 1024 + t7 * 128);
 #pragma unroll
     for (int i = 0; i < 4; ++i) x[i] = uint32_t(((4 * (qq & 1) + ((i + rot) & 3)) ^ t7) << 4);
 #pragma unroll
@@ -515,16 +532,18 @@ struct VOffsets {
 
 template <int VB>
 __device__ __noinline__ void fill_v_general(const AttnArgs& a, int u, int64_t tile_start,
-                                            uint8_t* vt, const uint8_t* rs, int tid);
+                                            uint8_t* vt, const uint8_t* rs, int tid, int perm_kb);
 
-// V tile: the whole-quantized-tile case inline, the rest out of line
-template <int VB>
+// V tile: the whole-quantized-tile case inline, the rest out of line.  Rows
+// follow the K tile's order: kpos when the tile's K is wholly quantized.
+template <int KB, int VB>
 __device__ __forceinline__ void fill_v_tile(const AttnArgs& a, int u, int64_t tile_start,
                                             uint8_t* vt, const uint8_t* rs, int tid,
-                                            const VOffsets& vo) {
+                                            const VOffsets<KB>& vo) {
   const CacheView& cv = a.c;
+  const bool k_whole = KB < 16 && tile_start + TT <= a.Lq;
   if constexpr (VB < 16) {
-    if (tile_start + TT <= a.L) {
+    if (KB < 16 ? k_whole : tile_start + TT <= a.L) {
       // whole tile quantized: one item per iteration (a rolled loop keeps
       // the hot code small)
       using W = typename std::conditional<VB == 4, uint4, uint2>::type;
@@ -555,12 +574,12 @@ __device__ __forceinline__ void fill_v_tile(const AttnArgs& a, int u, int64_t ti
       return;
     }
   }
-  fill_v_general<VB>(a, u, tile_start, vt, rs, tid);
+  fill_v_general<VB>(a, u, tile_start, vt, rs, tid, k_whole ? KB : 16);
 }
 
 template <int VB>
 __device__ __noinline__ void fill_v_general(const AttnArgs& a, int u, int64_t tile_start,
-                                            uint8_t* vt, const uint8_t* rs, int tid) {
+                                            uint8_t* vt, const uint8_t* rs, int tid, int perm_kb) {
   const CacheView& cv = a.c;
   const int d = kHeadDim;
 #pragma unroll 1
@@ -568,6 +587,8 @@ __device__ __noinline__ void fill_v_general(const AttnArgs& a, int u, int64_t ti
     const int item = tid + 256 * r;
     const int t = item >> 2, qq = item & 3;
     const int64_t pos = tile_start + t;
+    // row of token t (the K tile's order, see kpos)
+    const int p = perm_kb == 2 ? kpos<2>(t) : (perm_kb == 4 ? kpos<4>(t) : t);
     uint4 out[4];
     const uint16_t* raw = nullptr;
     bool codes = false;
@@ -612,7 +633,7 @@ __device__ __noinline__ void fill_v_general(const AttnArgs& a, int u, int64_t ti
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-      *reinterpret_cast<uint4*>(vt + vt_off(t, 32 * qq + 8 * ((i + rot) & 3))) = out[i];
+      *reinterpret_cast<uint4*>(vt + vt_off(p, 32 * qq + 8 * ((i + rot) & 3))) = out[i];
   }
 }
 
@@ -894,6 +915,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         a.part_ml[(size_t(u) * a.nsplit + sp) * cv.rows + r] = make_float2(rf, lt);
     }
   } else if (warp < 24) {
+    regs_dec<kRegProducer>();
     if (warp < 16) {
     // ------------------------------------------------------------ K producer
     const int c = (threadIdx.x - 256) & 127;   // channel
@@ -913,13 +935,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     } else {
     // ------------------------------------------------------------ V producer
     const int t = threadIdx.x - 512;
-    const VOffsets vo(t, cv.vw, cv.vgroups, cv.GV, VB < 16 ? VB : 16);
+    const VOffsets<KB> vo(t, cv.vw, cv.vgroups, cv.GV, VB < 16 ? VB : 16);
 #pragma unroll 1
     for (int j = 0; j < nt; ++j) {
       const int b = j & 1, st = j % kStages;
       if (!mbar_wait(bar(VEMPTY + b), ((j >> 1) & 1) ^ 1, abort_flag, cv.status)) break;
       if (!mbar_wait(bar(RFULL + st), (j / kStages) & 1, abort_flag, cv.status)) break;
-      fill_v_tile<VB>(a, u, (t_begin + j) * TT, sm + (b ? Smem::kV1 : Smem::kV0),
+      fill_v_tile<KB, VB>(a, u, (t_begin + j) * TT, sm + (b ? Smem::kV1 : Smem::kV0),
                       sm + Smem::kRing + st * Smem::kStageBytes, t, vo);
       fence_async_smem();
       mbar_arrive(bar(VFULL + b));

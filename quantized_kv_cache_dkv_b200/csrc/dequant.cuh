@@ -79,6 +79,34 @@ __device__ __forceinline__ void dequant2x16(uint32_t w, __half2 s2, __half2 z2, 
   hi.w = prmt(v[6], v[7], 0x7632);
 }
 
+// The same conversions without the element reordering (no prmt): 4-bit
+// halves come out as (e0, e4), (e1, e5), (e2, e6), (e3, e7); 2-bit halves as
+// a = (e0, e8), (e1, e9), (e2, e10), (e3, e11) and b = (e4, e12), ...,
+// (e7, e15).  A tile stored in this order holds its tokens permuted within
+// groups of 8 (4-bit) or 16 (2-bit) tokens.
+__device__ __forceinline__ uint4 dequant4x8_raw(uint32_t w, __half2 s2, __half2 z2) {
+  const uint32_t w8 = w >> 8;
+  uint4 r;
+  r.x = h2u(__hfma2(unbias(and_or(w, 0x000F000Fu, kMagic1024), 1.f, -1024.f), s2, z2));
+  r.y = h2u(__hfma2(unbias(and_or(w, 0x00F000F0u, kMagic1024), 0.0625f, -64.f), s2, z2));
+  r.z = h2u(__hfma2(unbias(and_or(w8, 0x000F000Fu, kMagic1024), 1.f, -1024.f), s2, z2));
+  r.w = h2u(__hfma2(unbias(and_or(w8, 0x00F000F0u, kMagic1024), 0.0625f, -64.f), s2, z2));
+  return r;
+}
+
+__device__ __forceinline__ void dequant2x16_raw(uint32_t w, __half2 s2, __half2 z2, uint4& a,
+                                                uint4& b) {
+  const uint32_t w8 = w >> 8;
+  a.x = h2u(__hfma2(unbias(and_or(w, 0x00030003u, kMagic1024), 1.f, -1024.f), s2, z2));
+  a.y = h2u(__hfma2(unbias(and_or(w, 0x000C000Cu, kMagic1024), 0.25f, -256.f), s2, z2));
+  a.z = h2u(__hfma2(unbias(and_or(w, 0x00300030u, kMagic1024), 0.0625f, -64.f), s2, z2));
+  a.w = h2u(__hfma2(unbias(and_or(w, 0x00C000C0u, kMagic1024), 0.015625f, -16.f), s2, z2));
+  b.x = h2u(__hfma2(unbias(and_or(w8, 0x00030003u, kMagic1024), 1.f, -1024.f), s2, z2));
+  b.y = h2u(__hfma2(unbias(and_or(w8, 0x000C000Cu, kMagic1024), 0.25f, -256.f), s2, z2));
+  b.z = h2u(__hfma2(unbias(and_or(w8, 0x00300030u, kMagic1024), 0.0625f, -64.f), s2, z2));
+  b.w = h2u(__hfma2(unbias(and_or(w8, 0x00C000C0u, kMagic1024), 0.015625f, -16.f), s2, z2));
+}
+
 // 8 bf16 -> 8 fp16 (exact inside fp16's normal range)
 __device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 x) {
   auto cvt = [](uint32_t w) -> uint32_t {
