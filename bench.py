@@ -359,49 +359,121 @@ def run_gpu(w: synth.Workload, K: int, W: int, want_e2e=True, log=print, kernel=
     # end to end through the public API from pinned host memory
     e2e = None
     if want_e2e:
-        pin = lambda a: torch.from_numpy(a).pin_memory()  # noqa: E731
         import numpy as np
-        hb = [(pin(a.view(np.int16)), pin(b.view(np.int16)), pin(m.view(np.int32)))
-              for a, b, m in host_blocks]
-        hs = [(pin(q.view(np.int16)), pin(ka.view(np.int16)), pin(va.view(np.int16)))
-              for q, ka, va in host_steps]
-        hout = torch.empty((w.B, w.Hq, w.blk, w.d), dtype=torch.int16).pin_memory()
-        dK = torch.empty((w.B, w.Hkv, w.blk, w.d), dtype=torch.int16, device=dev)
-        dV, dKa, dVa = torch.empty_like(dK), torch.empty_like(dK), torch.empty_like(dK)
-        dM = torch.empty((w.B, w.Hkv, w.blk // 32), dtype=torch.int32, device=dev)
-        dQ = torch.empty((w.B, w.Hq, w.blk, w.d), dtype=torch.int16, device=dev)
-        dO = torch.empty_like(dQ)
-        h2d = (dK.numel() * 2 * 2 + dM.numel() * 4 + dQ.numel() * 2 + dKa.numel() * 2 * 2)
-        d2h = dO.numel() * 2
+        # Three streams, two buffer sets: step k+1's inputs go up while step
+        # k computes, and step k's output comes down while step k+1 computes.
+        # Every step still copies its own inputs from pinned host memory and
+        # reads its own result back inside the timed region.
+        s_up, s_dn = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+        s_cp = stream
+        nb = 2
+        # One step's inputs -- K, V block and protect words (commit), Q and
+        # the active K, V (attention) -- packed in one pinned host buffer per
+        # (block, step) pair, so each step uploads them with one copy into a
+        # device buffer of the same layout (the API takes views into it).
+        n_kv = w.B * w.Hkv * w.blk * w.d
+        n_q = w.B * w.Hq * w.blk * w.d
+        n_m = w.B * w.Hkv * (w.blk // 32)
+        n_m16 = (2 * n_m + 7) // 8 * 8  # the words' int16 slots, padded to 16 bytes
+        offs = [0, n_kv, 2 * n_kv, 2 * n_kv + n_m16, 2 * n_kv + n_m16 + n_q,
+                3 * n_kv + n_m16 + n_q]  # int16 element offsets: K, V, M, Q, Ka, Va
+        n_in = 4 * n_kv + n_m16 + n_q
+        hin = {}
+        for c in range(C):
+            for st in range(S):
+                buf = torch.empty(n_in, dtype=torch.int16)
+                a_, b_, m_ = host_blocks[c]
+                q_, ka_, va_ = host_steps[st]
+                npb = buf.numpy()
+                npb[offs[0]:offs[1]] = a_.view(np.int16).ravel()
+                npb[offs[1]:offs[2]] = b_.view(np.int16).ravel()
+                npb[offs[2]:offs[2] + 2 * n_m] = m_.view(np.int32).ravel().view(np.int16)
+                npb[offs[3]:offs[4]] = q_.view(np.int16).ravel()
+                npb[offs[4]:offs[5]] = ka_.view(np.int16).ravel()
+                npb[offs[5]:] = va_.view(np.int16).ravel()
+                hin[(c, st)] = buf.pin_memory()
+        dIn = [torch.empty(n_in, dtype=torch.int16, device=dev) for _ in range(nb)]
+        shp_kv = (w.B, w.Hkv, w.blk, w.d)
+        shp_q = (w.B, w.Hq, w.blk, w.d)
+        views = []
+        for bf in dIn:
+            views.append((bf[offs[0]:offs[1]].view(shp_kv), bf[offs[1]:offs[2]].view(shp_kv),
+                          bf[offs[2]:offs[2] + 2 * n_m].view(torch.int32).view(w.B, w.Hkv, w.blk // 32),
+                          bf[offs[3]:offs[4]].view(shp_q), bf[offs[4]:offs[5]].view(shp_kv),
+                          bf[offs[5]:].view(shp_kv)))
+        dO = [torch.empty(shp_q, dtype=torch.int16, device=dev) for _ in range(nb)]
+        hout = [torch.empty(shp_q, dtype=torch.int16).pin_memory() for _ in range(nb)]
+        ev_up = [torch.cuda.Event() for _ in range(nb)]     # inputs of buffer b are on the device
+        ev_cp = [torch.cuda.Event() for _ in range(nb)]     # step using buffer b has computed
+        ev_dn = [torch.cuda.Event() for _ in range(nb)]     # output of buffer b is on the host
+        h2d = n_in * 2
+        d2h = dO[0].numel() * 2
+        used = [False] * nb
 
-        def e2e_step(k):
-            r = k % R
-            c = pos[r]
-            dK.copy_(hb[c][0], non_blocking=True)
-            dV.copy_(hb[c][1], non_blocking=True)
-            dM.copy_(hb[c][2], non_blocking=True)
+        def upload(k):
+            b = k % nb
+            with torch.cuda.stream(s_up):
+                if used[b]:
+                    s_up.wait_event(ev_cp[b])  # the step that read buffer b is done
+                dIn[b].copy_(hin[(pos_e[k % R], k % S)], non_blocking=True)
+                ev_up[b].record(s_up)
+
+        def compute(k):
+            b, r = k % nb, k % R
+            s_cp.wait_event(ev_up[b])
+            if used[b]:
+                s_cp.wait_event(ev_dn[b])  # the previous output in dO[b] has been read back
+            dK, dV, dM, dQ, dKa, dVa = views[b]
             dkv.dkv_commit_block(caches[r], dK, dV, dM)
-            q, ka, va = hs[k % S]
-            dQ.copy_(q, non_blocking=True)
-            dKa.copy_(ka, non_blocking=True)
-            dVa.copy_(va, non_blocking=True)
-            dkv.dkv_block_attention(caches[r], dQ, dKa, dVa, w.softmax_scale, dO)
-            hout.copy_(dO, non_blocking=True)
+            dkv.dkv_block_attention(caches[r], dQ, dKa, dVa, w.softmax_scale, dO[b])
+            ev_cp[b].record(s_cp)
             pos[r] += 1
             if pos[r] == C:
                 dkv.dkv_cache_truncate(caches[r], w.L)
                 pos[r] = 0
 
-        for k in range(W):
-            e2e_step(k)
+        def download(k):
+            b = k % nb
+            with torch.cuda.stream(s_dn):
+                s_dn.wait_event(ev_cp[b])
+                hout[b].copy_(dO[b], non_blocking=True)
+                ev_dn[b].record(s_dn)
+            used[b] = True
+
+        pos_e = [0] * R  # block index of the next commit of each cache, for uploads
+
+        def run(n):
+            for i in range(nb):
+                used[i] = False
+            for r in range(R):
+                pos_e[r] = pos[r]
+            upload(0)
+            pos_e[0 % R] = (pos_e[0 % R] + 1) % C
+            for k in range(n):
+                if k + 1 < n:
+                    upload(k + 1)
+                    pos_e[(k + 1) % R] = (pos_e[(k + 1) % R] + 1) % C
+                compute(k)
+                download(k)
+
+        def join_streams():
+            for st in (s_up, s_dn):
+                ev = torch.cuda.Event()
+                ev.record(st)
+                s_cp.wait_event(ev)
+
+        run(W)
+        join_streams()
         finish()
         torch.cuda.synchronize()
         barrier()
         torch.cuda.synchronize()
-        e0.record(stream)
-        for k in range(K):
-            e2e_step(k)
-        e1.record(stream)
+        e0.record(s_cp)
+        s_up.wait_stream(s_cp)
+        s_dn.wait_stream(s_cp)
+        run(K)
+        join_streams()
+        e1.record(s_cp)
         torch.cuda.synchronize()
         barrier()
         ems = e0.elapsed_time(e1)
