@@ -4,32 +4,35 @@
 // 128 rows, each padded with zero queries to the M = 128 MMA shape.  Attention is computed "directly
 // from low-bit KV" (MaskAhead / Q-MaskAhead abstract) at every denoising step.
 //
-// CTA = (unit, token split, row block), one CTA per SM, 24 warps (six
-// warpgroups; setmaxnreg moves registers from the producers and the control
-// warps to the softmax warpgroup):
-//   warps 0-7   softmax, two warpgroups: thread (r, h) owns query row r (=
-//               TMEM lane r) and columns [64h, 64h+64) of each S tile; loads
-//               its half of Q into TMEM, runs the online softmax (row maxima
-//               of the two halves exchanged through shared memory on an
-//               mbarrier), writes P (fp16) into its own half of S, rescales
-//               its half of O when the running max grows by > 2^8, and writes
-//               its half of the output / split partial at the end
+// CTA = (unit, token split, row block), one CTA per SM, 28 warps (seven
+// warpgroups; setmaxnreg: softmax 96 registers, producers 64, control 56):
+//   warps 0-7   softmax, two warpgroups: warpgroup h takes the 128-token
+//               tiles j = h (mod 2); thread = query row = TMEM lane, all 128
+//               columns.  Loads its half of Q into TMEM; per tile: the row
+//               max of S (pass 1), the reference max handed over from the
+//               previous tile through shared memory (raised only when the
+//               tile max exceeds it by more than 8 in log2 units, so P <= 2^8),
+//               P = 2^(s*scale - ref) as fp16 pairs written over the first 64
+//               columns of its S buffer (pass 2), O rescaled in TMEM when the
+//               reference rose; at the end the two warpgroups' row sums are
+//               merged and each writes half of the output / split partial
 //   warps 8-15  K producers: dequantize 128-token K tiles into shared memory
 //               (channel rows, tokens contiguous: MN-major, 128-byte swizzle);
 //               two warps per SM sub-partition, half a tile each
 //   warps 16-23 V producers: dequantize V tiles (token rows, channels
 //               contiguous: MN-major, 128-byte swizzle), half a tile each
-//   warp 24     allocates TMEM; one lane issues the MMAs:
+//   warp 25     allocates TMEM; one lane issues the MMAs:
 //               S_j = Q K_j^T (A = Q from TMEM), O += P_j V_j (A = P from TMEM)
-//   warp 25     one lane streams each tile's packed K/V codes and fp16
+//   warp 26     one lane streams each tile's packed K/V codes and fp16
 //               (scale, zero) pairs -- four contiguous ranges of the cache --
-//               into a 3-stage shared-memory ring with 1-D bulk copies
+//               and the tile's slice of the protected-K side table into a
+//               3-stage shared-memory ring with 1-D bulk copies
 //               (cp.async.bulk, completion counted on an mbarrier), so HBM
 //               latency overlaps the dequantization and the MMAs
 // Tensor memory (512 columns x 128 lanes x 32 bit): O [0,128), S0 [128,256),
-// S1 [256,384), Q [384,448).  P_j (fp16 pairs) overwrites, per half h, the
-// columns [64h, 64h+32) of S_(j mod 2) once that half's scores are read; the
-// PV MMAs take their A operand from those two 32-column pieces.
+// S1 [256,384), Q [384,448).  P_j (fp16 pairs) overwrites the first 64
+// columns of S_(j mod 2) once the scores are read; the PV MMAs take their A
+// operand there.
 // Hand-offs are mbarriers; MMA completion arrives through tcgen05.commit.
 // Every wait is bounded (about one second of %globaltimer): on expiry the
 // CTA raises DKV_FLAG_TIMEOUT, all roles leave their loops, the MMA lane waits
@@ -45,8 +48,11 @@ namespace {
 constexpr int TT = kTcTile;              // tokens per tile
 constexpr int kWarps = 28;  // seven warpgroups; warps 26, 27 only complete the last one
 constexpr int kThreads = kWarps * 32;
-constexpr int kMmaWarp = 24;
-constexpr int kLoadWarp = 25;
+// The MMA lane and the loader sit on sub-partitions 1 and 2: with query
+// groups of 32 rows all softmax work lands on sub-partition 0 (TMEM lanes
+// 0-31 belong to warps 0 and 4).
+constexpr int kMmaWarp = 25;
+constexpr int kLoadWarp = 26;
 constexpr int kStages = 3;  // ring of packed tiles
 constexpr int kStagedProt = 24;  // protected K rows staged per tile (more: read from global)
 constexpr uint32_t kTileBytes = 128 * 128 * 2;
