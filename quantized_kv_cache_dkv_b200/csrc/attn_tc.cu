@@ -336,7 +336,10 @@ __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
 // chunk i (0..7) holds tokens 64 qh + 8 i .. +7 of channel c.
 // Tiles whose K is wholly quantized are stored in the order the prmt-free
 // dequantization produces: the token at tile position kpos(t) is t, permuted
-// within groups of 16 (2-bit codes) or 8 (4-bit codes).  The V tile of such a
+// within groups of 16 (2-bit codes) or 8 (4-bit codes).  V tiles hold their
+// channels in the same kind of order for V's bit width (kpos<VB>, in every
+// tile, bf16 rows included), so O's column kpos<VB>(c) is channel c and the
+// epilogue reads it from there.  The V tile of such a
 // tile puts token t's row at the same position, so P V pairs every score with
 // its own value row; the softmax does not depend on column order.  Other
 // tiles (K tail, active block, bf16 K) keep the natural order.
@@ -561,17 +564,17 @@ __device__ __forceinline__ void fill_v_tile(const AttnArgs& a, int u, int64_t ti
         const __half2 sz = reinterpret_cast<const __half2*>(rs + Smem::kRVsz)[r ? vo.z[1] : vo.z[0]];
         const __half2 s2 = __half2half2(__low2half(sz));
         const __half2 z2 = __half2half2(__high2half(sz));
-        uint4 out[4];
+        uint4 out[4];  // channels in kpos<VB> order
         if constexpr (VB == 4) {
           if (rot) x = make_uint4(x.z, x.w, x.x, x.y);
-          out[0] = dequant4x8(x.x, s2, z2);
-          out[1] = dequant4x8(x.y, s2, z2);
-          out[2] = dequant4x8(x.z, s2, z2);
-          out[3] = dequant4x8(x.w, s2, z2);
+          out[0] = dequant4x8_raw(x.x, s2, z2);
+          out[1] = dequant4x8_raw(x.y, s2, z2);
+          out[2] = dequant4x8_raw(x.z, s2, z2);
+          out[3] = dequant4x8_raw(x.w, s2, z2);
         } else {
           if (rot) x = make_uint2(x.y, x.x);
-          dequant2x16(x.x, s2, z2, out[0], out[1]);
-          dequant2x16(x.y, s2, z2, out[2], out[3]);
+          dequant2x16_raw(x.x, s2, z2, out[0], out[1]);
+          dequant2x16_raw(x.y, s2, z2, out[2], out[3]);
         }
         uint8_t* dst = vt + vo.base + 16384u * uint32_t(r);
 #pragma unroll
@@ -617,22 +620,46 @@ __device__ __noinline__ void fill_v_general(const AttnArgs& a, int u, int64_t ti
         if constexpr (VB == 4) {
           uint4 w = *reinterpret_cast<const uint4*>(vc + qq * 4);
           if (rot) w = make_uint4(w.z, w.w, w.x, w.y);
-          out[0] = dequant4x8(w.x, s2, z2);
-          out[1] = dequant4x8(w.y, s2, z2);
-          out[2] = dequant4x8(w.z, s2, z2);
-          out[3] = dequant4x8(w.w, s2, z2);
+          out[0] = dequant4x8_raw(w.x, s2, z2);
+          out[1] = dequant4x8_raw(w.y, s2, z2);
+          out[2] = dequant4x8_raw(w.z, s2, z2);
+          out[3] = dequant4x8_raw(w.w, s2, z2);
         } else {
           uint2 w = *reinterpret_cast<const uint2*>(vc + qq * 2);
           if (rot) w = make_uint2(w.y, w.x);
-          dequant2x16(w.x, s2, z2, out[0], out[1]);
-          dequant2x16(w.y, s2, z2, out[2], out[3]);
+          dequant2x16_raw(w.x, s2, z2, out[0], out[1]);
+          dequant2x16_raw(w.y, s2, z2, out[2], out[3]);
         }
       }
     } else if (raw) {
+      uint4 nat[4];  // channels 32qq + 8k .. + 7, natural order
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        out[i] = bf16x8_to_f16x8(
-            __ldg(reinterpret_cast<const uint4*>(raw + qq * 32 + 8 * ((i + rot) & 3))));
+      for (int k = 0; k < 4; ++k)
+        nat[k] = bf16x8_to_f16x8(__ldg(reinterpret_cast<const uint4*>(raw + qq * 32 + 8 * k)));
+      uint4 pc[4];  // the same channels in kpos<VB> order (the quantized rows' order)
+      if constexpr (VB == 4) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          pc[k] = make_uint4(prmt(nat[k].x, nat[k].z, 0x5410), prmt(nat[k].x, nat[k].z, 0x7632),
+                             prmt(nat[k].y, nat[k].w, 0x5410), prmt(nat[k].y, nat[k].w, 0x7632));
+      } else if constexpr (VB == 2) {
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+          const uint4 A = nat[2 * g], B = nat[2 * g + 1];
+          pc[2 * g] = make_uint4(prmt(A.x, B.x, 0x5410), prmt(A.x, B.x, 0x7632),
+                                 prmt(A.y, B.y, 0x5410), prmt(A.y, B.y, 0x7632));
+          pc[2 * g + 1] = make_uint4(prmt(A.z, B.z, 0x5410), prmt(A.z, B.z, 0x7632),
+                                     prmt(A.w, B.w, 0x5410), prmt(A.w, B.w, 0x7632));
+        }
+      } else {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) pc[k] = nat[k];
+      }
+      // rot is 0 or 2
+      out[0] = rot ? pc[2] : pc[0];
+      out[1] = rot ? pc[3] : pc[1];
+      out[2] = rot ? pc[0] : pc[2];
+      out[3] = rot ? pc[1] : pc[3];
     } else {
 #pragma unroll
       for (int i = 0; i < 4; ++i) out[i] = make_uint4(0u, 0u, 0u, 0u);
@@ -902,8 +929,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             uint32_t w[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-              const __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(o[8 * i + 2 * k]) * inv,
-                                                             __uint_as_float(o[8 * i + 2 * k + 1]) * inv);
+              // O column kpos<VB>(c) holds channel c (the V tile's order)
+              const __nv_bfloat162 v = __floats2bfloat162_rn(
+                  __uint_as_float(o[kpos<VB>(8 * i + 2 * k)]) * inv,
+                  __uint_as_float(o[kpos<VB>(8 * i + 2 * k + 1)]) * inv);
               w[k] = *reinterpret_cast<const uint32_t*>(&v);
             }
             dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
@@ -913,8 +942,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
               a.part_o + ((size_t(u) * a.nsplit + sp) * cv.rows + r) * kHeadDim + col);
 #pragma unroll
           for (int i = 0; i < 8; ++i)
-            dst[i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
-                                 __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
+            dst[i] = make_float4(__uint_as_float(o[kpos<VB>(4 * i)]), __uint_as_float(o[kpos<VB>(4 * i + 1)]),
+                                 __uint_as_float(o[kpos<VB>(4 * i + 2)]), __uint_as_float(o[kpos<VB>(4 * i + 3)]));
         }
       }
       if (a.nsplit > 1 && row_ok && h == 0)

@@ -53,3 +53,41 @@ def test_tc_empty_and_ragged(dkv):
 def test_tc_many_splits_long_cache(dkv):
     w = SHRUNK["longprompt"].with_(L=4096, Hq=4, Hkv=1)
     _run_case(dkv, w, 128, steps=(2,), splits=(1, 7, 0), kernel=2, check_export=False)
+
+
+@pytest.mark.parametrize("kernel", [1, 2])
+@pytest.mark.parametrize("blk,hq,hkv,gk", [(64, 4, 2, 32), (96, 2, 2, 32), (128, 2, 1, 128),
+                                           (32, 5, 1, 64), (64, 2, 1, 128)])
+def test_block_sizes_and_row_counts(dkv, kernel, blk, hq, hkv, gk):
+    """Blocks of 64, 96 and 128 tokens and query groups of 96, 128, 160 and
+    256 rows (padding warps, two row blocks, K groups longer and shorter than
+    the block)."""
+    w = SHRUNK["batch32"].with_(blk=blk, Hq=hq, Hkv=hkv, k_group=gk, v_group=32,
+                                L=(640 // blk) * blk)
+    _run_case(dkv, w, w.L // w.blk, steps=(0,), splits=(0, 2), kernel=kernel)
+
+
+@pytest.mark.parametrize("kernel", [1, 2])
+@pytest.mark.parametrize("scale_mul", [-1.0, 0.0, 3.0])
+def test_softmax_scale_sign_zero_and_large(dkv, kernel, scale_mul):
+    """A negative scale (folded into Q on the tcgen05 path), zero (uniform
+    weights: the mean of V) and three times the workload's (peaked weights,
+    frequent reference rises; the fp16-operand score error grows with the
+    scale, so the bound does too)."""
+    import torch
+    from gpu_util import assert_close, default_P, default_cap, dev_bf16, host_bits, oracle_cache
+    w = SHRUNK["gqa7b"]
+    cache, _ = _run_case(dkv, w, w.L // w.blk, steps=(), kernel=kernel)
+    cap = default_cap(w, w.L // w.blk + 1)
+    ref_cache = oracle_cache(w, cap, default_P(w, cap))
+    for i in range(w.L // w.blk):
+        K, V, M = synth.block_inputs(w, i)
+        ref_cache.commit(K, V, M)
+    Q = synth.queries_bits(w, 4)
+    Ka, Va = synth.active_block_bits(w, 4)
+    scale = w.softmax_scale * scale_mul
+    out = torch.empty((w.B, w.Hq, w.blk, w.d), dtype=torch.bfloat16, device="cuda")
+    dkv.dkv_block_attention(cache, dev_bf16(Q), dev_bf16(Ka), dev_bf16(Va), scale, out)
+    torch.cuda.synchronize()
+    assert_close(host_bits(out), ref_cache.block_attention(Q, Ka, Va, scale),
+                 scale_mul=abs(scale_mul))
