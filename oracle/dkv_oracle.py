@@ -174,7 +174,7 @@ class OracleCache:
     """
 
     def __init__(self, B, Hq, Hkv, d, blk, k_bits, v_bits, k_group, v_group,
-                 max_protected, capacity):
+                 max_protected, capacity, sink_tokens=0):
         assert Hq % Hkv == 0
         assert k_bits in (2, 4, 16) and v_bits in (2, 4, 16)
         assert capacity % k_group == 0 and capacity % blk == 0
@@ -203,6 +203,14 @@ class OracleCache:
         self.prot_pos = np.full((U, max(max_protected, 0)), -1, np.int32)
         self.prot_k = np.zeros((U, max(max_protected, 0), d), np.uint16)
         self.prot_gstart = np.zeros((U, nG + 1), np.int32)
+        # Attention sink: the first sink_tokens positions of every sequence stay
+        # in full precision ("keeping the attention sink in full precision"
+        # matters at 2-bit KV -- SoloQ, KV-only paragraph).  Reading: their K
+        # is protected like any protected entry (side table), their V is kept
+        # as bf16 next to the codes (which are still computed and stored).
+        assert 0 <= sink_tokens <= capacity
+        self.sink = int(sink_tokens)
+        self.v_sink = np.zeros((U, self.sink, d), np.uint16)
 
     # -- derived sizes
     @property
@@ -233,6 +241,12 @@ class OracleCache:
             pw = np.asarray(protect_words, np.uint32).reshape(self.U, -1)
             prot = mask_words_to_bool(pw, blk)
         p0 = self.len
+        # sink positions: K always protected, V kept in bf16
+        ns = max(0, min(self.sink - p0, blk))
+        if ns:
+            prot = prot.copy()
+            prot[:, :ns] = True
+            self.v_sink[:, p0:p0 + ns] = V_bits[:, :ns]
         flags = 0
         for u in range(self.U):
             flags |= self._commit_v(u, p0, V_bits[u])
@@ -348,7 +362,11 @@ class OracleCache:
         q = q.reshape(L, d // GV, GV)
         s = self.v_sz[u, :L, :, 0].astype(np.float64)[..., None]
         z = self.v_sz[u, :L, :, 1].astype(np.float64)[..., None]
-        return (q * s + z).reshape(L, d)
+        v = (q * s + z).reshape(L, d)
+        ns = min(self.sink, L)
+        if ns:
+            v[:ns] = bf16_to_f64(self.v_sink[u, :ns])
+        return v
 
     # -- attention at one denoising step
     def block_attention(self, Q_bits, Kact_bits, Vact_bits, scale: float) -> np.ndarray:
@@ -390,6 +408,8 @@ class OracleCache:
             out["v_raw"] = self.v_raw[:, :L].copy()
         out["prot_pos"] = self.prot_pos.copy()
         out["prot_k"] = self.prot_k.copy()
+        if self.sink and self.vb < 16:
+            out["v_sink"] = self.v_sink[:, :min(self.sink, L)].copy()
         return out
 
 

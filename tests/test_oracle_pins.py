@@ -9,6 +9,7 @@ import numpy as np
 import pytest
 
 from oracle import (FLAG_CAPACITY, FLAG_RANGE, CapacityError, OracleCache, bf16_to_f64,
+                    bool_to_mask_words,
                     dense_attention_f64, mask_words_to_bool, pack_codes, quantize_groups,
                     quantize_stream_oneshot, to_fp16, unpack_codes)
 import synth
@@ -580,3 +581,55 @@ def test_truncate_then_recommit_equals_fresh_cache(gk):
         assert np.array_equal(a["prot_k"][u, :n], b["prot_k"][u, :n])
     with pytest.raises(ValueError):
         c.truncate(32 if gk == 64 else 33)
+
+
+# -- attention sink (positions [0, sink) kept in full precision)
+
+@pytest.mark.parametrize("sink,kb,gk", [(1, 4, 32), (5, 2, 64), (40, 4, 32), (96, 2, 32)])
+def test_sink_rows_exact_in_k_and_v(sink, kb, gk):
+    """Sink positions come back bit-exact in both K and V; V rows past the
+    sink are the quantized ones; K statistics leave the sink out exactly as
+    an explicit protection mask does."""
+    w = SMALL.with_(B=1, Hkv=2, Hq=2, prot_frac=0.0)
+    cap = 256
+    c = OracleCache(w.B, w.Hq, w.Hkv, w.d, w.blk, kb, kb, gk, 32, 128, cap, sink_tokens=sink)
+    ref = OracleCache(w.B, w.Hq, w.Hkv, w.d, w.blk, kb, kb, gk, 32, 128, cap)
+    nblk = 4
+    Ks, Vs = [], []
+    for i in range(nblk):
+        K, V, _ = synth.block_inputs(w, i)
+        Ks.append(K.reshape(2, w.blk, w.d))
+        Vs.append(V.reshape(2, w.blk, w.d))
+        c.commit(K, V, None)
+        # the same tokens protected explicitly in the reference cache
+        pos = np.arange(i * w.blk, (i + 1) * w.blk)
+        prot = np.broadcast_to(pos < sink, (2, w.blk))
+        ref.commit(K, V, bool_to_mask_words(prot).reshape(1, 2, -1))
+    Kall, Vall = np.concatenate(Ks, 1), np.concatenate(Vs, 1)   # [U, L, d]
+    ns = min(sink, nblk * w.blk)
+    sa, sr = c.snapshot(), ref.snapshot()
+    for key in ("k_codes", "prot_count", "prot_gstart", "prot_pos", "prot_k", "v_codes"):
+        assert np.array_equal(sa[key], sr[key]), key
+    for u in range(2):
+        assert sa["prot_pos"][u, :ns].tolist() == list(range(ns))
+        assert np.array_equal(c.dequant_k(u)[:ns], bf16_to_f64(Kall[u, :ns]))
+        vh = c.dequant_v(u)
+        assert np.array_equal(vh[:ns], bf16_to_f64(Vall[u, :ns]))
+        # past the sink V is the quantized value, as without a sink
+        assert np.array_equal(vh[ns:], ref.dequant_v(u)[ns:])
+        assert np.array_equal(sa["v_sink"][u], Vall[u, :ns])
+
+
+def test_sink_survives_truncation_and_recommit():
+    w = SMALL.with_(B=1, Hkv=1, Hq=1, prot_frac=0.0)
+    c = OracleCache(1, 1, 1, w.d, w.blk, 2, 2, 32, 32, 64, 256, sink_tokens=48)
+    blocks = [synth.block_inputs(w, i) for i in range(6)]
+    for K, V, _ in blocks[:3]:
+        c.commit(K, V, None)
+    c.truncate(32)
+    K5, V5, _ = blocks[5]
+    c.commit(K5, V5, None)     # positions 32..63: 32..47 are sink positions again
+    vh = c.dequant_v(0)
+    assert np.array_equal(vh[:32], bf16_to_f64(blocks[0][1].reshape(w.blk, w.d)))
+    assert np.array_equal(vh[32:48], bf16_to_f64(V5.reshape(w.blk, w.d)[:16]))
+    assert c.snapshot()["prot_pos"][0, :48].tolist() == list(range(48))
