@@ -82,6 +82,14 @@ typedef struct dkv_config {
   int32_t v_group;       /* GV: channels per V group (per token) */
   int32_t max_protected; /* side-table capacity per (sequence, kv-head) */
   int64_t max_tokens;    /* capacity per sequence */
+  int32_t sink_tokens;   /* attention sink: positions [0, sink_tokens) of every
+                            sequence stay in full precision -- K protected (a
+                            side-table entry each, counted in max_protected),
+                            V kept as bf16 beside its codes.  0 = none; at
+                            most 256 and max_tokens.  At 2-bit KV keeping the
+                            sink in full precision matters (SoloQ, KV-only
+                            paragraph). */
+  int32_t reserved;      /* must be 0 */
 } dkv_config;
 
 typedef struct dkv_cache dkv_cache; /* opaque; owns its device memory */
@@ -190,6 +198,7 @@ typedef struct dkv_export {
   int32_t* prot_pos;
   uint16_t* prot_k;
   int32_t* prot_gstart;
+  uint16_t* v_sink;      /* [U][min(sink_tokens, len)][d] bf16 (v_bits < 16) */
 } dkv_export;
 
 int dkv_cache_export(dkv_cache* cache, void* stream, dkv_export* out);

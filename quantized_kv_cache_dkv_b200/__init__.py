@@ -41,7 +41,8 @@ class dkv_config(ctypes.Structure):
                 ("block", ctypes.c_int32), ("k_bits", ctypes.c_int32),
                 ("v_bits", ctypes.c_int32), ("k_group", ctypes.c_int32),
                 ("v_group", ctypes.c_int32), ("max_protected", ctypes.c_int32),
-                ("max_tokens", ctypes.c_int64)]
+                ("max_tokens", ctypes.c_int64), ("sink_tokens", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
 
 
 _P = ctypes.c_void_p
@@ -50,7 +51,7 @@ _P = ctypes.c_void_p
 class dkv_export(ctypes.Structure):
     _fields_ = [(n, _P) for n in ("k_codes", "k_sz", "k_raw", "k_tail", "tail_mask", "v_codes",
                                    "v_sz", "v_raw", "prot_count", "prot_pos", "prot_k",
-                                   "prot_gstart")]
+                                   "prot_gstart", "v_sink")]
 
 
 def _sig(name, args):
@@ -105,9 +106,9 @@ def _ptr(t):
 
 
 def make_config(B, Hq, Hkv, d=128, blk=32, k_bits=4, v_bits=4, k_group=32, v_group=32,
-                max_protected=0, max_tokens=1024) -> dkv_config:
+                max_protected=0, max_tokens=1024, sink_tokens=0) -> dkv_config:
     return dkv_config(B, Hq, Hkv, d, blk, k_bits, v_bits, k_group, v_group, max_protected,
-                      max_tokens)
+                      max_tokens, sink_tokens, 0)
 
 
 class Cache:
@@ -249,6 +250,8 @@ def dkv_cache_export(cache: Cache, stream=None) -> dict:
     if c.v_bits < 16:
         out["v_codes"] = np.zeros((U, L, d * c.v_bits // 32), np.uint32)
         out["v_sz"] = np.zeros((U, L, d // c.v_group, 2), np.float16)
+        if c.sink_tokens > 0:
+            out["v_sink"] = np.zeros((U, min(c.sink_tokens, L), d), np.uint16)
     else:
         out["v_raw"] = np.zeros((U, L, d), np.uint16)
     e = dkv_export()

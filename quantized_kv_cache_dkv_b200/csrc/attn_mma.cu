@@ -145,6 +145,13 @@ __device__ __forceinline__ void fill_chunk(const AttnArgs& a, int u, int64_t pos
         const __half2 s2 = __half2half2(__low2half(sz));
         const __half2 z2 = __half2half2(__high2half(sz));
         uint4* dst = reinterpret_cast<uint4*>(Vt + (ch * 32 + t) * VT_LD + q * 32);
+        if (pos0 + t < c.sink) {  // sink position: its bf16 V row
+          const uint4* src = reinterpret_cast<const uint4*>(
+              c.v_sink + (size_t(u) * c.sink + size_t(pos0 + t)) * d + q * 32);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) dst[k] = bf16x8_to_f16x8(src[k]);
+          continue;
+        }
         if constexpr (VB == 4) {
           const uint4 w = *reinterpret_cast<const uint4*>(c.v_codes + tok * c.vw + q * 4);
           dst[0] = dequant4x8(w.x, s2, z2);

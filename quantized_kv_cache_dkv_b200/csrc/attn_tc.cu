@@ -545,14 +545,16 @@ __device__ __noinline__ void fill_v_general(const AttnArgs& a, int u, int64_t ti
 
 // V tile: the whole-quantized-tile case inline, the rest out of line.  Rows
 // follow the K tile's order: kpos when the tile's K is wholly quantized.
-template <int KB, int VB>
+template <int KB, int VB, bool SINK>
 __device__ __forceinline__ void fill_v_tile(const AttnArgs& a, int u, int64_t tile_start,
                                             uint8_t* vt, const uint8_t* rs, int tid,
                                             const VOffsets<KB>& vo) {
   const CacheView& cv = a.c;
   const bool k_whole = KB < 16 && tile_start + TT <= a.Lq;
   if constexpr (VB < 16) {
-    if (KB < 16 ? k_whole : tile_start + TT <= a.L) {
+    // (with a sink, tiles holding sink positions take the general path, which
+    // reads their bf16 rows)
+    if ((KB < 16 ? k_whole : tile_start + TT <= a.L) && (!SINK || tile_start >= cv.sink)) {
       // whole tile quantized: one item per iteration (a rolled loop keeps
       // the hot code small)
       using W = typename std::conditional<VB == 4, uint4, uint2>::type;
@@ -602,8 +604,12 @@ __device__ __noinline__ void fill_v_general(const AttnArgs& a, int u, int64_t ti
     const uint16_t* raw = nullptr;
     bool codes = false;
     if (pos < a.L) {
-      if constexpr (VB < 16) codes = true;
-      else raw = cv.v_raw + (size_t(u) * cv.cap + pos) * d;
+      if constexpr (VB < 16) {
+        if (pos < cv.sink) raw = cv.v_sink + (size_t(u) * cv.sink + size_t(pos)) * d;  // sink row
+        else codes = true;
+      } else {
+        raw = cv.v_raw + (size_t(u) * cv.cap + pos) * d;
+      }
     } else if (pos < a.n_tok) {
       raw = a.v_act + (size_t(u) * cv.blk + (pos - a.L)) * d;
     }
@@ -672,7 +678,7 @@ __device__ __noinline__ void fill_v_general(const AttnArgs& a, int u, int64_t ti
 
 // ------------------------------------------------------------------ kernel
 
-template <int KB, int VB>
+template <int KB, int VB, bool SINK>
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -976,7 +982,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       const int b = j & 1, st = j % kStages;
       if (!mbar_wait(bar(VEMPTY + b), ((j >> 1) & 1) ^ 1, abort_flag, cv.status)) break;
       if (!mbar_wait(bar(RFULL + st), (j / kStages) & 1, abort_flag, cv.status)) break;
-      fill_v_tile<KB, VB>(a, u, (t_begin + j) * TT, sm + (b ? Smem::kV1 : Smem::kV0),
+      fill_v_tile<KB, VB, SINK>(a, u, (t_begin + j) * TT, sm + (b ? Smem::kV1 : Smem::kV0),
                       sm + Smem::kRing + st * Smem::kStageBytes, t, vo);
       fence_async_smem();
       mbar_arrive(bar(VFULL + b));
@@ -1138,15 +1144,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   }
 }
 
-template <int KB, int VB>
-cudaError_t launch_kv(const AttnArgs& a, cudaStream_t s) {
+template <int KB, int VB, bool SINK>
+cudaError_t launch_kvs(const AttnArgs& a, cudaStream_t s) {
   const size_t smem = Smem::kBytes + 1024;
-  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<KB, VB>,
+  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<KB, VB, SINK>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   const unsigned nrb = unsigned((a.c.rows + 127) / 128);
-  attn_tc_kernel<KB, VB><<<unsigned(a.c.U) * unsigned(a.nsplit) * nrb, kThreads, smem, s>>>(a);
+  attn_tc_kernel<KB, VB, SINK><<<unsigned(a.c.U) * unsigned(a.nsplit) * nrb, kThreads, smem, s>>>(a);
   return cudaGetLastError();
+}
+
+// caches with a sink (and quantized V) run the instantiation that reads the
+// sink's bf16 V rows; the others the one without that check
+template <int KB, int VB>
+cudaError_t launch_kv(const AttnArgs& a, cudaStream_t s) {
+  if (VB < 16 && a.c.sink > 0) return launch_kvs<KB, VB, true>(a, s);
+  return launch_kvs<KB, VB, false>(a, s);
 }
 
 template <int KB>

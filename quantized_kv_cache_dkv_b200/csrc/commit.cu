@@ -94,6 +94,13 @@ __device__ __forceinline__ void stage_rows(uint16_t* dst, const uint16_t* src, i
 
 __device__ __forceinline__ float bf16_at(const uint16_t* p) { return bf16_bits_to_f32(*p); }
 
+// Protect bits of the sink positions [0, sink) among the 32 positions
+// starting at pos0.
+__device__ __forceinline__ uint32_t sink_bits(int64_t pos0, int sink) {
+  const int64_t n = sink - pos0;
+  return n <= 0 ? 0u : (n >= 32 ? 0xFFFFFFFFu : ((1u << uint32_t(n)) - 1u));
+}
+
 // One V group: G consecutive channels of one token (x: shared memory, 16-byte
 // aligned).  Rolled loops over 8-channel chunks and code words keep the code
 // small (each warp runs it once, so its instructions come from the cache).
@@ -222,6 +229,13 @@ commit_kernel(CacheView c, const uint16_t* __restrict__ k, const uint16_t* __res
       dst[i] = x;
     }
   } else if (tid >= 128) {
+    // sink positions keep their V row in bf16 too
+    const int64_t ns = c.sink - p0 < blk ? c.sink - p0 : blk;
+    for (int i = tid - 128; i < ns * (kHeadDim / 8); i += 128) {
+      const int t = i / (kHeadDim / 8), o = i % (kHeadDim / 8);
+      reinterpret_cast<uint4*>(c.v_sink + (size_t(u) * c.sink + size_t(p0 + t)) * d)[o] =
+          *reinterpret_cast<const uint4*>(sv + t * kRowPad + o * 8);
+    }
     const int GV = c.GV;
     const int ngr = d / GV;
     for (int it = tid - 128; it < blk * ngr; it += 128) {
@@ -254,7 +268,9 @@ commit_kernel(CacheView c, const uint16_t* __restrict__ k, const uint16_t* __res
         range_check8(x, range);
         dst[i] = x;
       }
-      if (tid < nbw) tmask[n_tail / 32 + tid] = pw ? pw[size_t(u) * nbw + tid] : 0u;
+      if (tid < nbw)
+        tmask[n_tail / 32 + tid] =
+            (pw ? pw[size_t(u) * nbw + tid] : 0u) | sink_bits(p0 + 32 * tid, c.sink);
     } else if (tid < 128) {
       // pending stream = tail[0, n_tail) ++ block[0, blk) (staged in sk);
       // quantize every complete group (k_group and block divide one another,
@@ -275,6 +291,7 @@ commit_kernel(CacheView c, const uint16_t* __restrict__ k, const uint16_t* __res
               gm[w] = tmask[pwi];
             else
               gm[w] = pw ? pw[size_t(u) * nbw + (pwi - n_tail / 32)] : 0u;
+            gm[w] |= sink_bits(j * GK + 32 * w, c.sink);
           }
         }
         // side table full: keep the first `room` protected tokens by position

@@ -89,6 +89,9 @@ int check_config(const dkv_config* c) {
     return fail(DKV_ERR_INVALID_ARG, "max_tokens must be a multiple of max(k_group, block)");
   if (c->max_tokens > (int64_t(1) << 30))
     return fail(DKV_ERR_INVALID_ARG, "max_tokens too large (limit 2^30)");
+  if (c->sink_tokens < 0 || c->sink_tokens > 256 || c->sink_tokens > c->max_tokens)
+    return fail(DKV_ERR_INVALID_ARG, "sink_tokens must be in [0, min(256, max_tokens)]");
+  if (c->reserved != 0) return fail(DKV_ERR_INVALID_ARG, "reserved must be 0");
   return DKV_OK;
 }
 
@@ -220,6 +223,7 @@ int dkv_cache_alloc(const dkv_config* cfg, void* stream, dkv_cache** out) {
   v.vgroups = v.d / v.GV;
   v.twords = (v.GK + 31) / 32;
   v.U = v.B * v.Hkv;
+  v.sink = cfg->sink_tokens;
   const size_t U = size_t(v.U);
 
   cudaError_t e = cudaGetDevice(&c->device);
@@ -255,6 +259,7 @@ int dkv_cache_alloc(const dkv_config* cfg, void* stream, dkv_cache** out) {
   Region r_st = take(4);
   Region r_po = take(U * size_t(c->max_splits) * v.rows * v.d * 4);
   Region r_pml = take(U * size_t(c->max_splits) * v.rows * 8);
+  Region r_vsink = take(vq ? U * size_t(v.sink) * v.d * 2 : 0);
   c->arena_bytes = off;
 
   e = cudaMalloc(&c->arena, c->arena_bytes);
@@ -279,6 +284,7 @@ int dkv_cache_alloc(const dkv_config* cfg, void* stream, dkv_cache** out) {
   v.status = static_cast<uint32_t*>(at(r_st));
   c->part_o = static_cast<float*>(at(r_po));
   c->part_ml = static_cast<float2*>(at(r_pml));
+  v.v_sink = static_cast<uint16_t*>(at(r_vsink));
 
   // zero everything that carries state (counters, masks, status) -- and the
   // rest, so exports of unused slots are deterministic; prot_pos unused = -1
@@ -449,6 +455,8 @@ int dkv_cache_export(dkv_cache* c, void* stream, dkv_export* o) {
   if (v.vb < 16) {
     DKV_CUDA(copy2d(o->v_codes, v.v_codes, L * v.vw * 4, v.cap * v.vw * 4));
     DKV_CUDA(copy2d(o->v_sz, v.v_sz, L * v.vgroups * 4, v.cap * v.vgroups * 4));
+    const int64_t ns = std::min<int64_t>(v.sink, L);
+    if (ns > 0) DKV_CUDA(copy2d(o->v_sink, v.v_sink, ns * v.d * 2, size_t(v.sink) * v.d * 2));
   } else {
     DKV_CUDA(copy2d(o->v_raw, v.v_raw, L * v.d * 2, v.cap * v.d * 2));
   }

@@ -39,6 +39,8 @@ struct CacheView {
   uint16_t* prot_k;     // [U][P][d]
   int32_t* prot_gstart; // [U][nG + 1]
   uint32_t* status;     // sticky DKV_FLAG_* bits
+  int32_t sink;         // positions [0, sink) in full precision (K protected, V bf16)
+  uint16_t* v_sink;     // [U][sink][d] bf16 V rows of the sink positions (vb < 16)
 };
 
 // Arguments of one attention call.

@@ -30,14 +30,14 @@ def host_bits(t) -> np.ndarray:
     return t.view(torch.int16).cpu().numpy().view(np.uint16)
 
 
-def gpu_config(dkv, w: synth.Workload, cap: int, P: int):
+def gpu_config(dkv, w: synth.Workload, cap: int, P: int, sink: int = 0):
     return dkv.make_config(w.B, w.Hq, w.Hkv, w.d, w.blk, w.k_bits, w.v_bits, w.k_group,
-                           w.v_group, P, cap)
+                           w.v_group, P, cap, sink)
 
 
-def oracle_cache(w: synth.Workload, cap: int, P: int, B=None, Hkv=None, Hq=None):
+def oracle_cache(w: synth.Workload, cap: int, P: int, B=None, Hkv=None, Hq=None, sink=0):
     return OracleCache(B or w.B, Hq or w.Hq, Hkv or w.Hkv, w.d, w.blk, w.k_bits, w.v_bits,
-                       w.k_group, w.v_group, P, cap)
+                       w.k_group, w.v_group, P, cap, sink)
 
 
 def default_cap(w: synth.Workload, n_blocks: int) -> int:
@@ -64,7 +64,7 @@ def compare_exports(gpu: dict, ref: dict, units=None):
     sel = (lambda a: a) if units is None else (lambda a: a[units])
     assert gpu["len"] == ref["len"]
     for key in ("k_codes", "k_tail", "tail_mask", "v_codes", "prot_count", "prot_gstart",
-                "k_raw", "v_raw"):
+                "k_raw", "v_raw", "v_sink"):
         if key in ref:
             g = sel(gpu[key])
             assert g.shape == ref[key].shape, (key, g.shape, ref[key].shape)

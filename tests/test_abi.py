@@ -44,6 +44,9 @@ def _alloc_rc(**over):
     (dict(k_group=64, max_tokens=96), dkv.DKV_ERR_INVALID_ARG),
     (dict(B=0), dkv.DKV_ERR_INVALID_ARG),
     (dict(max_protected=-1), dkv.DKV_ERR_INVALID_ARG),
+    (dict(sink_tokens=-1), dkv.DKV_ERR_INVALID_ARG),
+    (dict(sink_tokens=257), dkv.DKV_ERR_INVALID_ARG),
+    (dict(sink_tokens=64, max_tokens=32, blk=32), dkv.DKV_ERR_INVALID_ARG),
 ])
 def test_bad_config_rejected_on_host(over, code):
     rc, msg = _alloc_rc(**over)
