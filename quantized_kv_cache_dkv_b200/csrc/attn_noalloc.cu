@@ -30,6 +30,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 extern "C" int dkv_block_attention_noalloc(dkv_cache* cache, const void* q, const void* k_act,
                                            const void* v_act, float softmax_scale, void* out,
                                            void* stream) {
+  dkv::NvtxRange nvtx_range("dkv_block_attention_noalloc");
   using dkv::report_error;
   dkv::CacheInfo ci;
   if (!dkv::cache_info(cache, &ci) || !q || !k_act || !v_act || !out)

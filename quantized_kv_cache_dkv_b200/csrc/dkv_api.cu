@@ -193,6 +193,7 @@ extern "C" {
 const char* dkv_last_error(void) { return g_err.c_str(); }
 
 int dkv_cache_alloc(const dkv_config* cfg, void* stream, dkv_cache** out) {
+  dkv::NvtxRange nvtx_range("dkv_cache_alloc");
   g_err.clear();
   if (!out) return fail(DKV_ERR_INVALID_ARG, "out is NULL");
   *out = nullptr;
@@ -301,6 +302,7 @@ int dkv_cache_alloc(const dkv_config* cfg, void* stream, dkv_cache** out) {
 }
 
 int dkv_cache_free(dkv_cache* c) {
+  dkv::NvtxRange nvtx_range("dkv_cache_free");
   g_err.clear();
   if (!c) return fail(DKV_ERR_INVALID_ARG, "cache is NULL");
   cudaError_t e = cudaDeviceSynchronize();
@@ -323,6 +325,7 @@ int dkv_cache_len(const dkv_cache* c, int64_t* len) {
 }
 
 int dkv_cache_truncate(dkv_cache* c, int64_t new_len, void* stream) {
+  dkv::NvtxRange nvtx_range("dkv_cache_truncate");
   g_err.clear();
   if (!c) return fail(DKV_ERR_INVALID_ARG, "cache is NULL");
   if (new_len < 0 || new_len > c->len || new_len % c->v.blk)
@@ -353,6 +356,7 @@ static int apply_pending_truncate(dkv_cache* c, cudaStream_t s) {
 
 int dkv_commit_block(dkv_cache* c, const void* k, const void* v, const uint32_t* protect_words,
                      void* stream) {
+  dkv::NvtxRange nvtx_range("dkv_commit_block");
   g_err.clear();
   if (!c || !k || !v) return fail(DKV_ERR_INVALID_ARG, "NULL cache, k or v");
   if (!aligned16(k) || !aligned16(v) ||
@@ -374,6 +378,7 @@ int dkv_commit_block(dkv_cache* c, const void* k, const void* v, const uint32_t*
 
 int dkv_block_attention(dkv_cache* c, const void* q, const void* k_act, const void* v_act,
                         float softmax_scale, void* out, void* stream) {
+  dkv::NvtxRange nvtx_range("dkv_block_attention");
   g_err.clear();
   if (!c || !q || !k_act || !v_act || !out) return fail(DKV_ERR_INVALID_ARG, "NULL argument");
   if (!aligned16(q) || !aligned16(k_act) || !aligned16(v_act) || !aligned16(out))
@@ -415,6 +420,7 @@ int dkv_block_attention(dkv_cache* c, const void* q, const void* k_act, const vo
 }
 
 int dkv_cache_status(dkv_cache* c, void* stream, uint32_t* flags) {
+  dkv::NvtxRange nvtx_range("dkv_cache_status");
   g_err.clear();
   if (!c || !flags) return fail(DKV_ERR_INVALID_ARG, "NULL argument");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -425,6 +431,7 @@ int dkv_cache_status(dkv_cache* c, void* stream, uint32_t* flags) {
 }
 
 int dkv_cache_export(dkv_cache* c, void* stream, dkv_export* o) {
+  dkv::NvtxRange nvtx_range("dkv_cache_export");
   g_err.clear();
   if (!c || !o) return fail(DKV_ERR_INVALID_ARG, "NULL argument");
   const dkv::CacheView& v = c->v;

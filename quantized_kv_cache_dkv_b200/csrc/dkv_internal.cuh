@@ -8,7 +8,19 @@
 
 #include "dkv.h"
 
+#include <nvtx3/nvToolsExt.h>
+
 namespace dkv {
+
+// Host-side NVTX range around one library call (header-only NVTX: it costs a
+// few nanoseconds unless a profiler is attached, which then shows each call
+// on the timeline).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 constexpr int kHeadDim = 128;
 constexpr int kChunk = 32;  // token granularity of every segment boundary
