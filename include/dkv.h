@@ -60,9 +60,13 @@ enum {
   DKV_FLAG_CAPACITY = 0x1, /* side table full: later protected tokens were quantized normally */
   DKV_FLAG_RANGE = 0x2,    /* a committed K/V value was NaN/Inf or |x| > 65504; the
                               quantizer used NaN -> 0 and clamped to +-65504 */
-  DKV_FLAG_TIMEOUT = 0x4   /* an attention CTA gave up waiting on one of its own
+  DKV_FLAG_TIMEOUT = 0x4,  /* an attention CTA gave up waiting on one of its own
                               pipeline stages (bounded wait, about 1 s); that call's
                               output is undefined */
+  DKV_FLAG_BOUNDS = 0x8    /* bounds-checking build only (libdkv_bc.so, compiled
+                              with DKV_BOUNDS_CHECK): an index or copy range failed
+                              its check against its buffer and the access was
+                              skipped; that call's results are undefined */
 };
 
 /* Cache shape.  Supported: head_dim == 128; block a multiple of 32, <= 128;

@@ -13,7 +13,9 @@ import re
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libdkv.so")
+# DKV_LIB selects another build of the library (the bounds-checking
+# libdkv_bc.so, for tests); the default is the in-tree libdkv.so
+LIB_PATH = os.environ.get("DKV_LIB") or os.path.join(_HERE, "libdkv.so")
 HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "dkv.h")
 
 if not os.path.exists(LIB_PATH):
@@ -24,7 +26,7 @@ if not os.path.exists(LIB_PATH):
 _lib = ctypes.CDLL(LIB_PATH)
 
 DKV_OK, DKV_ERR_INVALID_ARG, DKV_ERR_UNSUPPORTED, DKV_ERR_CAPACITY, DKV_ERR_CUDA = 0, 1, 2, 3, 4
-DKV_FLAG_CAPACITY, DKV_FLAG_RANGE, DKV_FLAG_TIMEOUT = 0x1, 0x2, 0x4
+DKV_FLAG_CAPACITY, DKV_FLAG_RANGE, DKV_FLAG_TIMEOUT, DKV_FLAG_BOUNDS = 0x1, 0x2, 0x4, 0x8
 DKV_OPT_SPLITS, DKV_OPT_ATTN_KERNEL, DKV_OPT_PROFILE = 1, 2, 3
 DKV_KERNEL_ATTENTION, DKV_KERNEL_COMBINE, DKV_KERNEL_COMMIT, DKV_KERNEL_TRUNCATE = 0, 1, 2, 3
 

@@ -1,10 +1,13 @@
 """Build libdkv.so in-tree for sm_100a with nvcc.
 
-    python quantized_kv_cache_dkv_b200/build.py [--force] [-v]
+    python quantized_kv_cache_dkv_b200/build.py [--force] [-v] [--bounds-check]
 
 Objects go to quantized_kv_cache_dkv_b200/_build/, the library to
-quantized_kv_cache_dkv_b200/libdkv.so.  A source is recompiled when it or any
-header is newer than its object.
+quantized_kv_cache_dkv_b200/libdkv.so.  --bounds-check builds the
+bounds-checking variant instead (DKV_BOUNDS_CHECK: kernels check their index
+arithmetic and copy ranges, record DKV_FLAG_BOUNDS and skip the access) into
+_build_bc/ and libdkv_bc.so.  A source is recompiled when it or any header is
+newer than its object.
 """
 from __future__ import annotations
 
@@ -20,6 +23,8 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libdkv.so")
+BUILD_BC = os.path.join(HERE, "_build_bc")
+LIB_BC = os.path.join(HERE, "libdkv_bc.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2",
@@ -40,8 +45,9 @@ def _headers_mtime() -> float:
     return max((os.path.getmtime(h) for h in hs), default=0.0)
 
 
-def _compile(src: str, obj: str, verbose: bool) -> None:
-    cmd = [nvcc(), *ARCH, *COMMON, *PER_FILE.get(os.path.basename(src), []), "-c", src, "-o", obj]
+def _compile(src: str, obj: str, verbose: bool, extra=()) -> None:
+    cmd = [nvcc(), *ARCH, *COMMON, *PER_FILE.get(os.path.basename(src), []), *extra, "-c", src,
+           "-o", obj]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd), flush=True)
@@ -53,30 +59,32 @@ def _compile(src: str, obj: str, verbose: bool) -> None:
         raise RuntimeError(f"nvcc failed on {os.path.basename(src)}")
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, bounds_check: bool = False) -> str:
+    build_dir, lib = (BUILD_BC, LIB_BC) if bounds_check else (BUILD, LIB)
+    extra = ["-DDKV_BOUNDS_CHECK"] if bounds_check else []
+    os.makedirs(build_dir, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     hdr_t = _headers_mtime()
     jobs = []
     objs = []
     for s in srcs:
-        o = os.path.join(BUILD, os.path.basename(s)[:-3] + ".o")
+        o = os.path.join(build_dir, os.path.basename(s)[:-3] + ".o")
         objs.append(o)
         if force or not os.path.exists(o) or os.path.getmtime(o) < max(os.path.getmtime(s), hdr_t):
             jobs.append((s, o))
     if jobs:
         with concurrent.futures.ThreadPoolExecutor(max_workers=min(8, len(jobs))) as ex:
-            for f in [ex.submit(_compile, s, o, verbose) for s, o in jobs]:
+            for f in [ex.submit(_compile, s, o, verbose, extra) for s, o in jobs]:
                 f.result()
-    if jobs or not os.path.exists(LIB) or os.path.getmtime(LIB) < max(os.path.getmtime(o) for o in objs):
-        cmd = [nvcc(), *ARCH, "-shared", "-o", LIB, *objs, "-lcuda"]
+    if jobs or not os.path.exists(lib) or os.path.getmtime(lib) < max(os.path.getmtime(o) for o in objs):
+        cmd = [nvcc(), *ARCH, "-shared", "-o", lib, *objs, "-lcuda"]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode:
             sys.stderr.write(r.stdout + r.stderr)
-            raise RuntimeError("link of libdkv.so failed")
-    return LIB
+            raise RuntimeError(f"link of {os.path.basename(lib)} failed")
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose="-v" in sys.argv)
-    print(LIB)
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv,
+                bounds_check="--bounds-check" in sys.argv))

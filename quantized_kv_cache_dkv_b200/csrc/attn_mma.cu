@@ -68,12 +68,23 @@ __device__ __forceinline__ void fill_chunk(const AttnArgs& a, int u, int64_t pos
   } else {
     kind = SEG_ZERO;
   }
+  // bounds-checking build: the chunk lies inside the segment it reads (a
+  // chunk that does not is filled with zeros)
+  if (!DKV_IN_BOUNDS(pos0 >= 0 && (kind == SEG_ZERO ||
+                                   (kind == SEG_CODES ? pos0 + kChunk <= a.Lq && a.Lq <= c.cap &&
+                                                            a.Lq % c.GK == 0
+                                    : pos0 < a.Lq    ? pos0 + kChunk <= c.cap
+                                    : pos0 < a.L     ? pos0 + kChunk - a.Lq <= c.GK
+                                                     : pos0 + kChunk - a.L <= c.blk)),
+                     c.status))
+    kind = SEG_ZERO;
   if (kind == SEG_CODES) {
     if constexpr (KB < 16) {
       const int64_t j = pos0 / c.GK;
       const int o = int(pos0 % c.GK);
-      const int g0 = c.prot_gstart[size_t(u) * (c.nG + 1) + j];
-      const int g1 = c.prot_gstart[size_t(u) * (c.nG + 1) + j + 1];
+      int g0 = c.prot_gstart[size_t(u) * (c.nG + 1) + j];
+      int g1 = c.prot_gstart[size_t(u) * (c.nG + 1) + j + 1];
+      if (!DKV_IN_BOUNDS(g0 >= 0 && g0 <= g1 && g1 <= c.P, c.status)) g0 = g1 = 0;
       for (int cc = tid; cc < d; cc += nthr) {
         const size_t base = ((size_t(u) * c.nG + j) * d + cc) * c.kw + size_t(o) * KB / 32;
         const __half2 sz = c.k_sz[(size_t(u) * c.nG + j) * d + cc];
@@ -135,6 +146,11 @@ __device__ __forceinline__ void fill_chunk(const AttnArgs& a, int u, int64_t pos
   } else {
     kind = SEG_ZERO;
   }
+  if (!DKV_IN_BOUNDS(kind == SEG_ZERO ||
+                         (pos0 < a.L ? pos0 + kChunk <= a.L && a.L <= c.cap
+                                     : pos0 + kChunk - a.L <= c.blk),
+                     c.status))
+    kind = SEG_ZERO;
   if (kind == SEG_CODES) {
     if constexpr (VB < 16) {
       // item = (token t, quarter q of 32 channels)
@@ -145,7 +161,8 @@ __device__ __forceinline__ void fill_chunk(const AttnArgs& a, int u, int64_t pos
         const __half2 s2 = __half2half2(__low2half(sz));
         const __half2 z2 = __half2half2(__high2half(sz));
         uint4* dst = reinterpret_cast<uint4*>(Vt + (ch * 32 + t) * VT_LD + q * 32);
-        if (pos0 + t < c.sink) {  // sink position: its bf16 V row
+        if (pos0 + t < c.sink && DKV_IN_BOUNDS(c.sink <= c.cap, c.status)) {
+          // sink position: its bf16 V row
           const uint4* src = reinterpret_cast<const uint4*>(
               c.v_sink + (size_t(u) * c.sink + size_t(pos0 + t)) * d + q * 32);
 #pragma unroll

@@ -415,9 +415,13 @@ __device__ __forceinline__ void fill_k_tile(const AttnArgs& a, int u, int64_t ti
       const uint16_t* rpk = reinterpret_cast<const uint16_t*>(rs + Smem::kRPk);
 #pragma unroll 1
       for (int i = 0; i < n; ++i) {
+        if (!DKV_IN_BOUNDS(i < kStagedProt ? g0 + i - pbase >= 0 && g0 + i - pbase < 32
+                                           : g0 + i < cv.P, cv.status))
+          break;
         const int pos = i < kStagedProt ? rpos[g0 + i - pbase]
                                         : __ldg(cv.prot_pos + size_t(u) * cv.P + g0 + i);
         const int t = int(pos - tile_start);
+        if (!DKV_IN_BOUNDS(t >= 0 && t < TT, cv.status)) continue;
         if ((t >> 6) != qh) continue;
         const uint16_t kv = i < kStagedProt
                                 ? rpk[i * d + c]
@@ -498,6 +502,9 @@ __device__ __noinline__ void fill_k_general(const AttnArgs& a, int u, int64_t ti
         const int* rpos = reinterpret_cast<const int*>(rs + Smem::kRPos);
         const uint16_t* rpk = reinterpret_cast<const uint16_t*>(rs + Smem::kRPk);
         for (int i = 0; i < n; ++i) {
+          if (!DKV_IN_BOUNDS(i < kStagedProt ? g0 + i - pbase >= 0 && g0 + i - pbase < 32
+                                             : g0 + i < cv.P, cv.status))
+            break;
           const int pos = i < kStagedProt ? rpos[g0 + i - pbase]
                                           : __ldg(cv.prot_pos + size_t(u) * cv.P + g0 + i);
           if (pos >= pos0 && pos < pos0 + 32) {
@@ -1051,12 +1058,37 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           vc_b = nv * uint32_t(cv.vw) * 4u;
           vsz_b = nv * uint32_t(cv.vgroups) * 4u;
         }
+        const size_t ug = size_t(u) * size_t(cv.nG) + size_t(g_lo);
+        {
+          // bounds-checking build: each copy inside its buffer and its ring
+          // slot, else left out (the staged side table with it); the byte
+          // counts stay consistent with the expect_tx below
+          const size_t U = size_t(cv.U), P = size_t(cv.P), e = size_t(u) * P;
+          if (kc_b && !DKV_IN_BOUNDS(
+                          kc_b <= Smem::kRKsz - Smem::kRKc && ksz_b <= Smem::kRVc - Smem::kRKsz &&
+                          (ug * kHeadDim * cv.kw) * 4 + kc_b <= U * cv.nG * kHeadDim * cv.kw * 4 &&
+                          (ug * kHeadDim) * 4 + ksz_b <= U * cv.nG * kHeadDim * 4, cv.status))
+            kc_b = ksz_b = pos_b = pk_b = 0;
+          // (the staged positions are a 16-byte aligned superset: up to three
+          // entries past the unit's, inside the arena)
+          if (pos_b && !DKV_IN_BOUNDS(
+                           g0 >= 0 && pidx0 >= 0 && pos_b <= Smem::kRPk - Smem::kRPos &&
+                           pk_b <= Smem::kStageBytes - Smem::kRPk &&
+                           (e + size_t(pidx0)) * 4 + pos_b <= (U * P + 3) * 4 &&
+                           (e + size_t(g0)) * kHeadDim * 2 + pk_b <= U * P * kHeadDim * 2, cv.status))
+            pos_b = pk_b = 0;
+          const size_t ut = size_t(u) * size_t(cv.cap) + size_t(ts);
+          if (vc_b && !DKV_IN_BOUNDS(
+                          vc_b <= Smem::kRVsz - Smem::kRVc && vsz_b <= Smem::kRHdr - Smem::kRVsz &&
+                          ut * cv.vw * 4 + vc_b <= U * size_t(cv.cap) * cv.vw * 4 &&
+                          ut * cv.vgroups * 4 + vsz_b <= U * size_t(cv.cap) * cv.vgroups * 4, cv.status))
+            vc_b = vsz_b = 0;
+        }
         int* hdr = reinterpret_cast<int*>(sm + Smem::kRing + st * Smem::kStageBytes + Smem::kRHdr);
-        hdr[0] = kc_b ? n : 0;
+        hdr[0] = pos_b ? n : 0;  // pos_b is set exactly when the tile has protected rows
         hdr[1] = g0;
         hdr[2] = pidx0;
         mbar_arrive_expect_tx(bar(RFULL + st), kc_b + ksz_b + vc_b + vsz_b + pos_b + pk_b);
-        const size_t ug = size_t(u) * size_t(cv.nG) + size_t(g_lo);
         if (kc_b) {
           bulk_g2s(dst + Smem::kRKc, cv.k_codes + ug * kHeadDim * cv.kw, kc_b, bar(RFULL + st));
           bulk_g2s(dst + Smem::kRKsz, cv.k_sz + ug * kHeadDim, ksz_b, bar(RFULL + st));

@@ -202,6 +202,15 @@ commit_kernel(CacheView c, const uint16_t* __restrict__ k, const uint16_t* __res
   const int GK = c.GK;
   const int n_tail = KB < 16 ? int(p0 % GK) : 0;
   const bool completes = KB < 16 && n_tail + blk >= GK;
+  // bounds-checking build: the block lands inside the unit's capacity, an
+  // incomplete group stays inside the tail, the completed groups inside the
+  // group arrays (the condition is the same for every thread of the block)
+  if (!DKV_IN_BOUNDS(p0 >= 0 && p0 + blk <= c.cap && blk % 32 == 0 &&
+                         (KB == 16 || (completes ? (p0 + blk) / GK <= c.nG && (n_tail + blk) % GK == 0
+                                                 : n_tail + blk <= GK)) &&
+                         (VB == 16 || c.sink <= c.cap),
+                     c.status))
+    return;
 
   // a roll-back to p0 (a multiple of the K group) recorded since the last
   // commit: the side table keeps the entries of the groups before p0, the
@@ -325,6 +334,7 @@ commit_kernel(CacheView c, const uint16_t* __restrict__ k, const uint16_t* __res
             const int b = __ffs(m) - 1;
             m &= m - 1u;
             const int t = w * 32 + b;
+            if (!DKV_IN_BOUNDS(count < c.P, c.status)) break;
             if (tid == 0) c.prot_pos[size_t(u) * c.P + count] = int32_t(j * GK + t);
             c.prot_k[(size_t(u) * c.P + count) * d + ch] = sk[(gi * GK + t) * kRowPad + ch];
             ++count;

@@ -12,6 +12,17 @@
 
 namespace dkv {
 
+// Bounds checks of the bounds-checking build (DKV_BOUNDS_CHECK, built as
+// libdkv_bc.so): DKV_IN_BOUNDS(cond, status) is `cond`, and records
+// DKV_FLAG_BOUNDS in the sticky status when it fails, so the caller can skip
+// the access.  In the normal build it is `true` and costs nothing.
+#ifdef DKV_BOUNDS_CHECK
+#define DKV_IN_BOUNDS(cond, status) \
+  ((cond) ? true : (atomicOr((status), uint32_t(DKV_FLAG_BOUNDS)), false))
+#else
+#define DKV_IN_BOUNDS(cond, status) true
+#endif
+
 // Host-side NVTX range around one library call (header-only NVTX: it costs a
 // few nanoseconds unless a profiler is attached, which then shows each call
 // on the timeline).

@@ -9,17 +9,30 @@ import pytest
 import quantized_kv_cache_dkv_b200 as dkv
 
 
-def test_library_exports_every_header_symbol():
+def _check_exports(path):
     names = dkv.header_symbols()
     assert "dkv_commit_block" in names and "dkv_block_attention" in names
-    out = subprocess.run(["nm", "-D", "--defined-only", dkv.LIB_PATH], capture_output=True,
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True,
                          text=True, check=True).stdout
     exported = {ln.split()[-1] for ln in out.splitlines() if ln.strip()}
     missing = [n for n in names if n not in exported]
     assert not missing, missing
-    lib = ctypes.CDLL(dkv.LIB_PATH)
+    lib = ctypes.CDLL(path)
     for n in names:
         assert getattr(lib, n) is not None
+
+
+def test_library_exports_every_header_symbol():
+    _check_exports(dkv.LIB_PATH)
+
+
+def test_bounds_checking_library_exports_every_header_symbol():
+    """libdkv_bc.so (the DKV_BOUNDS_CHECK build) has the same boundary."""
+    import os
+    path = os.path.join(os.path.dirname(dkv.__file__), "libdkv_bc.so")
+    if not os.path.exists(path):
+        pytest.skip("libdkv_bc.so not built (build.py --bounds-check)")
+    _check_exports(path)
 
 
 def _alloc_rc(**over):
