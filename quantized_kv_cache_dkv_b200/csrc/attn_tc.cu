@@ -1070,9 +1070,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                           (ug * kHeadDim) * 4 + ksz_b <= U * cv.nG * kHeadDim * 4, cv.status))
             kc_b = ksz_b = pos_b = pk_b = 0;
           // (the staged positions are a 16-byte aligned superset: up to three
-          // entries past the unit's, inside the arena)
+          // entries before and after the unit's slice, inside the arena)
           if (pos_b && !DKV_IN_BOUNDS(
-                           g0 >= 0 && pidx0 >= 0 && pos_b <= Smem::kRPk - Smem::kRPos &&
+                           g0 >= 0 && int64_t(e) + pidx0 >= 0 &&
+                           pos_b <= Smem::kRPk - Smem::kRPos &&
                            pk_b <= Smem::kStageBytes - Smem::kRPk &&
                            (e + size_t(pidx0)) * 4 + pos_b <= (U * P + 3) * 4 &&
                            (e + size_t(g0)) * kHeadDim * 2 + pk_b <= U * P * kHeadDim * 2, cv.status))
