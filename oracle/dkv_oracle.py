@@ -41,6 +41,8 @@ from __future__ import annotations
 
 import numpy as np
 
+from . import krpbh
+
 FLAG_CAPACITY = 0x1   # protected side table full: extra protected tokens quantized normally
 FLAG_RANGE = 0x2      # a committed K/V value was non-finite or beyond fp16 range
 
@@ -174,7 +176,7 @@ class OracleCache:
     """
 
     def __init__(self, B, Hq, Hkv, d, blk, k_bits, v_bits, k_group, v_group,
-                 max_protected, capacity, sink_tokens=0):
+                 max_protected, capacity, sink_tokens=0, v_rotation=None):
         assert Hq % Hkv == 0
         assert k_bits in (2, 4, 16) and v_bits in (2, 4, 16)
         assert capacity % k_group == 0 and capacity % blk == 0
@@ -211,6 +213,16 @@ class OracleCache:
         assert 0 <= sink_tokens <= capacity
         self.sink = int(sink_tokens)
         self.v_sink = np.zeros((U, self.sink, d), np.uint16)
+        # Rotated V (K-RPBH, oracle/krpbh.py): (perm, mix, b) or None.  V rows
+        # are quantized in the rotated basis; the active block's V enters the
+        # attention rotated too (fp32 rotation rounded to bf16), and the
+        # output is rotated back.  Needs quantized V and no sink.
+        self.v_rot = None
+        if v_rotation is not None:
+            perm, mix, b = v_rotation
+            assert v_bits < 16 and self.sink == 0
+            krpbh.check_params(perm, mix, b, d)
+            self.v_rot = (np.asarray(perm, np.int64), np.asarray(mix, np.float32), int(b))
 
     # -- derived sizes
     @property
@@ -263,6 +275,10 @@ class OracleCache:
             self.v_raw[u, p0:p0 + blk] = vbits
             return flag
         x, _ = sanitize(x)
+        if self.v_rot is not None:
+            x = krpbh.rotate_f32(x, *self.v_rot)
+            flag |= FLAG_RANGE if (~np.isfinite(x) | (np.abs(x) > FP16_MAX)).any() else 0
+            x, _ = sanitize(x)
         # per token, one group per GV consecutive channels
         groups = x.reshape(blk * (d // GV), GV)
         q, s, z = quantize_groups(groups, np.ones_like(groups, bool), vb)
@@ -376,7 +392,10 @@ class OracleCache:
         g = Hq // Hkv
         Q = bf16_to_f64(np.asarray(Q_bits).reshape(B, Hq, blk, d))
         Ka = bf16_to_f64(np.asarray(Kact_bits).reshape(B, Hkv, blk, d))
-        Va = bf16_to_f64(np.asarray(Vact_bits).reshape(B, Hkv, blk, d))
+        Va_bits = np.asarray(Vact_bits, np.uint16).reshape(B, Hkv, blk, d)
+        if self.v_rot is not None:
+            Va_bits = krpbh.f32_to_bf16_bits(krpbh.rotate_f32(bf16_to_f32(Va_bits), *self.v_rot))
+        Va = bf16_to_f64(Va_bits)
         O = np.zeros((B, Hq, blk, d), np.float64)
         for b in range(B):
             for h in range(Hkv):
@@ -385,6 +404,9 @@ class OracleCache:
                 Vall = np.concatenate([self.dequant_v(u), Va[b, h]])
                 for hq in range(h * g, (h + 1) * g):
                     O[b, hq] = dense_attention_f64(Q[b, hq], Kall, Vall, scale)
+        if self.v_rot is not None:
+            perm, mix, rb = self.v_rot
+            O = krpbh.unrotate_f64(O, perm, mix.astype(np.float64), rb)
         return O
 
     # -- canonical snapshot of the committed state (what an export returns)

@@ -32,6 +32,7 @@ _TAG_PROT_PREFILL = 4
 _TAG_PROT_LATE = 5
 _TAG_ACTIVE = 6
 _TAG_GRID = 7
+_TAG_ROTATION = 8
 
 
 @dataclass(frozen=True)
@@ -281,3 +282,16 @@ def shrink(w: Workload, **kw) -> Workload:
     """A smaller case of the same recipe (for tests the oracle finishes in
     seconds): overrides sizes, keeps the distributions."""
     return w.with_(**kw)
+
+
+def krpbh_params(seed: int, b: int, d: int = 128):
+    """Random draws of a K-RPBH rotation with blocks of b coordinates: a
+    permutation of [0, d) (int32) and a Haar-random (d/b) x (d/b) orthogonal
+    mix (QR of a Gaussian matrix, column signs fixed by R's diagonal),
+    rounded to fp32 -- the form the library takes them in."""
+    k = d // b
+    r = _rng(seed, _TAG_ROTATION, b)
+    perm = r.permutation(d).astype(np.int32)
+    q, rr = np.linalg.qr(r.standard_normal((k, k)))
+    mix = (q * np.sign(np.diag(rr))[None, :]).astype(np.float32)
+    return perm, mix
