@@ -210,7 +210,8 @@ def whole_job_gbs(bytes_per_rank: float, max_ms: float, world: int) -> float:
     return world * bytes_per_rank / (max_ms / 1e3) / 1e9
 
 
-def run_gpu(w: synth.Workload, K: int, W: int, want_e2e=True, log=print, kernel=0):
+def run_gpu(w: synth.Workload, K: int, W: int, want_e2e=True, log=print, kernel=0,
+            v_rotation=0):
     import torch
     import quantized_kv_cache_dkv_b200 as dkv
 
@@ -228,6 +229,10 @@ def run_gpu(w: synth.Workload, K: int, W: int, want_e2e=True, log=print, kernel=
     cfg = dkv.make_config(w.B, w.Hq, w.Hkv, w.d, w.blk, w.k_bits, w.v_bits, w.k_group,
                           w.v_group, P, cap)
     caches = [dkv.dkv_cache_alloc(cfg) for _ in range(R)]
+    if v_rotation:
+        perm, mix = synth.krpbh_params(w.seed, v_rotation)
+        for c in caches:
+            dkv.dkv_cache_set_v_rotation(c, perm, mix, v_rotation)
     if kernel:
         for c in caches:
             dkv.dkv_cache_set_option(c, dkv.DKV_OPT_ATTN_KERNEL, kernel)
@@ -621,6 +626,8 @@ def main():
                     help="attention kernel: 0 = library's choice, 1 = mma.sync, 2 = tcgen05")
     ap.add_argument("--B", type=int, default=0, help="override the workload's batch (profiling)")
     ap.add_argument("--L", type=int, default=0, help="override the committed length (profiling)")
+    ap.add_argument("--v-rotation", type=int, default=0, choices=[0, 16, 32, 64, 128],
+                    help="K-RPBH rotation of V with this Hadamard block (0 = none)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -657,8 +664,11 @@ def main():
                                 device_id=torch.device("cuda", local))
     peaks, peak_kind = load_peaks()
     traffic = traffic_record()
-    r = run_gpu(w, args.steps, args.warmup, log=lambda *a: None, kernel=args.kernel)
+    r = run_gpu(w, args.steps, args.warmup, log=lambda *a: None, kernel=args.kernel,
+                v_rotation=args.v_rotation)
     line = base_line(w, args, r["value"], r["ms"] / args.steps, world)
+    if args.v_rotation:
+        line["config"]["v_rotation"] = f"K-RPBH, Hadamard block {args.v_rotation}"
     line["config"]["L2_policy"] = (f"{r['R']} cache replicas used round-robin"
                                    if r["R"] > 1 else "cache larger than L2")
     line["config"]["L_mean"] = r["L_mean"]
@@ -694,7 +704,7 @@ def main():
                 "commit_tokens_per_s": round(ww.B * ww.blk * rr["commit_n"] /
                                              (rr["commit_ms"] / 1e3), 1),
                 "plan": rr["plan"], "clocks_sm_mhz": (rr["clocks"] or {}).get("sm_mhz")}
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.v_rotation:
         gbs, steps, el, desc = oracle_sample(w, args.cpu_seconds)
         line["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": _blas_threads(),
                                 "kind": "oracle", "sample": desc}

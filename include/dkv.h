@@ -125,6 +125,34 @@ int dkv_block_attention(dkv_cache* cache, const void* q, const void* k_act,
                         const void* v_act, float softmax_scale, void* out,
                         void* stream);
 
+/* Rotated V (K-RPBH, "SoloQ: Calibration-Free Quantization for Diffusion
+ * Language Models", K-RPBH paragraph and the KV-cache paragraph): committed V
+ * rows are rotated by an orthogonal map R before their per-token
+ * quantization, the active block's V is rotated the same way (and rounded to
+ * bf16), and the attention output is rotated back, so the result is still
+ * softmax(...) V in the original basis; only the quantization error changes.
+ * For a row x of d = 128 channels and blocks of b channels (k = d / b):
+ *   y[i] = x[perm[i]];  each block of y <- (block) H_b / sqrt(b) with H_b the
+ *   Sylvester Hadamard matrix;  w[r*b + i] = sum_c mix[r*k + c] * y[c*b + i].
+ * Evaluated in fp32 in a fixed order (butterflies over strides 1, 2, ...,
+ * b/2; one multiply by fp32(1/sqrt(b)); the mix summed over c = 0..k-1 from
+ * 0; no fused multiply-add), so the stored codes are reproducible bit for bit.
+ *   perm  host int32 [128], a permutation of 0..127 (the caller's random draw)
+ *   mix   host fp32 [k * k], row-major, orthogonal (|mix mix^T - I| <= 1e-4)
+ *   block b in {16, 32, 64, 128}; block = 0 (perm, mix NULL) turns it off.
+ * Call before the first commit (len == 0) of a cache with v_bits < 16 and
+ * sink_tokens == 0.  The library copies the arguments (synchronously) and
+ * allocates a [B, Hkv, block, d] bf16 buffer for the rotated active block,
+ * so two attention calls on one handle must not overlap on the GPU.  Each
+ * attention call then also launches a small rotation kernel and always the
+ * combine kernel (which applies the inverse rotation in fp32).
+ * Errors: DKV_ERR_INVALID_ARG (len > 0, NULL or non-permutation perm, NULL,
+ * non-finite or non-orthogonal mix), DKV_ERR_UNSUPPORTED (block not in the
+ * set, v_bits == 16, sink_tokens > 0), DKV_ERR_CUDA; nothing changes on an
+ * error. */
+int dkv_cache_set_v_rotation(dkv_cache* cache, const int32_t* perm, const float* mix,
+                             int32_t block);
+
 /* Roll the cache back to its first new_len committed tokens (for instance to
  * reuse a shared prefix, the prefix-cache reuse of the Tai et al. abstract).
  * new_len must be a multiple of `block` and, when k_bits < 16, of k_group, so

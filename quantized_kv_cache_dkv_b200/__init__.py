@@ -76,6 +76,7 @@ _truncate = _sig("dkv_cache_truncate", [_P, ctypes.c_int64, _P])
 _status = _sig("dkv_cache_status", [_P, _P, ctypes.POINTER(ctypes.c_uint32)])
 _export = _sig("dkv_cache_export", [_P, _P, ctypes.POINTER(dkv_export)])
 _setopt = _sig("dkv_cache_set_option", [_P, ctypes.c_int32, ctypes.c_int64])
+_setrot = _sig("dkv_cache_set_v_rotation", [_P, _P, _P, ctypes.c_int32])
 _prof = _sig("dkv_profile_read", [_P, ctypes.c_int32, ctypes.POINTER(ctypes.c_double),
                                   ctypes.POINTER(ctypes.c_int64)])
 _plan = _sig("dkv_last_attention_plan", [_P, ctypes.POINTER(ctypes.c_int32),
@@ -200,6 +201,21 @@ def dkv_block_attention_noalloc(cache: Cache, q, k_act, v_act, softmax_scale: fl
 
 def dkv_cache_truncate(cache: Cache, new_len: int, stream=None) -> None:
     _check(_truncate(cache.h, new_len, _stream(stream)))
+
+
+def dkv_cache_set_v_rotation(cache: Cache, perm=None, mix=None, block: int = 0) -> None:
+    """K-RPBH rotation of V (before the first commit): perm int32 [128], a
+    permutation; mix float32 [k, k] orthogonal, k = 128 / block; block in
+    {16, 32, 64, 128}, or 0 (perm, mix None) to turn the rotation off."""
+    import numpy as np
+    if block == 0:
+        _check(_setrot(cache.h, None, None, 0))
+        return
+    p = np.ascontiguousarray(perm, dtype=np.int32)
+    m = np.ascontiguousarray(mix, dtype=np.float32)
+    if p.shape != (128,) or m.shape != (128 // block, 128 // block):
+        raise ValueError(f"perm must be [128] and mix [{128 // block}, {128 // block}]")
+    _check(_setrot(cache.h, p.ctypes.data_as(_P), m.ctypes.data_as(_P), int(block)))
 
 
 def dkv_cache_len(cache: Cache) -> int:

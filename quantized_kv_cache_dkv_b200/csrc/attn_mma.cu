@@ -331,7 +331,7 @@ attn_mma_kernel(AttnArgs a) {
   l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
   l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
 
-  if (a.nsplit == 1) {
+  if (a.final_out) {
     const float i0 = 1.f / l0, i1 = 1.f / l1;
     uint16_t* out0 = a.out + (size_t(u) * c.rows + r0) * kHeadDim;
     uint16_t* out1 = out0 + 8 * kHeadDim;
@@ -360,8 +360,51 @@ attn_mma_kernel(AttnArgs a) {
   }
 }
 
+// Inverse K-RPBH rotation of one output row held by a warp (lane: channels
+// 4 lane .. 4 lane + 3): mix^T across the k blocks, the per-block Hadamard
+// (butterflies, then 1/sqrt(b)), the inverse permutation (through `buf`, 128
+// floats of this warp's shared memory).  The attention of a rotated-V cache
+// sums rotated rows, so its output is the rotated output.
+__device__ __forceinline__ void unrotate_row(float (&x)[4], int b, float norm,
+                                          const int32_t* __restrict__ perm,
+                                          const float* __restrict__ mix, float* buf, int lane) {
+  const int k = kHeadDim / b, lb = b / 4;  // lanes per block
+  const int i_lane = lane % lb, r = lane / lb;           // this lane's block r
+  float y[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int rr = 0; rr < k; ++rr) {
+    const float m = __ldg(mix + rr * k + r);     // mix[rr][r]: y_r = sum_rr mix[rr][r] w_rr
+#pragma unroll
+    for (int e = 0; e < 4; ++e) y[e] += m * __shfl_sync(0xffffffffu, x[e], rr * lb + i_lane);
+  }
+#pragma unroll
+  for (int h = 1; h <= 2; h <<= 1) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (e & h) continue;
+      const float lo = y[e], hi = y[e + h];
+      y[e] = lo + hi;
+      y[e + h] = lo - hi;
+    }
+  }
+  for (int h = 4; h < b; h <<= 1) {
+    const bool upper = (lane & (h >> 2)) != 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float p = __shfl_xor_sync(0xffffffffu, y[e], h >> 2);
+      y[e] = upper ? p - y[e] : y[e] + p;
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 4; ++e) buf[__ldg(perm + 4 * lane + e)] = y[e] * norm;
+  __syncwarp();
+#pragma unroll
+  for (int e = 0; e < 4; ++e) x[e] = buf[4 * lane + e];
+}
+
 // One warp per (unit, row): out = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s
+// (rotated back first when V is stored rotated)
 __global__ void __launch_bounds__(128) combine_kernel(AttnArgs a) {
+  __shared__ float rbuf[4][kHeadDim];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t row = int64_t(blockIdx.x) * 4 + warp;
   const int rows = a.c.rows;
@@ -384,8 +427,11 @@ __global__ void __launch_bounds__(128) combine_kernel(AttnArgs a) {
     acc.w += w * x.w;
   }
   const float inv = 1.f / lsum;
-  const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
-  const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+  float x[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
+  if (a.c.vrot_b)
+    unrotate_row(x, a.c.vrot_b, a.c.vrot_norm, a.c.vrot_perm, a.c.vrot_mix, rbuf[warp], lane);
+  const __nv_bfloat162 lo = __floats2bfloat162_rn(x[0], x[1]);
+  const __nv_bfloat162 hi = __floats2bfloat162_rn(x[2], x[3]);
   uint2 pk;
   pk.x = *reinterpret_cast<const uint32_t*>(&lo);
   pk.y = *reinterpret_cast<const uint32_t*>(&hi);

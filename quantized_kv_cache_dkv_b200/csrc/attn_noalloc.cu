@@ -74,7 +74,7 @@ extern "C" int dkv_block_attention_noalloc(dkv_cache* cache, const void* q, cons
   const int prc = dkv::plan_attention(ci, &a, &kernel, &perr);
   if (prc != DKV_OK) return report_error(prc, perr);
 
-  if (a.nsplit > 1) {
+  if (!a.final_out) {
     const size_t rows_total = size_t(v.U) * size_t(a.nsplit) * size_t(v.rows);
     const size_t o_bytes = align256(rows_total * size_t(dkv::kHeadDim) * sizeof(float));
     const size_t need = o_bytes + rows_total * sizeof(float2);
@@ -89,10 +89,17 @@ extern "C" int dkv_block_attention_noalloc(dkv_cache* cache, const void* q, cons
   }
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (v.vrot_b) {
+    // the active block's V into the cache's rotated basis (cache-owned buffer)
+    e = dkv::launch_rotate_v_rows(v, a.v_act, ci.vrot_act, s);
+    if (e != cudaSuccess)
+      return report_error(DKV_ERR_CUDA, (std::string("rotation launch: ") + cudaGetErrorString(e)).c_str());
+    a.v_act = ci.vrot_act;
+  }
   e = kernel == 2 ? dkv::launch_attention_tc(a, s) : dkv::launch_attention_mma(a, s);
   if (e != cudaSuccess)
     return report_error(DKV_ERR_CUDA, (std::string("attention launch: ") + cudaGetErrorString(e)).c_str());
-  if (a.nsplit > 1) {
+  if (!a.final_out) {
     e = dkv::launch_combine(a, s);
     if (e != cudaSuccess)
       return report_error(DKV_ERR_CUDA, (std::string("combine launch: ") + cudaGetErrorString(e)).c_str());

@@ -935,7 +935,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         const int col = 64 * h + 32 * ch;
         if (!row_ok) {
           // padding row: nothing to write
-        } else if (a.nsplit == 1) {
+        } else if (a.final_out) {
           uint4* dst = reinterpret_cast<uint4*>(a.out + (size_t(u) * cv.rows + r) * kHeadDim + col);
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
@@ -959,7 +959,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                                  __uint_as_float(o[kpos<VB>(4 * i + 2)]), __uint_as_float(o[kpos<VB>(4 * i + 3)]));
         }
       }
-      if (a.nsplit > 1 && row_ok && h == 0)
+      if (!a.final_out && row_ok && h == 0)
         a.part_ml[(size_t(u) * a.nsplit + sp) * cv.rows + r] = make_float2(rf, lt);
     }
   } else if (warp < 24) {

@@ -136,6 +136,79 @@ __device__ __forceinline__ void quant_v_group(const uint16_t* x, int G, uint32_t
   *sz = q.sz;
 }
 
+// K-RPBH rotation of one V row held by a warp ("SoloQ", K-RPBH paragraph:
+// random permutation, per-block Hadamard, k x k orthogonal mix of the same
+// in-block coordinate across the k = d/b blocks).  On entry x[e] holds input
+// channel perm[4 lane + e] (the caller's gather applies the permutation); on
+// exit rotated channel 4 lane + e.  The fp32 order is fixed because the codes
+// depend on the last bit: butterflies (lo, hi) -> (lo + hi, lo - hi) over
+// strides 1, 2, 4, ..., b/2; one multiply by fp32(1/sqrt(b)); the mix as a
+// left-to-right sum over the k blocks of rounded products, starting from 0.
+__device__ __forceinline__ void rotate_row(float (&x)[4], int b, float norm,
+                                        const float* __restrict__ mix, int lane) {
+  const int k = kHeadDim / b, lb = b / 4;  // lanes per block
+#pragma unroll
+  for (int h = 1; h <= 2; h <<= 1) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (e & h) continue;
+      const float lo = x[e], hi = x[e + h];
+      x[e] = __fadd_rn(lo, hi);
+      x[e + h] = __fsub_rn(lo, hi);
+    }
+  }
+  for (int h = 4; h < b; h <<= 1) {
+    const bool upper = (lane & (h >> 2)) != 0;  // channel 4 lane + e has bit h set
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float p = __shfl_xor_sync(0xffffffffu, x[e], h >> 2);
+      x[e] = upper ? __fsub_rn(p, x[e]) : __fadd_rn(x[e], p);
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 4; ++e) x[e] = __fmul_rn(x[e], norm);
+  const int r = lane / lb, i_lane = lane % lb;  // output block r, in-block lane
+  float w[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int cc = 0; cc < k; ++cc) {
+    const float m = __ldg(mix + r * k + cc);  // mix[r][cc]
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      w[e] = __fadd_rn(w[e], __fmul_rn(m, __shfl_sync(0xffffffffu, x[e], cc * lb + i_lane)));
+  }
+#pragma unroll
+  for (int e = 0; e < 4; ++e) x[e] = w[e];
+}
+
+// Per-token quantization of a rotated V row held by a warp (channels 4 lane +
+// e): groups of G consecutive channels (G/4 lanes), the same quantizer as
+// quant_v_group, codes packed along channels.
+template <int VB>
+__device__ __forceinline__ void quant_v_rotated(float (&w)[4], int G, uint32_t* codes, __half2* sz,
+                                             int lane, bool& range) {
+  constexpr int levels = (1 << VB) - 1;
+  constexpr int lw = 8 / VB;  // lanes per code word (32 / VB channels)
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    range |= out_of_range(w[e]);
+    w[e] = sanitize(w[e]);
+  }
+  float mn = fminf(fminf(w[0], w[1]), fminf(w[2], w[3]));
+  float mx = fmaxf(fmaxf(w[0], w[1]), fmaxf(w[2], w[3]));
+  for (int o = 1; o < G / 4; o <<= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  const GroupQuant q = make_quant(mn, mx, levels);
+  uint32_t word = 0;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) word |= code_of(w[e], q, levels) << (e * VB);
+  word <<= (lane % lw) * 4 * VB;
+#pragma unroll
+  for (int o = 1; o < lw; o <<= 1) word |= __shfl_xor_sync(0xffffffffu, word, o);
+  if (lane % lw == 0) codes[lane / lw] = word;
+  if (lane % (G / 4) == 0) sz[lane / (G / 4)] = q.sz;
+}
+
 // One K group of channel ch: G tokens of the pending stream (rows of sk),
 // protected tokens (bits of gm) left out of min/max and given code 0.  Rolled
 // loops as above.
@@ -236,6 +309,24 @@ commit_kernel(CacheView c, const uint16_t* __restrict__ k, const uint16_t* __res
       const uint4 x = src[i];
       range_check8(x, range);
       dst[i] = x;
+    }
+  } else if (tid >= 128 && c.vrot_b) {
+    // rotated V (no sink): warp wv rotates and quantizes tokens wv, wv + 4, ...
+    const int lane = tid & 31;
+    int pm[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) pm[e] = __ldg(c.vrot_perm + 4 * lane + e);
+    for (int t = (tid - 128) >> 5; t < blk; t += 4) {
+      float x[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float f = bf16_at(sv + t * kRowPad + pm[e]);
+        range |= out_of_range(f);
+        x[e] = sanitize(f);
+      }
+      rotate_row(x, c.vrot_b, c.vrot_norm, c.vrot_mix, lane);
+      const size_t tok = size_t(u) * c.cap + size_t(p0 + t);
+      quant_v_rotated<VB>(x, c.GV, c.v_codes + tok * c.vw, c.v_sz + tok * c.vgroups, lane, range);
     }
   } else if (tid >= 128) {
     // sink positions keep their V row in bf16 too
@@ -349,6 +440,28 @@ commit_kernel(CacheView c, const uint16_t* __restrict__ k, const uint16_t* __res
   if (range) atomicOr(c.status, uint32_t(DKV_FLAG_RANGE));
 }
 
+// The active block's V rows rotated like committed rows and rounded to bf16
+// (attention sums them with the rotated cache rows).  One warp per row.
+__global__ void __launch_bounds__(256) rotate_rows_kernel(CacheView c,
+                                                          const uint16_t* __restrict__ src,
+                                                          uint16_t* __restrict__ dst,
+                                                          int64_t n_rows) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = int64_t(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (row >= n_rows) return;
+  const uint16_t* s = src + row * kHeadDim;
+  float x[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) x[e] = bf16_bits_to_f32(__ldg(s + __ldg(c.vrot_perm + 4 * lane + e)));
+  rotate_row(x, c.vrot_b, c.vrot_norm, c.vrot_mix, lane);
+  const __nv_bfloat162 lo = __floats2bfloat162_rn(x[0], x[1]);
+  const __nv_bfloat162 hi = __floats2bfloat162_rn(x[2], x[3]);
+  uint2 pk;
+  pk.x = *reinterpret_cast<const uint32_t*>(&lo);
+  pk.y = *reinterpret_cast<const uint32_t*>(&hi);
+  *reinterpret_cast<uint2*>(dst + row * kHeadDim + 4 * lane) = pk;
+}
+
 // Roll back to new_len (a multiple of the K group): the side table keeps the
 // entries stored before group new_len / GK; the tail is empty.
 __global__ void truncate_kernel(CacheView c, int64_t new_len) {
@@ -387,6 +500,13 @@ cudaError_t launch_k(const CacheView& c, const uint16_t* k, const uint16_t* v,
 
 cudaError_t launch_truncate(const CacheView& c, int64_t new_len, cudaStream_t s) {
   truncate_kernel<<<(c.U + 127) / 128, 128, 0, s>>>(c, new_len);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rotate_v_rows(const CacheView& c, const uint16_t* src, uint16_t* dst,
+                                 cudaStream_t s) {
+  const int64_t n_rows = int64_t(c.U) * c.blk;
+  rotate_rows_kernel<<<unsigned((n_rows + 7) / 8), 256, 0, s>>>(c, src, dst, n_rows);
   return cudaGetLastError();
 }
 

@@ -2,6 +2,7 @@
 // planning and kernel launches.  Every step of the path runs in the kernels
 // of commit.cu, attn_mma.cu and attn_tc.cu; this file only plans and launches.
 #include <algorithm>
+#include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <new>
@@ -29,6 +30,8 @@ struct dkv_cache {
   float* part_o = nullptr;
   float2* part_ml = nullptr;
   bool trunc_pending = false;  // a dkv_cache_truncate not yet applied on the device
+  void* vrot_mem = nullptr;      // rotation parameters + rotated active block (V rotation)
+  uint16_t* vrot_act = nullptr;  // [U][blk][d] bf16
   int32_t max_splits = 1;
   int32_t opt_splits = 0;
   int32_t opt_kernel = 0;
@@ -137,6 +140,7 @@ bool cache_info(const dkv_cache* c, CacheInfo* out) {
   out->opt_splits = c->opt_splits;
   out->opt_kernel = c->opt_kernel;
   out->max_splits = c->max_splits;
+  out->vrot_act = c->vrot_act;
   return true;
 }
 
@@ -182,6 +186,8 @@ int plan_attention(const CacheInfo& ci, AttnArgs* a, int* kernel_out, const char
   const int64_t tps = ceil_div(n_tiles, ns);
   a->nsplit = int(ceil_div(n_tiles, tps));  // no empty split
   a->tiles_per_split = int(tps);
+  // a rotated-V cache always goes through the combine kernel (inverse rotation)
+  a->final_out = (a->nsplit == 1 && v.vrot_b == 0) ? 1 : 0;
   *kernel_out = kernel;
   return DKV_OK;
 }
@@ -307,6 +313,10 @@ int dkv_cache_free(dkv_cache* c) {
   if (!c) return fail(DKV_ERR_INVALID_ARG, "cache is NULL");
   cudaError_t e = cudaDeviceSynchronize();
   cudaError_t e2 = cudaFree(c->arena);
+  if (c->vrot_mem) {
+    const cudaError_t e3 = cudaFree(c->vrot_mem);
+    if (e2 == cudaSuccess) e2 = e3;
+  }
   for (auto& r : c->prof) {
     cudaEventDestroy(r.start);
     cudaEventDestroy(r.stop);
@@ -403,15 +413,22 @@ int dkv_block_attention(dkv_cache* c, const void* q, const void* k_act, const vo
   if (prc != DKV_OK) return fail(prc, perr);
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int launches = 1;
+  if (v.vrot_b) {
+    // the active block's V into the rotated basis of the cache's V rows
+    cudaError_t e = dkv::launch_rotate_v_rows(v, a.v_act, c->vrot_act, s);
+    if (e != cudaSuccess) return fail(DKV_ERR_CUDA, std::string("rotation launch: ") + cudaGetErrorString(e));
+    a.v_act = c->vrot_act;
+    ++launches;
+  }
   cudaError_t e = timed_launch(c, DKV_KERNEL_ATTENTION, s, [&] {
     return kernel == 2 ? dkv::launch_attention_tc(a, s) : dkv::launch_attention_mma(a, s);
   });
   if (e != cudaSuccess) return fail(DKV_ERR_CUDA, std::string("attention launch: ") + cudaGetErrorString(e));
-  int launches = 1;
-  if (a.nsplit > 1) {
+  if (!a.final_out) {
     e = timed_launch(c, DKV_KERNEL_COMBINE, s, [&] { return dkv::launch_combine(a, s); });
     if (e != cudaSuccess) return fail(DKV_ERR_CUDA, std::string("combine launch: ") + cudaGetErrorString(e));
-    launches = 2;
+    ++launches;
   }
   c->last_kernel = kernel;
   c->last_splits = a.nsplit;
@@ -467,6 +484,71 @@ int dkv_cache_export(dkv_cache* c, void* stream, dkv_export* o) {
   } else {
     DKV_CUDA(copy2d(o->v_raw, v.v_raw, L * v.d * 2, v.cap * v.d * 2));
   }
+  return DKV_OK;
+}
+
+int dkv_cache_set_v_rotation(dkv_cache* c, const int32_t* perm, const float* mix,
+                             int32_t block) {
+  dkv::NvtxRange nvtx_range("dkv_cache_set_v_rotation");
+  g_err.clear();
+  if (!c) return fail(DKV_ERR_INVALID_ARG, "cache is NULL");
+  if (c->len != 0) return fail(DKV_ERR_INVALID_ARG, "set the V rotation before the first commit");
+  if (block == 0) {
+    if (c->vrot_mem) {
+      DKV_CUDA(cudaDeviceSynchronize());
+      DKV_CUDA(cudaFree(c->vrot_mem));
+    }
+    c->vrot_mem = nullptr;
+    c->vrot_act = nullptr;
+    c->v.vrot_b = 0;
+    c->v.vrot_perm = nullptr;
+    c->v.vrot_mix = nullptr;
+    return DKV_OK;
+  }
+  if (block != 16 && block != 32 && block != 64 && block != 128)
+    return fail(DKV_ERR_UNSUPPORTED, "rotation block must be 16, 32, 64 or 128");
+  if (c->v.vb == 16) return fail(DKV_ERR_UNSUPPORTED, "V rotation needs quantized V (v_bits < 16)");
+  if (c->v.sink > 0) return fail(DKV_ERR_UNSUPPORTED, "V rotation with an attention sink is not supported");
+  if (!perm || !mix) return fail(DKV_ERR_INVALID_ARG, "perm and mix must not be NULL");
+  const int d = dkv::kHeadDim, k = d / block;
+  std::vector<char> seen(d, 0);
+  for (int i = 0; i < d; ++i) {
+    if (perm[i] < 0 || perm[i] >= d || seen[perm[i]])
+      return fail(DKV_ERR_INVALID_ARG, "perm must be a permutation of 0..127");
+    seen[perm[i]] = 1;
+  }
+  for (int i = 0; i < k * k; ++i)
+    if (!std::isfinite(mix[i])) return fail(DKV_ERR_INVALID_ARG, "mix must be finite");
+  for (int r = 0; r < k; ++r)
+    for (int q = 0; q < k; ++q) {
+      double dot = 0.0;
+      for (int j = 0; j < k; ++j) dot += double(mix[r * k + j]) * double(mix[q * k + j]);
+      if (std::fabs(dot - (r == q ? 1.0 : 0.0)) > 1e-4)
+        return fail(DKV_ERR_INVALID_ARG, "mix must be orthogonal (|mix mix^T - I| <= 1e-4)");
+    }
+  // [perm d int32][mix k*k fp32] at 0, the rotated active block at 1024
+  const size_t act_bytes = size_t(c->v.U) * size_t(c->v.blk) * size_t(d) * 2;
+  void* mem = nullptr;
+  DKV_CUDA(cudaMalloc(&mem, 1024 + act_bytes));
+  std::vector<unsigned char> host(1024, 0);
+  std::memcpy(host.data(), perm, size_t(d) * 4);
+  std::memcpy(host.data() + size_t(d) * 4, mix, size_t(k) * k * 4);
+  cudaError_t e = cudaMemcpy(mem, host.data(), host.size(), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) {
+    cudaFree(mem);
+    return fail(DKV_ERR_CUDA, std::string("cudaMemcpy: ") + cudaGetErrorString(e));
+  }
+  if (c->vrot_mem) {
+    DKV_CUDA(cudaDeviceSynchronize());
+    DKV_CUDA(cudaFree(c->vrot_mem));
+  }
+  c->vrot_mem = mem;
+  unsigned char* base = static_cast<unsigned char*>(mem);
+  c->vrot_act = reinterpret_cast<uint16_t*>(base + 1024);
+  c->v.vrot_b = block;
+  c->v.vrot_norm = float(1.0 / std::sqrt(double(block)));
+  c->v.vrot_perm = reinterpret_cast<const int32_t*>(base);
+  c->v.vrot_mix = reinterpret_cast<const float*>(base + size_t(d) * 4);
   return DKV_OK;
 }
 

@@ -64,6 +64,11 @@ struct CacheView {
   uint32_t* status;     // sticky DKV_FLAG_* bits
   int32_t sink;         // positions [0, sink) in full precision (K protected, V bf16)
   uint16_t* v_sink;     // [U][sink][d] bf16 V rows of the sink positions (vb < 16)
+  // K-RPBH rotation of V (0: none): V rows are quantized in the rotated basis
+  int32_t vrot_b;             // Hadamard block b in {16, 32, 64, 128}
+  float vrot_norm;            // fp32(1 / sqrt(b))
+  const int32_t* vrot_perm;   // [d] permutation: y[i] = x[perm[i]]
+  const float* vrot_mix;      // [k][k] orthogonal mix, k = d / b
 };
 
 // Arguments of one attention call.
@@ -81,11 +86,17 @@ struct AttnArgs {
   int64_t n_tok;          // L + blk
   int32_t nsplit;
   int32_t tiles_per_split;  // in units of the kernel's token tile
+  int32_t final_out;        // 1: the attention kernel writes bf16 out (one split,
+                            // no rotation); 0: fp32 partials for combine_kernel
 };
 
 cudaError_t launch_commit(const CacheView& c, const uint16_t* k, const uint16_t* v,
                           const uint32_t* pw, int64_t p0, bool truncated, cudaStream_t s);
 cudaError_t launch_truncate(const CacheView& c, int64_t new_len, cudaStream_t s);
+// The active block's V [U][blk][d] bf16 rotated like committed V rows (same
+// fp32 order) and rounded to bf16 into dst (c.vrot_b > 0).
+cudaError_t launch_rotate_v_rows(const CacheView& c, const uint16_t* src, uint16_t* dst,
+                                 cudaStream_t s);
 
 // mma.sync kernel: token tile of 64.
 constexpr int kMmaTile = 64;
@@ -104,6 +115,7 @@ struct CacheInfo {
   int64_t len;
   int num_sms;
   int32_t opt_splits, opt_kernel, max_splits;
+  uint16_t* vrot_act;  // [U][blk][d] rotated active-block V (when c.v.vrot_b > 0)
 };
 bool cache_info(const dkv_cache* c, CacheInfo* out);
 

@@ -76,6 +76,7 @@ def test_null_arguments_rejected():
     assert dkv._len(None, ctypes.byref(n)) == dkv.DKV_ERR_INVALID_ARG
     assert dkv._free(None) == dkv.DKV_ERR_INVALID_ARG
     assert dkv._setopt(None, 1, 0) == dkv.DKV_ERR_INVALID_ARG
+    assert dkv._setrot(None, None, None, 32) == dkv.DKV_ERR_INVALID_ARG
     assert "NULL" in dkv._lib.dkv_last_error().decode()
 
 
