@@ -409,6 +409,32 @@ class OracleCache:
             O = krpbh.unrotate_f64(O, perm, mix.astype(np.float64), rb)
         return O
 
+    def block_attention_dual(self, suffix: "OracleCache", Q_bits, Kact_bits, Vact_bits,
+                             scale: float) -> np.ndarray:
+        """Dual-cache attention (Fast-dLLM-style prefix and dual cache reuse,
+        "KV Cache Quantization for Diffusion Language Models", abstract): the
+        active block's queries attend to this (prefix) cache, the active block
+        and a second cache holding the suffix region after the block, each
+        cache dequantized with its own parameters; softmax over all of them
+        (bidirectional, no mask).  Neither cache may rotate V; the suffix has
+        no sink."""
+        B, Hq, Hkv, blk, d = self.B, self.Hq, self.Hkv, self.blk, self.d
+        assert (suffix.B, suffix.Hq, suffix.Hkv, suffix.blk, suffix.d) == (B, Hq, Hkv, blk, d)
+        assert self.v_rot is None and suffix.v_rot is None and suffix.sink == 0
+        g = Hq // Hkv
+        Q = bf16_to_f64(np.asarray(Q_bits).reshape(B, Hq, blk, d))
+        Ka = bf16_to_f64(np.asarray(Kact_bits).reshape(B, Hkv, blk, d))
+        Va = bf16_to_f64(np.asarray(Vact_bits).reshape(B, Hkv, blk, d))
+        O = np.zeros((B, Hq, blk, d), np.float64)
+        for b in range(B):
+            for h in range(Hkv):
+                u = b * Hkv + h
+                Kall = np.concatenate([self.dequant_k(u), Ka[b, h], suffix.dequant_k(u)])
+                Vall = np.concatenate([self.dequant_v(u), Va[b, h], suffix.dequant_v(u)])
+                for hq in range(h * g, (h + 1) * g):
+                    O[b, hq] = dense_attention_f64(Q[b, hq], Kall, Vall, scale)
+        return O
+
     # -- canonical snapshot of the committed state (what an export returns)
     def snapshot(self) -> dict:
         L, GK = self.len, self.GK

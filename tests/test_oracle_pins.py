@@ -834,3 +834,78 @@ def test_rotation_spreads_v_outliers(seed):
                      for h in range(4)])
     err = [np.abs(c.block_attention(Q, Ka, Va, 1 / np.sqrt(d))[0] - want).mean() for c in caches]
     assert err[1] < 0.6 * err[0], err
+
+
+# ------------------------------------------------------------ dual cache
+
+def _dual_setup(kb=4, vb=4, gk=32, gv=32, nA=4, nB=3, prot=0.03):
+    w = synth.WORKLOADS["tiny"].with_(Hq=4, Hkv=2, k_bits=kb, v_bits=vb, k_group=gk,
+                                      v_group=gv, prot_frac=prot, seed=9)
+    mk = lambda cap: OracleCache(w.B, w.Hq, w.Hkv, w.d, w.blk, kb, vb, gk, gv, 64, cap)
+    blocks = [synth.block_inputs(w, i) for i in range(nA + nB)]
+    return w, mk, blocks[:nA], blocks[nA:]
+
+
+def test_dual_with_empty_suffix_is_single_cache_attention():
+    w, mk, A, _ = _dual_setup()
+    pre, suf = mk(256), mk(128)
+    for K, V, M in A:
+        pre.commit(K, V, M)
+    Q = synth.queries_bits(w, 0)
+    Ka, Va = synth.active_block_bits(w, 0)
+    assert np.array_equal(pre.block_attention_dual(suf, Q, Ka, Va, 0.1),
+                          pre.block_attention(Q, Ka, Va, 0.1))
+
+
+def test_dual_equals_one_cache_holding_both_regions():
+    """K groups of one block (GK = blk): each block quantizes on its own, so a
+    suffix cache holding blocks X gives the same dequantized keys and values as
+    appending X to the prefix; softmax attention does not depend on key order."""
+    w, mk, A, X = _dual_setup(kb=2, vb=4, gk=32, gv=64)
+    pre, suf, one = mk(256), mk(128), mk(384)
+    for K, V, M in A:
+        pre.commit(K, V, M)
+        one.commit(K, V, M)
+    for K, V, M in X:
+        suf.commit(K, V, M)
+        one.commit(K, V, M)
+    Q = synth.queries_bits(w, 1)
+    Ka, Va = synth.active_block_bits(w, 1)
+    np.testing.assert_allclose(pre.block_attention_dual(suf, Q, Ka, Va, 0.1),
+                               one.block_attention(Q, Ka, Va, 0.1), atol=1e-13)
+
+
+def test_dual_prefix_and_suffix_roles_swap():
+    """Attention is symmetric in which cache holds which region."""
+    w, mk, A, X = _dual_setup(kb=4, vb=2, gk=64, gv=32)
+    a1, b1, a2, b2 = mk(256), mk(256), mk(256), mk(256)
+    for K, V, M in A:
+        a1.commit(K, V, M)
+        a2.commit(K, V, M)
+    for K, V, M in X:
+        b1.commit(K, V, M)
+        b2.commit(K, V, M)
+    Q = synth.queries_bits(w, 2)
+    Ka, Va = synth.active_block_bits(w, 2)
+    np.testing.assert_allclose(a1.block_attention_dual(b1, Q, Ka, Va, 0.1),
+                               b2.block_attention_dual(a2, Q, Ka, Va, 0.1), atol=1e-13)
+
+
+def test_dual_passthrough_is_dense_attention():
+    w, mk, A, X = _dual_setup(kb=16, vb=16)
+    pre, suf = mk(256), mk(128)
+    for K, V, M in A:
+        pre.commit(K, V, M)
+    for K, V, M in X:
+        suf.commit(K, V, M)
+    Q = synth.queries_bits(w, 3)
+    Ka, Va = synth.active_block_bits(w, 3)
+    got = pre.block_attention_dual(suf, Q, Ka, Va, 0.1)
+    for h in range(w.Hkv):
+        Kall = bf16_to_f64(np.concatenate([b[0][0, h] for b in A] + [Ka[0, h]] +
+                                          [b[0][0, h] for b in X]))
+        Vall = bf16_to_f64(np.concatenate([b[1][0, h] for b in A] + [Va[0, h]] +
+                                          [b[1][0, h] for b in X]))
+        for hq in range(h * 2, h * 2 + 2):
+            want = dense_attention_f64(bf16_to_f64(Q[0, hq]), Kall, Vall, 0.1)
+            np.testing.assert_allclose(got[0, hq], want, atol=1e-13)
