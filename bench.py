@@ -210,8 +210,13 @@ def whole_job_gbs(bytes_per_rank: float, max_ms: float, world: int) -> float:
     return world * bytes_per_rank / (max_ms / 1e3) / 1e9
 
 
+def io_bytes(w: synth.Workload) -> float:
+    """Q, active K/V and output bytes of one attention call."""
+    return w.B * w.Hq * w.blk * w.d * 2 * 2 + 2 * w.B * w.Hkv * w.blk * w.d * 2
+
+
 def run_gpu(w: synth.Workload, K: int, W: int, want_e2e=True, log=print, kernel=0,
-            v_rotation=0):
+            v_rotation=0, suffix=0):
     import torch
     import quantized_kv_cache_dkv_b200 as dkv
 
@@ -229,6 +234,13 @@ def run_gpu(w: synth.Workload, K: int, W: int, want_e2e=True, log=print, kernel=
     cfg = dkv.make_config(w.B, w.Hq, w.Hkv, w.d, w.blk, w.k_bits, w.v_bits, w.k_group,
                           w.v_group, P, cap)
     caches = [dkv.dkv_cache_alloc(cfg) for _ in range(R)]
+    # dual cache: a suffix cache of `suffix` committed tokens per replica
+    sfx = []
+    if suffix:
+        cap_s = ((suffix + unit - 1) // unit) * unit
+        cfg_s = dkv.make_config(w.B, w.Hq, w.Hkv, w.d, w.blk, w.k_bits, w.v_bits, w.k_group,
+                                w.v_group, int(round(w.prot_frac * cap_s)) * 2 + 64, cap_s)
+        sfx = [dkv.dkv_cache_alloc(cfg_s) for _ in range(R)]
     if v_rotation:
         perm, mix = synth.krpbh_params(w.seed, v_rotation)
         for c in caches:
@@ -253,8 +265,19 @@ def run_gpu(w: synth.Workload, K: int, W: int, want_e2e=True, log=print, kernel=
         Kd, Vd, Md = up(K_), up(V_), upw(M_)
         for c in caches:
             dkv.dkv_commit_block(c, Kd, Vd, Md)
+    for i in range(suffix // w.blk):
+        K_, V_, M_ = synth.block_inputs(w, 100000 + i)
+        Kd, Vd, Md = up(K_), up(V_), upw(M_)
+        for c in sfx:
+            dkv.dkv_commit_block(c, Kd, Vd, Md)
     torch.cuda.synchronize()
     t_prefill = time.time() - t0
+
+    def attend(r, q, ka, va, out):
+        if sfx:
+            dkv.dkv_block_attention_dual(caches[r], sfx[r], q, ka, va, w.softmax_scale, out)
+        else:
+            dkv.dkv_block_attention(caches[r], q, ka, va, w.softmax_scale, out)
 
     # per-step inputs: C blocks to commit, S distinct query / active blocks
     blocks = [synth.block_inputs(w, nb + c) for c in range(C)]
@@ -277,7 +300,7 @@ def run_gpu(w: synth.Workload, K: int, W: int, want_e2e=True, log=print, kernel=
         Kd, Vd, Md = dblocks[c]
         dkv.dkv_commit_block(caches[r], Kd, Vd, Md)
         q, ka, va = dsteps[k % S]
-        dkv.dkv_block_attention(caches[r], q, ka, va, w.softmax_scale, outs[k % S])
+        attend(r, q, ka, va, outs[k % S])
         launches[0] += 1 + dkv.dkv_last_attention_plan(caches[r])[2]
         pos[r] += 1
         if pos[r] == C:  # back to the starting length (recorded; the next commit applies it)
@@ -333,11 +356,12 @@ def run_gpu(w: synth.Workload, K: int, W: int, want_e2e=True, log=print, kernel=
     ms = max_over_ranks(ms)
 
     Ls = step_lengths(w, K, R)
-    step_bytes = sum(attn_bytes(w, L + w.blk) + commit_bytes(w, L) for L in Ls)
+    sfx_bytes = attn_bytes(w, suffix) - io_bytes(w) if suffix else 0.0
+    step_bytes = sum(attn_bytes(w, L + w.blk) + sfx_bytes + commit_bytes(w, L) for L in Ls)
     value = whole_job_gbs(step_bytes, ms, world)
 
     # profiling pass: device time of each kernel kind (eager launches)
-    for c in caches:
+    for c in caches + sfx:
         dkv.dkv_cache_set_option(c, dkv.DKV_OPT_PROFILE, 1)
     Kp = max(K, 2 * R * C)
     for k in range(Kp):
@@ -353,12 +377,15 @@ def run_gpu(w: synth.Workload, K: int, W: int, want_e2e=True, log=print, kernel=
             tot += a
             n += b
         prof[name] = (tot, n)
-    for c in caches:
+    for c in caches + sfx:
         dkv.dkv_cache_set_option(c, dkv.DKV_OPT_PROFILE, 0)
     Lp = step_lengths(w, Kp, R)
     att_ms, att_n = prof["attention"]
-    att_bytes = sum(attn_bytes(w, L + w.blk) for L in Lp)
-    att_flops = sum(attn_flops(w, L + w.blk) for L in Lp)
+    # (a dual-cache step launches the attention kernel twice: its bytes and
+    # flops are those of both launches, averaged per launch below)
+    att_bytes = sum(attn_bytes(w, L + w.blk) + sfx_bytes for L in Lp)
+    att_flops = sum(attn_flops(w, L + w.blk) + 4.0 * w.rows * w.d * suffix * w.B * w.Hkv
+                    for L in Lp)
     com_ms, com_n = prof["commit"]
 
     # end to end through the public API from pinned host memory
@@ -430,7 +457,7 @@ def run_gpu(w: synth.Workload, K: int, W: int, want_e2e=True, log=print, kernel=
                 s_cp.wait_event(ev_dn[b])  # the previous output in dO[b] has been read back
             dK, dV, dM, dQ, dKa, dVa = views[b]
             dkv.dkv_commit_block(caches[r], dK, dV, dM)
-            dkv.dkv_block_attention(caches[r], dQ, dKa, dVa, w.softmax_scale, dO[b])
+            attend(r, dQ, dKa, dVa, dO[b])
             ev_cp[b].record(s_cp)
             pos[r] += 1
             if pos[r] == C:
@@ -488,7 +515,7 @@ def run_gpu(w: synth.Workload, K: int, W: int, want_e2e=True, log=print, kernel=
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": ems / K}
 
-    for c in caches:
+    for c in caches + sfx:
         dkv.dkv_cache_free(c)
     return {
         "ms": ms, "value": value, "R": R, "C": C, "cap": cap, "P": P, "plan": plan,
@@ -628,6 +655,8 @@ def main():
     ap.add_argument("--L", type=int, default=0, help="override the committed length (profiling)")
     ap.add_argument("--v-rotation", type=int, default=0, choices=[0, 16, 32, 64, 128],
                     help="K-RPBH rotation of V with this Hadamard block (0 = none)")
+    ap.add_argument("--suffix", type=int, default=0,
+                    help="dual cache: tokens in a second (suffix) cache attended with the prefix")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -664,17 +693,23 @@ def main():
                                 device_id=torch.device("cuda", local))
     peaks, peak_kind = load_peaks()
     traffic = traffic_record()
+    if args.suffix % w.blk:
+        raise SystemExit("--suffix must be a multiple of the block")
     r = run_gpu(w, args.steps, args.warmup, log=lambda *a: None, kernel=args.kernel,
-                v_rotation=args.v_rotation)
+                v_rotation=args.v_rotation, suffix=args.suffix)
     line = base_line(w, args, r["value"], r["ms"] / args.steps, world)
     if args.v_rotation:
         line["config"]["v_rotation"] = f"K-RPBH, Hadamard block {args.v_rotation}"
+    if args.suffix:
+        line["config"]["dual_cache_suffix_tokens"] = args.suffix
     line["config"]["L2_policy"] = (f"{r['R']} cache replicas used round-robin"
                                    if r["R"] > 1 else "cache larger than L2")
     line["config"]["L_mean"] = r["L_mean"]
     line["config"]["step"] = (f"1 commit + 1 attention; truncate to L every {r['C']} steps; "
                               "timed region = one CUDA graph replay of the steps")
     line["roofline"] = roofline(w, r, peaks, peak_kind, traffic)
+    if args.suffix:  # the recorded traffic is that of the single-cache launch
+        line["roofline"]["traffic"] = None
     line["clocks"] = r["clocks"]
     line["e2e"] = r["e2e"]
     line["gpu_launches"] = r["graph_launches"]
@@ -704,7 +739,8 @@ def main():
                 "commit_tokens_per_s": round(ww.B * ww.blk * rr["commit_n"] /
                                              (rr["commit_ms"] / 1e3), 1),
                 "plan": rr["plan"], "clocks_sm_mhz": (rr["clocks"] or {}).get("sm_mhz")}
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.v_rotation:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.v_rotation \
+            and not args.suffix:
         gbs, steps, el, desc = oracle_sample(w, args.cpu_seconds)
         line["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": _blas_threads(),
                                 "kind": "oracle", "sample": desc}

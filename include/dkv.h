@@ -125,6 +125,25 @@ int dkv_block_attention(dkv_cache* cache, const void* q, const void* k_act,
                         const void* v_act, float softmax_scale, void* out,
                         void* stream);
 
+/* Dual-cache attention (the prefix and dual cache reuse of Fast-dLLM-style
+ * decoding that "KV Cache Quantization for Diffusion Language Models"
+ * quantizes, abstract): the active block's queries attend to `prefix` (the
+ * committed tokens before the block), the active block, and `suffix`, a second
+ * cache holding the KV of the region after the block (for instance the masked
+ * tokens of later blocks, refreshed with dkv_cache_truncate(suffix, 0) and new
+ * commits).  out = softmax over all three segments, bidirectional, no mask;
+ * each cache is dequantized with its own bit widths and groups (a bf16 suffix
+ * uses bits = 16).  Arguments as in dkv_block_attention.  The two caches must
+ * have the same batch, heads, head_dim and block; neither may rotate V
+ * (DKV_ERR_UNSUPPORTED), the suffix may not have a sink.  An empty suffix
+ * gives exactly dkv_block_attention.  Launches: the split attention kernel on
+ * each cache (the suffix with its own DKV_OPT_* choices) writing into the
+ * prefix cache's split workspace, then one combine; no allocation.  Device
+ * flags raised while reading the suffix are reported by the suffix handle. */
+int dkv_block_attention_dual(dkv_cache* prefix, dkv_cache* suffix, const void* q,
+                             const void* k_act, const void* v_act, float softmax_scale,
+                             void* out, void* stream);
+
 /* Rotated V (K-RPBH, "SoloQ: Calibration-Free Quantization for Diffusion
  * Language Models", K-RPBH paragraph and the KV-cache paragraph): committed V
  * rows are rotated by an orthogonal map R before their per-token

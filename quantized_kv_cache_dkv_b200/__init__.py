@@ -77,6 +77,7 @@ _status = _sig("dkv_cache_status", [_P, _P, ctypes.POINTER(ctypes.c_uint32)])
 _export = _sig("dkv_cache_export", [_P, _P, ctypes.POINTER(dkv_export)])
 _setopt = _sig("dkv_cache_set_option", [_P, ctypes.c_int32, ctypes.c_int64])
 _setrot = _sig("dkv_cache_set_v_rotation", [_P, _P, _P, ctypes.c_int32])
+_attn_dual = _sig("dkv_block_attention_dual", [_P, _P, _P, _P, _P, ctypes.c_float, _P, _P])
 _prof = _sig("dkv_profile_read", [_P, ctypes.c_int32, ctypes.POINTER(ctypes.c_double),
                                   ctypes.POINTER(ctypes.c_int64)])
 _plan = _sig("dkv_last_attention_plan", [_P, ctypes.POINTER(ctypes.c_int32),
@@ -201,6 +202,22 @@ def dkv_block_attention_noalloc(cache: Cache, q, k_act, v_act, softmax_scale: fl
 
 def dkv_cache_truncate(cache: Cache, new_len: int, stream=None) -> None:
     _check(_truncate(cache.h, new_len, _stream(stream)))
+
+
+def dkv_block_attention_dual(prefix: Cache, suffix: Cache, q, k_act, v_act,
+                             softmax_scale: float, out, stream=None) -> None:
+    """Attention of the active block over prefix cache + active block +
+    suffix cache (dual-cache reuse); shapes as in dkv_block_attention."""
+    import torch
+    c = prefix.cfg
+    _tensor_check(q, (c.batch, c.q_heads, c.block, c.head_dim), "q", (torch.bfloat16, torch.int16))
+    shp = (c.batch, c.kv_heads, c.block, c.head_dim)
+    _tensor_check(k_act, shp, "k_act", (torch.bfloat16, torch.int16))
+    _tensor_check(v_act, shp, "v_act", (torch.bfloat16, torch.int16))
+    _tensor_check(out, (c.batch, c.q_heads, c.block, c.head_dim), "out",
+                  (torch.bfloat16, torch.int16))
+    _check(_attn_dual(prefix.h, suffix.h, _ptr(q), _ptr(k_act), _ptr(v_act),
+                      ctypes.c_float(softmax_scale), _ptr(out), _stream(stream)))
 
 
 def dkv_cache_set_v_rotation(cache: Cache, perm=None, mix=None, block: int = 0) -> None:

@@ -344,7 +344,7 @@ attn_mma_kernel(AttnArgs a) {
       *reinterpret_cast<__nv_bfloat162*>(out1 + col) = v1;
     }
   } else {
-    const size_t prow = (size_t(u) * a.nsplit + sp) * c.rows;
+    const size_t prow = (size_t(u) * a.part_stride + a.part_base + sp) * c.rows;
     float* po0 = a.part_o + (prow + r0) * kHeadDim;
     float* po1 = po0 + 8 * kHeadDim;
 #pragma unroll

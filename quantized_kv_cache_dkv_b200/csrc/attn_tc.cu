@@ -952,7 +952,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           }
         } else {
           float4* dst = reinterpret_cast<float4*>(
-              a.part_o + ((size_t(u) * a.nsplit + sp) * cv.rows + r) * kHeadDim + col);
+              a.part_o + ((size_t(u) * a.part_stride + a.part_base + sp) * cv.rows + r) * kHeadDim + col);
 #pragma unroll
           for (int i = 0; i < 8; ++i)
             dst[i] = make_float4(__uint_as_float(o[kpos<VB>(4 * i)]), __uint_as_float(o[kpos<VB>(4 * i + 1)]),
@@ -960,7 +960,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         }
       }
       if (!a.final_out && row_ok && h == 0)
-        a.part_ml[(size_t(u) * a.nsplit + sp) * cv.rows + r] = make_float2(rf, lt);
+        a.part_ml[(size_t(u) * a.part_stride + a.part_base + sp) * cv.rows + r] = make_float2(rf, lt);
     }
   } else if (warp < 24) {
     regs_dec<kRegProducer>();

@@ -146,11 +146,16 @@ bool cache_info(const dkv_cache* c, CacheInfo* out) {
 
 int report_error(int code, const char* msg) { return fail(code, msg); }
 
-int plan_attention(const CacheInfo& ci, AttnArgs* a, int* kernel_out, const char** err) {
+int plan_attention(const CacheInfo& ci, AttnArgs* a, int* kernel_out, const char** err,
+                   bool with_active) {
   const CacheView& v = ci.v;
   a->L = ci.len;
   a->Lq = v.kb < 16 ? (ci.len / v.GK) * v.GK : ci.len;
-  a->n_tok = ci.len + v.blk;
+  a->n_tok = ci.len + (with_active ? v.blk : 0);
+  if (a->n_tok <= 0) {
+    *err = "no tokens to attend to";
+    return DKV_ERR_INVALID_ARG;
+  }
   int kernel = ci.opt_kernel;
   if (kernel == 0) kernel = tc_supported(v) ? 2 : 1;
   if (kernel == 2 && !tc_supported(v)) {
@@ -188,6 +193,8 @@ int plan_attention(const CacheInfo& ci, AttnArgs* a, int* kernel_out, const char
   a->tiles_per_split = int(tps);
   // a rotated-V cache always goes through the combine kernel (inverse rotation)
   a->final_out = (a->nsplit == 1 && v.vrot_b == 0) ? 1 : 0;
+  a->part_base = 0;
+  a->part_stride = a->nsplit;
   *kernel_out = kernel;
   return DKV_OK;
 }
@@ -433,6 +440,78 @@ int dkv_block_attention(dkv_cache* c, const void* q, const void* k_act, const vo
   c->last_kernel = kernel;
   c->last_splits = a.nsplit;
   c->last_launches = launches;
+  return DKV_OK;
+}
+
+int dkv_block_attention_dual(dkv_cache* c, dkv_cache* sfx, const void* q, const void* k_act,
+                             const void* v_act, float softmax_scale, void* out, void* stream) {
+  dkv::NvtxRange nvtx_range("dkv_block_attention_dual");
+  g_err.clear();
+  if (!c || !sfx || !q || !k_act || !v_act || !out) return fail(DKV_ERR_INVALID_ARG, "NULL argument");
+  const dkv::CacheView& v = c->v;
+  const dkv::CacheView& vs = sfx->v;
+  if (vs.B != v.B || vs.Hq != v.Hq || vs.Hkv != v.Hkv || vs.d != v.d || vs.blk != v.blk)
+    return fail(DKV_ERR_INVALID_ARG, "prefix and suffix caches must share batch, heads, head_dim and block");
+  if (v.vrot_b || vs.vrot_b)
+    return fail(DKV_ERR_UNSUPPORTED, "dual-cache attention with rotated V is not supported");
+  if (vs.sink > 0) return fail(DKV_ERR_UNSUPPORTED, "the suffix cache cannot have an attention sink");
+  if (sfx->len == 0) {
+    // nothing after the active block: the single-cache call
+    const int rc = dkv_block_attention(c, q, k_act, v_act, softmax_scale, out, stream);
+    return rc;
+  }
+  if (!aligned16(q) || !aligned16(k_act) || !aligned16(v_act) || !aligned16(out))
+    return fail(DKV_ERR_INVALID_ARG, "q, k_act, v_act and out must be 16-byte aligned");
+  if (!(softmax_scale == softmax_scale) || softmax_scale > 3.0e38f || softmax_scale < -3.0e38f)
+    return fail(DKV_ERR_INVALID_ARG, "softmax_scale must be finite");
+
+  // prefix + active block: splits [0, n1); suffix: splits [n1, n1 + n2) of the
+  // prefix cache's partial workspace (room for max_splits per unit)
+  dkv::AttnArgs a1{}, a2{};
+  for (dkv::AttnArgs* a : {&a1, &a2}) {
+    a->q = static_cast<const uint16_t*>(q);
+    a->k_act = static_cast<const uint16_t*>(k_act);
+    a->v_act = static_cast<const uint16_t*>(v_act);
+    a->out = static_cast<uint16_t*>(out);
+    a->part_o = c->part_o;
+    a->part_ml = c->part_ml;
+    a->scale_log2 = softmax_scale * 1.4426950408889634f;
+  }
+  a1.c = v;
+  a2.c = vs;
+  dkv::CacheInfo ci1, ci2;
+  dkv::cache_info(c, &ci1);
+  dkv::cache_info(sfx, &ci2);
+  ci1.max_splits = c->max_splits - 1;
+  int k1 = 0, k2 = 0;
+  const char* perr = nullptr;
+  int prc = dkv::plan_attention(ci1, &a1, &k1, &perr, true);
+  if (prc != DKV_OK) return fail(prc, perr);
+  ci2.max_splits = c->max_splits - a1.nsplit;
+  prc = dkv::plan_attention(ci2, &a2, &k2, &perr, false);
+  if (prc != DKV_OK) return fail(prc, perr);
+  const int total = a1.nsplit + a2.nsplit;
+  a1.final_out = a2.final_out = 0;
+  a1.part_base = 0;
+  a2.part_base = a1.nsplit;
+  a1.part_stride = a2.part_stride = total;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = timed_launch(c, DKV_KERNEL_ATTENTION, s, [&] {
+    return k1 == 2 ? dkv::launch_attention_tc(a1, s) : dkv::launch_attention_mma(a1, s);
+  });
+  if (e != cudaSuccess) return fail(DKV_ERR_CUDA, std::string("attention launch: ") + cudaGetErrorString(e));
+  e = timed_launch(c, DKV_KERNEL_ATTENTION, s, [&] {
+    return k2 == 2 ? dkv::launch_attention_tc(a2, s) : dkv::launch_attention_mma(a2, s);
+  });
+  if (e != cudaSuccess) return fail(DKV_ERR_CUDA, std::string("suffix attention launch: ") + cudaGetErrorString(e));
+  dkv::AttnArgs ac = a1;
+  ac.nsplit = total;
+  e = timed_launch(c, DKV_KERNEL_COMBINE, s, [&] { return dkv::launch_combine(ac, s); });
+  if (e != cudaSuccess) return fail(DKV_ERR_CUDA, std::string("combine launch: ") + cudaGetErrorString(e));
+  c->last_kernel = k1;
+  c->last_splits = total;
+  c->last_launches = 3;
   return DKV_OK;
 }
 

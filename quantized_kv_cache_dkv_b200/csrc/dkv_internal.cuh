@@ -88,6 +88,8 @@ struct AttnArgs {
   int32_t tiles_per_split;  // in units of the kernel's token tile
   int32_t final_out;        // 1: the attention kernel writes bf16 out (one split,
                             // no rotation); 0: fp32 partials for combine_kernel
+  int32_t part_base;        // split sp of unit u writes partial u*part_stride +
+  int32_t part_stride;      // part_base + sp (one call: 0 and nsplit)
 };
 
 cudaError_t launch_commit(const CacheView& c, const uint16_t* k, const uint16_t* v,
@@ -122,7 +124,10 @@ bool cache_info(const dkv_cache* c, CacheInfo* out);
 // Launch plan of one attention call (kernel, split count, tiles per split);
 // fills a->L, Lq, n_tok, nsplit, tiles_per_split.  Returns DKV_OK or an error
 // code with *err set.
-int plan_attention(const CacheInfo& ci, AttnArgs* a, int* kernel, const char** err);
+// with_active = false: the tokens are the committed ones only (no active
+// block; the suffix cache of a dual-cache call).
+int plan_attention(const CacheInfo& ci, AttnArgs* a, int* kernel, const char** err,
+                   bool with_active = true);
 int report_error(int code, const char* msg);
 
 }  // namespace dkv

@@ -77,6 +77,8 @@ def test_null_arguments_rejected():
     assert dkv._free(None) == dkv.DKV_ERR_INVALID_ARG
     assert dkv._setopt(None, 1, 0) == dkv.DKV_ERR_INVALID_ARG
     assert dkv._setrot(None, None, None, 32) == dkv.DKV_ERR_INVALID_ARG
+    assert dkv._attn_dual(None, None, P(16), P(16), P(16), ctypes.c_float(1.0), P(16), None) == \
+        dkv.DKV_ERR_INVALID_ARG
     assert "NULL" in dkv._lib.dkv_last_error().decode()
 
 
