@@ -203,6 +203,8 @@ __global__ void __launch_bounds__(256)
 attn_mma_kernel(AttnArgs a) {
   __shared__ __align__(16) __half Kt[kHeadDim * KT_LD];
   __shared__ __align__(16) __half Vt[T * VT_LD];
+  pdl_wait();
+  pdl_trigger();
 
   const CacheView& c = a.c;
   const int nrb = (c.rows + kRowsPerCta - 1) / kRowsPerCta;
@@ -405,6 +407,8 @@ __device__ __forceinline__ void unrotate_row(float (&x)[4], int b, float norm,
 // (rotated back first when V is stored rotated)
 __global__ void __launch_bounds__(128) combine_kernel(AttnArgs a) {
   __shared__ float rbuf[4][kHeadDim];
+  pdl_wait();
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t row = int64_t(blockIdx.x) * 4 + warp;
   const int rows = a.c.rows;
@@ -445,7 +449,8 @@ cudaError_t launch_kv(const AttnArgs& a, cudaStream_t s) {
   if (a.c.rows % 16) return cudaErrorInvalidValue;
   const int threads = rows_cta * 2;  // one warp per 16 rows
   const unsigned grid = unsigned(a.c.U) * unsigned(a.nsplit) * unsigned(nrb);
-  attn_mma_kernel<KB, VB><<<grid, threads, 0, s>>>(a);
+  const cudaError_t e = launch_pdl(attn_mma_kernel<KB, VB>, dim3(grid), dim3(threads), 0, s, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -470,7 +475,8 @@ cudaError_t launch_attention_mma(const AttnArgs& a, cudaStream_t s) {
 
 cudaError_t launch_combine(const AttnArgs& a, cudaStream_t s) {
   const int64_t rows = int64_t(a.c.U) * a.c.rows;
-  combine_kernel<<<unsigned((rows + 3) / 4), 128, 0, s>>>(a);
+  const cudaError_t e = launch_pdl(combine_kernel, dim3(unsigned((rows + 3) / 4)), dim3(128), 0, s, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

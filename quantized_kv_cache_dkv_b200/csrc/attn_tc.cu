@@ -736,6 +736,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                  "r"(kTmemCols));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
+  pdl_wait();  // no global memory access above this line
+  pdl_trigger();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -1184,7 +1186,9 @@ cudaError_t launch_kvs(const AttnArgs& a, cudaStream_t s) {
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   const unsigned nrb = unsigned((a.c.rows + 127) / 128);
-  attn_tc_kernel<KB, VB, SINK><<<unsigned(a.c.U) * unsigned(a.nsplit) * nrb, kThreads, smem, s>>>(a);
+  e = launch_pdl(attn_tc_kernel<KB, VB, SINK>, dim3(unsigned(a.c.U) * unsigned(a.nsplit) * nrb),
+                 dim3(kThreads), smem, s, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

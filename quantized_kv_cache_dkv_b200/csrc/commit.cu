@@ -262,6 +262,8 @@ __global__ void __launch_bounds__(kThreads)
 commit_kernel(CacheView c, const uint16_t* __restrict__ k, const uint16_t* __restrict__ v,
               const uint32_t* __restrict__ pw, int64_t p0, int truncated) {
   extern __shared__ __align__(16) uint16_t sbuf[];
+  pdl_wait();
+  pdl_trigger();
   const int u = blockIdx.x;
   const int tid = threadIdx.x;
   const int d = kHeadDim;
@@ -446,6 +448,8 @@ __global__ void __launch_bounds__(256) rotate_rows_kernel(CacheView c,
                                                           const uint16_t* __restrict__ src,
                                                           uint16_t* __restrict__ dst,
                                                           int64_t n_rows) {
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int64_t row = int64_t(blockIdx.x) * 8 + (threadIdx.x >> 5);
   if (row >= n_rows) return;
@@ -465,6 +469,8 @@ __global__ void __launch_bounds__(256) rotate_rows_kernel(CacheView c,
 // Roll back to new_len (a multiple of the K group): the side table keeps the
 // entries stored before group new_len / GK; the tail is empty.
 __global__ void truncate_kernel(CacheView c, int64_t new_len) {
+  pdl_wait();
+  pdl_trigger();
   const int u = blockIdx.x * blockDim.x + threadIdx.x;
   if (u >= c.U) return;
   c.prot_count[u] = c.prot_gstart[size_t(u) * (c.nG + 1) + new_len / c.GK];
@@ -482,7 +488,9 @@ cudaError_t launch_kv(const CacheView& c, const uint16_t* k, const uint16_t* v,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     if (e != cudaSuccess) return e;
   }
-  commit_kernel<KB, VB><<<c.U, kThreads, smem, s>>>(c, k, v, pw, p0, truncated ? 1 : 0);
+  const cudaError_t e = launch_pdl(commit_kernel<KB, VB>, dim3(c.U), dim3(kThreads), smem, s, c, k,
+                                   v, pw, p0, truncated ? 1 : 0);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -499,14 +507,18 @@ cudaError_t launch_k(const CacheView& c, const uint16_t* k, const uint16_t* v,
 }  // namespace
 
 cudaError_t launch_truncate(const CacheView& c, int64_t new_len, cudaStream_t s) {
-  truncate_kernel<<<(c.U + 127) / 128, 128, 0, s>>>(c, new_len);
+  const cudaError_t e = launch_pdl(truncate_kernel, dim3((c.U + 127) / 128), dim3(128), 0, s, c,
+                                   new_len);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 cudaError_t launch_rotate_v_rows(const CacheView& c, const uint16_t* src, uint16_t* dst,
                                  cudaStream_t s) {
   const int64_t n_rows = int64_t(c.U) * c.blk;
-  rotate_rows_kernel<<<unsigned((n_rows + 7) / 8), 256, 0, s>>>(c, src, dst, n_rows);
+  const cudaError_t e = launch_pdl(rotate_rows_kernel, dim3(unsigned((n_rows + 7) / 8)), dim3(256),
+                                   0, s, c, src, dst, n_rows);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -23,6 +23,36 @@ namespace dkv {
 #define DKV_IN_BOUNDS(cond, status) true
 #endif
 
+// Programmatic dependent launch.  Every kernel of the library is launched
+// with launch_pdl, so the GPU may schedule it while the previous kernel of its
+// stream is still running; it calls pdl_wait() before its first global memory
+// access (the wait returns once the previous grid has completed and its
+// writes are visible) and then pdl_trigger(), which lets the next kernel be
+// scheduled as soon as every CTA of this grid has reached it.  What overlaps
+// is only launch latency and setup that touches no global memory (shared
+// memory barriers, TMEM allocation).  A dependent is scheduled only after all
+// CTAs of its predecessor are resident, so early CTAs cannot starve it.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KParams, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KParams...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // Host-side NVTX range around one library call (header-only NVTX: it costs a
 // few nanoseconds unless a profiler is attached, which then shows each call
 // on the timeline).
