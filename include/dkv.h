@@ -197,8 +197,11 @@ int dkv_cache_truncate(dkv_cache* cache, int64_t new_len, void* stream);
  *   - The buffer is a static __device__ array of DKV_NOALLOC_SCRATCH_BYTES
  *     (16 MiB); every GPU that loads libdkv holds it until the process exits.
  *   - A plan needing more scratch than that (B*Hkv * splits *
- *     (q_heads/kv_heads)*block * (4*head_dim + 8) bytes, when splits > 1)
- *     returns DKV_ERR_UNSUPPORTED with a message; lower DKV_OPT_SPLITS.
+ *     (q_heads/kv_heads)*block * (4*head_dim + 8) bytes, whenever the
+ *     combine kernel runs: splits > 1, or a rotated-V cache) returns
+ *     DKV_ERR_UNSUPPORTED with a message; lower DKV_OPT_SPLITS.
+ *   - A rotated-V cache rotates the active block's V into the buffer the
+ *     handle allocated in dkv_cache_set_v_rotation (no allocation here).
  *   - The first call on each device looks up the buffer's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
  *     before any stream capture.
@@ -274,9 +277,13 @@ enum { DKV_KERNEL_ATTENTION = 0, DKV_KERNEL_COMBINE = 1, DKV_KERNEL_COMMIT = 2,
        DKV_KERNEL_TRUNCATE = 3 };
 int dkv_profile_read(dkv_cache* cache, int32_t kind, double* total_ms, int64_t* launches);
 
-/* Launch description of the last dkv_block_attention on this handle: the
- * kernel used (1 = mma.sync, 2 = tcgen05), its split count, and how many
- * kernels it launched. */
+/* Launch description of the last dkv_block_attention (or
+ * dkv_block_attention_dual, recorded on the prefix handle) on this handle:
+ * the kernel used (1 = mma.sync, 2 = tcgen05; the prefix's for a dual call),
+ * the split count (prefix + suffix splits for a dual call), and how many
+ * kernels it launched (attention, plus the combine unless one split wrote
+ * the output directly, plus the active-block rotation of a rotated-V cache;
+ * 3 for a dual call). */
 int dkv_last_attention_plan(const dkv_cache* cache, int32_t* kernel,
                             int32_t* splits, int32_t* launches);
 
