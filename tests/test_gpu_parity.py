@@ -157,6 +157,36 @@ def test_gqa_equals_mha_with_replicated_kv(dkv):
     assert np.all(np.abs(a - b) <= ulp + 1e-3)
 
 
+@pytest.mark.parametrize("kernel", [1, 2])
+def test_permuting_whole_groups_leaves_output(dkv, kernel):
+    """Committing whole K groups (here one block each) in another order gives
+    the same attention: both orders are within the output bound of the
+    oracle's value for the original order (the oracle's own invariance is a
+    CPU pin)."""
+    torch = _torch()
+    w = SHRUNK["batch32"].with_(k_group=32)
+    order = [5, 0, 3, 1, 4, 2]
+    cap = default_cap(w, len(order) + 1)
+    P = default_P(w, cap)
+    oc = oracle_cache(w, cap, P)
+    outs = []
+    Q = synth.queries_bits(w, 3)
+    Ka, Va = synth.active_block_bits(w, 3)
+    for blocks in (sorted(order), order):
+        cache = dkv.dkv_cache_alloc(gpu_config(dkv, w, cap, P))
+        dkv.dkv_cache_set_option(cache, dkv.DKV_OPT_ATTN_KERNEL, kernel)
+        commit_both(dkv, cache, oc if blocks is not order else None, w, blocks)
+        out = torch.empty((w.B, w.Hq, w.blk, w.d), dtype=torch.bfloat16, device="cuda")
+        dkv.dkv_block_attention(cache, dev_bf16(Q), dev_bf16(Ka), dev_bf16(Va), w.softmax_scale,
+                                out)
+        torch.cuda.synchronize()
+        outs.append(host_bits(out))
+        dkv.dkv_cache_free(cache)
+    ref = oc.block_attention(Q, Ka, Va, w.softmax_scale)
+    for o in outs:
+        assert_close(o, ref, f"kernel {kernel}")
+
+
 def test_all_protected_group_and_side_table_overflow(dkv):
     w = SHRUNK["tiny"].with_(prot_frac=0.0)
     cap, P = 256, 40
