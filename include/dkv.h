@@ -134,7 +134,8 @@ int dkv_block_attention(dkv_cache* cache, const void* q, const void* k_act,
  * commits).  out = softmax over all three segments, bidirectional, no mask;
  * each cache is dequantized with its own bit widths and groups (a bf16 suffix
  * uses bits = 16).  Arguments as in dkv_block_attention.  The two caches must
- * have the same batch, heads, head_dim and block; neither may rotate V
+ * be on the same device and have the same batch, heads, head_dim and block
+ * (else DKV_ERR_INVALID_ARG); neither may rotate V
  * (DKV_ERR_UNSUPPORTED), the suffix may not have a sink.  An empty suffix
  * gives exactly dkv_block_attention.  Launches: the split attention kernel on
  * each cache (the suffix with its own DKV_OPT_* choices) writing into the

@@ -452,6 +452,8 @@ int dkv_block_attention_dual(dkv_cache* c, dkv_cache* sfx, const void* q, const 
   const dkv::CacheView& vs = sfx->v;
   if (vs.B != v.B || vs.Hq != v.Hq || vs.Hkv != v.Hkv || vs.d != v.d || vs.blk != v.blk)
     return fail(DKV_ERR_INVALID_ARG, "prefix and suffix caches must share batch, heads, head_dim and block");
+  if (sfx->device != c->device)
+    return fail(DKV_ERR_INVALID_ARG, "prefix and suffix caches must be on the same device");
   if (v.vrot_b || vs.vrot_b)
     return fail(DKV_ERR_UNSUPPORTED, "dual-cache attention with rotated V is not supported");
   if (vs.sink > 0) return fail(DKV_ERR_UNSUPPORTED, "the suffix cache cannot have an attention sink");
