@@ -435,6 +435,52 @@ class OracleCache:
                     O[b, hq] = dense_attention_f64(Q[b, hq], Kall, Vall, scale)
         return O
 
+    def block_attention_selected(self, Q_bits, Kact_bits, Vact_bits, scale: float,
+                                 budget: int):
+        """Attention over a selection of the committed entries (MaskAhead
+        abstract: the current block's mask queries rank KV entries by their
+        estimated contribution to the attention output and select the ones
+        the block attends to; Q-MaskAhead does selection and attention
+        directly from the low-bit KV).  Readings (the abstract gives no
+        formula): for each (sequence, kv-head) every committed entry j gets
+        c_j = (sum over the group's query rows i of p_ij) * ||v_hat_j||_2,
+        with p_ij the softmax weight of key j for row i over all committed
+        and active keys, from the dequantized cache; the `budget` entries of
+        largest c_j are kept (ties: the lower position), and every row
+        attends to those entries plus the whole active block.
+        Returns (O [B, Hq, blk, d] fp64, selected positions per unit, sorted)."""
+        B, Hq, Hkv, blk, d = self.B, self.Hq, self.Hkv, self.blk, self.d
+        assert self.v_rot is None and budget >= 0
+        g = Hq // Hkv
+        Q = bf16_to_f64(np.asarray(Q_bits).reshape(B, Hq, blk, d))
+        Ka = bf16_to_f64(np.asarray(Kact_bits).reshape(B, Hkv, blk, d))
+        Va = bf16_to_f64(np.asarray(Vact_bits).reshape(B, Hkv, blk, d))
+        O = np.zeros((B, Hq, blk, d), np.float64)
+        selected = []
+        L = self.len
+        for b in range(B):
+            for h in range(Hkv):
+                u = b * Hkv + h
+                Kc, Vc = self.dequant_k(u), self.dequant_v(u)
+                Kall = np.concatenate([Kc, Ka[b, h]])
+                Vall = np.concatenate([Vc, Va[b, h]])
+                mass = np.zeros(L, np.float64)
+                for hq in range(h * g, (h + 1) * g):
+                    s = scale * (Q[b, hq] @ Kall.T)                  # [blk, L + blk]
+                    p = np.exp(s - s.max(axis=1, keepdims=True))
+                    p /= p.sum(axis=1, keepdims=True)
+                    mass += p[:, :L].sum(axis=0)
+                contrib = mass * np.linalg.norm(Vc, axis=1)
+                # largest first; equal contributions keep the lower position
+                order = np.lexsort((np.arange(L), -contrib))
+                sel = np.sort(order[:min(budget, L)])
+                selected.append(sel)
+                Ks = np.concatenate([Kc[sel], Ka[b, h]])
+                Vs = np.concatenate([Vc[sel], Va[b, h]])
+                for hq in range(h * g, (h + 1) * g):
+                    O[b, hq] = dense_attention_f64(Q[b, hq], Ks, Vs, scale)
+        return O, selected
+
     # -- canonical snapshot of the committed state (what an export returns)
     def snapshot(self) -> dict:
         L, GK = self.len, self.GK

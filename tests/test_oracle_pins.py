@@ -909,3 +909,160 @@ def test_dual_passthrough_is_dense_attention():
         for hq in range(h * 2, h * 2 + 2):
             want = dense_attention_f64(bf16_to_f64(Q[0, hq]), Kall, Vall, 0.1)
             np.testing.assert_allclose(got[0, hq], want, atol=1e-13)
+
+
+# ------------------------------------------------------------ MaskAhead selection
+
+def _sel_cache(kb=4, vb=4, n_blocks=6, seed=0):
+    w = synth.WORKLOADS["tiny"].with_(Hq=4, Hkv=2, k_bits=kb, v_bits=vb, prot_frac=0.02,
+                                      seed=seed)
+    oc = OracleCache(w.B, w.Hq, w.Hkv, w.d, w.blk, kb, vb, 32, 32, 64, (n_blocks + 1) * 32)
+    for i in range(n_blocks):
+        oc.commit(*synth.block_inputs(w, i))
+    return w, oc
+
+
+def test_selection_with_full_budget_is_plain_attention():
+    w, oc = _sel_cache()
+    Q = synth.queries_bits(w, 0)
+    Ka, Va = synth.active_block_bits(w, 0)
+    O, sel = oc.block_attention_selected(Q, Ka, Va, w.softmax_scale, oc.len + 5)
+    assert all(np.array_equal(s, np.arange(oc.len)) for s in sel)
+    assert np.array_equal(O, oc.block_attention(Q, Ka, Va, w.softmax_scale))
+
+
+def test_selection_with_zero_budget_attends_the_active_block_only():
+    w, oc = _sel_cache()
+    Q = synth.queries_bits(w, 1)
+    Ka, Va = synth.active_block_bits(w, 1)
+    O, sel = oc.block_attention_selected(Q, Ka, Va, w.softmax_scale, 0)
+    assert all(s.size == 0 for s in sel)
+    empty = OracleCache(w.B, w.Hq, w.Hkv, w.d, w.blk, 4, 4, 32, 32, 0, 64)
+    np.testing.assert_allclose(O, empty.block_attention(Q, Ka, Va, w.softmax_scale), atol=1e-13)
+
+
+def test_selection_finds_planted_heavy_hitters():
+    """Keys pointing along a direction every query shares, with ordinary
+    values, take almost all attention mass: exactly they are selected."""
+    r = np.random.default_rng(3)
+    d, blk, nb = 128, 32, 4
+    L = nb * blk
+    oc = OracleCache(1, 2, 1, d, blk, 16, 16, 32, 32, 0, L + blk)
+    e0 = np.zeros(d)
+    e0[0] = 1.0
+    T = np.sort(r.choice(L, 9, replace=False))
+    K = r.standard_normal((L, d)) * 0.1
+    K[:, 0] = 0.0
+    K[T] += 6.0 * e0
+    V = r.standard_normal((L, d))
+    for i in range(nb):
+        sl = slice(i * blk, (i + 1) * blk)
+        oc.commit(synth.f32_to_bf16_bits(K[sl].astype(np.float32))[None, None],
+                  synth.f32_to_bf16_bits(V[sl].astype(np.float32))[None, None])
+    q = r.standard_normal((1, 2, blk, d)) * 0.3
+    q[..., 0] = 1.0
+    Q = synth.f32_to_bf16_bits(q.astype(np.float32))
+    Ka = synth.f32_to_bf16_bits((r.standard_normal((1, 1, blk, d)) * 0.1).astype(np.float32))
+    Va = synth.f32_to_bf16_bits(r.standard_normal((1, 1, blk, d)).astype(np.float32))
+    _, sel = oc.block_attention_selected(Q, Ka, Va, 1.0, len(T))
+    assert np.array_equal(sel[0], T)
+
+
+def test_selection_ties_keep_the_lowest_positions():
+    """Zero queries give every key the same weight; V rows that differ only
+    in signs have the same norm: all contributions tie exactly."""
+    d, blk, nb = 128, 32, 3
+    L = nb * blk
+    r = np.random.default_rng(4)
+    base = r.standard_normal(d)
+    oc = OracleCache(1, 1, 1, d, blk, 16, 16, 32, 32, 0, L + blk)
+    for i in range(nb):
+        V = base[None] * r.choice([-1.0, 1.0], (blk, d))
+        K = r.standard_normal((blk, d))
+        oc.commit(synth.f32_to_bf16_bits(K.astype(np.float32))[None, None],
+                  synth.f32_to_bf16_bits(V.astype(np.float32))[None, None])
+    Q = np.zeros((1, 1, blk, d), np.uint16)
+    Ka = synth.f32_to_bf16_bits(r.standard_normal((1, 1, blk, d)).astype(np.float32))
+    _, sel = oc.block_attention_selected(Q, Ka, Ka, 1.0, 40)
+    assert np.array_equal(sel[0], np.arange(40))
+
+
+def test_selection_follows_entries_when_blocks_are_permuted():
+    w, oc = _sel_cache(kb=2, vb=4, n_blocks=5, seed=2)
+    order = [3, 0, 4, 1, 2]
+    oc2 = OracleCache(w.B, w.Hq, w.Hkv, w.d, w.blk, 2, 4, 32, 32, 64, 6 * 32)
+    for i in order:
+        oc2.commit(*synth.block_inputs(w, i))
+    Q = synth.queries_bits(w, 2)
+    Ka, Va = synth.active_block_bits(w, 2)
+    O1, s1 = oc.block_attention_selected(Q, Ka, Va, w.softmax_scale, 37)
+    O2, s2 = oc2.block_attention_selected(Q, Ka, Va, w.softmax_scale, 37)
+    np.testing.assert_allclose(O1, O2, atol=1e-12)
+    # position p of block order[p // 32] in the permuted cache is position
+    # order[p // 32] * 32 + p % 32 of the original
+    for a, b in zip(s1, s2):
+        mapped = np.sort(np.array([order[p // 32] * 32 + p % 32 for p in b]))
+        assert np.array_equal(a, mapped)
+
+
+def test_selection_by_contribution_beats_random_selection():
+    """What the ranking is for: with peaked attention, keeping the entries of
+    largest estimated contribution approximates full attention better than
+    keeping as many random entries."""
+    r = np.random.default_rng(5)
+    d, blk, nb = 128, 32, 8
+    L = nb * blk
+    oc = OracleCache(1, 4, 1, d, blk, 4, 4, 32, 32, 0, L + blk)
+    K = r.standard_normal((L, d))
+    K[r.choice(L, 24, replace=False)] *= 3.0
+    V = r.standard_normal((L, d))
+    for i in range(nb):
+        sl = slice(i * blk, (i + 1) * blk)
+        oc.commit(synth.f32_to_bf16_bits(K[sl].astype(np.float32))[None, None],
+                  synth.f32_to_bf16_bits(V[sl].astype(np.float32))[None, None])
+    Q = synth.f32_to_bf16_bits(r.standard_normal((1, 4, blk, d)).astype(np.float32))
+    Ka = synth.f32_to_bf16_bits(r.standard_normal((1, 1, blk, d)).astype(np.float32))
+    Va = synth.f32_to_bf16_bits(r.standard_normal((1, 1, blk, d)).astype(np.float32))
+    scale = 1.0 / np.sqrt(d)
+    full = oc.block_attention(Q, Ka, Va, scale)
+    O, _ = oc.block_attention_selected(Q, Ka, Va, scale, 64)
+    err_sel = np.abs(O - full).mean()
+    # random subsets of the same size, attended the same way
+    Kc, Vc = oc.dequant_k(0), oc.dequant_v(0)
+    Qf, Kaf, Vaf = bf16_to_f64(Q[0]), bf16_to_f64(Ka[0, 0]), bf16_to_f64(Va[0, 0])
+    errs = []
+    for t in range(5):
+        sub = np.sort(r.choice(L, 64, replace=False))
+        Ks, Vs = np.concatenate([Kc[sub], Kaf]), np.concatenate([Vc[sub], Vaf])
+        Or = np.stack([dense_attention_f64(Qf[h], Ks, Vs, scale) for h in range(4)])
+        errs.append(np.abs(Or - full[0]).mean())
+    assert err_sel < 0.5 * min(errs), (err_sel, errs)
+
+
+def test_selection_weighs_attention_mass_by_value_norm():
+    """Entries A take more attention mass but carry values near zero; entries
+    B take less mass with large values.  Their contribution to the output is
+    B's, so B is selected."""
+    r = np.random.default_rng(6)
+    d, blk, nb = 128, 32, 4
+    L = nb * blk
+    oc = OracleCache(1, 1, 1, d, blk, 16, 16, 32, 32, 0, L + blk)
+    idx = r.permutation(L)
+    A, B = np.sort(idx[:6]), np.sort(idx[6:12])
+    K = r.standard_normal((L, d)) * 0.05
+    K[:, 0] = 0.0
+    K[A, 0] = 4.0
+    K[B, 0] = 3.0
+    V = r.standard_normal((L, d)) * 0.05
+    V[A] *= 0.01
+    V[B] *= 100.0
+    for i in range(nb):
+        sl = slice(i * blk, (i + 1) * blk)
+        oc.commit(synth.f32_to_bf16_bits(K[sl].astype(np.float32))[None, None],
+                  synth.f32_to_bf16_bits(V[sl].astype(np.float32))[None, None])
+    q = np.zeros((1, 1, blk, d))
+    q[..., 0] = 1.0
+    Q = synth.f32_to_bf16_bits(q.astype(np.float32))
+    Ka = np.zeros((1, 1, blk, d), np.uint16)
+    _, sel = oc.block_attention_selected(Q, Ka, Ka, 2.0, 6)
+    assert np.array_equal(sel[0], B)
