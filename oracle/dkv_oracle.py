@@ -116,24 +116,46 @@ def quantize_groups(x: np.ndarray, keep: np.ndarray, bits: int):
 
 
 def pack_codes(codes: np.ndarray, bits: int) -> np.ndarray:
-    """Little-endian packing along the last axis: element e lands at bits
-    [bits*e mod 32, +bits) of word floor(bits*e / 32)."""
-    per = 32 // bits
+    """Little-endian packing along the last axis: element e occupies bits
+    [bits*e, bits*e + bits) of the bit stream formed by the words, where bit i
+    of the stream is bit (i mod 32) of word floor(i / 32).  For bits 2 and 4
+    no element crosses a word (element e sits at bits [bits*e mod 32, +bits)
+    of word floor(bits*e / 32)); 3-bit elements do (32 of them fill 3 words)."""
     c = np.asarray(codes, dtype=np.uint32)
     n = c.shape[-1]
-    assert n % per == 0
-    c = c.reshape(c.shape[:-1] + (n // per, per))
-    shifts = (np.arange(per, dtype=np.uint32) * np.uint32(bits))
-    return np.bitwise_or.reduce(c << shifts, axis=-1).astype(np.uint32)
+    assert (n * bits) % 32 == 0
+    if 32 % bits == 0:
+        per = 32 // bits
+        c = c.reshape(c.shape[:-1] + (n // per, per))
+        shifts = (np.arange(per, dtype=np.uint32) * np.uint32(bits))
+        return np.bitwise_or.reduce(c << shifts, axis=-1).astype(np.uint32)
+    c = c.astype(np.uint64)
+    words = np.zeros(c.shape[:-1] + (n * bits // 32,), np.uint64)
+    for e in range(n):
+        w, off = divmod(bits * e, 32)
+        words[..., w] |= (c[..., e] << np.uint64(off)) & np.uint64(0xFFFFFFFF)
+        if off + bits > 32:                      # the high bits go to the next word
+            words[..., w + 1] |= c[..., e] >> np.uint64(32 - off)
+    return words.astype(np.uint32)
 
 
 def unpack_codes(words: np.ndarray, bits: int, n: int) -> np.ndarray:
-    per = 32 // bits
     w = np.asarray(words, dtype=np.uint32)
-    shifts = (np.arange(per, dtype=np.uint32) * np.uint32(bits))
-    c = (w[..., None] >> shifts) & np.uint32(2 ** bits - 1)
-    c = c.reshape(w.shape[:-1] + (w.shape[-1] * per,))
-    return c[..., :n].astype(np.uint8)
+    if 32 % bits == 0:
+        per = 32 // bits
+        shifts = (np.arange(per, dtype=np.uint32) * np.uint32(bits))
+        c = (w[..., None] >> shifts) & np.uint32(2 ** bits - 1)
+        c = c.reshape(w.shape[:-1] + (w.shape[-1] * per,))
+        return c[..., :n].astype(np.uint8)
+    w = w.astype(np.uint64)
+    out = np.zeros(w.shape[:-1] + (n,), np.uint64)
+    for e in range(n):
+        i, off = divmod(bits * e, 32)
+        v = w[..., i] >> np.uint64(off)
+        if off + bits > 32:
+            v = v | (w[..., i + 1] << np.uint64(32 - off))
+        out[..., e] = v & np.uint64(2 ** bits - 1)
+    return out.astype(np.uint8)
 
 
 def mask_words_to_bool(words: np.ndarray, n: int) -> np.ndarray:
@@ -178,7 +200,7 @@ class OracleCache:
     def __init__(self, B, Hq, Hkv, d, blk, k_bits, v_bits, k_group, v_group,
                  max_protected, capacity, sink_tokens=0, v_rotation=None):
         assert Hq % Hkv == 0
-        assert k_bits in (2, 4, 16) and v_bits in (2, 4, 16)
+        assert k_bits in (2, 3, 4, 16) and v_bits in (2, 3, 4, 16)
         assert capacity % k_group == 0 and capacity % blk == 0
         assert d % v_group == 0
         self.B, self.Hq, self.Hkv, self.d, self.blk = B, Hq, Hkv, d, blk

@@ -88,7 +88,7 @@ def _random_groups(rng, G, n, outliers=True):
     return synth.bf16_bits_to_f32(synth.f32_to_bf16_bits(x))
 
 
-@pytest.mark.parametrize("bits", [2, 4])
+@pytest.mark.parametrize("bits", [2, 3, 4])
 def test_quantizer_extremes_and_error_bound(bits):
     rng = np.random.default_rng(bits)
     x = _random_groups(rng, 512, 32)
@@ -107,7 +107,7 @@ def test_quantizer_extremes_and_error_bound(bits):
     assert np.all(np.abs(x - xhat) <= bound[:, None])
 
 
-@pytest.mark.parametrize("bits", [2, 4])
+@pytest.mark.parametrize("bits", [2, 3, 4])
 def test_quantizer_picks_nearest_code_bruteforce(bits):
     rng = np.random.default_rng(100 + bits)
     x = _random_groups(rng, 64, 32)
@@ -173,7 +173,8 @@ def test_packing_hand_derived_words(case):
     assert unpack_codes(got, bits, len(codes)).tolist() == codes
 
 
-@pytest.mark.parametrize("bits,n", [(2, 32), (2, 64), (4, 32), (4, 64), (4, 128)])
+@pytest.mark.parametrize("bits,n", [(2, 32), (2, 64), (4, 32), (4, 64), (4, 128), (3, 32),
+                                    (3, 64), (3, 128)])
 def test_pack_unpack_roundtrip(bits, n):
     rng = np.random.default_rng(bits * n)
     c = rng.integers(0, 2 ** bits, (7, 5, n)).astype(np.uint8)
@@ -200,7 +201,7 @@ SMALL = synth.WORKLOADS["batch32"].with_(B=2, Hq=4, Hkv=2, L=256, prot_frac=0.05
 
 
 @pytest.mark.parametrize("kb,vb,gk,gv", [(4, 4, 32, 32), (2, 2, 64, 64), (2, 4, 128, 32),
-                                         (4, 2, 64, 128)])
+                                         (4, 2, 64, 128), (3, 3, 64, 32), (3, 4, 32, 128)])
 def test_incremental_commits_equal_one_shot(kb, vb, gk, gv):
     w, c = _cache(SMALL, k_bits=kb, v_bits=vb, k_group=gk, v_group=gv)
     n_blocks = w.L // w.blk + 1          # ends with an incomplete K group when gk > blk
@@ -397,7 +398,8 @@ def _grid_block(rng, blk, d, bits, GK, GV, prot_rows):
     return synth.f32_to_bf16_bits(K.astype(np.float32)), synth.f32_to_bf16_bits(V.astype(np.float32))
 
 
-@pytest.mark.parametrize("bits,GK,GV", [(4, 32, 32), (2, 32, 64), (2, 32, 32), (4, 32, 128)])
+@pytest.mark.parametrize("bits,GK,GV", [(4, 32, 32), (2, 32, 64), (2, 32, 32), (4, 32, 128),
+                                        (3, 32, 32), (3, 32, 128)])
 def test_grid_exact_cache_attention_equals_dense(bits, GK, GV):
     """Commit + dequant + attention in quantized mode equal dense attention
     over the original K/V when the inputs sit on each group's grid."""
