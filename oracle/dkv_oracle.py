@@ -529,6 +529,46 @@ class OracleCache:
         return out
 
 
+class OracleRaggedCache:
+    """Per-sequence committed lengths: each sequence of the batch commits its
+    own blocks (block-diffusion sequences of one batch finish blocks at
+    different steps), and each attends over its own committed tokens plus its
+    active block.  Reading: the batch is B single-sequence caches with one
+    shared configuration; a commit names the sequences it appends to."""
+
+    def __init__(self, B, Hq, Hkv, d, blk, k_bits, v_bits, k_group, v_group,
+                 max_protected, capacity, sink_tokens=0):
+        self.B, self.Hq, self.Hkv, self.d, self.blk = B, Hq, Hkv, d, blk
+        self.seqs = [OracleCache(1, Hq, Hkv, d, blk, k_bits, v_bits, k_group, v_group,
+                                 max_protected, capacity, sink_tokens) for _ in range(B)]
+
+    @property
+    def lens(self) -> list:
+        return [c.len for c in self.seqs]
+
+    def commit(self, K_bits, V_bits, protect_words=None, seqs=None) -> int:
+        """Append one block to the sequences listed in `seqs` (all if None);
+        K_bits, V_bits [B, Hkv, blk, d], protect_words [B, Hkv, blk/32]: the
+        rows of other sequences are ignored.  Returns the OR of the flags."""
+        K = np.asarray(K_bits, np.uint16)
+        V = np.asarray(V_bits, np.uint16)
+        flags = 0
+        for b in (range(self.B) if seqs is None else seqs):
+            pw = None if protect_words is None else np.asarray(protect_words)[b:b + 1]
+            flags |= self.seqs[b].commit(K[b:b + 1], V[b:b + 1], pw)
+        return flags
+
+    def truncate(self, b: int, new_len: int) -> None:
+        self.seqs[b].truncate(new_len)
+
+    def block_attention(self, Q_bits, Kact_bits, Vact_bits, scale: float) -> np.ndarray:
+        Q = np.asarray(Q_bits, np.uint16)
+        Ka = np.asarray(Kact_bits, np.uint16)
+        Va = np.asarray(Vact_bits, np.uint16)
+        return np.concatenate([c.block_attention(Q[b:b + 1], Ka[b:b + 1], Va[b:b + 1], scale)
+                               for b, c in enumerate(self.seqs)])
+
+
 def dense_attention_f64(q, K, V, scale) -> np.ndarray:
     """Textbook softmax attention in fp64: softmax_j(scale * <q_i, K_j>) V_j.
     q [n, d], K [m, d], V [m, d] -> [n, d].  Subtracting the row maximum

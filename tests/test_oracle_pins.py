@@ -1068,3 +1068,55 @@ def test_selection_weighs_attention_mass_by_value_norm():
     Ka = np.zeros((1, 1, blk, d), np.uint16)
     _, sel = oc.block_attention_selected(Q, Ka, Ka, 2.0, 6)
     assert np.array_equal(sel[0], B)
+
+
+# ------------------------------------------------------------ per-sequence lengths
+
+from oracle import OracleRaggedCache  # noqa: E402
+
+
+def _ragged_setup():
+    w = synth.WORKLOADS["tiny"].with_(B=3, Hq=4, Hkv=2, prot_frac=0.03, seed=5)
+    args = (w.B, w.Hq, w.Hkv, w.d, w.blk, w.k_bits, w.v_bits, 64, w.v_group, 32, 256)
+    return w, args
+
+
+def test_ragged_with_every_sequence_committing_is_the_batched_cache():
+    w, args = _ragged_setup()
+    rc, bc = OracleRaggedCache(*args), OracleCache(*args)
+    for i in range(5):
+        K, V, M = synth.block_inputs(w, i)
+        assert rc.commit(K, V, M) == bc.commit(K, V, M)
+    Q = synth.queries_bits(w, 0)
+    Ka, Va = synth.active_block_bits(w, 0)
+    np.testing.assert_allclose(rc.block_attention(Q, Ka, Va, 0.1),
+                               bc.block_attention(Q, Ka, Va, 0.1), atol=1e-13)
+    snap = bc.snapshot()
+    for b in range(w.B):
+        one = rc.seqs[b].snapshot()
+        units = slice(b * w.Hkv, (b + 1) * w.Hkv)
+        for key in ("k_codes", "k_sz", "v_codes", "v_sz", "k_tail", "prot_count"):
+            assert np.array_equal(one[key], snap[key][units]), key
+
+
+def test_each_sequence_sees_only_its_own_commits():
+    """Sequence b's output equals that of a one-sequence cache given only the
+    blocks b committed (its rows of those blocks), whatever the others did."""
+    w, args = _ragged_setup()
+    rc = OracleRaggedCache(*args)
+    plan = [[0, 1, 2], [0, 2], [1], [0, 1, 2], [2], [0]]     # sequences per commit
+    for i, seqs in enumerate(plan):
+        rc.commit(*synth.block_inputs(w, i), seqs=seqs)
+    assert rc.lens == [4 * 32, 3 * 32, 4 * 32]
+    Q = synth.queries_bits(w, 1)
+    Ka, Va = synth.active_block_bits(w, 1)
+    O = rc.block_attention(Q, Ka, Va, 0.1)
+    for b in range(w.B):
+        one = OracleCache(1, *args[1:])
+        for i, seqs in enumerate(plan):
+            if b in seqs:
+                K, V, M = synth.block_inputs(w, i)
+                one.commit(K[b:b + 1], V[b:b + 1], M[b:b + 1])
+        np.testing.assert_allclose(O[b:b + 1], one.block_attention(Q[b:b + 1], Ka[b:b + 1],
+                                                                   Va[b:b + 1], 0.1),
+                                   atol=1e-13)
