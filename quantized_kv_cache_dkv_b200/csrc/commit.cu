@@ -435,6 +435,9 @@ commit_kernel(CacheView c, const uint16_t* __restrict__ k, const uint16_t* __res
         }
         if (tid == 0) c.prot_gstart[size_t(u) * (c.nG + 1) + j + 1] = count;
       }
+      // every K thread has read prot_count and the tail mask before either
+      // is rewritten (named barrier over the 128 K threads only)
+      asm volatile("bar.sync 1, 128;" ::: "memory");
       if (tid == 0) c.prot_count[u] = count;
       if (tid < c.twords) tmask[tid] = 0u;
     }
