@@ -67,6 +67,21 @@ def test_bad_config_rejected_on_host(over, code):
     assert msg
 
 
+def test_valid_config_without_a_device_fails_cleanly():
+    """On a machine without a usable CUDA device a valid configuration passes
+    the host checks and then fails with DKV_ERR_CUDA and a message; no handle
+    is returned."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a CUDA device is present")
+    c = dkv.make_config(1, 4, 1, 128, 32, 4, 4, 32, 32, 0, 256)
+    h = ctypes.c_void_p(12345)
+    rc = dkv._alloc(ctypes.byref(c), None, ctypes.byref(h))
+    assert rc == dkv.DKV_ERR_CUDA
+    assert h.value is None
+    assert dkv._lib.dkv_last_error().decode()
+
+
 def test_null_arguments_rejected():
     P = ctypes.c_void_p
     assert dkv._commit(None, P(16), P(16), None, None) == dkv.DKV_ERR_INVALID_ARG
