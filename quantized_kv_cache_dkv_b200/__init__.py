@@ -3,6 +3,24 @@
 Every operation runs in the CUDA kernels of libdkv.so.  torch tensors carry
 device memory and the current CUDA stream; nothing here computes the method.
 Importing fails loudly when libdkv.so has not been built.
+
+One block-diffusion layer, in outline (bf16 tensors on the GPU; K, V and the
+active block are [B, Hkv, block, 128], queries and output [B, Hq, block, 128]):
+
+    cfg = make_config(B, Hq, Hkv, 128, block, k_bits=4, v_bits=4, k_group=32,
+                      v_group=32, max_protected=P, max_tokens=capacity)
+    cache = dkv_cache_alloc(cfg)
+    for each denoising step of the active block:
+        dkv_block_attention(cache, q, k_act, v_act, softmax_scale, out)
+    dkv_commit_block(cache, k_block, v_block, protect_words)  # block done
+    ...
+    flags = dkv_cache_status(cache)     # DKV_FLAG_* raised on the device
+    dkv_cache_free(cache)
+
+Variants: dkv_block_attention_dual (a second, suffix cache),
+dkv_cache_set_v_rotation (K-RPBH-rotated V, before the first commit),
+dkv_block_attention_noalloc (no allocation, for stream capture),
+dkv_cache_truncate (roll back to a prefix).
 """
 from __future__ import annotations
 
