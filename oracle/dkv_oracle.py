@@ -458,7 +458,7 @@ class OracleCache:
         return O
 
     def block_attention_selected(self, Q_bits, Kact_bits, Vact_bits, scale: float,
-                                 budget: int):
+                                 budget: int, selection=None):
         """Attention over a selection of the committed entries (MaskAhead
         abstract: the current block's mask queries rank KV entries by their
         estimated contribution to the attention output and select the ones
@@ -470,7 +470,11 @@ class OracleCache:
         and active keys, from the dequantized cache; the `budget` entries of
         largest c_j are kept (ties: the lower position), and every row
         attends to those entries plus the whole active block.
-        Returns (O [B, Hq, blk, d] fp64, selected positions per unit, sorted)."""
+        `selection` (a list of position arrays, one per unit) replaces the
+        ranking: the attention then runs over exactly those entries (to
+        check another implementation's output on its own selection).
+        Returns (O [B, Hq, blk, d] fp64, selected positions per unit, sorted,
+        contributions per unit [L])."""
         B, Hq, Hkv, blk, d = self.B, self.Hq, self.Hkv, self.blk, self.d
         assert self.v_rot is None and budget >= 0
         g = Hq // Hkv
@@ -478,7 +482,7 @@ class OracleCache:
         Ka = bf16_to_f64(np.asarray(Kact_bits).reshape(B, Hkv, blk, d))
         Va = bf16_to_f64(np.asarray(Vact_bits).reshape(B, Hkv, blk, d))
         O = np.zeros((B, Hq, blk, d), np.float64)
-        selected = []
+        selected, contribs = [], []
         L = self.len
         for b in range(B):
             for h in range(Hkv):
@@ -493,15 +497,19 @@ class OracleCache:
                     p /= p.sum(axis=1, keepdims=True)
                     mass += p[:, :L].sum(axis=0)
                 contrib = mass * np.linalg.norm(Vc, axis=1)
-                # largest first; equal contributions keep the lower position
-                order = np.lexsort((np.arange(L), -contrib))
-                sel = np.sort(order[:min(budget, L)])
+                contribs.append(contrib)
+                if selection is not None:
+                    sel = np.sort(np.asarray(selection[u], np.int64))
+                else:
+                    # largest first; equal contributions keep the lower position
+                    order = np.lexsort((np.arange(L), -contrib))
+                    sel = np.sort(order[:min(budget, L)])
                 selected.append(sel)
                 Ks = np.concatenate([Kc[sel], Ka[b, h]])
                 Vs = np.concatenate([Vc[sel], Va[b, h]])
                 for hq in range(h * g, (h + 1) * g):
                     O[b, hq] = dense_attention_f64(Q[b, hq], Ks, Vs, scale)
-        return O, selected
+        return O, selected, contribs
 
     # -- canonical snapshot of the committed state (what an export returns)
     def snapshot(self) -> dict:

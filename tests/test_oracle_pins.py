@@ -928,7 +928,7 @@ def test_selection_with_full_budget_is_plain_attention():
     w, oc = _sel_cache()
     Q = synth.queries_bits(w, 0)
     Ka, Va = synth.active_block_bits(w, 0)
-    O, sel = oc.block_attention_selected(Q, Ka, Va, w.softmax_scale, oc.len + 5)
+    O, sel, _ = oc.block_attention_selected(Q, Ka, Va, w.softmax_scale, oc.len + 5)
     assert all(np.array_equal(s, np.arange(oc.len)) for s in sel)
     assert np.array_equal(O, oc.block_attention(Q, Ka, Va, w.softmax_scale))
 
@@ -937,7 +937,7 @@ def test_selection_with_zero_budget_attends_the_active_block_only():
     w, oc = _sel_cache()
     Q = synth.queries_bits(w, 1)
     Ka, Va = synth.active_block_bits(w, 1)
-    O, sel = oc.block_attention_selected(Q, Ka, Va, w.softmax_scale, 0)
+    O, sel, _ = oc.block_attention_selected(Q, Ka, Va, w.softmax_scale, 0)
     assert all(s.size == 0 for s in sel)
     empty = OracleCache(w.B, w.Hq, w.Hkv, w.d, w.blk, 4, 4, 32, 32, 0, 64)
     np.testing.assert_allclose(O, empty.block_attention(Q, Ka, Va, w.softmax_scale), atol=1e-13)
@@ -966,7 +966,7 @@ def test_selection_finds_planted_heavy_hitters():
     Q = synth.f32_to_bf16_bits(q.astype(np.float32))
     Ka = synth.f32_to_bf16_bits((r.standard_normal((1, 1, blk, d)) * 0.1).astype(np.float32))
     Va = synth.f32_to_bf16_bits(r.standard_normal((1, 1, blk, d)).astype(np.float32))
-    _, sel = oc.block_attention_selected(Q, Ka, Va, 1.0, len(T))
+    _, sel, _ = oc.block_attention_selected(Q, Ka, Va, 1.0, len(T))
     assert np.array_equal(sel[0], T)
 
 
@@ -985,7 +985,7 @@ def test_selection_ties_keep_the_lowest_positions():
                   synth.f32_to_bf16_bits(V.astype(np.float32))[None, None])
     Q = np.zeros((1, 1, blk, d), np.uint16)
     Ka = synth.f32_to_bf16_bits(r.standard_normal((1, 1, blk, d)).astype(np.float32))
-    _, sel = oc.block_attention_selected(Q, Ka, Ka, 1.0, 40)
+    _, sel, _ = oc.block_attention_selected(Q, Ka, Ka, 1.0, 40)
     assert np.array_equal(sel[0], np.arange(40))
 
 
@@ -997,8 +997,8 @@ def test_selection_follows_entries_when_blocks_are_permuted():
         oc2.commit(*synth.block_inputs(w, i))
     Q = synth.queries_bits(w, 2)
     Ka, Va = synth.active_block_bits(w, 2)
-    O1, s1 = oc.block_attention_selected(Q, Ka, Va, w.softmax_scale, 37)
-    O2, s2 = oc2.block_attention_selected(Q, Ka, Va, w.softmax_scale, 37)
+    O1, s1, _ = oc.block_attention_selected(Q, Ka, Va, w.softmax_scale, 37)
+    O2, s2, _ = oc2.block_attention_selected(Q, Ka, Va, w.softmax_scale, 37)
     np.testing.assert_allclose(O1, O2, atol=1e-12)
     # position p of block order[p // 32] in the permuted cache is position
     # order[p // 32] * 32 + p % 32 of the original
@@ -1027,7 +1027,7 @@ def test_selection_by_contribution_beats_random_selection():
     Va = synth.f32_to_bf16_bits(r.standard_normal((1, 1, blk, d)).astype(np.float32))
     scale = 1.0 / np.sqrt(d)
     full = oc.block_attention(Q, Ka, Va, scale)
-    O, _ = oc.block_attention_selected(Q, Ka, Va, scale, 64)
+    O, _, _ = oc.block_attention_selected(Q, Ka, Va, scale, 64)
     err_sel = np.abs(O - full).mean()
     # random subsets of the same size, attended the same way
     Kc, Vc = oc.dequant_k(0), oc.dequant_v(0)
@@ -1066,7 +1066,7 @@ def test_selection_weighs_attention_mass_by_value_norm():
     q[..., 0] = 1.0
     Q = synth.f32_to_bf16_bits(q.astype(np.float32))
     Ka = np.zeros((1, 1, blk, d), np.uint16)
-    _, sel = oc.block_attention_selected(Q, Ka, Ka, 2.0, 6)
+    _, sel, _ = oc.block_attention_selected(Q, Ka, Ka, 2.0, 6)
     assert np.array_equal(sel[0], B)
 
 
@@ -1120,3 +1120,20 @@ def test_each_sequence_sees_only_its_own_commits():
         np.testing.assert_allclose(O[b:b + 1], one.block_attention(Q[b:b + 1], Ka[b:b + 1],
                                                                    Va[b:b + 1], 0.1),
                                    atol=1e-13)
+
+
+def test_selection_given_explicitly_reproduces_the_ranking():
+    """Passing the ranking's own selection back gives the same output; a
+    different selection of the same size gives another output."""
+    w, oc = _sel_cache(seed=7)
+    Q = synth.queries_bits(w, 3)
+    Ka, Va = synth.active_block_bits(w, 3)
+    O, sel, contrib = oc.block_attention_selected(Q, Ka, Va, w.softmax_scale, 48)
+    O2, sel2, _ = oc.block_attention_selected(Q, Ka, Va, w.softmax_scale, 48, selection=sel)
+    assert np.array_equal(O, O2) and all(np.array_equal(a, b) for a, b in zip(sel, sel2))
+    # the selected entries hold the 48 largest contributions
+    for s, c in zip(sel, contrib):
+        assert c[s].min() >= np.sort(c)[-48]
+    other = [np.sort(np.setdiff1d(np.arange(oc.len), s))[:48] for s in sel]
+    O3, _, _ = oc.block_attention_selected(Q, Ka, Va, w.softmax_scale, 48, selection=other)
+    assert not np.allclose(O, O3)
