@@ -107,3 +107,36 @@ def test_package_refuses_to_load_without_library(tmp_path):
     r = subprocess.run([sys.executable, "-c", "import quantized_kv_cache_dkv_b200"],
                        cwd=tmp_path, capture_output=True, text=True)
     assert r.returncode != 0 and "libdkv.so is missing" in r.stderr
+
+
+def test_header_is_plain_c_and_links_from_c(tmp_path):
+    """include/dkv.h compiles as strict C99, and a C program links against
+    libdkv.so and gets the documented host-side error codes (no GPU call)."""
+    import os
+    import shutil
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    src = tmp_path / "abi_check.c"
+    src.write_text(
+        '#include <stdio.h>\n#include <string.h>\n#include "dkv.h"\n'
+        "int main(void) {\n"
+        "  int64_t n = 0;\n"
+        "  if (dkv_cache_len(0, &n) != DKV_ERR_INVALID_ARG) return 1;\n"
+        "  if (strlen(dkv_last_error()) == 0) return 2;\n"
+        "  if (dkv_cache_free(0) != DKV_ERR_INVALID_ARG) return 3;\n"
+        "  dkv_config c; memset(&c, 0, sizeof c);\n"
+        "  dkv_cache* h = 0;\n"
+        "  if (dkv_cache_alloc(&c, 0, &h) != DKV_ERR_INVALID_ARG || h != 0) return 4;\n"
+        '  printf("ok\\n");\n  return 0;\n}\n')
+    exe = tmp_path / "abi_check"
+    libdir = os.path.dirname(dkv.LIB_PATH)
+    libname = os.path.basename(dkv.LIB_PATH)
+    r = subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                        "-I", os.path.join(root, "include"), str(src), "-o", str(exe),
+                        os.path.join(libdir, libname), "-Wl,-rpath," + libdir],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", (r.returncode, r.stdout, r.stderr)
