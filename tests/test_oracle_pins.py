@@ -1137,3 +1137,24 @@ def test_selection_given_explicitly_reproduces_the_ranking():
     other = [np.sort(np.setdiff1d(np.arange(oc.len), s))[:48] for s in sel]
     O3, _, _ = oc.block_attention_selected(Q, Ka, Va, w.softmax_scale, 48, selection=other)
     assert not np.allclose(O, O3)
+
+
+def test_dual_with_a_sink_in_the_prefix_equals_one_cache():
+    """The prefix's sink positions keep full precision; the suffix has none.
+    With one-block K groups the combined cache (sink at its start, the
+    suffix appended) dequantizes to the same entries."""
+    w = synth.WORKLOADS["tiny"].with_(Hq=4, Hkv=2, k_bits=2, v_bits=2, prot_frac=0.02, seed=11)
+    mk = lambda cap, sink: OracleCache(w.B, w.Hq, w.Hkv, w.d, w.blk, 2, 2, 32, 32, 96, cap, sink)
+    pre, suf, one = mk(256, 40), mk(128, 0), mk(384, 40)
+    for i in range(4):
+        K, V, M = synth.block_inputs(w, i)
+        pre.commit(K, V, M)
+        one.commit(K, V, M)
+    for i in range(4, 7):
+        K, V, M = synth.block_inputs(w, i)
+        suf.commit(K, V, M)
+        one.commit(K, V, M)
+    Q = synth.queries_bits(w, 4)
+    Ka, Va = synth.active_block_bits(w, 4)
+    np.testing.assert_allclose(pre.block_attention_dual(suf, Q, Ka, Va, 0.1),
+                               one.block_attention(Q, Ka, Va, 0.1), atol=1e-13)
