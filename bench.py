@@ -216,7 +216,7 @@ def io_bytes(w: synth.Workload) -> float:
 
 
 def run_gpu(w: synth.Workload, K: int, W: int, want_e2e=True, log=print, kernel=0,
-            v_rotation=0, suffix=0):
+            v_rotation=0, suffix=0, time_build=False):
     import torch
     import quantized_kv_cache_dkv_b200 as dkv
 
@@ -260,11 +260,14 @@ def run_gpu(w: synth.Workload, K: int, W: int, want_e2e=True, log=print, kernel=
 
     t0 = time.time()
     nb = w.L // w.blk
+    kept = []
     for i in range(nb):
         K_, V_, M_ = synth.block_inputs(w, i)
         Kd, Vd, Md = up(K_), up(V_), upw(M_)
         for c in caches:
             dkv.dkv_commit_block(c, Kd, Vd, Md)
+        if time_build:
+            kept.append((Kd, Vd, Md))
     for i in range(suffix // w.blk):
         K_, V_, M_ = synth.block_inputs(w, 100000 + i)
         Kd, Vd, Md = up(K_), up(V_), upw(M_)
@@ -272,6 +275,35 @@ def run_gpu(w: synth.Workload, K: int, W: int, want_e2e=True, log=print, kernel=
             dkv.dkv_commit_block(c, Kd, Vd, Md)
     torch.cuda.synchronize()
     t_prefill = time.time() - t0
+    build = None
+    if time_build:
+        # The whole cache built again by its nb commits, captured in one CUDA
+        # graph: rolled back to 0 first, so every replay starts from an empty
+        # cache and rewrites the same state as the eager build above.
+        dkv.dkv_cache_truncate(caches[0], 0)
+        gb = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gb):
+            for Kd, Vd, Md in kept:
+                dkv.dkv_commit_block(caches[0], Kd, Vd, Md)
+        gb.replay()
+        torch.cuda.synchronize()
+        times = []
+        eb0 = torch.cuda.Event(enable_timing=True)
+        eb1 = torch.cuda.Event(enable_timing=True)
+        for _ in range(3):
+            eb0.record()
+            gb.replay()
+            eb1.record()
+            torch.cuda.synchronize()
+            times.append(eb0.elapsed_time(eb1))
+        bms = statistics.median(times)
+        build = {"commits": nb, "tokens": nb * w.blk, "ms": round(bms, 4),
+                 "us_per_commit": round(bms * 1e3 / nb, 3),
+                 "tokens_per_s": round(w.B * nb * w.blk / (bms / 1e3), 1),
+                 "method": "all commits captured in one CUDA graph; median of 3 replays "
+                           "(CUDA events)"}
+        del gb
+        kept.clear()
 
     def attend(r, q, ka, va, out):
         if sfx:
@@ -381,6 +413,14 @@ def run_gpu(w: synth.Workload, K: int, W: int, want_e2e=True, log=print, kernel=
         dkv.dkv_cache_set_option(c, dkv.DKV_OPT_PROFILE, 0)
     Lp = step_lengths(w, Kp, R)
     att_ms, att_n = prof["attention"]
+    # The timed region is a CUDA-graph replay whose kernels overlap their
+    # launch with the previous kernel (programmatic dependent launch), so the
+    # eager per-launch times above do not add up to its step time.  Each
+    # kernel's time in the timed execution is the graph's step time times that
+    # kernel's share of the eager device time.
+    eager_tot = sum(v[0] for v in prof.values())
+    share = {k: (v[0] / eager_tot if eager_tot > 0 else 0.0) for k, v in prof.items()}
+    step_ms_graph = ms / K
     # (a dual-cache step launches the attention kernel twice: its bytes and
     # flops are those of both launches, averaged per launch below)
     att_bytes = sum(attn_bytes(w, L + w.blk) + sfx_bytes for L in Lp)
@@ -523,13 +563,23 @@ def run_gpu(w: synth.Workload, K: int, W: int, want_e2e=True, log=print, kernel=
         "att_ms": att_ms, "att_n": att_n, "att_bytes": att_bytes, "att_flops": att_flops,
         "combine_ms": prof["combine"][0], "combine_n": prof["combine"][1],
         "commit_ms": com_ms, "commit_n": com_n, "e2e": e2e, "L_mean": sum(Ls) / len(Ls) + w.blk,
-        "step_bytes": step_bytes / K,
+        "step_bytes": step_bytes / K, "build": build, "Kp": Kp, "share": share,
+        # per-launch times in the timed (graph) execution
+        "att_us_graph": step_ms_graph * share["attention"] * Kp / max(att_n, 1) * 1e3,
+        "commit_us_graph": step_ms_graph * share["commit"] * Kp / max(com_n, 1) * 1e3,
+        "combine_us_graph": step_ms_graph * share["combine"] * Kp / max(prof["combine"][1], 1) * 1e3,
     }
 
 
+TIMING_METHOD = ("step time: CUDA events around one CUDA-graph replay of the K timed steps; "
+                 "per-kernel time in that execution = step time x the kernel's share of device "
+                 "time in an eager pass of the same steps with CUDA events around each launch")
+
+
 def roofline(w: synth.Workload, r: dict, peaks: dict, peak_kind: str, traffic):
-    """Roofline of the dominant kernel (the split attention kernel)."""
-    avg_s = r["att_ms"] / max(r["att_n"], 1) / 1e3
+    """Roofline of the dominant kernel (the split attention kernel), at its
+    per-launch time in the timed (graph) execution."""
+    avg_s = r["att_us_graph"] / 1e6
     bytes_launch = r["att_bytes"] / max(r["att_n"], 1)
     flops_launch = r["att_flops"] / max(r["att_n"], 1)
     ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
@@ -547,6 +597,8 @@ def roofline(w: synth.Workload, r: dict, peaks: dict, peak_kind: str, traffic):
             "frac": round(ach / peak, 4), "traffic": tr,
             "peak_source": f"{peak_kind} ({'hbm_gbs' if bound == 'hbm' else 'bf16_tflops burst'})",
             "kernel": "attention split kernel", "avg_launch_us": round(avg_s * 1e6, 3),
+            "avg_launch_us_eager": round(r["att_ms"] / max(r["att_n"], 1) * 1e3, 3),
+            "share_of_step": round(r["share"]["attention"], 4),
             "algorithmic_bytes_per_launch": int(bytes_launch),
             "algorithmic_flops_per_launch": int(flops_launch),
             "hbm_gbs_at_kernel": round(bytes_launch / avg_s / 1e9, 1),
@@ -572,7 +624,7 @@ def oracle_sample(w: synth.Workload, seconds: float, max_steps=None, warmup=0):
     from oracle import OracleCache
     nb = w.L // w.blk
     C = cycle_len(w)
-    units = [(0, 0)] if w.L >= 16384 else [(0, 0), (w.B - 1, w.Hkv - 1)]
+    units = [(0, 0)] if w.L >= 16384 or w.B * w.Hkv == 1 else [(0, 0), (w.B - 1, w.Hkv - 1)]
     cap = w.L + C * w.blk + max(w.k_group, w.blk)
     P = int(round(w.prot_frac * cap)) * 2 + 64
     ocs = []
@@ -640,15 +692,36 @@ def base_line(w, args, value, ms_per_step, world):
     }
 
 
+def kernel_fields(w: synth.Workload, r: dict) -> dict:
+    """Per-kernel figures of one run: times in the timed (graph) execution
+    and in the eager pass, commit rate, launch plan."""
+    att_us = r["att_us_graph"]
+    return {
+        "attention_gbs": round(r["att_bytes"] / max(r["att_n"], 1) / (att_us / 1e6) / 1e9, 1),
+        "pct_of_8tbs": round(100 * r["att_bytes"] / max(r["att_n"], 1) / (att_us / 1e6) / 8e12, 2),
+        "commit_tokens_per_s": round(w.B * w.blk / (r["commit_us_graph"] / 1e6), 1)
+        if r["commit_us_graph"] > 0 else None,
+        "kernel_us": {"attention": round(att_us, 3), "combine": round(r["combine_us_graph"], 3),
+                      "commit": round(r["commit_us_graph"], 3)},
+        "kernel_us_eager": {"attention": round(r["att_ms"] / max(r["att_n"], 1) * 1e3, 3),
+                            "combine": round(r["combine_ms"] / max(r["combine_n"], 1) * 1e3, 3),
+                            "commit": round(r["commit_ms"] / max(r["commit_n"], 1) * 1e3, 3)},
+        "attention_plan": {"kernel": ["", "mma.sync", "tcgen05"][r["plan"][0]],
+                           "splits": r["plan"][1], "launches": r["plan"][2]},
+    }
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=64)
     ap.add_argument("--warmup", type=int, default=4)
     ap.add_argument("--impl", choices=["dkv", "reference"], default="dkv")
-    ap.add_argument("--workload", default="mha8b", choices=list(synth.WORKLOADS))
-    ap.add_argument("--all-workloads", action="store_true",
-                    help="also run the other workloads and add a summary per workload")
+    ap.add_argument("--workload", default="batch32", choices=list(synth.WORKLOADS),
+                    help="the line's workload (default: the batch-32 decode profile, the "
+                         "largest single-GPU configuration)")
+    ap.add_argument("--no-sub-records", action="store_true",
+                    help="skip the per-workload records of the other configurations")
     ap.add_argument("--kernel", type=int, default=0, choices=[0, 1, 2],
                     help="attention kernel: 0 = library's choice, 1 = mma.sync, 2 = tcgen05")
     ap.add_argument("--B", type=int, default=0, help="override the workload's batch (profiling)")
@@ -696,7 +769,8 @@ def main():
     if args.suffix % w.blk:
         raise SystemExit("--suffix must be a multiple of the block")
     r = run_gpu(w, args.steps, args.warmup, log=lambda *a: None, kernel=args.kernel,
-                v_rotation=args.v_rotation, suffix=args.suffix)
+                v_rotation=args.v_rotation, suffix=args.suffix,
+                time_build=(w.name == "longprompt"))
     line = base_line(w, args, r["value"], r["ms"] / args.steps, world)
     if args.v_rotation:
         line["config"]["v_rotation"] = f"K-RPBH, Hadamard block {args.v_rotation}"
@@ -707,38 +781,39 @@ def main():
     line["config"]["L_mean"] = r["L_mean"]
     line["config"]["step"] = (f"1 commit + 1 attention; truncate to L every {r['C']} steps; "
                               "timed region = one CUDA graph replay of the steps")
+    line["config"]["timing"] = TIMING_METHOD
     line["roofline"] = roofline(w, r, peaks, peak_kind, traffic)
     if args.suffix:  # the recorded traffic is that of the single-cache launch
         line["roofline"]["traffic"] = None
     line["clocks"] = r["clocks"]
     line["e2e"] = r["e2e"]
     line["gpu_launches"] = r["graph_launches"]
-    line["attention_gbs"] = round(r["att_bytes"] / (r["att_ms"] / 1e3) / 1e9, 1)
-    line["pct_of_8tbs"] = round(100 * line["attention_gbs"] / 8000.0, 2)
-    line["commit_tokens_per_s"] = round(w.B * w.blk * r["commit_n"] / (r["commit_ms"] / 1e3), 1) \
-        if r["commit_ms"] > 0 else None
-    line["kernel_ms"] = {"attention": round(r["att_ms"] / max(r["att_n"], 1), 5),
-                         "combine": round(r["combine_ms"] / max(r["combine_n"], 1), 5),
-                         "commit": round(r["commit_ms"] / max(r["commit_n"], 1), 5)}
-    line["attention_plan"] = {"kernel": ["", "mma.sync", "tcgen05"][r["plan"][0]],
-                              "splits": r["plan"][1], "launches": r["plan"][2]}
-    if args.all_workloads:
+    line.update(kernel_fields(w, r))
+    if r["build"]:
+        line["build"] = r["build"]
+    if not args.no_sub_records:
+        # every other configuration of the workload set, each with its own
+        # roofline (same timing method, no end-to-end or oracle leg)
         line["workloads"] = {}
         for name in synth.WORKLOAD_ORDER:
             if name == w.name:
                 continue
             ww = synth.WORKLOADS[name]
-            kern = args.kernel if (args.kernel != 2 or ww.rows == 128) else 0
-            rr = run_gpu(ww, min(args.steps, 16), args.warmup, want_e2e=False, kernel=kern)
-            rf = roofline(ww, rr, peaks, peak_kind, traffic)
-            line["workloads"][name] = {
-                "value_gbs": round(rr["value"], 1),
-                "attention_gbs": round(rr["att_bytes"] / (rr["att_ms"] / 1e3) / 1e9, 1),
-                "attention_us": round(rr["att_ms"] / max(rr["att_n"], 1) * 1e3, 2),
-                "roofline": {k: rf[k] for k in ("bound", "achieved", "peak", "unit", "frac")},
-                "commit_tokens_per_s": round(ww.B * ww.blk * rr["commit_n"] /
-                                             (rr["commit_ms"] / 1e3), 1),
-                "plan": rr["plan"], "clocks_sm_mhz": (rr["clocks"] or {}).get("sm_mhz")}
+            kern = args.kernel if (args.kernel != 2 or ww.rows % 32 == 0) else 0
+            rr = run_gpu(ww, args.steps, args.warmup, want_e2e=False, kernel=kern,
+                         time_build=(name == "longprompt"))
+            rec = {"value_gbs": round(rr["value"], 1),
+                   "ms_per_step": round(rr["ms"] / args.steps, 6),
+                   "config": {k: getattr(ww, k) for k in ("B", "Hq", "Hkv", "L", "k_bits",
+                                                          "v_bits", "k_group", "v_group",
+                                                          "prot_frac")},
+                   "roofline": roofline(ww, rr, peaks, peak_kind, traffic),
+                   "clocks_sm_mhz": (rr["clocks"] or {}).get("sm_mhz"),
+                   "clock_reasons": (rr["clocks"] or {}).get("reasons")}
+            rec.update(kernel_fields(ww, rr))
+            if rr["build"]:
+                rec["build"] = rr["build"]
+            line["workloads"][name] = rec
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.v_rotation \
             and not args.suffix:
         gbs, steps, el, desc = oracle_sample(w, args.cpu_seconds)

@@ -32,8 +32,9 @@
  *     export synchronize `stream`.
  *   - Caller buffers are device memory (cudaMalloc or torch), contiguous,
  *     16-byte aligned, bf16 = IEEE bfloat16 bit patterns.  The library keeps
- *     no caller pointer past the call.  Calls on the current CUDA device,
- *     which must be the one the cache was allocated on.
+ *     no caller pointer past the call.  Commit and attention calls run on the
+ *     current CUDA device, which must be the one the cache was allocated on
+ *     (else DKV_ERR_INVALID_ARG).
  *   - Errors found while kernels run (protected side table full, committed
  *     value out of fp16 range) are sticky flags read by dkv_cache_status.
  */
@@ -264,8 +265,16 @@ int dkv_cache_export(dkv_cache* cache, void* stream, dkv_export* out);
  *     rounding for any split count.
  *   DKV_OPT_ATTN_KERNEL: 0 = best available (default), 1 = warp-level
  *     mma.sync kernel, 2 = tcgen05 tensor-memory kernel (DKV_ERR_UNSUPPORTED
- *     if the shape has no tcgen05 variant). */
-enum { DKV_OPT_SPLITS = 1, DKV_OPT_ATTN_KERNEL = 2, DKV_OPT_PROFILE = 3 };
+ *     if the shape has no tcgen05 variant).
+ *   DKV_OPT_TEST_STALL: bounds-checking build (libdkv_bc.so) only, else
+ *     DKV_ERR_UNSUPPORTED.  A test of the bounded waits: value t >= 0 makes the
+ *     tcgen05 kernel's loader withhold the copies of tile t (0 = the first
+ *     tile of each CTA's token range), so the waits on that stage run out;
+ *     while it is set every bounded wait gives up after 2 ms instead of about
+ *     1 s.  The call then raises DKV_FLAG_TIMEOUT, every CTA leaves its
+ *     loops, waits for its own copies and MMAs in flight and frees its tensor
+ *     memory; the output is undefined.  -1 (default) turns it off. */
+enum { DKV_OPT_SPLITS = 1, DKV_OPT_ATTN_KERNEL = 2, DKV_OPT_PROFILE = 3, DKV_OPT_TEST_STALL = 4 };
 int dkv_cache_set_option(dkv_cache* cache, int32_t key, int64_t value);
 
 /* With DKV_OPT_PROFILE = 1, every kernel launch on this handle (outside CUDA

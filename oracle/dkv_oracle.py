@@ -8,8 +8,8 @@ tables); the two meet only through the seeded inputs of the `synth` module and
 the canonical cache layout written out below.
 
 What it follows (the pages print no formula, kernel or bit layout; the
-textbook meaning of the names they use is taken, and every reading is listed
-in DESIGN.md):
+textbook meaning of the names they use is taken, and each reading of a step
+the pages leave open is stated beside the function that takes it):
 
 * "SoloQ: Calibration-Free Quantization for Diffusion Language Models"
   (block-diffusion paragraph): KV entries are quantized only when a block is

@@ -45,7 +45,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 DKV_OK, DKV_ERR_INVALID_ARG, DKV_ERR_UNSUPPORTED, DKV_ERR_CAPACITY, DKV_ERR_CUDA = 0, 1, 2, 3, 4
 DKV_FLAG_CAPACITY, DKV_FLAG_RANGE, DKV_FLAG_TIMEOUT, DKV_FLAG_BOUNDS = 0x1, 0x2, 0x4, 0x8
-DKV_OPT_SPLITS, DKV_OPT_ATTN_KERNEL, DKV_OPT_PROFILE = 1, 2, 3
+DKV_OPT_SPLITS, DKV_OPT_ATTN_KERNEL, DKV_OPT_PROFILE, DKV_OPT_TEST_STALL = 1, 2, 3, 4
 DKV_KERNEL_ATTENTION, DKV_KERNEL_COMBINE, DKV_KERNEL_COMMIT, DKV_KERNEL_TRUNCATE = 0, 1, 2, 3
 
 

@@ -15,14 +15,14 @@ namespace {
 constexpr size_t kScratchBytes = DKV_NOALLOC_SCRATCH_BYTES;
 constexpr int kMaxDevices = 64;
 
-// Split partials: [U][splits][rows][d] fp32, then [U][splits][rows] float2.
-// Host code must not use this name as an address: it is a host-side stand-in.
+// Split partials, laid out as the handle's workspace (split_o_bytes of fp32
+// partial outputs, then split_ml_bytes of (max, sum) pairs).  Host code must
+// not use this name as an address: it is a host-side stand-in.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
 std::mutex g_mu;
 void* g_scratch_addr[kMaxDevices] = {};  // device address per device ordinal
 
-size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 }  // namespace
@@ -40,11 +40,13 @@ extern "C" int dkv_block_attention_noalloc(dkv_cache* cache, const void* q, cons
   if (!(softmax_scale == softmax_scale) || softmax_scale > 3.0e38f || softmax_scale < -3.0e38f)
     return report_error(DKV_ERR_INVALID_ARG, "softmax_scale must be finite");
 
-  // once per device, with that device current: the buffer's device address
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return report_error(DKV_ERR_CUDA, cudaGetErrorString(e));
+  // the call runs on the cache's device, which must be the current one (the
+  // static buffer exists once per device)
+  const int drc = dkv::check_device(ci);
+  if (drc != DKV_OK) return drc;
+  const int dev = ci.device;
   if (dev < 0 || dev >= kMaxDevices) return report_error(DKV_ERR_UNSUPPORTED, "device ordinal >= 64");
+  cudaError_t e = cudaSuccess;
   void* scratch = nullptr;
   {
     std::lock_guard<std::mutex> lk(g_mu);
@@ -75,9 +77,8 @@ extern "C" int dkv_block_attention_noalloc(dkv_cache* cache, const void* q, cons
   if (prc != DKV_OK) return report_error(prc, perr);
 
   if (!a.final_out) {
-    const size_t rows_total = size_t(v.U) * size_t(a.nsplit) * size_t(v.rows);
-    const size_t o_bytes = align256(rows_total * size_t(dkv::kHeadDim) * sizeof(float));
-    const size_t need = o_bytes + rows_total * sizeof(float2);
+    const size_t o_bytes = dkv::split_o_bytes(v.U, a.nsplit, v.rows);
+    const size_t need = o_bytes + dkv::split_ml_bytes(v.U, a.nsplit, v.rows);
     if (need > kScratchBytes)
       return report_error(
           DKV_ERR_UNSUPPORTED,

@@ -57,7 +57,6 @@ constexpr int kStages = 3;  // ring of packed tiles
 constexpr int kStagedProt = 24;  // protected K rows staged per tile (more: read from global)
 constexpr uint32_t kTileBytes = 128 * 128 * 2;
 constexpr uint32_t kColO = 0, kColS0 = 128, kColS1 = 256, kColQ = 384, kTmemCols = 512;
-constexpr uint64_t kTimeoutNs = 1000000000ull;
 
 // instruction descriptor: D f32, A f16 (K-major), B f16 (MN-major), M = N = 128
 constexpr uint32_t kIdesc = (1u << 4) | (0u << 7) | (0u << 10) | (0u << 15) | (1u << 16) |
@@ -131,11 +130,13 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
 }
 
 // Waits for the phase of `parity`; false on abort (unless drain) or after
-// ~1 s (then the CTA-wide abort flag and the sticky timeout flag are set).
-// `drain` waits that ignore the abort flag are used only for the CTA's own
-// copies and MMAs in flight before it releases shared and tensor memory.
-__device__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                          uint32_t* status, bool drain = false) {
+// a.wait_limit_ns (about 1 s; then the CTA-wide abort flag and the sticky
+// timeout flag are set).  `drain` waits that ignore the abort flag are used
+// only for the CTA's own copies and MMAs in flight before it releases shared
+// and tensor memory.  (`a` is the kernel's __grid_constant__ parameter: its
+// fields are read from the parameter bank, not held in registers.)
+__device__ bool mbar_wait(uint32_t bar, uint32_t parity, const AttnArgs& a,
+                          volatile int* abort_flag, bool drain = false) {
   uint64_t t0 = 0;
   for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -144,9 +145,9 @@ __device__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_fla
       const uint64_t now = globaltimer();
       if (t0 == 0) {
         t0 = now;
-      } else if (now - t0 > kTimeoutNs) {
+      } else if (now - t0 > a.wait_limit_ns) {
         *abort_flag = 1;
-        atomicOr(status, uint32_t(DKV_FLAG_TIMEOUT));
+        atomicOr(a.c.status, uint32_t(DKV_FLAG_TIMEOUT));
         return false;
       }
     }
@@ -792,7 +793,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       const int b = h;  // S buffer, reference slot and barriers of this warpgroup's tiles
       const uint32_t s_col = b ? kColS1 : kColS0;
       // tcgen05.ld/st are warp-collective: every branch around them is warp-uniform
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(SFULL + b), (j >> 1) & 1, abort_flag, cv.status))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(SFULL + b), (j >> 1) & 1, a, abort_flag))) {
         ok = false;
         break;
       }
@@ -830,7 +831,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       float r_prev = -__int_as_float(0x7f800000);
       if (j > 0) {
         if (!__all_sync(0xffffffffu, mbar_wait(bar(RREADY + (b ^ 1)), ((j - 1) >> 1) & 1,
-                                               abort_flag, cv.status))) {
+                                               a, abort_flag))) {
           ok = false;
           break;
         }
@@ -884,7 +885,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         // done; PV(j) waits for this warpgroup's arrive below
         const float alpha = fast_exp2(r_prev - r_j);
         if (!__all_sync(0xffffffffu, mbar_wait(bar(VEMPTY + (b ^ 1)), ((j - 1) >> 1) & 1,
-                                               abort_flag, cv.status))) {
+                                               a, abort_flag))) {
           ok = false;
           break;
         }
@@ -914,13 +915,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     if (ok && nt > 0) {
       const int jl = nt - 1;
       ok = __all_sync(0xffffffffu,
-                      mbar_wait(bar(VEMPTY + (jl & 1)), (jl >> 1) & 1, abort_flag, cv.status));
+                      mbar_wait(bar(VEMPTY + (jl & 1)), (jl >> 1) & 1, a, abort_flag));
     }
     if (ok) {
       lsum[h * 128 + lr] = l;
       lsum[256 + h * 128 + lr] = r_w;
       mbar_arrive(bar(LSUM));
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(LSUM), 0, abort_flag, cv.status));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(LSUM), 0, a, abort_flag));
     }
     if (ok && warp_rows) {
       tc_fence_after();
@@ -974,8 +975,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 #pragma unroll 1
     for (int j = 0; j < nt; ++j) {
       const int b = j & 1, st = j % kStages;
-      if (!mbar_wait(bar(KEMPTY + b), ((j >> 1) & 1) ^ 1, abort_flag, cv.status)) break;
-      if (!mbar_wait(bar(RFULL + st), (j / kStages) & 1, abort_flag, cv.status)) break;
+      if (!mbar_wait(bar(KEMPTY + b), ((j >> 1) & 1) ^ 1, a, abort_flag)) break;
+      if (!mbar_wait(bar(RFULL + st), (j / kStages) & 1, a, abort_flag)) break;
       fill_k_tile<KB>(a, u, (t_begin + j) * TT, sm + (b ? Smem::kK1 : Smem::kK0),
                       sm + Smem::kRing + st * Smem::kStageBytes, c, qh, ko);
       fence_async_smem();
@@ -989,8 +990,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 #pragma unroll 1
     for (int j = 0; j < nt; ++j) {
       const int b = j & 1, st = j % kStages;
-      if (!mbar_wait(bar(VEMPTY + b), ((j >> 1) & 1) ^ 1, abort_flag, cv.status)) break;
-      if (!mbar_wait(bar(RFULL + st), (j / kStages) & 1, abort_flag, cv.status)) break;
+      if (!mbar_wait(bar(VEMPTY + b), ((j >> 1) & 1) ^ 1, a, abort_flag)) break;
+      if (!mbar_wait(bar(RFULL + st), (j / kStages) & 1, a, abort_flag)) break;
       fill_v_tile<KB, VB, SINK>(a, u, (t_begin + j) * TT, sm + (b ? Smem::kV1 : Smem::kV0),
                       sm + Smem::kRing + st * Smem::kStageBytes, t, vo);
       fence_async_smem();
@@ -1009,7 +1010,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     const int gks = KB < 16 ? __ffs(cv.GK) - 1 : 0;
     const int Lq = int(a.Lq), Lc = int(a.L), t0 = int(t_begin) * TT;
     const int32_t* gs = cv.prot_gstart + size_t(u) * size_t(cv.nG + 1);
-    int issued = 0;
+    int issued = 0;     // tiles 0 .. issued-1 went through the ring
+    int stalled = -1;   // (bounds-checking build) the tile whose copies were withheld
     int pf0 = 0, pf1 = 0;  // this lane's prefetched gstart values (tile j0 + lane)
 #pragma unroll 1
     for (int j = 0; j < nt; ++j) {
@@ -1029,9 +1031,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       const int g1 = __shfl_sync(0xffffffffu, pf1, j & 31);
       const int st = j % kStages;
       if (!__all_sync(0xffffffffu, mbar_wait(bar(REMPTY + st), ((j / kStages) & 1) ^ 1,
-                                             abort_flag, cv.status)))
+                                             a, abort_flag)))
         break;
       ++issued;
+#ifdef DKV_BOUNDS_CHECK
+      if (j == a.test_stall_tile) {
+        // test hook: nothing is copied and nothing arrives on this stage, so
+        // the producers' bounded waits on it run out (DKV_FLAG_TIMEOUT)
+        stalled = j;
+        continue;
+      }
+#endif
       if (lane == 0) {
         const int ts = t0 + j * TT;
         const uint32_t dst = sm_base + Smem::kRing + st * Smem::kStageBytes;
@@ -1113,10 +1123,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     // drain: the last copies issued have landed before shared memory is released
     if (lane == 0)
       for (int j = issued > kStages ? issued - kStages : 0; j < issued; ++j)
-        mbar_wait(bar(RFULL + j % kStages), (j / kStages) & 1, abort_flag, cv.status, true);
+        if (j != stalled) mbar_wait(bar(RFULL + j % kStages), (j / kStages) & 1, a, abort_flag, true);
     } else if (warp == kMmaWarp && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
-    bool ok = mbar_wait(bar(QREADY), 0, abort_flag, cv.status);
+    bool ok = mbar_wait(bar(QREADY), 0, a, abort_flag);
     tc_fence_after();
     // QK(j) needs K_j (KFULL) and S_(j mod 2) free, i.e. PV(j-2) issued; PV(i)
     // needs P_i (PFULL) and V_i (VFULL).  Every QK that is ready and allowed
@@ -1143,13 +1153,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       while (nq < nt && nq <= np + 1 && mbar_test(bar(KFULL + (nq & 1)), (nq >> 1) & 1)) issue_qk();
       if (np == nq) {
         // nothing to multiply by P yet: wait for the next K tile
-        ok = mbar_wait(bar(KFULL + (nq & 1)), (nq >> 1) & 1, abort_flag, cv.status);
+        ok = mbar_wait(bar(KFULL + (nq & 1)), (nq >> 1) & 1, a, abort_flag);
         if (ok) issue_qk();
         continue;
       }
       const int bb = np & 1;
-      if (!mbar_wait(bar(PFULL + bb), (np >> 1) & 1, abort_flag, cv.status) ||
-          !mbar_wait(bar(VFULL + bb), (np >> 1) & 1, abort_flag, cv.status)) {
+      if (!mbar_wait(bar(PFULL + bb), (np >> 1) & 1, a, abort_flag) ||
+          !mbar_wait(bar(VFULL + bb), (np >> 1) & 1, a, abort_flag)) {
         ok = false;
         break;
       }
@@ -1167,7 +1177,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     }
     // drain: every MMA issued above completes before TMEM is released
     mma_commit(bar(DONE));
-    mbar_wait(bar(DONE), 0, abort_flag, cv.status, /*drain=*/true);
+    mbar_wait(bar(DONE), 0, a, abort_flag, /*drain=*/true);
     }
   }
 

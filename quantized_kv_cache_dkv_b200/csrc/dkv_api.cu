@@ -35,6 +35,7 @@ struct dkv_cache {
   int32_t max_splits = 1;
   int32_t opt_splits = 0;
   int32_t opt_kernel = 0;
+  int32_t opt_test_stall = -1;
   int32_t last_kernel = 0, last_splits = 0, last_launches = 0;
   bool profile = false;
   std::vector<ProfRecord> prof;  // event pool; the first prof_used are pending
@@ -136,15 +137,27 @@ bool cache_info(const dkv_cache* c, CacheInfo* out) {
   if (!c || !out) return false;
   out->v = c->v;
   out->len = c->len;
+  out->device = c->device;
   out->num_sms = c->num_sms;
   out->opt_splits = c->opt_splits;
   out->opt_kernel = c->opt_kernel;
+  out->opt_test_stall = c->opt_test_stall;
   out->max_splits = c->max_splits;
   out->vrot_act = c->vrot_act;
   return true;
 }
 
 int report_error(int code, const char* msg) { return fail(code, msg); }
+
+int check_device(const CacheInfo& ci) {
+  int dev = -1;
+  const cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(DKV_ERR_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(e));
+  if (dev != ci.device)
+    return fail(DKV_ERR_INVALID_ARG, "the current CUDA device (" + std::to_string(dev) +
+                                         ") is not the cache's device (" + std::to_string(ci.device) + ")");
+  return DKV_OK;
+}
 
 int plan_attention(const CacheInfo& ci, AttnArgs* a, int* kernel_out, const char** err,
                    bool with_active) {
@@ -195,6 +208,9 @@ int plan_attention(const CacheInfo& ci, AttnArgs* a, int* kernel_out, const char
   a->final_out = (a->nsplit == 1 && v.vrot_b == 0) ? 1 : 0;
   a->part_base = 0;
   a->part_stride = a->nsplit;
+  // bounded waits give up after about 1 s; the stall test hook shortens that
+  a->test_stall_tile = ci.opt_test_stall;
+  a->wait_limit_ns = ci.opt_test_stall >= 0 ? 2000000ull : 1000000000ull;
   *kernel_out = kernel;
   return DKV_OK;
 }
@@ -271,8 +287,8 @@ int dkv_cache_alloc(const dkv_config* cfg, void* stream, dkv_cache** out) {
   Region r_pk = take(U * size_t(v.P) * v.d * 2);
   Region r_pg = take(U * (v.nG + 1) * 4);
   Region r_st = take(4);
-  Region r_po = take(U * size_t(c->max_splits) * v.rows * v.d * 4);
-  Region r_pml = take(U * size_t(c->max_splits) * v.rows * 8);
+  Region r_po = take(dkv::split_o_bytes(v.U, c->max_splits, v.rows));
+  Region r_pml = take(dkv::split_ml_bytes(v.U, c->max_splits, v.rows));
   Region r_vsink = take(vq ? U * size_t(v.sink) * v.d * 2 : 0);
   c->arena_bytes = off;
 
@@ -381,6 +397,12 @@ int dkv_commit_block(dkv_cache* c, const void* k, const void* v, const uint32_t*
     return fail(DKV_ERR_INVALID_ARG, "k and v must be 16-byte aligned, protect_words 4-byte");
   if (c->len + c->v.blk > c->v.cap)
     return fail(DKV_ERR_CAPACITY, "len + block exceeds max_tokens");
+  {
+    dkv::CacheInfo ci;
+    dkv::cache_info(c, &ci);
+    const int drc = dkv::check_device(ci);
+    if (drc != DKV_OK) return drc;
+  }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = timed_launch(c, DKV_KERNEL_COMMIT, s, [&] {
     return dkv::launch_commit(c->v, static_cast<const uint16_t*>(k),
@@ -414,6 +436,8 @@ int dkv_block_attention(dkv_cache* c, const void* q, const void* k_act, const vo
   a.scale_log2 = softmax_scale * 1.4426950408889634f;
   dkv::CacheInfo ci;
   dkv::cache_info(c, &ci);
+  const int drc = dkv::check_device(ci);
+  if (drc != DKV_OK) return drc;
   int kernel = 0;
   const char* perr = nullptr;
   const int prc = dkv::plan_attention(ci, &a, &kernel, &perr);
@@ -484,6 +508,8 @@ int dkv_block_attention_dual(dkv_cache* c, dkv_cache* sfx, const void* q, const 
   dkv::CacheInfo ci1, ci2;
   dkv::cache_info(c, &ci1);
   dkv::cache_info(sfx, &ci2);
+  const int drc = dkv::check_device(ci1);
+  if (drc != DKV_OK) return drc;
   ci1.max_splits = c->max_splits - 1;
   int k1 = 0, k2 = 0;
   const char* perr = nullptr;
@@ -648,6 +674,15 @@ int dkv_cache_set_option(dkv_cache* c, int32_t key, int64_t value) {
         return fail(DKV_ERR_UNSUPPORTED, "no tcgen05 attention variant for this shape");
       c->opt_kernel = int32_t(value);
       return DKV_OK;
+    case DKV_OPT_TEST_STALL:
+#ifdef DKV_BOUNDS_CHECK
+      if (value < -1 || value > (int64_t(1) << 30))
+        return fail(DKV_ERR_INVALID_ARG, "test stall tile must be -1 (off) or a tile index");
+      c->opt_test_stall = int32_t(value);
+      return DKV_OK;
+#else
+      return fail(DKV_ERR_UNSUPPORTED, "DKV_OPT_TEST_STALL exists only in the bounds-checking build");
+#endif
     case DKV_OPT_PROFILE:
       if (value != 0 && value != 1) return fail(DKV_ERR_INVALID_ARG, "profile must be 0 or 1");
       c->profile = value == 1;

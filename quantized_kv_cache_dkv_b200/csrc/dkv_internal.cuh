@@ -120,6 +120,9 @@ struct AttnArgs {
                             // no rotation); 0: fp32 partials for combine_kernel
   int32_t part_base;        // split sp of unit u writes partial u*part_stride +
   int32_t part_stride;      // part_base + sp (one call: 0 and nsplit)
+  uint64_t wait_limit_ns;   // limit of one bounded wait in the tcgen05 kernel
+  int32_t test_stall_tile;  // bounds-checking build: tile whose copies the
+                            // tcgen05 loader withholds (-1: none)
 };
 
 cudaError_t launch_commit(const CacheView& c, const uint16_t* k, const uint16_t* v,
@@ -140,13 +143,27 @@ constexpr int kTcTile = 128;
 bool tc_supported(const CacheView& c);
 cudaError_t launch_attention_tc(const AttnArgs& a, cudaStream_t s);
 
+// Split workspace of one attention call: fp32 partial outputs
+// [U][splits][rows][d], then (running max, sum) pairs [U][splits][rows],
+// starting at the next 256-byte boundary.  The handle's workspace and the
+// no-allocation entry point's static buffer are both sized by these.
+inline size_t split_o_bytes(int64_t U, int64_t splits, int64_t rows) {
+  return (size_t(U) * size_t(splits) * size_t(rows) * kHeadDim * sizeof(float) + 255) &
+         ~size_t(255);
+}
+inline size_t split_ml_bytes(int64_t U, int64_t splits, int64_t rows) {
+  return size_t(U) * size_t(splits) * size_t(rows) * sizeof(float2);
+}
+
 // Read-only view of a cache handle, and the thread-local error message, for
 // entry points defined outside dkv_api.cu.
 struct CacheInfo {
   CacheView v;
   int64_t len;
+  int device;  // CUDA device the cache was allocated on
   int num_sms;
   int32_t opt_splits, opt_kernel, max_splits;
+  int32_t opt_test_stall;  // DKV_OPT_TEST_STALL (bounds-checking build), -1 = off
   uint16_t* vrot_act;  // [U][blk][d] rotated active-block V (when c.v.vrot_b > 0)
 };
 bool cache_info(const dkv_cache* c, CacheInfo* out);
@@ -159,5 +176,8 @@ bool cache_info(const dkv_cache* c, CacheInfo* out);
 int plan_attention(const CacheInfo& ci, AttnArgs* a, int* kernel, const char** err,
                    bool with_active = true);
 int report_error(int code, const char* msg);
+// DKV_OK when the current CUDA device is the cache's, else DKV_ERR_INVALID_ARG
+// (or DKV_ERR_CUDA) with the error message set.
+int check_device(const CacheInfo& ci);
 
 }  // namespace dkv

@@ -10,7 +10,7 @@ Workload shapes follow the five synthetic configurations the pages' setting
 implies (8B-class dLLM heads, 32-token blocks, long prompts; the block
 diffusion description in "SoloQ: Calibration-Free Quantization for Diffusion
 Language Models", and MaskAhead's batch-32 systems profile).  The pages print
-no head counts or distributions; those are fixed here and listed in the design doc.
+no head counts or distributions; those are fixed here, in WORKLOADS below.
 
 Every random draw is addressable by position: the K/V of one 32-token block of
 one (batch, kv-head) unit comes from its own PCG64 stream keyed by
