@@ -4,16 +4,17 @@
  *
  * The operations follow three passages of the source pages:
  *   - "SoloQ: Calibration-Free Quantization for Diffusion Language Models",
- *     block-diffusion paragraph: KV entries are quantized only when a block
- *     is committed, the block being denoised stays in full precision, and
- *     keys use KIVI-style per-channel asymmetric quantization.
+ *     block-diffusion paragraph: the cache is quantized when a block is
+ *     committed and not before, the block under denoising keeps full
+ *     precision, and K is quantized per channel on an asymmetric grid, as in
+ *     KIVI.
  *   - "KV Cache Quantization for Diffusion Language Models" (Tai et al.,
- *     Findings of EMNLP 2026), abstract: KIVI adapted to prefix-cache reuse;
- *     KProtect keeps chosen K entries in high precision while V gets
- *     standard low-bit quantization.
- *   - MaskAhead / Q-MaskAhead abstract: block-diffusion models attend to the
- *     cache at every denoising step, computing attention directly from the
- *     low-bit KV.
+ *     Findings of EMNLP 2026), abstract: KIVI carried over to prefix-cache
+ *     reuse; KProtect holds a chosen set of K entries in high precision
+ *     while V is stored at low bit width.
+ *   - MaskAhead / Q-MaskAhead abstract: every denoising step of a block
+ *     model reads the whole committed cache, and the quantized variant runs
+ *     that attention on the low-bit cache itself.
  *
  * Quantizer of one group (b bits): s = fp16((max - min) / (2^b - 1)),
  * z = fp16(min), q = clamp(rint((x - z) / s), 0, 2^b - 1), all fp32 with

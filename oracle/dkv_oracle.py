@@ -12,15 +12,16 @@ textbook meaning of the names they use is taken, and each reading of a step
 the pages leave open is stated beside the function that takes it):
 
 * "SoloQ: Calibration-Free Quantization for Diffusion Language Models"
-  (block-diffusion paragraph): KV entries are quantized only when a block is
-  committed; the block being denoised stays in full precision; keys use
-  KIVI-style per-channel asymmetric quantization.
+  (block-diffusion paragraph): the cache is quantized at commit time and
+  never earlier; the block under denoising keeps full precision; K is
+  quantized per channel on an asymmetric grid, as in KIVI.
 * "KV Cache Quantization for Diffusion Language Models" (Tai et al., Findings
-  of EMNLP 2026, abstract): KIVI adapted to prefix-cache reuse; KProtect keeps
-  chosen K entries in high precision while values get standard low-bit
-  quantization.
-* MaskAhead / Q-MaskAhead abstract: block models attend to the cache at every
-  denoising step; attention is computed directly from the low-bit KV.
+  of EMNLP 2026, abstract): KIVI carried over to prefix-cache reuse; KProtect
+  holds a chosen set of K entries in high precision, and V is stored at low
+  bit width in the usual way.
+* MaskAhead / Q-MaskAhead abstract: each denoising step of a block model
+  reads the whole committed cache; the quantized variant does so on the
+  low-bit cache itself.
 
 Asymmetric quantizer of one group (b bits, 2^b - 1 levels), in fp32 with
 round-to-nearest-even and no fused multiply-add:
@@ -228,8 +229,8 @@ class OracleCache:
         self.prot_k = np.zeros((U, max(max_protected, 0), d), np.uint16)
         self.prot_gstart = np.zeros((U, nG + 1), np.int32)
         # Attention sink: the first sink_tokens positions of every sequence stay
-        # in full precision ("keeping the attention sink in full precision"
-        # matters at 2-bit KV -- SoloQ, KV-only paragraph).  Reading: their K
+        # in full precision (SoloQ, KV-only paragraph: at 2-bit KV, a
+        # full-precision sink makes a large difference).  Reading: their K
         # is protected like any protected entry (side table), their V is kept
         # as bf16 next to the codes (which are still computed and stored).
         assert 0 <= sink_tokens <= capacity
@@ -258,7 +259,7 @@ class OracleCache:
     def tail_mask(self) -> np.ndarray:
         return bool_to_mask_words(self.tail_prot)
 
-    # -- commit ("KV entries are quantized only when a block is committed")
+    # -- commit (quantization happens here, when a block is committed)
     def commit(self, K_bits, V_bits, protect_words=None) -> int:
         """Append one block.  K_bits, V_bits: uint16 [B, Hkv, blk, d] bf16
         patterns; protect_words: uint32 [B, Hkv, ceil(blk/32)] (bit t = token
@@ -460,10 +461,10 @@ class OracleCache:
     def block_attention_selected(self, Q_bits, Kact_bits, Vact_bits, scale: float,
                                  budget: int, selection=None):
         """Attention over a selection of the committed entries (MaskAhead
-        abstract: the current block's mask queries rank KV entries by their
-        estimated contribution to the attention output and select the ones
-        the block attends to; Q-MaskAhead does selection and attention
-        directly from the low-bit KV).  Readings (the abstract gives no
+        abstract: the mask queries of the block being denoised score every
+        cached entry by how much it is expected to add to the attention
+        output, and the block attends to the best-scored ones; the quantized
+        variant scores and attends on the low-bit cache).  Readings (the abstract gives no
         formula): for each (sequence, kv-head) every committed entry j gets
         c_j = (sum over the group's query rows i of p_ij) * ||v_hat_j||_2,
         with p_ij the softmax weight of key j for row i over all committed

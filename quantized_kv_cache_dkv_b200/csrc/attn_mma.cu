@@ -1,6 +1,7 @@
 // Bidirectional block attention over the low-bit cache, warp-level mma.sync
-// variant ("attend to it at every denoising step", computed "directly from
-// low-bit KV" -- MaskAhead / Q-MaskAhead abstract).
+// variant.  Block-diffusion decoding reads the whole committed cache at each
+// denoising step, and Q-MaskAhead runs that attention on the low-bit cache
+// itself (MaskAhead / Q-MaskAhead abstract).
 //
 // CTA = (unit, token split).  Each warp owns 16 query rows of the unit (rows =
 // query heads of the kv-head x block tokens, contiguous in q and out).  Per

@@ -1,8 +1,10 @@
 // Bidirectional block attention over the low-bit cache on the 5th-generation
 // tensor cores (tcgen05 + tensor memory).  A query group (query heads per
 // kv-head x block tokens, 32..256 rows) is processed in row blocks of at most
-// 128 rows, each padded with zero queries to the M = 128 MMA shape.  Attention is computed "directly
-// from low-bit KV" (MaskAhead / Q-MaskAhead abstract) at every denoising step.
+// 128 rows, each padded with zero queries to the M = 128 MMA shape.  The
+// scores and the weighted sum read the packed codes themselves, at each
+// denoising step (MaskAhead / Q-MaskAhead abstract: Q-MaskAhead attends over
+// the low-bit cache without a dequantized copy).
 //
 // CTA = (unit, token split, row block), one CTA per SM, 28 warps (seven
 // warpgroups; setmaxnreg: softmax 96 registers, producers 64, control 56):

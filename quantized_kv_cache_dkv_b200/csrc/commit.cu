@@ -1,8 +1,10 @@
-// Quantize-on-commit ("KV entries are quantized only when a block is
-// committed; the block still being denoised stays in full precision; keys use
-// KIVI-style per-channel asymmetric quantization" -- SoloQ, block-diffusion
-// paragraph; protected K entries kept in high precision with standard low-bit
-// V -- "KV Cache Quantization for Diffusion Language Models", abstract).
+// Quantize-on-commit.  In block-diffusion decoding the cache is quantized at
+// the moment a block is committed and never before; the block under
+// denoising keeps its full precision; K is quantized per channel with an
+// asymmetric (min / max) grid, as KIVI does (SoloQ, block-diffusion
+// paragraph).  A chosen set of K entries keeps high precision while V is
+// stored at low bit width (KProtect, "KV Cache Quantization for Diffusion
+// Language Models", abstract).
 //
 // One CTA of 256 threads per (sequence, kv-head) unit.  The block's V and,
 // when a K group completes, the pending K stream (bf16 tail + block) are first
@@ -71,8 +73,11 @@ __device__ __forceinline__ uint32_t code_of(float x, const GroupQuant& q, int le
   return uint32_t(c);
 }
 
-constexpr int kThreads = 256;         // 128 K channels and up to 128 V groups side by side
-constexpr int kRowPad = kHeadDim + 8;  // shared-memory row stride in halves (272 B)
+constexpr int kThreads = 256;
+// CTAs per (sequence, kv-head) unit: slice sl takes K channels
+// [32 sl, 32 sl + 32) and V tokens [sl blk/4, (sl + 1) blk/4) of the block.
+constexpr int kSlices = 4;
+constexpr int kSliceCh = kHeadDim / kSlices;
 
 __device__ __forceinline__ void range_check8(uint4 x, bool& range) {
   const uint32_t w[4] = {x.x, x.y, x.z, x.w};
@@ -83,17 +88,6 @@ __device__ __forceinline__ void range_check8(uint4 x, bool& range) {
   }
 }
 
-// rows [0, n) of a [n][d] bf16 block -> shared rows of kRowPad halves
-__device__ __forceinline__ void stage_rows(uint16_t* dst, const uint16_t* src, int n, int tid) {
-  for (int i = tid; i < n * (kHeadDim / 8); i += kThreads) {
-    const int t = i / (kHeadDim / 8), o = i % (kHeadDim / 8);
-    *reinterpret_cast<uint4*>(dst + t * kRowPad + o * 8) =
-        __ldg(reinterpret_cast<const uint4*>(src + size_t(t) * kHeadDim + o * 8));
-  }
-}
-
-__device__ __forceinline__ float bf16_at(const uint16_t* p) { return bf16_bits_to_f32(*p); }
-
 // Protect bits of the sink positions [0, sink) among the 32 positions
 // starting at pos0.
 __device__ __forceinline__ uint32_t sink_bits(int64_t pos0, int sink) {
@@ -101,42 +95,7 @@ __device__ __forceinline__ uint32_t sink_bits(int64_t pos0, int sink) {
   return n <= 0 ? 0u : (n >= 32 ? 0xFFFFFFFFu : ((1u << uint32_t(n)) - 1u));
 }
 
-// One V group: G consecutive channels of one token (x: shared memory, 16-byte
-// aligned).  Rolled loops over 8-channel chunks and code words keep the code
-// small (each warp runs it once, so its instructions come from the cache).
-template <int VB>
-__device__ __forceinline__ void quant_v_group(const uint16_t* x, int G, uint32_t* codes,
-                                              __half2* sz, bool& range) {
-  constexpr int levels = (1 << VB) - 1;
-  constexpr int per = 32 / VB;
-  float mn2[2] = {__int_as_float(0x7f800000), __int_as_float(0x7f800000)};
-  float mx2[2] = {-__int_as_float(0x7f800000), -__int_as_float(0x7f800000)};
-#pragma unroll 1
-  for (int i8 = 0; i8 < G; i8 += 8) {
-    const uint4 q8 = *reinterpret_cast<const uint4*>(x + i8);
-    const uint32_t w[4] = {q8.x, q8.y, q8.z, q8.w};
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      float f = bf16_bits_to_f32(uint16_t(w[j >> 1] >> (16 * (j & 1))));
-      range |= out_of_range(f);
-      f = sanitize(f);
-      mn2[j & 1] = fminf(mn2[j & 1], f);
-      mx2[j & 1] = fmaxf(mx2[j & 1], f);
-    }
-  }
-  const GroupQuant q = make_quant(fminf(mn2[0], mn2[1]), fmaxf(mx2[0], mx2[1]), levels);
-#pragma unroll 1
-  for (int w = 0; w < G / per; ++w) {
-    uint32_t word = 0;
-#pragma unroll
-    for (int e = 0; e < per; ++e)
-      word |= code_of(sanitize(bf16_at(x + w * per + e)), q, levels) << (e * VB);
-    codes[w] = word;
-  }
-  *sz = q.sz;
-}
-
-// K-RPBH rotation of one V row held by a warp ("SoloQ", K-RPBH paragraph:
+// K-RPBH rotation of one V row held by a warp (SoloQ, K-RPBH paragraph:
 // random permutation, per-block Hadamard, k x k orthogonal mix of the same
 // in-block coordinate across the k = d/b blocks).  On entry x[e] holds input
 // channel perm[4 lane + e] (the caller's gather applies the permutation); on
@@ -209,71 +168,76 @@ __device__ __forceinline__ void quant_v_rotated(float (&w)[4], int G, uint32_t* 
   if (lane % (G / 4) == 0) sz[lane / (G / 4)] = q.sz;
 }
 
-// One K group of channel ch: G tokens of the pending stream (rows of sk),
-// protected tokens (bits of gm) left out of min/max and given code 0.  Rolled
-// loops as above.
-template <int KB>
-__device__ __forceinline__ GroupQuant quant_k_group(const uint16_t* sk, int G, int row0, int ch,
-                                                    const uint32_t (&gm)[4], int check_row,
-                                                    uint32_t* codes, bool& range) {
-  constexpr int levels = (1 << KB) - 1;
-  constexpr int per = 32 / KB;
-  float mn2[2] = {__int_as_float(0x7f800000), __int_as_float(0x7f800000)};
-  float mx2[2] = {-__int_as_float(0x7f800000), -__int_as_float(0x7f800000)};
-#pragma unroll 1
-  for (int t8 = 0; t8 < G; t8 += 8) {
-    const uint32_t m8 = (gm[t8 >> 5] >> (t8 & 31)) & 0xFFu;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int t = t8 + i;
-      float f = bf16_at(sk + (row0 + t) * kRowPad + ch);
-      if (row0 + t >= check_row) range |= out_of_range(f);
-      f = sanitize(f);
-      if (!((m8 >> i) & 1u)) {
-        mn2[i & 1] = fminf(mn2[i & 1], f);
-        mx2[i & 1] = fmaxf(mx2[i & 1], f);
-      }
-    }
+// min / max over the `lanes` consecutive lanes of one group (lanes a power
+// of two dividing 32, the group aligned to it)
+__device__ __forceinline__ void group_minmax(float& mn, float& mx, int lanes) {
+  for (int o = 1; o < lanes; o <<= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
   }
-  float mn = fminf(mn2[0], mn2[1]);
-  float mx = fmaxf(mx2[0], mx2[1]);
-  if (mn > mx) mn = mx = 0.f;  // every token protected
-  const GroupQuant q = make_quant(mn, mx, levels);
-#pragma unroll 1
-  for (int w = 0; w < G / per; ++w) {
-    const uint32_t mw = (gm[(w * per) >> 5] >> ((w * per) & 31));  // per <= 16 bits of mask
-    uint32_t word = 0;
-#pragma unroll
-    for (int e = 0; e < per; ++e) {
-      const uint32_t cq =
-          code_of(sanitize(bf16_at(sk + (row0 + w * per + e) * kRowPad + ch)), q, levels);
-      if (!((mw >> e) & 1u)) word |= cq << (e * KB);  // protected slot: code 0
-    }
-    codes[w] = word;
-  }
-  return q;
 }
 
-// Shared memory: the V block [blk][kRowPad] (quantized V), then the pending
-// K stream [max(k_group, blk)][kRowPad] (quantized K, when a group completes).
-// Threads [0, 128): K (channel = thread); threads [128, 256): V groups.
+// Protect words of K group gi of the pending stream (the tail's slots, then
+// the block), with the sink positions, cut to the side table's room: the
+// first `room` protected tokens by position stay protected.  Returns how
+// many stay; `cut` is set when some did not fit.
+__device__ __forceinline__ int group_mask(const CacheView& c, const uint32_t* tmask,
+                                          const uint32_t* pwu, int n_tail, int gi, int64_t j,
+                                          int room, uint32_t (&gm)[4], bool& cut) {
+  const int GK = c.GK;
+  int want = 0;
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    gm[w] = 0u;
+    if (w < GK / 32) {
+      const int pwi = gi * GK / 32 + w;  // word of the pending stream
+      gm[w] = pwi < n_tail / 32 ? tmask[pwi] : (pwu ? pwu[pwi - n_tail / 32] : 0u);
+      gm[w] |= sink_bits(j * GK + 32 * w, c.sink);
+      want += __popc(gm[w]);
+    }
+  }
+  if (want <= room) return want;
+  cut = true;
+  int kept = 0;
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    uint32_t m = gm[w], nm = 0u;
+    while (m && kept < room) {
+      const uint32_t low = m & (0u - m);
+      nm |= low;
+      m ^= low;
+      ++kept;
+    }
+    gm[w] = nm;
+  }
+  return kept;
+}
+
+// Quantize-on-commit of one block.  Grid: kSlices CTAs per unit.  Every
+// thread produces one packed code word: K item (group, channel, word) covers
+// the 32/KB tokens of one word of one channel's group, V item (token, word)
+// the 32/VB channels of one word of one token.  A group's min / max is
+// reduced across the lanes holding its words (shuffles), so no thread runs a
+// serial loop over a whole group.  Values are read straight from global
+// memory (the K tail / the caller's block).  The K side table's running count
+// is taken from the group index written by earlier commits (entries before
+// the first group this commit completes), which no CTA of this launch
+// writes, so the CTAs of one unit need no ordering among themselves.
 template <int KB, int VB>
 __global__ void __launch_bounds__(kThreads)
 commit_kernel(CacheView c, const uint16_t* __restrict__ k, const uint16_t* __restrict__ v,
               const uint32_t* __restrict__ pw, int64_t p0, int truncated) {
-  extern __shared__ __align__(16) uint16_t sbuf[];
   pdl_wait();
   pdl_trigger();
-  const int u = blockIdx.x;
-  const int tid = threadIdx.x;
+  const int u = blockIdx.x / kSlices, sl = blockIdx.x % kSlices;
+  const int tid = threadIdx.x, lane = tid & 31;
   const int d = kHeadDim;
   const int blk = c.blk;
   const uint16_t* ku = k + size_t(u) * blk * d;
   const uint16_t* vu = v + size_t(u) * blk * d;
   const int nbw = blk / 32;
+  const uint32_t* pwu = pw ? pw + size_t(u) * nbw : nullptr;
   bool range = false;
-  uint16_t* sv = sbuf;
-  uint16_t* sk = sbuf + (VB < 16 ? blk * kRowPad : 0);
   const int GK = c.GK;
   const int n_tail = KB < 16 ? int(p0 % GK) : 0;
   const bool completes = KB < 16 && n_tail + blk >= GK;
@@ -286,160 +250,198 @@ commit_kernel(CacheView c, const uint16_t* __restrict__ k, const uint16_t* __res
                          (VB == 16 || c.sink <= c.cap),
                      c.status))
     return;
+  const int tpc = blk / kSlices;  // V (and raw K) tokens of this CTA
+  const int t_lo = sl * tpc;
 
-  // a roll-back to p0 (a multiple of the K group) recorded since the last
-  // commit: the side table keeps the entries of the groups before p0, the
-  // tail is empty; applied here, before any thread reads either
-  if (KB < 16 && truncated) {
-    if (tid == 0) c.prot_count[u] = c.prot_gstart[size_t(u) * size_t(c.nG + 1) + size_t(p0 / GK)];
-    if (tid < c.twords) c.tail_mask[size_t(u) * c.twords + tid] = 0u;
-  }
-
-  // ------------------------------------------------------------------ stage
-  if constexpr (VB < 16) stage_rows(sv, vu, blk, tid);
-  if (completes) {
-    stage_rows(sk, c.k_tail + size_t(u) * GK * d, n_tail, tid);
-    stage_rows(sk + n_tail * kRowPad, ku, blk, tid);
-  }
-  __syncthreads();
-
-  // ------------------------------------------------------------------ V
-  if constexpr (VB == 16) {
-    const uint4* src = reinterpret_cast<const uint4*>(vu);
-    uint4* dst = reinterpret_cast<uint4*>(c.v_raw + (size_t(u) * c.cap + p0) * d);
-    for (int i = tid; i < blk * d / 8; i += kThreads) {
+  // ------------------------------------------------------------------ K
+  int nK = 0;  // K items of this CTA (a multiple of 32)
+  constexpr int kper = KB < 16 ? 32 / KB : 1;  // tokens per K code word
+  const int kw = c.kw;                         // words per (group, channel)
+  int nfull = 0;
+  int64_t j0 = 0;
+  int count0 = 0;
+  if constexpr (KB == 16) {
+    const uint4* src = reinterpret_cast<const uint4*>(ku + size_t(t_lo) * d);
+    uint4* dst = reinterpret_cast<uint4*>(c.k_raw + (size_t(u) * c.cap + p0 + t_lo) * d);
+    for (int i = tid; i < tpc * d / 8; i += kThreads) {
       const uint4 x = src[i];
       range_check8(x, range);
       dst[i] = x;
     }
-  } else if (tid >= 128 && c.vrot_b) {
-    // rotated V (no sink): warp wv rotates and quantizes tokens wv, wv + 4, ...
-    const int lane = tid & 31;
-    int pm[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) pm[e] = __ldg(c.vrot_perm + 4 * lane + e);
-    for (int t = (tid - 128) >> 5; t < blk; t += 4) {
-      float x[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float f = bf16_at(sv + t * kRowPad + pm[e]);
-        range |= out_of_range(f);
-        x[e] = sanitize(f);
-      }
-      rotate_row(x, c.vrot_b, c.vrot_norm, c.vrot_mix, lane);
-      const size_t tok = size_t(u) * c.cap + size_t(p0 + t);
-      quant_v_rotated<VB>(x, c.GV, c.v_codes + tok * c.vw, c.v_sz + tok * c.vgroups, lane, range);
+  } else if (!completes) {
+    // the group stays incomplete: this CTA's channels of the block go to the
+    // bf16 tail; the slice-0 CTA writes the tail's protect words
+    uint16_t* tail = c.k_tail + size_t(u) * GK * d;
+    for (int i = tid; i < blk * (kSliceCh / 8); i += kThreads) {
+      const int t = i / (kSliceCh / 8), o = i % (kSliceCh / 8);
+      const uint4 x = *reinterpret_cast<const uint4*>(ku + size_t(t) * d + kSliceCh * sl + 8 * o);
+      range_check8(x, range);
+      *reinterpret_cast<uint4*>(tail + size_t(n_tail + t) * d + kSliceCh * sl + 8 * o) = x;
     }
-  } else if (tid >= 128) {
-    // sink positions keep their V row in bf16 too
-    const int64_t ns = c.sink - p0 < blk ? c.sink - p0 : blk;
-    for (int i = tid - 128; i < ns * (kHeadDim / 8); i += 128) {
-      const int t = i / (kHeadDim / 8), o = i % (kHeadDim / 8);
-      reinterpret_cast<uint4*>(c.v_sink + (size_t(u) * c.sink + size_t(p0 + t)) * d)[o] =
-          *reinterpret_cast<const uint4*>(sv + t * kRowPad + o * 8);
-    }
-    const int GV = c.GV;
-    const int ngr = d / GV;
-    for (int it = tid - 128; it < blk * ngr; it += 128) {
-      const int t = it / ngr, gi = it % ngr;
-      const uint16_t* x = sv + t * kRowPad + gi * GV;
-      uint32_t* codes = c.v_codes + (size_t(u) * c.cap + p0 + t) * c.vw + gi * GV * VB / 32;
-      __half2* sz = c.v_sz + (size_t(u) * c.cap + p0 + t) * ngr + gi;
-      quant_v_group<VB>(x, GV, codes, sz, range);
-    }
+    if (sl == 0 && tid < nbw)
+      c.tail_mask[size_t(u) * c.twords + n_tail / 32 + tid] =
+          (pwu ? pwu[tid] : 0u) | sink_bits(p0 + 32 * tid, c.sink);
+    // a roll-back recorded since the last commit (p0 is then a multiple of
+    // the K group): the side table's count restarts at the group index
+    if (sl == 0 && tid == 0 && truncated)
+      c.prot_count[u] = c.prot_gstart[size_t(u) * size_t(c.nG + 1) + size_t(p0 / GK)];
+  } else {
+    // pending stream = tail[0, n_tail) ++ block[0, blk); every complete group
+    // is quantized (k_group and block divide one another: nothing is left)
+    nfull = (n_tail + blk) / GK;
+    j0 = (p0 - n_tail) / GK;
+    count0 = c.prot_gstart[size_t(u) * size_t(c.nG + 1) + size_t(j0)];
+    nK = nfull * kSliceCh * kw;
   }
 
-  // ------------------------------------------------------------------ K
-  if constexpr (KB == 16) {
-    const uint4* src = reinterpret_cast<const uint4*>(ku);
-    uint4* dst = reinterpret_cast<uint4*>(c.k_raw + (size_t(u) * c.cap + p0) * d);
-    for (int i = tid; i < blk * d / 8; i += kThreads) {
+  // ------------------------------------------------------------------ V
+  constexpr int vper = VB < 16 ? 32 / VB : 1;  // channels per V code word
+  const int vw = c.vw;
+  const int nV = (VB < 16 && !c.vrot_b) ? tpc * vw : 0;
+  if constexpr (VB == 16) {
+    const uint4* src = reinterpret_cast<const uint4*>(vu + size_t(t_lo) * d);
+    uint4* dst = reinterpret_cast<uint4*>(c.v_raw + (size_t(u) * c.cap + p0 + t_lo) * d);
+    for (int i = tid; i < tpc * d / 8; i += kThreads) {
       const uint4 x = src[i];
       range_check8(x, range);
       dst[i] = x;
     }
   } else {
-    uint16_t* tail = c.k_tail + size_t(u) * GK * d;
-    uint32_t* tmask = c.tail_mask + size_t(u) * c.twords;
-    if (!completes) {
-      // the group stays incomplete: append the block to the bf16 tail
-      const uint4* src = reinterpret_cast<const uint4*>(ku);
-      uint4* dst = reinterpret_cast<uint4*>(tail + size_t(n_tail) * d);
-      for (int i = tid; i < blk * d / 8; i += kThreads) {
-        const uint4 x = src[i];
-        range_check8(x, range);
-        dst[i] = x;
+    // sink positions keep their V row in bf16 too
+    const int64_t s_end = c.sink - p0 < int64_t(t_lo + tpc) ? c.sink - p0 : int64_t(t_lo + tpc);
+    for (int i = tid; i < (s_end - t_lo) * (kHeadDim / 8); i += kThreads) {
+      const int t = t_lo + i / (kHeadDim / 8), o = i % (kHeadDim / 8);
+      reinterpret_cast<uint4*>(c.v_sink + (size_t(u) * c.sink + size_t(p0 + t)) * d)[o] =
+          reinterpret_cast<const uint4*>(vu + size_t(t) * d)[o];
+    }
+    if (c.vrot_b) {
+      // rotated V (no sink): warp wv rotates and quantizes tokens t_lo + wv, + 8, ...
+      int pm[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) pm[e] = __ldg(c.vrot_perm + 4 * lane + e);
+      for (int t = t_lo + (tid >> 5); t < t_lo + tpc; t += kThreads / 32) {
+        float x[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float f = bf16_bits_to_f32(__ldg(vu + size_t(t) * d + pm[e]));
+          range |= out_of_range(f);
+          x[e] = sanitize(f);
+        }
+        rotate_row(x, c.vrot_b, c.vrot_norm, c.vrot_mix, lane);
+        const size_t tok = size_t(u) * c.cap + size_t(p0 + t);
+        quant_v_rotated<VB>(x, c.GV, c.v_codes + tok * c.vw, c.v_sz + tok * c.vgroups, lane, range);
       }
-      if (tid < nbw)
-        tmask[n_tail / 32 + tid] =
-            (pw ? pw[size_t(u) * nbw + tid] : 0u) | sink_bits(p0 + 32 * tid, c.sink);
-    } else if (tid < 128) {
-      // pending stream = tail[0, n_tail) ++ block[0, blk) (staged in sk);
-      // quantize every complete group (k_group and block divide one another,
-      // so nothing is left over)
-      const int npend = n_tail + blk;
-      const int nfull = npend / GK;
-      const int ch = tid;  // channel
-      int count = c.prot_count[u];
-      const int64_t j0 = (p0 - n_tail) / GK;
-      for (int gi = 0; gi < nfull; ++gi) {
+    }
+  }
+
+  // one code word per item; items are warp-aligned (nK, nV multiples of 32)
+  for (int it = tid; it < nK + nV; it += kThreads) {
+    if constexpr (KB < 16) {
+      if (it < nK) {
+        constexpr int levels = (1 << KB) - 1;
+        const int w = it % kw, cl = (it / kw) % kSliceCh, gi = it / (kw * kSliceCh);
+        const int ch = kSliceCh * sl + cl;
         const int64_t j = j0 + gi;
-        uint32_t gm[4] = {0u, 0u, 0u, 0u};
+        const uint32_t* tmask = c.tail_mask + size_t(u) * c.twords;
+        // side-table entries stored before group gi (groups of this commit
+        // in order; the same arithmetic in every thread)
+        int before = count0;
+        bool cut = false;
+        uint32_t gm[4];
+        for (int g = 0; g < gi; ++g)
+          before += group_mask(c, tmask, pwu, n_tail, g, j0 + g, c.P - before, gm, cut);
+        const int kept = group_mask(c, tmask, pwu, n_tail, gi, j, c.P - before, gm, cut);
+        if (cut && cl == 0 && w == 0) atomicOr(c.status, uint32_t(DKV_FLAG_CAPACITY));
+        // this word's tokens: t = w kper + e of the group, pending index
+        // gi GK + t (tail slot below n_tail, else block row)
+        const int tw = w * kper;
+        // (a select chain, not a dynamic index: gm stays in registers)
+        const int wi = tw >> 5;
+        const uint32_t gw = wi == 0 ? gm[0] : (wi == 1 ? gm[1] : (wi == 2 ? gm[2] : gm[3]));
+        const uint32_t mw = (gw >> (tw & 31)) & ((kper == 32 ? 0u : (1u << kper)) - 1u);
+        float x[kper];
+        uint16_t raw[kper];
+        float mn = __int_as_float(0x7f800000), mx = -__int_as_float(0x7f800000);
 #pragma unroll
-        for (int w = 0; w < 4; ++w) {
-          if (w < GK / 32) {
-            const int pwi = gi * GK / 32 + w;  // word of the pending stream
-            if (pwi < n_tail / 32)
-              gm[w] = tmask[pwi];
-            else
-              gm[w] = pw ? pw[size_t(u) * nbw + (pwi - n_tail / 32)] : 0u;
-            gm[w] |= sink_bits(j * GK + 32 * w, c.sink);
+        for (int e = 0; e < kper; ++e) {
+          const int pi = gi * GK + tw + e;
+          const uint16_t b = pi < n_tail ? c.k_tail[(size_t(u) * GK + pi) * d + ch]
+                                         : ku[size_t(pi - n_tail) * d + ch];
+          raw[e] = b;
+          float f = bf16_bits_to_f32(b);
+          if (pi >= n_tail) range |= out_of_range(f);
+          f = sanitize(f);
+          x[e] = f;
+          if (!((mw >> e) & 1u)) {
+            mn = fminf(mn, f);
+            mx = fmaxf(mx, f);
           }
         }
-        // side table full: keep the first `room` protected tokens by position
-        int want = 0;
+        group_minmax(mn, mx, kw);
+        if (mn > mx) mn = mx = 0.f;  // every token protected
+        const GroupQuant q = make_quant(mn, mx, levels);
+        uint32_t word = 0;
 #pragma unroll
-        for (int w = 0; w < 4; ++w) want += __popc(gm[w]);
-        const int room = c.P - count;
-        if (want > room) {
-          int kept = 0;
+        for (int e = 0; e < kper; ++e)
+          if (!((mw >> e) & 1u)) word |= code_of(x[e], q, levels) << (e * KB);  // protected: 0
+        const size_t gidx = (size_t(u) * c.nG + size_t(j)) * d + ch;
+        c.k_codes[gidx * kw + w] = word;
+        if (w == 0) c.k_sz[gidx] = q.sz;
+        // protected tokens of this word: side-table entry = entries before the
+        // group + protected tokens of the group before this one
+        if (mw) {
+          int rank = before;
 #pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            uint32_t m = gm[w], nm = 0u;
-            while (m && kept < room) {
-              const uint32_t low = m & (0u - m);
-              nm |= low;
-              m ^= low;
-              ++kept;
+          for (int ww = 0; ww < 4; ++ww)
+            if (32 * ww < tw) rank += __popc(gm[ww] & (32 * ww + 32 <= tw ? 0xFFFFFFFFu
+                                                                           : ((1u << (tw & 31)) - 1u)));
+#pragma unroll
+          for (int e = 0; e < kper; ++e) {
+            if (!((mw >> e) & 1u)) continue;
+            if (DKV_IN_BOUNDS(rank < c.P, c.status)) {
+              c.prot_k[(size_t(u) * c.P + rank) * d + ch] = raw[e];
+              if (ch == 0) c.prot_pos[size_t(u) * c.P + rank] = int32_t(j * GK + tw + e);
             }
-            gm[w] = nm;
-          }
-          if (tid == 0) atomicOr(c.status, uint32_t(DKV_FLAG_CAPACITY));
-        }
-        uint32_t* codes = c.k_codes + ((size_t(u) * c.nG + j) * d + ch) * c.kw;
-        const GroupQuant q = quant_k_group<KB>(sk, GK, gi * GK, ch, gm, n_tail, codes, range);
-        c.k_sz[(size_t(u) * c.nG + j) * d + ch] = q.sz;
-        // side-table entries, ascending positions
-#pragma unroll
-        for (int w = 0; w < 4; ++w) {
-          uint32_t m = gm[w];
-          while (m) {
-            const int b = __ffs(m) - 1;
-            m &= m - 1u;
-            const int t = w * 32 + b;
-            if (!DKV_IN_BOUNDS(count < c.P, c.status)) break;
-            if (tid == 0) c.prot_pos[size_t(u) * c.P + count] = int32_t(j * GK + t);
-            c.prot_k[(size_t(u) * c.P + count) * d + ch] = sk[(gi * GK + t) * kRowPad + ch];
-            ++count;
+            ++rank;
           }
         }
-        if (tid == 0) c.prot_gstart[size_t(u) * (c.nG + 1) + j + 1] = count;
+        if (ch == 0 && w == 0) {
+          c.prot_gstart[size_t(u) * (c.nG + 1) + size_t(j) + 1] = before + kept;
+          if (gi == nfull - 1) c.prot_count[u] = before + kept;
+        }
+        continue;
       }
-      // every K thread has read prot_count and the tail mask before either
-      // is rewritten (named barrier over the 128 K threads only)
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      if (tid == 0) c.prot_count[u] = count;
-      if (tid < c.twords) tmask[tid] = 0u;
+    }
+    if constexpr (VB < 16) {
+      constexpr int levels = (1 << VB) - 1;
+      const int iv = it - nK;
+      const int w = iv % vw, t = t_lo + iv / vw;
+      const int wpg = c.GV / vper;  // words per V group
+      const uint16_t* src = vu + size_t(t) * d + w * vper;
+      float x[vper];
+      float mn = __int_as_float(0x7f800000), mx = -__int_as_float(0x7f800000);
+#pragma unroll
+      for (int o = 0; o < vper / 8; ++o) {
+        const uint4 q8 = *reinterpret_cast<const uint4*>(src + 8 * o);
+        const uint32_t ww[4] = {q8.x, q8.y, q8.z, q8.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          float f = bf16_bits_to_f32(uint16_t(ww[e >> 1] >> (16 * (e & 1))));
+          range |= out_of_range(f);
+          f = sanitize(f);
+          x[8 * o + e] = f;
+          mn = fminf(mn, f);
+          mx = fmaxf(mx, f);
+        }
+      }
+      group_minmax(mn, mx, wpg);
+      const GroupQuant q = make_quant(mn, mx, levels);
+      uint32_t word = 0;
+#pragma unroll
+      for (int e = 0; e < vper; ++e) word |= code_of(x[e], q, levels) << (e * VB);
+      const size_t tok = size_t(u) * c.cap + size_t(p0 + t);
+      c.v_codes[tok * vw + w] = word;
+      if (w % wpg == 0) c.v_sz[tok * c.vgroups + w / wpg] = q.sz;
     }
   }
   if (range) atomicOr(c.status, uint32_t(DKV_FLAG_RANGE));
@@ -483,16 +485,8 @@ __global__ void truncate_kernel(CacheView c, int64_t new_len) {
 template <int KB, int VB>
 cudaError_t launch_kv(const CacheView& c, const uint16_t* k, const uint16_t* v,
                       const uint32_t* pw, int64_t p0, bool truncated, cudaStream_t s) {
-  const int krows = KB < 16 ? (c.GK > c.blk ? c.GK : c.blk) : 0;
-  const int vrows = VB < 16 ? c.blk : 0;
-  const size_t smem = size_t(krows + vrows) * kRowPad * 2;
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(commit_kernel<KB, VB>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-    if (e != cudaSuccess) return e;
-  }
-  const cudaError_t e = launch_pdl(commit_kernel<KB, VB>, dim3(c.U), dim3(kThreads), smem, s, c, k,
-                                   v, pw, p0, truncated ? 1 : 0);
+  const cudaError_t e = launch_pdl(commit_kernel<KB, VB>, dim3(unsigned(c.U) * kSlices),
+                                   dim3(kThreads), 0, s, c, k, v, pw, p0, truncated ? 1 : 0);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

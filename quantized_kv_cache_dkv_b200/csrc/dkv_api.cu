@@ -575,6 +575,12 @@ int dkv_cache_export(dkv_cache* c, void* stream, dkv_export* o) {
     DKV_CUDA(copy2d(o->k_sz, v.k_sz, nGq * v.d * 4, v.nG * v.d * 4));
     DKV_CUDA(copy2d(o->k_tail, v.k_tail, (L - Lq) * v.d * 2, size_t(v.GK) * v.d * 2));
     DKV_CUDA(copy2d(o->tail_mask, v.tail_mask, v.twords * 4, v.twords * 4));
+    // Only the words of the occupied tail slots are meaningful (the commit
+    // kernel writes a slot's word when tokens enter the tail and leaves it
+    // when their group completes): the canonical view has the rest zero.
+    if (o->tail_mask)
+      for (size_t uu = 0; uu < U; ++uu)
+        for (int w = int((L - Lq) / 32); w < v.twords; ++w) o->tail_mask[uu * v.twords + w] = 0u;
     DKV_CUDA(copy2d(o->prot_count, v.prot_count, 4, 4));
     DKV_CUDA(copy2d(o->prot_pos, v.prot_pos, size_t(v.P) * 4, size_t(v.P) * 4));
     DKV_CUDA(copy2d(o->prot_k, v.prot_k, size_t(v.P) * v.d * 2, size_t(v.P) * v.d * 2));

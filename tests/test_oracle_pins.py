@@ -1009,7 +1009,7 @@ def test_selection_follows_entries_when_blocks_are_permuted():
 
 def test_selection_by_contribution_beats_random_selection():
     """What the ranking is for: with peaked attention, keeping the entries of
-    largest estimated contribution approximates full attention better than
+    highest contribution score approximates full attention better than
     keeping as many random entries."""
     r = np.random.default_rng(5)
     d, blk, nb = 128, 32, 8
