@@ -77,7 +77,9 @@ enum {
  * k_group in {32, 64, 128} with k_group % block == 0 or block % k_group == 0;
  * v_group in {32, 64, 128}; max_tokens a multiple of max(k_group, block). */
 typedef struct dkv_config {
-  int32_t batch;         /* B: sequences (all share one committed length) */
+  int32_t batch;         /* B: sequences, at most 512 (each has its own committed
+                            length; they stay equal unless dkv_commit_block_seqs or
+                            dkv_cache_truncate_seq make them differ) */
   int32_t q_heads;       /* Hq */
   int32_t kv_heads;      /* Hkv; query head h reads kv-head h / (Hq/Hkv) */
   int32_t head_dim;      /* d */
@@ -115,6 +117,27 @@ int dkv_cache_free(dkv_cache* cache);
  * at once).  Returns DKV_ERR_CAPACITY if len + block > max_tokens. */
 int dkv_commit_block(dkv_cache* cache, const void* k, const void* v,
                      const uint32_t* protect_words, void* stream);
+
+/* Per-sequence lengths (sequences of one batch finish their blocks at
+ * different denoising steps -- SoloQ, block-diffusion paragraph: each block is
+ * quantized when it is committed).  Commit one block to the sequences listed
+ * in `seqs` (host int32 array of n_seqs distinct indices in [0, B); n_seqs = 0
+ * does nothing): each appends at its own committed length.  k, v and
+ * protect_words have the shapes of dkv_commit_block; the rows of sequences not
+ * listed are not read.  DKV_ERR_CAPACITY if a listed sequence would pass
+ * max_tokens (nothing changes).  Attention then runs every sequence over its
+ * own committed tokens plus its active block. */
+int dkv_commit_block_seqs(dkv_cache* cache, const void* k, const void* v,
+                          const uint32_t* protect_words, const int32_t* seqs,
+                          int32_t n_seqs, void* stream);
+
+/* Committed tokens of every sequence: lens is a host array of B entries
+ * (host mirror, no synchronization). */
+int dkv_cache_seq_lens(const dkv_cache* cache, int64_t* lens);
+
+/* dkv_cache_truncate for one sequence: roll sequence `seq` back to new_len
+ * (same rules as dkv_cache_truncate, against that sequence's length). */
+int dkv_cache_truncate_seq(dkv_cache* cache, int32_t seq, int64_t new_len, void* stream);
 
 /* One denoising-step attention: q bf16 [B, Hq, block, d], the active block
  * k_act, v_act bf16 [B, Hkv, block, d] (kept in full precision), out bf16
@@ -180,7 +203,8 @@ int dkv_cache_set_v_rotation(dkv_cache* cache, const int32_t* perm, const float*
  * new_len must be a multiple of `block` and, when k_bits < 16, of k_group, so
  * that no incomplete K group remains; 0 <= new_len <= len.  The side table
  * keeps the entries of the surviving groups.  len changes at once on the
- * host.  No kernel runs here: the device-side count of side-table entries
+ * host.  Every sequence is rolled back (new_len must not exceed any
+ * sequence's length).  No kernel runs here: the device-side count of side-table entries
  * and the tail mask are reset by the next dkv_commit_block, or by
  * dkv_cache_export if that comes first (on its stream), which is all that
  * reads them; dkv_block_attention reads neither.  `stream` is unused. */
@@ -217,7 +241,8 @@ int dkv_block_attention_noalloc(dkv_cache* cache, const void* q, const void* k_a
                                 const void* v_act, float softmax_scale, void* out,
                                 void* stream);
 
-/* Committed tokens per sequence (host mirror, no synchronization). */
+/* Committed tokens of the longest sequence (host mirror, no synchronization);
+ * the committed length of every sequence when they are all equal. */
 int dkv_cache_len(const dkv_cache* cache, int64_t* len);
 
 /* Synchronize `stream`, return the sticky DKV_FLAG_* bits and clear them. */
@@ -259,6 +284,11 @@ typedef struct dkv_export {
 } dkv_export;
 
 int dkv_cache_export(dkv_cache* cache, void* stream, dkv_export* out);
+
+/* dkv_cache_export of one sequence: its Hkv units (U = kv_heads, in kv-head
+ * order) at its own committed length.  dkv_cache_export itself requires all
+ * sequences to have the same length (else DKV_ERR_INVALID_ARG). */
+int dkv_cache_export_seq(dkv_cache* cache, int32_t seq, void* stream, dkv_export* out);
 
 /* Tuning knobs (testing and benchmarking).  Values persist on the handle.
  *   DKV_OPT_SPLITS: token splits per (sequence, kv-head) in attention;

@@ -86,6 +86,10 @@ _lib.dkv_last_error.restype = ctypes.c_char_p
 _alloc = _sig("dkv_cache_alloc", [ctypes.POINTER(dkv_config), _P, ctypes.POINTER(_P)])
 _free = _sig("dkv_cache_free", [_P])
 _commit = _sig("dkv_commit_block", [_P, _P, _P, _P, _P])
+_commit_seqs = _sig("dkv_commit_block_seqs", [_P, _P, _P, _P, _P, ctypes.c_int32, _P])
+_seq_lens = _sig("dkv_cache_seq_lens", [_P, _P])
+_truncate_seq = _sig("dkv_cache_truncate_seq", [_P, ctypes.c_int32, ctypes.c_int64, _P])
+_export_seq = _sig("dkv_cache_export_seq", [_P, ctypes.c_int32, _P, ctypes.POINTER(dkv_export)])
 _attn = _sig("dkv_block_attention", [_P, _P, _P, _P, ctypes.c_float, _P, _P])
 _attn_noalloc = _sig("dkv_block_attention_noalloc", [_P, _P, _P, _P, ctypes.c_float, _P, _P])
 DKV_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -183,6 +187,32 @@ def dkv_commit_block(cache: Cache, k, v, protect_words=None, stream=None) -> Non
         _tensor_check(protect_words, (c.batch, c.kv_heads, c.block // 32), "protect_words",
                       (torch.int32,))
     _check(_commit(cache.h, _ptr(k), _ptr(v), _ptr(protect_words), _stream(stream)))
+
+
+def dkv_commit_block_seqs(cache: Cache, k, v, protect_words=None, seqs=(), stream=None) -> None:
+    """Commit one block to the listed sequences only (each at its own
+    length); shapes as in dkv_commit_block, other sequences' rows unread."""
+    import torch
+    c = cache.cfg
+    shp = (c.batch, c.kv_heads, c.block, c.head_dim)
+    _tensor_check(k, shp, "k", (torch.bfloat16, torch.int16))
+    _tensor_check(v, shp, "v", (torch.bfloat16, torch.int16))
+    if protect_words is not None:
+        _tensor_check(protect_words, (c.batch, c.kv_heads, c.block // 32), "protect_words",
+                      (torch.int32,))
+    s = np.ascontiguousarray(np.asarray(list(seqs), dtype=np.int32))
+    _check(_commit_seqs(cache.h, _ptr(k), _ptr(v), _ptr(protect_words),
+                        s.ctypes.data_as(_P) if s.size else None, int(s.size), _stream(stream)))
+
+
+def dkv_cache_seq_lens(cache: Cache) -> list:
+    out = np.zeros(cache.cfg.batch, np.int64)
+    _check(_seq_lens(cache.h, out.ctypes.data_as(_P)))
+    return [int(x) for x in out]
+
+
+def dkv_cache_truncate_seq(cache: Cache, seq: int, new_len: int, stream=None) -> None:
+    _check(_truncate_seq(cache.h, int(seq), int(new_len), _stream(stream)))
 
 
 def dkv_block_attention(cache: Cache, q, k_act, v_act, softmax_scale: float, out,
@@ -285,7 +315,20 @@ def dkv_last_attention_plan(cache: Cache):
 def dkv_cache_export(cache: Cache, stream=None) -> dict:
     """Canonical host copies of the committed state (numpy arrays)."""
     c = cache.cfg
-    U, d, L = c.batch * c.kv_heads, c.head_dim, dkv_cache_len(cache)
+    return _export_arrays(cache, c.batch * c.kv_heads, dkv_cache_len(cache),
+                          lambda e: _export(cache.h, _stream(stream), ctypes.byref(e)))
+
+
+def dkv_cache_export_seq(cache: Cache, seq: int, stream=None) -> dict:
+    """Canonical host copies of one sequence's units at its own length."""
+    c = cache.cfg
+    return _export_arrays(cache, c.kv_heads, dkv_cache_seq_lens(cache)[seq],
+                          lambda e: _export_seq(cache.h, int(seq), _stream(stream), ctypes.byref(e)))
+
+
+def _export_arrays(cache: Cache, U: int, L: int, call) -> dict:
+    c = cache.cfg
+    d = c.head_dim
     out = {"len": L}
     if c.k_bits < 16:
         Lq = (L // c.k_group) * c.k_group
@@ -312,5 +355,5 @@ def dkv_cache_export(cache: Cache, stream=None) -> dict:
         arr = out.get(name)
         if arr is not None and arr.size:
             setattr(e, name, arr.ctypes.data)
-    _check(_export(cache.h, _stream(stream), ctypes.byref(e)))
+    _check(call(e))
     return out

@@ -46,37 +46,37 @@ __device__ __forceinline__ uint32_t bf16x2_to_h2(uint32_t w) {
 // Fill K tile columns [32*ch, 32*ch + 32) (one 32-token chunk at absolute
 // position pos0) and V tile rows of the same chunk.
 template <int KB, int VB>
-__device__ __forceinline__ void fill_chunk(const AttnArgs& a, int u, int64_t pos0, int ch,
+__device__ __forceinline__ void fill_chunk(const AttnArgs& a, const UnitLen ul, int u, int64_t pos0, int ch,
                                            __half* Kt, __half* Vt, int tid, int nthr) {
   const CacheView& c = a.c;
   const int d = kHeadDim;
   // ---- K
   int kind;
   const uint16_t* kraw = nullptr;  // token-major bf16 rows (stride d)
-  if (pos0 < a.Lq) {
+  if (pos0 < ul.Lq) {
     if constexpr (KB < 16) {
       kind = SEG_CODES;
     } else {
       kind = SEG_RAW;
       kraw = c.k_raw + (size_t(u) * c.cap + pos0) * d;
     }
-  } else if (pos0 < a.L) {
+  } else if (pos0 < ul.L) {
     kind = SEG_RAW;
-    kraw = c.k_tail + (size_t(u) * c.GK + (pos0 - a.Lq)) * d;
-  } else if (pos0 < a.n_tok) {
+    kraw = c.k_tail + (size_t(u) * c.GK + (pos0 - ul.Lq)) * d;
+  } else if (pos0 < ul.n_tok) {
     kind = SEG_RAW;
-    kraw = a.k_act + (size_t(u) * c.blk + (pos0 - a.L)) * d;
+    kraw = a.k_act + (size_t(u) * c.blk + (pos0 - ul.L)) * d;
   } else {
     kind = SEG_ZERO;
   }
   // bounds-checking build: the chunk lies inside the segment it reads (a
   // chunk that does not is filled with zeros)
   if (!DKV_IN_BOUNDS(pos0 >= 0 && (kind == SEG_ZERO ||
-                                   (kind == SEG_CODES ? pos0 + kChunk <= a.Lq && a.Lq <= c.cap &&
-                                                            a.Lq % c.GK == 0
-                                    : pos0 < a.Lq    ? pos0 + kChunk <= c.cap
-                                    : pos0 < a.L     ? pos0 + kChunk - a.Lq <= c.GK
-                                                     : pos0 + kChunk - a.L <= c.blk)),
+                                   (kind == SEG_CODES ? pos0 + kChunk <= ul.Lq && ul.Lq <= c.cap &&
+                                                            ul.Lq % c.GK == 0
+                                    : pos0 < ul.Lq    ? pos0 + kChunk <= c.cap
+                                    : pos0 < ul.L     ? pos0 + kChunk - ul.Lq <= c.GK
+                                                     : pos0 + kChunk - ul.L <= c.blk)),
                      c.status))
     kind = SEG_ZERO;
   if (kind == SEG_CODES) {
@@ -134,22 +134,22 @@ __device__ __forceinline__ void fill_chunk(const AttnArgs& a, int u, int64_t pos
 
   // ---- V
   const uint16_t* vraw = nullptr;
-  if (pos0 < a.L) {
+  if (pos0 < ul.L) {
     if constexpr (VB < 16) {
       kind = SEG_CODES;
     } else {
       kind = SEG_RAW;
       vraw = c.v_raw + (size_t(u) * c.cap + pos0) * d;
     }
-  } else if (pos0 < a.n_tok) {
+  } else if (pos0 < ul.n_tok) {
     kind = SEG_RAW;
-    vraw = a.v_act + (size_t(u) * c.blk + (pos0 - a.L)) * d;
+    vraw = a.v_act + (size_t(u) * c.blk + (pos0 - ul.L)) * d;
   } else {
     kind = SEG_ZERO;
   }
   if (!DKV_IN_BOUNDS(kind == SEG_ZERO ||
-                         (pos0 < a.L ? pos0 + kChunk <= a.L && a.L <= c.cap
-                                     : pos0 + kChunk - a.L <= c.blk),
+                         (pos0 < ul.L ? pos0 + kChunk <= ul.L && ul.L <= c.cap
+                                     : pos0 + kChunk - ul.L <= c.blk),
                      c.status))
     kind = SEG_ZERO;
   if (kind == SEG_CODES) {
@@ -201,7 +201,7 @@ constexpr int kRowsPerCta = 128;  // 8 warps; a larger query group takes several
 
 template <int KB, int VB>
 __global__ void __launch_bounds__(256)
-attn_mma_kernel(AttnArgs a) {
+attn_mma_kernel(const __grid_constant__ AttnArgs a) {
   __shared__ __align__(16) __half Kt[kHeadDim * KT_LD];
   __shared__ __align__(16) __half Vt[T * VT_LD];
   pdl_wait();
@@ -219,8 +219,9 @@ attn_mma_kernel(AttnArgs a) {
   // warps past the last row only help fill the tiles
   const bool active = rb * kRowsPerCta + warp * 16 < c.rows;
   const int cq = 2 * (lane & 3);           // column pair inside an 8-wide n tile
+  const UnitLen ul = unit_len(a, u);       // this unit's sequence length
 
-  const int64_t n_tiles = (a.n_tok + T - 1) / T;
+  const int64_t n_tiles = (ul.n_tok + T - 1) / T;
   const int64_t t_begin = int64_t(sp) * a.tiles_per_split;
   const int64_t t_end = t_begin + a.tiles_per_split < n_tiles ? t_begin + a.tiles_per_split : n_tiles;
 
@@ -251,8 +252,8 @@ attn_mma_kernel(AttnArgs a) {
   for (int64_t tile = t_begin; tile < t_end; ++tile) {
     const int64_t tile_start = tile * T;
     __syncthreads();
-    fill_chunk<KB, VB>(a, u, tile_start, 0, Kt, Vt, tid, nthr);
-    fill_chunk<KB, VB>(a, u, tile_start + kChunk, 1, Kt, Vt, tid, nthr);
+    fill_chunk<KB, VB>(a, ul, u, tile_start, 0, Kt, Vt, tid, nthr);
+    fill_chunk<KB, VB>(a, ul, u, tile_start + kChunk, 1, Kt, Vt, tid, nthr);
     __syncthreads();
     if (!active) continue;
 
@@ -280,7 +281,7 @@ attn_mma_kernel(AttnArgs a) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int64_t pos = tile_start + nt * 8 + cq + (i & 1);
-        s[nt][i] = pos < a.n_tok ? s[nt][i] * a.scale_log2 : -__int_as_float(0x7f800000);
+        s[nt][i] = pos < ul.n_tok ? s[nt][i] * a.scale_log2 : -__int_as_float(0x7f800000);
       }
       mx0 = fmaxf(mx0, fmaxf(s[nt][0], s[nt][1]));
       mx1 = fmaxf(mx1, fmaxf(s[nt][2], s[nt][3]));
@@ -406,7 +407,7 @@ __device__ __forceinline__ void unrotate_row(float (&x)[4], int b, float norm,
 
 // One warp per (unit, row): out = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s
 // (rotated back first when V is stored rotated)
-__global__ void __launch_bounds__(128) combine_kernel(AttnArgs a) {
+__global__ void __launch_bounds__(128) combine_kernel(const __grid_constant__ AttnArgs a) {
   __shared__ float rbuf[4][kHeadDim];
   pdl_wait();
   pdl_trigger();

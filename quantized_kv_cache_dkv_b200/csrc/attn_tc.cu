@@ -79,8 +79,8 @@ struct Smem {
   static constexpr uint32_t kBar = kRing + kStages * kStageBytes;  // 32 mbarriers
   static constexpr uint32_t kRef = kBar + 32 * 8;   // [tile parity][128] reference max per row
   static constexpr uint32_t kLsum = kRef + 1024;    // [warpgroup][128] row sum, then its reference
-  static constexpr uint32_t kMisc = kLsum + 2048;   // tmem base, abort flag
-  static constexpr uint32_t kBytes = kMisc + 16;
+  static constexpr uint32_t kMisc = kLsum + 2048;   // tmem base, abort flag, then the unit's lengths
+  static constexpr uint32_t kBytes = kMisc + 32;
 };
 enum Bar {
   KFULL = 0, KEMPTY = 2, VFULL = 4, VEMPTY = 6, SFULL = 8, PFULL = 10, QREADY = 12, DONE = 13,
@@ -371,7 +371,7 @@ struct KOffsets {
 };
 
 template <int KB>
-__device__ __noinline__ void fill_k_general(const AttnArgs& a, int u, int64_t tile_start,
+__device__ __noinline__ void fill_k_general(const AttnArgs& a, const UnitLen ul, int u, int64_t tile_start,
                                             uint8_t* kt, const uint8_t* rs, int c, int qh);
 
 // K tile, channel c, token chunks 2qh, 2qh+1.  The whole-quantized-tile case
@@ -379,13 +379,13 @@ __device__ __noinline__ void fill_k_general(const AttnArgs& a, int u, int64_t ti
 // out-of-line general path (at most two per call), which keeps the hot loop's
 // code small.
 template <int KB>
-__device__ __forceinline__ void fill_k_tile(const AttnArgs& a, int u, int64_t tile_start,
+__device__ __forceinline__ void fill_k_tile(const AttnArgs& a, const UnitLen ul, int u, int64_t tile_start,
                                             uint8_t* kt, const uint8_t* rs, int c, int qh,
                                             const KOffsets& ko) {
   const CacheView& cv = a.c;
   const int d = kHeadDim;
   if constexpr (KB < 16) {
-    if (tile_start + TT <= a.Lq) {
+    if (tile_start + TT <= ul.Lq) {
       // whole tile quantized: one 32-token chunk per iteration (a rolled
       // loop keeps the hot code small)
       using W = typename std::conditional<KB == 4, uint4, uint2>::type;
@@ -436,11 +436,11 @@ __device__ __forceinline__ void fill_k_tile(const AttnArgs& a, int u, int64_t ti
       return;
     }
   }
-  fill_k_general<KB>(a, u, tile_start, kt, rs, c, qh);
+  fill_k_general<KB>(a, ul, u, tile_start, kt, rs, c, qh);
 }
 
 template <int KB>
-__device__ __noinline__ void fill_k_general(const AttnArgs& a, int u, int64_t tile_start,
+__device__ __noinline__ void fill_k_general(const AttnArgs& a, const UnitLen ul, int u, int64_t tile_start,
                                             uint8_t* kt, const uint8_t* rs, int c, int qh) {
   const CacheView& cv = a.c;
   const int d = kHeadDim;
@@ -450,13 +450,13 @@ __device__ __noinline__ void fill_k_general(const AttnArgs& a, int u, int64_t ti
     uint4 out[4];
     const uint16_t* raw = nullptr;
     bool codes = false;
-    if (pos0 < a.Lq) {
+    if (pos0 < ul.Lq) {
       if constexpr (KB < 16) codes = true;
       else raw = cv.k_raw + (size_t(u) * cv.cap + pos0) * d;
-    } else if (pos0 < a.L) {
-      raw = cv.k_tail + (size_t(u) * cv.GK + (pos0 - a.Lq)) * d;
-    } else if (pos0 < a.n_tok) {
-      raw = a.k_act + (size_t(u) * cv.blk + (pos0 - a.L)) * d;
+    } else if (pos0 < ul.L) {
+      raw = cv.k_tail + (size_t(u) * cv.GK + (pos0 - ul.Lq)) * d;
+    } else if (pos0 < ul.n_tok) {
+      raw = a.k_act + (size_t(u) * cv.blk + (pos0 - ul.L)) * d;
     }
     if (codes) {
       if constexpr (KB < 16) {
@@ -550,21 +550,21 @@ struct VOffsets {
 };
 
 template <int VB>
-__device__ __noinline__ void fill_v_general(const AttnArgs& a, int u, int64_t tile_start,
+__device__ __noinline__ void fill_v_general(const AttnArgs& a, const UnitLen ul, int u, int64_t tile_start,
                                             uint8_t* vt, const uint8_t* rs, int tid, int perm_kb);
 
 // V tile: the whole-quantized-tile case inline, the rest out of line.  Rows
 // follow the K tile's order: kpos when the tile's K is wholly quantized.
 template <int KB, int VB, bool SINK>
-__device__ __forceinline__ void fill_v_tile(const AttnArgs& a, int u, int64_t tile_start,
+__device__ __forceinline__ void fill_v_tile(const AttnArgs& a, const UnitLen ul, int u, int64_t tile_start,
                                             uint8_t* vt, const uint8_t* rs, int tid,
                                             const VOffsets<KB>& vo) {
   const CacheView& cv = a.c;
-  const bool k_whole = KB < 16 && tile_start + TT <= a.Lq;
+  const bool k_whole = KB < 16 && tile_start + TT <= ul.Lq;
   if constexpr (VB < 16) {
     // (with a sink, tiles holding sink positions take the general path, which
     // reads their bf16 rows)
-    if ((KB < 16 ? k_whole : tile_start + TT <= a.L) && (!SINK || tile_start >= cv.sink)) {
+    if ((KB < 16 ? k_whole : tile_start + TT <= ul.L) && (!SINK || tile_start >= cv.sink)) {
       // whole tile quantized: one item per iteration (a rolled loop keeps
       // the hot code small)
       using W = typename std::conditional<VB == 4, uint4, uint2>::type;
@@ -595,11 +595,11 @@ __device__ __forceinline__ void fill_v_tile(const AttnArgs& a, int u, int64_t ti
       return;
     }
   }
-  fill_v_general<VB>(a, u, tile_start, vt, rs, tid, k_whole ? KB : 16);
+  fill_v_general<VB>(a, ul, u, tile_start, vt, rs, tid, k_whole ? KB : 16);
 }
 
 template <int VB>
-__device__ __noinline__ void fill_v_general(const AttnArgs& a, int u, int64_t tile_start,
+__device__ __noinline__ void fill_v_general(const AttnArgs& a, const UnitLen ul, int u, int64_t tile_start,
                                             uint8_t* vt, const uint8_t* rs, int tid, int perm_kb) {
   const CacheView& cv = a.c;
   const int d = kHeadDim;
@@ -613,15 +613,15 @@ __device__ __noinline__ void fill_v_general(const AttnArgs& a, int u, int64_t ti
     uint4 out[4];
     const uint16_t* raw = nullptr;
     bool codes = false;
-    if (pos < a.L) {
+    if (pos < ul.L) {
       if constexpr (VB < 16) {
         if (pos < cv.sink) raw = cv.v_sink + (size_t(u) * cv.sink + size_t(pos)) * d;  // sink row
         else codes = true;
       } else {
         raw = cv.v_raw + (size_t(u) * cv.cap + pos) * d;
       }
-    } else if (pos < a.n_tok) {
-      raw = a.v_act + (size_t(u) * cv.blk + (pos - a.L)) * d;
+    } else if (pos < ul.n_tok) {
+      raw = a.v_act + (size_t(u) * cv.blk + (pos - ul.L)) * d;
     }
     // out[i] holds channels 32qq + 8((i + rot) & 3): lanes of a quarter warp
     // (tokens t, t+1 x quarters 0..3) then store to 8 distinct bank groups
@@ -708,12 +708,32 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   const int u = (blockIdx.x / nrb) / a.nsplit;
   const int sp = (blockIdx.x / nrb) % a.nsplit;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t n_tiles = (a.n_tok + TT - 1) / TT;
+  const UnitLen ul = unit_len(a, u);  // this unit's sequence length
+  const int64_t n_tiles = (ul.n_tok + TT - 1) / TT;
   const int64_t t_begin = int64_t(sp) * a.tiles_per_split;
   const int64_t t_end = t_begin + a.tiles_per_split < n_tiles ? t_begin + a.tiles_per_split : n_tiles;
-  const int nt = int(t_end - t_begin);
+  const int nt = t_end > t_begin ? int(t_end - t_begin) : 0;
+  if (nt == 0) {
+    // a split past the end of a shorter sequence (the plan follows the
+    // longest): an empty partial -- max -inf, sum 0, O = 0 -- which the
+    // combine gives weight 0.  (With one split every unit has tiles.)
+    pdl_wait();
+    pdl_trigger();
+    if (!a.final_out) {
+      const size_t prow = (size_t(u) * a.part_stride + a.part_base + sp) * cv.rows + size_t(rb) * rpb;
+      for (int i = threadIdx.x; i < rpb * (kHeadDim / 4); i += kThreads)
+        reinterpret_cast<float4*>(a.part_o + prow * kHeadDim)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int i = threadIdx.x; i < rpb; i += kThreads)
+        a.part_ml[prow + i] = make_float2(-__int_as_float(0x7f800000), 0.f);
+    }
+    return;
+  }
 
+  // the unit's lengths live in shared memory from here on: read where used,
+  // not held in registers through the role loops
+  const UnitLen* uls = reinterpret_cast<const UnitLen*>(sm + Smem::kMisc + 16);
   if (threadIdx.x == 0) {
+    *reinterpret_cast<UnitLen*>(sm + Smem::kMisc + 16) = ul;
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar(KFULL + b), 256);
       mbar_init(bar(KEMPTY + b), 1);
@@ -806,7 +826,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         continue;
       }
       const int64_t tile_start = (t_begin + j) * TT;
-      const int valid = a.n_tok - tile_start < TT ? int(a.n_tok - tile_start) : TT;
+      const int n_tok = uls->n_tok;
+      const int valid = n_tok - tile_start < TT ? int(n_tok - tile_start) : TT;
       // Token counts are multiples of 32, so a tile holds n32 = valid / 32
       // whole 32-column chunks of scores; columns past them are never read
       // (and the PV MMAs stop at the same token).
@@ -979,7 +1000,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       const int b = j & 1, st = j % kStages;
       if (!mbar_wait(bar(KEMPTY + b), ((j >> 1) & 1) ^ 1, a, abort_flag)) break;
       if (!mbar_wait(bar(RFULL + st), (j / kStages) & 1, a, abort_flag)) break;
-      fill_k_tile<KB>(a, u, (t_begin + j) * TT, sm + (b ? Smem::kK1 : Smem::kK0),
+      fill_k_tile<KB>(a, *uls, u, (t_begin + j) * TT, sm + (b ? Smem::kK1 : Smem::kK0),
                       sm + Smem::kRing + st * Smem::kStageBytes, c, qh, ko);
       fence_async_smem();
       mbar_arrive(bar(KFULL + b));
@@ -994,7 +1015,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       const int b = j & 1, st = j % kStages;
       if (!mbar_wait(bar(VEMPTY + b), ((j >> 1) & 1) ^ 1, a, abort_flag)) break;
       if (!mbar_wait(bar(RFULL + st), (j / kStages) & 1, a, abort_flag)) break;
-      fill_v_tile<KB, VB, SINK>(a, u, (t_begin + j) * TT, sm + (b ? Smem::kV1 : Smem::kV0),
+      fill_v_tile<KB, VB, SINK>(a, *uls, u, (t_begin + j) * TT, sm + (b ? Smem::kV1 : Smem::kV0),
                       sm + Smem::kRing + st * Smem::kStageBytes, t, vo);
       fence_async_smem();
       mbar_arrive(bar(VFULL + b));
@@ -1010,7 +1031,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     // (capacity <= 2^30) and K groups are 32, 64 or 128 tokens, so the group
     // arithmetic is 32-bit shifts.
     const int gks = KB < 16 ? __ffs(cv.GK) - 1 : 0;
-    const int Lq = int(a.Lq), Lc = int(a.L), t0 = int(t_begin) * TT;
+    const int Lq = uls->Lq, Lc = uls->L, t0 = int(t_begin) * TT;
     const int32_t* gs = cv.prot_gstart + size_t(u) * size_t(cv.nG + 1);
     int issued = 0;     // tiles 0 .. issued-1 went through the ring
     int stalled = -1;   // (bounds-checking build) the tile whose copies were withheld
@@ -1169,7 +1190,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       const uint32_t vbase = sm_base + (bb ? Smem::kV1 : Smem::kV0);
       const uint32_t p_col = bb ? kColS1 : kColS0;
       const int64_t pv_start = (t_begin + np) * TT;
-      const int nk = a.n_tok - pv_start < TT ? int(a.n_tok - pv_start) >> 4 : TT / 16;
+      const int n_tok = uls->n_tok;
+      const int nk = n_tok - pv_start < TT ? int(n_tok - pv_start) >> 4 : TT / 16;
 #pragma unroll 1
       for (int kk = 0; kk < nk; ++kk)  // tokens 16kk..16kk+15: packed P columns 8kk..8kk+7
         mma_ts(tmem + kColO, tmem + p_col + 8 * kk, sdesc_sw128(vbase + 4096 * kk, 1024, 2048),

@@ -225,11 +225,17 @@ __device__ __forceinline__ int group_mask(const CacheView& c, const uint32_t* tm
 // writes, so the CTAs of one unit need no ordering among themselves.
 template <int KB, int VB>
 __global__ void __launch_bounds__(kThreads)
-commit_kernel(CacheView c, const uint16_t* __restrict__ k, const uint16_t* __restrict__ v,
-              const uint32_t* __restrict__ pw, int64_t p0, int truncated) {
+commit_kernel(const __grid_constant__ CacheView c, const uint16_t* __restrict__ k,
+              const uint16_t* __restrict__ v, const uint32_t* __restrict__ pw,
+              const __grid_constant__ CommitArgs ca) {
   pdl_wait();
   pdl_trigger();
   const int u = blockIdx.x / kSlices, sl = blockIdx.x % kSlices;
+  // the unit's sequence: does it commit, at which position, after a roll-back?
+  const int sq = u / c.Hkv;
+  if (!((ca.commit[sq >> 5] >> (sq & 31)) & 1u)) return;
+  const int64_t p0 = ca.p0.len[sq];
+  const bool truncated = (ca.trunc[sq >> 5] >> (sq & 31)) & 1u;
   const int tid = threadIdx.x, lane = tid & 31;
   const int d = kHeadDim;
   const int blk = c.blk;
@@ -471,41 +477,44 @@ __global__ void __launch_bounds__(256) rotate_rows_kernel(CacheView c,
   *reinterpret_cast<uint2*>(dst + row * kHeadDim + 4 * lane) = pk;
 }
 
-// Roll back to new_len (a multiple of the K group): the side table keeps the
-// entries stored before group new_len / GK; the tail is empty.
-__global__ void truncate_kernel(CacheView c, int64_t new_len) {
+// Roll back the sequences with a trunc bit to their length ca.p0 (a multiple
+// of the K group): the side table keeps the entries stored before group
+// len / GK; the tail is empty.
+__global__ void truncate_kernel(const __grid_constant__ CacheView c,
+                                const __grid_constant__ CommitArgs ca) {
   pdl_wait();
   pdl_trigger();
   const int u = blockIdx.x * blockDim.x + threadIdx.x;
   if (u >= c.U) return;
-  c.prot_count[u] = c.prot_gstart[size_t(u) * (c.nG + 1) + new_len / c.GK];
+  const int sq = u / c.Hkv;
+  if (!((ca.trunc[sq >> 5] >> (sq & 31)) & 1u)) return;
+  c.prot_count[u] = c.prot_gstart[size_t(u) * (c.nG + 1) + ca.p0.len[sq] / c.GK];
   for (int w = 0; w < c.twords; ++w) c.tail_mask[size_t(u) * c.twords + w] = 0u;
 }
 
 template <int KB, int VB>
 cudaError_t launch_kv(const CacheView& c, const uint16_t* k, const uint16_t* v,
-                      const uint32_t* pw, int64_t p0, bool truncated, cudaStream_t s) {
+                      const uint32_t* pw, const CommitArgs& ca, cudaStream_t s) {
   const cudaError_t e = launch_pdl(commit_kernel<KB, VB>, dim3(unsigned(c.U) * kSlices),
-                                   dim3(kThreads), 0, s, c, k, v, pw, p0, truncated ? 1 : 0);
+                                   dim3(kThreads), 0, s, c, k, v, pw, ca);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 template <int KB>
 cudaError_t launch_k(const CacheView& c, const uint16_t* k, const uint16_t* v,
-                     const uint32_t* pw, int64_t p0, bool truncated, cudaStream_t s) {
+                     const uint32_t* pw, const CommitArgs& ca, cudaStream_t s) {
   switch (c.vb) {
-    case 2: return launch_kv<KB, 2>(c, k, v, pw, p0, truncated, s);
-    case 4: return launch_kv<KB, 4>(c, k, v, pw, p0, truncated, s);
-    default: return launch_kv<KB, 16>(c, k, v, pw, p0, truncated, s);
+    case 2: return launch_kv<KB, 2>(c, k, v, pw, ca, s);
+    case 4: return launch_kv<KB, 4>(c, k, v, pw, ca, s);
+    default: return launch_kv<KB, 16>(c, k, v, pw, ca, s);
   }
 }
 
 }  // namespace
 
-cudaError_t launch_truncate(const CacheView& c, int64_t new_len, cudaStream_t s) {
-  const cudaError_t e = launch_pdl(truncate_kernel, dim3((c.U + 127) / 128), dim3(128), 0, s, c,
-                                   new_len);
+cudaError_t launch_truncate(const CacheView& c, const CommitArgs& ca, cudaStream_t s) {
+  const cudaError_t e = launch_pdl(truncate_kernel, dim3((c.U + 127) / 128), dim3(128), 0, s, c, ca);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -520,11 +529,11 @@ cudaError_t launch_rotate_v_rows(const CacheView& c, const uint16_t* src, uint16
 }
 
 cudaError_t launch_commit(const CacheView& c, const uint16_t* k, const uint16_t* v,
-                          const uint32_t* pw, int64_t p0, bool truncated, cudaStream_t s) {
+                          const uint32_t* pw, const CommitArgs& ca, cudaStream_t s) {
   switch (c.kb) {
-    case 2: return launch_k<2>(c, k, v, pw, p0, truncated, s);
-    case 4: return launch_k<4>(c, k, v, pw, p0, truncated, s);
-    default: return launch_k<16>(c, k, v, pw, p0, truncated, s);
+    case 2: return launch_k<2>(c, k, v, pw, ca, s);
+    case 4: return launch_k<4>(c, k, v, pw, ca, s);
+    default: return launch_k<16>(c, k, v, pw, ca, s);
   }
 }
 

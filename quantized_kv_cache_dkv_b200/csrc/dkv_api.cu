@@ -24,12 +24,12 @@ struct dkv_cache {
   dkv::CacheView v;
   int device = 0;
   int num_sms = 148;
-  int64_t len = 0;
+  std::vector<int64_t> lens;       // committed tokens per sequence (the host is the authority)
+  std::vector<char> trunc;         // a roll-back of that sequence not yet applied on the device
   void* arena = nullptr;
   size_t arena_bytes = 0;
   float* part_o = nullptr;
   float2* part_ml = nullptr;
-  bool trunc_pending = false;  // a dkv_cache_truncate not yet applied on the device
   void* vrot_mem = nullptr;      // rotation parameters + rotated active block (V rotation)
   uint16_t* vrot_act = nullptr;  // [U][blk][d] bf16
   int32_t max_splits = 1;
@@ -69,6 +69,8 @@ int check_config(const dkv_config* c) {
   if (c->batch < 1 || c->q_heads < 1 || c->kv_heads < 1 || c->head_dim < 1 || c->block < 1 ||
       c->max_tokens < 1 || c->max_protected < 0)
     return fail(DKV_ERR_INVALID_ARG, "non-positive size in config");
+  if (c->batch > dkv::kMaxSeqs)
+    return fail(DKV_ERR_UNSUPPORTED, "batch must be <= " + std::to_string(dkv::kMaxSeqs));
   if (c->q_heads % c->kv_heads)
     return fail(DKV_ERR_INVALID_ARG, "q_heads must be a multiple of kv_heads");
   if (c->head_dim != dkv::kHeadDim) return fail(DKV_ERR_UNSUPPORTED, "head_dim must be 128");
@@ -124,6 +126,30 @@ cudaError_t timed_launch(dkv_cache* c, int kind, cudaStream_t s, F&& launch) {
   return e;
 }
 
+int64_t max_len(const dkv_cache* c) {
+  int64_t m = 0;
+  for (int64_t l : c->lens) m = std::max(m, l);
+  return m;
+}
+
+bool any_trunc(const dkv_cache* c) {
+  for (char t : c->trunc)
+    if (t) return true;
+  return false;
+}
+
+// lengths, commit set and roll-back marks of one commit / truncate launch
+dkv::CommitArgs commit_args(const dkv_cache* c, const std::vector<char>& commits) {
+  dkv::CommitArgs ca;
+  std::memset(&ca, 0, sizeof(ca));
+  for (size_t b = 0; b < c->lens.size(); ++b) {
+    ca.p0.len[b] = int32_t(c->lens[b]);
+    if (commits[b]) ca.commit[b >> 5] |= 1u << (b & 31);
+    if (c->trunc[b]) ca.trunc[b >> 5] |= 1u << (b & 31);
+  }
+  return ca;
+}
+
 int split_cap(int U, int sms) {
   int64_t s = ceil_div(int64_t(8) * sms, U);
   return int(std::min<int64_t>(64, std::max<int64_t>(4, s)));
@@ -136,7 +162,9 @@ namespace dkv {
 bool cache_info(const dkv_cache* c, CacheInfo* out) {
   if (!c || !out) return false;
   out->v = c->v;
-  out->len = c->len;
+  out->len = max_len(c);
+  std::memset(&out->lens, 0, sizeof(out->lens));
+  for (size_t b = 0; b < c->lens.size(); ++b) out->lens.len[b] = int32_t(c->lens[b]);
   out->device = c->device;
   out->num_sms = c->num_sms;
   out->opt_splits = c->opt_splits;
@@ -165,6 +193,8 @@ int plan_attention(const CacheInfo& ci, AttnArgs* a, int* kernel_out, const char
   a->L = ci.len;
   a->Lq = v.kb < 16 ? (ci.len / v.GK) * v.GK : ci.len;
   a->n_tok = ci.len + (with_active ? v.blk : 0);
+  a->lens = ci.lens;
+  a->with_active = with_active ? 1 : 0;
   if (a->n_tok <= 0) {
     *err = "no tokens to attend to";
     return DKV_ERR_INVALID_ARG;
@@ -233,6 +263,8 @@ int dkv_cache_alloc(const dkv_config* cfg, void* stream, dkv_cache** out) {
   dkv_cache* c = new (std::nothrow) dkv_cache();
   if (!c) return fail(DKV_ERR_INVALID_ARG, "host allocation failed");
   c->cfg = *cfg;
+  c->lens.assign(size_t(cfg->batch), 0);
+  c->trunc.assign(size_t(cfg->batch), 0);
   dkv::CacheView& v = c->v;
   v.B = cfg->batch;
   v.Hq = cfg->q_heads;
@@ -353,50 +385,79 @@ int dkv_cache_free(dkv_cache* c) {
 int dkv_cache_len(const dkv_cache* c, int64_t* len) {
   g_err.clear();
   if (!c || !len) return fail(DKV_ERR_INVALID_ARG, "NULL argument");
-  *len = c->len;
+  *len = max_len(c);
   return DKV_OK;
 }
 
+int dkv_cache_seq_lens(const dkv_cache* c, int64_t* lens) {
+  g_err.clear();
+  if (!c || !lens) return fail(DKV_ERR_INVALID_ARG, "NULL argument");
+  for (size_t b = 0; b < c->lens.size(); ++b) lens[b] = c->lens[b];
+  return DKV_OK;
+}
+
+static int check_truncate(const dkv_cache* c, int64_t cur, int64_t new_len) {
+  if (new_len < 0 || new_len > cur || new_len % c->v.blk)
+    return fail(DKV_ERR_INVALID_ARG, "new_len must be a multiple of block within [0, len]");
+  if (c->v.kb < 16 && new_len % c->v.GK)
+    return fail(DKV_ERR_INVALID_ARG, "new_len must be a multiple of k_group");
+  return DKV_OK;
+}
+
+// The device side (side-table count, tail mask) is read only by the next
+// commit and by export, so a roll-back is recorded here and applied by
+// whichever of them comes first: no launch of its own.
 int dkv_cache_truncate(dkv_cache* c, int64_t new_len, void* stream) {
   dkv::NvtxRange nvtx_range("dkv_cache_truncate");
   g_err.clear();
   if (!c) return fail(DKV_ERR_INVALID_ARG, "cache is NULL");
-  if (new_len < 0 || new_len > c->len || new_len % c->v.blk)
-    return fail(DKV_ERR_INVALID_ARG, "new_len must be a multiple of block within [0, len]");
-  if (c->v.kb < 16) {
-    if (new_len % c->v.GK) return fail(DKV_ERR_INVALID_ARG, "new_len must be a multiple of k_group");
-    // The device side (side-table count, tail mask) is read only by the next
-    // commit and by export, so the roll-back is recorded here and applied by
-    // whichever of them comes first: no launch of its own.
-    c->trunc_pending = true;
+  for (int64_t l : c->lens) {
+    const int rc = check_truncate(c, l, new_len);
+    if (rc != DKV_OK) return rc;
   }
   (void)stream;
-  c->len = new_len;
+  for (size_t b = 0; b < c->lens.size(); ++b) {
+    if (c->v.kb < 16) c->trunc[b] = 1;
+    c->lens[b] = new_len;
+  }
   return DKV_OK;
 }
 
-// Applies a recorded roll-back to the device state (export without an
+int dkv_cache_truncate_seq(dkv_cache* c, int32_t seq, int64_t new_len, void* stream) {
+  dkv::NvtxRange nvtx_range("dkv_cache_truncate_seq");
+  g_err.clear();
+  if (!c) return fail(DKV_ERR_INVALID_ARG, "cache is NULL");
+  if (seq < 0 || seq >= c->v.B) return fail(DKV_ERR_INVALID_ARG, "seq out of range");
+  const int rc = check_truncate(c, c->lens[size_t(seq)], new_len);
+  if (rc != DKV_OK) return rc;
+  (void)stream;
+  if (c->v.kb < 16) c->trunc[size_t(seq)] = 1;
+  c->lens[size_t(seq)] = new_len;
+  return DKV_OK;
+}
+
+// Applies recorded roll-backs to the device state (export without an
 // intervening commit).
 static int apply_pending_truncate(dkv_cache* c, cudaStream_t s) {
-  if (!c->trunc_pending) return DKV_OK;
+  if (!any_trunc(c)) return DKV_OK;
+  const dkv::CommitArgs ca = commit_args(c, std::vector<char>(c->lens.size(), 0));
   cudaError_t e = timed_launch(c, DKV_KERNEL_TRUNCATE, s,
-                               [&] { return dkv::launch_truncate(c->v, c->len, s); });
+                               [&] { return dkv::launch_truncate(c->v, ca, s); });
   if (e != cudaSuccess)
     return fail(DKV_ERR_CUDA, std::string("truncate launch: ") + cudaGetErrorString(e));
-  c->trunc_pending = false;
+  std::fill(c->trunc.begin(), c->trunc.end(), 0);
   return DKV_OK;
 }
 
-int dkv_commit_block(dkv_cache* c, const void* k, const void* v, const uint32_t* protect_words,
-                     void* stream) {
-  dkv::NvtxRange nvtx_range("dkv_commit_block");
-  g_err.clear();
-  if (!c || !k || !v) return fail(DKV_ERR_INVALID_ARG, "NULL cache, k or v");
+static int commit_some(dkv_cache* c, const void* k, const void* v, const uint32_t* protect_words,
+                       const std::vector<char>& commits, void* stream) {
+  if (!k || !v) return fail(DKV_ERR_INVALID_ARG, "NULL cache, k or v");
   if (!aligned16(k) || !aligned16(v) ||
       (reinterpret_cast<uintptr_t>(protect_words) & 3u))
     return fail(DKV_ERR_INVALID_ARG, "k and v must be 16-byte aligned, protect_words 4-byte");
-  if (c->len + c->v.blk > c->v.cap)
-    return fail(DKV_ERR_CAPACITY, "len + block exceeds max_tokens");
+  for (size_t b = 0; b < c->lens.size(); ++b)
+    if (commits[b] && c->lens[b] + c->v.blk > c->v.cap)
+      return fail(DKV_ERR_CAPACITY, "len + block exceeds max_tokens");
   {
     dkv::CacheInfo ci;
     dkv::cache_info(c, &ci);
@@ -404,15 +465,43 @@ int dkv_commit_block(dkv_cache* c, const void* k, const void* v, const uint32_t*
     if (drc != DKV_OK) return drc;
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const dkv::CommitArgs ca = commit_args(c, commits);
   cudaError_t e = timed_launch(c, DKV_KERNEL_COMMIT, s, [&] {
     return dkv::launch_commit(c->v, static_cast<const uint16_t*>(k),
-                              static_cast<const uint16_t*>(v), protect_words, c->len,
-                              c->trunc_pending, s);
+                              static_cast<const uint16_t*>(v), protect_words, ca, s);
   });
   if (e != cudaSuccess) return fail(DKV_ERR_CUDA, std::string("commit launch: ") + cudaGetErrorString(e));
-  c->trunc_pending = false;
-  c->len += c->v.blk;
+  for (size_t b = 0; b < c->lens.size(); ++b)
+    if (commits[b]) {
+      c->trunc[b] = 0;
+      c->lens[b] += c->v.blk;
+    }
   return DKV_OK;
+}
+
+int dkv_commit_block(dkv_cache* c, const void* k, const void* v, const uint32_t* protect_words,
+                     void* stream) {
+  dkv::NvtxRange nvtx_range("dkv_commit_block");
+  g_err.clear();
+  if (!c) return fail(DKV_ERR_INVALID_ARG, "NULL cache, k or v");
+  return commit_some(c, k, v, protect_words, std::vector<char>(c->lens.size(), 1), stream);
+}
+
+int dkv_commit_block_seqs(dkv_cache* c, const void* k, const void* v,
+                          const uint32_t* protect_words, const int32_t* seqs, int32_t n_seqs,
+                          void* stream) {
+  dkv::NvtxRange nvtx_range("dkv_commit_block_seqs");
+  g_err.clear();
+  if (!c) return fail(DKV_ERR_INVALID_ARG, "NULL cache, k or v");
+  if (n_seqs < 0 || (n_seqs > 0 && !seqs)) return fail(DKV_ERR_INVALID_ARG, "bad sequence list");
+  std::vector<char> commits(c->lens.size(), 0);
+  for (int32_t i = 0; i < n_seqs; ++i) {
+    if (seqs[i] < 0 || seqs[i] >= c->v.B) return fail(DKV_ERR_INVALID_ARG, "sequence index out of range");
+    if (commits[size_t(seqs[i])]) return fail(DKV_ERR_INVALID_ARG, "sequence listed twice");
+    commits[size_t(seqs[i])] = 1;
+  }
+  if (n_seqs == 0) return DKV_OK;
+  return commit_some(c, k, v, protect_words, commits, stream);
 }
 
 int dkv_block_attention(dkv_cache* c, const void* q, const void* k_act, const void* v_act,
@@ -481,7 +570,7 @@ int dkv_block_attention_dual(dkv_cache* c, dkv_cache* sfx, const void* q, const 
   if (v.vrot_b || vs.vrot_b)
     return fail(DKV_ERR_UNSUPPORTED, "dual-cache attention with rotated V is not supported");
   if (vs.sink > 0) return fail(DKV_ERR_UNSUPPORTED, "the suffix cache cannot have an attention sink");
-  if (sfx->len == 0) {
+  if (max_len(sfx) == 0) {
     // nothing after the active block: the single-cache call
     const int rc = dkv_block_attention(c, q, k_act, v_act, softmax_scale, out, stream);
     return rc;
@@ -554,21 +643,20 @@ int dkv_cache_status(dkv_cache* c, void* stream, uint32_t* flags) {
   return DKV_OK;
 }
 
-int dkv_cache_export(dkv_cache* c, void* stream, dkv_export* o) {
-  dkv::NvtxRange nvtx_range("dkv_cache_export");
-  g_err.clear();
-  if (!c || !o) return fail(DKV_ERR_INVALID_ARG, "NULL argument");
+// Host copies of units [u0, u0 + nU), all of committed length L.
+static int export_units(dkv_cache* c, size_t u0, size_t nU, int64_t L, void* stream,
+                        dkv_export* o) {
   const dkv::CacheView& v = c->v;
   const int trc = apply_pending_truncate(c, static_cast<cudaStream_t>(stream));
   if (trc != DKV_OK) return trc;
   DKV_CUDA(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
-  const int64_t L = c->len;
   const int64_t Lq = v.kb < 16 ? (L / v.GK) * v.GK : L;
   const int64_t nGq = v.kb < 16 ? Lq / v.GK : 0;
-  const size_t U = size_t(v.U);
+  // row = one unit: `width` bytes of a unit's `pitch`-byte region
   auto copy2d = [&](void* dst, const void* src, size_t width, size_t pitch) -> cudaError_t {
     if (!dst || !src || width == 0) return cudaSuccess;
-    return cudaMemcpy2D(dst, width, src, pitch, width, U, cudaMemcpyDeviceToHost);
+    return cudaMemcpy2D(dst, width, static_cast<const char*>(src) + u0 * pitch, pitch, width, nU,
+                        cudaMemcpyDeviceToHost);
   };
   if (v.kb < 16) {
     DKV_CUDA(copy2d(o->k_codes, v.k_codes, nGq * v.d * v.kw * 4, v.nG * v.d * v.kw * 4));
@@ -579,7 +667,7 @@ int dkv_cache_export(dkv_cache* c, void* stream, dkv_export* o) {
     // kernel writes a slot's word when tokens enter the tail and leaves it
     // when their group completes): the canonical view has the rest zero.
     if (o->tail_mask)
-      for (size_t uu = 0; uu < U; ++uu)
+      for (size_t uu = 0; uu < nU; ++uu)
         for (int w = int((L - Lq) / 32); w < v.twords; ++w) o->tail_mask[uu * v.twords + w] = 0u;
     DKV_CUDA(copy2d(o->prot_count, v.prot_count, 4, 4));
     DKV_CUDA(copy2d(o->prot_pos, v.prot_pos, size_t(v.P) * 4, size_t(v.P) * 4));
@@ -587,7 +675,7 @@ int dkv_cache_export(dkv_cache* c, void* stream, dkv_export* o) {
     DKV_CUDA(copy2d(o->prot_gstart, v.prot_gstart, (nGq + 1) * 4, (v.nG + 1) * 4));
   } else {
     DKV_CUDA(copy2d(o->k_raw, v.k_raw, L * v.d * 2, v.cap * v.d * 2));
-    if (o->prot_count) std::memset(o->prot_count, 0, U * 4);
+    if (o->prot_count) std::memset(o->prot_count, 0, nU * 4);
   }
   if (v.vb < 16) {
     DKV_CUDA(copy2d(o->v_codes, v.v_codes, L * v.vw * 4, v.cap * v.vw * 4));
@@ -600,12 +688,32 @@ int dkv_cache_export(dkv_cache* c, void* stream, dkv_export* o) {
   return DKV_OK;
 }
 
+int dkv_cache_export(dkv_cache* c, void* stream, dkv_export* o) {
+  dkv::NvtxRange nvtx_range("dkv_cache_export");
+  g_err.clear();
+  if (!c || !o) return fail(DKV_ERR_INVALID_ARG, "NULL argument");
+  for (int64_t l : c->lens)
+    if (l != c->lens[0])
+      return fail(DKV_ERR_INVALID_ARG,
+                  "sequences have different lengths: export them with dkv_cache_export_seq");
+  return export_units(c, 0, size_t(c->v.U), c->lens[0], stream, o);
+}
+
+int dkv_cache_export_seq(dkv_cache* c, int32_t seq, void* stream, dkv_export* o) {
+  dkv::NvtxRange nvtx_range("dkv_cache_export_seq");
+  g_err.clear();
+  if (!c || !o) return fail(DKV_ERR_INVALID_ARG, "NULL argument");
+  if (seq < 0 || seq >= c->v.B) return fail(DKV_ERR_INVALID_ARG, "seq out of range");
+  return export_units(c, size_t(seq) * size_t(c->v.Hkv), size_t(c->v.Hkv), c->lens[size_t(seq)],
+                      stream, o);
+}
+
 int dkv_cache_set_v_rotation(dkv_cache* c, const int32_t* perm, const float* mix,
                              int32_t block) {
   dkv::NvtxRange nvtx_range("dkv_cache_set_v_rotation");
   g_err.clear();
   if (!c) return fail(DKV_ERR_INVALID_ARG, "cache is NULL");
-  if (c->len != 0) return fail(DKV_ERR_INVALID_ARG, "set the V rotation before the first commit");
+  if (max_len(c) != 0) return fail(DKV_ERR_INVALID_ARG, "set the V rotation before the first commit");
   if (block == 0) {
     if (c->vrot_mem) {
       DKV_CUDA(cudaDeviceSynchronize());

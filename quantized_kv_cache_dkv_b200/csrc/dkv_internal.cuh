@@ -101,9 +101,18 @@ struct CacheView {
   const float* vrot_mix;      // [k][k] orthogonal mix, k = d / b
 };
 
+// Committed tokens of every sequence, passed by value to each launch (the
+// host keeps the lengths; a CUDA graph captures them with the launch).
+constexpr int kMaxSeqs = 512;
+struct SeqLens {
+  int32_t len[kMaxSeqs];
+};
+
 // Arguments of one attention call.
 struct AttnArgs {
   CacheView c;
+  SeqLens lens;           // committed tokens per sequence
+  int32_t with_active;    // 1: the active block follows each sequence's tokens
   const uint16_t* q;      // [B][Hq][blk][d] bf16
   const uint16_t* k_act;  // [B][Hkv][blk][d] bf16
   const uint16_t* v_act;  // [B][Hkv][blk][d] bf16
@@ -111,9 +120,9 @@ struct AttnArgs {
   float* part_o;          // [U][nsplit][rows][d] fp32 (unnormalised)
   float2* part_ml;        // [U][nsplit][rows] (running max in log2 units, sum)
   float scale_log2;       // softmax_scale * log2(e)
-  int64_t L;              // committed tokens
-  int64_t Lq;             // tokens whose K is in complete groups (or raw)
-  int64_t n_tok;          // L + blk
+  int64_t L;              // committed tokens of the longest sequence (planning)
+  int64_t Lq;             // its tokens whose K is in complete groups (or raw)
+  int64_t n_tok;          // L + blk (L without the active block)
   int32_t nsplit;
   int32_t tiles_per_split;  // in units of the kernel's token tile
   int32_t final_out;        // 1: the attention kernel writes bf16 out (one split,
@@ -125,9 +134,35 @@ struct AttnArgs {
                             // tcgen05 loader withholds (-1: none)
 };
 
+// Token counts of one unit (u = b * Hkv + h) in one attention call: L
+// committed, Lq of them with K in complete groups (or raw), n_tok attended
+// (L plus the active block when there is one).  Capacities are at most 2^30
+// tokens, so 32 bits hold them.
+struct UnitLen {
+  int32_t L, Lq, n_tok;
+};
+__device__ __forceinline__ UnitLen unit_len(const AttnArgs& a, int u) {
+  const int32_t L = a.lens.len[u / a.c.Hkv];
+  UnitLen r;
+  r.L = L;
+  r.Lq = a.c.kb < 16 ? (L / a.c.GK) * a.c.GK : L;
+  r.n_tok = L + (a.with_active ? a.c.blk : 0);
+  return r;
+}
+
+// One commit launch: the sequences that append a block (bit b of commit[]),
+// each at its own position p0.len[b]; trunc[] marks sequences with a
+// roll-back recorded since their last commit.
+struct CommitArgs {
+  SeqLens p0;
+  uint32_t commit[kMaxSeqs / 32];
+  uint32_t trunc[kMaxSeqs / 32];
+};
 cudaError_t launch_commit(const CacheView& c, const uint16_t* k, const uint16_t* v,
-                          const uint32_t* pw, int64_t p0, bool truncated, cudaStream_t s);
-cudaError_t launch_truncate(const CacheView& c, int64_t new_len, cudaStream_t s);
+                          const uint32_t* pw, const CommitArgs& ca, cudaStream_t s);
+// Applies recorded roll-backs (sequences with a trunc bit, to lens) to the
+// side-table count and tail mask.
+cudaError_t launch_truncate(const CacheView& c, const CommitArgs& ca, cudaStream_t s);
 // The active block's V [U][blk][d] bf16 rotated like committed V rows (same
 // fp32 order) and rounded to bf16 into dst (c.vrot_b > 0).
 cudaError_t launch_rotate_v_rows(const CacheView& c, const uint16_t* src, uint16_t* dst,
@@ -159,7 +194,8 @@ inline size_t split_ml_bytes(int64_t U, int64_t splits, int64_t rows) {
 // entry points defined outside dkv_api.cu.
 struct CacheInfo {
   CacheView v;
-  int64_t len;
+  int64_t len;       // the longest sequence's committed tokens
+  SeqLens lens;      // every sequence's
   int device;  // CUDA device the cache was allocated on
   int num_sms;
   int32_t opt_splits, opt_kernel, max_splits;
