@@ -73,7 +73,8 @@ enum {
 
 /* Cache shape.  Supported: head_dim == 128; block a multiple of 32, <= 128;
  * q_heads a multiple of kv_heads with (q_heads/kv_heads)*block <= 256;
- * k_bits, v_bits in {2, 4, 16} (16 = store bf16, quantization off);
+ * k_bits, v_bits in {2, 3, 4, 16} (16 = store bf16, quantization off; 3-bit
+ * caches attend with the mma.sync kernel, and 3-bit V cannot be rotated);
  * k_group in {32, 64, 128} with k_group % block == 0 or block % k_group == 0;
  * v_group in {32, 64, 128}; max_tokens a multiple of max(k_group, block). */
 typedef struct dkv_config {
@@ -253,8 +254,10 @@ int dkv_cache_status(dkv_cache* cache, void* stream, uint32_t* flags);
  * = L when k_bits == 16; nG = Lq / k_group).  Every pointer is a host buffer
  * owned by the caller, or NULL to skip that array.  Synchronizes `stream`.
  *   k_codes   uint32 [U, nG, d, k_group*k_bits/32]  codes of one (group,
- *             channel) packed along its tokens: token t at bits
- *             [k_bits*t mod 32, +k_bits) of word k_bits*t/32
+ *             channel) packed along its tokens, a little-endian bit stream:
+ *             token t at bits [k_bits*t, +k_bits) of the stream, where bit i
+ *             is bit i mod 32 of word i/32 (at 3 bits codes 10 and 21 of
+ *             every 32 straddle two words)
  *   k_sz      uint16 [U, nG, d, 2]    fp16 (scale, zero) per (group, channel)
  *   k_raw     uint16 [U, L, d]        bf16 K when k_bits == 16
  *   k_tail    uint16 [U, L - Lq, d]   bf16 K of the incomplete group

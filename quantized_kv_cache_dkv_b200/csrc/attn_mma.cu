@@ -92,7 +92,13 @@ __device__ __forceinline__ void fill_chunk(const AttnArgs& a, const UnitLen ul, 
         const __half2 s2 = __half2half2(__low2half(sz));
         const __half2 z2 = __half2half2(__high2half(sz));
         uint4* dst = reinterpret_cast<uint4*>(Kt + cc * KT_LD + ch * 32);
-        if constexpr (KB == 4) {
+        if constexpr (KB == 3) {
+          const uint32_t* kc = c.k_codes + base;  // 3 words, 4-byte aligned
+          uint4 o4[4];
+          dequant3x32(kc[0], kc[1], kc[2], s2, z2, o4);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) dst[k] = o4[k];
+        } else if constexpr (KB == 4) {
           const uint4 w = *reinterpret_cast<const uint4*>(c.k_codes + base);
           dst[0] = dequant4x8(w.x, s2, z2);
           dst[1] = dequant4x8(w.y, s2, z2);
@@ -170,7 +176,13 @@ __device__ __forceinline__ void fill_chunk(const AttnArgs& a, const UnitLen ul, 
           for (int k = 0; k < 4; ++k) dst[k] = bf16x8_to_f16x8(src[k]);
           continue;
         }
-        if constexpr (VB == 4) {
+        if constexpr (VB == 3) {
+          const uint32_t* vc = c.v_codes + tok * c.vw + q * 3;  // 3 words, 4-byte aligned
+          uint4 o4[4];
+          dequant3x32(vc[0], vc[1], vc[2], s2, z2, o4);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) dst[k] = o4[k];
+        } else if constexpr (VB == 4) {
           const uint4 w = *reinterpret_cast<const uint4*>(c.v_codes + tok * c.vw + q * 4);
           dst[0] = dequant4x8(w.x, s2, z2);
           dst[1] = dequant4x8(w.y, s2, z2);
@@ -460,6 +472,7 @@ template <int KB>
 cudaError_t launch_k(const AttnArgs& a, cudaStream_t s) {
   switch (a.c.vb) {
     case 2: return launch_kv<KB, 2>(a, s);
+    case 3: return launch_kv<KB, 3>(a, s);
     case 4: return launch_kv<KB, 4>(a, s);
     default: return launch_kv<KB, 16>(a, s);
   }
@@ -470,6 +483,7 @@ cudaError_t launch_k(const AttnArgs& a, cudaStream_t s) {
 cudaError_t launch_attention_mma(const AttnArgs& a, cudaStream_t s) {
   switch (a.c.kb) {
     case 2: return launch_k<2>(a, s);
+    case 3: return launch_k<3>(a, s);
     case 4: return launch_k<4>(a, s);
     default: return launch_k<16>(a, s);
   }

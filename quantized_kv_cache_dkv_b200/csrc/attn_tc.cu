@@ -1246,8 +1246,10 @@ cudaError_t launch_k(const AttnArgs& a, cudaStream_t s) {
 }  // namespace
 
 // any query group of 32..256 rows (a multiple of 32): M = 128 per row block
+// (3-bit codes take the mma.sync kernel)
 bool tc_supported(const CacheView& c) {
-  return c.d == kHeadDim && c.rows >= 32 && c.rows <= 256 && c.rows % 32 == 0;
+  return c.d == kHeadDim && c.rows >= 32 && c.rows <= 256 && c.rows % 32 == 0 && c.kb != 3 &&
+         c.vb != 3;
 }
 
 cudaError_t launch_attention_tc(const AttnArgs& a, cudaStream_t s) {

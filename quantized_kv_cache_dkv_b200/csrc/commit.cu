@@ -168,6 +168,30 @@ __device__ __forceinline__ void quant_v_rotated(float (&w)[4], int G, uint32_t* 
   if (lane % (G / 4) == 0) sz[lane / (G / 4)] = q.sz;
 }
 
+// Packs n codes (code(e), e = 0..n-1, each < 2^B) little-endian into the
+// bit stream of words[]: code e at bits [B e, B e + B).  n B is 32 (one
+// word) or, at 3 bits, 96 (three words; codes 10 and 21 straddle words).
+template <int B, int n, class F>
+__device__ __forceinline__ void pack_codes(F code, uint32_t (&words)[n * B / 32]) {
+  uint64_t lo = 0, hi = 0;  // bits [0, 64) and [64, 128) of the stream
+#pragma unroll
+  for (int e = 0; e < n; ++e) {
+    const uint64_t cq = code(e);
+    const int pos = B * e;
+    if (pos + B <= 64) {
+      lo |= cq << pos;
+    } else if (pos >= 64) {
+      hi |= cq << (pos - 64);
+    } else {
+      lo |= cq << pos;
+      hi |= cq >> (64 - pos);
+    }
+  }
+  words[0] = uint32_t(lo);
+  if constexpr (n * B / 32 > 1) words[1] = uint32_t(lo >> 32);
+  if constexpr (n * B / 32 > 2) words[2] = uint32_t(hi);
+}
+
 // min / max over the `lanes` consecutive lanes of one group (lanes a power
 // of two dividing 32, the group aligned to it)
 __device__ __forceinline__ void group_minmax(float& mn, float& mx, int lanes) {
@@ -261,8 +285,12 @@ commit_kernel(const __grid_constant__ CacheView c, const uint16_t* __restrict__ 
 
   // ------------------------------------------------------------------ K
   int nK = 0;  // K items of this CTA (a multiple of 32)
-  constexpr int kper = KB < 16 ? 32 / KB : 1;  // tokens per K code word
-  const int kw = c.kw;                         // words per (group, channel)
+  // One thread codes kper tokens of one (group, channel) into kwpt packed
+  // words: one word (32 / KB tokens) at 2 and 4 bits; at 3 bits 32 tokens,
+  // whose codes fill exactly 3 words.  kthr threads share a group.
+  constexpr int kper = KB < 16 ? (KB == 3 ? 32 : 32 / KB) : 1;
+  constexpr int kwpt = KB == 3 ? 3 : 1;
+  const int kthr = GK / kper;
   int nfull = 0;
   int64_t j0 = 0;
   int count0 = 0;
@@ -297,13 +325,15 @@ commit_kernel(const __grid_constant__ CacheView c, const uint16_t* __restrict__ 
     nfull = (n_tail + blk) / GK;
     j0 = (p0 - n_tail) / GK;
     count0 = c.prot_gstart[size_t(u) * size_t(c.nG + 1) + size_t(j0)];
-    nK = nfull * kSliceCh * kw;
+    nK = nfull * kSliceCh * kthr;
   }
 
   // ------------------------------------------------------------------ V
-  constexpr int vper = VB < 16 ? 32 / VB : 1;  // channels per V code word
-  const int vw = c.vw;
-  const int nV = (VB < 16 && !c.vrot_b) ? tpc * vw : 0;
+  // likewise for V: vper channels of one token into vwpt words per thread
+  constexpr int vper = VB < 16 ? (VB == 3 ? 32 : 32 / VB) : 1;
+  constexpr int vwpt = VB == 3 ? 3 : 1;
+  const int vthr = kHeadDim / vper;  // threads per token
+  const int nV = (VB < 16 && !c.vrot_b) ? tpc * vthr : 0;
   if constexpr (VB == 16) {
     const uint4* src = reinterpret_cast<const uint4*>(vu + size_t(t_lo) * d);
     uint4* dst = reinterpret_cast<uint4*>(c.v_raw + (size_t(u) * c.cap + p0 + t_lo) * d);
@@ -320,8 +350,8 @@ commit_kernel(const __grid_constant__ CacheView c, const uint16_t* __restrict__ 
       reinterpret_cast<uint4*>(c.v_sink + (size_t(u) * c.sink + size_t(p0 + t)) * d)[o] =
           reinterpret_cast<const uint4*>(vu + size_t(t) * d)[o];
     }
-    if (c.vrot_b) {
-      // rotated V (no sink): warp wv rotates and quantizes tokens t_lo + wv, + 8, ...
+    if (VB != 3 && c.vrot_b) {
+      // rotated V (no sink; 2 or 4 bits): warp wv rotates and quantizes tokens t_lo + wv, + 8, ...
       int pm[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) pm[e] = __ldg(c.vrot_perm + 4 * lane + e);
@@ -335,7 +365,8 @@ commit_kernel(const __grid_constant__ CacheView c, const uint16_t* __restrict__ 
         }
         rotate_row(x, c.vrot_b, c.vrot_norm, c.vrot_mix, lane);
         const size_t tok = size_t(u) * c.cap + size_t(p0 + t);
-        quant_v_rotated<VB>(x, c.GV, c.v_codes + tok * c.vw, c.v_sz + tok * c.vgroups, lane, range);
+        quant_v_rotated<VB == 3 ? 4 : VB>(x, c.GV, c.v_codes + tok * c.vw, c.v_sz + tok * c.vgroups,
+                                          lane, range);
       }
     }
   }
@@ -345,7 +376,7 @@ commit_kernel(const __grid_constant__ CacheView c, const uint16_t* __restrict__ 
     if constexpr (KB < 16) {
       if (it < nK) {
         constexpr int levels = (1 << KB) - 1;
-        const int w = it % kw, cl = (it / kw) % kSliceCh, gi = it / (kw * kSliceCh);
+        const int w = it % kthr, cl = (it / kthr) % kSliceCh, gi = it / (kthr * kSliceCh);
         const int ch = kSliceCh * sl + cl;
         const int64_t j = j0 + gi;
         const uint32_t* tmask = c.tail_mask + size_t(u) * c.twords;
@@ -358,7 +389,7 @@ commit_kernel(const __grid_constant__ CacheView c, const uint16_t* __restrict__ 
           before += group_mask(c, tmask, pwu, n_tail, g, j0 + g, c.P - before, gm, cut);
         const int kept = group_mask(c, tmask, pwu, n_tail, gi, j, c.P - before, gm, cut);
         if (cut && cl == 0 && w == 0) atomicOr(c.status, uint32_t(DKV_FLAG_CAPACITY));
-        // this word's tokens: t = w kper + e of the group, pending index
+        // this thread's tokens: t = w kper + e of the group, pending index
         // gi GK + t (tail slot below n_tail, else block row)
         const int tw = w * kper;
         // (a select chain, not a dynamic index: gm stays in registers)
@@ -383,15 +414,16 @@ commit_kernel(const __grid_constant__ CacheView c, const uint16_t* __restrict__ 
             mx = fmaxf(mx, f);
           }
         }
-        group_minmax(mn, mx, kw);
+        group_minmax(mn, mx, kthr);
         if (mn > mx) mn = mx = 0.f;  // every token protected
         const GroupQuant q = make_quant(mn, mx, levels);
-        uint32_t word = 0;
-#pragma unroll
-        for (int e = 0; e < kper; ++e)
-          if (!((mw >> e) & 1u)) word |= code_of(x[e], q, levels) << (e * KB);  // protected: 0
+        uint32_t words[kwpt];
+        pack_codes<KB, kper>(
+            [&](int e) { return ((mw >> e) & 1u) ? 0u : code_of(x[e], q, levels); },  // protected: 0
+            words);
         const size_t gidx = (size_t(u) * c.nG + size_t(j)) * d + ch;
-        c.k_codes[gidx * kw + w] = word;
+#pragma unroll
+        for (int i = 0; i < kwpt; ++i) c.k_codes[gidx * c.kw + w * kwpt + i] = words[i];
         if (w == 0) c.k_sz[gidx] = q.sz;
         // protected tokens of this word: side-table entry = entries before the
         // group + protected tokens of the group before this one
@@ -421,8 +453,8 @@ commit_kernel(const __grid_constant__ CacheView c, const uint16_t* __restrict__ 
     if constexpr (VB < 16) {
       constexpr int levels = (1 << VB) - 1;
       const int iv = it - nK;
-      const int w = iv % vw, t = t_lo + iv / vw;
-      const int wpg = c.GV / vper;  // words per V group
+      const int w = iv % vthr, t = t_lo + iv / vthr;
+      const int wpg = c.GV / vper;  // threads per V group
       const uint16_t* src = vu + size_t(t) * d + w * vper;
       float x[vper];
       float mn = __int_as_float(0x7f800000), mx = -__int_as_float(0x7f800000);
@@ -442,11 +474,11 @@ commit_kernel(const __grid_constant__ CacheView c, const uint16_t* __restrict__ 
       }
       group_minmax(mn, mx, wpg);
       const GroupQuant q = make_quant(mn, mx, levels);
-      uint32_t word = 0;
-#pragma unroll
-      for (int e = 0; e < vper; ++e) word |= code_of(x[e], q, levels) << (e * VB);
+      uint32_t words[vwpt];
+      pack_codes<VB, vper>([&](int e) { return code_of(x[e], q, levels); }, words);
       const size_t tok = size_t(u) * c.cap + size_t(p0 + t);
-      c.v_codes[tok * vw + w] = word;
+#pragma unroll
+      for (int i = 0; i < vwpt; ++i) c.v_codes[tok * c.vw + w * vwpt + i] = words[i];
       if (w % wpg == 0) c.v_sz[tok * c.vgroups + w / wpg] = q.sz;
     }
   }
@@ -506,6 +538,7 @@ cudaError_t launch_k(const CacheView& c, const uint16_t* k, const uint16_t* v,
                      const uint32_t* pw, const CommitArgs& ca, cudaStream_t s) {
   switch (c.vb) {
     case 2: return launch_kv<KB, 2>(c, k, v, pw, ca, s);
+    case 3: return launch_kv<KB, 3>(c, k, v, pw, ca, s);
     case 4: return launch_kv<KB, 4>(c, k, v, pw, ca, s);
     default: return launch_kv<KB, 16>(c, k, v, pw, ca, s);
   }
@@ -532,6 +565,7 @@ cudaError_t launch_commit(const CacheView& c, const uint16_t* k, const uint16_t*
                           const uint32_t* pw, const CommitArgs& ca, cudaStream_t s) {
   switch (c.kb) {
     case 2: return launch_k<2>(c, k, v, pw, ca, s);
+    case 3: return launch_k<3>(c, k, v, pw, ca, s);
     case 4: return launch_k<4>(c, k, v, pw, ca, s);
     default: return launch_k<16>(c, k, v, pw, ca, s);
   }

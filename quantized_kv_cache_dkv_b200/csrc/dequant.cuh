@@ -107,6 +107,41 @@ __device__ __forceinline__ void dequant2x16_raw(uint32_t w, __half2 s2, __half2 
   b.w = h2u(__hfma2(unbias(and_or(w8, 0x00C000C0u, kMagic1024), 0.015625f, -16.f), s2, z2));
 }
 
+// Code e (0..31) of 32 three-bit codes packed little-endian into the 96-bit
+// stream w2:w1:w0 (codes 10 and 21 straddle two words).
+template <int e>
+__device__ __forceinline__ uint32_t code3(uint32_t w0, uint32_t w1, uint32_t w2) {
+  constexpr int pos = 3 * e, wi = pos / 32, off = pos % 32;
+  const uint32_t a = wi == 0 ? w0 : (wi == 1 ? w1 : w2);
+  if constexpr (off <= 29) {
+    return (a >> off) & 7u;
+  } else {
+    const uint32_t b = wi == 0 ? w1 : w2;
+    return __funnelshift_r(a, b, off) & 7u;
+  }
+}
+
+template <int i>
+__device__ __forceinline__ uint32_t dequant3_pair(uint32_t w0, uint32_t w1, uint32_t w2,
+                                                  __half2 s2, __half2 z2) {
+  // 1024 + c in each half (exact), minus 1024 (exact), then c * s + z (one rounding)
+  const uint32_t x = code3<2 * i>(w0, w1, w2) | (code3<2 * i + 1>(w0, w1, w2) << 16) | kMagic1024;
+  return h2u(__hfma2(__hsub2(u2h(x), h2c(1024.f)), s2, z2));
+}
+
+// 32 three-bit codes -> 32 halves q*s+z in element order (out[k] = e 8k..8k+7)
+__device__ __forceinline__ void dequant3x32(uint32_t w0, uint32_t w1, uint32_t w2, __half2 s2,
+                                            __half2 z2, uint4 (&out)[4]) {
+  out[0] = make_uint4(dequant3_pair<0>(w0, w1, w2, s2, z2), dequant3_pair<1>(w0, w1, w2, s2, z2),
+                      dequant3_pair<2>(w0, w1, w2, s2, z2), dequant3_pair<3>(w0, w1, w2, s2, z2));
+  out[1] = make_uint4(dequant3_pair<4>(w0, w1, w2, s2, z2), dequant3_pair<5>(w0, w1, w2, s2, z2),
+                      dequant3_pair<6>(w0, w1, w2, s2, z2), dequant3_pair<7>(w0, w1, w2, s2, z2));
+  out[2] = make_uint4(dequant3_pair<8>(w0, w1, w2, s2, z2), dequant3_pair<9>(w0, w1, w2, s2, z2),
+                      dequant3_pair<10>(w0, w1, w2, s2, z2), dequant3_pair<11>(w0, w1, w2, s2, z2));
+  out[3] = make_uint4(dequant3_pair<12>(w0, w1, w2, s2, z2), dequant3_pair<13>(w0, w1, w2, s2, z2),
+                      dequant3_pair<14>(w0, w1, w2, s2, z2), dequant3_pair<15>(w0, w1, w2, s2, z2));
+}
+
 // 8 bf16 -> 8 fp16 (exact inside fp16's normal range)
 __device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 x) {
   auto cvt = [](uint32_t w) -> uint32_t {

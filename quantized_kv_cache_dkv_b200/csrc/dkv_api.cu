@@ -78,9 +78,9 @@ int check_config(const dkv_config* c) {
     return fail(DKV_ERR_UNSUPPORTED, "block must be a multiple of 32 and <= 128");
   if ((c->q_heads / c->kv_heads) * c->block > 256)
     return fail(DKV_ERR_UNSUPPORTED, "(q_heads/kv_heads)*block must be <= 256");
-  auto okbits = [](int b) { return b == 2 || b == 4 || b == 16; };
+  auto okbits = [](int b) { return b == 2 || b == 3 || b == 4 || b == 16; };
   if (!okbits(c->k_bits) || !okbits(c->v_bits))
-    return fail(DKV_ERR_UNSUPPORTED, "k_bits/v_bits must be 2, 4 or 16");
+    return fail(DKV_ERR_UNSUPPORTED, "k_bits/v_bits must be 2, 3, 4 or 16");
   auto okgrp = [](int g) { return g == 32 || g == 64 || g == 128; };
   if (c->k_bits < 16) {
     if (!okgrp(c->k_group)) return fail(DKV_ERR_UNSUPPORTED, "k_group must be 32, 64 or 128");
@@ -729,6 +729,7 @@ int dkv_cache_set_v_rotation(dkv_cache* c, const int32_t* perm, const float* mix
   if (block != 16 && block != 32 && block != 64 && block != 128)
     return fail(DKV_ERR_UNSUPPORTED, "rotation block must be 16, 32, 64 or 128");
   if (c->v.vb == 16) return fail(DKV_ERR_UNSUPPORTED, "V rotation needs quantized V (v_bits < 16)");
+  if (c->v.vb == 3) return fail(DKV_ERR_UNSUPPORTED, "V rotation needs 2- or 4-bit V");
   if (c->v.sink > 0) return fail(DKV_ERR_UNSUPPORTED, "V rotation with an attention sink is not supported");
   if (!perm || !mix) return fail(DKV_ERR_INVALID_ARG, "perm and mix must not be NULL");
   const int d = dkv::kHeadDim, k = d / block;

@@ -7,7 +7,8 @@ record DKV_FLAG_BOUNDS instead of making an out-of-range access).
 
 Each case draws bit widths, group sizes, block, heads, fill level (empty up
 to a full cache), side-table size (some too small, so the capacity path
-runs), sink length, a roll-back and recommit; commits through the library and
+runs), sink length, a roll-back and recommit (bit widths 2, 3, 4 and 16);
+commits through the library and
 the oracle, compares the exported state bit for bit and the status flags
 exactly (the oracle never sets DKV_FLAG_BOUNDS), and the block attention of
 both attention kernels, with and without splits, within the output bound.
@@ -27,7 +28,7 @@ from gpu_util import (assert_close, commit_both, compare_exports, dev_bf16,  # n
 
 
 def draw_case(r: np.random.Generator, i: int):
-    kb, vb = (int(x) for x in r.choice([2, 4, 16], 2))
+    kb, vb = (int(x) for x in r.choice([2, 3, 4, 16], 2))
     gk, gv = (int(x) for x in r.choice([32, 64, 128], 2))
     blk = int(r.choice([32, 64, 128]))
     g = int(r.choice([g for g in (1, 2, 4, 8) if g * blk <= 256]))
@@ -71,7 +72,7 @@ def run_case(dkv, torch, w, n_blocks, cap, P, sink, trunc):
     Q = synth.queries_bits(w, 0)
     Ka, Va = synth.active_block_bits(w, 0)
     ref = oc.block_attention(Q, Ka, Va, w.softmax_scale)
-    for kernel in (1, 2):
+    for kernel in ((1,) if 3 in (w.k_bits, w.v_bits) else (1, 2)):   # 3 bits: mma.sync only
         dkv.dkv_cache_set_option(cache, dkv.DKV_OPT_ATTN_KERNEL, kernel)
         for sp in (0, 2):
             dkv.dkv_cache_set_option(cache, dkv.DKV_OPT_SPLITS, sp)

@@ -46,7 +46,8 @@ def _alloc_rc(**over):
 
 @pytest.mark.parametrize("over,code", [
     (dict(d=64), dkv.DKV_ERR_UNSUPPORTED),
-    (dict(k_bits=3), dkv.DKV_ERR_UNSUPPORTED),
+    (dict(k_bits=5), dkv.DKV_ERR_UNSUPPORTED),
+    (dict(B=513), dkv.DKV_ERR_UNSUPPORTED),
     (dict(v_bits=8), dkv.DKV_ERR_UNSUPPORTED),
     (dict(k_group=48), dkv.DKV_ERR_UNSUPPORTED),
     (dict(v_group=16), dkv.DKV_ERR_UNSUPPORTED),
