@@ -151,6 +151,35 @@ int dkv_block_attention(dkv_cache* cache, const void* q, const void* k_act,
                         const void* v_act, float softmax_scale, void* out,
                         void* stream);
 
+/* Q-MaskAhead selection (MaskAhead / Q-MaskAhead abstract: the queries of the
+ * block being denoised score the cached entries by their expected share of
+ * the attention output, the block attends to the best-scored ones, and the
+ * quantized variant scores and attends on the low-bit cache).  The abstract
+ * gives no formula; the reading taken here: for every (sequence, kv-head)
+ * unit and committed token j,
+ *   c_j = (sum over the unit's query rows i of p_ij) * ||v_hat_j||_2,
+ * p_ij the softmax weight of token j for row i in the full attention of this
+ * call (committed tokens and active block, from the dequantized cache);
+ * the min(budget, len) tokens of largest c_j are kept (equal scores: the
+ * lower position first), and every query row attends to them plus the
+ * whole active block: out = softmax(softmax_scale * q K_sel^T) V_sel, bf16.
+ * Arguments as in dkv_block_attention, and:
+ *   budget    tokens kept per unit, 0 <= budget <= max_tokens
+ *   selected  device int32 [B, Hkv, budget], or NULL: the kept positions of
+ *             each unit in increasing order, -1 after the last
+ *   scores    device fp32 [B, Hkv, max_tokens], or NULL: c_j at [.., j] for
+ *             j < the sequence's length
+ * Launches: the split attention kernel (for each row's softmax max and sum),
+ * a scoring kernel, a per-unit top-k kernel (radix select), the mma.sync
+ * attention over the gathered tokens, and the combine when it splits.  The
+ * first call on a handle allocates its workspace ([B*Hkv, max_tokens] x 3
+ * fp32/int32 words); make it before any stream capture.  Not available on a
+ * rotated-V cache (DKV_ERR_UNSUPPORTED); query groups must be a multiple of
+ * 16 rows. */
+int dkv_block_attention_selected(dkv_cache* cache, const void* q, const void* k_act,
+                                 const void* v_act, float softmax_scale, int32_t budget,
+                                 void* out, int32_t* selected, float* scores, void* stream);
+
 /* Dual-cache attention (the prefix and dual cache reuse of Fast-dLLM-style
  * decoding that "KV Cache Quantization for Diffusion Language Models"
  * quantizes, abstract): the active block's queries attend to `prefix` (the

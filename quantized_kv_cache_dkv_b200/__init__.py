@@ -91,6 +91,8 @@ _seq_lens = _sig("dkv_cache_seq_lens", [_P, _P])
 _truncate_seq = _sig("dkv_cache_truncate_seq", [_P, ctypes.c_int32, ctypes.c_int64, _P])
 _export_seq = _sig("dkv_cache_export_seq", [_P, ctypes.c_int32, _P, ctypes.POINTER(dkv_export)])
 _attn = _sig("dkv_block_attention", [_P, _P, _P, _P, ctypes.c_float, _P, _P])
+_attn_sel = _sig("dkv_block_attention_selected", [_P, _P, _P, _P, ctypes.c_float, ctypes.c_int32,
+                                                  _P, _P, _P, _P])
 _attn_noalloc = _sig("dkv_block_attention_noalloc", [_P, _P, _P, _P, ctypes.c_float, _P, _P])
 DKV_NOALLOC_SCRATCH_BYTES = 16 << 20
 _len = _sig("dkv_cache_len", [_P, ctypes.POINTER(ctypes.c_int64)])
@@ -227,6 +229,29 @@ def dkv_block_attention(cache: Cache, q, k_act, v_act, softmax_scale: float, out
                   (torch.bfloat16, torch.int16))
     _check(_attn(cache.h, _ptr(q), _ptr(k_act), _ptr(v_act), ctypes.c_float(softmax_scale),
                  _ptr(out), _stream(stream)))
+
+
+def dkv_block_attention_selected(cache: Cache, q, k_act, v_act, softmax_scale: float,
+                                 budget: int, out, selected=None, scores=None,
+                                 stream=None) -> None:
+    """Q-MaskAhead selection: attention over the `budget` committed tokens
+    of largest contribution score per (sequence, kv-head) plus the active
+    block.  selected: int32 [B, Hkv, budget] or None (the kept positions,
+    ascending, -1 after them); scores: float32 [B, Hkv, max_tokens] or None."""
+    import torch
+    c = cache.cfg
+    _tensor_check(q, (c.batch, c.q_heads, c.block, c.head_dim), "q", (torch.bfloat16, torch.int16))
+    shp = (c.batch, c.kv_heads, c.block, c.head_dim)
+    _tensor_check(k_act, shp, "k_act", (torch.bfloat16, torch.int16))
+    _tensor_check(v_act, shp, "v_act", (torch.bfloat16, torch.int16))
+    _tensor_check(out, (c.batch, c.q_heads, c.block, c.head_dim), "out",
+                  (torch.bfloat16, torch.int16))
+    if selected is not None:
+        _tensor_check(selected, (c.batch, c.kv_heads, budget), "selected", (torch.int32,))
+    if scores is not None:
+        _tensor_check(scores, (c.batch, c.kv_heads, c.max_tokens), "scores", (torch.float32,))
+    _check(_attn_sel(cache.h, _ptr(q), _ptr(k_act), _ptr(v_act), ctypes.c_float(softmax_scale),
+                     int(budget), _ptr(out), _ptr(selected), _ptr(scores), _stream(stream)))
 
 
 def dkv_block_attention_noalloc(cache: Cache, q, k_act, v_act, softmax_scale: float, out,

@@ -30,6 +30,7 @@ struct dkv_cache {
   size_t arena_bytes = 0;
   float* part_o = nullptr;
   float2* part_ml = nullptr;
+  void* sel_mem = nullptr;       // selection workspace (first dkv_block_attention_selected)
   void* vrot_mem = nullptr;      // rotation parameters + rotated active block (V rotation)
   uint16_t* vrot_act = nullptr;  // [U][blk][d] bf16
   int32_t max_splits = 1;
@@ -368,8 +369,9 @@ int dkv_cache_free(dkv_cache* c) {
   if (!c) return fail(DKV_ERR_INVALID_ARG, "cache is NULL");
   cudaError_t e = cudaDeviceSynchronize();
   cudaError_t e2 = cudaFree(c->arena);
-  if (c->vrot_mem) {
-    const cudaError_t e3 = cudaFree(c->vrot_mem);
+  for (void* m : {c->vrot_mem, c->sel_mem}) {
+    if (!m) continue;
+    const cudaError_t e3 = cudaFree(m);
     if (e2 == cudaSuccess) e2 = e3;
   }
   for (auto& r : c->prof) {
@@ -629,6 +631,91 @@ int dkv_block_attention_dual(dkv_cache* c, dkv_cache* sfx, const void* q, const 
   c->last_kernel = k1;
   c->last_splits = total;
   c->last_launches = 3;
+  return DKV_OK;
+}
+
+int dkv_block_attention_selected(dkv_cache* c, const void* q, const void* k_act,
+                                 const void* v_act, float softmax_scale, int32_t budget, void* out,
+                                 int32_t* selected, float* scores, void* stream) {
+  dkv::NvtxRange nvtx_range("dkv_block_attention_selected");
+  g_err.clear();
+  if (!c || !q || !k_act || !v_act || !out) return fail(DKV_ERR_INVALID_ARG, "NULL argument");
+  if (!aligned16(q) || !aligned16(k_act) || !aligned16(v_act) || !aligned16(out) ||
+      (reinterpret_cast<uintptr_t>(selected) & 3u) || (reinterpret_cast<uintptr_t>(scores) & 3u))
+    return fail(DKV_ERR_INVALID_ARG, "q, k_act, v_act and out must be 16-byte aligned, "
+                                     "selected and scores 4-byte aligned");
+  if (!(softmax_scale == softmax_scale) || softmax_scale > 3.0e38f || softmax_scale < -3.0e38f)
+    return fail(DKV_ERR_INVALID_ARG, "softmax_scale must be finite");
+  const dkv::CacheView& v = c->v;
+  if (budget < 0 || budget > v.cap) return fail(DKV_ERR_INVALID_ARG, "budget must be in [0, max_tokens]");
+  if (v.vrot_b) return fail(DKV_ERR_UNSUPPORTED, "selection over a rotated-V cache is not supported");
+  if (v.rows % 16) return fail(DKV_ERR_UNSUPPORTED, "(q_heads/kv_heads)*block must be a multiple of 16");
+  dkv::CacheInfo ci;
+  dkv::cache_info(c, &ci);
+  const int drc = dkv::check_device(ci);
+  if (drc != DKV_OK) return drc;
+  // workspace, [U][cap] each: row-block shares of the scores, scores, selection
+  const int nrb = dkv::score_row_blocks(v);
+  const size_t cells = size_t(v.U) * size_t(v.cap);
+  const size_t part_b = align256(cells * nrb * 4), sc_b = align256(cells * 4);
+  if (!c->sel_mem) DKV_CUDA(cudaMalloc(&c->sel_mem, part_b + sc_b + cells * 4));
+  float* part = static_cast<float*>(c->sel_mem);
+  float* sc = scores ? scores : reinterpret_cast<float*>(static_cast<char*>(c->sel_mem) + part_b);
+  int32_t* sel = selected ? selected
+                          : reinterpret_cast<int32_t*>(static_cast<char*>(c->sel_mem) + part_b + sc_b);
+  const int32_t sel_ld = selected ? budget : int32_t(v.cap);
+
+  dkv::AttnArgs a{};
+  a.c = v;
+  a.q = static_cast<const uint16_t*>(q);
+  a.k_act = static_cast<const uint16_t*>(k_act);
+  a.v_act = static_cast<const uint16_t*>(v_act);
+  a.out = static_cast<uint16_t*>(out);
+  a.part_o = c->part_o;
+  a.part_ml = c->part_ml;
+  a.scale_log2 = softmax_scale * 1.4426950408889634f;
+  int kernel = 0;
+  const char* perr = nullptr;
+  int prc = dkv::plan_attention(ci, &a, &kernel, &perr);
+  if (prc != DKV_OK) return fail(prc, perr);
+  a.final_out = 0;  // the first pass keeps every row's (max, sum) in the split partials
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = timed_launch(c, DKV_KERNEL_ATTENTION, s, [&] {
+    return kernel == 2 ? dkv::launch_attention_tc(a, s) : dkv::launch_attention_mma(a, s);
+  });
+  if (e != cudaSuccess) return fail(DKV_ERR_CUDA, std::string("attention launch: ") + cudaGetErrorString(e));
+  // contributions of the committed tokens, then the selection
+  dkv::AttnArgs sa = a;
+  sa.with_active = 0;
+  sa.sel = sel;
+  sa.sel_ld = sel_ld;
+  sa.budget = budget;
+  e = dkv::launch_scores(sa, part, v.cap, s);
+  if (e == cudaSuccess) e = dkv::launch_topk(sa, part, v.cap, sc, sel, s);
+  if (e != cudaSuccess) return fail(DKV_ERR_CUDA, std::string("selection launch: ") + cudaGetErrorString(e));
+  // attention over the selected tokens and the active block (mma.sync gather)
+  dkv::CacheInfo cg = ci;
+  cg.len = std::min<int64_t>(budget, ci.len);
+  cg.opt_kernel = 1;
+  dkv::AttnArgs ga = a;
+  prc = dkv::plan_attention(cg, &ga, &kernel, &perr);
+  if (prc != DKV_OK) return fail(prc, perr);
+  ga.lens = ci.lens;  // unit_len takes min(budget, each sequence's length)
+  ga.gather = 1;
+  ga.sel = sel;
+  ga.sel_ld = sel_ld;
+  ga.budget = budget;
+  e = timed_launch(c, DKV_KERNEL_ATTENTION, s, [&] { return dkv::launch_attention_mma(ga, s); });
+  if (e != cudaSuccess) return fail(DKV_ERR_CUDA, std::string("selected attention launch: ") + cudaGetErrorString(e));
+  int launches = 4;
+  if (!ga.final_out) {
+    e = timed_launch(c, DKV_KERNEL_COMBINE, s, [&] { return dkv::launch_combine(ga, s); });
+    if (e != cudaSuccess) return fail(DKV_ERR_CUDA, std::string("combine launch: ") + cudaGetErrorString(e));
+    ++launches;
+  }
+  c->last_kernel = 1;
+  c->last_splits = ga.nsplit;
+  c->last_launches = launches;
   return DKV_OK;
 }
 

@@ -129,6 +129,12 @@ struct AttnArgs {
                             // no rotation); 0: fp32 partials for combine_kernel
   int32_t part_base;        // split sp of unit u writes partial u*part_stride +
   int32_t part_stride;      // part_base + sp (one call: 0 and nsplit)
+  // Attention over selected committed tokens (mma.sync kernel, gather = 1):
+  // slot i < min(budget, L) of unit u is token sel[u * sel_ld + i]
+  const int32_t* sel;
+  int32_t sel_ld;
+  int32_t budget;
+  int32_t gather;
   uint64_t wait_limit_ns;   // limit of one bounded wait in the tcgen05 kernel
   int32_t test_stall_tile;  // bounds-checking build: tile whose copies the
                             // tcgen05 loader withholds (-1: none)
@@ -144,9 +150,14 @@ struct UnitLen {
 __device__ __forceinline__ UnitLen unit_len(const AttnArgs& a, int u) {
   const int32_t L = a.lens.len[u / a.c.Hkv];
   UnitLen r;
-  r.L = L;
-  r.Lq = a.c.kb < 16 ? (L / a.c.GK) * a.c.GK : L;
-  r.n_tok = L + (a.with_active ? a.c.blk : 0);
+  if (a.gather) {
+    // the selected slots take the place of the committed tokens
+    r.L = r.Lq = L < a.budget ? L : a.budget;
+  } else {
+    r.L = L;
+    r.Lq = a.c.kb < 16 ? (L / a.c.GK) * a.c.GK : L;
+  }
+  r.n_tok = r.L + (a.with_active ? a.c.blk : 0);
   return r;
 }
 
@@ -172,6 +183,17 @@ cudaError_t launch_rotate_v_rows(const CacheView& c, const uint16_t* src, uint16
 constexpr int kMmaTile = 64;
 cudaError_t launch_attention_mma(const AttnArgs& a, cudaStream_t s);
 cudaError_t launch_combine(const AttnArgs& a, cudaStream_t s);
+// Q-MaskAhead selection (mma.sync kernels).  Scores: for every committed
+// token j of unit u and row block rb, part[(u * nrb + rb) * ld + j] = (sum
+// over the block's rows i of p_ij) * ||v_hat_j||, with p_ij the softmax weight
+// of the whole call, from the split partials a.part_ml (a.with_active = 0).
+int score_row_blocks(const CacheView& c);
+cudaError_t launch_scores(const AttnArgs& a, float* part, int64_t ld, cudaStream_t s);
+// Per unit: scores[u * ld + j] = sum over row blocks of part, then the
+// min(budget, L) largest (ties: lower position) into sel[u * sel_ld + ...]
+// in increasing position order, -1 after them.
+cudaError_t launch_topk(const AttnArgs& a, const float* part, int64_t ld, float* scores,
+                        int32_t* sel, cudaStream_t s);
 
 // tcgen05 kernel: token tile of 128, rows == 128.
 constexpr int kTcTile = 128;
