@@ -692,6 +692,14 @@ def base_line(w, args, value, ms_per_step, world):
     }
 
 
+def plan_name(w: synth.Workload, kernel: int) -> str:
+    if kernel == 1:
+        return "mma.sync"
+    if kernel == 2 and w.rows == 32:
+        return "tcgen05 (tokens on TMEM lanes)"
+    return "tcgen05 (query-row blocks)" if kernel in (2, 3) else str(kernel)
+
+
 def kernel_fields(w: synth.Workload, r: dict) -> dict:
     """Per-kernel figures of one run: times in the timed (graph) execution
     and in the eager pass, commit rate, launch plan."""
@@ -706,7 +714,7 @@ def kernel_fields(w: synth.Workload, r: dict) -> dict:
         "kernel_us_eager": {"attention": round(r["att_ms"] / max(r["att_n"], 1) * 1e3, 3),
                             "combine": round(r["combine_ms"] / max(r["combine_n"], 1) * 1e3, 3),
                             "commit": round(r["commit_ms"] / max(r["commit_n"], 1) * 1e3, 3)},
-        "attention_plan": {"kernel": ["", "mma.sync", "tcgen05"][r["plan"][0]],
+        "attention_plan": {"kernel": plan_name(w, r["plan"][0]),
                            "splits": r["plan"][1], "launches": r["plan"][2]},
     }
 
@@ -722,8 +730,9 @@ def main():
                          "largest single-GPU configuration)")
     ap.add_argument("--no-sub-records", action="store_true",
                     help="skip the per-workload records of the other configurations")
-    ap.add_argument("--kernel", type=int, default=0, choices=[0, 1, 2],
-                    help="attention kernel: 0 = library's choice, 1 = mma.sync, 2 = tcgen05")
+    ap.add_argument("--kernel", type=int, default=0, choices=[0, 1, 2, 3],
+                    help="attention kernel: 0 = library's choice, 1 = mma.sync, 2 = tcgen05, "
+                         "3 = tcgen05 with query-row blocks for every group")
     ap.add_argument("--B", type=int, default=0, help="override the workload's batch (profiling)")
     ap.add_argument("--L", type=int, default=0, help="override the committed length (profiling)")
     ap.add_argument("--v-rotation", type=int, default=0, choices=[0, 16, 32, 64, 128],

@@ -327,8 +327,10 @@ int dkv_cache_export_seq(dkv_cache* cache, int32_t seq, void* stream, dkv_export
  *     0 = chosen from the SM count (default).  Results agree within fp32
  *     rounding for any split count.
  *   DKV_OPT_ATTN_KERNEL: 0 = best available (default), 1 = warp-level
- *     mma.sync kernel, 2 = tcgen05 tensor-memory kernel (DKV_ERR_UNSUPPORTED
- *     if the shape has no tcgen05 variant).
+ *     mma.sync kernel, 2 = tcgen05 tensor-memory kernel (tokens on the TMEM
+ *     lanes for 32-row query groups, query-row blocks of up to 128 rows
+ *     otherwise), 3 = tcgen05 with query-row blocks for every group
+ *     (DKV_ERR_UNSUPPORTED for 2 and 3 if the shape has no tcgen05 variant).
  *   DKV_OPT_TEST_STALL: bounds-checking build (libdkv_bc.so) only, else
  *     DKV_ERR_UNSUPPORTED.  A test of the bounded waits: value t >= 0 makes the
  *     tcgen05 kernel's loader withhold the copies of tile t (0 = the first
@@ -352,7 +354,8 @@ int dkv_profile_read(dkv_cache* cache, int32_t kind, double* total_ms, int64_t* 
 
 /* Launch description of the last dkv_block_attention (or
  * dkv_block_attention_dual, recorded on the prefix handle) on this handle:
- * the kernel used (1 = mma.sync, 2 = tcgen05; the prefix's for a dual call),
+ * the kernel used (1 = mma.sync, 2 or 3 = tcgen05 as in DKV_OPT_ATTN_KERNEL;
+ * the prefix's for a dual call),
  * the split count (prefix + suffix splits for a dual call), and how many
  * kernels it launched (attention, plus the combine unless one split wrote
  * the output directly, plus the active-block rotation of a rotated-V cache;

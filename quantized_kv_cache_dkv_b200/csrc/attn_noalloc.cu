@@ -97,7 +97,7 @@ extern "C" int dkv_block_attention_noalloc(dkv_cache* cache, const void* q, cons
       return report_error(DKV_ERR_CUDA, (std::string("rotation launch: ") + cudaGetErrorString(e)).c_str());
     a.v_act = ci.vrot_act;
   }
-  e = kernel == 2 ? dkv::launch_attention_tc(a, s) : dkv::launch_attention_mma(a, s);
+  e = kernel >= 2 ? dkv::launch_attention_tc(a, s) : dkv::launch_attention_mma(a, s);
   if (e != cudaSuccess)
     return report_error(DKV_ERR_CUDA, (std::string("attention launch: ") + cudaGetErrorString(e)).c_str());
   if (!a.final_out) {

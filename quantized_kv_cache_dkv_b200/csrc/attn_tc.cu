@@ -686,6 +686,189 @@ __device__ __noinline__ void fill_v_general(const AttnArgs& a, const UnitLen ul,
   }
 }
 
+// ------------------------------------------------------------ shared pipeline loops
+
+// Shared-memory addresses of one kernel's pipeline: the ring of packed
+// tiles, the two dequantized K and V tile buffers, and the barriers that
+// hand them over (entry i of a barrier pair or ring at +8 i).
+struct Pipe {
+  uint8_t* sm;
+  uint32_t sm_base;
+  uint32_t ring;              // offset of ring stage 0 (stages kStageBytes apart)
+  uint32_t k_buf0, v_buf0;    // offsets of K / V tile buffer 0 (buffer 1 at + kTileBytes)
+  uint32_t kfull, kempty, vfull, vempty, rfull, rempty;  // barrier addresses
+};
+
+// K producer thread pt (0..255): channel pt % 128, token chunks 2 qh, 2 qh + 1
+// of every tile, qh = pt / 128.
+template <int KB, int STAGES>
+__device__ __forceinline__ void k_producer_loop(const AttnArgs& a, const UnitLen* uls, int u,
+                                                int64_t t_begin, int nt, const Pipe& p,
+                                                volatile int* abort_flag, int pt) {
+  const CacheView& cv = a.c;
+  const int c = pt & 127;   // channel
+  const int qh = pt >> 7;   // chunks 2qh, 2qh+1 of each tile
+  const KOffsets ko(c, qh, cv.GK, cv.kw, KB < 16 ? KB : 16);
+#pragma unroll 1
+  for (int j = 0; j < nt; ++j) {
+    const int b = j & 1, st = j % STAGES;
+    if (!mbar_wait(p.kempty + 8u * b, ((j >> 1) & 1) ^ 1, a, abort_flag)) break;
+    if (!mbar_wait(p.rfull + 8u * st, (j / STAGES) & 1, a, abort_flag)) break;
+    fill_k_tile<KB>(a, *uls, u, (t_begin + j) * TT, p.sm + p.k_buf0 + b * kTileBytes,
+                    p.sm + p.ring + st * Smem::kStageBytes, c, qh, ko);
+    fence_async_smem();
+    mbar_arrive(p.kfull + 8u * b);
+    mbar_arrive(p.rempty + 8u * st);
+  }
+}
+
+// V producer thread pt (0..255).
+template <int KB, int VB, bool SINK, int STAGES>
+__device__ __forceinline__ void v_producer_loop(const AttnArgs& a, const UnitLen* uls, int u,
+                                                int64_t t_begin, int nt, const Pipe& p,
+                                                volatile int* abort_flag, int pt) {
+  const CacheView& cv = a.c;
+  const VOffsets<KB> vo(pt, cv.vw, cv.vgroups, cv.GV, VB < 16 ? VB : 16);
+#pragma unroll 1
+  for (int j = 0; j < nt; ++j) {
+    const int b = j & 1, st = j % STAGES;
+    if (!mbar_wait(p.vempty + 8u * b, ((j >> 1) & 1) ^ 1, a, abort_flag)) break;
+    if (!mbar_wait(p.rfull + 8u * st, (j / STAGES) & 1, a, abort_flag)) break;
+    fill_v_tile<KB, VB, SINK>(a, *uls, u, (t_begin + j) * TT, p.sm + p.v_buf0 + b * kTileBytes,
+                              p.sm + p.ring + st * Smem::kStageBytes, pt, vo);
+    fence_async_smem();
+    mbar_arrive(p.vfull + 8u * b);
+    mbar_arrive(p.rempty + 8u * st);
+  }
+}
+
+// Loader warp: lanes prefetch the side-table group index of 32 tiles at a
+// time; lane 0 issues the bulk copies of each tile into the ring.  Token
+// positions fit in 32 bits (capacity <= 2^30) and K groups are 32, 64 or 128
+// tokens, so the group arithmetic is 32-bit shifts.
+template <int KB, int VB, int STAGES>
+__device__ __forceinline__ void loader_loop(const AttnArgs& a, const UnitLen* uls, int u,
+                                            int64_t t_begin, int nt, const Pipe& p,
+                                            volatile int* abort_flag, int lane) {
+  const CacheView& cv = a.c;
+  const int gks = KB < 16 ? __ffs(cv.GK) - 1 : 0;
+  const int Lq = uls->Lq, Lc = uls->L, t0 = int(t_begin) * TT;
+  const int32_t* gs = cv.prot_gstart + size_t(u) * size_t(cv.nG + 1);
+  int issued = 0;     // tiles 0 .. issued-1 went through the ring
+  int stalled = -1;   // (bounds-checking build) the tile whose copies were withheld
+  int pf0 = 0, pf1 = 0;  // this lane's prefetched gstart values (tile j0 + lane)
+#pragma unroll 1
+  for (int j = 0; j < nt; ++j) {
+    if constexpr (KB < 16) {
+      if ((j & 31) == 0) {
+        pf0 = pf1 = 0;
+        const int jj = j + lane;
+        const int ts = t0 + jj * TT;
+        if (jj < nt && ts < Lq && cv.P > 0) {
+          const int q_end = ts + TT < Lq ? ts + TT : Lq;
+          pf0 = __ldg(gs + (ts >> gks));
+          pf1 = __ldg(gs + (q_end >> gks));
+        }
+      }
+    }
+    const int g0 = __shfl_sync(0xffffffffu, pf0, j & 31);
+    const int g1 = __shfl_sync(0xffffffffu, pf1, j & 31);
+    const int st = j % STAGES;
+    const uint32_t rfull = p.rfull + 8u * st;
+    if (!__all_sync(0xffffffffu, mbar_wait(p.rempty + 8u * st, ((j / STAGES) & 1) ^ 1, a, abort_flag)))
+      break;
+    ++issued;
+#ifdef DKV_BOUNDS_CHECK
+    if (j == a.test_stall_tile) {
+      // test hook: nothing is copied and nothing arrives on this stage, so
+      // the producers' bounded waits on it run out (DKV_FLAG_TIMEOUT)
+      stalled = j;
+      continue;
+    }
+#endif
+    if (lane == 0) {
+      const int ts = t0 + j * TT;
+      const uint32_t dst = p.sm_base + p.ring + st * Smem::kStageBytes;
+      uint32_t kc_b = 0, ksz_b = 0, vc_b = 0, vsz_b = 0, pos_b = 0, pk_b = 0;
+      int g_lo = 0, pidx0 = 0;  // pidx0: first staged position, relative to the unit
+      const int n = g1 - g0;
+      if (KB < 16 && ts < Lq) {
+        g_lo = ts >> gks;
+        const int q_end = ts + TT < Lq ? ts + TT : Lq;  // multiple of GK
+        const uint32_t ng = uint32_t((q_end >> gks) - g_lo);
+        kc_b = ng * kHeadDim * uint32_t(cv.kw) * 4u;
+        ksz_b = ng * kHeadDim * 4u;
+        if (n > 0) {
+          const int nst = n < kStagedProt ? n : kStagedProt;
+          // 16-byte aligned superset of the staged positions (the unit's
+          // slice starts at u * P entries)
+          const int64_t e0 = int64_t(u) * cv.P + g0;
+          const int64_t ea = e0 & ~int64_t(3);
+          pidx0 = int(ea - int64_t(u) * cv.P);
+          pos_b = uint32_t(((e0 + nst + 3) & ~int64_t(3)) - ea) * 4u;
+          pk_b = uint32_t(nst) * kHeadDim * 2u;
+        }
+      }
+      if (VB < 16 && ts < Lc) {
+        const uint32_t nv = uint32_t((ts + TT < Lc ? ts + TT : Lc) - ts);
+        vc_b = nv * uint32_t(cv.vw) * 4u;
+        vsz_b = nv * uint32_t(cv.vgroups) * 4u;
+      }
+      const size_t ug = size_t(u) * size_t(cv.nG) + size_t(g_lo);
+      {
+        // bounds-checking build: each copy inside its buffer and its ring
+        // slot, else left out (the staged side table with it); the byte
+        // counts stay consistent with the expect_tx below
+        const size_t U = size_t(cv.U), P = size_t(cv.P), e = size_t(u) * P;
+        if (kc_b && !DKV_IN_BOUNDS(
+                        kc_b <= Smem::kRKsz - Smem::kRKc && ksz_b <= Smem::kRVc - Smem::kRKsz &&
+                        (ug * kHeadDim * cv.kw) * 4 + kc_b <= U * cv.nG * kHeadDim * cv.kw * 4 &&
+                        (ug * kHeadDim) * 4 + ksz_b <= U * cv.nG * kHeadDim * 4, cv.status))
+          kc_b = ksz_b = pos_b = pk_b = 0;
+        // (the staged positions are a 16-byte aligned superset: up to three
+        // entries before and after the unit's slice, inside the arena)
+        if (pos_b && !DKV_IN_BOUNDS(
+                         g0 >= 0 && int64_t(e) + pidx0 >= 0 &&
+                         pos_b <= Smem::kRPk - Smem::kRPos &&
+                         pk_b <= Smem::kStageBytes - Smem::kRPk &&
+                         (e + size_t(pidx0)) * 4 + pos_b <= (U * P + 3) * 4 &&
+                         (e + size_t(g0)) * kHeadDim * 2 + pk_b <= U * P * kHeadDim * 2, cv.status))
+          pos_b = pk_b = 0;
+        const size_t ut = size_t(u) * size_t(cv.cap) + size_t(ts);
+        if (vc_b && !DKV_IN_BOUNDS(
+                        vc_b <= Smem::kRVsz - Smem::kRVc && vsz_b <= Smem::kRHdr - Smem::kRVsz &&
+                        ut * cv.vw * 4 + vc_b <= U * size_t(cv.cap) * cv.vw * 4 &&
+                        ut * cv.vgroups * 4 + vsz_b <= U * size_t(cv.cap) * cv.vgroups * 4, cv.status))
+          vc_b = vsz_b = 0;
+      }
+      int* hdr = reinterpret_cast<int*>(p.sm + p.ring + st * Smem::kStageBytes + Smem::kRHdr);
+      hdr[0] = pos_b ? n : 0;  // pos_b is set exactly when the tile has protected rows
+      hdr[1] = g0;
+      hdr[2] = pidx0;
+      mbar_arrive_expect_tx(rfull, kc_b + ksz_b + vc_b + vsz_b + pos_b + pk_b);
+      if (kc_b) {
+        bulk_g2s(dst + Smem::kRKc, cv.k_codes + ug * kHeadDim * cv.kw, kc_b, rfull);
+        bulk_g2s(dst + Smem::kRKsz, cv.k_sz + ug * kHeadDim, ksz_b, rfull);
+      }
+      if (pos_b) {
+        const size_t e = size_t(u) * size_t(cv.P);
+        bulk_g2s(dst + Smem::kRPos, cv.prot_pos + e + size_t(pidx0), pos_b, rfull);
+        bulk_g2s(dst + Smem::kRPk, cv.prot_k + (e + size_t(g0)) * kHeadDim, pk_b, rfull);
+      }
+      if (vc_b) {
+        const size_t ut = size_t(u) * size_t(cv.cap) + size_t(ts);
+        bulk_g2s(dst + Smem::kRVc, cv.v_codes + ut * cv.vw, vc_b, rfull);
+        bulk_g2s(dst + Smem::kRVsz, cv.v_sz + ut * cv.vgroups, vsz_b, rfull);
+      }
+    }
+    __syncwarp();
+  }
+  // drain: the last copies issued have landed before shared memory is released
+  if (lane == 0)
+    for (int j = issued > STAGES ? issued - STAGES : 0; j < issued; ++j)
+      if (j != stalled) mbar_wait(p.rfull + 8u * (j % STAGES), (j / STAGES) & 1, a, abort_flag, true);
+}
+
 // ------------------------------------------------------------------ kernel
 
 template <int KB, int VB, bool SINK>
@@ -732,6 +915,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   // the unit's lengths live in shared memory from here on: read where used,
   // not held in registers through the role loops
   const UnitLen* uls = reinterpret_cast<const UnitLen*>(sm + Smem::kMisc + 16);
+  const Pipe pipe{sm, sm_base, Smem::kRing, Smem::kK0, Smem::kV0, bar(KFULL), bar(KEMPTY),
+                  bar(VFULL), bar(VEMPTY), bar(RFULL), bar(REMPTY)};
   if (threadIdx.x == 0) {
     *reinterpret_cast<UnitLen*>(sm + Smem::kMisc + 16) = ul;
     for (int b = 0; b < 2; ++b) {
@@ -990,163 +1175,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     }
   } else if (warp < 24) {
     regs_dec<kRegProducer>();
-    if (warp < 16) {
-    // ------------------------------------------------------------ K producer
-    const int c = (threadIdx.x - 256) & 127;   // channel
-    const int qh = (threadIdx.x - 256) >> 7;    // chunks 2qh, 2qh+1 of each tile
-    const KOffsets ko(c, qh, cv.GK, cv.kw, KB < 16 ? KB : 16);
-#pragma unroll 1
-    for (int j = 0; j < nt; ++j) {
-      const int b = j & 1, st = j % kStages;
-      if (!mbar_wait(bar(KEMPTY + b), ((j >> 1) & 1) ^ 1, a, abort_flag)) break;
-      if (!mbar_wait(bar(RFULL + st), (j / kStages) & 1, a, abort_flag)) break;
-      fill_k_tile<KB>(a, *uls, u, (t_begin + j) * TT, sm + (b ? Smem::kK1 : Smem::kK0),
-                      sm + Smem::kRing + st * Smem::kStageBytes, c, qh, ko);
-      fence_async_smem();
-      mbar_arrive(bar(KFULL + b));
-      mbar_arrive(bar(REMPTY + st));
-    }
-    } else {
-    // ------------------------------------------------------------ V producer
-    const int t = threadIdx.x - 512;
-    const VOffsets<KB> vo(t, cv.vw, cv.vgroups, cv.GV, VB < 16 ? VB : 16);
-#pragma unroll 1
-    for (int j = 0; j < nt; ++j) {
-      const int b = j & 1, st = j % kStages;
-      if (!mbar_wait(bar(VEMPTY + b), ((j >> 1) & 1) ^ 1, a, abort_flag)) break;
-      if (!mbar_wait(bar(RFULL + st), (j / kStages) & 1, a, abort_flag)) break;
-      fill_v_tile<KB, VB, SINK>(a, *uls, u, (t_begin + j) * TT, sm + (b ? Smem::kV1 : Smem::kV0),
-                      sm + Smem::kRing + st * Smem::kStageBytes, t, vo);
-      fence_async_smem();
-      mbar_arrive(bar(VFULL + b));
-      mbar_arrive(bar(REMPTY + st));
-    }
-    }
+    if (warp < 16)
+      k_producer_loop<KB, kStages>(a, uls, u, t_begin, nt, pipe, abort_flag, threadIdx.x - 256);
+    else
+      v_producer_loop<KB, VB, SINK, kStages>(a, uls, u, t_begin, nt, pipe, abort_flag,
+                                             threadIdx.x - 512);
   } else {
     regs_dec<kRegControl>();
     if (warp == kLoadWarp) {
-    // ------------------------------------------------------------ loader
-    // lanes prefetch the side-table group index of 32 tiles at a time; lane 0
-    // issues the bulk copies of each tile.  Token positions fit in 32 bits
-    // (capacity <= 2^30) and K groups are 32, 64 or 128 tokens, so the group
-    // arithmetic is 32-bit shifts.
-    const int gks = KB < 16 ? __ffs(cv.GK) - 1 : 0;
-    const int Lq = uls->Lq, Lc = uls->L, t0 = int(t_begin) * TT;
-    const int32_t* gs = cv.prot_gstart + size_t(u) * size_t(cv.nG + 1);
-    int issued = 0;     // tiles 0 .. issued-1 went through the ring
-    int stalled = -1;   // (bounds-checking build) the tile whose copies were withheld
-    int pf0 = 0, pf1 = 0;  // this lane's prefetched gstart values (tile j0 + lane)
-#pragma unroll 1
-    for (int j = 0; j < nt; ++j) {
-      if constexpr (KB < 16) {
-        if ((j & 31) == 0) {
-          pf0 = pf1 = 0;
-          const int jj = j + lane;
-          const int ts = t0 + jj * TT;
-          if (jj < nt && ts < Lq && cv.P > 0) {
-            const int q_end = ts + TT < Lq ? ts + TT : Lq;
-            pf0 = __ldg(gs + (ts >> gks));
-            pf1 = __ldg(gs + (q_end >> gks));
-          }
-        }
-      }
-      const int g0 = __shfl_sync(0xffffffffu, pf0, j & 31);
-      const int g1 = __shfl_sync(0xffffffffu, pf1, j & 31);
-      const int st = j % kStages;
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(REMPTY + st), ((j / kStages) & 1) ^ 1,
-                                             a, abort_flag)))
-        break;
-      ++issued;
-#ifdef DKV_BOUNDS_CHECK
-      if (j == a.test_stall_tile) {
-        // test hook: nothing is copied and nothing arrives on this stage, so
-        // the producers' bounded waits on it run out (DKV_FLAG_TIMEOUT)
-        stalled = j;
-        continue;
-      }
-#endif
-      if (lane == 0) {
-        const int ts = t0 + j * TT;
-        const uint32_t dst = sm_base + Smem::kRing + st * Smem::kStageBytes;
-        uint32_t kc_b = 0, ksz_b = 0, vc_b = 0, vsz_b = 0, pos_b = 0, pk_b = 0;
-        int g_lo = 0, pidx0 = 0;  // pidx0: first staged position, relative to the unit
-        const int n = g1 - g0;
-        if (KB < 16 && ts < Lq) {
-          g_lo = ts >> gks;
-          const int q_end = ts + TT < Lq ? ts + TT : Lq;  // multiple of GK
-          const uint32_t ng = uint32_t((q_end >> gks) - g_lo);
-          kc_b = ng * kHeadDim * uint32_t(cv.kw) * 4u;
-          ksz_b = ng * kHeadDim * 4u;
-          if (n > 0) {
-            const int nst = n < kStagedProt ? n : kStagedProt;
-            // 16-byte aligned superset of the staged positions (the unit's
-            // slice starts at u * P entries)
-            const int64_t e0 = int64_t(u) * cv.P + g0;
-            const int64_t ea = e0 & ~int64_t(3);
-            pidx0 = int(ea - int64_t(u) * cv.P);
-            pos_b = uint32_t(((e0 + nst + 3) & ~int64_t(3)) - ea) * 4u;
-            pk_b = uint32_t(nst) * kHeadDim * 2u;
-          }
-        }
-        if (VB < 16 && ts < Lc) {
-          const uint32_t nv = uint32_t((ts + TT < Lc ? ts + TT : Lc) - ts);
-          vc_b = nv * uint32_t(cv.vw) * 4u;
-          vsz_b = nv * uint32_t(cv.vgroups) * 4u;
-        }
-        const size_t ug = size_t(u) * size_t(cv.nG) + size_t(g_lo);
-        {
-          // bounds-checking build: each copy inside its buffer and its ring
-          // slot, else left out (the staged side table with it); the byte
-          // counts stay consistent with the expect_tx below
-          const size_t U = size_t(cv.U), P = size_t(cv.P), e = size_t(u) * P;
-          if (kc_b && !DKV_IN_BOUNDS(
-                          kc_b <= Smem::kRKsz - Smem::kRKc && ksz_b <= Smem::kRVc - Smem::kRKsz &&
-                          (ug * kHeadDim * cv.kw) * 4 + kc_b <= U * cv.nG * kHeadDim * cv.kw * 4 &&
-                          (ug * kHeadDim) * 4 + ksz_b <= U * cv.nG * kHeadDim * 4, cv.status))
-            kc_b = ksz_b = pos_b = pk_b = 0;
-          // (the staged positions are a 16-byte aligned superset: up to three
-          // entries before and after the unit's slice, inside the arena)
-          if (pos_b && !DKV_IN_BOUNDS(
-                           g0 >= 0 && int64_t(e) + pidx0 >= 0 &&
-                           pos_b <= Smem::kRPk - Smem::kRPos &&
-                           pk_b <= Smem::kStageBytes - Smem::kRPk &&
-                           (e + size_t(pidx0)) * 4 + pos_b <= (U * P + 3) * 4 &&
-                           (e + size_t(g0)) * kHeadDim * 2 + pk_b <= U * P * kHeadDim * 2, cv.status))
-            pos_b = pk_b = 0;
-          const size_t ut = size_t(u) * size_t(cv.cap) + size_t(ts);
-          if (vc_b && !DKV_IN_BOUNDS(
-                          vc_b <= Smem::kRVsz - Smem::kRVc && vsz_b <= Smem::kRHdr - Smem::kRVsz &&
-                          ut * cv.vw * 4 + vc_b <= U * size_t(cv.cap) * cv.vw * 4 &&
-                          ut * cv.vgroups * 4 + vsz_b <= U * size_t(cv.cap) * cv.vgroups * 4, cv.status))
-            vc_b = vsz_b = 0;
-        }
-        int* hdr = reinterpret_cast<int*>(sm + Smem::kRing + st * Smem::kStageBytes + Smem::kRHdr);
-        hdr[0] = pos_b ? n : 0;  // pos_b is set exactly when the tile has protected rows
-        hdr[1] = g0;
-        hdr[2] = pidx0;
-        mbar_arrive_expect_tx(bar(RFULL + st), kc_b + ksz_b + vc_b + vsz_b + pos_b + pk_b);
-        if (kc_b) {
-          bulk_g2s(dst + Smem::kRKc, cv.k_codes + ug * kHeadDim * cv.kw, kc_b, bar(RFULL + st));
-          bulk_g2s(dst + Smem::kRKsz, cv.k_sz + ug * kHeadDim, ksz_b, bar(RFULL + st));
-        }
-        if (pos_b) {
-          const size_t e = size_t(u) * size_t(cv.P);
-          bulk_g2s(dst + Smem::kRPos, cv.prot_pos + e + size_t(pidx0), pos_b, bar(RFULL + st));
-          bulk_g2s(dst + Smem::kRPk, cv.prot_k + (e + size_t(g0)) * kHeadDim, pk_b,
-                   bar(RFULL + st));
-        }
-        if (vc_b) {
-          const size_t ut = size_t(u) * size_t(cv.cap) + size_t(ts);
-          bulk_g2s(dst + Smem::kRVc, cv.v_codes + ut * cv.vw, vc_b, bar(RFULL + st));
-          bulk_g2s(dst + Smem::kRVsz, cv.v_sz + ut * cv.vgroups, vsz_b, bar(RFULL + st));
-        }
-      }
-      __syncwarp();
-    }
-    // drain: the last copies issued have landed before shared memory is released
-    if (lane == 0)
-      for (int j = issued > kStages ? issued - kStages : 0; j < issued; ++j)
-        if (j != stalled) mbar_wait(bar(RFULL + j % kStages), (j / kStages) & 1, a, abort_flag, true);
+      loader_loop<KB, VB, kStages>(a, uls, u, t_begin, nt, pipe, abort_flag, lane);
     } else if (warp == kMmaWarp && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
     bool ok = mbar_wait(bar(QREADY), 0, a, abort_flag);
@@ -1213,8 +1250,457 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   }
 }
 
+
+// ------------------------------------------------------------ tokens on lanes
+
+// Query groups of 32 rows (one query head per kv-head and 32-token blocks).
+// The scores are computed transposed, S^T = K_hat Q^T, so the 128 tokens of
+// a tile sit on the 128 TMEM lanes and all four warps of the softmax
+// warpgroup work (thread = token, 32 scores per thread), and O^T = V_hat^T P^T
+// accumulates with the channels on the lanes.  Both MMAs are M = 128, N = 64
+// (the 32 query rows zero-padded; every operand MN-major, 128-byte swizzle):
+//   S^T[token][row] += K_hat tile (A: tokens x channels, as dequantized) *
+//                      Q^T (B: channels x rows, staged once)
+//   O^T[chan][row]  += V_hat^T (A: channels x tokens, the V tile as
+//                      dequantized) * P^T (B: tokens x rows, written by the
+//                      softmax threads)
+// The producers, the loader and the ring are the row-block kernel's.  Each
+// row keeps a reference max in registers (the same in every thread), raised
+// only when a tile's score exceeds it by more than 8 (log2 units), as in the
+// row-block kernel; raising takes a 128-thread reduction and rescales O and
+// the per-thread partial row sums.  Per-thread partial row sums (one per
+// row) are reduced once at the end.
+// Warps: 0-3 softmax, 4-11 K producers, 12-19 V producers, 21 TMEM and MMA
+// lane, 22 loader (20, 23 idle); one CTA per SM.
+namespace tl {
+constexpr int kWarps = 24;
+constexpr int kThreads = kWarps * 32;
+constexpr int kRows = 32;  // query rows per unit
+constexpr int kN = 64;     // MMA N (rows padded)
+constexpr int kMmaWarp = 21, kLoadWarp = 22;
+constexpr int kStages = 2;
+constexpr uint32_t kColS0 = 0, kColS1 = 64, kColO = 128, kTmemCols = 256;
+// D f32, A and B f16, both MN-major, M = 128, N = 64
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 15) | (1u << 16) | ((uint32_t(kN) >> 3) << 17) |
+                            ((128u >> 4) << 24);
+// launch: 80 registers x 768 threads = 61440; softmax 152 x 128, producers
+// 64 x 512, control 56 x 128 = 59392
+constexpr int kRegSoftmax = 152, kRegProducer = 64, kRegControl = 56;
+
+struct Smem {
+  static constexpr uint32_t kK0 = 0, kV0 = 2 * kTileBytes;
+  static constexpr uint32_t kP = 4 * kTileBytes;                   // P^T tile [128 tokens][64 rows]
+  static constexpr uint32_t kQ = kP + 128 * kN * 2;                // Q^T [128 channels][64 rows]
+  static constexpr uint32_t kRing = kQ + 128 * kN * 2;
+  static constexpr uint32_t kBar = kRing + kStages * ::dkv::Smem::kStageBytes;  // 32 mbarriers
+  static constexpr uint32_t kFlag = kBar + 32 * 8;                 // [2][4] raise votes
+  static constexpr uint32_t kRed = kFlag + 64;                     // [3][4 warps][32 rows] floats
+  static constexpr uint32_t kMisc = kRed + 3 * 4 * kRows * 4;      // tmem, abort, lengths
+  static constexpr uint32_t kBytes = kMisc + 32;
+};
+// (VOTE, RED, EPI: the softmax threads' exchanges, bounded waits like every
+// other hand-off, so a CTA that aborts cannot leave a thread waiting)
+enum Bar {
+  KFULL = 0, KEMPTY = 2, VFULL = 4, VEMPTY = 6, SFULL = 8, SFREE = 10, PFULL = 12, QREADY = 13,
+  DONE = 14, VOTE = 15, RED = 16, EPI = 17, RFULL = 18, REMPTY = RFULL + kStages
+};
+
+// the 16-byte chunk of rows 8k..8k+7 of token / channel t in a [128][64]
+// MN-major tile (one 64-element atom per 8 tokens: atom t/8 at (t/8) * 1024)
+__device__ __forceinline__ uint32_t nt_off(int t, int k) {
+  return uint32_t((t >> 3) * 1024 + (t & 7) * 128 + ((k ^ (t & 7)) << 4));
+}
+
+// max over the 32 lanes of every one of the 32 values v[i], the result for
+// i = lane returned (a butterfly that halves the values held at each step)
+__device__ __forceinline__ float transpose_max(float (&v)[32], int lane) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < o; ++i) {
+      // keep rows i (lane bit clear) or i + o (set); send the other
+      const float send = up ? v[i] : v[i + o];
+      const float keep = up ? v[i + o] : v[i];
+      v[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, o));
+    }
+  }
+  return v[0];  // row = lane
+}
+__device__ __forceinline__ float transpose_sum(float (&v)[32], int lane) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < o; ++i) {
+      const float send = up ? v[i] : v[i + o];
+      const float keep = up ? v[i + o] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+  return v[0];
+}
+
+// channel of O^T's lane p: the V tile holds its channels in kpos<VB> order
+template <int VB>
+__device__ __forceinline__ int kpos_inv(int p) {
+  for (int t = p & ~15; t < (p & ~15) + 16; ++t)
+    if (kpos<VB>(t) == p) return t;
+  return p;
+}
+}  // namespace tl
+
+template <int KB, int VB, bool SINK>
+__global__ void __launch_bounds__(tl::kThreads, 1) attn_tl_kernel(const __grid_constant__ AttnArgs a) {
+  using S = tl::Smem;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~uintptr_t(1023));
+  const uint32_t sm_base = smem_u32(sm);
+  const uint32_t bar0 = sm_base + S::kBar;
+  auto bar = [&](int i) { return bar0 + 8u * uint32_t(i); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + S::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + S::kMisc + 4);
+
+  const CacheView& cv = a.c;
+  const int u = blockIdx.x / a.nsplit;
+  const int sp = blockIdx.x % a.nsplit;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const UnitLen ul = unit_len(a, u);
+  const int64_t n_tiles = (ul.n_tok + TT - 1) / TT;
+  const int64_t t_begin = int64_t(sp) * a.tiles_per_split;
+  const int64_t t_end = t_begin + a.tiles_per_split < n_tiles ? t_begin + a.tiles_per_split : n_tiles;
+  const int nt = t_end > t_begin ? int(t_end - t_begin) : 0;
+  if (nt == 0) {
+    // a split past the end of a shorter sequence: an empty partial
+    pdl_wait();
+    pdl_trigger();
+    if (!a.final_out) {
+      const size_t prow = (size_t(u) * a.part_stride + a.part_base + sp) * tl::kRows;
+      for (int i = threadIdx.x; i < tl::kRows * (kHeadDim / 4); i += tl::kThreads)
+        reinterpret_cast<float4*>(a.part_o + prow * kHeadDim)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int i = threadIdx.x; i < tl::kRows; i += tl::kThreads)
+        a.part_ml[prow + i] = make_float2(-__int_as_float(0x7f800000), 0.f);
+    }
+    return;
+  }
+  const UnitLen* uls = reinterpret_cast<const UnitLen*>(sm + S::kMisc + 16);
+  const Pipe pipe{sm, sm_base, S::kRing, S::kK0, S::kV0, bar(tl::KFULL), bar(tl::KEMPTY),
+                  bar(tl::VFULL), bar(tl::VEMPTY), bar(tl::RFULL), bar(tl::REMPTY)};
+  if (threadIdx.x == 0) {
+    *reinterpret_cast<UnitLen*>(sm + S::kMisc + 16) = ul;
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(tl::KFULL + b), 256);
+      mbar_init(bar(tl::KEMPTY + b), 1);
+      mbar_init(bar(tl::VFULL + b), 256);
+      mbar_init(bar(tl::VEMPTY + b), 1);
+      mbar_init(bar(tl::SFULL + b), 1);
+      mbar_init(bar(tl::SFREE + b), 128);
+    }
+    mbar_init(bar(tl::PFULL), 128);
+    mbar_init(bar(tl::QREADY), 128);
+    mbar_init(bar(tl::DONE), 1);
+    mbar_init(bar(tl::VOTE), 128);
+    mbar_init(bar(tl::RED), 128);
+    mbar_init(bar(tl::EPI), 128);
+    for (int st = 0; st < tl::kStages; ++st) {
+      mbar_init(bar(tl::RFULL + st), 1);
+      mbar_init(bar(tl::REMPTY + st), 512);
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == tl::kMmaWarp) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(tl::kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  pdl_wait();  // no global memory access above this line
+  pdl_trigger();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp < 4) {
+    // ------------------------------------------------------------ softmax
+    regs_inc<tl::kRegSoftmax>();
+    const int l = threadIdx.x;  // TMEM lane: token of a tile, then channel of O^T
+    const uint32_t lane_base = tmem + (uint32_t(warp * 32) << 16);
+    float* red = reinterpret_cast<float*>(sm + S::kRed);     // [3][4][32]
+    int* flag = reinterpret_cast<int*>(sm + S::kFlag);         // [2][4]
+    const bool qneg = a.scale_log2 < 0.f;
+    const float sc = fmaxf(fabsf(a.scale_log2), 1e-30f);
+    {
+      // Q^T into shared memory: thread = channel l, its 32 rows (bf16 ->
+      // fp16, the sign of a negative scale folded in); rows 32..63 zero.  The
+      // P^T tile's rows 32..63 (never written again) are zeroed too.
+      uint32_t q2[16];
+      const uint16_t* qc = a.q + size_t(u) * tl::kRows * kHeadDim + l;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float lo = __uint_as_float(uint32_t(__ldg(qc + size_t(2 * i) * kHeadDim)) << 16);
+        const float hi = __uint_as_float(uint32_t(__ldg(qc + size_t(2 * i + 1) * kHeadDim)) << 16);
+        q2[i] = pack_h2(qneg ? -lo : lo, qneg ? -hi : hi);
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        *reinterpret_cast<uint4*>(sm + S::kQ + tl::nt_off(l, k)) =
+            make_uint4(q2[4 * k], q2[4 * k + 1], q2[4 * k + 2], q2[4 * k + 3]);
+#pragma unroll
+      for (int k = 4; k < 8; ++k) {
+        *reinterpret_cast<uint4*>(sm + S::kQ + tl::nt_off(l, k)) = make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(sm + S::kP + tl::nt_off(l, k)) = make_uint4(0u, 0u, 0u, 0u);
+      }
+      fence_async_smem();
+      mbar_arrive(bar(tl::QREADY));
+    }
+    float ref[tl::kRows];    // reference max per row (log2 units), the same in every thread
+    float lsum[tl::kRows];   // this thread's (token's) share of each row sum, relative to ref
+#pragma unroll
+    for (int i = 0; i < tl::kRows; ++i) {
+      ref[i] = -__int_as_float(0x7f800000);
+      lsum[i] = 0.f;
+    }
+    bool ok = true;
+    int n_raise = 0;  // phases of the tl::RED barrier used so far
+#pragma unroll 1
+    for (int j = 0; j < nt && ok; ++j) {
+      const int b = j & 1;
+      // tcgen05.ld is warp-collective: every branch around it is warp-uniform
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(tl::SFULL + b), (j >> 1) & 1, a, abort_flag))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t s_col = lane_base + (b ? tl::kColS1 : tl::kColS0);
+      float x[tl::kRows];
+      auto load_scores = [&]() {
+        uint32_t sv[32];
+        tmem_ld32(s_col, sv);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < tl::kRows; ++i) x[i] = __uint_as_float(sv[i]) * sc;
+      };
+      load_scores();
+      const int64_t tile_start = (t_begin + j) * TT;
+      const int n_tok = uls->n_tok;
+      const bool valid = tile_start + l < n_tok;  // (past-the-end tokens have zero K and V)
+      // raise the reference where a score exceeds it by more than 8
+      bool raise = false;
+      if (valid)
+#pragma unroll
+        for (int i = 0; i < tl::kRows; ++i) raise |= x[i] > ref[i] + 8.f;
+      raise = __any_sync(0xffffffffu, raise);
+      if (lane == 0) flag[b * 4 + warp] = raise;
+      mbar_arrive(bar(tl::VOTE));
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(tl::VOTE), j & 1, a, abort_flag))) {
+        ok = false;
+        break;
+      }
+      raise = flag[b * 4] | flag[b * 4 + 1] | flag[b * 4 + 2] | flag[b * 4 + 3];
+      if (raise) {
+        // tile max of every row over the 128 tokens (the reduction takes x
+        // apart; the scores are read again from tensor memory after it)
+        if (!valid)
+#pragma unroll
+          for (int i = 0; i < tl::kRows; ++i) x[i] = -__int_as_float(0x7f800000);
+        red[(b * 4 + warp) * tl::kRows + lane] = tl::transpose_max(x, lane);
+        mbar_arrive(bar(tl::RED));
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(tl::RED), n_raise & 1, a, abort_flag))) {
+          ok = false;
+          break;
+        }
+        ++n_raise;
+        float alpha[tl::kRows];
+#pragma unroll
+        for (int i = 0; i < tl::kRows; ++i) {
+          const float* rr = red + b * 4 * tl::kRows + i;
+          const float tm = fmaxf(fmaxf(rr[0], rr[tl::kRows]), fmaxf(rr[2 * tl::kRows], rr[3 * tl::kRows]));
+          const float nr = tm > ref[i] + 8.f ? fmaxf(ref[i], tm) : ref[i];
+          alpha[i] = fast_exp2(ref[i] - nr);  // 1 when unchanged, 0 from -inf
+          ref[i] = nr;
+          lsum[i] *= alpha[i];
+        }
+        if (j > 0) {
+          // O^T holds PV up to tile j-1 relative to the old references: scale
+          // its row columns once that PV has completed
+          if (!__all_sync(0xffffffffu, mbar_wait(bar(tl::VEMPTY + ((j - 1) & 1)), ((j - 1) >> 1) & 1, a,
+                                                 abort_flag))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            uint32_t o[16];
+            tmem_ld16(lane_base + tl::kColO + 16 * h, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha[16 * h + i]);
+            tmem_st16(lane_base + tl::kColO + 16 * h, o);
+          }
+          tmem_st_wait();
+        }
+        load_scores();
+      }
+      // P = 2^(x - ref) (0 past the end), fp16 pairs; row sums in fp32
+      uint32_t pk[tl::kRows / 2];
+#pragma unroll
+      for (int i = 0; i < tl::kRows; i += 2) {
+        const float p0 = valid ? fast_exp2(x[i] - ref[i]) : 0.f;
+        const float p1 = valid ? fast_exp2(x[i + 1] - ref[i + 1]) : 0.f;
+        lsum[i] += p0;
+        lsum[i + 1] += p1;
+        pk[i / 2] = pack_h2(p0, p1);
+      }
+      // the P^T tile is free once PV(j-1) has completed
+      if (j > 0 && !__all_sync(0xffffffffu, mbar_wait(bar(tl::VEMPTY + ((j - 1) & 1)),
+                                                      ((j - 1) >> 1) & 1, a, abort_flag))) {
+        ok = false;
+        break;
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        *reinterpret_cast<uint4*>(sm + S::kP + tl::nt_off(l, k)) =
+            make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar(tl::PFULL));
+      mbar_arrive(bar(tl::SFREE + b));  // (S_b was last read above)
+    }
+    // epilogue: row sums over the 128 tokens, then O^T / l per row
+    if (ok) {
+      const int jl = nt - 1;
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait(bar(tl::VEMPTY + (jl & 1)), (jl >> 1) & 1, a, abort_flag));
+    }
+    if (ok) {
+      float* rs = red + 2 * 4 * tl::kRows;  // (the raise path's halves stay untouched)
+      rs[warp * tl::kRows + lane] = tl::transpose_sum(lsum, lane);
+      mbar_arrive(bar(tl::EPI));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(tl::EPI), 0, a, abort_flag));
+    }
+    if (ok) {
+      const float* rs = red + 2 * 4 * tl::kRows;
+      tc_fence_after();
+      uint32_t o[32];
+      tmem_ld32(lane_base + tl::kColO, o);
+      tmem_ld_wait();
+      const int ch = tl::kpos_inv<VB>(l);  // O^T lane l holds channel kpos^-1(l)
+#pragma unroll
+      for (int i = 0; i < tl::kRows; ++i) {
+        const float lt = (rs[i] + rs[tl::kRows + i]) + (rs[2 * tl::kRows + i] + rs[3 * tl::kRows + i]);
+        const float ov = __uint_as_float(o[i]);
+        if (a.final_out) {
+          const __nv_bfloat16 v = __float2bfloat16_rn(ov / lt);
+          a.out[(size_t(u) * tl::kRows + i) * kHeadDim + ch] = *reinterpret_cast<const uint16_t*>(&v);
+        } else {
+          const size_t prow = (size_t(u) * a.part_stride + a.part_base + sp) * tl::kRows + i;
+          a.part_o[prow * kHeadDim + ch] = ov;
+          if (l == 0) a.part_ml[prow] = make_float2(ref[i], lt);
+        }
+      }
+    }
+  } else if (warp < 20) {
+    regs_dec<tl::kRegProducer>();
+    if (warp < 12)
+      k_producer_loop<KB, tl::kStages>(a, uls, u, t_begin, nt, pipe, abort_flag, threadIdx.x - 128);
+    else
+      v_producer_loop<KB, VB, SINK, tl::kStages>(a, uls, u, t_begin, nt, pipe, abort_flag,
+                                             threadIdx.x - 384);
+  } else {
+    regs_dec<tl::kRegControl>();
+    if (warp == tl::kLoadWarp) {
+      loader_loop<KB, VB, tl::kStages>(a, uls, u, t_begin, nt, pipe, abort_flag, lane);
+    } else if (warp == tl::kMmaWarp && lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
+      // QK(j) needs K_j and S_(j mod 2) read (tl::SFREE of tile j-2); PV(j) needs
+      // P_j (tl::PFULL, phase j) and V_j.  QK runs up to one tile ahead of PV.
+      bool ok = mbar_wait(bar(tl::QREADY), 0, a, abort_flag);
+      tc_fence_after();
+      const uint32_t qbase = sm_base + S::kQ, pbase = sm_base + S::kP;
+      int nq = 0, np = 0;
+      auto issue_qk = [&]() {
+        tc_fence_after();
+        const int b = nq & 1;
+        const uint32_t kbase = sm_base + S::kK0 + b * kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)  // channels 16kk .. 16kk + 15
+          asm volatile(
+              "{\n\t.reg .pred p;\n\t"
+              "setp.ne.b32 p, %4, 0;\n\t"
+              "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(
+                  tmem + (b ? tl::kColS1 : tl::kColS0)),
+              "l"(sdesc_sw128(kbase + 4096 * kk, 1024, 2048)), "l"(sdesc_sw128(qbase + 2048 * kk, 8192, 1024)),
+              "r"(tl::kIdesc), "r"(kk > 0 ? 1u : 0u)
+              : "memory");
+        mma_commit(bar(tl::KEMPTY + b));
+        mma_commit(bar(tl::SFULL + b));
+        ++nq;
+      };
+#pragma unroll 1
+      while (ok && np < nt) {
+        // issue every QK that is ready and allowed (at most one ahead of PV)
+        while (nq < nt && nq <= np + 1 && mbar_test(bar(tl::KFULL + (nq & 1)), (nq >> 1) & 1) &&
+               (nq < 2 || mbar_test(bar(tl::SFREE + (nq & 1)), ((nq - 2) >> 1) & 1)))
+          issue_qk();
+        if (np == nq) {
+          ok = mbar_wait(bar(tl::KFULL + (nq & 1)), (nq >> 1) & 1, a, abort_flag) &&
+               (nq < 2 || mbar_wait(bar(tl::SFREE + (nq & 1)), ((nq - 2) >> 1) & 1, a, abort_flag));
+          if (ok) issue_qk();
+          continue;
+        }
+        const int bb = np & 1;
+        if (!mbar_wait(bar(tl::PFULL), np & 1, a, abort_flag) ||
+            !mbar_wait(bar(tl::VFULL + bb), (np >> 1) & 1, a, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t vbase = sm_base + S::kV0 + bb * kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)  // tokens 16kk .. 16kk + 15
+          asm volatile(
+              "{\n\t.reg .pred p;\n\t"
+              "setp.ne.b32 p, %4, 0;\n\t"
+              "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem + tl::kColO),
+              "l"(sdesc_sw128(vbase + 4096 * kk, 1024, 2048)), "l"(sdesc_sw128(pbase + 2048 * kk, 8192, 1024)),
+              "r"(tl::kIdesc), "r"((np > 0 || kk > 0) ? 1u : 0u)
+              : "memory");
+        mma_commit(bar(tl::VEMPTY + bb));
+        ++np;
+      }
+      // drain: every MMA issued above completes before TMEM is released
+      mma_commit(bar(tl::DONE));
+      mbar_wait(bar(tl::DONE), 0, a, abort_flag, /*drain=*/true);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == tl::kMmaWarp) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(tl::kTmemCols));
+  }
+}
+
+template <int KB, int VB, bool SINK>
+cudaError_t launch_tl(const AttnArgs& a, cudaStream_t s) {
+  const size_t smem = tl::Smem::kBytes + 1024;
+  cudaError_t e = cudaFuncSetAttribute(attn_tl_kernel<KB, VB, SINK>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e != cudaSuccess) return e;
+  e = launch_pdl(attn_tl_kernel<KB, VB, SINK>, dim3(unsigned(a.c.U) * unsigned(a.nsplit)),
+                 dim3(tl::kThreads), smem, s, a);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
 template <int KB, int VB, bool SINK>
 cudaError_t launch_kvs(const AttnArgs& a, cudaStream_t s) {
+  if (a.tc_layout == 1) return launch_tl<KB, VB, SINK>(a, s);
   const size_t smem = Smem::kBytes + 1024;
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<KB, VB, SINK>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));

@@ -200,15 +200,18 @@ int plan_attention(const CacheInfo& ci, AttnArgs* a, int* kernel_out, const char
     *err = "no tokens to attend to";
     return DKV_ERR_INVALID_ARG;
   }
+  // kernel 2: tcgen05, tokens on TMEM lanes for 32-row query groups, query-row
+  // blocks otherwise; 3: tcgen05 with query-row blocks for every group
   int kernel = ci.opt_kernel;
   if (kernel == 0) kernel = tc_supported(v) ? 2 : 1;
-  if (kernel == 2 && !tc_supported(v)) {
+  if (kernel >= 2 && !tc_supported(v)) {
     *err = "no tcgen05 attention variant for this shape";
     return DKV_ERR_UNSUPPORTED;
   }
-  const int tile = kernel == 2 ? kTcTile : kMmaTile;
+  a->tc_layout = (kernel == 2 && v.rows == 32) ? 1 : 0;
+  const int tile = kernel >= 2 ? kTcTile : kMmaTile;
   const int64_t n_tiles = ceil_div(a->n_tok, tile);
-  const int64_t nrb = kernel == 2 ? (v.rows + 127) / 128 : 1;
+  const int64_t nrb = kernel >= 2 ? (v.rows + 127) / 128 : 1;
   const int64_t cap = std::max<int64_t>(1, std::min<int64_t>(n_tiles, ci.max_splits));
   int64_t ns;
   if (ci.opt_splits > 0) {
@@ -544,7 +547,7 @@ int dkv_block_attention(dkv_cache* c, const void* q, const void* k_act, const vo
     ++launches;
   }
   cudaError_t e = timed_launch(c, DKV_KERNEL_ATTENTION, s, [&] {
-    return kernel == 2 ? dkv::launch_attention_tc(a, s) : dkv::launch_attention_mma(a, s);
+    return kernel >= 2 ? dkv::launch_attention_tc(a, s) : dkv::launch_attention_mma(a, s);
   });
   if (e != cudaSuccess) return fail(DKV_ERR_CUDA, std::string("attention launch: ") + cudaGetErrorString(e));
   if (!a.final_out) {
@@ -617,11 +620,11 @@ int dkv_block_attention_dual(dkv_cache* c, dkv_cache* sfx, const void* q, const 
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = timed_launch(c, DKV_KERNEL_ATTENTION, s, [&] {
-    return k1 == 2 ? dkv::launch_attention_tc(a1, s) : dkv::launch_attention_mma(a1, s);
+    return k1 >= 2 ? dkv::launch_attention_tc(a1, s) : dkv::launch_attention_mma(a1, s);
   });
   if (e != cudaSuccess) return fail(DKV_ERR_CUDA, std::string("attention launch: ") + cudaGetErrorString(e));
   e = timed_launch(c, DKV_KERNEL_ATTENTION, s, [&] {
-    return k2 == 2 ? dkv::launch_attention_tc(a2, s) : dkv::launch_attention_mma(a2, s);
+    return k2 >= 2 ? dkv::launch_attention_tc(a2, s) : dkv::launch_attention_mma(a2, s);
   });
   if (e != cudaSuccess) return fail(DKV_ERR_CUDA, std::string("suffix attention launch: ") + cudaGetErrorString(e));
   dkv::AttnArgs ac = a1;
@@ -681,7 +684,7 @@ int dkv_block_attention_selected(dkv_cache* c, const void* q, const void* k_act,
   a.final_out = 0;  // the first pass keeps every row's (max, sum) in the split partials
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = timed_launch(c, DKV_KERNEL_ATTENTION, s, [&] {
-    return kernel == 2 ? dkv::launch_attention_tc(a, s) : dkv::launch_attention_mma(a, s);
+    return kernel >= 2 ? dkv::launch_attention_tc(a, s) : dkv::launch_attention_mma(a, s);
   });
   if (e != cudaSuccess) return fail(DKV_ERR_CUDA, std::string("attention launch: ") + cudaGetErrorString(e));
   // contributions of the committed tokens, then the selection
@@ -871,8 +874,8 @@ int dkv_cache_set_option(dkv_cache* c, int32_t key, int64_t value) {
       c->opt_splits = int32_t(value);
       return DKV_OK;
     case DKV_OPT_ATTN_KERNEL:
-      if (value < 0 || value > 2) return fail(DKV_ERR_INVALID_ARG, "kernel must be 0, 1 or 2");
-      if (value == 2 && !dkv::tc_supported(c->v))
+      if (value < 0 || value > 3) return fail(DKV_ERR_INVALID_ARG, "kernel must be 0, 1, 2 or 3");
+      if (value >= 2 && !dkv::tc_supported(c->v))
         return fail(DKV_ERR_UNSUPPORTED, "no tcgen05 attention variant for this shape");
       c->opt_kernel = int32_t(value);
       return DKV_OK;

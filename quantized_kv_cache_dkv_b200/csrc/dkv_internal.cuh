@@ -135,6 +135,7 @@ struct AttnArgs {
   int32_t sel_ld;
   int32_t budget;
   int32_t gather;
+  int32_t tc_layout;        // tcgen05 kernel: 0 query-row blocks, 1 tokens on lanes (32 rows)
   uint64_t wait_limit_ns;   // limit of one bounded wait in the tcgen05 kernel
   int32_t test_stall_tile;  // bounds-checking build: tile whose copies the
                             // tcgen05 loader withholds (-1: none)

@@ -26,11 +26,17 @@ from gpu_util import (assert_close, commit_both, default_P, default_cap, dev_bf1
 
 
 def main():
-    import torch
     import quantized_kv_cache_dkv_b200 as dkv
     print("library:", os.path.basename(dkv.LIB_PATH), flush=True)
-    # 128-row query groups (4 query heads x 32-token blocks): the tcgen05 kernel
-    w = synth.WORKLOADS["tiny"].with_(B=2, Hq=8, Hkv=2, L=1024, prot_frac=0.02)
+    # 128-row query groups (4 query heads x 32-token blocks): the row-block
+    # kernel; 32-row groups (one query head per kv-head): tokens on lanes
+    check(dkv, synth.WORKLOADS["tiny"].with_(B=2, Hq=8, Hkv=2, L=1024, prot_frac=0.02))
+    check(dkv, synth.WORKLOADS["tiny"].with_(B=2, Hq=2, Hkv=2, L=1024, prot_frac=0.02))
+    print("OK timeout path", flush=True)
+
+
+def check(dkv, w):
+    import torch
     n_blocks = w.L // w.blk
     cap = default_cap(w, n_blocks + 1)
     P = default_P(w, cap)
@@ -83,7 +89,6 @@ def main():
     assert dkv.dkv_cache_status(cache2) == 0
     dkv.dkv_cache_free(cache2)
     dkv.dkv_cache_free(cache)
-    print("OK timeout path", flush=True)
 
 
 if __name__ == "__main__":
