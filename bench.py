@@ -216,7 +216,7 @@ def io_bytes(w: synth.Workload) -> float:
 
 
 def run_gpu(w: synth.Workload, K: int, W: int, want_e2e=True, log=print, kernel=0,
-            v_rotation=0, suffix=0, time_build=False):
+            v_rotation=0, suffix=0, time_build=False, select_budget=0):
     import torch
     import quantized_kv_cache_dkv_b200 as dkv
 
@@ -306,7 +306,10 @@ def run_gpu(w: synth.Workload, K: int, W: int, want_e2e=True, log=print, kernel=
         kept.clear()
 
     def attend(r, q, ka, va, out):
-        if sfx:
+        if select_budget:
+            dkv.dkv_block_attention_selected(caches[r], q, ka, va, w.softmax_scale,
+                                             select_budget, out)
+        elif sfx:
             dkv.dkv_block_attention_dual(caches[r], sfx[r], q, ka, va, w.softmax_scale, out)
         else:
             dkv.dkv_block_attention(caches[r], q, ka, va, w.softmax_scale, out)
@@ -413,6 +416,10 @@ def run_gpu(w: synth.Workload, K: int, W: int, want_e2e=True, log=print, kernel=
         dkv.dkv_cache_set_option(c, dkv.DKV_OPT_PROFILE, 0)
     Lp = step_lengths(w, Kp, R)
     att_ms, att_n = prof["attention"]
+    if select_budget:
+        # one selection call = four kernels timed as attention (statistics,
+        # scores, top-k, attention over the kept tokens): per-call figures
+        att_n = att_n // 4
     # The timed region is a CUDA-graph replay whose kernels overlap their
     # launch with the previous kernel (programmatic dependent launch), so the
     # eager per-launch times above do not add up to its step time.  Each
@@ -739,6 +746,9 @@ def main():
                     help="K-RPBH rotation of V with this Hadamard block (0 = none)")
     ap.add_argument("--suffix", type=int, default=0,
                     help="dual cache: tokens in a second (suffix) cache attended with the prefix")
+    ap.add_argument("--select-budget", type=int, default=0,
+                    help="Q-MaskAhead selection: each step attends to this many committed tokens "
+                         "per (sequence, kv-head), chosen by contribution score, plus the block")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -779,12 +789,18 @@ def main():
         raise SystemExit("--suffix must be a multiple of the block")
     r = run_gpu(w, args.steps, args.warmup, log=lambda *a: None, kernel=args.kernel,
                 v_rotation=args.v_rotation, suffix=args.suffix,
-                time_build=(w.name == "longprompt"))
+                time_build=(w.name == "longprompt"), select_budget=args.select_budget)
     line = base_line(w, args, r["value"], r["ms"] / args.steps, world)
     if args.v_rotation:
         line["config"]["v_rotation"] = f"K-RPBH, Hadamard block {args.v_rotation}"
     if args.suffix:
         line["config"]["dual_cache_suffix_tokens"] = args.suffix
+    if args.select_budget:
+        line["config"]["select_budget"] = args.select_budget
+        line["config"]["select_bytes"] = ("the packed cache counted once per step (the scores read "
+                                          "all of it); the attention kernel figures sum its two "
+                                          "launches (softmax statistics over the whole cache, "
+                                          "then the gathered tokens)")
     line["config"]["L2_policy"] = (f"{r['R']} cache replicas used round-robin"
                                    if r["R"] > 1 else "cache larger than L2")
     line["config"]["L_mean"] = r["L_mean"]
@@ -792,7 +808,7 @@ def main():
                               "timed region = one CUDA graph replay of the steps")
     line["config"]["timing"] = TIMING_METHOD
     line["roofline"] = roofline(w, r, peaks, peak_kind, traffic)
-    if args.suffix:  # the recorded traffic is that of the single-cache launch
+    if args.suffix or args.select_budget:  # the recorded traffic is that of the plain launch
         line["roofline"]["traffic"] = None
     line["clocks"] = r["clocks"]
     line["e2e"] = r["e2e"]
@@ -800,7 +816,7 @@ def main():
     line.update(kernel_fields(w, r))
     if r["build"]:
         line["build"] = r["build"]
-    if not args.no_sub_records:
+    if not args.no_sub_records and not (args.select_budget or args.suffix or args.v_rotation):
         # every other configuration of the workload set, each with its own
         # roofline (same timing method, no end-to-end or oracle leg)
         line["workloads"] = {}
@@ -824,7 +840,7 @@ def main():
                 rec["build"] = rr["build"]
             line["workloads"][name] = rec
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.v_rotation \
-            and not args.suffix:
+            and not args.suffix and not args.select_budget:
         gbs, steps, el, desc = oracle_sample(w, args.cpu_seconds)
         line["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": _blas_threads(),
                                 "kind": "oracle", "sample": desc}

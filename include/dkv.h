@@ -346,7 +346,9 @@ int dkv_cache_set_option(dkv_cache* cache, int32_t key, int64_t value);
  * graph capture) is bracketed by CUDA events recorded on its stream.  This
  * call waits for them and returns, per kernel kind, the summed device time in
  * milliseconds and the launch count since the last read, then resets them.
- * kind: DKV_KERNEL_ATTENTION (the split attention kernel), DKV_KERNEL_COMBINE,
+ * kind: DKV_KERNEL_ATTENTION (the split attention kernel; for
+ * dkv_block_attention_selected also its scoring and top-k kernels and the
+ * attention over the kept tokens), DKV_KERNEL_COMBINE,
  * DKV_KERNEL_COMMIT, DKV_KERNEL_TRUNCATE. */
 enum { DKV_KERNEL_ATTENTION = 0, DKV_KERNEL_COMBINE = 1, DKV_KERNEL_COMMIT = 2,
        DKV_KERNEL_TRUNCATE = 3 };

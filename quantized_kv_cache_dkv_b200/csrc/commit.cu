@@ -78,6 +78,7 @@ constexpr int kThreads = 256;
 // [32 sl, 32 sl + 32) and V tokens [sl blk/4, (sl + 1) blk/4) of the block.
 constexpr int kSlices = 4;
 constexpr int kSliceCh = kHeadDim / kSlices;
+constexpr int kPendStride = 128 + 8;  // tokens per staged channel row (pending <= 128), padded
 
 __device__ __forceinline__ void range_check8(uint4 x, bool& range) {
   const uint32_t w[4] = {x.x, x.y, x.z, x.w};
@@ -252,6 +253,9 @@ __global__ void __launch_bounds__(kThreads)
 commit_kernel(const __grid_constant__ CacheView c, const uint16_t* __restrict__ k,
               const uint16_t* __restrict__ v, const uint32_t* __restrict__ pw,
               const __grid_constant__ CommitArgs ca) {
+  // the pending K stream of this CTA's 32 channels, channel-major (a
+  // thread's tokens are contiguous), filled by coalesced row loads
+  __shared__ __align__(16) uint16_t sk[kSliceCh * kPendStride];
   pdl_wait();
   pdl_trigger();
   const int u = blockIdx.x / kSlices, sl = blockIdx.x % kSlices;
@@ -326,7 +330,22 @@ commit_kernel(const __grid_constant__ CacheView c, const uint16_t* __restrict__ 
     j0 = (p0 - n_tail) / GK;
     count0 = c.prot_gstart[size_t(u) * size_t(c.nG + 1) + size_t(j0)];
     nK = nfull * kSliceCh * kthr;
+    // stage: item (token t, octet o) = 8 channels of one row, 16-byte loads;
+    // the block's values are range-checked (the tail's were on entry)
+    const int npend = n_tail + blk;
+    for (int i = tid; i < npend * (kSliceCh / 8); i += kThreads) {
+      const int t = i / (kSliceCh / 8), o = i % (kSliceCh / 8);
+      const uint16_t* src = t < n_tail ? c.k_tail + (size_t(u) * GK + t) * d
+                                       : ku + size_t(t - n_tail) * d;
+      const uint4 x = *reinterpret_cast<const uint4*>(src + kSliceCh * sl + 8 * o);
+      if (t >= n_tail) range_check8(x, range);
+      const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        sk[(8 * o + e) * kPendStride + t] = uint16_t(w4[e >> 1] >> (16 * (e & 1)));
+    }
   }
+  __syncthreads();
 
   // ------------------------------------------------------------------ V
   // likewise for V: vper channels of one token into vwpt words per thread
@@ -397,17 +416,24 @@ commit_kernel(const __grid_constant__ CacheView c, const uint16_t* __restrict__ 
         const uint32_t gw = wi == 0 ? gm[0] : (wi == 1 ? gm[1] : (wi == 2 ? gm[2] : gm[3]));
         const uint32_t mw = (gw >> (tw & 31)) & ((kper == 32 ? 0u : (1u << kper)) - 1u);
         float x[kper];
-        uint16_t raw[kper];
+        uint32_t raw2[kper / 2];  // the tokens' bf16 bits, two per word
         float mn = __int_as_float(0x7f800000), mx = -__int_as_float(0x7f800000);
+        {
+          // this thread's kper tokens: kper / 8 16-byte reads of its channel row
+          const uint4* row = reinterpret_cast<const uint4*>(sk + cl * kPendStride + gi * GK + tw);
+#pragma unroll
+          for (int o = 0; o < kper / 8; ++o) {
+            const uint4 x8 = row[o];
+            raw2[4 * o] = x8.x;
+            raw2[4 * o + 1] = x8.y;
+            raw2[4 * o + 2] = x8.z;
+            raw2[4 * o + 3] = x8.w;
+          }
+        }
+        auto raw = [&](int e) { return uint16_t(raw2[e >> 1] >> (16 * (e & 1))); };
 #pragma unroll
         for (int e = 0; e < kper; ++e) {
-          const int pi = gi * GK + tw + e;
-          const uint16_t b = pi < n_tail ? c.k_tail[(size_t(u) * GK + pi) * d + ch]
-                                         : ku[size_t(pi - n_tail) * d + ch];
-          raw[e] = b;
-          float f = bf16_bits_to_f32(b);
-          if (pi >= n_tail) range |= out_of_range(f);
-          f = sanitize(f);
+          float f = sanitize(bf16_bits_to_f32(raw(e)));
           x[e] = f;
           if (!((mw >> e) & 1u)) {
             mn = fminf(mn, f);
@@ -437,7 +463,7 @@ commit_kernel(const __grid_constant__ CacheView c, const uint16_t* __restrict__ 
           for (int e = 0; e < kper; ++e) {
             if (!((mw >> e) & 1u)) continue;
             if (DKV_IN_BOUNDS(rank < c.P, c.status)) {
-              c.prot_k[(size_t(u) * c.P + rank) * d + ch] = raw[e];
+              c.prot_k[(size_t(u) * c.P + rank) * d + ch] = raw(e);
               if (ch == 0) c.prot_pos[size_t(u) * c.P + rank] = int32_t(j * GK + tw + e);
             }
             ++rank;

@@ -693,8 +693,10 @@ int dkv_block_attention_selected(dkv_cache* c, const void* q, const void* k_act,
   sa.sel = sel;
   sa.sel_ld = sel_ld;
   sa.budget = budget;
-  e = dkv::launch_scores(sa, part, v.cap, s);
-  if (e == cudaSuccess) e = dkv::launch_topk(sa, part, v.cap, sc, sel, s);
+  e = timed_launch(c, DKV_KERNEL_ATTENTION, s, [&] { return dkv::launch_scores(sa, part, v.cap, s); });
+  if (e == cudaSuccess)
+    e = timed_launch(c, DKV_KERNEL_ATTENTION, s,
+                     [&] { return dkv::launch_topk(sa, part, v.cap, sc, sel, s); });
   if (e != cudaSuccess) return fail(DKV_ERR_CUDA, std::string("selection launch: ") + cudaGetErrorString(e));
   // attention over the selected tokens and the active block (mma.sync gather)
   dkv::CacheInfo cg = ci;
