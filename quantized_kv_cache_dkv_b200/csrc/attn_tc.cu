@@ -59,7 +59,7 @@ constexpr int kThreads = kWarps * 32;
 constexpr int kMmaWarp = 25;
 constexpr int kLoadWarp = 26;
 constexpr int kStages = 2;  // ring of packed tiles
-constexpr int kStagedProt = 24;  // protected K rows staged per tile (more: read from global)
+constexpr int kStagedProt = 4;  // protected K rows staged per tile (more: read from global)
 constexpr uint32_t kTileBytes = 128 * 128 * 2;
 // TMEM: O and three score buffers (tile j uses S_(j mod 3)), so three tiles'
 // QK -> softmax -> PV chains overlap; Q is an A operand in shared memory
@@ -83,7 +83,7 @@ struct Smem {
   // g0, index base of the staged positions}, positions (aligned superset),
   // and the bf16 K rows of the first kStagedProt entries
   static constexpr uint32_t kRHdr = 20480, kRPos = 20496, kRPk = 20624;
-  static constexpr uint32_t kStageBytes = 27648;
+  static constexpr uint32_t kStageBytes = kRPk + kStagedProt * 256;  // 21648
   static constexpr uint32_t kRing = kQ + 2 * 16384;
   static constexpr uint32_t kBar = kRing + kStages * kStageBytes;  // 32 mbarriers
   static constexpr uint32_t kRef = kBar + 32 * 8;   // [tile parity][128] reference max per row
@@ -1309,7 +1309,9 @@ constexpr int kRows = 32;  // query rows per unit
 constexpr int kN = 64;     // MMA N (rows padded)
 constexpr int kMmaWarp = 21, kLoadWarp = 22;
 constexpr int kStages = 2;
-constexpr uint32_t kColS0 = 0, kColS1 = 64, kColO = 128, kTmemCols = 256;
+// TMEM: four score buffers (tile j uses S_(j mod 4)) and O^T
+constexpr int kSBufs = 4;
+constexpr uint32_t kColS0 = 0, kColO = 256, kTmemCols = 512;
 // D f32, A and B f16, both MN-major, M = 128, N = 64
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 15) | (1u << 16) | ((uint32_t(kN) >> 3) << 17) |
                             ((128u >> 4) << 24);
@@ -1319,8 +1321,8 @@ constexpr int kRegSoftmax = 152, kRegProducer = 64, kRegControl = 56;
 
 struct Smem {
   static constexpr uint32_t kK0 = 0, kV0 = 2 * kTileBytes;
-  static constexpr uint32_t kP = 4 * kTileBytes;                   // P^T tile [128 tokens][64 rows]
-  static constexpr uint32_t kQ = kP + 128 * kN * 2;                // Q^T [128 channels][64 rows]
+  static constexpr uint32_t kP = 4 * kTileBytes;                   // 2 P^T tiles [128 tokens][64 rows]
+  static constexpr uint32_t kQ = kP + 2 * 128 * kN * 2;            // Q^T [128 channels][64 rows]
   static constexpr uint32_t kRing = kQ + 128 * kN * 2;
   static constexpr uint32_t kBar = kRing + kStages * ::dkv::Smem::kStageBytes;  // 32 mbarriers
   static constexpr uint32_t kFlag = kBar + 32 * 8;                 // [2][4] raise votes
@@ -1331,8 +1333,8 @@ struct Smem {
 // (VOTE, RED, EPI: the softmax threads' exchanges, bounded waits like every
 // other hand-off, so a CTA that aborts cannot leave a thread waiting)
 enum Bar {
-  KFULL = 0, KEMPTY = 2, VFULL = 4, VEMPTY = 6, SFULL = 8, SFREE = 10, PFULL = 12, QREADY = 13,
-  DONE = 14, VOTE = 15, RED = 16, EPI = 17, RFULL = 18, REMPTY = RFULL + kStages
+  KFULL = 0, KEMPTY = 2, VFULL = 4, VEMPTY = 6, SFULL = 8, SFREE = 12, PFULL = 16, QREADY = 18,
+  DONE = 19, VOTE = 20, RED = 21, EPI = 22, RFULL = 23, REMPTY = RFULL + kStages
 };
 
 // the 16-byte chunk of rows 8k..8k+7 of token / channel t in a [128][64]
@@ -1424,10 +1426,12 @@ __global__ void __launch_bounds__(tl::kThreads, 1) attn_tl_kernel(const __grid_c
       mbar_init(bar(tl::KEMPTY + b), 1);
       mbar_init(bar(tl::VFULL + b), 256);
       mbar_init(bar(tl::VEMPTY + b), 1);
+      mbar_init(bar(tl::PFULL + b), 128);
+    }
+    for (int b = 0; b < tl::kSBufs; ++b) {
       mbar_init(bar(tl::SFULL + b), 1);
       mbar_init(bar(tl::SFREE + b), 128);
     }
-    mbar_init(bar(tl::PFULL), 128);
     mbar_init(bar(tl::QREADY), 128);
     mbar_init(bar(tl::DONE), 1);
     mbar_init(bar(tl::VOTE), 128);
@@ -1482,6 +1486,7 @@ __global__ void __launch_bounds__(tl::kThreads, 1) attn_tl_kernel(const __grid_c
       for (int k = 4; k < 8; ++k) {
         *reinterpret_cast<uint4*>(sm + S::kQ + tl::nt_off(l, k)) = make_uint4(0u, 0u, 0u, 0u);
         *reinterpret_cast<uint4*>(sm + S::kP + tl::nt_off(l, k)) = make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(sm + S::kP + 16384 + tl::nt_off(l, k)) = make_uint4(0u, 0u, 0u, 0u);
       }
       fence_async_smem();
       mbar_arrive(bar(tl::QREADY));
@@ -1497,14 +1502,15 @@ __global__ void __launch_bounds__(tl::kThreads, 1) attn_tl_kernel(const __grid_c
     int n_raise = 0;  // phases of the tl::RED barrier used so far
 #pragma unroll 1
     for (int j = 0; j < nt && ok; ++j) {
-      const int b = j & 1;
+      const int b = j & 1;               // vote slot, P buffer
+      const int bs = j % tl::kSBufs;     // score buffer (its (j / 4)-th use)
       // tcgen05.ld is warp-collective: every branch around it is warp-uniform
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(tl::SFULL + b), (j >> 1) & 1, a, abort_flag))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(tl::SFULL + bs), (j / tl::kSBufs) & 1, a, abort_flag))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const uint32_t s_col = lane_base + (b ? tl::kColS1 : tl::kColS0);
+      const uint32_t s_col = lane_base + tl::kColS0 + 64u * uint32_t(bs);
       float x[tl::kRows];
       auto load_scores = [&]() {
         uint32_t sv[32];
@@ -1585,20 +1591,20 @@ __global__ void __launch_bounds__(tl::kThreads, 1) attn_tl_kernel(const __grid_c
         lsum[i + 1] += p1;
         pk[i / 2] = pack_h2(p0, p1);
       }
-      // the P^T tile is free once PV(j-1) has completed
-      if (j > 0 && !__all_sync(0xffffffffu, mbar_wait(bar(tl::VEMPTY + ((j - 1) & 1)),
-                                                      ((j - 1) >> 1) & 1, a, abort_flag))) {
+      // P^T buffer b is free once PV(j-2) has completed
+      if (j > 1 && !__all_sync(0xffffffffu, mbar_wait(bar(tl::VEMPTY + b), ((j - 2) >> 1) & 1, a,
+                                                      abort_flag))) {
         ok = false;
         break;
       }
 #pragma unroll
       for (int k = 0; k < 4; ++k)
-        *reinterpret_cast<uint4*>(sm + S::kP + tl::nt_off(l, k)) =
+        *reinterpret_cast<uint4*>(sm + S::kP + 16384u * uint32_t(b) + tl::nt_off(l, k)) =
             make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
       fence_async_smem();
       tc_fence_before();
-      mbar_arrive(bar(tl::PFULL));
-      mbar_arrive(bar(tl::SFREE + b));  // (S_b was last read above)
+      mbar_arrive(bar(tl::PFULL + b));
+      mbar_arrive(bar(tl::SFREE + bs));  // (S_bs was last read above)
     }
     // epilogue: row sums over the 128 tokens, then O^T / l per row
     if (ok) {
@@ -1646,15 +1652,15 @@ __global__ void __launch_bounds__(tl::kThreads, 1) attn_tl_kernel(const __grid_c
       loader_loop<KB, VB, tl::kStages>(a, uls, u, t_begin, nt, pipe, abort_flag, lane);
     } else if (warp == tl::kMmaWarp && lane == 0) {
       // ------------------------------------------------------------ MMA issuer
-      // QK(j) needs K_j and S_(j mod 2) read (tl::SFREE of tile j-2); PV(j) needs
-      // P_j (tl::PFULL, phase j) and V_j.  QK runs up to one tile ahead of PV.
+      // QK(j) needs K_j and S_(j mod 4) read (SFREE of tile j-4); PV(j) needs
+      // P_j (PFULL of buffer j mod 2) and V_j.  QK runs up to three tiles ahead of PV.
       bool ok = mbar_wait(bar(tl::QREADY), 0, a, abort_flag);
       tc_fence_after();
-      const uint32_t qbase = sm_base + S::kQ, pbase = sm_base + S::kP;
+      const uint32_t qbase = sm_base + S::kQ;
       int nq = 0, np = 0;
       auto issue_qk = [&]() {
         tc_fence_after();
-        const int b = nq & 1;
+        const int b = nq & 1, bs = nq % tl::kSBufs;
         const uint32_t kbase = sm_base + S::kK0 + b * kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)  // channels 16kk .. 16kk + 15
@@ -1662,34 +1668,40 @@ __global__ void __launch_bounds__(tl::kThreads, 1) attn_tl_kernel(const __grid_c
               "{\n\t.reg .pred p;\n\t"
               "setp.ne.b32 p, %4, 0;\n\t"
               "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(
-                  tmem + (b ? tl::kColS1 : tl::kColS0)),
+                  tmem + tl::kColS0 + 64u * uint32_t(bs)),
               "l"(sdesc_sw128(kbase + 4096 * kk, 1024, 2048)), "l"(sdesc_sw128(qbase + 2048 * kk, 8192, 1024)),
               "r"(tl::kIdesc), "r"(kk > 0 ? 1u : 0u)
               : "memory");
         mma_commit(bar(tl::KEMPTY + b));
-        mma_commit(bar(tl::SFULL + b));
+        mma_commit(bar(tl::SFULL + bs));
         ++nq;
       };
 #pragma unroll 1
       while (ok && np < nt) {
         // issue every QK that is ready and allowed (at most one ahead of PV)
-        while (nq < nt && nq <= np + 1 && mbar_test(bar(tl::KFULL + (nq & 1)), (nq >> 1) & 1) &&
-               (nq < 2 || mbar_test(bar(tl::SFREE + (nq & 1)), ((nq - 2) >> 1) & 1)))
+        auto s_free = [&](bool wait) {  // S_(nq mod 4) read by the softmax of tile nq - 4
+          if (nq < tl::kSBufs) return true;
+          const uint32_t sb = bar(tl::SFREE + nq % tl::kSBufs);
+          const uint32_t ph = ((nq - tl::kSBufs) / tl::kSBufs) & 1;
+          return wait ? mbar_wait(sb, ph, a, abort_flag) : mbar_test(sb, ph);
+        };
+        while (nq < nt && nq <= np + tl::kSBufs - 1 &&
+               mbar_test(bar(tl::KFULL + (nq & 1)), (nq >> 1) & 1) && s_free(false))
           issue_qk();
         if (np == nq) {
-          ok = mbar_wait(bar(tl::KFULL + (nq & 1)), (nq >> 1) & 1, a, abort_flag) &&
-               (nq < 2 || mbar_wait(bar(tl::SFREE + (nq & 1)), ((nq - 2) >> 1) & 1, a, abort_flag));
+          ok = mbar_wait(bar(tl::KFULL + (nq & 1)), (nq >> 1) & 1, a, abort_flag) && s_free(true);
           if (ok) issue_qk();
           continue;
         }
         const int bb = np & 1;
-        if (!mbar_wait(bar(tl::PFULL), np & 1, a, abort_flag) ||
+        if (!mbar_wait(bar(tl::PFULL + bb), (np >> 1) & 1, a, abort_flag) ||
             !mbar_wait(bar(tl::VFULL + bb), (np >> 1) & 1, a, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint32_t vbase = sm_base + S::kV0 + bb * kTileBytes;
+        const uint32_t pbase = sm_base + S::kP + 16384u * uint32_t(bb);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)  // tokens 16kk .. 16kk + 15
           asm volatile(
