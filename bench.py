@@ -700,11 +700,8 @@ def base_line(w, args, value, ms_per_step, world):
 
 
 def plan_name(w: synth.Workload, kernel: int) -> str:
-    if kernel == 1:
-        return "mma.sync"
-    if kernel == 2 and w.rows == 32:
-        return "tcgen05 (tokens on TMEM lanes)"
-    return "tcgen05 (query-row blocks)" if kernel in (2, 3) else str(kernel)
+    return {1: "mma.sync", 2: "tcgen05 (query-row blocks)",
+            3: "tcgen05 (tokens on TMEM lanes)"}.get(kernel, str(kernel))
 
 
 def kernel_fields(w: synth.Workload, r: dict) -> dict:
@@ -738,8 +735,9 @@ def main():
     ap.add_argument("--no-sub-records", action="store_true",
                     help="skip the per-workload records of the other configurations")
     ap.add_argument("--kernel", type=int, default=0, choices=[0, 1, 2, 3],
-                    help="attention kernel: 0 = library's choice, 1 = mma.sync, 2 = tcgen05, "
-                         "3 = tcgen05 with query-row blocks for every group")
+                    help="attention kernel: 0 = library's choice, 1 = mma.sync, 2 = tcgen05 "
+                         "(query-row blocks), 3 = tcgen05 with the tokens on the TMEM lanes "
+                         "(32-row query groups)")
     ap.add_argument("--B", type=int, default=0, help="override the workload's batch (profiling)")
     ap.add_argument("--L", type=int, default=0, help="override the committed length (profiling)")
     ap.add_argument("--v-rotation", type=int, default=0, choices=[0, 16, 32, 64, 128],
@@ -824,7 +822,7 @@ def main():
             if name == w.name:
                 continue
             ww = synth.WORKLOADS[name]
-            kern = args.kernel if (args.kernel != 2 or ww.rows % 32 == 0) else 0
+            kern = args.kernel if (args.kernel != 3 or ww.rows == 32) else 0
             rr = run_gpu(ww, args.steps, args.warmup, want_e2e=False, kernel=kern,
                          time_build=(name == "longprompt"))
             rec = {"value_gbs": round(rr["value"], 1),

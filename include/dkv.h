@@ -326,11 +326,11 @@ int dkv_cache_export_seq(dkv_cache* cache, int32_t seq, void* stream, dkv_export
  *   DKV_OPT_SPLITS: token splits per (sequence, kv-head) in attention;
  *     0 = chosen from the SM count (default).  Results agree within fp32
  *     rounding for any split count.
- *   DKV_OPT_ATTN_KERNEL: 0 = best available (default), 1 = warp-level
- *     mma.sync kernel, 2 = tcgen05 tensor-memory kernel (tokens on the TMEM
- *     lanes for 32-row query groups, query-row blocks of up to 128 rows
- *     otherwise), 3 = tcgen05 with query-row blocks for every group
- *     (DKV_ERR_UNSUPPORTED for 2 and 3 if the shape has no tcgen05 variant).
+ *   DKV_OPT_ATTN_KERNEL: 0 = best available (default: 2 where the shape has a
+ *     tcgen05 variant, else 1), 1 = warp-level mma.sync kernel, 2 = tcgen05
+ *     tensor-memory kernel with query-row blocks of up to 128 rows, 3 =
+ *     tcgen05 with the tokens on the TMEM lanes, for 32-row query groups only
+ *     (DKV_ERR_UNSUPPORTED for 2 and 3 where the shape has no such variant).
  *   DKV_OPT_TEST_STALL: bounds-checking build (libdkv_bc.so) only, else
  *     DKV_ERR_UNSUPPORTED.  A test of the bounded waits: value t >= 0 makes the
  *     tcgen05 kernel's loader withhold the copies of tile t (0 = the first

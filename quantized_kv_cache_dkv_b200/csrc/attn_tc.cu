@@ -24,20 +24,17 @@
 //   warps 16-23 V producers: dequantize V tiles (token rows, channels
 //               contiguous: MN-major, 128-byte swizzle), half a tile each
 //   warp 25     allocates TMEM; one lane issues the MMAs:
-//               S_j = Q K_j^T (A = Q from shared memory), O += P_j V_j (A = P
-//               from TMEM)
+//               S_j = Q K_j^T (A = Q from TMEM), O += P_j V_j (A = P from TMEM)
 //   warp 26     one lane streams each tile's packed K/V codes and fp16
 //               (scale, zero) pairs -- four contiguous ranges of the cache --
 //               and the tile's slice of the protected-K side table into a
-//               2-stage shared-memory ring with 1-D bulk copies
+//               3-stage shared-memory ring with 1-D bulk copies
 //               (cp.async.bulk, completion counted on an mbarrier), so HBM
 //               latency overlaps the dequantization and the MMAs
 // Tensor memory (512 columns x 128 lanes x 32 bit): O [0,128), S0 [128,256),
-// S1 [256,384), S2 [384,512): three score buffers, so the QK -> softmax -> PV
-// chains of three tiles overlap (the chain of one tile is longer than a
-// tile's share of the MMA and issue time).  P_j (fp16 pairs) overwrites the
-// first 64 columns of S_(j mod 3) once the scores are read; the PV MMAs take
-// their A operand there.
+// S1 [256,384), Q [384,448).  P_j (fp16 pairs) overwrites the first 64
+// columns of S_(j mod 2) once the scores are read; the PV MMAs take their A
+// operand there.
 // Hand-offs are mbarriers; MMA completion arrives through tcgen05.commit.
 // Every wait is bounded (about one second of %globaltimer): on expiry the
 // CTA raises DKV_FLAG_TIMEOUT, all roles leave their loops, the MMA lane waits
@@ -58,13 +55,10 @@ constexpr int kThreads = kWarps * 32;
 // 0-31 belong to warps 0 and 4).
 constexpr int kMmaWarp = 25;
 constexpr int kLoadWarp = 26;
-constexpr int kStages = 2;  // ring of packed tiles
-constexpr int kStagedProt = 4;  // protected K rows staged per tile (more: read from global)
+constexpr int kStages = 3;  // ring of packed tiles
+constexpr int kStagedProt = 8;  // protected K rows staged per tile (more: read from global)
 constexpr uint32_t kTileBytes = 128 * 128 * 2;
-// TMEM: O and three score buffers (tile j uses S_(j mod 3)), so three tiles'
-// QK -> softmax -> PV chains overlap; Q is an A operand in shared memory
-constexpr uint32_t kColO = 0, kColS0 = 128, kTmemCols = 512;
-constexpr int kSBufs = 3;
+constexpr uint32_t kColO = 0, kColS0 = 128, kColS1 = 256, kColQ = 384, kTmemCols = 512;
 
 // instruction descriptor: D f32, A f16 (K-major), B f16 (MN-major), M = N = 128
 constexpr uint32_t kIdesc = (1u << 4) | (0u << 7) | (0u << 10) | (0u << 15) | (1u << 16) |
@@ -73,9 +67,6 @@ constexpr uint32_t kIdesc = (1u << 4) | (0u << 7) | (0u << 10) | (0u << 15) | (1
 struct Smem {
   // offsets into the 1024-byte aligned dynamic shared memory
   static constexpr uint32_t kK0 = 0, kK1 = kTileBytes, kV0 = 2 * kTileBytes, kV1 = 3 * kTileBytes;
-  // Q, the A operand of QK: [128 rows][128 channels] fp16, K-major with the
-  // 128-byte swizzle, as two halves of 64 channels (16 KB each)
-  static constexpr uint32_t kQ = 4 * kTileBytes;
   // one ring stage: packed K codes (<= 8 KB: 128 tokens x 128 channels x 4 bit),
   // K (scale, zero) (<= 2 KB), packed V codes (<= 8 KB), V (scale, zero) (<= 2 KB)
   static constexpr uint32_t kRKc = 0, kRKsz = 8192, kRVc = 10240, kRVsz = 18432;
@@ -83,8 +74,8 @@ struct Smem {
   // g0, index base of the staged positions}, positions (aligned superset),
   // and the bf16 K rows of the first kStagedProt entries
   static constexpr uint32_t kRHdr = 20480, kRPos = 20496, kRPk = 20624;
-  static constexpr uint32_t kStageBytes = kRPk + kStagedProt * 256;  // 21648
-  static constexpr uint32_t kRing = kQ + 2 * 16384;
+  static constexpr uint32_t kStageBytes = kRPk + kStagedProt * 256;  // 22672
+  static constexpr uint32_t kRing = 4 * kTileBytes;
   static constexpr uint32_t kBar = kRing + kStages * kStageBytes;  // 32 mbarriers
   static constexpr uint32_t kRef = kBar + 32 * 8;   // [tile parity][128] reference max per row
   static constexpr uint32_t kLsum = kRef + 1024;    // [warpgroup][128] row sum, then its reference
@@ -92,8 +83,8 @@ struct Smem {
   static constexpr uint32_t kBytes = kMisc + 32;
 };
 enum Bar {
-  KFULL = 0, KEMPTY = 2, VFULL = 4, VEMPTY = 6, SFULL = 8, PFULL = 11, QREADY = 14, DONE = 15,
-  RFULL = 16, REMPTY = RFULL + kStages, RREADY = REMPTY + kStages, LSUM = RREADY + 2
+  KFULL = 0, KEMPTY = 2, VFULL = 4, VEMPTY = 6, SFULL = 8, PFULL = 10, QREADY = 12, DONE = 13,
+  RFULL = 14, REMPTY = 14 + kStages, RREADY = 14 + 2 * kStages, LSUM = RREADY + 2
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -310,17 +301,6 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       "setp.ne.b32 p, %3, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %4, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(accumulate), "r"(kIdesc)
-      : "memory");
-}
-
-// D[tmem] (+)= A[smem] * B[smem]^T
-__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                       uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %3, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %4, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(accumulate), "r"(kIdesc)
       : "memory");
 }
 
@@ -944,11 +924,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       mbar_init(bar(KEMPTY + b), 1);
       mbar_init(bar(VFULL + b), 256);
       mbar_init(bar(VEMPTY + b), 1);
-      mbar_init(bar(RREADY + b), 128);
-    }
-    for (int b = 0; b < kSBufs; ++b) {
       mbar_init(bar(SFULL + b), 1);
       mbar_init(bar(PFULL + b), 128);
+      mbar_init(bar(RREADY + b), 128);
     }
     mbar_init(bar(QREADY), 256);
     mbar_init(bar(LSUM), 256);
@@ -1004,14 +982,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         qv[4 * i + 2] = y.z;
         qv[4 * i + 3] = y.w;
       }
-      // row lr, channels [64h, 64h + 64): the 16-byte chunk c of the row at
-      // chunk c ^ (row mod 8) of its 128-byte line (K-major, 128-byte swizzle)
-      uint8_t* qh = sm + Smem::kQ + h * 16384 + lr * 128;
-#pragma unroll
-      for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<uint4*>(qh + ((c ^ (lr & 7)) << 4)) =
-            make_uint4(qv[4 * c], qv[4 * c + 1], qv[4 * c + 2], qv[4 * c + 3]);
-      fence_async_smem();
+      tmem_st32(lane_base + kColQ + 32 * h, qv);
+      tmem_st_wait();
+      tc_fence_before();
       mbar_arrive(bar(QREADY));
     }
     // Every tile j has one reference max per row, r_j (log2 units), non-
@@ -1024,18 +997,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     bool ok = true;
 #pragma unroll 1
     for (int j = h; j < nt && ok; j += 2) {
-      const int b = h;  // reference slot and RREADY barrier of this warpgroup's tiles
-      const int bs = j % kSBufs;  // score buffer of tile j (its (j / 3)-th use)
-      const uint32_t s_col = kColS0 + 128u * uint32_t(bs);
+      const int b = h;  // S buffer, reference slot and barriers of this warpgroup's tiles
+      const uint32_t s_col = b ? kColS1 : kColS0;
       // tcgen05.ld/st are warp-collective: every branch around them is warp-uniform
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(SFULL + bs), (j / kSBufs) & 1, a, abort_flag))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(SFULL + b), (j >> 1) & 1, a, abort_flag))) {
         ok = false;
         break;
       }
       tc_fence_after();
       if (!warp_rows) {
         mbar_arrive(bar(RREADY + b));
-        mbar_arrive(bar(PFULL + bs));
+        mbar_arrive(bar(PFULL + b));
         continue;
       }
       const int64_t tile_start = (t_begin + j) * TT;
@@ -1144,7 +1116,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(bar(PFULL + bs));
+      mbar_arrive(bar(PFULL + b));
     }
     // epilogue: wait for the last PV, combine the two warpgroups' row sums at
     // the final reference (the largest, references never decrease), write O
@@ -1216,46 +1188,44 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     // ------------------------------------------------------------ MMA issuer
     bool ok = mbar_wait(bar(QREADY), 0, a, abort_flag);
     tc_fence_after();
-    // QK(j) needs K_j (KFULL) and S_(j mod 3) free, i.e. PV(j-3) issued (MMAs
-    // run in issue order); PV(i) needs P_i (PFULL) and V_i (VFULL).  Every QK
-    // that is ready and allowed is issued at once; otherwise the lane sleeps
-    // (suspending mbarrier wait) on the barrier it needs next: P of the
-    // oldest un-issued PV, or K of the next QK when no PV is pending.  Barrier
-    // phases cannot run ahead: each next phase needs an MMA issued here first.
+    // QK(j) needs K_j (KFULL) and S_(j mod 2) free, i.e. PV(j-2) issued; PV(i)
+    // needs P_i (PFULL) and V_i (VFULL).  Every QK that is ready and allowed
+    // is issued at once; otherwise the lane sleeps (suspending mbarrier wait)
+    // on the barrier it needs next: P of the oldest un-issued PV, or K of the
+    // next QK when no PV is pending.  Barrier phases cannot run ahead: each
+    // next phase needs an MMA issued here first.
     int nq = 0, np = 0;
-    const uint32_t qbase = sm_base + Smem::kQ;
     auto issue_qk = [&]() {
       tc_fence_after();
-      const int b = nq & 1, bs = nq % kSBufs;
+      const int b = nq & 1;
       const uint32_t kbase = sm_base + (b ? Smem::kK1 : Smem::kK0);
-      const uint32_t s_col = kColS0 + 128u * uint32_t(bs);
+      const uint32_t s_col = b ? kColS1 : kColS0;
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk)  // channels 16kk .. 16kk + 15: Q half kk / 4, 32 bytes in
-        mma_ss(tmem + s_col, sdesc_sw128(qbase + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-               sdesc_sw128(kbase + 4096 * kk, 1024, 2048), kk > 0 ? 1u : 0u);
+      for (int kk = 0; kk < 8; ++kk)
+        mma_ts(tmem + s_col, tmem + kColQ + 8 * kk, sdesc_sw128(kbase + 4096 * kk, 1024, 2048),
+               kk > 0 ? 1u : 0u);
       mma_commit(bar(KEMPTY + b));
-      mma_commit(bar(SFULL + bs));
+      mma_commit(bar(SFULL + b));
       ++nq;
     };
 #pragma unroll 1
     while (ok && np < nt) {
-      while (nq < nt && nq <= np + kSBufs - 1 && mbar_test(bar(KFULL + (nq & 1)), (nq >> 1) & 1))
-        issue_qk();
+      while (nq < nt && nq <= np + 1 && mbar_test(bar(KFULL + (nq & 1)), (nq >> 1) & 1)) issue_qk();
       if (np == nq) {
         // nothing to multiply by P yet: wait for the next K tile
         ok = mbar_wait(bar(KFULL + (nq & 1)), (nq >> 1) & 1, a, abort_flag);
         if (ok) issue_qk();
         continue;
       }
-      const int bb = np & 1, bps = np % kSBufs;
-      if (!mbar_wait(bar(PFULL + bps), (np / kSBufs) & 1, a, abort_flag) ||
+      const int bb = np & 1;
+      if (!mbar_wait(bar(PFULL + bb), (np >> 1) & 1, a, abort_flag) ||
           !mbar_wait(bar(VFULL + bb), (np >> 1) & 1, a, abort_flag)) {
         ok = false;
         break;
       }
       tc_fence_after();
       const uint32_t vbase = sm_base + (bb ? Smem::kV1 : Smem::kV0);
-      const uint32_t p_col = kColS0 + 128u * uint32_t(bps);
+      const uint32_t p_col = bb ? kColS1 : kColS0;
       const int64_t pv_start = (t_begin + np) * TT;
       const int n_tok = uls->n_tok;
       const int nk = n_tok - pv_start < TT ? int(n_tok - pv_start) >> 4 : TT / 16;

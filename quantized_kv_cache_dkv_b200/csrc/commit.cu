@@ -76,8 +76,10 @@ __device__ __forceinline__ uint32_t code_of(float x, const GroupQuant& q, int le
 constexpr int kThreads = 256;
 // CTAs per (sequence, kv-head) unit: slice sl takes K channels
 // [32 sl, 32 sl + 32) and V tokens [sl blk/4, (sl + 1) blk/4) of the block.
-constexpr int kSlices = 4;
-constexpr int kSliceCh = kHeadDim / kSlices;
+// CTAs per (sequence, kv-head) unit, chosen per launch from the unit count
+// (1, 2 or 4, about two CTAs per SM): slice sl of nsl takes K channels
+// [sl 128/nsl, (sl + 1) 128/nsl) and V tokens [sl blk/nsl, (sl + 1) blk/nsl).
+constexpr int kMaxSlices = 4;
 constexpr int kPendStride = 128 + 8;  // tokens per staged channel row (pending <= 128), padded
 
 __device__ __forceinline__ void range_check8(uint4 x, bool& range) {
@@ -238,7 +240,7 @@ __device__ __forceinline__ int group_mask(const CacheView& c, const uint32_t* tm
   return kept;
 }
 
-// Quantize-on-commit of one block.  Grid: kSlices CTAs per unit.  Every
+// Quantize-on-commit of one block.  Grid: nsl CTAs per unit.  Every
 // thread produces one packed code word: K item (group, channel, word) covers
 // the 32/KB tokens of one word of one channel's group, V item (token, word)
 // the 32/VB channels of one word of one token.  A group's min / max is
@@ -252,13 +254,14 @@ template <int KB, int VB>
 __global__ void __launch_bounds__(kThreads)
 commit_kernel(const __grid_constant__ CacheView c, const uint16_t* __restrict__ k,
               const uint16_t* __restrict__ v, const uint32_t* __restrict__ pw,
-              const __grid_constant__ CommitArgs ca) {
+              const __grid_constant__ CommitArgs ca, int nsl) {
   // the pending K stream of this CTA's 32 channels, channel-major (a
   // thread's tokens are contiguous), filled by coalesced row loads
-  __shared__ __align__(16) uint16_t sk[kSliceCh * kPendStride];
+  __shared__ __align__(16) uint16_t sk[kHeadDim * kPendStride];
   pdl_wait();
   pdl_trigger();
-  const int u = blockIdx.x / kSlices, sl = blockIdx.x % kSlices;
+  const int u = blockIdx.x / nsl, sl = blockIdx.x % nsl;
+  const int sch = kHeadDim / nsl;  // K channels of this CTA
   // the unit's sequence: does it commit, at which position, after a roll-back?
   const int sq = u / c.Hkv;
   if (!((ca.commit[sq >> 5] >> (sq & 31)) & 1u)) return;
@@ -284,7 +287,7 @@ commit_kernel(const __grid_constant__ CacheView c, const uint16_t* __restrict__ 
                          (VB == 16 || c.sink <= c.cap),
                      c.status))
     return;
-  const int tpc = blk / kSlices;  // V (and raw K) tokens of this CTA
+  const int tpc = blk / nsl;  // V (and raw K) tokens of this CTA
   const int t_lo = sl * tpc;
 
   // ------------------------------------------------------------------ K
@@ -310,11 +313,11 @@ commit_kernel(const __grid_constant__ CacheView c, const uint16_t* __restrict__ 
     // the group stays incomplete: this CTA's channels of the block go to the
     // bf16 tail; the slice-0 CTA writes the tail's protect words
     uint16_t* tail = c.k_tail + size_t(u) * GK * d;
-    for (int i = tid; i < blk * (kSliceCh / 8); i += kThreads) {
-      const int t = i / (kSliceCh / 8), o = i % (kSliceCh / 8);
-      const uint4 x = *reinterpret_cast<const uint4*>(ku + size_t(t) * d + kSliceCh * sl + 8 * o);
+    for (int i = tid; i < blk * (sch / 8); i += kThreads) {
+      const int t = i / (sch / 8), o = i % (sch / 8);
+      const uint4 x = *reinterpret_cast<const uint4*>(ku + size_t(t) * d + sch * sl + 8 * o);
       range_check8(x, range);
-      *reinterpret_cast<uint4*>(tail + size_t(n_tail + t) * d + kSliceCh * sl + 8 * o) = x;
+      *reinterpret_cast<uint4*>(tail + size_t(n_tail + t) * d + sch * sl + 8 * o) = x;
     }
     if (sl == 0 && tid < nbw)
       c.tail_mask[size_t(u) * c.twords + n_tail / 32 + tid] =
@@ -329,15 +332,15 @@ commit_kernel(const __grid_constant__ CacheView c, const uint16_t* __restrict__ 
     nfull = (n_tail + blk) / GK;
     j0 = (p0 - n_tail) / GK;
     count0 = c.prot_gstart[size_t(u) * size_t(c.nG + 1) + size_t(j0)];
-    nK = nfull * kSliceCh * kthr;
+    nK = nfull * sch * kthr;
     // stage: item (token t, octet o) = 8 channels of one row, 16-byte loads;
     // the block's values are range-checked (the tail's were on entry)
     const int npend = n_tail + blk;
-    for (int i = tid; i < npend * (kSliceCh / 8); i += kThreads) {
-      const int t = i / (kSliceCh / 8), o = i % (kSliceCh / 8);
+    for (int i = tid; i < npend * (sch / 8); i += kThreads) {
+      const int t = i / (sch / 8), o = i % (sch / 8);
       const uint16_t* src = t < n_tail ? c.k_tail + (size_t(u) * GK + t) * d
                                        : ku + size_t(t - n_tail) * d;
-      const uint4 x = *reinterpret_cast<const uint4*>(src + kSliceCh * sl + 8 * o);
+      const uint4 x = *reinterpret_cast<const uint4*>(src + sch * sl + 8 * o);
       if (t >= n_tail) range_check8(x, range);
       const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
@@ -395,8 +398,8 @@ commit_kernel(const __grid_constant__ CacheView c, const uint16_t* __restrict__ 
     if constexpr (KB < 16) {
       if (it < nK) {
         constexpr int levels = (1 << KB) - 1;
-        const int w = it % kthr, cl = (it / kthr) % kSliceCh, gi = it / (kthr * kSliceCh);
-        const int ch = kSliceCh * sl + cl;
+        const int w = it % kthr, cl = (it / kthr) % sch, gi = it / (kthr * sch);
+        const int ch = sch * sl + cl;
         const int64_t j = j0 + gi;
         const uint32_t* tmask = c.tail_mask + size_t(u) * c.twords;
         // side-table entries stored before group gi (groups of this commit
@@ -553,8 +556,10 @@ __global__ void truncate_kernel(const __grid_constant__ CacheView c,
 template <int KB, int VB>
 cudaError_t launch_kv(const CacheView& c, const uint16_t* k, const uint16_t* v,
                       const uint32_t* pw, const CommitArgs& ca, cudaStream_t s) {
-  const cudaError_t e = launch_pdl(commit_kernel<KB, VB>, dim3(unsigned(c.U) * kSlices),
-                                   dim3(kThreads), 0, s, c, k, v, pw, ca);
+  // about two CTAs per SM (148 SMs): four slices for small batches, one for large
+  const int nsl = c.U >= 296 ? 1 : (c.U >= 148 ? 2 : kMaxSlices);
+  const cudaError_t e = launch_pdl(commit_kernel<KB, VB>, dim3(unsigned(c.U) * unsigned(nsl)),
+                                   dim3(kThreads), 0, s, c, k, v, pw, ca, nsl);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

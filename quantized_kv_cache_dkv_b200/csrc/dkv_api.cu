@@ -200,15 +200,15 @@ int plan_attention(const CacheInfo& ci, AttnArgs* a, int* kernel_out, const char
     *err = "no tokens to attend to";
     return DKV_ERR_INVALID_ARG;
   }
-  // kernel 2: tcgen05, tokens on TMEM lanes for 32-row query groups, query-row
-  // blocks otherwise; 3: tcgen05 with query-row blocks for every group
+  // kernel 2: tcgen05 with query-row blocks; 3: tcgen05 with the tokens on
+  // the TMEM lanes (32-row query groups only)
   int kernel = ci.opt_kernel;
   if (kernel == 0) kernel = tc_supported(v) ? 2 : 1;
-  if (kernel >= 2 && !tc_supported(v)) {
+  if ((kernel >= 2 && !tc_supported(v)) || (kernel == 3 && v.rows != 32)) {
     *err = "no tcgen05 attention variant for this shape";
     return DKV_ERR_UNSUPPORTED;
   }
-  a->tc_layout = (kernel == 2 && v.rows == 32) ? 1 : 0;
+  a->tc_layout = kernel == 3 ? 1 : 0;
   const int tile = kernel >= 2 ? kTcTile : kMmaTile;
   const int64_t n_tiles = ceil_div(a->n_tok, tile);
   const int64_t nrb = kernel >= 2 ? (v.rows + 127) / 128 : 1;
@@ -877,7 +877,7 @@ int dkv_cache_set_option(dkv_cache* c, int32_t key, int64_t value) {
       return DKV_OK;
     case DKV_OPT_ATTN_KERNEL:
       if (value < 0 || value > 3) return fail(DKV_ERR_INVALID_ARG, "kernel must be 0, 1, 2 or 3");
-      if (value >= 2 && !dkv::tc_supported(c->v))
+      if ((value >= 2 && !dkv::tc_supported(c->v)) || (value == 3 && c->v.rows != 32))
         return fail(DKV_ERR_UNSUPPORTED, "no tcgen05 attention variant for this shape");
       c->opt_kernel = int32_t(value);
       return DKV_OK;

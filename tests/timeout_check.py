@@ -28,14 +28,16 @@ from gpu_util import (assert_close, commit_both, default_P, default_cap, dev_bf1
 def main():
     import quantized_kv_cache_dkv_b200 as dkv
     print("library:", os.path.basename(dkv.LIB_PATH), flush=True)
-    # 128-row query groups (4 query heads x 32-token blocks): the row-block
-    # kernel; 32-row groups (one query head per kv-head): tokens on lanes
-    check(dkv, synth.WORKLOADS["tiny"].with_(B=2, Hq=8, Hkv=2, L=1024, prot_frac=0.02))
-    check(dkv, synth.WORKLOADS["tiny"].with_(B=2, Hq=2, Hkv=2, L=1024, prot_frac=0.02))
+    # 128-row query groups (4 query heads x 32-token blocks) and 32-row groups
+    # (one query head per kv-head) on the row-block kernel; 32-row groups with
+    # the tokens on the TMEM lanes
+    check(dkv, synth.WORKLOADS["tiny"].with_(B=2, Hq=8, Hkv=2, L=1024, prot_frac=0.02), 2)
+    check(dkv, synth.WORKLOADS["tiny"].with_(B=2, Hq=2, Hkv=2, L=1024, prot_frac=0.02), 2)
+    check(dkv, synth.WORKLOADS["tiny"].with_(B=2, Hq=2, Hkv=2, L=1024, prot_frac=0.02), 3)
     print("OK timeout path", flush=True)
 
 
-def check(dkv, w):
+def check(dkv, w, kernel):
     import torch
     n_blocks = w.L // w.blk
     cap = default_cap(w, n_blocks + 1)
@@ -43,7 +45,7 @@ def check(dkv, w):
 
     def built():
         cache = dkv.dkv_cache_alloc(gpu_config(dkv, w, cap, P))
-        dkv.dkv_cache_set_option(cache, dkv.DKV_OPT_ATTN_KERNEL, 2)
+        dkv.dkv_cache_set_option(cache, dkv.DKV_OPT_ATTN_KERNEL, kernel)
         return cache
 
     cache = built()
