@@ -1,13 +1,15 @@
 """Build libdkv.so in-tree for sm_100a with nvcc.
 
-    python quantized_kv_cache_dkv_b200/build.py [--force] [-v] [--bounds-check]
+    python quantized_kv_cache_dkv_b200/build.py [--force] [-v] [--bounds-check | --trace]
 
 Objects go to quantized_kv_cache_dkv_b200/_build/, the library to
 quantized_kv_cache_dkv_b200/libdkv.so.  --bounds-check builds the
 bounds-checking variant instead (DKV_BOUNDS_CHECK: kernels check their index
 arithmetic and copy ranges, record DKV_FLAG_BOUNDS and skip the access) into
-_build_bc/ and libdkv_bc.so.  A source is recompiled when it or any header is
-newer than its object.
+_build_bc/ and libdkv_bc.so; --trace the pipeline-trace variant (DKV_TRACE:
+the tcgen05 kernels stamp the clock at each hand-off of CTA 0, read by
+pipeline_trace.py) into _build_trace/ and libdkv_trace.so.  A source is
+recompiled when it or any header is newer than its object.
 """
 from __future__ import annotations
 
@@ -25,6 +27,8 @@ BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libdkv.so")
 BUILD_BC = os.path.join(HERE, "_build_bc")
 LIB_BC = os.path.join(HERE, "libdkv_bc.so")
+BUILD_TRACE = os.path.join(HERE, "_build_trace")
+LIB_TRACE = os.path.join(HERE, "libdkv_trace.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2",
@@ -59,9 +63,14 @@ def _compile(src: str, obj: str, verbose: bool, extra=()) -> None:
         raise RuntimeError(f"nvcc failed on {os.path.basename(src)}")
 
 
-def build(force: bool = False, verbose: bool = False, bounds_check: bool = False) -> str:
-    build_dir, lib = (BUILD_BC, LIB_BC) if bounds_check else (BUILD, LIB)
-    extra = ["-DDKV_BOUNDS_CHECK"] if bounds_check else []
+def build(force: bool = False, verbose: bool = False, bounds_check: bool = False,
+          trace: bool = False) -> str:
+    if bounds_check:
+        build_dir, lib, extra = BUILD_BC, LIB_BC, ["-DDKV_BOUNDS_CHECK"]
+    elif trace:
+        build_dir, lib, extra = BUILD_TRACE, LIB_TRACE, ["-DDKV_TRACE"]
+    else:
+        build_dir, lib, extra = BUILD, LIB, []
     os.makedirs(build_dir, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     hdr_t = _headers_mtime()
@@ -87,4 +96,4 @@ def build(force: bool = False, verbose: bool = False, bounds_check: bool = False
 
 if __name__ == "__main__":
     print(build(force="--force" in sys.argv, verbose="-v" in sys.argv,
-                bounds_check="--bounds-check" in sys.argv))
+                bounds_check="--bounds-check" in sys.argv, trace="--trace" in sys.argv))

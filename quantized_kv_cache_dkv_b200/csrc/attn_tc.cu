@@ -47,6 +47,25 @@
 namespace dkv {
 namespace {
 
+// Pipeline trace (trace build, DKV_TRACE, libdkv_trace.so): clock64 stamps of
+// CTA 0 of the last launch, per event and tile (first 64 tiles), read with
+// dkv_trace_read.  In the normal build the stamps compile to nothing.
+#ifdef DKV_TRACE
+__device__ unsigned long long g_trace[16][64];
+#define DKV_TR(e, j)                                                            \
+  do {                                                                          \
+    if (blockIdx.x == 0 && (j) < 64) g_trace[e][j] = static_cast<unsigned long long>(clock64()); \
+  } while (0)
+#else
+#define DKV_TR(e, j) \
+  do {               \
+  } while (0)
+#endif
+// events: 0 loader issues the tile's copies, 1/2 K producer starts/ends the
+// tile, 11/3/4 V producer has its buffer / starts / ends, 5 QK issued, 6
+// softmax has the scores, 12 softmax after its first pass or vote, 7 P
+// written, 8 PV issued, 9 CTA start, 10 CTA end
+
 constexpr int TT = kTcTile;              // tokens per tile
 constexpr int kWarps = 28;  // seven warpgroups; warps 26, 27 only complete the last one
 constexpr int kThreads = kWarps * 32;
@@ -714,9 +733,11 @@ __device__ __forceinline__ void k_producer_loop(const AttnArgs& a, const UnitLen
     const int b = j & 1, st = j % STAGES;
     if (!mbar_wait(p.kempty + 8u * b, ((j >> 1) & 1) ^ 1, a, abort_flag)) break;
     if (!mbar_wait(p.rfull + 8u * st, (j / STAGES) & 1, a, abort_flag)) break;
+    if (pt == 0) DKV_TR(1, j);
     fill_k_tile<KB>(a, *uls, u, (t_begin + j) * TT, p.sm + p.k_buf0 + b * kTileBytes,
                     p.sm + p.ring + st * Smem::kStageBytes, c, qh, ko);
     fence_async_smem();
+    if (pt == 0) DKV_TR(2, j);
     mbar_arrive(p.kfull + 8u * b);
     mbar_arrive(p.rempty + 8u * st);
   }
@@ -733,10 +754,13 @@ __device__ __forceinline__ void v_producer_loop(const AttnArgs& a, const UnitLen
   for (int j = 0; j < nt; ++j) {
     const int b = j & 1, st = j % STAGES;
     if (!mbar_wait(p.vempty + 8u * b, ((j >> 1) & 1) ^ 1, a, abort_flag)) break;
+    if (pt == 0) DKV_TR(11, j);
     if (!mbar_wait(p.rfull + 8u * st, (j / STAGES) & 1, a, abort_flag)) break;
+    if (pt == 0) DKV_TR(3, j);
     fill_v_tile<KB, VB, SINK>(a, *uls, u, (t_begin + j) * TT, p.sm + p.v_buf0 + b * kTileBytes,
                               p.sm + p.ring + st * Smem::kStageBytes, pt, vo);
     fence_async_smem();
+    if (pt == 0) DKV_TR(4, j);
     mbar_arrive(p.vfull + 8u * b);
     mbar_arrive(p.rempty + 8u * st);
   }
@@ -777,6 +801,7 @@ __device__ __forceinline__ void loader_loop(const AttnArgs& a, const UnitLen* ul
     const uint32_t rfull = p.rfull + 8u * st;
     if (!__all_sync(0xffffffffu, mbar_wait(p.rempty + 8u * st, ((j / STAGES) & 1) ^ 1, a, abort_flag)))
       break;
+    if (lane == 0) DKV_TR(0, j);
     ++issued;
 #ifdef DKV_BOUNDS_CHECK
     if (j == a.test_stall_tile) {
@@ -949,6 +974,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (threadIdx.x == 0) DKV_TR(9, 0);
   const uint32_t tmem = *tmem_slot;
 
   if (warp < 8) {
@@ -1005,6 +1031,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         break;
       }
       tc_fence_after();
+      if ((threadIdx.x & 127) == 0) DKV_TR(6, j);
       if (!warp_rows) {
         mbar_arrive(bar(RREADY + b));
         mbar_arrive(bar(PFULL + b));
@@ -1046,6 +1073,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         r_prev = ref[(b ^ 1) * 128 + lr];
       }
       // lazy rescale, decided per warp; rows whose max did not grow keep r_prev
+      if ((threadIdx.x & 127) == 0) DKV_TR(12, j);
       const bool rescale = __any_sync(0xffffffffu, mx > r_prev + 8.f);
       const float r_j = rescale ? fmaxf(r_prev, mx) : r_prev;
       ref[b * 128 + lr] = r_j;
@@ -1116,6 +1144,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       }
       tmem_st_wait();
       tc_fence_before();
+      if ((threadIdx.x & 127) == 0) DKV_TR(7, j);
       mbar_arrive(bar(PFULL + b));
     }
     // epilogue: wait for the last PV, combine the two warpgroups' row sums at
@@ -1196,6 +1225,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     // next phase needs an MMA issued here first.
     int nq = 0, np = 0;
     auto issue_qk = [&]() {
+      DKV_TR(5, nq);
       tc_fence_after();
       const int b = nq & 1;
       const uint32_t kbase = sm_base + (b ? Smem::kK1 : Smem::kK0);
@@ -1224,6 +1254,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         break;
       }
       tc_fence_after();
+      DKV_TR(8, np);
       const uint32_t vbase = sm_base + (bb ? Smem::kV1 : Smem::kV0);
       const uint32_t p_col = bb ? kColS1 : kColS0;
       const int64_t pv_start = (t_begin + np) * TT;
@@ -1244,6 +1275,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 
   tc_fence_before();
   __syncthreads();
+  if (threadIdx.x == 0) DKV_TR(10, 0);
   if (warp == kMmaWarp) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
@@ -1425,6 +1457,7 @@ __global__ void __launch_bounds__(tl::kThreads, 1) attn_tl_kernel(const __grid_c
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (threadIdx.x == 0) DKV_TR(9, 0);
   const uint32_t tmem = *tmem_slot;
 
   if (warp < 4) {
@@ -1480,6 +1513,7 @@ __global__ void __launch_bounds__(tl::kThreads, 1) attn_tl_kernel(const __grid_c
         break;
       }
       tc_fence_after();
+      if (threadIdx.x == 0) DKV_TR(6, j);
       const uint32_t s_col = lane_base + tl::kColS0 + 64u * uint32_t(bs);
       float x[tl::kRows];
       auto load_scores = [&]() {
@@ -1505,6 +1539,7 @@ __global__ void __launch_bounds__(tl::kThreads, 1) attn_tl_kernel(const __grid_c
         ok = false;
         break;
       }
+      if (threadIdx.x == 0) DKV_TR(12, j);
       raise = flag[b * 4] | flag[b * 4 + 1] | flag[b * 4 + 2] | flag[b * 4 + 3];
       if (raise) {
         // tile max of every row over the 128 tokens (the reduction takes x
@@ -1573,6 +1608,7 @@ __global__ void __launch_bounds__(tl::kThreads, 1) attn_tl_kernel(const __grid_c
             make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
       fence_async_smem();
       tc_fence_before();
+      if (threadIdx.x == 0) DKV_TR(7, j);
       mbar_arrive(bar(tl::PFULL + b));
       mbar_arrive(bar(tl::SFREE + bs));  // (S_bs was last read above)
     }
@@ -1630,6 +1666,7 @@ __global__ void __launch_bounds__(tl::kThreads, 1) attn_tl_kernel(const __grid_c
       int nq = 0, np = 0;
       auto issue_qk = [&]() {
         tc_fence_after();
+        DKV_TR(5, nq);
         const int b = nq & 1, bs = nq % tl::kSBufs;
         const uint32_t kbase = sm_base + S::kK0 + b * kTileBytes;
 #pragma unroll
@@ -1670,6 +1707,7 @@ __global__ void __launch_bounds__(tl::kThreads, 1) attn_tl_kernel(const __grid_c
           break;
         }
         tc_fence_after();
+        DKV_TR(8, np);
         const uint32_t vbase = sm_base + S::kV0 + bb * kTileBytes;
         const uint32_t pbase = sm_base + S::kP + 16384u * uint32_t(bb);
 #pragma unroll
@@ -1692,6 +1730,7 @@ __global__ void __launch_bounds__(tl::kThreads, 1) attn_tl_kernel(const __grid_c
 
   tc_fence_before();
   __syncthreads();
+  if (threadIdx.x == 0) DKV_TR(10, 0);
   if (warp == tl::kMmaWarp) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(tl::kTmemCols));
@@ -1760,3 +1799,15 @@ cudaError_t launch_attention_tc(const AttnArgs& a, cudaStream_t s) {
 }
 
 }  // namespace dkv
+
+#ifdef DKV_TRACE
+// trace build only: the stamps of the last traced launch (16 x 64 uint64, host
+// buffer), and their reset to zero
+extern "C" int dkv_trace_read(unsigned long long* out) {
+  return int(cudaMemcpyFromSymbol(out, dkv::g_trace, sizeof(dkv::g_trace)));
+}
+extern "C" int dkv_trace_clear(void) {
+  static unsigned long long zero[16][64] = {};
+  return int(cudaMemcpyToSymbol(dkv::g_trace, zero, sizeof(zero)));
+}
+#endif
