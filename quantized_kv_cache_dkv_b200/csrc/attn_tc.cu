@@ -64,7 +64,8 @@ __device__ unsigned long long g_trace[16][64];
 // events: 0 loader issues the tile's copies, 1/2 K producer starts/ends the
 // tile, 11/3/4 V producer has its buffer / starts / ends, 5 QK issued, 6
 // softmax has the scores, 12 softmax after its first pass or vote, 7 P
-// written, 8 PV issued, 9 CTA start, 10 CTA end
+// written, 8 PV issue starts, 13 PV issued and committed, 14 QK issued and
+// committed, 9 CTA start, 10 CTA end
 
 constexpr int TT = kTcTile;              // tokens per tile
 constexpr int kWarps = 28;  // seven warpgroups; warps 26, 27 only complete the last one
@@ -1236,6 +1237,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                kk > 0 ? 1u : 0u);
       mma_commit(bar(KEMPTY + b));
       mma_commit(bar(SFULL + b));
+      DKV_TR(14, nq);
       ++nq;
     };
 #pragma unroll 1
@@ -1265,6 +1267,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         mma_ts(tmem + kColO, tmem + p_col + 8 * kk, sdesc_sw128(vbase + 4096 * kk, 1024, 2048),
                (np > 0 || kk > 0) ? 1u : 0u);
       mma_commit(bar(VEMPTY + bb));
+      DKV_TR(13, np);
       ++np;
     }
     // drain: every MMA issued above completes before TMEM is released

@@ -9,9 +9,11 @@ One attention call on a cache of the workload's shape (seeded synthetic
 inputs), then one line per tile with the cycles since the CTA started of:
 the loader issuing the tile's copies (load), the K producer starting and
 ending the tile (k_beg, k_end), the V producer getting its buffer, starting
-and ending (v_wt, v_beg, v_end), the QK MMAs issued (qk), the softmax
+and ending (v_wt, v_beg, v_end), the QK MMAs' issue starting and ending
+(qk, qk_end), the softmax
 holding the scores (sm_beg), after its first pass / vote (sm_mid), P
-written (p_out), the PV MMAs issued (pv); and the steady-state period (pv
+written (p_out), the PV MMAs' issue starting and ending (pv, pv_end); and
+the steady-state period (pv
 issue to pv issue over the last two thirds of the tiles).  The stamps cost
 a few instructions in CTA 0 only; times of a trace-build call are not
 benchmark figures."""
@@ -27,7 +29,8 @@ sys.path.insert(0, ROOT)
 import numpy as np  # noqa: E402
 
 EVENTS = [(0, "load"), (1, "k_beg"), (2, "k_end"), (11, "v_wt"), (3, "v_beg"), (4, "v_end"),
-          (5, "qk"), (6, "sm_beg"), (12, "sm_mid"), (7, "p_out"), (8, "pv")]
+          (5, "qk"), (14, "qk_end"), (6, "sm_beg"), (12, "sm_mid"), (7, "p_out"), (8, "pv"),
+          (13, "pv_end")]
 
 
 def trace(workload="batch32", kernel=2, B=0, L=0, splits=1):
