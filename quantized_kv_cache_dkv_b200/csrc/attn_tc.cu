@@ -76,36 +76,66 @@ constexpr int kThreads = kWarps * 32;
 constexpr int kMmaWarp = 25;
 constexpr int kLoadWarp = 26;
 constexpr int kStages = 3;  // ring of packed tiles
-constexpr int kStagedProt = 8;  // protected K rows staged per tile (more: read from global)
 constexpr uint32_t kTileBytes = 128 * 128 * 2;
-constexpr uint32_t kColO = 0, kColS0 = 128, kColS1 = 256, kColQ = 384, kTmemCols = 512;
+// TMEM columns: O, two score buffers, two P buffers (fp16 pairs).  A score
+// buffer is free for the next QK once the softmax has read it, before its P
+// is written or multiplied.
+constexpr uint32_t kColO = 0, kColS0 = 128, kColS1 = 256, kColP0 = 384, kColP1 = 448,
+                   kTmemCols = 512;
 
 // instruction descriptor: D f32, A f16 (K-major), B f16 (MN-major), M = N = 128
 constexpr uint32_t kIdesc = (1u << 4) | (0u << 7) | (0u << 10) | (0u << 15) | (1u << 16) |
                             ((128u >> 3) << 17) | ((128u >> 4) << 24);
 
+// One ring stage of a tile's packed data, sized for the code widths (byte
+// offsets, all multiples of 16): packed K codes (128 tokens x 128 channels x
+// KB bits), K (scale, zero) pairs (at most 4 groups x 128 channels), the
+// side-table slice of the tile's K groups (header {entries n, first entry
+// g0, index base of the staged positions}, positions as an aligned superset,
+// the bf16 K rows of the first kProt entries; later ones are read from
+// global memory), packed V codes, V (scale, zero) pairs (128 tokens x at
+// most 4 groups).
+template <int KB, int VB>
+struct Stage {
+  static constexpr uint32_t kCodesK = KB < 16 ? 2048u * KB : 0u;
+  static constexpr uint32_t kCodesV = VB < 16 ? 2048u * VB : 0u;
+  static constexpr int kProt = KB >= 16 ? 0 : (KB == 4 && VB == 4 ? 3 : 8);
+  static constexpr uint32_t kRKc = 0, kRKsz = kCodesK, kRHdr = kRKsz + (KB < 16 ? 2048u : 0u),
+                            kRPos = kRHdr + 16, kRPk = kRPos + 128, kRVc = kRPk + 256u * kProt,
+                            kRVsz = kRVc + kCodesV, kBytes = kRVsz + (VB < 16 ? 2048u : 0u);
+};
+constexpr uint32_t kMaxStageBytes = Stage<4, 4>::kBytes > Stage<2, 4>::kBytes
+                                        ? (Stage<4, 4>::kBytes > Stage<4, 2>::kBytes ? Stage<4, 4>::kBytes
+                                                                                      : Stage<4, 2>::kBytes)
+                                        : Stage<2, 4>::kBytes;
+static_assert(Stage<2, 2>::kBytes <= kMaxStageBytes && Stage<2, 16>::kBytes <= kMaxStageBytes &&
+                  Stage<4, 16>::kBytes <= kMaxStageBytes && Stage<16, 4>::kBytes <= kMaxStageBytes,
+              "largest ring stage");
+
 struct Smem {
-  // offsets into the 1024-byte aligned dynamic shared memory
+  // offsets into the 1024-byte aligned dynamic shared memory: the two K and
+  // the two V tile buffers, Q (the A operand of QK: [128 rows][128
+  // channels] fp16, K-major with the 128-byte swizzle, as two halves of 64
+  // channels), then the ring
   static constexpr uint32_t kK0 = 0, kK1 = kTileBytes, kV0 = 2 * kTileBytes, kV1 = 3 * kTileBytes;
-  // one ring stage: packed K codes (<= 8 KB: 128 tokens x 128 channels x 4 bit),
-  // K (scale, zero) (<= 2 KB), packed V codes (<= 8 KB), V (scale, zero) (<= 2 KB)
-  static constexpr uint32_t kRKc = 0, kRKsz = 8192, kRVc = 10240, kRVsz = 18432;
-  // side-table slice of the tile's K groups: header {entries n, first entry
-  // g0, index base of the staged positions}, positions (aligned superset),
-  // and the bf16 K rows of the first kStagedProt entries
-  static constexpr uint32_t kRHdr = 20480, kRPos = 20496, kRPk = 20624;
-  static constexpr uint32_t kStageBytes = kRPk + kStagedProt * 256;  // 22672
-  static constexpr uint32_t kRing = 4 * kTileBytes;
-  static constexpr uint32_t kBar = kRing + kStages * kStageBytes;  // 32 mbarriers
+  static constexpr uint32_t kQ = 4 * kTileBytes;
+  static constexpr uint32_t kRing = kQ + kTileBytes;
+};
+template <int KB, int VB>
+struct SmemTail {
+  static constexpr uint32_t kBar = Smem::kRing + kStages * Stage<KB, VB>::kBytes;  // 32 mbarriers
   static constexpr uint32_t kRef = kBar + 32 * 8;   // [tile parity][128] reference max per row
   static constexpr uint32_t kLsum = kRef + 1024;    // [warpgroup][128] row sum, then its reference
   static constexpr uint32_t kMisc = kLsum + 2048;   // tmem base, abort flag, then the unit's lengths
   static constexpr uint32_t kBytes = kMisc + 32;
+  // plus 1024 bytes of alignment slack
+  static_assert(kBytes + 1024 <= 232448, "shared memory per block");
 };
 enum Bar {
-  KFULL = 0, KEMPTY = 2, VFULL = 4, VEMPTY = 6, SFULL = 8, PFULL = 10, QREADY = 12, DONE = 13,
-  RFULL = 14, REMPTY = 14 + kStages, RREADY = 14 + 2 * kStages, LSUM = RREADY + 2
+  KFULL = 0, VFULL = 4, VEMPTY = 6, SFULL = 8, PFULL = 10, QREADY = 12, DONE = 13,
+  RFULL = 14, REMPTY = 14 + kStages, RREADY = 14 + 2 * kStages, LSUM = RREADY + 2, SFREE = LSUM + 1
 };
+static_assert(SFREE + 2 <= 32, "barrier slots");
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -174,6 +204,15 @@ __device__ bool mbar_wait(uint32_t bar, uint32_t parity, const AttnArgs& a,
       }
     }
   }
+}
+
+// For the producer, loader and MMA loops: the common case -- the phase has
+// already completed -- costs one non-blocking test inline; otherwise the
+// bounded wait.
+__device__ __forceinline__ bool mbar_wait_fast(uint32_t bar, uint32_t parity, const AttnArgs& a,
+                                               volatile int* abort_flag) {
+  if (mbar_test(bar, parity)) return true;
+  return mbar_wait(bar, parity, a, abort_flag);
 }
 
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
@@ -324,6 +363,17 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       : "memory");
 }
 
+// D[tmem] (+)= A[smem] * B[smem]^T
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %3, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %4, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(accumulate), "r"(kIdesc)
+      : "memory");
+}
+
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                    bar)
@@ -390,7 +440,7 @@ struct KOffsets {
   }
 };
 
-template <int KB>
+template <int KB, int VB>
 __device__ __noinline__ void fill_k_general(const AttnArgs& a, const UnitLen ul, int u, int64_t tile_start,
                                             uint8_t* kt, const uint8_t* rs, int c, int qh);
 
@@ -398,10 +448,11 @@ __device__ __noinline__ void fill_k_general(const AttnArgs& a, const UnitLen ul,
 // is inline; tiles that reach the bf16 tail or the active block take the
 // out-of-line general path (at most two per call), which keeps the hot loop's
 // code small.
-template <int KB>
+template <int KB, int VB>
 __device__ __forceinline__ void fill_k_tile(const AttnArgs& a, const UnitLen ul, int u, int64_t tile_start,
                                             uint8_t* kt, const uint8_t* rs, int c, int qh,
                                             const KOffsets& ko) {
+  using ST = Stage<KB, VB>;
   const CacheView& cv = a.c;
   const int d = kHeadDim;
   if constexpr (KB < 16) {
@@ -411,9 +462,9 @@ __device__ __forceinline__ void fill_k_tile(const AttnArgs& a, const UnitLen ul,
       using W = typename std::conditional<KB == 4, uint4, uint2>::type;
 #pragma unroll 1
       for (int qi = 0; qi < 2; ++qi) {
-        const W w = *reinterpret_cast<const W*>(reinterpret_cast<const uint32_t*>(rs + Smem::kRKc) +
+        const W w = *reinterpret_cast<const W*>(reinterpret_cast<const uint32_t*>(rs + ST::kRKc) +
                                                 (qi ? ko.w[1] : ko.w[0]));
-        const __half2 sz = reinterpret_cast<const __half2*>(rs + Smem::kRKsz)[qi ? ko.z[1] : ko.z[0]];
+        const __half2 sz = reinterpret_cast<const __half2*>(rs + ST::kRKsz)[qi ? ko.z[1] : ko.z[0]];
         const __half2 s2 = __half2half2(__low2half(sz));
         const __half2 z2 = __half2half2(__high2half(sz));
         uint4 out[4];  // tokens in kpos order
@@ -432,36 +483,40 @@ __device__ __forceinline__ void fill_k_tile(const AttnArgs& a, const UnitLen ul,
         for (int i = 0; i < 4; ++i) *reinterpret_cast<uint4*>(dst + ko.o[i]) = out[i];
       }
       // protected rows of this thread's two chunks
-      const int* hdr = reinterpret_cast<const int*>(rs + Smem::kRHdr);
+      const int* hdr = reinterpret_cast<const int*>(rs + ST::kRHdr);
       const int n = hdr[0], g0 = hdr[1], pbase = hdr[2];
-      const int* rpos = reinterpret_cast<const int*>(rs + Smem::kRPos);
-      const uint16_t* rpk = reinterpret_cast<const uint16_t*>(rs + Smem::kRPk);
-#pragma unroll 1
-      for (int i = 0; i < n; ++i) {
-        if (!DKV_IN_BOUNDS(i < kStagedProt ? g0 + i - pbase >= 0 && g0 + i - pbase < 32
-                                           : g0 + i < cv.P, cv.status))
-          break;
-        const int pos = i < kStagedProt ? rpos[g0 + i - pbase]
-                                        : __ldg(cv.prot_pos + size_t(u) * cv.P + g0 + i);
+      const int* rpos = reinterpret_cast<const int*>(rs + ST::kRPos);
+      const uint16_t* rpk = reinterpret_cast<const uint16_t*>(rs + ST::kRPk);
+      auto put = [&](int pos, uint16_t kv) {
         const int t = int(pos - tile_start);
-        if (!DKV_IN_BOUNDS(t >= 0 && t < TT, cv.status)) continue;
-        if ((t >> 6) != qh) continue;
-        const uint16_t kv = i < kStagedProt
-                                ? rpk[i * d + c]
-                                : __ldg(cv.prot_k + (size_t(u) * cv.P + g0 + i) * d + c);
+        if (!DKV_IN_BOUNDS(t >= 0 && t < TT, cv.status)) return;
+        if ((t >> 6) != qh) return;
         const int p = kpos<KB>(t);
         __half* dst = reinterpret_cast<__half*>(kt + kt_off(c, p & ~7)) + (p & 7);
         *dst = bf16_to_half(kv);
+      };
+      const int ns = n < ST::kProt ? n : ST::kProt;
+#pragma unroll 1
+      for (int i = 0; i < ns; ++i) {  // staged entries
+        if (!DKV_IN_BOUNDS(g0 + i - pbase >= 0 && g0 + i - pbase < 32, cv.status)) break;
+        put(rpos[g0 + i - pbase], rpk[i * d + c]);
+      }
+#pragma unroll 1
+      for (int i = ns; i < n; ++i) {  // the rest from global memory
+        if (!DKV_IN_BOUNDS(g0 + i < cv.P, cv.status)) break;
+        put(__ldg(cv.prot_pos + size_t(u) * cv.P + g0 + i),
+            __ldg(cv.prot_k + (size_t(u) * cv.P + g0 + i) * d + c));
       }
       return;
     }
   }
-  fill_k_general<KB>(a, ul, u, tile_start, kt, rs, c, qh);
+  fill_k_general<KB, VB>(a, ul, u, tile_start, kt, rs, c, qh);
 }
 
-template <int KB>
+template <int KB, int VB>
 __device__ __noinline__ void fill_k_general(const AttnArgs& a, const UnitLen ul, int u, int64_t tile_start,
                                             uint8_t* kt, const uint8_t* rs, int c, int qh) {
+  using ST = Stage<KB, VB>;
   const CacheView& cv = a.c;
   const int d = kHeadDim;
 #pragma unroll 1
@@ -482,9 +537,9 @@ __device__ __noinline__ void fill_k_general(const AttnArgs& a, const UnitLen ul,
       if constexpr (KB < 16) {
         const int gi = (32 * q) / cv.GK;  // group within the tile
         const int o = (32 * q) % cv.GK;
-        const uint32_t* kc = reinterpret_cast<const uint32_t*>(rs + Smem::kRKc) +
+        const uint32_t* kc = reinterpret_cast<const uint32_t*>(rs + ST::kRKc) +
                              (gi * d + c) * cv.kw + o * KB / 32;
-        const __half2 sz = reinterpret_cast<const __half2*>(rs + Smem::kRKsz)[gi * d + c];
+        const __half2 sz = reinterpret_cast<const __half2*>(rs + ST::kRKsz)[gi * d + c];
         const __half2 s2 = __half2half2(__low2half(sz));
         const __half2 z2 = __half2half2(__high2half(sz));
         if constexpr (KB == 4) {
@@ -519,20 +574,20 @@ __device__ __noinline__ void fill_k_general(const AttnArgs& a, const UnitLen ul,
     if constexpr (KB < 16) {
       if (codes) {
         // protected rows of this chunk: their bf16 K from the staged side-table
-        // slice (entries past kStagedProt from global memory)
-        const int* hdr = reinterpret_cast<const int*>(rs + Smem::kRHdr);
+        // slice (entries past the staged ones from global memory)
+        const int* hdr = reinterpret_cast<const int*>(rs + ST::kRHdr);
         const int n = hdr[0], g0 = hdr[1], pbase = hdr[2];
-        const int* rpos = reinterpret_cast<const int*>(rs + Smem::kRPos);
-        const uint16_t* rpk = reinterpret_cast<const uint16_t*>(rs + Smem::kRPk);
+        const int* rpos = reinterpret_cast<const int*>(rs + ST::kRPos);
+        const uint16_t* rpk = reinterpret_cast<const uint16_t*>(rs + ST::kRPk);
         for (int i = 0; i < n; ++i) {
-          if (!DKV_IN_BOUNDS(i < kStagedProt ? g0 + i - pbase >= 0 && g0 + i - pbase < 32
+          if (!DKV_IN_BOUNDS(i < ST::kProt ? g0 + i - pbase >= 0 && g0 + i - pbase < 32
                                              : g0 + i < cv.P, cv.status))
             break;
-          const int pos = i < kStagedProt ? rpos[g0 + i - pbase]
+          const int pos = i < ST::kProt ? rpos[g0 + i - pbase]
                                           : __ldg(cv.prot_pos + size_t(u) * cv.P + g0 + i);
           if (pos >= pos0 && pos < pos0 + 32) {
             const int t = 32 * q + int(pos - pos0);
-            const uint16_t kv = i < kStagedProt
+            const uint16_t kv = i < ST::kProt
                                     ? rpk[i * d + c]
                                     : __ldg(cv.prot_k + (size_t(u) * cv.P + g0 + i) * d + c);
             __half* dst = reinterpret_cast<__half*>(kt + kt_off(c, t & ~7)) + (t & 7);
@@ -569,7 +624,7 @@ struct VOffsets {
   }
 };
 
-template <int VB>
+template <int KB, int VB>
 __device__ __noinline__ void fill_v_general(const AttnArgs& a, const UnitLen ul, int u, int64_t tile_start,
                                             uint8_t* vt, const uint8_t* rs, int tid, int perm_kb);
 
@@ -579,6 +634,7 @@ template <int KB, int VB, bool SINK>
 __device__ __forceinline__ void fill_v_tile(const AttnArgs& a, const UnitLen ul, int u, int64_t tile_start,
                                             uint8_t* vt, const uint8_t* rs, int tid,
                                             const VOffsets<KB>& vo) {
+  using ST = Stage<KB, VB>;
   const CacheView& cv = a.c;
   const bool k_whole = KB < 16 && tile_start + TT <= ul.Lq;
   if constexpr (VB < 16) {
@@ -591,9 +647,9 @@ __device__ __forceinline__ void fill_v_tile(const AttnArgs& a, const UnitLen ul,
       const bool rot = (tid & 2) != 0;
 #pragma unroll 1
       for (int r = 0; r < 2; ++r) {
-        W x = *reinterpret_cast<const W*>(reinterpret_cast<const uint32_t*>(rs + Smem::kRVc) +
+        W x = *reinterpret_cast<const W*>(reinterpret_cast<const uint32_t*>(rs + ST::kRVc) +
                                           (r ? vo.w[1] : vo.w[0]));
-        const __half2 sz = reinterpret_cast<const __half2*>(rs + Smem::kRVsz)[r ? vo.z[1] : vo.z[0]];
+        const __half2 sz = reinterpret_cast<const __half2*>(rs + ST::kRVsz)[r ? vo.z[1] : vo.z[0]];
         const __half2 s2 = __half2half2(__low2half(sz));
         const __half2 z2 = __half2half2(__high2half(sz));
         uint4 out[4];  // channels in kpos<VB> order
@@ -615,12 +671,13 @@ __device__ __forceinline__ void fill_v_tile(const AttnArgs& a, const UnitLen ul,
       return;
     }
   }
-  fill_v_general<VB>(a, ul, u, tile_start, vt, rs, tid, k_whole ? KB : 16);
+  fill_v_general<KB, VB>(a, ul, u, tile_start, vt, rs, tid, k_whole ? KB : 16);
 }
 
-template <int VB>
+template <int KB, int VB>
 __device__ __noinline__ void fill_v_general(const AttnArgs& a, const UnitLen ul, int u, int64_t tile_start,
                                             uint8_t* vt, const uint8_t* rs, int tid, int perm_kb) {
+  using ST = Stage<KB, VB>;  // KB: the ring stage's layout (the row order is perm_kb)
   const CacheView& cv = a.c;
   const int d = kHeadDim;
 #pragma unroll 1
@@ -649,10 +706,10 @@ __device__ __noinline__ void fill_v_general(const AttnArgs& a, const UnitLen ul,
     if (codes) {
       if constexpr (VB < 16) {
         const __half2 sz =
-            reinterpret_cast<const __half2*>(rs + Smem::kRVsz)[t * cv.vgroups + (qq * 32) / cv.GV];
+            reinterpret_cast<const __half2*>(rs + ST::kRVsz)[t * cv.vgroups + (qq * 32) / cv.GV];
         const __half2 s2 = __half2half2(__low2half(sz));
         const __half2 z2 = __half2half2(__high2half(sz));
-        const uint32_t* vc = reinterpret_cast<const uint32_t*>(rs + Smem::kRVc) + t * cv.vw;
+        const uint32_t* vc = reinterpret_cast<const uint32_t*>(rs + ST::kRVc) + t * cv.vw;
         if constexpr (VB == 4) {
           uint4 w = *reinterpret_cast<const uint4*>(vc + qq * 4);
           if (rot) w = make_uint4(w.z, w.w, w.x, w.y);
@@ -714,17 +771,18 @@ __device__ __noinline__ void fill_v_general(const AttnArgs& a, const UnitLen ul,
 struct Pipe {
   uint8_t* sm;
   uint32_t sm_base;
-  uint32_t ring;              // offset of ring stage 0 (stages kStageBytes apart)
+  uint32_t ring;              // offset of ring stage 0 (stages Stage<KB, VB>::kBytes apart)
   uint32_t k_buf0, v_buf0;    // offsets of K / V tile buffer 0 (buffer 1 at + kTileBytes)
   uint32_t kfull, kempty, vfull, vempty, rfull, rempty;  // barrier addresses
 };
 
 // K producer thread pt (0..255): channel pt % 128, token chunks 2 qh, 2 qh + 1
 // of every tile, qh = pt / 128.
-template <int KB, int STAGES>
+template <int KB, int VB, int STAGES>
 __device__ __forceinline__ void k_producer_loop(const AttnArgs& a, const UnitLen* uls, int u,
                                                 int64_t t_begin, int nt, const Pipe& p,
                                                 volatile int* abort_flag, int pt) {
+  using ST = Stage<KB, VB>;
   const CacheView& cv = a.c;
   const int c = pt & 127;   // channel
   const int qh = pt >> 7;   // chunks 2qh, 2qh+1 of each tile
@@ -732,11 +790,11 @@ __device__ __forceinline__ void k_producer_loop(const AttnArgs& a, const UnitLen
 #pragma unroll 1
   for (int j = 0; j < nt; ++j) {
     const int b = j & 1, st = j % STAGES;
-    if (!mbar_wait(p.kempty + 8u * b, ((j >> 1) & 1) ^ 1, a, abort_flag)) break;
-    if (!mbar_wait(p.rfull + 8u * st, (j / STAGES) & 1, a, abort_flag)) break;
+    if (!mbar_wait_fast(p.kempty + 8u * b, ((j >> 1) & 1) ^ 1, a, abort_flag)) break;
+    if (!mbar_wait_fast(p.rfull + 8u * st, (j / STAGES) & 1, a, abort_flag)) break;
     if (pt == 0) DKV_TR(1, j);
-    fill_k_tile<KB>(a, *uls, u, (t_begin + j) * TT, p.sm + p.k_buf0 + b * kTileBytes,
-                    p.sm + p.ring + st * Smem::kStageBytes, c, qh, ko);
+    fill_k_tile<KB, VB>(a, *uls, u, (t_begin + j) * TT, p.sm + p.k_buf0 + b * kTileBytes,
+                    p.sm + p.ring + st * ST::kBytes, c, qh, ko);
     fence_async_smem();
     if (pt == 0) DKV_TR(2, j);
     mbar_arrive(p.kfull + 8u * b);
@@ -749,17 +807,18 @@ template <int KB, int VB, bool SINK, int STAGES>
 __device__ __forceinline__ void v_producer_loop(const AttnArgs& a, const UnitLen* uls, int u,
                                                 int64_t t_begin, int nt, const Pipe& p,
                                                 volatile int* abort_flag, int pt) {
+  using ST = Stage<KB, VB>;
   const CacheView& cv = a.c;
   const VOffsets<KB> vo(pt, cv.vw, cv.vgroups, cv.GV, VB < 16 ? VB : 16);
 #pragma unroll 1
   for (int j = 0; j < nt; ++j) {
     const int b = j & 1, st = j % STAGES;
-    if (!mbar_wait(p.vempty + 8u * b, ((j >> 1) & 1) ^ 1, a, abort_flag)) break;
+    if (!mbar_wait_fast(p.vempty + 8u * b, ((j >> 1) & 1) ^ 1, a, abort_flag)) break;
     if (pt == 0) DKV_TR(11, j);
-    if (!mbar_wait(p.rfull + 8u * st, (j / STAGES) & 1, a, abort_flag)) break;
+    if (!mbar_wait_fast(p.rfull + 8u * st, (j / STAGES) & 1, a, abort_flag)) break;
     if (pt == 0) DKV_TR(3, j);
     fill_v_tile<KB, VB, SINK>(a, *uls, u, (t_begin + j) * TT, p.sm + p.v_buf0 + b * kTileBytes,
-                              p.sm + p.ring + st * Smem::kStageBytes, pt, vo);
+                              p.sm + p.ring + st * ST::kBytes, pt, vo);
     fence_async_smem();
     if (pt == 0) DKV_TR(4, j);
     mbar_arrive(p.vfull + 8u * b);
@@ -775,6 +834,7 @@ template <int KB, int VB, int STAGES>
 __device__ __forceinline__ void loader_loop(const AttnArgs& a, const UnitLen* uls, int u,
                                             int64_t t_begin, int nt, const Pipe& p,
                                             volatile int* abort_flag, int lane) {
+  using ST = Stage<KB, VB>;
   const CacheView& cv = a.c;
   const int gks = KB < 16 ? __ffs(cv.GK) - 1 : 0;
   const int Lq = uls->Lq, Lc = uls->L, t0 = int(t_begin) * TT;
@@ -800,7 +860,7 @@ __device__ __forceinline__ void loader_loop(const AttnArgs& a, const UnitLen* ul
     const int g1 = __shfl_sync(0xffffffffu, pf1, j & 31);
     const int st = j % STAGES;
     const uint32_t rfull = p.rfull + 8u * st;
-    if (!__all_sync(0xffffffffu, mbar_wait(p.rempty + 8u * st, ((j / STAGES) & 1) ^ 1, a, abort_flag)))
+    if (!__all_sync(0xffffffffu, mbar_wait_fast(p.rempty + 8u * st, ((j / STAGES) & 1) ^ 1, a, abort_flag)))
       break;
     if (lane == 0) DKV_TR(0, j);
     ++issued;
@@ -814,7 +874,7 @@ __device__ __forceinline__ void loader_loop(const AttnArgs& a, const UnitLen* ul
 #endif
     if (lane == 0) {
       const int ts = t0 + j * TT;
-      const uint32_t dst = p.sm_base + p.ring + st * Smem::kStageBytes;
+      const uint32_t dst = p.sm_base + p.ring + st * ST::kBytes;
       uint32_t kc_b = 0, ksz_b = 0, vc_b = 0, vsz_b = 0, pos_b = 0, pk_b = 0;
       int g_lo = 0, pidx0 = 0;  // pidx0: first staged position, relative to the unit
       const int n = g1 - g0;
@@ -825,7 +885,7 @@ __device__ __forceinline__ void loader_loop(const AttnArgs& a, const UnitLen* ul
         kc_b = ng * kHeadDim * uint32_t(cv.kw) * 4u;
         ksz_b = ng * kHeadDim * 4u;
         if (n > 0) {
-          const int nst = n < kStagedProt ? n : kStagedProt;
+          const int nst = n < ST::kProt ? n : ST::kProt;
           // 16-byte aligned superset of the staged positions (the unit's
           // slice starts at u * P entries)
           const int64_t e0 = int64_t(u) * cv.P + g0;
@@ -847,7 +907,7 @@ __device__ __forceinline__ void loader_loop(const AttnArgs& a, const UnitLen* ul
         // counts stay consistent with the expect_tx below
         const size_t U = size_t(cv.U), P = size_t(cv.P), e = size_t(u) * P;
         if (kc_b && !DKV_IN_BOUNDS(
-                        kc_b <= Smem::kRKsz - Smem::kRKc && ksz_b <= Smem::kRVc - Smem::kRKsz &&
+                        kc_b <= ST::kRKsz - ST::kRKc && ksz_b <= ST::kRHdr - ST::kRKsz &&
                         (ug * kHeadDim * cv.kw) * 4 + kc_b <= U * cv.nG * kHeadDim * cv.kw * 4 &&
                         (ug * kHeadDim) * 4 + ksz_b <= U * cv.nG * kHeadDim * 4, cv.status))
           kc_b = ksz_b = pos_b = pk_b = 0;
@@ -855,36 +915,36 @@ __device__ __forceinline__ void loader_loop(const AttnArgs& a, const UnitLen* ul
         // entries before and after the unit's slice, inside the arena)
         if (pos_b && !DKV_IN_BOUNDS(
                          g0 >= 0 && int64_t(e) + pidx0 >= 0 &&
-                         pos_b <= Smem::kRPk - Smem::kRPos &&
-                         pk_b <= Smem::kStageBytes - Smem::kRPk &&
+                         pos_b <= ST::kRPk - ST::kRPos &&
+                         pk_b <= ST::kRVc - ST::kRPk &&
                          (e + size_t(pidx0)) * 4 + pos_b <= (U * P + 3) * 4 &&
                          (e + size_t(g0)) * kHeadDim * 2 + pk_b <= U * P * kHeadDim * 2, cv.status))
           pos_b = pk_b = 0;
         const size_t ut = size_t(u) * size_t(cv.cap) + size_t(ts);
         if (vc_b && !DKV_IN_BOUNDS(
-                        vc_b <= Smem::kRVsz - Smem::kRVc && vsz_b <= Smem::kRHdr - Smem::kRVsz &&
+                        vc_b <= ST::kRVsz - ST::kRVc && vsz_b <= ST::kBytes - ST::kRVsz &&
                         ut * cv.vw * 4 + vc_b <= U * size_t(cv.cap) * cv.vw * 4 &&
                         ut * cv.vgroups * 4 + vsz_b <= U * size_t(cv.cap) * cv.vgroups * 4, cv.status))
           vc_b = vsz_b = 0;
       }
-      int* hdr = reinterpret_cast<int*>(p.sm + p.ring + st * Smem::kStageBytes + Smem::kRHdr);
+      int* hdr = reinterpret_cast<int*>(p.sm + p.ring + st * ST::kBytes + ST::kRHdr);
       hdr[0] = pos_b ? n : 0;  // pos_b is set exactly when the tile has protected rows
       hdr[1] = g0;
       hdr[2] = pidx0;
       mbar_arrive_expect_tx(rfull, kc_b + ksz_b + vc_b + vsz_b + pos_b + pk_b);
       if (kc_b) {
-        bulk_g2s(dst + Smem::kRKc, cv.k_codes + ug * kHeadDim * cv.kw, kc_b, rfull);
-        bulk_g2s(dst + Smem::kRKsz, cv.k_sz + ug * kHeadDim, ksz_b, rfull);
+        bulk_g2s(dst + ST::kRKc, cv.k_codes + ug * kHeadDim * cv.kw, kc_b, rfull);
+        bulk_g2s(dst + ST::kRKsz, cv.k_sz + ug * kHeadDim, ksz_b, rfull);
       }
       if (pos_b) {
         const size_t e = size_t(u) * size_t(cv.P);
-        bulk_g2s(dst + Smem::kRPos, cv.prot_pos + e + size_t(pidx0), pos_b, rfull);
-        bulk_g2s(dst + Smem::kRPk, cv.prot_k + (e + size_t(g0)) * kHeadDim, pk_b, rfull);
+        bulk_g2s(dst + ST::kRPos, cv.prot_pos + e + size_t(pidx0), pos_b, rfull);
+        bulk_g2s(dst + ST::kRPk, cv.prot_k + (e + size_t(g0)) * kHeadDim, pk_b, rfull);
       }
       if (vc_b) {
         const size_t ut = size_t(u) * size_t(cv.cap) + size_t(ts);
-        bulk_g2s(dst + Smem::kRVc, cv.v_codes + ut * cv.vw, vc_b, rfull);
-        bulk_g2s(dst + Smem::kRVsz, cv.v_sz + ut * cv.vgroups, vsz_b, rfull);
+        bulk_g2s(dst + ST::kRVc, cv.v_codes + ut * cv.vw, vc_b, rfull);
+        bulk_g2s(dst + ST::kRVsz, cv.v_sz + ut * cv.vgroups, vsz_b, rfull);
       }
     }
     __syncwarp();
@@ -903,10 +963,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~uintptr_t(1023));
   const uint32_t sm_base = smem_u32(sm);
-  const uint32_t bar0 = sm_base + Smem::kBar;
+  const uint32_t bar0 = sm_base + SmemTail<KB, VB>::kBar;
   auto bar = [&](int i) { return bar0 + 8u * uint32_t(i); };
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + Smem::kMisc);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + Smem::kMisc + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SmemTail<KB, VB>::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + SmemTail<KB, VB>::kMisc + 4);
 
   const CacheView& cv = a.c;
   // CTA = (unit, split, row block): a query group of more than 128 rows is
@@ -940,17 +1000,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 
   // the unit's lengths live in shared memory from here on: read where used,
   // not held in registers through the role loops
-  const UnitLen* uls = reinterpret_cast<const UnitLen*>(sm + Smem::kMisc + 16);
-  const Pipe pipe{sm, sm_base, Smem::kRing, Smem::kK0, Smem::kV0, bar(KFULL), bar(KEMPTY),
+  const UnitLen* uls = reinterpret_cast<const UnitLen*>(sm + SmemTail<KB, VB>::kMisc + 16);
+  const Pipe pipe{sm, sm_base, Smem::kRing, Smem::kK0, Smem::kV0, bar(KFULL), bar(SFULL),
                   bar(VFULL), bar(VEMPTY), bar(RFULL), bar(REMPTY)};
   if (threadIdx.x == 0) {
-    *reinterpret_cast<UnitLen*>(sm + Smem::kMisc + 16) = ul;
+    *reinterpret_cast<UnitLen*>(sm + SmemTail<KB, VB>::kMisc + 16) = ul;
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar(KFULL + b), 256);
-      mbar_init(bar(KEMPTY + b), 1);
       mbar_init(bar(VFULL + b), 256);
       mbar_init(bar(VEMPTY + b), 1);
-      mbar_init(bar(SFULL + b), 1);
+      mbar_init(bar(SFULL + b), 1);  // also tells the K producers that K_b is free
+      mbar_init(bar(SFREE + b), 128);
       mbar_init(bar(PFULL + b), 128);
       mbar_init(bar(RREADY + b), 128);
     }
@@ -989,8 +1049,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     const bool warp_rows = (warp & 3) * 32 < rpb;
     const int r = rb * rpb + lr;        // query row of the unit
     const uint32_t lane_base = tmem + (uint32_t((warp & 3) * 32) << 16);
-    float* ref = reinterpret_cast<float*>(sm + Smem::kRef);    // [tile parity][row]
-    float* lsum = reinterpret_cast<float*>(sm + Smem::kLsum);  // [warpgroup][row], then refs
+    float* ref = reinterpret_cast<float*>(sm + SmemTail<KB, VB>::kRef);    // [tile parity][row]
+    float* lsum = reinterpret_cast<float*>(sm + SmemTail<KB, VB>::kLsum);  // [warpgroup][row], then refs
     // a negative scale is folded into Q (an exact fp16 sign flip), so scores
     // are always multiplied by sc > 0; scale 0 (uniform weights) uses 1e-30
     const bool qneg = a.scale_log2 < 0.f;
@@ -1009,9 +1069,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         qv[4 * i + 2] = y.z;
         qv[4 * i + 3] = y.w;
       }
-      tmem_st32(lane_base + kColQ + 32 * h, qv);
-      tmem_st_wait();
-      tc_fence_before();
+      // row lr, channels [64h, 64h + 64): the 16-byte chunk c of the row at
+      // chunk c ^ (row mod 8) of its 128-byte line (K-major, 128-byte swizzle)
+      uint8_t* qh = sm + Smem::kQ + h * 16384 + lr * 128;
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<uint4*>(qh + ((c ^ (lr & 7)) << 4)) =
+            make_uint4(qv[4 * c], qv[4 * c + 1], qv[4 * c + 2], qv[4 * c + 3]);
+      fence_async_smem();
       mbar_arrive(bar(QREADY));
     }
     // Every tile j has one reference max per row, r_j (log2 units), non-
@@ -1024,8 +1089,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     bool ok = true;
 #pragma unroll 1
     for (int j = h; j < nt && ok; j += 2) {
-      const int b = h;  // S buffer, reference slot and barriers of this warpgroup's tiles
-      const uint32_t s_col = b ? kColS1 : kColS0;
+      const int b = h;  // S and P buffers, reference slot and barriers of this warpgroup's tiles
+      const uint32_t s_col = b ? kColS1 : kColS0, p_col = b ? kColP1 : kColP0;
       // tcgen05.ld/st are warp-collective: every branch around them is warp-uniform
       if (!__all_sync(0xffffffffu, mbar_wait(bar(SFULL + b), (j >> 1) & 1, a, abort_flag))) {
         ok = false;
@@ -1035,6 +1100,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       if ((threadIdx.x & 127) == 0) DKV_TR(6, j);
       if (!warp_rows) {
         mbar_arrive(bar(RREADY + b));
+        mbar_arrive(bar(SFREE + b));
         mbar_arrive(bar(PFULL + b));
         continue;
       }
@@ -1081,8 +1147,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       mbar_arrive(bar(RREADY + b));
       l *= fast_exp2(r_w - r_j);  // 1 when unchanged, 0 on this warpgroup's first tile
       r_w = r_j;
-      // pass 2: P = 2^(s*sc - r_j) as fp16 pairs into columns [0, 64) of S_b;
-      // 16-column chunks, the load of chunk c+1 in flight while chunk c is computed
+      // pass 2: P = 2^(s*sc - r_j) as fp16 pairs into P_b, once PV(j-2) has
+      // read it (QK(j) is issued before PV(j-2)); 16-column chunks, the load
+      // of chunk c+1 in flight while chunk c is computed; S_b is released to
+      // QK(j+2) after its last load
+      if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(bar(VEMPTY + b), ((j - 2) >> 1) & 1, a,
+                                                        abort_flag))) {
+        ok = false;
+        break;
+      }
       const uint64_t sc2 = f2pack(sc, sc), nm2 = f2pack(-r_j, -r_j);
       uint64_t l2[2] = {0ull, 0ull};  // two packed pairs of partial row sums
       uint32_t va[16], vb[16];
@@ -1097,7 +1170,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           l2[i & 1] = fadd2(l2[i & 1], f2pack(p0, p1));
           pv[i] = pack_h2(p0, p1);
         }
-        tmem_st8(lane_base + s_col + 8 * c, pv);
+        tmem_st8(lane_base + p_col + 8 * c, pv);
       };
       const int n16 = 2 * n32;
       tmem_ld16(lane_base + s_col, va);
@@ -1107,7 +1180,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         tmem_ld16(lane_base + s_col + 16 * (c + 1), vb);
         chunk(va, c);
         tmem_ld_wait();
-        if (c + 2 < n16) tmem_ld16(lane_base + s_col + 16 * (c + 2), va);
+        if (c + 2 < n16) {
+          tmem_ld16(lane_base + s_col + 16 * (c + 2), va);
+        } else {
+          tc_fence_before();
+          mbar_arrive(bar(SFREE + b));
+        }
         chunk(vb, c + 1);
         if (c + 2 < n16) tmem_ld_wait();
       }
@@ -1206,7 +1284,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   } else if (warp < 24) {
     regs_dec<kRegProducer>();
     if (warp < 16)
-      k_producer_loop<KB, kStages>(a, uls, u, t_begin, nt, pipe, abort_flag, threadIdx.x - 256);
+      k_producer_loop<KB, VB, kStages>(a, uls, u, t_begin, nt, pipe, abort_flag, threadIdx.x - 256);
     else
       v_producer_loop<KB, VB, SINK, kStages>(a, uls, u, t_begin, nt, pipe, abort_flag,
                                              threadIdx.x - 512);
@@ -1218,57 +1296,78 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     // ------------------------------------------------------------ MMA issuer
     bool ok = mbar_wait(bar(QREADY), 0, a, abort_flag);
     tc_fence_after();
-    // QK(j) needs K_j (KFULL) and S_(j mod 2) free, i.e. PV(j-2) issued; PV(i)
-    // needs P_i (PFULL) and V_i (VFULL).  Every QK that is ready and allowed
-    // is issued at once; otherwise the lane sleeps (suspending mbarrier wait)
-    // on the barrier it needs next: P of the oldest un-issued PV, or K of the
-    // next QK when no PV is pending.  Barrier phases cannot run ahead: each
-    // next phase needs an MMA issued here first.
-    int nq = 0, np = 0;
-    auto issue_qk = [&]() {
-      DKV_TR(5, nq);
+    // A fixed order: QK(0), QK(1), then for each tile j QK(j+2) and PV(j).
+    // QK(j+2) needs K_(j+2) (KFULL) and S_(j mod 2) read out by the softmax
+    // of tile j (SFREE, before P_j is complete); PV(j) needs P_j (PFULL) and
+    // V_j (VFULL).  MMAs run in issue order, so when the softmax of tile j
+    // starts (QK(j) complete), PV(j-3) and every earlier PV are complete:
+    // its parity waits on VEMPTY for PV(j-1) and PV(j-2) cannot match an
+    // older phase.  The QK's commit on SFULL also frees its K buffer for the
+    // K producers.
+    // operand descriptors, computed once: a K-step adds a fixed offset to the
+    // start-address field (address / 16, 14 bits; shared memory stays below
+    // 256 KB, so the field never carries)
+    const uint64_t dq = sdesc_sw128(sm_base + Smem::kQ, 16, 1024);
+    const uint64_t dk0 = sdesc_sw128(sm_base + Smem::kK0, 1024, 2048);
+    const uint64_t dk1 = sdesc_sw128(sm_base + Smem::kK1, 1024, 2048);
+    const uint64_t dv0 = sdesc_sw128(sm_base + Smem::kV0, 1024, 2048);
+    const uint64_t dv1 = sdesc_sw128(sm_base + Smem::kV1, 1024, 2048);
+    auto issue_qk = [&](int q) {
+      DKV_TR(5, q);
       tc_fence_after();
-      const int b = nq & 1;
-      const uint32_t kbase = sm_base + (b ? Smem::kK1 : Smem::kK0);
-      const uint32_t s_col = b ? kColS1 : kColS0;
+      const int b = q & 1;
+      const uint64_t db = b ? dk1 : dk0;
+      const uint32_t d_s = tmem + (b ? kColS1 : kColS0);
+      // channels 16kk .. 16kk + 15: Q half kk / 4 (16 KB apart), 32 bytes into
+      // its 128-byte rows; K tile rows 16kk.. (4 KB per 16 channels)
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)
-        mma_ts(tmem + s_col, tmem + kColQ + 8 * kk, sdesc_sw128(kbase + 4096 * kk, 1024, 2048),
+        mma_ss(d_s, dq + uint64_t((kk >> 2) * 1024 + (kk & 3) * 2), db + uint64_t(256 * kk),
                kk > 0 ? 1u : 0u);
-      mma_commit(bar(KEMPTY + b));
       mma_commit(bar(SFULL + b));
-      DKV_TR(14, nq);
-      ++nq;
+      DKV_TR(14, q);
+    };
+    auto issue_pv = [&](int p) {
+      tc_fence_after();
+      DKV_TR(8, p);
+      const int bb = p & 1;
+      const uint64_t dv = bb ? dv1 : dv0;
+      const uint32_t a_p = tmem + (bb ? kColP1 : kColP0);
+      const int64_t pv_start = (t_begin + p) * TT;
+      const int n_tok = uls->n_tok;
+      const uint32_t acc0 = p > 0 ? 1u : 0u;
+      // tokens 16kk..16kk+15: packed P columns 8kk..8kk+7, V rows 16kk.. (4 KB)
+      if (n_tok - pv_start >= TT) {
+#pragma unroll
+        for (int kk = 0; kk < TT / 16; ++kk)
+          mma_ts(tmem + kColO, a_p + 8 * kk, dv + uint64_t(256 * kk), kk > 0 ? 1u : acc0);
+      } else {
+        const int nk = int(n_tok - pv_start) >> 4;  // the last tile stops at its last token
+#pragma unroll 1
+        for (int kk = 0; kk < nk; ++kk)
+          mma_ts(tmem + kColO, a_p + 8 * kk, dv + uint64_t(256 * kk), kk > 0 ? 1u : acc0);
+      }
+      mma_commit(bar(VEMPTY + bb));
+      DKV_TR(13, p);
     };
 #pragma unroll 1
-    while (ok && np < nt) {
-      while (nq < nt && nq <= np + 1 && mbar_test(bar(KFULL + (nq & 1)), (nq >> 1) & 1)) issue_qk();
-      if (np == nq) {
-        // nothing to multiply by P yet: wait for the next K tile
-        ok = mbar_wait(bar(KFULL + (nq & 1)), (nq >> 1) & 1, a, abort_flag);
-        if (ok) issue_qk();
-        continue;
-      }
-      const int bb = np & 1;
-      if (!mbar_wait(bar(PFULL + bb), (np >> 1) & 1, a, abort_flag) ||
-          !mbar_wait(bar(VFULL + bb), (np >> 1) & 1, a, abort_flag)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      DKV_TR(8, np);
-      const uint32_t vbase = sm_base + (bb ? Smem::kV1 : Smem::kV0);
-      const uint32_t p_col = bb ? kColS1 : kColS0;
-      const int64_t pv_start = (t_begin + np) * TT;
-      const int n_tok = uls->n_tok;
-      const int nk = n_tok - pv_start < TT ? int(n_tok - pv_start) >> 4 : TT / 16;
+    for (int q = 0; ok && q < 2 && q < nt; ++q) {
+      ok = mbar_wait_fast(bar(KFULL + q), 0, a, abort_flag);
+      if (ok) issue_qk(q);
+    }
 #pragma unroll 1
-      for (int kk = 0; kk < nk; ++kk)  // tokens 16kk..16kk+15: packed P columns 8kk..8kk+7
-        mma_ts(tmem + kColO, tmem + p_col + 8 * kk, sdesc_sw128(vbase + 4096 * kk, 1024, 2048),
-               (np > 0 || kk > 0) ? 1u : 0u);
-      mma_commit(bar(VEMPTY + bb));
-      DKV_TR(13, np);
-      ++np;
+    for (int j = 0; ok && j < nt; ++j) {
+      const int q = j + 2;
+      if (q < nt) {
+        ok = mbar_wait_fast(bar(SFREE + (q & 1)), (j >> 1) & 1, a, abort_flag) &&
+             mbar_wait_fast(bar(KFULL + (q & 1)), (q >> 1) & 1, a, abort_flag);
+        if (!ok) break;
+        issue_qk(q);
+      }
+      ok = mbar_wait_fast(bar(PFULL + (j & 1)), (j >> 1) & 1, a, abort_flag) &&
+           mbar_wait_fast(bar(VFULL + (j & 1)), (j >> 1) & 1, a, abort_flag);
+      if (!ok) break;
+      issue_pv(j);
     }
     // drain: every MMA issued above completes before TMEM is released
     mma_commit(bar(DONE));
@@ -1329,7 +1428,7 @@ struct Smem {
   static constexpr uint32_t kP = 4 * kTileBytes;                   // 2 P^T tiles [128 tokens][64 rows]
   static constexpr uint32_t kQ = kP + 2 * 128 * kN * 2;            // Q^T [128 channels][64 rows]
   static constexpr uint32_t kRing = kQ + 128 * kN * 2;
-  static constexpr uint32_t kBar = kRing + kStages * ::dkv::Smem::kStageBytes;  // 32 mbarriers
+  static constexpr uint32_t kBar = kRing + kStages * ::dkv::kMaxStageBytes;  // 32 mbarriers
   static constexpr uint32_t kFlag = kBar + 32 * 8;                 // [2][4] raise votes
   static constexpr uint32_t kRed = kFlag + 64;                     // [3][4 warps][32 rows] floats
   static constexpr uint32_t kMisc = kRed + 3 * 4 * kRows * 4;      // tmem, abort, lengths
@@ -1651,7 +1750,7 @@ __global__ void __launch_bounds__(tl::kThreads, 1) attn_tl_kernel(const __grid_c
   } else if (warp < 20) {
     regs_dec<tl::kRegProducer>();
     if (warp < 12)
-      k_producer_loop<KB, tl::kStages>(a, uls, u, t_begin, nt, pipe, abort_flag, threadIdx.x - 128);
+      k_producer_loop<KB, VB, tl::kStages>(a, uls, u, t_begin, nt, pipe, abort_flag, threadIdx.x - 128);
     else
       v_producer_loop<KB, VB, SINK, tl::kStages>(a, uls, u, t_begin, nt, pipe, abort_flag,
                                              threadIdx.x - 384);
@@ -1755,7 +1854,7 @@ cudaError_t launch_tl(const AttnArgs& a, cudaStream_t s) {
 template <int KB, int VB, bool SINK>
 cudaError_t launch_kvs(const AttnArgs& a, cudaStream_t s) {
   if (a.tc_layout == 1) return launch_tl<KB, VB, SINK>(a, s);
-  const size_t smem = Smem::kBytes + 1024;
+  const size_t smem = SmemTail<KB, VB>::kBytes + 1024;
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<KB, VB, SINK>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
