@@ -70,10 +70,10 @@ __device__ unsigned long long g_trace[16][64];
 constexpr int TT = kTcTile;              // tokens per tile
 constexpr int kWarps = 28;  // seven warpgroups; warps 26, 27 only complete the last one
 constexpr int kThreads = kWarps * 32;
-// The MMA lane and the loader sit on sub-partitions 1 and 2: with query
+// The MMA lane and the loader sit on sub-partitions 3 and 2: with query
 // groups of 32 rows all softmax work lands on sub-partition 0 (TMEM lanes
 // 0-31 belong to warps 0 and 4).
-constexpr int kMmaWarp = 25;
+constexpr int kMmaWarp = 27;  // sub-partition 3: the MMA issue rate follows its share of issue slots
 constexpr int kLoadWarp = 26;
 constexpr int kStages = 3;  // ring of packed tiles
 constexpr uint32_t kTileBytes = 128 * 128 * 2;
@@ -363,14 +363,62 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       : "memory");
 }
 
-// D[tmem] (+)= A[smem] * B[smem]^T
-__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                       uint32_t accumulate) {
+// Eight MMAs over K = 128 (eight K-steps of 16) into one accumulator, in one
+// asm block: between MMAs only the 32-bit start-address words of the
+// descriptors advance (shared-memory operands: address / 16, so a 32-byte
+// step within a 128-byte swizzled row is +2 and a 4 KB step +256), which keeps
+// the issuing thread's instruction count per MMA at three.  A from shared
+// memory, K-major over two 16 KB halves (steps +2, +2, +2, +1018 to the next
+// half, ...); B from shared memory with +256 per step.
+__device__ __forceinline__ void mma8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                        uint32_t accumulate) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %3, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %4, p;\n\t}" ::"r"(d_tmem),
+      "{\n\t.reg .pred p, t;\n\t.reg .b32 al, ah, bl, bh;\n\t.reg .b64 a, b;\n\t"
+      "setp.ne.b32 p, %3, 0;\n\tsetp.eq.b32 t, 0, 0;\n\t"
+      "mov.b64 {al, ah}, %1;\n\tmov.b64 {bl, bh}, %2;\n\t"
+      "mov.b64 a, {al, ah};\n\tmov.b64 b, {bl, bh};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %4, p;\n\t"
+      "add.u32 al, al, 2;\n\tadd.u32 bl, bl, 256;\n\tmov.b64 a, {al, ah};\n\tmov.b64 b, {bl, bh};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %4, t;\n\t"
+      "add.u32 al, al, 2;\n\tadd.u32 bl, bl, 256;\n\tmov.b64 a, {al, ah};\n\tmov.b64 b, {bl, bh};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %4, t;\n\t"
+      "add.u32 al, al, 2;\n\tadd.u32 bl, bl, 256;\n\tmov.b64 a, {al, ah};\n\tmov.b64 b, {bl, bh};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %4, t;\n\t"
+      "add.u32 al, al, 1018;\n\tadd.u32 bl, bl, 256;\n\tmov.b64 a, {al, ah};\n\tmov.b64 b, {bl, bh};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %4, t;\n\t"
+      "add.u32 al, al, 2;\n\tadd.u32 bl, bl, 256;\n\tmov.b64 a, {al, ah};\n\tmov.b64 b, {bl, bh};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %4, t;\n\t"
+      "add.u32 al, al, 2;\n\tadd.u32 bl, bl, 256;\n\tmov.b64 a, {al, ah};\n\tmov.b64 b, {bl, bh};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %4, t;\n\t"
+      "add.u32 al, al, 2;\n\tadd.u32 bl, bl, 256;\n\tmov.b64 a, {al, ah};\n\tmov.b64 b, {bl, bh};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %4, t;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(accumulate), "r"(kIdesc)
+      : "memory");
+}
+
+// The same with A in TMEM (eight columns per K-step: +8 to the TMEM address).
+__device__ __forceinline__ void mma8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                        uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, t;\n\t.reg .b32 a, bl, bh;\n\t.reg .b64 b;\n\t"
+      "setp.ne.b32 p, %3, 0;\n\tsetp.eq.b32 t, 0, 0;\n\t"
+      "mov.b32 a, %1;\n\tmov.b64 {bl, bh}, %2;\n\tmov.b64 b, {bl, bh};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, p;\n\t"
+      "add.u32 a, a, 8;\n\tadd.u32 bl, bl, 256;\n\tmov.b64 b, {bl, bh};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, t;\n\t"
+      "add.u32 a, a, 8;\n\tadd.u32 bl, bl, 256;\n\tmov.b64 b, {bl, bh};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, t;\n\t"
+      "add.u32 a, a, 8;\n\tadd.u32 bl, bl, 256;\n\tmov.b64 b, {bl, bh};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, t;\n\t"
+      "add.u32 a, a, 8;\n\tadd.u32 bl, bl, 256;\n\tmov.b64 b, {bl, bh};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, t;\n\t"
+      "add.u32 a, a, 8;\n\tadd.u32 bl, bl, 256;\n\tmov.b64 b, {bl, bh};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, t;\n\t"
+      "add.u32 a, a, 8;\n\tadd.u32 bl, bl, 256;\n\tmov.b64 b, {bl, bh};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, t;\n\t"
+      "add.u32 a, a, 8;\n\tadd.u32 bl, bl, 256;\n\tmov.b64 b, {bl, bh};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %4, t;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(accumulate), "r"(kIdesc)
       : "memory");
 }
 
@@ -1320,10 +1368,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       const uint32_t d_s = tmem + (b ? kColS1 : kColS0);
       // channels 16kk .. 16kk + 15: Q half kk / 4 (16 KB apart), 32 bytes into
       // its 128-byte rows; K tile rows 16kk.. (4 KB per 16 channels)
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        mma_ss(d_s, dq + uint64_t((kk >> 2) * 1024 + (kk & 3) * 2), db + uint64_t(256 * kk),
-               kk > 0 ? 1u : 0u);
+      mma8_ss(d_s, dq, db, 0u);
       mma_commit(bar(SFULL + b));
       DKV_TR(14, q);
     };
@@ -1338,9 +1383,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       const uint32_t acc0 = p > 0 ? 1u : 0u;
       // tokens 16kk..16kk+15: packed P columns 8kk..8kk+7, V rows 16kk.. (4 KB)
       if (n_tok - pv_start >= TT) {
-#pragma unroll
-        for (int kk = 0; kk < TT / 16; ++kk)
-          mma_ts(tmem + kColO, a_p + 8 * kk, dv + uint64_t(256 * kk), kk > 0 ? 1u : acc0);
+        mma8_ts(tmem + kColO, a_p, dv, acc0);
       } else {
         const int nk = int(n_tok - pv_start) >> 4;  // the last tile stops at its last token
 #pragma unroll 1
