@@ -74,11 +74,10 @@ __device__ __forceinline__ uint32_t code_of(float x, const GroupQuant& q, int le
 }
 
 constexpr int kThreads = 256;
-// CTAs per (sequence, kv-head) unit: slice sl takes K channels
-// [32 sl, 32 sl + 32) and V tokens [sl blk/4, (sl + 1) blk/4) of the block.
 // CTAs per (sequence, kv-head) unit, chosen per launch from the unit count
-// (1, 2 or 4, about two CTAs per SM): slice sl of nsl takes K channels
-// [sl 128/nsl, (sl + 1) 128/nsl) and V tokens [sl blk/nsl, (sl + 1) blk/nsl).
+// (1, 2 or 4, so that all CTAs fit one wave of four per SM): slice sl of nsl
+// takes K channels [sl 128/nsl, (sl + 1) 128/nsl) and V tokens
+// [sl blk/nsl, (sl + 1) blk/nsl).
 constexpr int kMaxSlices = 4;
 constexpr int kPendStride = 128 + 8;  // tokens per staged channel row (pending <= 128), padded
 
@@ -195,6 +194,62 @@ __device__ __forceinline__ void pack_codes(F code, uint32_t (&words)[n * B / 32]
   if constexpr (n * B / 32 > 2) words[2] = uint32_t(hi);
 }
 
+// Codes of n values (val(e); code 0 where bit e of `zero` is set) packed
+// little-endian as in pack_codes, with code_of's arithmetic split in two
+// passes: the unrolled pass takes the reciprocal estimate for every value and
+// notes those near a tie; a rolled pass then replaces their codes with the
+// exact division's (rare).  The unrolled loop holds no call, so the values
+// need not stay live across one.
+template <int B, int n, class V>
+__device__ __forceinline__ void quantize_pack(V val, uint32_t zero, const GroupQuant& q, int levels,
+                                              uint32_t (&words)[n * B / 32]) {
+  uint64_t lo = 0, hi = 0;  // bits [0, 64) and [64, 128) of the stream
+  auto put = [&](int e, uint64_t cq) {
+    const int pos = B * e;
+    if (pos + B <= 64) {
+      lo |= cq << pos;
+    } else if (pos >= 64) {
+      hi |= cq << (pos - 64);
+    } else {
+      lo |= cq << pos;
+      hi |= cq >> (64 - pos);
+    }
+  };
+  if (q.s32 > 0.f) {
+    uint32_t tie = 0u;
+#pragma unroll
+    for (int e = 0; e < n; ++e) {
+      if ((zero >> e) & 1u) continue;
+      const float t = __fmul_rn(__fsub_rn(val(e), q.z32), q.rs);
+      if (fabsf(fabsf(__fsub_rn(t, rintf(t))) - 0.5f) < 2.44140625e-4f) tie |= 1u << e;
+      int c = __float2int_rn(t);
+      c = c < 0 ? 0 : (c > levels ? levels : c);
+      put(e, uint64_t(c));
+    }
+#pragma unroll 1
+    while (tie) {
+      const int e = __ffs(tie) - 1;
+      tie &= tie - 1u;
+      int c = __float2int_rn(exact_quotient(__fsub_rn(val(e), q.z32), q.s32));
+      c = c < 0 ? 0 : (c > levels ? levels : c);
+      // replace the estimate's code at bits [B e, B e + B)
+      const int pos = B * e;
+      const uint64_t m = (uint64_t(1) << B) - 1;
+      if (pos + B <= 64) {
+        lo = (lo & ~(m << pos)) | (uint64_t(c) << pos);
+      } else if (pos >= 64) {
+        hi = (hi & ~(m << (pos - 64))) | (uint64_t(c) << (pos - 64));
+      } else {
+        lo = (lo & ~(m << pos)) | (uint64_t(c) << pos);
+        hi = (hi & ~(m >> (64 - pos))) | (uint64_t(c) >> (64 - pos));
+      }
+    }
+  }
+  words[0] = uint32_t(lo);
+  if constexpr (n * B / 32 > 1) words[1] = uint32_t(lo >> 32);
+  if constexpr (n * B / 32 > 2) words[2] = uint32_t(hi);
+}
+
 // min / max over the `lanes` consecutive lanes of one group (lanes a power
 // of two dividing 32, the group aligned to it)
 __device__ __forceinline__ void group_minmax(float& mn, float& mx, int lanes) {
@@ -251,7 +306,7 @@ __device__ __forceinline__ int group_mask(const CacheView& c, const uint32_t* tm
 // the first group this commit completes), which no CTA of this launch
 // writes, so the CTAs of one unit need no ordering among themselves.
 template <int KB, int VB>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 4)  // four CTAs per SM: one wave up to 592 CTAs
 commit_kernel(const __grid_constant__ CacheView c, const uint16_t* __restrict__ k,
               const uint16_t* __restrict__ v, const uint32_t* __restrict__ pw,
               const __grid_constant__ CommitArgs ca, int nsl) {
@@ -418,8 +473,8 @@ commit_kernel(const __grid_constant__ CacheView c, const uint16_t* __restrict__ 
         const int wi = tw >> 5;
         const uint32_t gw = wi == 0 ? gm[0] : (wi == 1 ? gm[1] : (wi == 2 ? gm[2] : gm[3]));
         const uint32_t mw = (gw >> (tw & 31)) & ((kper == 32 ? 0u : (1u << kper)) - 1u);
-        float x[kper];
-        uint32_t raw2[kper / 2];  // the tokens' bf16 bits, two per word
+        uint32_t raw2[kper / 2];  // the tokens' bf16 bits, two per word (values are
+                                  // re-derived from them, not held as floats)
         float mn = __int_as_float(0x7f800000), mx = -__int_as_float(0x7f800000);
         {
           // this thread's kper tokens: kper / 8 16-byte reads of its channel row
@@ -434,10 +489,10 @@ commit_kernel(const __grid_constant__ CacheView c, const uint16_t* __restrict__ 
           }
         }
         auto raw = [&](int e) { return uint16_t(raw2[e >> 1] >> (16 * (e & 1))); };
+        auto val = [&](int e) { return sanitize(bf16_bits_to_f32(raw(e))); };
 #pragma unroll
         for (int e = 0; e < kper; ++e) {
-          float f = sanitize(bf16_bits_to_f32(raw(e)));
-          x[e] = f;
+          const float f = val(e);
           if (!((mw >> e) & 1u)) {
             mn = fminf(mn, f);
             mx = fmaxf(mx, f);
@@ -447,9 +502,7 @@ commit_kernel(const __grid_constant__ CacheView c, const uint16_t* __restrict__ 
         if (mn > mx) mn = mx = 0.f;  // every token protected
         const GroupQuant q = make_quant(mn, mx, levels);
         uint32_t words[kwpt];
-        pack_codes<KB, kper>(
-            [&](int e) { return ((mw >> e) & 1u) ? 0u : code_of(x[e], q, levels); },  // protected: 0
-            words);
+        quantize_pack<KB, kper>(val, mw, q, levels, words);  // protected tokens: code 0
         const size_t gidx = (size_t(u) * c.nG + size_t(j)) * d + ch;
 #pragma unroll
         for (int i = 0; i < kwpt; ++i) c.k_codes[gidx * c.kw + w * kwpt + i] = words[i];
@@ -485,26 +538,29 @@ commit_kernel(const __grid_constant__ CacheView c, const uint16_t* __restrict__ 
       const int w = iv % vthr, t = t_lo + iv / vthr;
       const int wpg = c.GV / vper;  // threads per V group
       const uint16_t* src = vu + size_t(t) * d + w * vper;
-      float x[vper];
-      float mn = __int_as_float(0x7f800000), mx = -__int_as_float(0x7f800000);
+      uint32_t raw2[vper / 2];  // the channels' bf16 bits, two per word
 #pragma unroll
       for (int o = 0; o < vper / 8; ++o) {
         const uint4 q8 = *reinterpret_cast<const uint4*>(src + 8 * o);
-        const uint32_t ww[4] = {q8.x, q8.y, q8.z, q8.w};
+        raw2[4 * o] = q8.x;
+        raw2[4 * o + 1] = q8.y;
+        raw2[4 * o + 2] = q8.z;
+        raw2[4 * o + 3] = q8.w;
+      }
+      auto bits = [&](int e) { return uint16_t(raw2[e >> 1] >> (16 * (e & 1))); };
+      auto val = [&](int e) { return sanitize(bf16_bits_to_f32(bits(e))); };
+      float mn = __int_as_float(0x7f800000), mx = -__int_as_float(0x7f800000);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          float f = bf16_bits_to_f32(uint16_t(ww[e >> 1] >> (16 * (e & 1))));
-          range |= out_of_range(f);
-          f = sanitize(f);
-          x[8 * o + e] = f;
-          mn = fminf(mn, f);
-          mx = fmaxf(mx, f);
-        }
+      for (int e = 0; e < vper; ++e) {
+        range |= out_of_range(bf16_bits_to_f32(bits(e)));
+        const float f = val(e);
+        mn = fminf(mn, f);
+        mx = fmaxf(mx, f);
       }
       group_minmax(mn, mx, wpg);
       const GroupQuant q = make_quant(mn, mx, levels);
       uint32_t words[vwpt];
-      pack_codes<VB, vper>([&](int e) { return code_of(x[e], q, levels); }, words);
+      quantize_pack<VB, vper>(val, 0u, q, levels, words);
       const size_t tok = size_t(u) * c.cap + size_t(p0 + t);
 #pragma unroll
       for (int i = 0; i < vwpt; ++i) c.v_codes[tok * c.vw + w * vwpt + i] = words[i];
@@ -556,7 +612,7 @@ __global__ void truncate_kernel(const __grid_constant__ CacheView c,
 template <int KB, int VB>
 cudaError_t launch_kv(const CacheView& c, const uint16_t* k, const uint16_t* v,
                       const uint32_t* pw, const CommitArgs& ca, cudaStream_t s) {
-  // about two CTAs per SM (148 SMs): four slices for small batches, one for large
+  // one wave of at most four CTAs per SM (148 SMs): four slices for small batches, one for large
   const int nsl = c.U >= 296 ? 1 : (c.U >= 148 ? 2 : kMaxSlices);
   const cudaError_t e = launch_pdl(commit_kernel<KB, VB>, dim3(unsigned(c.U) * unsigned(nsl)),
                                    dim3(kThreads), 0, s, c, k, v, pw, ca, nsl);
