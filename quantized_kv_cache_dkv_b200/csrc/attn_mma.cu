@@ -550,20 +550,40 @@ __global__ void __launch_bounds__(128) combine_kernel(const __grid_constant__ At
   if (row >= int64_t(a.c.U) * rows) return;
   const int64_t u = row / rows, r = row % rows;
   const size_t base = size_t(u) * a.nsplit * rows + r;  // split s at base + s*rows
+  // Splits merged in a fixed order, four at a time with all their loads in
+  // flight: a running max M, the sum and O rescaled when it rises.  Empty
+  // splits (max -inf, sum 0, O 0) get weight 1 against an equal -inf max
+  // instead of 2^(-inf + inf).
   float M = -__int_as_float(0x7f800000);
-  for (int s = 0; s < a.nsplit; ++s) M = fmaxf(M, a.part_ml[base + size_t(s) * rows].x);
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float lsum = 0.f;
-  for (int s = 0; s < a.nsplit; ++s) {
-    const float2 ml = a.part_ml[base + size_t(s) * rows];
-    const float w = fast_exp2(ml.x - M);
-    lsum += w * ml.y;
-    const float4 x =
-        *reinterpret_cast<const float4*>(a.part_o + (base + size_t(s) * rows) * kHeadDim + lane * 4);
-    acc.x += w * x.x;
-    acc.y += w * x.y;
-    acc.z += w * x.z;
-    acc.w += w * x.w;
+#pragma unroll 1
+  for (int s0 = 0; s0 < a.nsplit; s0 += 4) {
+    const int n = a.nsplit - s0 < 4 ? a.nsplit - s0 : 4;
+    float2 ml[4];
+    float4 x[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if (i < n) {
+        const size_t ps = base + size_t(s0 + i) * rows;
+        ml[i] = a.part_ml[ps];
+        x[i] = *reinterpret_cast<const float4*>(a.part_o + ps * kHeadDim + lane * 4);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if (i < n) {
+        const float Mn = fmaxf(M, ml[i].x);
+        const float c = M == Mn ? 1.f : fast_exp2(M - Mn);
+        const float w = ml[i].x == Mn ? 1.f : fast_exp2(ml[i].x - Mn);
+        lsum = lsum * c + w * ml[i].y;
+        acc.x = acc.x * c + w * x[i].x;
+        acc.y = acc.y * c + w * x[i].y;
+        acc.z = acc.z * c + w * x[i].z;
+        acc.w = acc.w * c + w * x[i].w;
+        M = Mn;
+      }
+    }
   }
   const float inv = 1.f / lsum;
   float x[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
