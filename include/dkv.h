@@ -254,7 +254,7 @@ int dkv_cache_truncate(dkv_cache* cache, int64_t new_len, void* stream);
  *   - The buffer is a static __device__ array of DKV_NOALLOC_SCRATCH_BYTES
  *     (16 MiB); every GPU that loads libdkv holds it until the process exits.
  *   - A plan needing more scratch than that (B*Hkv * splits *
- *     (q_heads/kv_heads)*block * (4*head_dim + 8) bytes, whenever the
+ *     (q_heads/kv_heads)*block * (2*head_dim + 8) bytes, whenever the
  *     combine kernel runs: splits > 1, or a rotated-V cache) returns
  *     DKV_ERR_UNSUPPORTED with a message; lower DKV_OPT_SPLITS.
  *   - A rotated-V cache rotates the active block's V into the buffer the

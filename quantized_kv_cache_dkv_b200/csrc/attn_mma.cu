@@ -10,7 +10,8 @@
 // from the side table, tail / active-block tokens converted from bf16), then
 // each warp runs S = Q K^T, an online softmax in the log2 domain, and
 // O += P V with m16n8k16 fp16 MMAs and fp32 accumulators.  Split partials
-// (unnormalised O, running max, running sum) are merged by combine_kernel.
+// (the split's O divided by its row sum in fp16, its running max and row sum)
+// are merged by combine_kernel.
 #include "dequant.cuh"
 #include "dkv_internal.cuh"
 
@@ -482,13 +483,16 @@ attn_mma_kernel(const __grid_constant__ AttnArgs a) {
     }
   } else {
     const size_t prow = (size_t(u) * a.part_stride + a.part_base + sp) * c.rows;
-    float* po0 = a.part_o + (prow + r0) * kHeadDim;
-    float* po1 = po0 + 8 * kHeadDim;
+    // the split's output divided by its row sum, in fp16 (an empty split --
+    // past the end of a shorter sequence -- has sum 0 and O 0: zeros)
+    const float i0 = l0 > 0.f ? 1.f / l0 : 0.f, i1 = l1 > 0.f ? 1.f / l1 : 0.f;
+    __half* po0 = a.part_o + (prow + r0) * kHeadDim;
+    __half* po1 = po0 + 8 * kHeadDim;
 #pragma unroll
     for (int nd = 0; nd < 16; ++nd) {
       const int col = nd * 8 + cq;
-      *reinterpret_cast<float2*>(po0 + col) = make_float2(o[nd][0], o[nd][1]);
-      *reinterpret_cast<float2*>(po1 + col) = make_float2(o[nd][2], o[nd][3]);
+      *reinterpret_cast<__half2*>(po0 + col) = __floats2half2_rn(o[nd][0] * i0, o[nd][1] * i0);
+      *reinterpret_cast<__half2*>(po1 + col) = __floats2half2_rn(o[nd][2] * i1, o[nd][3] * i1);
     }
     if ((lane & 3) == 0) {
       a.part_ml[prow + r0] = make_float2(m0, l0);
@@ -561,13 +565,13 @@ __global__ void __launch_bounds__(128) combine_kernel(const __grid_constant__ At
   for (int s0 = 0; s0 < a.nsplit; s0 += 4) {
     const int n = a.nsplit - s0 < 4 ? a.nsplit - s0 : 4;
     float2 ml[4];
-    float4 x[4];
+    uint2 x[4];  // four fp16 channels of the split's normalised output
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       if (i < n) {
         const size_t ps = base + size_t(s0 + i) * rows;
         ml[i] = a.part_ml[ps];
-        x[i] = *reinterpret_cast<const float4*>(a.part_o + ps * kHeadDim + lane * 4);
+        x[i] = *reinterpret_cast<const uint2*>(a.part_o + ps * kHeadDim + lane * 4);
       }
     }
 #pragma unroll
@@ -575,12 +579,14 @@ __global__ void __launch_bounds__(128) combine_kernel(const __grid_constant__ At
       if (i < n) {
         const float Mn = fmaxf(M, ml[i].x);
         const float c = M == Mn ? 1.f : fast_exp2(M - Mn);
-        const float w = ml[i].x == Mn ? 1.f : fast_exp2(ml[i].x - Mn);
-        lsum = lsum * c + w * ml[i].y;
-        acc.x = acc.x * c + w * x[i].x;
-        acc.y = acc.y * c + w * x[i].y;
-        acc.z = acc.z * c + w * x[i].z;
-        acc.w = acc.w * c + w * x[i].w;
+        const float wl = (ml[i].x == Mn ? 1.f : fast_exp2(ml[i].x - Mn)) * ml[i].y;
+        const float2 o01 = __half22float2(*reinterpret_cast<const __half2*>(&x[i].x));
+        const float2 o23 = __half22float2(*reinterpret_cast<const __half2*>(&x[i].y));
+        lsum = lsum * c + wl;
+        acc.x = acc.x * c + wl * o01.x;
+        acc.y = acc.y * c + wl * o01.y;
+        acc.z = acc.z * c + wl * o23.x;
+        acc.w = acc.w * c + wl * o23.y;
         M = Mn;
       }
     }

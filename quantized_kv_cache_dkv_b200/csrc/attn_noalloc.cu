@@ -85,7 +85,7 @@ extern "C" int dkv_block_attention_noalloc(dkv_cache* cache, const void* q, cons
           ("this plan needs " + std::to_string(need) + " bytes of split scratch; the static buffer "
            "holds " + std::to_string(kScratchBytes) + ": lower DKV_OPT_SPLITS or use "
            "dkv_block_attention").c_str());
-    a.part_o = static_cast<float*>(scratch);
+    a.part_o = static_cast<__half*>(scratch);
     a.part_ml = reinterpret_cast<float2*>(static_cast<unsigned char*>(scratch) + o_bytes);
   }
 

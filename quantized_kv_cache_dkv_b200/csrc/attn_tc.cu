@@ -1038,8 +1038,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     pdl_trigger();
     if (!a.final_out) {
       const size_t prow = (size_t(u) * a.part_stride + a.part_base + sp) * cv.rows + size_t(rb) * rpb;
-      for (int i = threadIdx.x; i < rpb * (kHeadDim / 4); i += kThreads)
-        reinterpret_cast<float4*>(a.part_o + prow * kHeadDim)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int i = threadIdx.x; i < rpb * (kHeadDim / 8); i += kThreads)
+        reinterpret_cast<uint4*>(a.part_o + prow * kHeadDim)[i] = make_uint4(0u, 0u, 0u, 0u);
       for (int i = threadIdx.x; i < rpb; i += kThreads)
         a.part_ml[prow + i] = make_float2(-__int_as_float(0x7f800000), 0.f);
     }
@@ -1318,12 +1318,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
           }
         } else {
-          float4* dst = reinterpret_cast<float4*>(
+          // the split's output divided by its row sum, in fp16
+          uint4* dst = reinterpret_cast<uint4*>(
               a.part_o + ((size_t(u) * a.part_stride + a.part_base + sp) * cv.rows + r) * kHeadDim + col);
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            dst[i] = make_float4(__uint_as_float(o[kpos<VB>(4 * i)]), __uint_as_float(o[kpos<VB>(4 * i + 1)]),
-                                 __uint_as_float(o[kpos<VB>(4 * i + 2)]), __uint_as_float(o[kpos<VB>(4 * i + 3)]));
+          for (int i = 0; i < 4; ++i) {
+            uint32_t w[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              w[k] = pack_h2(__uint_as_float(o[kpos<VB>(8 * i + 2 * k)]) * inv,
+                             __uint_as_float(o[kpos<VB>(8 * i + 2 * k + 1)]) * inv);
+            dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
         }
       }
       if (!a.final_out && row_ok && h == 0)
@@ -1556,8 +1562,8 @@ __global__ void __launch_bounds__(tl::kThreads, 1) attn_tl_kernel(const __grid_c
     pdl_trigger();
     if (!a.final_out) {
       const size_t prow = (size_t(u) * a.part_stride + a.part_base + sp) * tl::kRows;
-      for (int i = threadIdx.x; i < tl::kRows * (kHeadDim / 4); i += tl::kThreads)
-        reinterpret_cast<float4*>(a.part_o + prow * kHeadDim)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int i = threadIdx.x; i < tl::kRows * (kHeadDim / 8); i += tl::kThreads)
+        reinterpret_cast<uint4*>(a.part_o + prow * kHeadDim)[i] = make_uint4(0u, 0u, 0u, 0u);
       for (int i = threadIdx.x; i < tl::kRows; i += tl::kThreads)
         a.part_ml[prow + i] = make_float2(-__int_as_float(0x7f800000), 0.f);
     }
@@ -1785,7 +1791,7 @@ __global__ void __launch_bounds__(tl::kThreads, 1) attn_tl_kernel(const __grid_c
           a.out[(size_t(u) * tl::kRows + i) * kHeadDim + ch] = *reinterpret_cast<const uint16_t*>(&v);
         } else {
           const size_t prow = (size_t(u) * a.part_stride + a.part_base + sp) * tl::kRows + i;
-          a.part_o[prow * kHeadDim + ch] = ov;
+          a.part_o[prow * kHeadDim + ch] = __float2half_rn(ov / lt);
           if (l == 0) a.part_ml[prow] = make_float2(ref[i], lt);
         }
       }

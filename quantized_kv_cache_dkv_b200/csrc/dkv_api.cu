@@ -28,7 +28,7 @@ struct dkv_cache {
   std::vector<char> trunc;         // a roll-back of that sequence not yet applied on the device
   void* arena = nullptr;
   size_t arena_bytes = 0;
-  float* part_o = nullptr;
+  __half* part_o = nullptr;
   float2* part_ml = nullptr;
   void* sel_mem = nullptr;       // selection workspace (first dkv_block_attention_selected)
   void* vrot_mem = nullptr;      // rotation parameters + rotated active block (V rotation)
@@ -348,7 +348,7 @@ int dkv_cache_alloc(const dkv_config* cfg, void* stream, dkv_cache** out) {
   v.prot_k = static_cast<uint16_t*>(at(r_pk));
   v.prot_gstart = static_cast<int32_t*>(at(r_pg));
   v.status = static_cast<uint32_t*>(at(r_st));
-  c->part_o = static_cast<float*>(at(r_po));
+  c->part_o = static_cast<__half*>(at(r_po));
   c->part_ml = static_cast<float2*>(at(r_pml));
   v.v_sink = static_cast<uint16_t*>(at(r_vsink));
 

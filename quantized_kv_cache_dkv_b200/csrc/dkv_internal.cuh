@@ -117,7 +117,7 @@ struct AttnArgs {
   const uint16_t* k_act;  // [B][Hkv][blk][d] bf16
   const uint16_t* v_act;  // [B][Hkv][blk][d] bf16
   uint16_t* out;          // [B][Hq][blk][d] bf16
-  float* part_o;          // [U][nsplit][rows][d] fp32 (unnormalised)
+  __half* part_o;         // [U][nsplit][rows][d] fp16: the split's output divided by its row sum
   float2* part_ml;        // [U][nsplit][rows] (running max in log2 units, sum)
   float scale_log2;       // softmax_scale * log2(e)
   int64_t L;              // committed tokens of the longest sequence (planning)
@@ -206,7 +206,7 @@ cudaError_t launch_attention_tc(const AttnArgs& a, cudaStream_t s);
 // starting at the next 256-byte boundary.  The handle's workspace and the
 // no-allocation entry point's static buffer are both sized by these.
 inline size_t split_o_bytes(int64_t U, int64_t splits, int64_t rows) {
-  return (size_t(U) * size_t(splits) * size_t(rows) * kHeadDim * sizeof(float) + 255) &
+  return (size_t(U) * size_t(splits) * size_t(rows) * kHeadDim * sizeof(__half) + 255) &
          ~size_t(255);
 }
 inline size_t split_ml_bytes(int64_t U, int64_t splits, int64_t rows) {

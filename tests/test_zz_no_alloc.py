@@ -140,9 +140,10 @@ def test_noalloc_rotated_v(dkv):
 
 def test_noalloc_rejects_scratch_beyond_buffer(dkv):
     import torch
-    w = CASES["groups128"].with_(B=8, Hkv=8, Hq=32, L=2048)
+    w = CASES["groups128"].with_(B=16, Hkv=8, Hq=32, L=2048)
     cache, _ = _built(dkv, w, with_oracle=False)
-    # 64 units x 8 splits x 128 rows x 520 bytes = 34 MB > 16 MiB
+    # 17 tiles in splits of 3: 128 units x 6 splits x 128 rows x 264 bytes
+    # (fp16 partial + (max, sum)) = 26 MB > 16 MiB
     dkv.dkv_cache_set_option(cache, dkv.DKV_OPT_SPLITS, 8)
     Q = dev_bf16(synth.queries_bits(w, 0))
     Ka, Va = [dev_bf16(x) for x in synth.active_block_bits(w, 0)]
