@@ -1147,6 +1147,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       tc_fence_after();
       if ((threadIdx.x & 127) == 0) DKV_TR(6, j);
       if (!warp_rows) {
+        // Arrivals for tile j only once PV(j-2) is complete (so are all
+        // arrivals for tile j-2): QK(j) can complete while the row warps are
+        // still in tile j-2 after their SFREE, and early arrivals here would
+        // count toward tile j-2's RREADY / PFULL phases.
+        if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(bar(VEMPTY + b), ((j - 2) >> 1) & 1, a,
+                                                          abort_flag))) {
+          ok = false;
+          break;
+        }
         mbar_arrive(bar(RREADY + b));
         mbar_arrive(bar(SFREE + b));
         mbar_arrive(bar(PFULL + b));

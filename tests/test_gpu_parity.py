@@ -357,3 +357,33 @@ def test_full_size_sampled_units(dkv, name):
     # every output finite and bounded by the largest |V| of the cache
     allv = synth.bf16_bits_to_f32(got)
     assert np.all(np.isfinite(allv))
+
+
+@pytest.mark.parametrize("kernel,splits", [(2, 1), (2, 4), (2, 0), (1, 0)])
+def test_repeat_bit_identical_mha8b(dkv, kernel, splits):
+    """The attention of a fixed plan is deterministic: repeated calls give the
+    same bits in every unit.  The 32-row query groups of the 8B MHA workload
+    leave three of the four warps of each softmax warpgroup with padding rows
+    only; a hand-off that lets those warps run a tile ahead of the row warps
+    shows up as rows that change from call to call."""
+    torch = _torch()
+    w = synth.WORKLOADS["mha8b"]
+    n_blocks = w.L // w.blk
+    cap = default_cap(w, n_blocks + 1)
+    P = default_P(w, cap)
+    cache = dkv.dkv_cache_alloc(gpu_config(dkv, w, cap, P))
+    commit_both(dkv, cache, None, w, range(n_blocks))
+    dkv.dkv_cache_set_option(cache, dkv.DKV_OPT_ATTN_KERNEL, kernel)
+    dkv.dkv_cache_set_option(cache, dkv.DKV_OPT_SPLITS, splits)
+    q, ka, va = (dev_bf16(x) for x in (synth.queries_bits(w, 0), *synth.active_block_bits(w, 0)))
+    outs = []
+    for _ in range(8):
+        out = torch.empty((w.B, w.Hq, w.blk, w.d), dtype=torch.bfloat16, device="cuda")
+        dkv.dkv_block_attention(cache, q, ka, va, w.softmax_scale, out)
+        outs.append(out)
+    torch.cuda.synchronize()
+    assert dkv.dkv_cache_status(cache) == 0
+    first = host_bits(outs[0])
+    for i, o in enumerate(outs[1:], 1):
+        diff = np.argwhere(host_bits(o) != first)
+        assert diff.size == 0, f"call {i} differs from call 0 at (b, head, row, ch) {diff[:4].tolist()}"
