@@ -648,24 +648,41 @@ __device__ __noinline__ void fill_k_general(const AttnArgs& a, const UnitLen ul,
 }
 
 // V tile: thread `tid` (0..255) fills items (token t, channel quarter qq) with
-// qq = item % 4, t = item / 4, item = tid + 256 r (r = 0, 1), so a warp reads
-// 512 contiguous bytes of the ring stage ([token][vw words]).
+// qq = tid % 4 and t = v_slot_token(tid / 4) + 64 r (r = 0, 1): a warp reads
+// its eight tokens' code words from the ring stage ([token][vw words]) in
+// 32-byte pieces or larger.
+
+// Token (0..63 of a half tile) whose V row the V producer slot s (= tid / 4,
+// four threads per token) fills.  In the K tile's row order (kpos) tokens t
+// and t + 1 sit 2 rows apart modulo 8, which gives their 16-byte chunks the
+// same bank groups; a quarter warp (two slots) therefore takes tokens t and
+// t + 8 (2-bit K) or t + 4 (4-bit K), which sit 1 row apart modulo 8, and
+// its eight 16-byte stores fall in eight distinct bank groups.
+template <int KB>
+__device__ __forceinline__ int v_slot_token(int s) {
+  if constexpr (KB == 2) return (s & ~15) | ((s & 15) >> 1) | ((s & 1) << 3);
+  else if constexpr (KB == 4) return (s & ~7) | ((s & 7) >> 1) | ((s & 1) << 2);
+  else return s;
+}
+
 // Byte offsets of the 16-byte chunks a V producer thread stores: item r
-// (token (tid >> 2) + 64 r, quarter tid & 3), store i = chunk (i + rot) & 3.
+// (token t0 + 64 r, quarter tid & 3), store i = chunk (i + rot) & 3.
 template <int KB>
 struct VOffsets {
   uint32_t base, x[4];
   uint32_t w[2], z[2];  // ring offsets of item r: code words (uint32), (scale, zero) pairs
   __device__ VOffsets(int tid, int vw, int vgroups, int GV, int vb) {
-    // row of token tid >> 2 (and + 64): its kpos position (identity for bf16 K)
-    const int p = kpos<KB>(tid >> 2);
+    // row of this thread's token t0 (and t0 + 64): its kpos position
+    // (identity for bf16 K)
+    const int t0 = v_slot_token<KB>(tid >> 2);
+    const int p = kpos<KB>(t0);
     const int qq = tid & 3, t7 = p & 7, rot = qq & 2;
     base = uint32_t(((p >> 3) * 2 + (qq >> 1)) * 1024 + t7 * 128);
 #pragma unroll
     for (int i = 0; i < 4; ++i) x[i] = uint32_t(((4 * (qq & 1) + ((i + rot) & 3)) ^ t7) << 4);
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
-      const int t = (tid + 256 * r) >> 2;
+      const int t = t0 + 64 * r;
       w[r] = uint32_t(t * vw + qq * (vb == 4 ? 4 : 2));
       z[r] = uint32_t(t * vgroups + (qq * 32) / GV);
     }
@@ -730,8 +747,9 @@ __device__ __noinline__ void fill_v_general(const AttnArgs& a, const UnitLen ul,
   const int d = kHeadDim;
 #pragma unroll 1
   for (int r = 0; r < 2; ++r) {
-    const int item = tid + 256 * r;
-    const int t = item >> 2, qq = item & 3;
+    const int sl = tid >> 2, qq = tid & 3;
+    const int t = (perm_kb == 2 ? v_slot_token<2>(sl) : (perm_kb == 4 ? v_slot_token<4>(sl) : sl)) +
+                  64 * r;
     const int64_t pos = tile_start + t;
     // row of token t (the K tile's order, see kpos)
     const int p = perm_kb == 2 ? kpos<2>(t) : (perm_kb == 4 ? kpos<4>(t) : t);
@@ -749,7 +767,8 @@ __device__ __noinline__ void fill_v_general(const AttnArgs& a, const UnitLen ul,
       raw = a.v_act + (size_t(u) * cv.blk + (pos - ul.L)) * d;
     }
     // out[i] holds channels 32qq + 8((i + rot) & 3): lanes of a quarter warp
-    // (tokens t, t+1 x quarters 0..3) then store to 8 distinct bank groups
+    // (two tokens one row apart modulo 8, see v_slot_token, x quarters 0..3)
+    // then store to 8 distinct bank groups
     const int rot = qq & 2;
     if (codes) {
       if constexpr (VB < 16) {
