@@ -1037,13 +1037,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 
   const CacheView& cv = a.c;
   // CTA = (unit, split, row block): a query group of more than 128 rows is
-  // cut into row blocks of 128 and the rest (rows are multiples of 32, so a
-  // short block leaves whole warps of padding rows, which skip the softmax
-  // arithmetic); blocks are zero-padded to M = 128
+  // cut into row blocks of rows/nrb; smaller blocks are zero-padded to M = 128
   const int nrb = (cv.rows + 127) / 128;
+  const int rpb = cv.rows / nrb;
   const int rb = blockIdx.x % nrb;
-  const int r0 = rb * 128;                                   // first query row of the block
-  const int rpb = cv.rows - r0 < 128 ? cv.rows - r0 : 128;  // rows of the block
   const int u = (blockIdx.x / nrb) / a.nsplit;
   const int sp = (blockIdx.x / nrb) % a.nsplit;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1059,7 +1056,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     pdl_wait();
     pdl_trigger();
     if (!a.final_out) {
-      const size_t prow = (size_t(u) * a.part_stride + a.part_base + sp) * cv.rows + size_t(r0);
+      const size_t prow = (size_t(u) * a.part_stride + a.part_base + sp) * cv.rows + size_t(rb) * rpb;
       for (int i = threadIdx.x; i < rpb * (kHeadDim / 8); i += kThreads)
         reinterpret_cast<uint4*>(a.part_o + prow * kHeadDim)[i] = make_uint4(0u, 0u, 0u, 0u);
       for (int i = threadIdx.x; i < rpb; i += kThreads)
@@ -1117,7 +1114,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     // a warp holding only padding rows skips the softmax arithmetic (its P
     // rows feed only padding rows of O, which are never read)
     const bool warp_rows = (warp & 3) * 32 < rpb;
-    const int r = r0 + lr;              // query row of the unit
+    const int r = rb * rpb + lr;        // query row of the unit
     const uint32_t lane_base = tmem + (uint32_t((warp & 3) * 32) << 16);
     float* ref = reinterpret_cast<float*>(sm + SmemTail<KB, VB>::kRef);    // [tile parity][row]
     float* lsum = reinterpret_cast<float*>(sm + SmemTail<KB, VB>::kLsum);  // [warpgroup][row], then refs
