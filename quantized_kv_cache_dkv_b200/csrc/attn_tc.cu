@@ -109,7 +109,10 @@ constexpr uint32_t kMaxStageBytes = Stage<4, 4>::kBytes > Stage<2, 4>::kBytes
                                                                                       : Stage<4, 2>::kBytes)
                                         : Stage<2, 4>::kBytes;
 static_assert(Stage<2, 2>::kBytes <= kMaxStageBytes && Stage<2, 16>::kBytes <= kMaxStageBytes &&
-                  Stage<4, 16>::kBytes <= kMaxStageBytes && Stage<16, 4>::kBytes <= kMaxStageBytes,
+                  Stage<4, 16>::kBytes <= kMaxStageBytes && Stage<16, 4>::kBytes <= kMaxStageBytes &&
+                  Stage<3, 4>::kBytes <= kMaxStageBytes && Stage<4, 3>::kBytes <= kMaxStageBytes &&
+                  Stage<3, 3>::kBytes <= kMaxStageBytes && Stage<3, 16>::kBytes <= kMaxStageBytes &&
+                  Stage<16, 3>::kBytes <= kMaxStageBytes,
               "largest ring stage");
 
 struct Smem {
@@ -457,7 +460,9 @@ __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
 // chunk i (0..7) holds tokens 64 qh + 8 i .. +7 of channel c.
 // Tiles whose K is wholly quantized are stored in the order the prmt-free
 // dequantization produces: the token at tile position kpos(t) is t, permuted
-// within groups of 16 (2-bit codes) or 8 (4-bit codes).  V tiles hold their
+// within groups of 16 (2-bit codes) or 8 (4-bit codes); 3-bit codes (32 to
+// three words, two of them straddling words) are extracted one by one and
+// keep the natural order.  V tiles hold their
 // channels in the same kind of order for V's bit width (kpos<VB>, in every
 // tile, bf16 rows included), so O's column kpos<VB>(c) is channel c and the
 // epilogue reads it from there.  The V tile of such a
@@ -507,21 +512,23 @@ __device__ __forceinline__ void fill_k_tile(const AttnArgs& a, const UnitLen ul,
     if (tile_start + TT <= ul.Lq) {
       // whole tile quantized: one 32-token chunk per iteration (a rolled
       // loop keeps the hot code small)
-      using W = typename std::conditional<KB == 4, uint4, uint2>::type;
 #pragma unroll 1
       for (int qi = 0; qi < 2; ++qi) {
-        const W w = *reinterpret_cast<const W*>(reinterpret_cast<const uint32_t*>(rs + ST::kRKc) +
-                                                (qi ? ko.w[1] : ko.w[0]));
+        const uint32_t* wp = reinterpret_cast<const uint32_t*>(rs + ST::kRKc) + (qi ? ko.w[1] : ko.w[0]);
         const __half2 sz = reinterpret_cast<const __half2*>(rs + ST::kRKsz)[qi ? ko.z[1] : ko.z[0]];
         const __half2 s2 = __half2half2(__low2half(sz));
         const __half2 z2 = __half2half2(__high2half(sz));
         uint4 out[4];  // tokens in kpos order
         if constexpr (KB == 4) {
+          const uint4 w = *reinterpret_cast<const uint4*>(wp);
           out[0] = dequant4x8_raw(w.x, s2, z2);
           out[1] = dequant4x8_raw(w.y, s2, z2);
           out[2] = dequant4x8_raw(w.z, s2, z2);
           out[3] = dequant4x8_raw(w.w, s2, z2);
+        } else if constexpr (KB == 3) {
+          dequant3x32(wp[0], wp[1], wp[2], s2, z2, out);  // 4-byte aligned words
         } else {
+          const uint2 w = *reinterpret_cast<const uint2*>(wp);
           dequant2x16_raw(w.x, s2, z2, out[0], out[1]);
           dequant2x16_raw(w.y, s2, z2, out[2], out[3]);
         }
@@ -596,6 +603,8 @@ __device__ __noinline__ void fill_k_general(const AttnArgs& a, const UnitLen ul,
           out[1] = dequant4x8(w.y, s2, z2);
           out[2] = dequant4x8(w.z, s2, z2);
           out[3] = dequant4x8(w.w, s2, z2);
+        } else if constexpr (KB == 3) {
+          dequant3x32(kc[0], kc[1], kc[2], s2, z2, out);
         } else {
           const uint2 w = *reinterpret_cast<const uint2*>(kc);
           dequant2x16(w.x, s2, z2, out[0], out[1]);
@@ -683,7 +692,7 @@ struct VOffsets {
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
       const int t = t0 + 64 * r;
-      w[r] = uint32_t(t * vw + qq * (vb == 4 ? 4 : 2));
+      w[r] = uint32_t(t * vw + qq * (vb < 16 ? vb : 0));  // a channel quarter: vb words
       z[r] = uint32_t(t * vgroups + (qq * 32) / GV);
     }
   }
@@ -708,23 +717,30 @@ __device__ __forceinline__ void fill_v_tile(const AttnArgs& a, const UnitLen ul,
     if ((KB < 16 ? k_whole : tile_start + TT <= ul.L) && (!SINK || tile_start >= cv.sink)) {
       // whole tile quantized: one item per iteration (a rolled loop keeps
       // the hot code small)
-      using W = typename std::conditional<VB == 4, uint4, uint2>::type;
       const bool rot = (tid & 2) != 0;
 #pragma unroll 1
       for (int r = 0; r < 2; ++r) {
-        W x = *reinterpret_cast<const W*>(reinterpret_cast<const uint32_t*>(rs + ST::kRVc) +
-                                          (r ? vo.w[1] : vo.w[0]));
+        const uint32_t* xp = reinterpret_cast<const uint32_t*>(rs + ST::kRVc) + (r ? vo.w[1] : vo.w[0]);
         const __half2 sz = reinterpret_cast<const __half2*>(rs + ST::kRVsz)[r ? vo.z[1] : vo.z[0]];
         const __half2 s2 = __half2half2(__low2half(sz));
         const __half2 z2 = __half2half2(__high2half(sz));
         uint4 out[4];  // channels in kpos<VB> order
-        if constexpr (VB == 4) {
+        if constexpr (VB == 3) {
+          uint4 nat[4];  // 4-byte aligned words; channels in natural order
+          dequant3x32(xp[0], xp[1], xp[2], s2, z2, nat);
+          out[0] = rot ? nat[2] : nat[0];
+          out[1] = rot ? nat[3] : nat[1];
+          out[2] = rot ? nat[0] : nat[2];
+          out[3] = rot ? nat[1] : nat[3];
+        } else if constexpr (VB == 4) {
+          uint4 x = *reinterpret_cast<const uint4*>(xp);
           if (rot) x = make_uint4(x.z, x.w, x.x, x.y);
           out[0] = dequant4x8_raw(x.x, s2, z2);
           out[1] = dequant4x8_raw(x.y, s2, z2);
           out[2] = dequant4x8_raw(x.z, s2, z2);
           out[3] = dequant4x8_raw(x.w, s2, z2);
         } else {
+          uint2 x = *reinterpret_cast<const uint2*>(xp);
           if (rot) x = make_uint2(x.y, x.x);
           dequant2x16_raw(x.x, s2, z2, out[0], out[1]);
           dequant2x16_raw(x.y, s2, z2, out[2], out[3]);
@@ -777,7 +793,14 @@ __device__ __noinline__ void fill_v_general(const AttnArgs& a, const UnitLen ul,
         const __half2 s2 = __half2half2(__low2half(sz));
         const __half2 z2 = __half2half2(__high2half(sz));
         const uint32_t* vc = reinterpret_cast<const uint32_t*>(rs + ST::kRVc) + t * cv.vw;
-        if constexpr (VB == 4) {
+        if constexpr (VB == 3) {
+          uint4 nat[4];
+          dequant3x32(vc[qq * 3], vc[qq * 3 + 1], vc[qq * 3 + 2], s2, z2, nat);
+          out[0] = rot ? nat[2] : nat[0];
+          out[1] = rot ? nat[3] : nat[1];
+          out[2] = rot ? nat[0] : nat[2];
+          out[3] = rot ? nat[1] : nat[3];
+        } else if constexpr (VB == 4) {
           uint4 w = *reinterpret_cast<const uint4*>(vc + qq * 4);
           if (rot) w = make_uint4(w.z, w.w, w.x, w.y);
           out[0] = dequant4x8_raw(w.x, s2, z2);
@@ -1954,6 +1977,7 @@ template <int KB>
 cudaError_t launch_k(const AttnArgs& a, cudaStream_t s) {
   switch (a.c.vb) {
     case 2: return launch_kv<KB, 2>(a, s);
+    case 3: return launch_kv<KB, 3>(a, s);
     case 4: return launch_kv<KB, 4>(a, s);
     default: return launch_kv<KB, 16>(a, s);
   }
@@ -1962,16 +1986,15 @@ cudaError_t launch_k(const AttnArgs& a, cudaStream_t s) {
 }  // namespace
 
 // any query group of 32..256 rows (a multiple of 32): M = 128 per row block
-// (3-bit codes take the mma.sync kernel)
 bool tc_supported(const CacheView& c) {
-  return c.d == kHeadDim && c.rows >= 32 && c.rows <= 256 && c.rows % 32 == 0 && c.kb != 3 &&
-         c.vb != 3;
+  return c.d == kHeadDim && c.rows >= 32 && c.rows <= 256 && c.rows % 32 == 0;
 }
 
 cudaError_t launch_attention_tc(const AttnArgs& a, cudaStream_t s) {
   if (!tc_supported(a.c)) return cudaErrorNotSupported;
   switch (a.c.kb) {
     case 2: return launch_k<2>(a, s);
+    case 3: return launch_k<3>(a, s);
     case 4: return launch_k<4>(a, s);
     default: return launch_k<16>(a, s);
   }

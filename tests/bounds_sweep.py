@@ -72,7 +72,7 @@ def run_case(dkv, torch, w, n_blocks, cap, P, sink, trunc):
     Q = synth.queries_bits(w, 0)
     Ka, Va = synth.active_block_bits(w, 0)
     ref = oc.block_attention(Q, Ka, Va, w.softmax_scale)
-    for kernel in ((1,) if 3 in (w.k_bits, w.v_bits) else (1, 2)):   # 3 bits: mma.sync only
+    for kernel in (1, 2):
         dkv.dkv_cache_set_option(cache, dkv.DKV_OPT_ATTN_KERNEL, kernel)
         for sp in (0, 2):
             dkv.dkv_cache_set_option(cache, dkv.DKV_OPT_SPLITS, sp)

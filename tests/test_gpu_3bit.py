@@ -1,8 +1,10 @@
 """3-bit K and V (SoloQ summary: KV-only results near 3 bits, and the KV2 sink
 ablation): commit codes, scales and zero points bit for bit against the
 oracle -- 32 codes fill three words, codes 10 and 21 straddle two -- and
-attention within the output bound.  3-bit caches attend with the mma.sync
-kernel (the tcgen05 kernel refuses them)."""
+attention within the output bound on every attention kernel: mma.sync,
+tcgen05 with query-row blocks, and tcgen05 with the tokens on the TMEM lanes
+for 32-row query groups.  The tcgen05 producers extract the 32 codes of three
+words one by one and keep the natural token / channel order."""
 import pytest
 
 import synth
@@ -44,22 +46,31 @@ def test_three_bit_commit_and_attention(dkv, name, over, sink):
     commit_both(dkv, cache, oc, w, range(n_blocks))
     compare_exports(dkv.dkv_cache_export(cache), oc.snapshot())
     assert dkv.dkv_cache_status(cache) == oc.flags
+    rows = (w.Hq // w.Hkv) * w.blk
+    kernels = (1, 2, 3) if rows == 32 else (1, 2)
     for step in (0, 1):
         Q = synth.queries_bits(w, step)
         Ka, Va = synth.active_block_bits(w, step)
         ref = oc.block_attention(Q, Ka, Va, w.softmax_scale)
-        for sp in (0, 1, 3):
-            dkv.dkv_cache_set_option(cache, dkv.DKV_OPT_SPLITS, sp)
-            out = torch.empty((w.B, w.Hq, w.blk, w.d), dtype=torch.bfloat16, device="cuda")
-            dkv.dkv_block_attention(cache, dev_bf16(Q), dev_bf16(Ka), dev_bf16(Va),
-                                    w.softmax_scale, out)
-            torch.cuda.synchronize()
-            assert_close(host_bits(out), ref, f"{name} {over} step {step} splits {sp}")
-            assert dkv.dkv_last_attention_plan(cache)[0] == 1
-    # no tcgen05 variant and no rotated V at 3 bits
-    with pytest.raises(dkv.DkvError) as ei:
-        dkv.dkv_cache_set_option(cache, dkv.DKV_OPT_ATTN_KERNEL, 2)
-    assert ei.value.code == dkv.DKV_ERR_UNSUPPORTED
+        for kernel in kernels:
+            dkv.dkv_cache_set_option(cache, dkv.DKV_OPT_ATTN_KERNEL, kernel)
+            for sp in (0, 1, 3):
+                dkv.dkv_cache_set_option(cache, dkv.DKV_OPT_SPLITS, sp)
+                out = torch.empty((w.B, w.Hq, w.blk, w.d), dtype=torch.bfloat16, device="cuda")
+                dkv.dkv_block_attention(cache, dev_bf16(Q), dev_bf16(Ka), dev_bf16(Va),
+                                        w.softmax_scale, out)
+                torch.cuda.synchronize()
+                assert_close(host_bits(out), ref,
+                             f"{name} {over} step {step} kernel {kernel} splits {sp}")
+                assert dkv.dkv_last_attention_plan(cache)[0] == kernel
+    assert dkv.dkv_cache_status(cache) == oc.flags
+    # the default plan of a 3-bit cache is the row-block tcgen05 kernel
+    dkv.dkv_cache_set_option(cache, dkv.DKV_OPT_ATTN_KERNEL, 0)
+    out = torch.empty((w.B, w.Hq, w.blk, w.d), dtype=torch.bfloat16, device="cuda")
+    dkv.dkv_block_attention(cache, dev_bf16(Q), dev_bf16(Ka), dev_bf16(Va), w.softmax_scale, out)
+    torch.cuda.synchronize()
+    assert dkv.dkv_last_attention_plan(cache)[0] == 2
+    # no rotated V at 3 bits
     if w.v_bits == 3:
         fresh = dkv.dkv_cache_alloc(gpu_config(dkv, w, cap, P))
         perm, mix = synth.krpbh_params(0, 32)
