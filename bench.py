@@ -740,6 +740,10 @@ def main():
                          "(32-row query groups)")
     ap.add_argument("--B", type=int, default=0, help="override the workload's batch (profiling)")
     ap.add_argument("--L", type=int, default=0, help="override the committed length (profiling)")
+    ap.add_argument("--k-bits", type=int, default=0, choices=[0, 2, 3, 4, 16],
+                    help="override the line's K code width (0 = the workload's)")
+    ap.add_argument("--v-bits", type=int, default=0, choices=[0, 2, 3, 4, 16],
+                    help="override the line's V code width (0 = the workload's)")
     ap.add_argument("--v-rotation", type=int, default=0, choices=[0, 16, 32, 64, 128],
                     help="K-RPBH rotation of V with this Hadamard block (0 = none)")
     ap.add_argument("--suffix", type=int, default=0,
@@ -758,6 +762,10 @@ def main():
         w = w.with_(B=args.B)
     if args.L:
         w = w.with_(L=args.L)
+    if args.k_bits:
+        w = w.with_(k_bits=args.k_bits)
+    if args.v_bits:
+        w = w.with_(v_bits=args.v_bits)
 
     if args.impl == "reference":
         if rank != 0:
@@ -806,7 +814,8 @@ def main():
                               "timed region = one CUDA graph replay of the steps")
     line["config"]["timing"] = TIMING_METHOD
     line["roofline"] = roofline(w, r, peaks, peak_kind, traffic)
-    if args.suffix or args.select_budget:  # the recorded traffic is that of the plain launch
+    if args.suffix or args.select_budget or args.k_bits or args.v_bits:
+        # the recorded traffic is that of the plain launch at the workload's own code widths
         line["roofline"]["traffic"] = None
     line["clocks"] = r["clocks"]
     line["e2e"] = r["e2e"]

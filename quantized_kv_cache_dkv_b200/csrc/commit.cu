@@ -194,15 +194,23 @@ __device__ __forceinline__ void pack_codes(F code, uint32_t (&words)[n * B / 32]
   if constexpr (n * B / 32 > 2) words[2] = uint32_t(hi);
 }
 
-// Codes of n values (val(e); code 0 where bit e of `zero` is set) packed
+// Codes of n values (val(e), called with compile-time e only; val_slow(e),
+// the same value for a run-time e; code 0 where bit e of `zero` is set) packed
 // little-endian as in pack_codes, with code_of's arithmetic split in two
 // passes: the unrolled pass takes the reciprocal estimate for every value and
 // notes those near a tie; a rolled pass then replaces their codes with the
 // exact division's (rare).  The unrolled loop holds no call, so the values
-// need not stay live across one.
-template <int B, int n, class V>
-__device__ __forceinline__ void quantize_pack(V val, uint32_t zero, const GroupQuant& q, int levels,
-                                              uint32_t (&words)[n * B / 32]) {
+// need not stay live across one.  The unrolled pass clamps the estimate to
+// [0, levels] before rounding it: rounding to nearest is monotone and both
+// bounds are integers, so this gives clamp(rint(t)); the only ties that can
+// change a code (k + 1/2, k = 0 .. levels - 1) lie inside the range, where
+// the clamp leaves t as it is.  Adding 1.5 * 2^23 rounds t in [0, 15] to an
+// integer (round to nearest even, as rint) in the low mantissa bits, and
+// subtracting it back gives rint(t) exactly, so t - rint(t) is exact and
+// |t - rint(t)| > 1/2 - 2^-12 is the same tie test as code_of's.
+template <int B, int n, class V, class VS>
+__device__ __forceinline__ void quantize_pack(V val, VS val_slow, uint32_t zero, const GroupQuant& q,
+                                              int levels, uint32_t (&words)[n * B / 32]) {
   uint64_t lo = 0, hi = 0;  // bits [0, 64) and [64, 128) of the stream
   auto put = [&](int e, uint64_t cq) {
     const int pos = B * e;
@@ -217,20 +225,21 @@ __device__ __forceinline__ void quantize_pack(V val, uint32_t zero, const GroupQ
   };
   if (q.s32 > 0.f) {
     uint32_t tie = 0u;
+    const float lv = float(levels);
+    constexpr float kRound = 12582912.f;  // 1.5 * 2^23
 #pragma unroll
     for (int e = 0; e < n; ++e) {
       if ((zero >> e) & 1u) continue;
-      const float t = __fmul_rn(__fsub_rn(val(e), q.z32), q.rs);
-      if (fabsf(fabsf(__fsub_rn(t, rintf(t))) - 0.5f) < 2.44140625e-4f) tie |= 1u << e;
-      int c = __float2int_rn(t);
-      c = c < 0 ? 0 : (c > levels ? levels : c);
-      put(e, uint64_t(c));
+      const float t = fminf(fmaxf(__fmul_rn(__fsub_rn(val(e), q.z32), q.rs), 0.f), lv);
+      const float y = __fadd_rn(t, kRound);
+      if (fabsf(__fsub_rn(t, __fsub_rn(y, kRound))) > 0.499755859375f) tie |= 1u << e;
+      put(e, uint64_t(__float_as_uint(y) & uint32_t(levels)));
     }
 #pragma unroll 1
     while (tie) {
       const int e = __ffs(tie) - 1;
       tie &= tie - 1u;
-      int c = __float2int_rn(exact_quotient(__fsub_rn(val(e), q.z32), q.s32));
+      int c = __float2int_rn(exact_quotient(__fsub_rn(val_slow(e), q.z32), q.s32));
       c = c < 0 ? 0 : (c > levels ? levels : c);
       // replace the estimate's code at bits [B e, B e + B)
       const int pos = B * e;
@@ -489,7 +498,17 @@ commit_kernel(const __grid_constant__ CacheView c, const uint16_t* __restrict__ 
           }
         }
         auto raw = [&](int e) { return uint16_t(raw2[e >> 1] >> (16 * (e & 1))); };
-        auto val = [&](int e) { return sanitize(bf16_bits_to_f32(raw(e))); };
+        // the values, converted once where they fit in registers (2 and 4 bits)
+        float fv[kper <= 16 ? kper : 1];
+        auto val_slow = [&](int e) { return sanitize(bf16_bits_to_f32(raw(e))); };
+        auto val = [&](int e) {
+          if constexpr (kper <= 16) return fv[e];
+          else return val_slow(e);
+        };
+        if constexpr (kper <= 16) {
+#pragma unroll
+          for (int e = 0; e < kper; ++e) fv[e] = sanitize(bf16_bits_to_f32(raw(e)));
+        }
 #pragma unroll
         for (int e = 0; e < kper; ++e) {
           const float f = val(e);
@@ -502,7 +521,7 @@ commit_kernel(const __grid_constant__ CacheView c, const uint16_t* __restrict__ 
         if (mn > mx) mn = mx = 0.f;  // every token protected
         const GroupQuant q = make_quant(mn, mx, levels);
         uint32_t words[kwpt];
-        quantize_pack<KB, kper>(val, mw, q, levels, words);  // protected tokens: code 0
+        quantize_pack<KB, kper>(val, val_slow, mw, q, levels, words);  // protected tokens: code 0
         const size_t gidx = (size_t(u) * c.nG + size_t(j)) * d + ch;
 #pragma unroll
         for (int i = 0; i < kwpt; ++i) c.k_codes[gidx * c.kw + w * kwpt + i] = words[i];
@@ -548,19 +567,27 @@ commit_kernel(const __grid_constant__ CacheView c, const uint16_t* __restrict__ 
         raw2[4 * o + 3] = q8.w;
       }
       auto bits = [&](int e) { return uint16_t(raw2[e >> 1] >> (16 * (e & 1))); };
-      auto val = [&](int e) { return sanitize(bf16_bits_to_f32(bits(e))); };
+      // the values, converted once where they fit in registers (2 and 4 bits)
+      float fv[vper <= 16 ? vper : 1];
+      auto val_slow = [&](int e) { return sanitize(bf16_bits_to_f32(bits(e))); };
+      auto val = [&](int e) {
+        if constexpr (vper <= 16) return fv[e];
+        else return val_slow(e);
+      };
       float mn = __int_as_float(0x7f800000), mx = -__int_as_float(0x7f800000);
 #pragma unroll
       for (int e = 0; e < vper; ++e) {
-        range |= out_of_range(bf16_bits_to_f32(bits(e)));
-        const float f = val(e);
+        const float r = bf16_bits_to_f32(bits(e));
+        range |= out_of_range(r);
+        const float f = sanitize(r);
+        if constexpr (vper <= 16) fv[e] = f;
         mn = fminf(mn, f);
         mx = fmaxf(mx, f);
       }
       group_minmax(mn, mx, wpg);
       const GroupQuant q = make_quant(mn, mx, levels);
       uint32_t words[vwpt];
-      quantize_pack<VB, vper>(val, 0u, q, levels, words);
+      quantize_pack<VB, vper>(val, val_slow, 0u, q, levels, words);
       const size_t tok = size_t(u) * c.cap + size_t(p0 + t);
 #pragma unroll
       for (int i = 0; i < vwpt; ++i) c.v_codes[tok * c.vw + w * vwpt + i] = words[i];
