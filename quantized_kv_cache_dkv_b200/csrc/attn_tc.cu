@@ -223,7 +223,7 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                : "memory");
 }
 
-// 1-D bulk copy global -> shared (no multicast); completion counted on `bar`
+// 1-D bulk copy global -> this CTA's own shared memory; completion counted on `bar`
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes,
                                          uint32_t bar) {
   asm volatile(
