@@ -542,14 +542,16 @@ __device__ __forceinline__ void unrotate_row(float (&x)[4], int b, float norm,
   for (int e = 0; e < 4; ++e) x[e] = buf[4 * lane + e];
 }
 
+constexpr int kCombineWarps = 4;  // rows (one per warp) per combine CTA
+
 // One warp per (unit, row): out = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s
 // (rotated back first when V is stored rotated)
-__global__ void __launch_bounds__(128) combine_kernel(const __grid_constant__ AttnArgs a) {
-  __shared__ float rbuf[4][kHeadDim];
+__global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(const __grid_constant__ AttnArgs a) {
+  __shared__ float rbuf[kCombineWarps][kHeadDim];
   pdl_wait();
   pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t row = int64_t(blockIdx.x) * 4 + warp;
+  const int64_t row = int64_t(blockIdx.x) * kCombineWarps + warp;
   const int rows = a.c.rows;
   if (row >= int64_t(a.c.U) * rows) return;
   const int64_t u = row / rows, r = row % rows;
@@ -944,7 +946,8 @@ cudaError_t launch_topk(const AttnArgs& a, const float* part, int64_t ld, float*
 
 cudaError_t launch_combine(const AttnArgs& a, cudaStream_t s) {
   const int64_t rows = int64_t(a.c.U) * a.c.rows;
-  const cudaError_t e = launch_pdl(combine_kernel, dim3(unsigned((rows + 3) / 4)), dim3(128), 0, s, a);
+  const cudaError_t e = launch_pdl(combine_kernel, dim3(unsigned((rows + kCombineWarps - 1) / kCombineWarps)),
+                                   dim3(32 * kCombineWarps), 0, s, a);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
