@@ -27,7 +27,9 @@ def _cache_bytes(oc: OracleCache) -> int:
 
 @pytest.mark.parametrize("kb,vb,gk,gv,n_blocks", [(4, 4, 32, 32, 8), (2, 2, 64, 64, 9),
                                                   (2, 4, 32, 128, 5), (16, 4, 32, 32, 4),
-                                                  (4, 16, 128, 32, 7), (16, 16, 32, 32, 3)])
+                                                  (4, 16, 128, 32, 7), (16, 16, 32, 32, 3),
+                                                  (3, 3, 64, 64, 9), (3, 4, 32, 32, 6),
+                                                  (2, 3, 128, 32, 5)])
 def test_attention_bytes_match_the_cache_arrays(kb, vb, gk, gv, n_blocks):
     """No protected tokens: bench.attn_bytes equals the cache arrays plus Q,
     the active block and the output, exactly."""
