@@ -107,39 +107,35 @@ __device__ __forceinline__ void dequant2x16_raw(uint32_t w, __half2 s2, __half2 
   b.w = h2u(__hfma2(unbias(and_or(w8, 0x00C000C0u, kMagic1024), 0.015625f, -16.f), s2, z2));
 }
 
-// Code e (0..31) of 32 three-bit codes packed little-endian into the 96-bit
-// stream w2:w1:w0 (codes 10 and 21 straddle two words).
-template <int e>
-__device__ __forceinline__ uint32_t code3(uint32_t w0, uint32_t w1, uint32_t w2) {
-  constexpr int pos = 3 * e, wi = pos / 32, off = pos % 32;
-  const uint32_t a = wi == 0 ? w0 : (wi == 1 ? w1 : w2);
-  if constexpr (off <= 29) {
-    return (a >> off) & 7u;
-  } else {
-    const uint32_t b = wi == 0 ? w1 : w2;
-    return __funnelshift_r(a, b, off) & 7u;
-  }
+// Four three-bit codes at bits 0-2, 3-5, 6-8 and 9-11 of t -> two pairs of
+// halves q*s+z, (c0, c1) and (c2, c3).  t << 13 brings c1 to bits 16-18 and
+// c3 to bits 22-24, so one mask-and-or per pair forms 1024 + c0 | 1024 + c1
+// and 1024 + 64 c2 | 1024 + 64 c3 (exact in fp16); the unbias fma removes the
+// offset and the factor 64 exactly, and the second fma gives q*s+z with one
+// rounding.
+__device__ __forceinline__ void dequant3x4(uint32_t t, __half2 s2, __half2 z2, uint32_t& p01,
+                                           uint32_t& p23) {
+  const uint32_t t13 = t << 13;
+  const uint32_t a = and_or(t13, 0x00070000u, and_or(t, 0x00000007u, kMagic1024));
+  const uint32_t b = and_or(t13, 0x01C00000u, and_or(t, 0x000001C0u, kMagic1024));
+  p01 = h2u(__hfma2(unbias(a, 1.f, -1024.f), s2, z2));
+  p23 = h2u(__hfma2(unbias(b, 0.015625f, -16.f), s2, z2));
 }
 
-template <int i>
-__device__ __forceinline__ uint32_t dequant3_pair(uint32_t w0, uint32_t w1, uint32_t w2,
-                                                  __half2 s2, __half2 z2) {
-  // 1024 + c in each half (exact), minus 1024 (exact), then c * s + z (one rounding)
-  const uint32_t x = code3<2 * i>(w0, w1, w2) | (code3<2 * i + 1>(w0, w1, w2) << 16) | kMagic1024;
-  return h2u(__hfma2(__hsub2(u2h(x), h2c(1024.f)), s2, z2));
-}
-
-// 32 three-bit codes -> 32 halves q*s+z in element order (out[k] = e 8k..8k+7)
+// 32 three-bit codes packed little-endian into the 96-bit stream w2:w1:w0
+// (code e at bits 3e; codes 10 and 21 straddle two words) -> 32 halves q*s+z
+// in element order (out[k] = e 8k..8k+7).  Codes 4g..4g+3 sit at stream bits
+// 12g..12g+11, which a shift (a funnel shift across a word boundary) moves to
+// bits 0-11.
 __device__ __forceinline__ void dequant3x32(uint32_t w0, uint32_t w1, uint32_t w2, __half2 s2,
                                             __half2 z2, uint4 (&out)[4]) {
-  out[0] = make_uint4(dequant3_pair<0>(w0, w1, w2, s2, z2), dequant3_pair<1>(w0, w1, w2, s2, z2),
-                      dequant3_pair<2>(w0, w1, w2, s2, z2), dequant3_pair<3>(w0, w1, w2, s2, z2));
-  out[1] = make_uint4(dequant3_pair<4>(w0, w1, w2, s2, z2), dequant3_pair<5>(w0, w1, w2, s2, z2),
-                      dequant3_pair<6>(w0, w1, w2, s2, z2), dequant3_pair<7>(w0, w1, w2, s2, z2));
-  out[2] = make_uint4(dequant3_pair<8>(w0, w1, w2, s2, z2), dequant3_pair<9>(w0, w1, w2, s2, z2),
-                      dequant3_pair<10>(w0, w1, w2, s2, z2), dequant3_pair<11>(w0, w1, w2, s2, z2));
-  out[3] = make_uint4(dequant3_pair<12>(w0, w1, w2, s2, z2), dequant3_pair<13>(w0, w1, w2, s2, z2),
-                      dequant3_pair<14>(w0, w1, w2, s2, z2), dequant3_pair<15>(w0, w1, w2, s2, z2));
+  const uint32_t t[8] = {w0,      w0 >> 12, __funnelshift_r(w0, w1, 24), w1 >> 4,
+                         w1 >> 16, __funnelshift_r(w1, w2, 28), w2 >> 8, w2 >> 20};
+  uint32_t p[16];
+#pragma unroll
+  for (int g = 0; g < 8; ++g) dequant3x4(t[g], s2, z2, p[2 * g], p[2 * g + 1]);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) out[k] = make_uint4(p[4 * k], p[4 * k + 1], p[4 * k + 2], p[4 * k + 3]);
 }
 
 // 8 bf16 -> 8 fp16 (exact inside fp16's normal range)
