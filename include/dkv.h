@@ -73,8 +73,7 @@ enum {
 
 /* Cache shape.  Supported: head_dim == 128; block a multiple of 32, <= 128;
  * q_heads a multiple of kv_heads with (q_heads/kv_heads)*block <= 256;
- * k_bits, v_bits in {2, 3, 4, 16} (16 = store bf16, quantization off; 3-bit
- * V cannot be rotated);
+ * k_bits, v_bits in {2, 3, 4, 16} (16 = store bf16, quantization off);
  * k_group in {32, 64, 128} with k_group % block == 0 or block % k_group == 0;
  * v_group in {32, 64, 128}; max_tokens a multiple of max(k_group, block). */
 typedef struct dkv_config {

@@ -142,12 +142,14 @@ __device__ __forceinline__ void rotate_row(float (&x)[4], int b, float norm,
 
 // Per-token quantization of a rotated V row held by a warp (channels 4 lane +
 // e): groups of G consecutive channels (G/4 lanes), the same quantizer as
-// quant_v_group, codes packed along channels.
+// quant_v_group, codes packed along channels.  At 3 bits the 12 code bits of
+// a lane sit at stream bits 12 (lane % 8) of its 32-channel block, whose 96
+// bits fill three words (lanes 2 and 5 straddle a word boundary).
 template <int VB>
 __device__ __forceinline__ void quant_v_rotated(float (&w)[4], int G, uint32_t* codes, __half2* sz,
                                              int lane, bool& range) {
   constexpr int levels = (1 << VB) - 1;
-  constexpr int lw = 8 / VB;  // lanes per code word (32 / VB channels)
+  constexpr int lw = VB == 3 ? 8 : 8 / VB;  // lanes per code word (32 / VB channels; 3 words at 3 bits)
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
     range |= out_of_range(w[e]);
@@ -163,10 +165,26 @@ __device__ __forceinline__ void quant_v_rotated(float (&w)[4], int G, uint32_t* 
   uint32_t word = 0;
 #pragma unroll
   for (int e = 0; e < 4; ++e) word |= code_of(w[e], q, levels) << (e * VB);
-  word <<= (lane % lw) * 4 * VB;
+  if constexpr (VB == 3) {
+    const int pos = 12 * (lane & 7), wi = pos >> 5, off = pos & 31;
+    uint32_t part[3];
 #pragma unroll
-  for (int o = 1; o < lw; o <<= 1) word |= __shfl_xor_sync(0xffffffffu, word, o);
-  if (lane % lw == 0) codes[lane / lw] = word;
+    for (int k = 0; k < 3; ++k) {
+      part[k] = wi == k ? word << off : 0u;
+      if (off > 20 && wi + 1 == k) part[k] |= word >> (32 - off);
+#pragma unroll
+      for (int o = 1; o < 8; o <<= 1) part[k] |= __shfl_xor_sync(0xffffffffu, part[k], o);
+    }
+    if ((lane & 7) == 0) {
+#pragma unroll
+      for (int k = 0; k < 3; ++k) codes[(lane >> 3) * 3 + k] = part[k];
+    }
+  } else {
+    word <<= (lane % lw) * 4 * VB;
+#pragma unroll
+    for (int o = 1; o < lw; o <<= 1) word |= __shfl_xor_sync(0xffffffffu, word, o);
+    if (lane % lw == 0) codes[lane / lw] = word;
+  }
   if (lane % (G / 4) == 0) sz[lane / (G / 4)] = q.sz;
 }
 
@@ -436,8 +454,8 @@ commit_kernel(const __grid_constant__ CacheView c, const uint16_t* __restrict__ 
       reinterpret_cast<uint4*>(c.v_sink + (size_t(u) * c.sink + size_t(p0 + t)) * d)[o] =
           reinterpret_cast<const uint4*>(vu + size_t(t) * d)[o];
     }
-    if (VB != 3 && c.vrot_b) {
-      // rotated V (no sink; 2 or 4 bits): warp wv rotates and quantizes tokens t_lo + wv, + 8, ...
+    if (c.vrot_b) {
+      // rotated V (no sink): warp wv rotates and quantizes tokens t_lo + wv, + 8, ...
       int pm[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) pm[e] = __ldg(c.vrot_perm + 4 * lane + e);
@@ -451,8 +469,7 @@ commit_kernel(const __grid_constant__ CacheView c, const uint16_t* __restrict__ 
         }
         rotate_row(x, c.vrot_b, c.vrot_norm, c.vrot_mix, lane);
         const size_t tok = size_t(u) * c.cap + size_t(p0 + t);
-        quant_v_rotated<VB == 3 ? 4 : VB>(x, c.GV, c.v_codes + tok * c.vw, c.v_sz + tok * c.vgroups,
-                                          lane, range);
+        quant_v_rotated<VB>(x, c.GV, c.v_codes + tok * c.vw, c.v_sz + tok * c.vgroups, lane, range);
       }
     }
   }

@@ -821,7 +821,6 @@ int dkv_cache_set_v_rotation(dkv_cache* c, const int32_t* perm, const float* mix
   if (block != 16 && block != 32 && block != 64 && block != 128)
     return fail(DKV_ERR_UNSUPPORTED, "rotation block must be 16, 32, 64 or 128");
   if (c->v.vb == 16) return fail(DKV_ERR_UNSUPPORTED, "V rotation needs quantized V (v_bits < 16)");
-  if (c->v.vb == 3) return fail(DKV_ERR_UNSUPPORTED, "V rotation needs 2- or 4-bit V");
   if (c->v.sink > 0) return fail(DKV_ERR_UNSUPPORTED, "V rotation with an attention sink is not supported");
   if (!perm || !mix) return fail(DKV_ERR_INVALID_ARG, "perm and mix must not be NULL");
   const int d = dkv::kHeadDim, k = d / block;

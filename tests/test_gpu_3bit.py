@@ -70,10 +70,3 @@ def test_three_bit_commit_and_attention(dkv, name, over, sink):
     dkv.dkv_block_attention(cache, dev_bf16(Q), dev_bf16(Ka), dev_bf16(Va), w.softmax_scale, out)
     torch.cuda.synchronize()
     assert dkv.dkv_last_attention_plan(cache)[0] == 2
-    # no rotated V at 3 bits
-    if w.v_bits == 3:
-        fresh = dkv.dkv_cache_alloc(gpu_config(dkv, w, cap, P))
-        perm, mix = synth.krpbh_params(0, 32)
-        with pytest.raises(dkv.DkvError) as ei:
-            dkv.dkv_cache_set_v_rotation(fresh, perm, mix, 32)
-        assert ei.value.code == dkv.DKV_ERR_UNSUPPORTED

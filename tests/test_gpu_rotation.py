@@ -1,7 +1,7 @@
 """Rotated V (K-RPBH before per-token V quantization, output rotated back) on
-both attention kernels against the oracle: codes, scales and zero points bit
-for bit (the rotation runs in the same fp32 order on both sides), attention
-within the output bound."""
+both attention kernels against the oracle, at 2, 3 and 4 bits: codes, scales
+and zero points bit for bit (the rotation runs in the same fp32 order on both
+sides), attention within the output bound."""
 import numpy as np
 import pytest
 
@@ -43,7 +43,10 @@ def _attend(dkv, cache, Q, Ka, Va, w, noalloc=False):
 
 CASES = [("mha8b", 16, {}), ("mha8b", 128, {}), ("batch32", 32, {}), ("gqa7b", 64, {}),
          ("tiny", 32, {"v_group": 128}), ("tiny", 16, {"v_bits": 2, "v_group": 64}),
-         ("longprompt", 32, {"L": 320})]
+         ("longprompt", 32, {"L": 320}),
+         # 3-bit V: a lane's 12 code bits straddle words in lanes 2 and 5 of each 8
+         ("batch32", 64, {"k_bits": 3, "v_bits": 3, "v_group": 32}),
+         ("tiny", 128, {"v_bits": 3, "v_group": 128}), ("mha8b", 32, {"v_bits": 3, "v_group": 64})]
 
 
 @pytest.mark.parametrize("name,b,over", CASES)
