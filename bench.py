@@ -348,8 +348,10 @@ def run_gpu(w: synth.Workload, K: int, W: int, want_e2e=True, log=print, kernel=
                 dkv.dkv_cache_truncate(caches[r], w.L)
                 pos[r] = 0
 
-    # warm-up (eager), then capture exactly K steps in one CUDA graph
-    for k in range(W):
+    # warm-up (eager; at least one step per cache replica, so that every
+    # handle has made its first call -- which may allocate -- before the
+    # capture), then capture exactly K steps in one CUDA graph
+    for k in range(max(W, R)):
         step(k)
     finish()
     torch.cuda.synchronize()
