@@ -868,9 +868,19 @@ template <int KB, int VB>
 cudaError_t launch_scores_kv(const AttnArgs& a, float* part, int64_t ld, cudaStream_t s) {
   const int nrb = (a.c.rows + kRowsPerCta - 1) / kRowsPerCta;
   const int64_t n_tiles = (a.L + T - 1) / T;
-  // about 2 CTAs per SM over the whole grid
-  const int64_t want = (2 * 148 + int64_t(a.c.U) * nrb - 1) / (int64_t(a.c.U) * nrb);
-  const int64_t tpc = n_tiles < 1 ? 1 : (n_tiles + want - 1) / want;
+  // chunks of tiles per (unit, row block): the count whose waves (two CTAs
+  // per SM resident) times tiles per chunk is least, i.e. the grid that
+  // loses the least to a partly filled last wave
+  const int64_t slots = 2 * 148, cells = int64_t(a.c.U) * nrb;
+  int64_t tpc = n_tiles < 1 ? 1 : n_tiles, best = -1;
+  for (int64_t nc = 1; n_tiles > 0 && nc <= n_tiles && nc <= 64; ++nc) {
+    const int64_t t = (n_tiles + nc - 1) / nc;
+    const int64_t waves = (cells * ((n_tiles + t - 1) / t) + slots - 1) / slots;
+    if (best < 0 || waves * (t + 1) < best) {
+      best = waves * (t + 1);
+      tpc = t;
+    }
+  }
   const int nchunk = int(n_tiles < 1 ? 1 : (n_tiles + tpc - 1) / tpc);
   const unsigned grid = unsigned(a.c.U) * unsigned(nrb) * unsigned(nchunk);
   const cudaError_t e = launch_pdl(score_kernel<KB, VB>, dim3(grid), dim3(256), 0, s, a, part, ld,
