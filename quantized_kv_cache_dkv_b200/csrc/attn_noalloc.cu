@@ -15,7 +15,7 @@ namespace {
 constexpr size_t kScratchBytes = DKV_NOALLOC_SCRATCH_BYTES;
 constexpr int kMaxDevices = 64;
 
-// Split partials, laid out as the handle's workspace (split_o_bytes of fp32
+// Split partials, laid out as the handle's workspace (split_o_bytes of fp16
 // partial outputs, then split_ml_bytes of (max, sum) pairs).  Host code must
 // not use this name as an address: it is a host-side stand-in.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];

@@ -126,7 +126,7 @@ struct AttnArgs {
   int32_t nsplit;
   int32_t tiles_per_split;  // in units of the kernel's token tile
   int32_t final_out;        // 1: the attention kernel writes bf16 out (one split,
-                            // no rotation); 0: fp32 partials for combine_kernel
+                            // no rotation); 0: fp16 partials for combine_kernel
   int32_t part_base;        // split sp of unit u writes partial u*part_stride +
   int32_t part_stride;      // part_base + sp (one call: 0 and nsplit)
   // Attention over selected committed tokens (mma.sync kernel, gather = 1):
@@ -201,8 +201,9 @@ constexpr int kTcTile = 128;
 bool tc_supported(const CacheView& c);
 cudaError_t launch_attention_tc(const AttnArgs& a, cudaStream_t s);
 
-// Split workspace of one attention call: fp32 partial outputs
-// [U][splits][rows][d], then (running max, sum) pairs [U][splits][rows],
+// Split workspace of one attention call: fp16 partial outputs (each split's
+// output divided by its row sum) [U][splits][rows][d], then (max, sum)
+// pairs in fp32 [U][splits][rows],
 // starting at the next 256-byte boundary.  The handle's workspace and the
 // no-allocation entry point's static buffer are both sized by these.
 inline size_t split_o_bytes(int64_t U, int64_t splits, int64_t rows) {
